@@ -1,0 +1,391 @@
+"""Pins of the fp64 oracle to things other than itself (CPU only).
+
+Each test checks one oracle function against a closed form, a library routine (torch SDPA,
+scikit-learn k-means, numpy lstsq, scipy orth), brute force on a tiny input, or a hand-worked
+fixture under tests/golden/ whose derivation is written in the fixture.  They are chosen so
+that a plausible slip (a dropped term, a wrong sign or scale, a transposed operand, an
+off-by-one in a sampling formula) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+from oracle import sparsepr_oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- random draws
+def test_splitmix64_published_vectors():
+    for case in _gold("splitmix64_vectors.json")["cases"]:
+        r = O.SplitMix64(case["seed"])
+        assert [r.next() for _ in case["outputs"]] == case["outputs"]
+
+
+def test_kmeans_init_ids_is_a_partial_fisher_yates():
+    # Brute force: the same shuffle on an explicit full array.
+    for n, c, seed in [(10, 10, 3), (1000, 16, 77), (37, 5, 2**63 + 11)]:
+        arr = list(range(n))
+        r = O.SplitMix64(seed)
+        for i in range(c):
+            j = i + r.next() % (n - i)
+            arr[i], arr[j] = arr[j], arr[i]
+        ids = O.kmeans_init_ids(n, c, seed)
+        assert ids == arr[:c]
+        assert len(set(ids)) == c and all(0 <= x < n for x in ids)
+    assert sorted(O.kmeans_init_ids(50, 50, 9)) == list(range(50))
+
+
+def test_stream_seeds_differ_per_head_and_stage():
+    seeds = {O.stream_seed(5, bh, st) for bh in range(4) for st in range(2)}
+    assert len(seeds) == 8
+
+
+# ---------------------------------------------------------------- sampling
+def test_sample_query_rows_formula():
+    assert list(O.sample_query_rows(8, 8)) == list(range(8))
+    assert list(O.sample_query_rows(10, 1)) == [5]
+    assert list(O.sample_query_rows(10, 2)) == [2, 7]
+    r = O.sample_query_rows(118800, 1024)
+    assert np.all(np.diff(r) > 0) and r[0] >= 0 and r[-1] < 118800
+
+
+# ---------------------------------------------------------------- attention
+def _sdpa(q, k, v, mask=None):
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x))[None, None]
+    m = None if mask is None else torch.from_numpy(mask)[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), attn_mask=m)[0, 0].numpy()
+
+
+def test_dense_attention_matches_torch_sdpa():
+    rng = np.random.default_rng(0)
+    q, k, v = rng.standard_normal((7, 16)), rng.standard_normal((23, 16)), rng.standard_normal((23, 5))
+    np.testing.assert_allclose(O.attention(q * 3, k, v), _sdpa(q * 3, k, v), rtol=1e-12, atol=1e-12)
+
+
+def test_dense_attention_special_cases():
+    rng = np.random.default_rng(1)
+    q, k = rng.standard_normal((4, 8)), rng.standard_normal((9, 8))
+    v = np.tile(rng.standard_normal((1, 3)), (9, 1))
+    np.testing.assert_allclose(O.attention(q, k, v), np.tile(v[:1], (4, 1)), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(O.attention(q, k[:1], v[:1] * 2), np.tile(v[:1] * 2, (4, 1)), atol=1e-14)
+    # a key far more aligned than the others takes all the mass
+    kk = np.zeros((3, 8)); kk[1, 0] = 1000.0
+    qq = np.zeros((1, 8)); qq[0, 0] = 1.0
+    vv = np.eye(3)
+    np.testing.assert_allclose(O.attention(qq, kk, vv), [[0, 1, 0]], atol=1e-12)
+
+
+def test_sparse_attention_matches_masked_sdpa():
+    rng = np.random.default_rng(2)
+    N, d = 40, 8
+    q, k, v = rng.standard_normal((N, d)), rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    ql = rng.integers(0, 3, N)
+    kl = rng.integers(0, 4, N)
+    route = np.array([[1, 0, 1, 0], [0, 1, 0, 0], [1, 1, 1, 1]], dtype=bool)
+    mask = route[ql][:, kl]
+    np.testing.assert_allclose(O.sparse_attention(q, k, v, ql, kl, route), _sdpa(q, k, v, mask),
+                               rtol=1e-12, atol=1e-12)
+    full = np.ones((3, 4), dtype=bool)
+    np.testing.assert_allclose(O.sparse_attention(q, k, v, ql, kl, full), O.attention(q, k, v), atol=1e-13)
+
+
+# ---------------------------------------------------------------- k-means
+def _blobs(rng, n_per, centres, spread):
+    pts = [c + spread * rng.standard_normal((n_per, centres.shape[1])) for c in centres]
+    return np.concatenate(pts)
+
+
+def test_lloyd_matches_scikit_learn():
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(3)
+    X = _blobs(rng, 30, 4.0 * rng.standard_normal((6, 5)), 1.0)
+    init = X[[0, 31, 62, 95, 130, 170]]
+    res = O.lloyd(X, init, iters=100, tol=0.0)
+    km = KMeans(n_clusters=6, init=init, n_init=1, max_iter=100, tol=0.0, algorithm="lloyd").fit(X)
+    assert np.array_equal(res.labels, km.labels_)
+    np.testing.assert_allclose(res.centroids, km.cluster_centers_, rtol=1e-12, atol=1e-12)
+
+
+def test_lloyd_objective_non_increasing_and_fixed_point():
+    rng = np.random.default_rng(4)
+    X = rng.standard_normal((300, 4))
+    res = O.lloyd(X, X[:12], iters=50, tol=0.0)
+    J = np.array(res.objective)
+    assert np.all(np.diff(J) <= 1e-9 * J[:-1])
+    again = O.lloyd(X, res.centroids, iters=1, tol=0.0)
+    assert np.array_equal(again.labels, res.labels)
+    np.testing.assert_allclose(again.centroids, res.centroids, atol=1e-13)
+
+
+def test_lloyd_recovers_generator_tiles():
+    from free_block_sparse_02_b200 import configs, gen
+    w = configs.workload(0)
+    Q, K, V = gen.make_qkv(w)
+    k = gen.as_f64(K)[0, 0]
+    tiles = gen.token_tiles(w)
+    first = [int(np.flatnonzero(tiles == t)[0]) for t in range(w.n_tiles)]
+    res = O.lloyd(k, k[first], iters=20, tol=0.0)
+    assert np.array_equal(res.labels, tiles)
+
+
+def test_lloyd_empty_group_keeps_centroid_and_shadow():
+    X = np.array([[0.0], [0.1], [10.0]])
+    init = np.array([[0.0], [10.0], [100.0]])
+    res = O.lloyd(X, init, iters=3, tol=0.0, shadow=X * 2, shadow_init=init * 2)
+    assert list(res.labels) == [0, 0, 1]
+    assert res.centroids[2, 0] == 100.0 and res.shadow[2, 0] == 200.0
+    np.testing.assert_allclose(res.shadow[:2, 0], [0.1, 20.0])
+
+
+def test_lloyd_tolerance_stop_rule():
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((400, 3))
+    res = O.lloyd(X, X[:8], iters=100, tol=1e-2)
+    J = res.objective
+    assert res.n_iter == len(J)
+    if res.n_iter < 100:
+        assert J[-2] - J[-1] <= 1e-2 * J[-2]
+    for a, b in zip(J[:-2], J[1:-1]):
+        assert a - b > 1e-2 * a
+    never = O.lloyd(X, X[:8], iters=7, tol=-1.0)
+    assert never.n_iter == 7
+
+
+def test_near_tie_margin_flags_equidistant_point():
+    X = np.array([[0.0], [1.0], [2.0]])
+    labels, d1, margin = O.assign(X, np.array([[0.0], [2.0]]))
+    assert list(labels) == [0, 0, 1]          # the midpoint goes to the lower index
+    assert margin[1] == 0.0 and margin[0] == np.inf
+
+
+def test_key_response_kmeans_equals_metric_kmeans_in_key_space():
+    """k-means on rows of F = K Qs^T / sqrt(d) equals Euclidean k-means on K L with
+    L L^T = Qs^T Qs / d (a different space and a library k-means)."""
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(6)
+    d, s = 6, 20
+    K = _blobs(rng, 25, 3.0 * rng.standard_normal((5, d)), 0.7)
+    Qs = rng.standard_normal((s, d))
+    F = K @ Qs.T / math.sqrt(d)
+    ids = [0, 26, 52, 77, 101]
+    res = O.lloyd(F, F[ids], iters=60, tol=0.0, shadow=K, shadow_init=K[ids])
+    L = np.linalg.cholesky(Qs.T @ Qs / d)
+    Z = K @ L
+    km = KMeans(n_clusters=5, init=Z[ids], n_init=1, max_iter=60, tol=0.0, algorithm="lloyd").fit(Z)
+    assert np.array_equal(res.labels, km.labels_)
+    # the shadow (key-space) centroids map onto the response-space centroids
+    np.testing.assert_allclose(res.shadow @ Qs.T / math.sqrt(d), res.centroids, rtol=1e-10, atol=1e-10)
+
+
+# ---------------------------------------------------------------- responses
+def test_query_responses_and_rms():
+    rng = np.random.default_rng(7)
+    q, c = rng.standard_normal((5, 16)), rng.standard_normal((3, 16))
+    R = O.query_responses(q, c)
+    np.testing.assert_allclose(R[2, 1], float(q[2] @ c[1]) / 4.0, rtol=1e-14)
+    Rt = O.rms_normalize(R)
+    np.testing.assert_allclose(np.mean(Rt ** 2, axis=1), 1.0, rtol=1e-9)
+    np.testing.assert_allclose(O.rms_normalize(7.5 * R), Rt, rtol=1e-10)  # the 1e-12 epsilon
+    assert np.all(np.sign(Rt) == np.sign(R))
+    assert np.all(O.rms_normalize(np.zeros((2, 3))) == 0.0)
+
+
+# ---------------------------------------------------------------- routing
+def test_route_group_hand_cases():
+    g = _gold("routing_cases.json")
+    S, m = np.array(g["scores"]), np.array(g["sizes"])
+    for case in g["cases"]:
+        assert O.route_group(S, m, case["fixed_k"], case["kappa"]) == case["expected"], case
+
+
+def test_routing_scores_hand_case():
+    c = _gold("routing_cases.json")["score_case"]
+    S = O.routing_scores(np.array(c["R"]), np.array(c["qlabels"]), c["n_qgroups"], np.array(c["ksizes"]))
+    np.testing.assert_allclose(S[0], c["expected_row0"], rtol=1e-15)
+    assert np.all(np.isneginf(S[1]))
+
+
+def test_routing_scores_pool_by_linearity():
+    # mean of responses == response of the mean query (a different computation path)
+    rng = np.random.default_rng(8)
+    q, kc = rng.standard_normal((30, 8)), rng.standard_normal((4, 8))
+    ql = rng.integers(0, 3, 30)
+    m = np.array([3, 0, 5, 9])
+    S = O.routing_scores(O.query_responses(q, kc), ql, 3, m)
+    for g in range(3):
+        qbar = q[ql == g].mean(axis=0)
+        ref = kc @ qbar / math.sqrt(8) + np.log(np.where(m > 0, m, 1))
+        np.testing.assert_allclose(S[g][m > 0], ref[m > 0], rtol=1e-12)
+        assert np.isneginf(S[g][1])
+
+
+def test_per_row_key_budget():
+    # kappa*N + (s + Ck + P)*N == rho*N^2 : the target counts routing and probe pairs
+    N, s, Ck, P = 16384, 256, 64, 128
+    kap = O.per_row_key_budget(0.22, N, s, Ck, P)
+    assert abs((kap + s + Ck + P) * N / N ** 2 - float(np.float32(0.22))) < 1e-12
+
+
+# ---------------------------------------------------------------- probes
+def test_probes_uniform_formula():
+    t, w = O.probes_uniform(10, 2)
+    assert list(t) == [2, 7] and list(w) == [1.0, 1.0]
+    t, _ = O.probes_uniform(1024, 32)
+    assert t[0] == 16 and t[-1] == 1008 and np.all(np.diff(t) == 32)
+
+
+def test_probes_stratified_hand_cases():
+    for c in _gold("stratified_probe_cases.json")["cases"]:
+        t, w = O.probes_stratified(np.array(c["labels"]), c["n_qgroups"], c["P"])
+        assert list(t) == c["tokens"]
+        np.testing.assert_allclose(w, c["weights"], rtol=1e-14)
+
+
+def test_probes_stratified_invariants():
+    rng = np.random.default_rng(9)
+    ql = rng.integers(0, 17, 5000)
+    ql[ql == 3] = 4                       # an empty group
+    t, w = O.probes_stratified(ql, 17, 128)
+    assert len(t) == 128 and len(set(t.tolist())) == 128 and np.all(np.diff(t) > 0)
+    np.testing.assert_allclose(w.sum(), 128.0, rtol=1e-13)
+    n = np.bincount(ql, minlength=17)
+    m = np.bincount(ql[t], minlength=17)
+    assert np.all(np.abs(m - 128 * n / 5000) < 1.0 + 1e-12) and m[3] == 0
+
+
+# ---------------------------------------------------------------- ridge and projection
+def test_ridge_exact_when_residual_is_affine():
+    rng = np.random.default_rng(10)
+    P, d = 40, 6
+    osp = rng.standard_normal((P, d))
+    Btrue = rng.standard_normal((d + 1, d))
+    od = osp + np.hstack([osp, np.ones((P, 1))]) @ Btrue
+    A, lam = O.ridge_fit(osp, od, rng.uniform(0.5, 2.0, P), 0.0)
+    assert lam == 0.0
+    np.testing.assert_allclose(A, Btrue, rtol=1e-10, atol=1e-10)
+
+
+def test_ridge_matches_augmented_lstsq():
+    rng = np.random.default_rng(11)
+    P, d = 25, 5
+    osp, od, w = rng.standard_normal((P, d)), rng.standard_normal((P, d)), rng.uniform(0.2, 3.0, P)
+    A, lam = O.ridge_fit(osp, od, w, -1.0)
+    X = np.hstack([osp, np.ones((P, 1))])
+    G = X.T @ (w[:, None] * X)
+    assert lam == pytest.approx(1e-3 * np.trace(G) / (d + 1), rel=1e-14)
+    Xa = np.vstack([np.sqrt(w)[:, None] * X, math.sqrt(lam) * np.eye(d + 1)])
+    Ra = np.vstack([np.sqrt(w)[:, None] * (od - osp), np.zeros((d + 1, d))])
+    ref = np.linalg.lstsq(Xa, Ra, rcond=None)[0]
+    np.testing.assert_allclose(A, ref, rtol=1e-10, atol=1e-11)
+    # normal equations: X^T W (R - X A) = lam A
+    np.testing.assert_allclose(X.T @ (w[:, None] * ((od - osp) - X @ A)), lam * A, atol=1e-11)
+    A1, lam1 = O.ridge_fit(osp, od, w, 1.0)
+    assert lam1 == 1.0 and not np.allclose(A1, A)
+
+
+def test_ridge_mean_only_special_case():
+    rng = np.random.default_rng(12)
+    P, d = 9, 4
+    R, w = rng.standard_normal((P, d)), rng.uniform(0.5, 1.5, P)
+    A, _ = O.weighted_ridge(np.ones((P, 1)), R, w, 0.0)
+    np.testing.assert_allclose(A[0], (w[:, None] * R).sum(0) / w.sum(), rtol=1e-13)
+    A, lam = O.weighted_ridge(np.ones((P, 1)), R, w, 2.0)
+    np.testing.assert_allclose(A[0], (w[:, None] * R).sum(0) / (w.sum() + 2.0), rtol=1e-13)
+
+
+def test_residual_span_projection():
+    rng = np.random.default_rng(13)
+    P, d = 5, 12                                     # rank-deficient: span has dimension 5
+    R, w = rng.standard_normal((P, d)), rng.uniform(0.5, 1.5, P)
+    U = O.residual_span_basis(R, w)
+    assert U.shape == (d, P)
+    Qo = scipy.linalg.orth(R.T)
+    np.testing.assert_allclose(U @ U.T, Qo @ Qo.T, atol=1e-12)
+    A = rng.standard_normal((d + 1, d))
+    PA = O.restrict_to_residual_span(A, R, w)
+    np.testing.assert_allclose(PA, A @ Qo @ Qo.T, atol=1e-12)
+    np.testing.assert_allclose(O.restrict_to_residual_span(PA, R, w), PA, atol=1e-12)
+    # the ridge solution already lies in the span: the projection leaves it unchanged
+    osp = rng.standard_normal((P, d))
+    A2, _ = O.ridge_fit(osp, osp + R, w, 0.5)
+    np.testing.assert_allclose(O.restrict_to_residual_span(A2, R, w), A2, atol=1e-12)
+    assert O.residual_span_basis(np.zeros((3, 4)), np.ones(3)).shape == (4, 0)
+
+
+def test_apply_correction_and_row_errors():
+    osp = np.array([[1.0, 2.0]])
+    A = np.array([[1.0, 0.0], [0.0, 2.0], [0.5, -1.0]])
+    np.testing.assert_allclose(O.apply_correction(osp, A), [[1 + 1 + 0.5, 2 + 4 - 1]])
+    e = O.row_errors(np.array([[3.0, 4.0], [1.0, 1.0]]), np.array([[0.0, 0.0], [1.0, 1.0]]))
+    np.testing.assert_allclose(e, [5.0 / 1e-8, 0.0])
+
+
+# ---------------------------------------------------------------- whole call
+class _Cfg:
+    s, n_kgroups, n_qgroups, density, fixed_k, P, probe_mode = 16, 4, 4, 0.5, 0, 6, 1
+    lam, km_iters, km_iters_warm, km_tol, seed = -1.0, 8, 2, 1e-4, 99
+
+
+def _small_inputs(seed=14, N=96, d=8):
+    rng = np.random.default_rng(seed)
+    centres = 2.0 * rng.standard_normal((6, d))
+    lab = np.repeat(np.arange(6), N // 6)
+    q = centres[lab] + 0.5 * rng.standard_normal((N, d))
+    k = centres[lab] + 0.5 * rng.standard_normal((N, d))
+    return q, k, rng.standard_normal((N, d))
+
+
+def test_call_with_every_group_kept_is_dense():
+    q, k, v = _small_inputs()
+    cfg = _Cfg()
+    cfg.fixed_k = cfg.n_kgroups
+    r = O.call_head(q, k, v, cfg, 0)
+    dense = O.attention(q, k, v)
+    np.testing.assert_allclose(r["osp"], dense, atol=1e-13)
+    np.testing.assert_allclose(r["O"], dense, atol=1e-13)
+    assert np.abs(r["A"]).max() < 1e-12
+    N = q.shape[0]
+    assert r["sparse_pairs"] == N * N
+    assert r["density"] == pytest.approx(1.0 + (cfg.s + cfg.n_kgroups + cfg.P) / N)
+
+
+def test_call_constant_values_are_exact():
+    q, k, v = _small_inputs(15)
+    v[:] = np.array([0.5, -1.0, 2.0, 0.0, 1.0, 3.0, -2.0, 0.25])
+    r = O.call_head(q, k, v, _Cfg(), 0)
+    np.testing.assert_allclose(r["O"], np.tile(v[:1], (q.shape[0], 1)), atol=1e-12)
+
+
+def test_call_partition_is_consistent():
+    q, k, v = _small_inputs(16)
+    cfg = _Cfg()
+    r = O.call_head(q, k, v, cfg, 3)
+    assert np.array_equal(np.bincount(r["klabels"], minlength=4), r["ksizes"])
+    # key-space centroids are the means of their groups' keys
+    for j in range(4):
+        if r["ksizes"][j]:
+            np.testing.assert_allclose(r["kcent"][j], k[r["klabels"] == j].mean(0), atol=1e-13)
+    assert np.all(r["route"].sum(1)[r["qsizes"] > 0] >= 1)
+    assert np.all(r["O"][r["probes"]] == r["odense"])
+    # warm start from the state of this call runs the warm iteration limit
+    r2 = O.call_head(q, k, v, cfg, 3, warm=O.warm_state(r))
+    assert r2["kmeans_k"].n_iter <= cfg.km_iters_warm
+    assert np.array_equal(r2["klabels"], r["klabels"])
+
+
+def test_table2_error_reduction_arithmetic():
+    t = _gold("table2_error_reduction.json")
+    red = [100 * (1 - b / a) for a, b in zip(t["semantic_mean"], t["sparsepr_mean"])]
+    lo, hi = t["stated_reduction_range_pct"]
+    assert round(min(red), 1) == lo and round(max(red), 1) == hi
