@@ -1,0 +1,302 @@
+#!/usr/bin/env python
+"""Throughput of the SparsePR per-call sparse attention operator on B200.
+
+One step = one whole operator call (plan: response-coupled partitioning, routing, probes;
+attention: block-sparse + dense probe rows; fit_apply: weighted ridge + residual add) over
+one batch of seeded synthetic video-latent Q/K/V of the chosen workload (default: the
+mid-size bf16 call, B=1 H=8 N=16384 d=64 at 22% density).
+
+  python bench.py [--gpus N --steps K --warmup W] [--workload I] [--impl reference]
+
+Prints one JSON line (rank 0).  `value` is dense-equivalent TFLOPS of all ranks
+(4*B*H*N^2*d per call / device time); `ms_per_step` is milliseconds per call (max over
+ranks).  With N > 1 (torchrun) every rank runs its own independent call on its own inputs
+(heads never exchange data: weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from free_block_sparse_02_b200 import configs, gen  # noqa: E402
+
+METRIC = "SparsePR ms/call & dense-equiv TFLOPS at 22% density; % bf16 TC peak"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def workload_config(w, extra=None):
+    c = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "density": w.density, "s": w.s,
+         "n_kgroups": w.n_kgroups, "n_qgroups": w.n_qgroups, "P": w.P,
+         "probes": "stratified" if w.probe_mode else "uniform", "km_iters": w.km_iters, "km_tol": w.km_tol,
+         "generator": f"clustered Gaussian tiles {w.tile} on grid {w.grid}" + (" + 3D RoPE" if w.rope else "")}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ------------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={uuid}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------ CPU baseline
+def oracle_sample(w, budget_s: float, max_heads=None):
+    """Time the fp64 oracle on whole heads of the workload until `budget_s` is spent."""
+    from oracle import sparsepr_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        cores = os.cpu_count()
+    times = []
+    h = 0
+    max_heads = max_heads or w.H
+    while h < max_heads and (sum(times) < budget_s or not times):
+        Q, K, V = gen.make_qkv(w, heads=[(0, h)])
+        q, k, v = (gen.as_f64(x)[0, h] for x in (Q, K, V))
+        t0 = time.perf_counter()
+        O.call_head(q, k, v, w, h)
+        times.append(time.perf_counter() - t0)
+        h += 1
+    per_call_s = statistics.mean(times) * w.B * w.H
+    return {"value": w.dense_flops() / per_call_s / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+            "sample": f"{len(times)} of {w.B * w.H} heads of one call (fp64 NumPy oracle, whole per-head "
+                      f"call), mean {statistics.mean(times):.2f} s/head extrapolated x{w.B * w.H}",
+            "s_per_call": per_call_s}
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(w, 0.0, max_heads=1)
+    t0 = time.perf_counter()
+    runs = [oracle_sample(w, 0.0, max_heads=1) for _ in range(args.steps)]
+    wall = time.perf_counter() - t0
+    s_per_call = statistics.mean(r["s_per_call"] for r in runs)
+    val = w.dense_flops() / s_per_call / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": s_per_call * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, {"l2": "n/a (CPU)"}),
+            "cpu_baseline": {"kind": "oracle", "cores": runs[0]["cores"], "value": val, "unit": "TFLOPS",
+                             "sample": "each step: head 0 of the call through the fp64 NumPy oracle, "
+                                       f"extrapolated x{w.B * w.H} heads"},
+            "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s": wall}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------ GPU arm
+def run_ours(args, w, world, rank, local):
+    from free_block_sparse_02_b200 import _lib as S
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    S.load()
+    Qc, Kc, Vc = gen.make_qkv(w, variant=rank)
+    Q, K, V = Qc.to(dev), Kc.to(dev), Vc.to(dev)
+    op = S.SparsePR(w, device=dev)
+    O = torch.empty(Q.shape, dtype=Q.dtype, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        op(Q, K, V, O=O)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    st = op.stats()
+    pairs = sum(s["sparse_pairs"] for s in st)
+    realised = statistics.mean(s["density"] for s in st)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in kev:  # torch creates the CUDA event on first record; the library records it again
+        a.record(stream)
+        b.record(stream)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    launches0 = S.launch_count()
+    for i in range(args.steps):
+        flush.zero_()                         # L2 flush between timed steps, outside the events
+        op.set_kernel_events(*kev[i])
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    launches = S.launch_count() - launches0
+    clk = clocks.stop()
+    op.set_kernel_events(None, None)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    kern_ms = [a.elapsed_time(b) for a, b in kev]
+    ms = statistics.mean(step_ms)
+    kms = statistics.mean(kern_ms)
+    t = torch.tensor([ms, kms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max, kms_max = float(t[0]), float(t[1])
+
+    # end to end through the public API with host buffers (pinned), copies inside the region
+    Qh, Kh, Vh = Qc.pin_memory(), Kc.pin_memory(), Vc.pin_memory()
+    Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps + 1):
+        flush.zero_()
+        if i > 0:
+            e2e_ev[i - 1][0].record(stream)
+        Q.copy_(Qh, non_blocking=True)
+        K.copy_(Kh, non_blocking=True)
+        V.copy_(Vh, non_blocking=True)
+        op(Q, K, V, O=O)
+        Oh.copy_(O, non_blocking=True)
+        if i > 0:
+            e2e_ev[i - 1][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in e2e_ev)
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t[0])
+
+    if rank == 0:
+        pk = peaks()
+        flops = w.dense_flops()
+        value = world * flops / (ms_max * 1e-3) / 1e12
+        kflops = 4.0 * w.d * pairs
+        achieved = kflops / (kms_max * 1e-3) / 1e12
+        peak = pk["bf16_tflops"]
+        elt = Q.element_size()
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.dtype == configs.BF16 else "f32", "data": "synthetic",
+            "config": workload_config(w, {"l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
+                                          "realised_density": realised,
+                                          "parallelism": f"{world} independent calls, one per GPU"}),
+            "ms_per_call": ms_max,
+            "executed_tflops": world * (kflops + 4.0 * w.d * w.B * w.H * w.P * w.N) / (ms_max * 1e-3) / 1e12,
+            "kernel_ms": {"block_sparse_attention": kms_max},
+            "roofline": {"bound": "tensor", "kernel": "block-sparse attention", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{pk['source']} bf16 dense (burst)",
+                         "algorithmic": f"4*d*executed pairs = {kflops:.4g} flop per launch"},
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+                    "h2d_bytes_per_step": 3 * Q.numel() * elt, "d2h_bytes_per_step": O.numel() * O.element_size(),
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample(w, args.cpu_budget)
+            line["cpu_baseline"].pop("s_per_call", None)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", type=int, default=1, help="index into configs.WORKLOADS")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_env()
+    w = configs.workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, w, world, rank)
+    else:
+        run_ours(args, w, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

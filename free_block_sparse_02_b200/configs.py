@@ -53,7 +53,7 @@ class Workload:
     def n_tiles(self) -> int:
         T, Y, X = self.grid
         a, b, c = self.tile
-        return (T // a) * (Y // b) * (X // c)
+        return (-(-T // a)) * (-(-Y // b)) * (-(-X // c))
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)

@@ -1,0 +1,169 @@
+// Shared definitions of the SparsePR CUDA library: the workspace layout every kernel receives
+// by value, element conversions, warp reductions and launch checking.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <type_traits>
+#include <utility>
+
+#include "../../include/sparsepr.h"
+
+namespace sparsepr {
+
+constexpr int kMaxGroups = 1024;  // C_k, C_q upper bound (route rows fit one CTA's smem)
+constexpr int kMaxProbes = 4096;
+
+// Device status word values (a subset of sparsepr_status).
+constexpr int kDevOk = 0;
+constexpr int kDevNumeric = SPARSEPR_ERR_NUMERIC;
+constexpr int kDevTimeout = SPARSEPR_ERR_TIMEOUT;
+
+// Everything a kernel needs to find its data: sizes and device pointers carved from the
+// caller's workspace.  Arrays are head-major: head bh = b*H + h owns one contiguous slice.
+struct Layout {
+  int BH, H, N, d, s, Ck, Cq, P;
+  int dtype;            // SPARSEPR_F32 / SPARSEPR_BF16 of Q, K, V
+  int fixed_k;
+  int iters_cap;        // length of the per-iteration objective arrays
+  int probe_mode;
+  float density;
+  float km_tol;
+  double lambda;
+  uint64_t seed;
+  int n_gram_parts;     // N-chunks of the key Gram reduction
+
+  // status + per-head statistics
+  int* status;                    // [1]
+  sparsepr_head_stats* stats;     // [BH]
+
+  // key responses: metric M = Qs^T Qs / d and the key Gram for the objective constant
+  double* M;                      // [BH, d, d]
+  double* gram_part;              // [BH, n_gram_parts, d, d]
+  double* T0k;                    // [BH]  sum_t ||f_t||^2
+  double* T0q;                    // [BH]  sum_q ||r~_q||^2
+
+  // k-means shared scratch
+  int* init_ids;                  // [BH, max(Ck, Cq)]
+  int* fy;                        // [BH, N] Fisher-Yates slots
+  int* iters_run;                 // [BH, 2] iterations for keys / queries (run-time state)
+  int* stop_at;                   // [BH, 2] iteration at which the loop stopped
+  int* warm;                      // [1] 1 = warm start from stored centroids
+
+  // key k-means (features: keys with metric M)
+  double* kcent;                  // [BH, Ck, d]   key-space centroids
+  double* kW64;                   // [BH, Ck, d]   M c_j
+  float* kW32;                    // [BH, Ck, d]
+  double* kbias64;                // [BH, Ck]      c_j^T M c_j
+  float* kbias32;                 // [BH, Ck]
+  float* kwnorm;                  // [BH, Ck]      ||W_j||_2
+  double* ksum;                   // [BH, Ck, d]
+  int* kcount;                    // [BH, Ck]
+  int* klabel;                    // [BH, N]
+  double* kJ;                     // [BH, iters_cap]
+  int* krefined;                  // [BH]
+
+  // query responses and query k-means (features: RMS-normalised responses)
+  double* r64;                    // [BH, N, Ck]
+  float* r32;                     // [BH, N, Ck]
+  double* qcent;                  // [BH, Cq, Ck]
+  float* qW32;                    // [BH, Cq, Ck]
+  double* qbias64;                // [BH, Cq]
+  float* qbias32;                 // [BH, Cq]
+  float* qwnorm;                  // [BH, Cq]
+  double* qsum;                   // [BH, Cq, Ck]
+  int* qcount;                    // [BH, Cq]
+  int* qlabel;                    // [BH, N]
+  double* qJ;                     // [BH, iters_cap]
+  int* qrefined;                  // [BH]
+
+  // group-contiguous order (stable counting sort)
+  int* kperm;                     // [BH, N]   position -> token
+  int* kinv;                      // [BH, N]   token -> position
+  int* koff;                      // [BH, Ck+1]
+  int* qperm;
+  int* qinv;
+  int* qoff;                      // [BH, Cq+1]
+
+  // routing
+  unsigned char* route;           // [BH, Cq, Ck]
+  int* route_list;                // [BH, Cq, Ck]  kept key groups, ascending
+  int* route_cnt;                 // [BH, Cq]
+  int* route_keys;                // [BH, Cq]      keys visible to the group (sum of m_j)
+  int* tile_off;                  // [BH, Cq+1]    prefix of query tiles per group
+
+  // probes
+  int* probe_tok;                 // [BH, P]
+  double* probe_w;                // [BH, P]
+  int* probe_of;                  // [BH, N]  token -> probe index or -1
+
+  // permuted operands (input dtype) and outputs
+  void* Qp;                       // [BH, N, d]
+  void* Kp;
+  void* Vp;
+  void* Qprobe;                   // [BH, P, d]
+  float* Osp;                     // [BH, N, d]  permuted (query-group) order
+  float* Odense;                  // [BH, P, d]
+
+  // ridge
+  double* ridgeG;                 // [BH, d+1, d+1]
+  double* ridgeB;                 // [BH, d+1, d]
+  double* spanS;                  // [BH, d, d]   R^T W R
+  double* A64;                    // [BH, d+1, d]
+  float* A32;                     // [BH, d+1, d]
+};
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide sum of a double; every thread gets the result.  `red` needs blockDim/32 doubles.
+__device__ __forceinline__ double block_sum(double v, double* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  double t = 0.0;
+  for (int i = 0; i < nw; ++i) t += red[i];
+  return t;
+}
+
+__host__ __device__ inline size_t elt_size(int dtype) { return dtype == SPARSEPR_F32 ? 4 : 2; }
+
+// Kernels launched by this library since it was loaded (read by sparsepr_launch_count).
+extern std::atomic<long long> g_launches;
+
+// Every kernel of the library is launched through this helper, which counts the launch.
+template <typename... KArgs, typename... Args>
+inline void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   Args&&... args) {
+  kernel<<<grid, block, smem, st>>>(std::forward<Args>(args)...);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+}  // namespace sparsepr
+
+#define SPR_LAUNCH_CHECK()                                   \
+  do {                                                       \
+    cudaError_t e_ = cudaGetLastError();                     \
+    if (e_ != cudaSuccess) return SPARSEPR_ERR_CUDA;         \
+  } while (0)

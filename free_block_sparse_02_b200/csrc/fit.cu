@@ -1,0 +1,326 @@
+// Probe-Fitted Residual Reconstruction of the SparsePR operator.
+//
+// "Partition the Support, Reconstruct the Residual" (arXiv 2608.18484), abstract: "fit an
+// affine correction to the differences between their dense and sparse outputs using
+// weighted ridge regression.  The fitted map predicts a residual for each unprobed query,
+// which we add to its sparse output"; arXiv abstract: the correction acts "within the output
+// subspace observed in the probe residuals"; project page method column "Probe-Fitted
+// Residual Reconstruction".
+//
+// Per head, with X_p = [O_sp(p), 1], R_p = O_dense(p) - O_sp(p), W = diag(w):
+//   A = (X^T W X + lam I)^-1 X^T W R,   lam = 1e-3 tr(X^T W X)/(d+1) unless given,
+//   A <- A U U^T with U an orthonormal basis of span{R_p},
+//   O_i = O_sp,i + [O_sp,i, 1] A for unprobed rows, O_dense for probe rows.
+// The normal equations and the span basis are solved in fp64 by one CTA per head.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace sparsepr {
+
+constexpr int kRidgeRows = 8;    // rows of G/B/S per block
+constexpr int kRidgeChunk = 32;  // probes staged per step
+
+// G = X^T W X ((d+1)^2), B = X^T W R ((d+1) x d), S = R^T W R (d x d): rows
+// [8 y, 8 y + 8) of each, summed over the probes in a fixed order.
+__global__ void __launch_bounds__(256) ridge_gram_kernel(Layout L) {
+  extern __shared__ double shr[];
+  const int bh = blockIdx.x, d = L.d, n1 = d + 1, P = L.P, tid = threadIdx.x;
+  double* X = shr;                       // [32][n1]
+  double* R = X + kRidgeChunk * n1;      // [32][d]
+  double* w = R + kRidgeChunk * d;       // [32]
+  const int a0 = blockIdx.y * kRidgeRows;
+  // outputs owned by this thread: index o over [8 rows] x [n1 (G) + d (B) + d (S)]
+  const int per_row = n1 + 2 * d;
+  const int n_out = kRidgeRows * per_row;
+  double acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.0;
+  const int* tok = L.probe_tok + (size_t)bh * P;
+  const int* qinv = L.qinv + (size_t)bh * L.N;
+  const float* osp = L.Osp + (size_t)bh * L.N * d;
+  const float* od = L.Odense + (size_t)bh * P * d;
+  for (int p0 = 0; p0 < P; p0 += kRidgeChunk) {
+    const int np = min(kRidgeChunk, P - p0);
+    __syncthreads();
+    for (int e = tid; e < kRidgeChunk * n1; e += 256) {
+      const int p = e / n1, a = e % n1;
+      double v = 0.0;
+      if (p < np) v = a < d ? (double)osp[(size_t)qinv[tok[p0 + p]] * d + a] : 1.0;
+      X[e] = v;
+    }
+    for (int e = tid; e < kRidgeChunk * d; e += 256) {
+      const int p = e / d, a = e % d;
+      R[e] = p < np ? (double)od[(size_t)(p0 + p) * d + a] - (double)osp[(size_t)qinv[tok[p0 + p]] * d + a] : 0.0;
+    }
+    if (tid < kRidgeChunk) w[tid] = tid < np ? L.probe_w[(size_t)bh * P + p0 + tid] : 0.0;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int o = tid + i * 256;
+      if (o >= n_out) break;
+      const int rr = o / per_row, c = o % per_row, a = a0 + rr;
+      if (a >= n1) continue;
+      double s = 0.0;
+      if (c < n1) {
+        for (int p = 0; p < np; ++p) s += w[p] * X[p * n1 + a] * X[p * n1 + c];
+      } else if (c < n1 + d) {
+        const int cc = c - n1;
+        for (int p = 0; p < np; ++p) s += w[p] * X[p * n1 + a] * R[p * d + cc];
+      } else {
+        const int cc = c - n1 - d;
+        if (a < d)
+          for (int p = 0; p < np; ++p) s += w[p] * R[p * d + a] * R[p * d + cc];
+      }
+      acc[i] += s;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int o = tid + i * 256;
+    if (o >= n_out) break;
+    const int rr = o / per_row, c = o % per_row, a = a0 + rr;
+    if (a >= n1) continue;
+    if (c < n1) L.ridgeG[((size_t)bh * n1 + a) * n1 + c] = acc[i];
+    else if (c < n1 + d) L.ridgeB[((size_t)bh * n1 + a) * d + (c - n1)] = acc[i];
+    else if (a < d) L.spanS[((size_t)bh * d + a) * d + (c - n1 - d)] = acc[i];
+  }
+}
+
+// In-place lower Cholesky of the n x n matrix in shared memory; false if a pivot is not > 0.
+__device__ bool chol_smem(double* G, int n, int ld) {
+  __shared__ int fail;
+  if (threadIdx.x == 0) fail = 0;
+  __syncthreads();
+  for (int k = 0; k < n; ++k) {
+    if (threadIdx.x == 0) {
+      const double piv = G[k * ld + k];
+      if (!(piv > 0.0) || !isfinite(piv)) fail = 1;
+      else G[k * ld + k] = sqrt(piv);
+    }
+    __syncthreads();
+    if (fail) return false;
+    const double lkk = G[k * ld + k];
+    for (int i = k + 1 + threadIdx.x; i < n; i += blockDim.x) G[i * ld + k] /= lkk;
+    __syncthreads();
+    const int m = n - k - 1;
+    for (int e = threadIdx.x; e < m * m; e += blockDim.x) {
+      const int i = k + 1 + e / m, j = k + 1 + e % m;
+      if (j <= i) G[i * ld + j] -= G[i * ld + k] * G[j * ld + k];
+    }
+    __syncthreads();
+  }
+  return true;
+}
+
+// One CTA per head: lam, Cholesky with up to three x10 jitter retries, the d right-hand sides,
+// then the residual-span basis by column-pivoted Gram-Schmidt on S = R^T W R and A <- A U U^T.
+__global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
+  extern __shared__ double shs[];
+  const int bh = blockIdx.x, d = L.d, n1 = d + 1, tid = threadIdx.x;
+  double* G = shs;  // [n1][n1], later S [d][d]
+  __shared__ double red[8];
+  __shared__ int s_piv;
+  __shared__ double s_norm;
+  const double* Gg = L.ridgeG + (size_t)bh * n1 * n1;
+  double* A = L.A64 + (size_t)bh * n1 * d;
+  sparsepr_head_stats& st = L.stats[bh];
+
+  if (L.P == 0) {
+    for (int e = tid; e < n1 * d; e += blockDim.x) {
+      A[e] = 0.0;
+      L.A32[(size_t)bh * n1 * d + e] = 0.f;
+    }
+    if (tid == 0) {
+      st.lambda = 0.0;
+      st.fit_retries = 0;
+      st.span_rank = 0;
+    }
+    return;
+  }
+  double tr = 0.0;
+  for (int i = tid; i < n1; i += blockDim.x) tr += Gg[i * n1 + i];
+  tr = block_sum(tr, red);
+  double lam = L.lambda >= 0.0 ? L.lambda : 1e-3 * tr / n1;
+  int retries = 0;
+  bool ok = false;
+  for (; retries <= 3; ++retries) {
+    for (int e = tid; e < n1 * n1; e += blockDim.x) G[e] = Gg[e] + ((e / n1) == (e % n1) ? lam : 0.0);
+    __syncthreads();
+    ok = chol_smem(G, n1, n1);
+    if (ok) break;
+    lam = lam > 0.0 ? lam * 10.0 : (tr > 0.0 ? 1e-12 * tr / n1 : 1e-30);
+  }
+  if (!ok) {
+    if (tid == 0) {
+      atomicCAS(L.status, kDevOk, kDevNumeric);
+      st.fit_retries = retries;
+    }
+    for (int e = tid; e < n1 * d; e += blockDim.x) {
+      A[e] = 0.0;
+      L.A32[(size_t)bh * n1 * d + e] = 0.f;
+    }
+    return;
+  }
+  // solve L L^T x = b for every column of B; A is the scratch of each thread's column
+  const double* Bg = L.ridgeB + (size_t)bh * n1 * d;
+  for (int c = tid; c < d; c += blockDim.x) {
+    for (int i = 0; i < n1; ++i) {
+      double v = Bg[i * d + c];
+      for (int k = 0; k < i; ++k) v -= G[i * n1 + k] * A[k * d + c];
+      A[i * d + c] = v / G[i * n1 + i];
+    }
+    for (int i = n1 - 1; i >= 0; --i) {
+      double v = A[i * d + c];
+      for (int k = i + 1; k < n1; ++k) v -= G[k * n1 + i] * A[k * d + c];
+      A[i * d + c] = v / G[i * n1 + i];
+    }
+  }
+  __syncthreads();
+  // span basis: columns of S (they span range(S) = span{R_p}); pivoted Gram-Schmidt in place
+  double* S = G;
+  const double* Sg = L.spanS + (size_t)bh * d * d;
+  for (int e = tid; e < d * d; e += blockDim.x) S[e] = Sg[e];  // S[i*d + c]: column c, entry i
+  __shared__ double cn[128];
+  __shared__ int used[128];
+  __syncthreads();
+  for (int c = tid; c < d; c += blockDim.x) {
+    double s = 0.0;
+    for (int i = 0; i < d; ++i) s += S[i * d + c] * S[i * d + c];
+    cn[c] = s;
+    used[c] = 0;
+  }
+  __syncthreads();
+  __shared__ double s_tol;
+  if (tid == 0) {
+    double mx = 0.0;
+    for (int c = 0; c < d; ++c) mx = fmax(mx, cn[c]);
+    // column norms of S scale like eigenvalue^2; the span keeps eigenvalues > 1e-10 of the top
+    s_tol = mx * 1e-20;
+  }
+  __syncthreads();
+  int rank = 0;
+  int basis[128];
+  for (int step = 0; step < d; ++step) {
+    if (tid == 0) {
+      int best = -1;
+      double bv = 0.0;
+      for (int c = 0; c < d; ++c)
+        if (!used[c] && cn[c] > bv) {
+          bv = cn[c];
+          best = c;
+        }
+      s_piv = (best >= 0 && bv > s_tol && bv > 0.0) ? best : -1;
+      if (s_piv >= 0) {
+        used[s_piv] = 1;
+        double s = 0.0;
+        for (int i = 0; i < d; ++i) s += S[i * d + s_piv] * S[i * d + s_piv];
+        s_norm = sqrt(s);
+      }
+    }
+    __syncthreads();
+    const int pv = s_piv;
+    if (pv < 0) break;
+    for (int i = tid; i < d; i += blockDim.x) S[i * d + pv] /= s_norm;
+    __syncthreads();
+    for (int c = tid; c < d; c += blockDim.x) {
+      if (used[c]) continue;
+      double dot = 0.0;
+      for (int i = 0; i < d; ++i) dot += S[i * d + pv] * S[i * d + c];
+      double s = 0.0;
+      for (int i = 0; i < d; ++i) {
+        const double v = S[i * d + c] - dot * S[i * d + pv];
+        S[i * d + c] = v;
+        s += v * v;
+      }
+      cn[c] = s;
+    }
+    basis[rank++] = pv;
+    __syncthreads();
+  }
+  // A <- (A U) U^T, one row of A per thread
+  for (int a = tid; a < n1; a += blockDim.x) {
+    double t[128];
+    for (int r = 0; r < rank; ++r) {
+      double s = 0.0;
+      for (int i = 0; i < d; ++i) s += A[a * d + i] * S[i * d + basis[r]];
+      t[r] = s;
+    }
+    for (int i = 0; i < d; ++i) {
+      double s = 0.0;
+      for (int r = 0; r < rank; ++r) s += t[r] * S[i * d + basis[r]];
+      A[a * d + i] = s;
+      L.A32[((size_t)bh * n1 + a) * d + i] = (float)s;
+    }
+  }
+  if (tid == 0) {
+    st.lambda = lam;
+    st.fit_retries = retries;
+    st.span_rank = rank;
+  }
+}
+
+// a10: O[token] = O_sp + [O_sp, 1] A for unprobed rows, O_dense for probe rows; 64 permuted
+// rows per block, written back to original token order.
+template <typename To, int D>
+__global__ void __launch_bounds__(256) apply_kernel(Layout L, To* __restrict__ O) {
+  extern __shared__ float sha[];
+  float* As = sha;                  // [(D+1)][D]
+  float* Xs = As + (D + 1) * D;     // [64][D]
+  const int bh = blockIdx.y, tid = threadIdx.x;
+  const int r0 = blockIdx.x * 64, nr = min(64, L.N - r0);
+  const float* A = L.A32 + (size_t)bh * (D + 1) * D;
+  for (int e = tid; e < (D + 1) * D; e += 256) As[e] = A[e];
+  const float* osp = L.Osp + ((size_t)bh * L.N + r0) * D;
+  for (int e = tid; e < 64 * D; e += 256) Xs[e] = e / D < nr ? osp[e] : 0.f;
+  __syncthreads();
+  const int* perm = L.qperm + (size_t)bh * L.N;
+  const int* pof = L.probe_of + (size_t)bh * L.N;
+  const float* od = L.Odense + (size_t)bh * L.P * D;
+  for (int e = tid; e < nr * D; e += 256) {
+    const int r = e / D, c = e % D;
+    const int t = perm[r0 + r];
+    const int p = pof[t];
+    float v;
+    if (p >= 0) {
+      v = od[(size_t)p * D + c];
+    } else {
+      float acc = As[D * D + c];
+      const float* x = Xs + r * D;
+#pragma unroll 8
+      for (int a = 0; a < D; ++a) acc = fmaf(x[a], As[a * D + c], acc);
+      v = x[c] + acc;
+    }
+    To* orow = O + ((size_t)bh * L.N + t) * D;
+    if constexpr (std::is_same<To, float>::value) orow[c] = v;
+    else orow[c] = __float2bfloat16_rn(v);
+  }
+}
+
+template <typename To, int D>
+static sparsepr_status launch_apply(const Layout& L, void* O, cudaStream_t st) {
+  const size_t smem = (size_t)((D + 1) * D + 64 * D) * 4;
+  cudaFuncSetAttribute(apply_kernel<To, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  launch(apply_kernel<To, D>, dim3((L.N + 63) / 64, L.BH), 256, smem, st, L, (To*)O);
+  SPR_LAUNCH_CHECK();
+  return SPARSEPR_OK;
+}
+
+sparsepr_status launch_fit_apply(const Layout& L, void* O, int out_dtype, cudaStream_t st) {
+  const int d = L.d, n1 = d + 1;
+  if (L.P > 0) {
+    const size_t gsm = (size_t)(kRidgeChunk * n1 + kRidgeChunk * d + kRidgeChunk) * sizeof(double);
+    cudaFuncSetAttribute(ridge_gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm);
+    launch(ridge_gram_kernel, dim3(L.BH, (n1 + kRidgeRows - 1) / kRidgeRows), 256, gsm, st, L);
+  }
+  const size_t ssm = (size_t)n1 * n1 * sizeof(double);
+  cudaFuncSetAttribute(ridge_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
+  launch(ridge_solve_kernel, L.BH, 256, ssm, st, L);
+  SPR_LAUNCH_CHECK();
+  if (out_dtype == SPARSEPR_F32)
+    return d == 64 ? launch_apply<float, 64>(L, O, st) : launch_apply<float, 128>(L, O, st);
+  return d == 64 ? launch_apply<__nv_bfloat16, 64>(L, O, st) : launch_apply<__nv_bfloat16, 128>(L, O, st);
+}
+
+}  // namespace sparsepr

@@ -1,0 +1,899 @@
+// Response-Coupled Partitioning, routing and probe choice of the SparsePR operator.
+//
+// "Partition the Support, Reconstruct the Residual" (arXiv 2608.18484), abstract: keys are
+// grouped by their responses to sampled queries (paired K/V groups), queries by their
+// responses to the key-group centroids (shared sparse routing); project page "SparsePR:
+// Training-Free Sparse Attention for Video Generation", method pipeline steps 01-03.
+//
+// Key responses f_t = Q_s k_t / sqrt(d) (s-dimensional) are never materialised: for a group
+// mean mu_j = Q_s c_j / sqrt(d) (c_j = mean of the member keys), linearity gives
+//   ||f_t - mu_j||^2 = (k_t - c_j)^T M (k_t - c_j),   M = Q_s^T Q_s / d,
+// so the assignment is argmin_j ( c_j^T M c_j - 2 k_t . (M c_j) ) over d-dimensional keys.
+//
+// Exactness: scores are computed in fp32 with a rigorous rounding bound; a point whose best
+// two scores are within that bound is re-decided over all groups in fp64, so labels agree
+// with an fp64 evaluation except at ties far below the fp32 resolution.  Group sums are fp64.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace sparsepr {
+
+// ------------------------------------------------------------------------------------------
+// a1 + a2 prologue: M = Q_s^T Q_s / d (fp64, exact products) per head.
+// ------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void metric_kernel(Layout L, const T* __restrict__ Q) {
+  const int bh = blockIdx.x, a = blockIdx.y, b = threadIdx.x;
+  if (b >= L.d) return;
+  const T* q = Q + (size_t)bh * L.N * L.d;
+  double acc = 0.0;
+  for (int i = 0; i < L.s; ++i) {
+    const long long row = ((2LL * i + 1) * L.N) / (2LL * L.s);
+    acc += (double)to_f32(q[row * L.d + a]) * (double)to_f32(q[row * L.d + b]);
+  }
+  L.M[((size_t)bh * L.d + a) * L.d + b] = acc / L.d;
+}
+
+// Partial key Gram G = sum_t k_t k_t^T over one N-chunk (fp64).  Used only for the constant
+// sum_t ||f_t||^2 = <M, G> of the k-means objective.
+template <typename T>
+__global__ void __launch_bounds__(256) gram_part_kernel(Layout L, const T* __restrict__ K) {
+  extern __shared__ double sh_rows[];  // [32][d]
+  const int bh = blockIdx.x, part = blockIdx.y, d = L.d;
+  const int chunk = (L.N + L.n_gram_parts - 1) / L.n_gram_parts;
+  const int t0 = part * chunk, t1 = min(L.N, t0 + chunk);
+  const T* k = K + (size_t)bh * L.N * d;
+  const int ne = d * d;
+  double acc[64];
+#pragma unroll
+  for (int i = 0; i < 64; ++i) acc[i] = 0.0;
+  for (int base = t0; base < t1; base += 32) {
+    const int nr = min(32, t1 - base);
+    __syncthreads();
+    for (int e = threadIdx.x; e < nr * d; e += blockDim.x)
+      sh_rows[e] = (double)to_f32(k[(size_t)(base + e / d) * d + (e % d)]);
+    __syncthreads();
+    for (int r = 0; r < nr; ++r) {
+      const double* row = sh_rows + r * d;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const int e = threadIdx.x + i * 256;
+        if (e < ne) acc[i] += row[e / d] * row[e % d];
+      }
+    }
+  }
+  double* out = L.gram_part + ((size_t)bh * L.n_gram_parts + part) * ne;
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    const int e = threadIdx.x + i * 256;
+    if (e < ne) out[e] = acc[i];
+  }
+}
+
+__global__ void __launch_bounds__(256) gram_reduce_kernel(Layout L) {
+  __shared__ double red[8];
+  const int bh = blockIdx.x, ne = L.d * L.d;
+  double v = 0.0;
+  for (int e = threadIdx.x; e < ne; e += blockDim.x) {
+    double g = 0.0;
+    for (int p = 0; p < L.n_gram_parts; ++p) g += L.gram_part[((size_t)bh * L.n_gram_parts + p) * ne + e];
+    v += g * L.M[(size_t)bh * ne + e];
+  }
+  v = block_sum(v, red);
+  if (threadIdx.x == 0) L.T0k[bh] = v;
+}
+
+// ------------------------------------------------------------------------------------------
+// k-means initial points: SplitMix64 (Steele, Lea & Flood 2014) partial Fisher-Yates.
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t splitmix64_next(uint64_t& state) {
+  state += 0x9E3779B97F4A7C15ULL;
+  uint64_t z = state;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+  return z ^ (z >> 31);
+}
+
+// One thread per head.  The slots touched by C swaps live in a shared-memory hash map
+// (slot -> value), so the identity array of N slots is never written.
+__global__ void km_draw_kernel(Layout L, int stage, int C) {
+  constexpr int kTab = 4096;  // >= 2 * 2 * kMaxGroups
+  __shared__ int keys[kTab];
+  __shared__ int vals[kTab];
+  const int bh = blockIdx.x;
+  for (int i = threadIdx.x; i < kTab; i += blockDim.x) keys[i] = -1;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  auto slot_ref = [&](int slot) -> int* {
+    unsigned h = ((unsigned)slot * 2654435761u) >> 20;  // 12 bits
+    while (true) {
+      if (keys[h] == slot) return &vals[h];
+      if (keys[h] == -1) {
+        keys[h] = slot;
+        vals[h] = slot;
+        return &vals[h];
+      }
+      h = (h + 1) & (kTab - 1);
+    }
+  };
+  uint64_t state = L.seed + 2ULL * (uint64_t)bh + (uint64_t)stage;
+  const uint64_t n = (uint64_t)L.N;
+  int* out = L.init_ids + (size_t)bh * max(L.Ck, L.Cq);
+  for (int i = 0; i < C; ++i) {
+    const uint64_t r = splitmix64_next(state);
+    const int j = i + (int)(r % (n - (uint64_t)i));
+    int* pi = slot_ref(i);
+    int* pj = slot_ref(j);
+    const int vi = *pi, vj = *pj;
+    *pi = vj;
+    *pj = vi;
+    out[i] = vj;
+  }
+}
+
+template <typename T>
+__global__ void kcent_init_kernel(Layout L, const T* __restrict__ K) {
+  const int bh = blockIdx.x, j = blockIdx.y, a = threadIdx.x;
+  if (a >= L.d) return;
+  const int t = L.init_ids[(size_t)bh * max(L.Ck, L.Cq) + j];
+  L.kcent[((size_t)bh * L.Ck + j) * L.d + a] = (double)to_f32(K[((size_t)bh * L.N + t) * L.d + a]);
+}
+
+__global__ void qcent_init_kernel(Layout L) {
+  const int bh = blockIdx.x, g = blockIdx.y;
+  const int t = L.init_ids[(size_t)bh * max(L.Ck, L.Cq) + g];
+  for (int a = threadIdx.x; a < L.Ck; a += blockDim.x)
+    L.qcent[((size_t)bh * L.Cq + g) * L.Ck + a] = L.r64[((size_t)bh * L.N + t) * L.Ck + a];
+}
+
+// J arrays start at the objective constant; the stop marker starts at the iteration limit.
+__global__ void km_reset_kernel(Layout L, int which, int iters) {
+  const int bh = blockIdx.x;
+  double* J = (which == 0 ? L.kJ : L.qJ) + (size_t)bh * L.iters_cap;
+  const double c = which == 0 ? L.T0k[bh] : L.T0q[bh];
+  for (int i = threadIdx.x; i < L.iters_cap; i += blockDim.x) J[i] = c;
+  if (threadIdx.x == 0) {
+    L.stop_at[bh * 2 + which] = iters;
+    (which == 0 ? L.krefined : L.qrefined)[bh] = 0;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Lloyd step 1 of iteration `it`: centroid update from the sums of assignment it-1, the stop
+// test, then the score weights of the next assignment.  Grid (BH, C), one block per group.
+//   keys:    c_j (key space), W_j = M c_j, bias_j = c_j^T M c_j
+//   queries: nu_g (response space), W_g = nu_g, bias_g = ||nu_g||^2
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ bool km_should_stop(const double* J, int it, int iters, float tol) {
+  if (it >= iters) return true;
+  if (it >= 2 && tol >= 0.f) {
+    const double Jp = J[it - 2], Jc = J[it - 1];
+    return Jp - Jc <= (double)tol * Jp;
+  }
+  return false;
+}
+
+__global__ void __launch_bounds__(128) kprep_kernel(Layout L, int it, int iters) {
+  __shared__ double c[128];
+  __shared__ double red[4];
+  const int bh = blockIdx.x, j = blockIdx.y, a = threadIdx.x, d = L.d;
+  if (it > L.stop_at[bh * 2 + 0]) return;
+  double* cj = L.kcent + ((size_t)bh * L.Ck + j) * d;
+  const size_t gj = (size_t)bh * L.Ck + j;
+  if (it > 0) {
+    const int cnt = L.kcount[gj];
+    if (cnt > 0 && a < d) cj[a] = L.ksum[gj * d + a] / (double)cnt;
+  }
+  if (km_should_stop(L.kJ + (size_t)bh * L.iters_cap, it, iters, L.km_tol)) {
+    if (a == 0 && j == 0) L.stop_at[bh * 2 + 0] = it;
+    return;
+  }
+  if (a < d) c[a] = cj[a];
+  __syncthreads();
+  double w = 0.0;
+  if (a < d) {
+    const double* Mr = L.M + ((size_t)bh * d + a) * d;
+    for (int b = 0; b < d; ++b) w += Mr[b] * c[b];
+    L.kW64[gj * d + a] = w;
+    L.kW32[gj * d + a] = (float)w;
+    L.ksum[gj * d + a] = 0.0;
+  }
+  const double bias = block_sum(a < d ? c[a] * w : 0.0, red);
+  const double wn = block_sum(a < d ? w * w : 0.0, red);
+  if (a == 0) {
+    L.kbias64[gj] = bias;
+    L.kbias32[gj] = (float)bias;
+    L.kcount[gj] = 0;
+    L.kwnorm[gj] = (float)sqrt(wn);
+  }
+}
+
+__global__ void __launch_bounds__(128) qprep_kernel(Layout L, int it, int iters) {
+  __shared__ double red[4];
+  const int bh = blockIdx.x, g = blockIdx.y, D = L.Ck;
+  if (it > L.stop_at[bh * 2 + 1]) return;
+  const size_t gg = (size_t)bh * L.Cq + g;
+  double* nu = L.qcent + gg * D;
+  if (it > 0) {
+    const int cnt = L.qcount[gg];
+    if (cnt > 0)
+      for (int a = threadIdx.x; a < D; a += blockDim.x) nu[a] = L.qsum[gg * D + a] / (double)cnt;
+  }
+  if (km_should_stop(L.qJ + (size_t)bh * L.iters_cap, it, iters, L.km_tol)) {
+    if (threadIdx.x == 0 && g == 0) L.stop_at[bh * 2 + 1] = it;
+    return;
+  }
+  double nn = 0.0;
+  for (int a = threadIdx.x; a < D; a += blockDim.x) {
+    const double v = nu[a];
+    nn += v * v;
+    L.qW32[gg * D + a] = (float)v;
+    L.qsum[gg * D + a] = 0.0;
+  }
+  nn = block_sum(nn, red);
+  if (threadIdx.x == 0) {
+    L.qbias64[gg] = nn;
+    L.qbias32[gg] = (float)nn;
+    L.qcount[gg] = 0;
+    L.qwnorm[gg] = (float)sqrt(nn);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Lloyd step 2: assignment of 64 points per block against all groups, with fp64 sums.
+// Thread (pg, cg) = (tid / 16, tid % 16) scores points 4pg..4pg+3 against groups cg + 16i of
+// the current 64-group chunk.  Feature rows: keys (d dims, exact in fp32 and fp64) or the
+// normalised responses (C_k dims; fp32 copy for scoring, fp64 for tie-breaks and sums).
+// ------------------------------------------------------------------------------------------
+struct KeyFeat {};
+struct QueryFeat {};
+
+constexpr int kAsgPts = 64;
+constexpr int kAsgChunk = 64;
+
+template <typename T, typename Feat>
+__global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* __restrict__ K, int it) {
+  constexpr bool kKeys = std::is_same<Feat, KeyFeat>::value;
+  const int bh = blockIdx.y;
+  const int which = kKeys ? 0 : 1;
+  if (it >= L.stop_at[bh * 2 + which]) return;
+  const int D = kKeys ? L.d : L.Ck;
+  const int C = kKeys ? L.Ck : L.Cq;
+  const int DP = D + 1;
+  const int p0 = blockIdx.x * kAsgPts;
+  const int np = min(kAsgPts, L.N - p0);
+  if (np <= 0) return;
+
+  const float* W32 = kKeys ? L.kW32 + (size_t)bh * C * D : L.qW32 + (size_t)bh * C * D;
+  const float* B32 = kKeys ? L.kbias32 + (size_t)bh * C : L.qbias32 + (size_t)bh * C;
+  const double* W64 = kKeys ? L.kW64 + (size_t)bh * C * D : L.qcent + (size_t)bh * C * D;
+  const double* B64 = kKeys ? L.kbias64 + (size_t)bh * C : L.qbias64 + (size_t)bh * C;
+  const float* WN = kKeys ? L.kwnorm + (size_t)bh * C : L.qwnorm + (size_t)bh * C;
+
+  extern __shared__ float smem[];
+  float* Xs = smem;                        // [64][DP]
+  float* Ws = Xs + kAsgPts * DP;           // [64][DP]
+  float* Bs = Ws + kAsgChunk * DP;         // [64]
+  float* xnorm = Bs + kAsgChunk;           // [64]
+  int* lab = (int*)(xnorm + kAsgPts);      // [64]
+  int* order = lab + kAsgPts;              // [64]
+  double* a64 = (double*)(order + kAsgPts);  // [64]
+  __shared__ float s_wmax, s_bmax;
+  __shared__ int s_refine[kAsgPts];
+  __shared__ double red[8];
+
+  const int tid = threadIdx.x;
+  // features
+  for (int e = tid; e < kAsgPts * D; e += 256) {
+    const int p = e / D, a = e % D;
+    float v = 0.f;
+    if (p < np) {
+      if constexpr (kKeys) v = to_f32(K[((size_t)bh * L.N + p0 + p) * D + a]);
+      else v = L.r32[((size_t)bh * L.N + p0 + p) * D + a];
+    }
+    Xs[p * DP + a] = v;
+  }
+  if (tid == 0) {
+    float wm = 0.f, bm = 0.f;
+    for (int j = 0; j < C; ++j) {
+      wm = fmaxf(wm, WN[j]);
+      bm = fmaxf(bm, fabsf(B32[j]));
+    }
+    s_wmax = wm;
+    s_bmax = bm;
+  }
+  __syncthreads();
+  if (tid < kAsgPts) {
+    float s = 0.f;
+    for (int a = 0; a < D; ++a) s += Xs[tid * DP + a] * Xs[tid * DP + a];
+    xnorm[tid] = sqrtf(s);
+  }
+
+  const int pg = tid >> 4, cg = tid & 15;
+  float b1[4], b2[4];
+  int i1[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    b1[r] = INFINITY;
+    b2[r] = INFINITY;
+    i1[r] = 0x7fffffff;
+  }
+  for (int c0 = 0; c0 < C; c0 += kAsgChunk) {
+    const int nc = min(kAsgChunk, C - c0);
+    __syncthreads();
+    for (int e = tid; e < kAsgChunk * D; e += 256) {
+      const int j = e / D, a = e % D;
+      Ws[j * DP + a] = j < nc ? W32[(size_t)(c0 + j) * D + a] : 0.f;
+    }
+    if (tid < kAsgChunk) Bs[tid] = tid < nc ? B32[c0 + tid] : 0.f;
+    __syncthreads();
+    float acc[4][4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[r][i] = 0.f;
+    for (int a = 0; a < D; ++a) {
+      float x[4], w[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) x[r] = Xs[(pg * 4 + r) * DP + a];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w[i] = Ws[(cg + 16 * i) * DP + a];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[r][i] = fmaf(x[r], w[i], acc[r][i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = cg + 16 * i;
+      if (j >= nc) continue;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float sc = Bs[j] - 2.f * acc[r][i];
+        const int gj = c0 + j;
+        if (sc < b1[r] || (sc == b1[r] && gj < i1[r])) {
+          b2[r] = b1[r];
+          b1[r] = sc;
+          i1[r] = gj;
+        } else if (sc < b2[r]) {
+          b2[r] = sc;
+        }
+      }
+    }
+  }
+  // merge the 16 partial top-2 lists of each point (lanes of one half-warp)
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) {
+      const float ob1 = __shfl_xor_sync(0xffffffffu, b1[r], o);
+      const float ob2 = __shfl_xor_sync(0xffffffffu, b2[r], o);
+      const int oi1 = __shfl_xor_sync(0xffffffffu, i1[r], o);
+      if (ob1 < b1[r] || (ob1 == b1[r] && oi1 < i1[r])) {
+        b2[r] = fminf(b1[r], ob2);
+        b1[r] = ob1;
+        i1[r] = oi1;
+      } else {
+        b2[r] = fminf(b2[r], ob1);
+      }
+    }
+  }
+  const float u = 5.9604645e-8f;  // 2^-24
+  if (cg == 0) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int p = pg * 4 + r;
+      const float delta = 4.f * (D + 2) * u * xnorm[p] * s_wmax + 2.f * u * s_bmax;
+      lab[p] = (i1[r] >= 0 && i1[r] < C) ? i1[r] : 0;  // non-finite scores never yield a bad label
+      s_refine[p] = (p < np) && !(b2[r] - b1[r] > 2.f * delta);
+    }
+  }
+  __syncthreads();
+
+  // fp64 re-decision of points whose best two scores are within the rounding bound, and the
+  // exact score of every chosen group (for the objective).
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int p = warp; p < np; p += 8) {
+    const size_t row = (size_t)bh * L.N + p0 + p;
+    auto xval = [&](int a) -> double {
+      if constexpr (kKeys) return (double)to_f32(K[row * D + a]);
+      else return L.r64[row * D + a];
+    };
+    int best = lab[p];
+    double bestv;
+    if (s_refine[p]) {
+      bestv = INFINITY;
+      best = 0x7fffffff;
+      for (int j = 0; j < C; ++j) {
+        double dot = 0.0;
+        for (int a = lane; a < D; a += 32) dot += xval(a) * W64[(size_t)j * D + a];
+        dot = warp_sum(dot);
+        const double sc = B64[j] - 2.0 * dot;
+        if (sc < bestv) {  // ascending j: strict < keeps the lowest index on ties
+          bestv = sc;
+          best = j;
+        }
+      }
+    } else {
+      double dot = 0.0;
+      for (int a = lane; a < D; a += 32) dot += xval(a) * W64[(size_t)best * D + a];
+      dot = warp_sum(dot);
+      bestv = B64[best] - 2.0 * dot;
+    }
+    if (lane == 0) {
+      lab[p] = (best >= 0 && best < C) ? best : 0;
+      a64[p] = bestv;
+    }
+  }
+  __syncthreads();
+  // labels out, objective, refined count
+  int* labels = (kKeys ? L.klabel : L.qlabel) + (size_t)bh * L.N;
+  if (tid < np) labels[p0 + tid] = lab[tid];
+  const double jsum = block_sum(tid < np ? a64[tid] : 0.0, red);
+  int nref = 0;
+  if (tid < np) nref = s_refine[tid];
+  nref = __syncthreads_count(nref);
+  if (tid == 0) {
+    atomicAdd((kKeys ? L.kJ : L.qJ) + (size_t)bh * L.iters_cap + it, jsum);
+    if (nref) atomicAdd((kKeys ? L.krefined : L.qrefined) + bh, nref);
+  }
+  // stable order of the block's points by label, then one fp64 atomic per (run, dim)
+  if (tid < np) {
+    const int l = lab[tid];
+    int rk = 0;
+    for (int q = 0; q < np; ++q) {
+      const int lq = lab[q];
+      rk += (lq < l) || (lq == l && q < tid);
+    }
+    order[rk] = tid;
+  }
+  __syncthreads();
+  double* sums = (kKeys ? L.ksum : L.qsum) + (size_t)bh * C * D;
+  int* counts = (kKeys ? L.kcount : L.qcount) + (size_t)bh * C;
+  for (int a = tid; a < D; a += 256) {
+    double acc = 0.0;
+    for (int q = 0; q < np; ++q) {
+      const int p = order[q];
+      const size_t row = (size_t)bh * L.N + p0 + p;
+      double v;
+      if constexpr (kKeys) v = (double)to_f32(K[row * D + a]);
+      else v = L.r64[row * D + a];
+      acc += v;
+      if (q == np - 1 || lab[order[q + 1]] != lab[p]) {
+        atomicAdd(sums + (size_t)lab[p] * D + a, acc);
+        acc = 0.0;
+      }
+    }
+  }
+  if (tid == 0) {
+    int run = 0;
+    for (int q = 0; q < np; ++q) {
+      ++run;
+      const int l = lab[order[q]];
+      if (q == np - 1 || lab[order[q + 1]] != l) {
+        atomicAdd(counts + l, run);
+        run = 0;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// a3: query responses r_q = q . c_j / sqrt(d) (fp64) and per-query RMS normalisation
+// (Table D.1, "Per query RMS"): r~ = r / sqrt(mean_j r_j^2 + 1e-12).  32 queries per block.
+// ------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) qresp_kernel(Layout L, const T* __restrict__ Q) {
+  extern __shared__ double shq[];
+  const int d = L.d, Ck = L.Ck, bh = blockIdx.y;
+  const int p0 = blockIdx.x * 32, np = min(32, L.N - p0);
+  double* qs = shq;                 // [32][d+1]
+  double* cs = qs + 32 * (d + 1);   // [32][d+1]
+  double* rs = cs + 32 * (d + 1);   // [32][Ck]
+  __shared__ double inv[32];
+  __shared__ double red[8];
+  const int tid = threadIdx.x;
+  for (int e = tid; e < 32 * d; e += 256) {
+    const int p = e / d, a = e % d;
+    qs[p * (d + 1) + a] = p < np ? (double)to_f32(Q[((size_t)bh * L.N + p0 + p) * d + a]) : 0.0;
+  }
+  const double rsd = 1.0 / sqrt((double)d);
+  for (int c0 = 0; c0 < Ck; c0 += 32) {
+    const int nc = min(32, Ck - c0);
+    __syncthreads();
+    for (int e = tid; e < 32 * d; e += 256) {
+      const int j = e / d, a = e % d;
+      cs[j * (d + 1) + a] = j < nc ? L.kcent[((size_t)bh * Ck + c0 + j) * d + a] : 0.0;
+    }
+    __syncthreads();
+    for (int e = tid; e < 32 * 32; e += 256) {
+      const int p = e >> 5, j = e & 31;
+      if (j >= nc) continue;
+      double acc = 0.0;
+      for (int a = 0; a < d; ++a) acc += qs[p * (d + 1) + a] * cs[j * (d + 1) + a];
+      rs[p * Ck + c0 + j] = acc * rsd;
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    double ms = 0.0;
+    for (int j = 0; j < Ck; ++j) ms += rs[tid * Ck + j] * rs[tid * Ck + j];
+    inv[tid] = 1.0 / sqrt(ms / Ck + 1e-12);
+  }
+  __syncthreads();
+  double nrm = 0.0;
+  for (int e = tid; e < 32 * Ck; e += 256) {
+    const int p = e / Ck, j = e % Ck;
+    if (p >= np) continue;
+    const double v = rs[p * Ck + j] * inv[p];
+    const size_t o = ((size_t)bh * L.N + p0 + p) * Ck + j;
+    L.r64[o] = v;
+    L.r32[o] = (float)v;
+    nrm += v * v;
+  }
+  nrm = block_sum(nrm, red);
+  if (tid == 0) atomicAdd(L.T0q + bh, nrm);
+}
+
+// ------------------------------------------------------------------------------------------
+// a6 prologue: stable counting sort of the labels (one warp per (head, side)).  Members of a
+// group keep ascending token order.  perm[pos] = token, inv[token] = pos, off = group starts.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(32) group_sort_kernel(Layout L) {
+  __shared__ int cursor[kMaxGroups + 1];
+  const int bh = blockIdx.x, side = blockIdx.y, lane = threadIdx.x;
+  const int C = side == 0 ? L.Ck : L.Cq;
+  const int* labels = (side == 0 ? L.klabel : L.qlabel) + (size_t)bh * L.N;
+  int* perm = (side == 0 ? L.kperm : L.qperm) + (size_t)bh * L.N;
+  int* inv = (side == 0 ? L.kinv : L.qinv) + (size_t)bh * L.N;
+  int* off = (side == 0 ? L.koff : L.qoff) + (size_t)bh * (C + 1);
+  for (int c = lane; c <= C; c += 32) cursor[c] = 0;
+  __syncwarp();
+  for (int t = lane; t < L.N; t += 32) atomicAdd(&cursor[labels[t]], 1);
+  __syncwarp();
+  if (lane == 0) {
+    int run = 0;
+    for (int c = 0; c < C; ++c) {
+      const int n = cursor[c];
+      off[c] = run;
+      cursor[c] = run;
+      run += n;
+    }
+    off[C] = run;
+  }
+  __syncwarp();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = 0; base < L.N; base += 32) {
+    const int t = base + lane;
+    const bool valid = t < L.N;
+    const int l = valid ? labels[t] : -1;
+    const unsigned m = __match_any_sync(0xffffffffu, l);
+    const int pos = valid ? cursor[l] + __popc(m & lt) : 0;
+    __syncwarp();
+    if (valid && (m & lt) == 0) cursor[l] += __popc(m);
+    __syncwarp();
+    if (valid) {
+      perm[pos] = t;
+      inv[t] = pos;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// a5: routing.  S[g,j] = (mean query of group g) . c_j / sqrt(d) + ln m_j over non-empty key
+// groups, visited by score (ties: lower j).  fixed_k > 0 keeps the first fixed_k; otherwise
+// the top one is kept and every later one iff it brings the running key count strictly
+// closer to kappa = density*N - (s + C_k + P).
+// ------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(128) route_select_kernel(Layout L, const T* __restrict__ Q) {
+  __shared__ double qbar[128];
+  __shared__ double S[kMaxGroups];
+  __shared__ int ord[kMaxGroups];
+  const int bh = blockIdx.x, g = blockIdx.y, d = L.d, Ck = L.Ck, tid = threadIdx.x;
+  const int* qoff = L.qoff + (size_t)bh * (L.Cq + 1);
+  const int* koff = L.koff + (size_t)bh * (Ck + 1);
+  unsigned char* route = L.route + ((size_t)bh * L.Cq + g) * Ck;
+  const int r0 = qoff[g], n = qoff[g + 1] - r0;
+  for (int j = tid; j < Ck; j += blockDim.x) route[j] = 0;
+  if (n == 0) return;
+  if (tid < d) {
+    double acc = 0.0;
+    const int* perm = L.qperm + (size_t)bh * L.N;
+    for (int i = 0; i < n; ++i) acc += (double)to_f32(Q[((size_t)bh * L.N + perm[r0 + i]) * d + tid]);
+    qbar[tid] = acc / (double)n;
+  }
+  __syncthreads();
+  const double rsd = 1.0 / sqrt((double)d);
+  for (int j = tid; j < Ck; j += blockDim.x) {
+    const int m = koff[j + 1] - koff[j];
+    double v = -INFINITY;
+    if (m > 0) {
+      const double* c = L.kcent + ((size_t)bh * Ck + j) * d;
+      double dot = 0.0;
+      for (int a = 0; a < d; ++a) dot += qbar[a] * c[a];
+      v = dot * rsd + log((double)m);
+    }
+    S[j] = v;
+  }
+  __syncthreads();
+  for (int j = tid; j < Ck; j += blockDim.x) {
+    if (koff[j + 1] - koff[j] == 0) continue;
+    const double sj = S[j];
+    int rk = 0;
+    for (int i = 0; i < Ck; ++i) {
+      if (koff[i + 1] - koff[i] == 0) continue;
+      rk += (S[i] > sj) || (S[i] == sj && i < j);
+    }
+    ord[rk] = j;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int nne = 0;
+    for (int j = 0; j < Ck; ++j) nne += koff[j + 1] - koff[j] > 0;
+    if (L.fixed_k > 0) {
+      for (int r = 0; r < min(L.fixed_k, nne); ++r) route[ord[r]] = 1;
+    } else {
+      const double kappa = (double)L.density * (double)L.N - (double)(L.s + Ck + L.P);
+      double cum = 0.0;
+      for (int r = 0; r < nne; ++r) {
+        const int j = ord[r];
+        const double m = (double)(koff[j + 1] - koff[j]);
+        if (r == 0 || fabs((cum + m) - kappa) < fabs(cum - kappa)) {
+          route[j] = 1;
+          cum += m;
+        }
+      }
+    }
+  }
+}
+
+// Route lists (ascending key-group ids), visible keys per group, query-tile prefix and the
+// realised density.  One block per head.
+__global__ void __launch_bounds__(256) route_build_kernel(Layout L, int tile_m) {
+  __shared__ int tiles[kMaxGroups + 1];
+  __shared__ long long pairs[kMaxGroups];
+  const int bh = blockIdx.x, Ck = L.Ck, Cq = L.Cq;
+  const int* koff = L.koff + (size_t)bh * (Ck + 1);
+  const int* qoff = L.qoff + (size_t)bh * (Cq + 1);
+  for (int g = threadIdx.x; g < Cq; g += blockDim.x) {
+    const unsigned char* route = L.route + ((size_t)bh * Cq + g) * Ck;
+    int* list = L.route_list + ((size_t)bh * Cq + g) * Ck;
+    int cnt = 0, keys = 0;
+    for (int j = 0; j < Ck; ++j)
+      if (route[j]) {
+        list[cnt++] = j;
+        keys += koff[j + 1] - koff[j];
+      }
+    const int n = qoff[g + 1] - qoff[g];
+    L.route_cnt[(size_t)bh * Cq + g] = cnt;
+    L.route_keys[(size_t)bh * Cq + g] = keys;
+    tiles[g] = (n + tile_m - 1) / tile_m;
+    pairs[g] = (long long)n * keys;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int* toff = L.tile_off + (size_t)bh * (Cq + 1);
+    int run = 0;
+    long long tot = 0;
+    for (int g = 0; g < Cq; ++g) {
+      toff[g] = run;
+      run += tiles[g];
+      tot += pairs[g];
+    }
+    toff[Cq] = run;
+    const double N = (double)L.N;
+    L.stats[bh].sparse_pairs = tot;
+    L.stats[bh].density = ((double)L.s * N + (double)Ck * N + (double)L.P * N + (double)tot) / (N * N);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Probe rows (Table 4).  Uniform spatiotemporal: rows floor((2i+1)N/(2P)), weight 1.
+// Query-group stratified: m_g = floor(P n_g / N) plus one for the largest remainders
+// (P n_g mod N, ties to the lower g); member floor((2i+1) n_g / (2 m_g)) of group g in token
+// order; weight n_g / m_g scaled to sum P.  Output in ascending token order.
+// ------------------------------------------------------------------------------------------
+constexpr size_t kProbeSmem = kMaxProbes * (sizeof(double) + sizeof(int)) + kMaxGroups * sizeof(long long) +
+                              (2 * kMaxGroups + 1) * sizeof(int);
+
+__global__ void __launch_bounds__(1024) probe_select_kernel(Layout L) {
+  extern __shared__ double shp[];
+  double* cw = shp;                                  // [kMaxProbes]
+  long long* rem = (long long*)(cw + kMaxProbes);    // [kMaxGroups]
+  int* ctok = (int*)(rem + kMaxGroups);              // [kMaxProbes]
+  int* mg = ctok + kMaxProbes;                       // [kMaxGroups]
+  int* slot = mg + kMaxGroups;                       // [kMaxGroups + 1]
+  __shared__ double s_sum;
+  const int bh = blockIdx.x, P = L.P, Cq = L.Cq, N = L.N, tid = threadIdx.x;
+  int* pof = L.probe_of + (size_t)bh * N;
+  for (int t = tid; t < N; t += blockDim.x) pof[t] = -1;
+  if (P == 0) return;
+  if (L.probe_mode == SPARSEPR_PROBE_UNIFORM) {
+    for (int i = tid; i < P; i += blockDim.x) {
+      ctok[i] = (int)(((2LL * i + 1) * N) / (2LL * P));
+      cw[i] = 1.0;
+    }
+    if (tid == 0) s_sum = (double)P;
+  } else {
+    const int* qoff = L.qoff + (size_t)bh * (Cq + 1);
+    const int* qperm = L.qperm + (size_t)bh * N;
+    for (int g = tid; g < Cq; g += blockDim.x) {
+      const long long n = qoff[g + 1] - qoff[g];
+      mg[g] = (int)((P * n) / N);
+      rem[g] = (P * n) % N;
+    }
+    __syncthreads();
+    __shared__ int s_extra;
+    if (tid == 0) {
+      int tot = 0;
+      for (int g = 0; g < Cq; ++g) tot += mg[g];
+      s_extra = P - tot;
+    }
+    __syncthreads();
+    for (int g = tid; g < Cq; g += blockDim.x) {
+      int rk = 0;
+      for (int h = 0; h < Cq; ++h) rk += (rem[h] > rem[g]) || (rem[h] == rem[g] && h < g);
+      if (rk < s_extra) mg[g] += 1;  // each g is written by its own thread only
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int run = 0;
+      for (int g = 0; g < Cq; ++g) {
+        slot[g] = run;
+        run += mg[g];
+      }
+      slot[Cq] = run;
+    }
+    __syncthreads();
+    for (int g = tid; g < Cq; g += blockDim.x) {
+      const int n = qoff[g + 1] - qoff[g], m = mg[g];
+      for (int i = 0; i < m; ++i) {
+        ctok[slot[g] + i] = qperm[qoff[g] + (int)(((2LL * i + 1) * n) / (2LL * m))];
+        cw[slot[g] + i] = (double)n / (double)m;
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      double s = 0.0;
+      for (int i = 0; i < P; ++i) s += cw[i];
+      s_sum = s;
+    }
+  }
+  __syncthreads();
+  int* tok = L.probe_tok + (size_t)bh * P;
+  double* w = L.probe_w + (size_t)bh * P;
+  const double scale = (double)P / s_sum;
+  for (int i = tid; i < P; i += blockDim.x) {
+    const int t = ctok[i];
+    int rk = 0;
+    for (int k = 0; k < P; ++k) rk += ctok[k] < t;
+    tok[rk] = t;
+    w[rk] = cw[i] * scale;
+    pof[t] = rk;
+  }
+}
+
+// probe_of from an installed probe list (sparsepr_set_partition).
+__global__ void probe_index_kernel(Layout L) {
+  const int bh = blockIdx.x;
+  int* pof = L.probe_of + (size_t)bh * L.N;
+  for (int t = threadIdx.x; t < L.N; t += blockDim.x) pof[t] = -1;
+  __syncthreads();
+  for (int i = threadIdx.x; i < L.P; i += blockDim.x) pof[L.probe_tok[(size_t)bh * L.P + i]] = i;
+}
+
+// Per-head k-means statistics after both loops.
+__global__ void plan_stats_kernel(Layout L) {
+  const int bh = blockIdx.x * blockDim.x + threadIdx.x;
+  if (bh >= L.BH) return;
+  sparsepr_head_stats& st = L.stats[bh];
+  const int ki = L.stop_at[bh * 2 + 0], qi = L.stop_at[bh * 2 + 1];
+  st.k_iters = ki;
+  st.q_iters = qi;
+  st.k_refined = L.krefined[bh];
+  st.q_refined = L.qrefined[bh];
+  st.k_objective = ki > 0 ? L.kJ[(size_t)bh * L.iters_cap + ki - 1] : 0.0;
+  st.q_objective = qi > 0 ? L.qJ[(size_t)bh * L.iters_cap + qi - 1] : 0.0;
+}
+
+// ------------------------------------------------------------------------------------------
+// a6: gather rows into group-contiguous order (one warp per row, 16-byte chunks).
+// ------------------------------------------------------------------------------------------
+__global__ void permute_rows_kernel(Layout L, const void* __restrict__ src, void* __restrict__ dst,
+                                    const int* __restrict__ perm, int rows_per_head, int src_rows_per_head) {
+  const int bh = blockIdx.y;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= rows_per_head) return;
+  const size_t rb = (size_t)L.d * elt_size(L.dtype);
+  const int chunks = (int)(rb / 16);
+  const int t = perm[(size_t)bh * rows_per_head + warp];
+  const uint4* s = (const uint4*)((const char*)src + ((size_t)bh * src_rows_per_head + t) * rb);
+  uint4* o = (uint4*)((char*)dst + ((size_t)bh * rows_per_head + warp) * rb);
+  for (int c = lane; c < chunks; c += 32) o[c] = s[c];
+}
+
+// ------------------------------------------------------------------------------------------
+// Host launchers.
+// ------------------------------------------------------------------------------------------
+template <typename T>
+static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool warm, int iters,
+                                  cudaStream_t st) {
+  const int d = L.d;
+  launch(metric_kernel<T>, dim3(L.BH, d), 128, 0, st, L, Q);
+  launch(gram_part_kernel<T>, dim3(L.BH, L.n_gram_parts), 256, 32 * d * sizeof(double), st, L, K);
+  launch(gram_reduce_kernel, L.BH, 256, 0, st, L);
+  if (!warm) {
+    launch(km_draw_kernel, L.BH, 128, 0, st, L, 0, L.Ck);
+    launch(kcent_init_kernel<T>, dim3(L.BH, L.Ck), 128, 0, st, L, K);
+  }
+  SPR_LAUNCH_CHECK();
+  launch(km_reset_kernel, L.BH, 128, 0, st, L, 0, iters);
+  cudaMemsetAsync(L.T0q, 0, sizeof(double) * L.BH, st);
+  const size_t asg_smem_k = (size_t)(kAsgPts + kAsgChunk) * (d + 1) * 4 + (kAsgChunk + kAsgPts) * 4 +
+                            2 * kAsgPts * 4 + kAsgPts * 8;
+  const int nblk = (L.N + kAsgPts - 1) / kAsgPts;
+  cudaFuncSetAttribute(kmeans_assign_kernel<T, KeyFeat>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asg_smem_k);
+  for (int it = 0; it <= iters; ++it) {
+    launch(kprep_kernel, dim3(L.BH, L.Ck), 128, 0, st, L, it, iters);
+    if (it < iters)
+      launch(kmeans_assign_kernel<T, KeyFeat>, dim3(nblk, L.BH), 256, asg_smem_k, st, L, K, it);
+  }
+  SPR_LAUNCH_CHECK();
+  const size_t qr_smem = (size_t)(2 * 32 * (d + 1) + 32 * L.Ck) * sizeof(double);
+  cudaFuncSetAttribute(qresp_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qr_smem);
+  launch(qresp_kernel<T>, dim3((L.N + 31) / 32, L.BH), 256, qr_smem, st, L, Q);
+  if (!warm) {
+    launch(km_draw_kernel, L.BH, 128, 0, st, L, 1, L.Cq);
+    launch(qcent_init_kernel, dim3(L.BH, L.Cq), 128, 0, st, L);
+  }
+  launch(km_reset_kernel, L.BH, 128, 0, st, L, 1, iters);
+  SPR_LAUNCH_CHECK();
+  const size_t asg_smem_q = (size_t)(kAsgPts + kAsgChunk) * (L.Ck + 1) * 4 + (kAsgChunk + kAsgPts) * 4 +
+                            2 * kAsgPts * 4 + kAsgPts * 8;
+  cudaFuncSetAttribute(kmeans_assign_kernel<T, QueryFeat>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asg_smem_q);
+  for (int it = 0; it <= iters; ++it) {
+    launch(qprep_kernel, dim3(L.BH, L.Cq), 128, 0, st, L, it, iters);
+    if (it < iters)
+      launch(kmeans_assign_kernel<T, QueryFeat>, dim3(nblk, L.BH), 256, asg_smem_q, st, L, K, it);
+  }
+  SPR_LAUNCH_CHECK();
+  launch(group_sort_kernel, dim3(L.BH, 2), 32, 0, st, L);
+  launch(route_select_kernel<T>, dim3(L.BH, L.Cq), 128, 0, st, L, Q);
+  launch(route_build_kernel, L.BH, 256, 0, st, L, kAttnTileM);
+  cudaFuncSetAttribute(probe_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kProbeSmem);
+  launch(probe_select_kernel, L.BH, 1024, kProbeSmem, st, L);
+  launch(plan_stats_kernel, (L.BH + 127) / 128, 128, 0, st, L);
+  SPR_LAUNCH_CHECK();
+  return SPARSEPR_OK;
+}
+
+sparsepr_status launch_plan(const Layout& L, const void* Q, const void* K, bool warm, int iters,
+                            cudaStream_t st) {
+  if (L.dtype == SPARSEPR_F32) return plan_typed<float>(L, (const float*)Q, (const float*)K, warm, iters, st);
+  return plan_typed<__nv_bfloat16>(L, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, warm, iters, st);
+}
+
+sparsepr_status launch_installed_partition(const Layout& L, cudaStream_t st) {
+  launch(group_sort_kernel, dim3(L.BH, 2), 32, 0, st, L);
+  launch(route_build_kernel, L.BH, 256, 0, st, L, kAttnTileM);
+  launch(probe_index_kernel, L.BH, 1024, 0, st, L);
+  SPR_LAUNCH_CHECK();
+  return SPARSEPR_OK;
+}
+
+sparsepr_status launch_permute(const Layout& L, const void* Q, const void* K, const void* V,
+                               cudaStream_t st) {
+  const dim3 grid((L.N * 32 + 255) / 256, L.BH);
+  launch(permute_rows_kernel, grid, 256, 0, st, L, Q, L.Qp, L.qperm, L.N, L.N);
+  launch(permute_rows_kernel, grid, 256, 0, st, L, K, L.Kp, L.kperm, L.N, L.N);
+  launch(permute_rows_kernel, grid, 256, 0, st, L, V, L.Vp, L.kperm, L.N, L.N);
+  if (L.P > 0)
+    launch(permute_rows_kernel, dim3((L.P * 32 + 255) / 256, L.BH), 256, 0, st, L, Q, L.Qprobe, L.probe_tok, L.P, L.N);
+  SPR_LAUNCH_CHECK();
+  return SPARSEPR_OK;
+}
+
+}  // namespace sparsepr

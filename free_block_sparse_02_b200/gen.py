@@ -43,7 +43,8 @@ def token_tiles(w: Workload) -> np.ndarray:
     T, Y, X = w.grid
     a, b, c = w.tile
     t, y, x = np.meshgrid(np.arange(T), np.arange(Y), np.arange(X), indexing="ij")
-    tid = ((t // a) * (Y // b) + (y // b)) * (X // c) + (x // c)
+    ny, nx = -(-Y // b), -(-X // c)          # tiles per axis (a ragged last tile is allowed)
+    tid = ((t // a) * ny + (y // b)) * nx + (x // c)
     return tid.reshape(-1)
 
 

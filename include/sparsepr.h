@@ -1,0 +1,189 @@
+/*
+ * sparsepr.h -- C ABI of the B200 (sm_100a) SparsePR per-call sparse attention operator.
+ *
+ * The operator is the one described in "Partition the Support, Reconstruct the Residual:
+ * Training-Free Sparse Attention for Video Generation and World Models" (Taghavi, Langari,
+ * Pandey, arXiv 2608.18484): abstract, and the method pipeline of the project page
+ * "SparsePR: Training-Free Sparse Attention for Video Generation" (steps 01 sample responses,
+ * 02 partition support, 03 execute sparse routes, 04 reconstruct residual).
+ *
+ * One call on Q, K, V of shape [B, H, N, d] runs, independently for every (b, h) head:
+ *   sparsepr_plan       Response-Coupled Partitioning and routing (abstract: "group paired
+ *                       key/value tokens by how their keys respond to sampled queries", "group
+ *                       queries by their responses to the resulting key-group centroids for
+ *                       shared sparse routing"), plus the choice of probe rows (Table 4).
+ *   sparsepr_attention  block-sparse attention over the kept (query group, key group) cells
+ *                       and exact dense attention of the probe rows (abstract: "compute exact
+ *                       attention on a small set of query rows").
+ *   sparsepr_fit_apply  Probe-Fitted Residual Reconstruction: weighted ridge fit of an affine
+ *                       map [O_sp, 1] -> O_dense - O_sp on the probe rows, restricted to the
+ *                       span of the probe residuals, added to every unprobed row; probe rows
+ *                       take their exact output.
+ *
+ * Conventions
+ *   - All tensor arguments are DEVICE pointers to contiguous row-major [B, H, N, d] arrays of
+ *     the configured dtype (SPARSEPR_F32 or SPARSEPR_BF16); d is 64 or 128.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Every
+ *     call only enqueues work on that stream and returns without waiting, except
+ *     sparsepr_plan_query and sparsepr_sync, which wait for the stream.
+ *   - The caller owns Q, K, V, O and the workspace; the plan owns a small host structure and
+ *     pointers into the caller's workspace.  Inputs are never written.
+ *   - Errors: arguments are checked before anything is enqueued (SPARSEPR_ERR_INVALID_ARG /
+ *     _UNSUPPORTED / _WORKSPACE, nothing launched).  Launch failures return SPARSEPR_ERR_CUDA.
+ *     Faults found by the kernels themselves (a ridge system that stays indefinite after the
+ *     jitter retries, a bounded wait that expired) are written to a device status word in the
+ *     workspace and returned by the next sparsepr_sync or sparsepr_plan_query.  No exception
+ *     crosses the ABI; no call allocates device memory.
+ */
+#ifndef SPARSEPR_H_
+#define SPARSEPR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sparsepr_status {
+  SPARSEPR_OK = 0,
+  SPARSEPR_ERR_INVALID_ARG = 1,  /* null pointer, size out of range, inconsistent config     */
+  SPARSEPR_ERR_UNSUPPORTED = 2,  /* valid but not built: d not in {64,128}, too many groups  */
+  SPARSEPR_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed               */
+  SPARSEPR_ERR_WORKSPACE = 4,    /* workspace null, too small or not 256-byte aligned         */
+  SPARSEPR_ERR_NUMERIC = 5,      /* ridge system not positive definite after jitter retries  */
+  SPARSEPR_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up                       */
+  SPARSEPR_ERR_STATE = 7         /* call out of order (attention before plan, ...)           */
+} sparsepr_status;
+
+enum { SPARSEPR_F32 = 0, SPARSEPR_BF16 = 1 };
+enum { SPARSEPR_PROBE_UNIFORM = 0, SPARSEPR_PROBE_STRATIFIED = 1 };
+
+/* Parameters of one call, as the paper states the problem (abstract; Table C.1; Table 4). */
+typedef struct sparsepr_config {
+  int32_t B, H, N, d;       /* Q/K/V shape [B,H,N,d]; N >= 1, d in {64, 128}                   */
+  int32_t dtype;            /* SPARSEPR_F32 or SPARSEPR_BF16 for Q, K, V                        */
+  int32_t s;                /* sampled queries per head, 1 <= s <= N; rows floor((2i+1)N/(2s)) */
+  int32_t n_kgroups;        /* C_k paired K/V groups, 1 <= C_k <= min(N, 1024)                */
+  int32_t n_qgroups;        /* C_q query groups,      1 <= C_q <= min(N, 1024)                */
+  float density;            /* target executed-pair density in (0, 1], counting the s*N routing,
+                               C_k*N centroid and P*N probe pairs; per-row key budget
+                               kappa = density*N - (s + C_k + P)                                */
+  int32_t fixed_k;          /* > 0: every query group keeps exactly min(fixed_k, non-empty)
+                               key groups and `density` is ignored                              */
+  int32_t P;                /* probe rows per head, 0 <= P <= min(N, 4096)                     */
+  int32_t probe_mode;       /* SPARSEPR_PROBE_UNIFORM or SPARSEPR_PROBE_STRATIFIED              */
+  double lambda;            /* ridge lambda >= 0; < 0 selects 1e-3 * tr(X^T W X) / (d+1)       */
+  int32_t km_iters;         /* Lloyd iteration limit of a cold plan (>= 1)                     */
+  int32_t km_iters_warm;    /* limit of a re-plan warm-started from the previous centroids;
+                               0 = every plan starts cold                                      */
+  float km_tol;             /* stop when J_prev - J <= km_tol * J_prev; < 0 = never early      */
+  uint64_t seed;            /* k-means initial points: SplitMix64 stream seed + 2*(b*H+h) + stage */
+} sparsepr_config;
+
+/* Per-head statistics, read with sparsepr_plan_query(SPARSEPR_Q_STATS). */
+typedef struct sparsepr_head_stats {
+  int32_t k_iters;          /* Lloyd iterations run for the key groups                          */
+  int32_t q_iters;          /* ... for the query groups                                         */
+  int32_t k_refined;        /* key labels decided by the float64 tie-break at the last pass     */
+  int32_t q_refined;        /* query labels decided by the float64 tie-break at the last pass   */
+  int32_t fit_retries;      /* ridge jitter retries (lambda x10 each); 0 normally               */
+  int32_t span_rank;        /* rank of the probe-residual span                                  */
+  int64_t sparse_pairs;     /* executed (query, key) pairs of the block-sparse pass             */
+  double density;           /* realised density: (s*N + C_k*N + P*N + sparse_pairs) / N^2      */
+  double k_objective;       /* J at the last key assignment                                     */
+  double q_objective;       /* J at the last query assignment                                   */
+  double lambda;            /* ridge lambda used                                                */
+} sparsepr_head_stats;
+
+/* What sparsepr_plan_query copies to host memory (all heads, head-major). */
+enum {
+  SPARSEPR_Q_KLABELS = 1,   /* int32  [B*H, N]       key-group label of every key token        */
+  SPARSEPR_Q_QLABELS = 2,   /* int32  [B*H, N]       query-group label of every query token    */
+  SPARSEPR_Q_ROUTE = 3,     /* uint8  [B*H, C_q, C_k] 1 = key group kept by the query group     */
+  SPARSEPR_Q_PROBES = 4,    /* int32  [B*H, P]       probe token ids, ascending                 */
+  SPARSEPR_Q_PROBE_W = 5,   /* double [B*H, P]       probe weights (sum P per head)             */
+  SPARSEPR_Q_FIT = 6,       /* double [B*H, d+1, d]  fitted affine map A (last row: intercept) */
+  SPARSEPR_Q_KCENT = 7,     /* double [B*H, C_k, d]  key-group centroids (key space)            */
+  SPARSEPR_Q_QCENT = 8,     /* double [B*H, C_q, C_k] query-group centroids (response space)    */
+  SPARSEPR_Q_OSP = 9,       /* float  [B*H, N, d]    block-sparse output, original token order */
+  SPARSEPR_Q_ODENSE = 10,   /* float  [B*H, P, d]    exact output of the probe rows            */
+  SPARSEPR_Q_STATS = 11,    /* sparsepr_head_stats [B*H]                                        */
+  SPARSEPR_Q_KOBJ = 12,     /* double [B*H, km_iters] key objective per iteration (0 = not run) */
+  SPARSEPR_Q_QOBJ = 13      /* double [B*H, km_iters] query objective per iteration             */
+};
+
+typedef struct sparsepr_plan_s sparsepr_plan_t;
+
+/* Bytes of device workspace the configuration needs.  Returns INVALID_ARG / UNSUPPORTED for a
+ * configuration that the other calls would reject. */
+sparsepr_status sparsepr_workspace_size(const sparsepr_config* cfg, size_t* bytes);
+
+/* Creates a plan bound to `workspace` (device memory of at least sparsepr_workspace_size
+ * bytes, 256-byte aligned, owned by the caller and kept alive until sparsepr_plan_destroy).
+ * Allocates the small host plan structure and clears the device status word and statistics
+ * with a blocking cudaMemset; enqueues nothing on any stream. */
+sparsepr_status sparsepr_plan_create(const sparsepr_config* cfg, void* workspace,
+                                     size_t ws_bytes, sparsepr_plan_t** plan);
+
+/* Response-Coupled Partitioning, routing and probe choice for Q, K (device pointers).
+ * The first plan of a plan object starts k-means from SplitMix64-drawn points and runs up
+ * to km_iters; later plans start from the previous call's centroids and run up to
+ * km_iters_warm when km_iters_warm > 0 (Table C.1: 25 initial / 2 subsequent iterations). */
+sparsepr_status sparsepr_plan(sparsepr_plan_t* plan, const void* Q, const void* K, void* stream);
+
+/* Debug/injection entry: installs a partition given in HOST memory instead of computing one
+ * (klabels, qlabels int32 [B*H, N] with values in [0, C_k) / [0, C_q); route uint8
+ * [B*H, C_q, C_k]; probes int32 [B*H, P] distinct token ids; probe_w double [B*H, P]).
+ * Copies synchronously; afterwards attention / fit_apply run as after sparsepr_plan. */
+sparsepr_status sparsepr_set_partition(sparsepr_plan_t* plan, const int32_t* klabels,
+                                       const int32_t* qlabels, const uint8_t* route,
+                                       const int32_t* probes, const double* probe_w,
+                                       void* stream);
+
+/* Block-sparse attention of every query over the keys of its group's kept key groups, and
+ * exact dense attention of the probe rows.  Q, K, V: the same tensors as the plan's. */
+sparsepr_status sparsepr_attention(sparsepr_plan_t* plan, const void* Q, const void* K,
+                                   const void* V, void* stream);
+
+/* Weighted ridge fit on the probe rows, projection onto the probe-residual span, and the
+ * corrected output O [B,H,N,d] in original token order (out_dtype SPARSEPR_F32 or _BF16). */
+sparsepr_status sparsepr_fit_apply(sparsepr_plan_t* plan, void* O, int32_t out_dtype,
+                                   void* stream);
+
+/* Waits for the plan's last stream and copies one result (SPARSEPR_Q_*) to host memory;
+ * `bytes` must equal the item's size.  Returns a pending device fault if there is one. */
+sparsepr_status sparsepr_plan_query(const sparsepr_plan_t* plan, int32_t what, void* host_dst,
+                                    size_t bytes);
+
+/* Waits for the plan's last stream and returns (and clears) the device status word. */
+sparsepr_status sparsepr_sync(sparsepr_plan_t* plan);
+
+/* Frees the host plan structure (not the caller's workspace).  NULL is ignored. */
+void sparsepr_plan_destroy(sparsepr_plan_t* plan);
+
+/* Static string naming a status code. */
+const char* sparsepr_status_string(sparsepr_status status);
+
+/* Library version, e.g. 100 for 0.1.0. */
+int32_t sparsepr_version(void);
+
+/* Kernels whose launches sparsepr_set_kernel_events can bracket. */
+enum { SPARSEPR_KERNEL_BLOCK_SPARSE = 0 };
+
+/* Optional timing hook for measurement.  When set, sparsepr_attention records `start_event`
+ * on its stream immediately before launching the block-sparse attention kernel and
+ * `stop_event` immediately after it, so cudaEventElapsedTime gives that kernel's duration.
+ * Events are cudaEvent_t handles passed as void*, created and owned by the caller; passing
+ * NULL for both removes the hook.  Returns INVALID_ARG for an unknown kernel id. */
+sparsepr_status sparsepr_set_kernel_events(sparsepr_plan_t* plan, int32_t kernel, void* start_event,
+                                           void* stop_event);
+
+/* Number of CUDA kernels this library has launched since it was loaded (all plans). */
+int64_t sparsepr_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSEPR_H_ */

@@ -422,6 +422,7 @@ def call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int,
     scale = 1.0 / math.sqrt(d)
     Ck, Cq = cfg.n_kgroups, cfg.n_qgroups
     seed = getattr(cfg, "seed", 0)
+    tol = float(np.float32(cfg.km_tol))  # the operator's tolerance is a float32 argument
 
     # 1-2: key responses to the sampled queries and paired K/V groups.
     rows = sample_query_rows(N, cfg.s)
@@ -433,7 +434,7 @@ def call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int,
     else:
         C0 = (warm.key_centroids @ Qs.T) * scale
         S0, iters = warm.key_centroids, cfg.km_iters_warm
-    kk = lloyd(F, C0, iters, cfg.km_tol, shadow=k, shadow_init=S0, keep_history=keep_history)
+    kk = lloyd(F, C0, iters, tol, shadow=k, shadow_init=S0, keep_history=keep_history)
     klabels = kk.labels
     kcent = kk.shadow
 
@@ -445,7 +446,7 @@ def call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int,
         C0q, iters = Rt[ids], cfg.km_iters
     else:
         C0q, iters = warm.query_centroids, cfg.km_iters_warm
-    qq = lloyd(Rt, C0q, iters, cfg.km_tol, keep_history=keep_history)
+    qq = lloyd(Rt, C0q, iters, tol, keep_history=keep_history)
     qlabels = qq.labels
 
     # 5: routing.

@@ -1,0 +1,81 @@
+"""The C-ABI library loads and exports every entry point declared in include/sparsepr.h, and
+its host-side argument checks reject bad configurations before touching a GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from free_block_sparse_02_b200 import build, configs
+from free_block_sparse_02_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "sparsepr.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sparsepr_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_version(lib):
+    assert lib.sparsepr_version() >= 100
+    for code in range(8):
+        assert lib.sparsepr_status_string(code)
+    assert lib.sparsepr_status_string(0) == b"ok"
+
+
+def test_workspace_size_for_every_workload(lib):
+    for w in configs.WORKLOADS:
+        n = _lib.workspace_size(_lib.config_from(w))
+        assert n > 0 and n % 256 == 0
+    small = _lib.workspace_size(_lib.config_from(configs.workload(0)))
+    big = _lib.workspace_size(_lib.config_from(configs.workload(2)))
+    assert big > 100 * small
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("d", 96, 2), ("d", 0, 2), ("N", 0, 1), ("s", 0, 1), ("s", 2000, 1), ("n_kgroups", 0, 1),
+    ("n_kgroups", 1025, 1), ("n_kgroups", 300, 2), ("n_qgroups", 2000, 1), ("P", -1, 1),
+    ("P", 5000, 1), ("probe_mode", 7, 1), ("dtype", 3, 1), ("km_iters", 0, 1), ("km_iters_warm", -2, 1),
+])
+def test_invalid_configs_are_rejected_on_the_host(lib, field, value, code):
+    w = configs.workload(0)
+    cfg = _lib.config_from(w, **{field: value})
+    n = ctypes.c_size_t(0)
+    assert lib.sparsepr_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == code
+
+
+def test_density_is_checked_only_without_fixed_k(lib):
+    n = ctypes.c_size_t(0)
+    cfg = _lib.config_from(configs.workload(1), density=0.0)
+    assert lib.sparsepr_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == 1
+    cfg = _lib.config_from(configs.workload(0), density=0.0)  # fixed_k > 0
+    assert lib.sparsepr_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == 0
+
+
+def test_null_and_misaligned_arguments(lib):
+    cfg = _lib.config_from(configs.workload(0))
+    h = ctypes.c_void_p()
+    assert lib.sparsepr_workspace_size(None, None) == 1
+    assert lib.sparsepr_plan_create(ctypes.byref(cfg), None, 1 << 30, ctypes.byref(h)) == 4
+    assert lib.sparsepr_plan_create(ctypes.byref(cfg), 4096 + 16, 1 << 30, ctypes.byref(h)) == 4
+    assert lib.sparsepr_plan_create(ctypes.byref(cfg), 4096, 16, ctypes.byref(h)) == 4
+    assert lib.sparsepr_plan(None, None, None, None) == 1
+    assert lib.sparsepr_attention(None, None, None, None, None) == 1
+    assert lib.sparsepr_fit_apply(None, None, 0, None) == 1
+    assert lib.sparsepr_sync(None) == 1
+    lib.sparsepr_plan_destroy(None)
