@@ -76,6 +76,9 @@ def compare_outputs(op, out, qf, kf, vf, w, atol, rel_l2):
                                         pw[bh], w.lam)
         for name, got, exp in (("O_sp", osp[bh], ref["osp"]), ("O_dense", od[bh], ref["odense"]),
                                ("O", O_gpu[bh], ref["O"])):
+            if exp.size == 0:
+                assert got.size == 0
+                continue
             diff = np.abs(got - exp)
             rl2 = np.linalg.norm(got - exp) / max(np.linalg.norm(exp), 1e-30)
             assert diff.max() <= atol, f"head {bh} {name}: max-abs {diff.max():.3e} > {atol}"
