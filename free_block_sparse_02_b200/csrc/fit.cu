@@ -324,3 +324,17 @@ sparsepr_status launch_fit_apply(const Layout& L, void* O, int out_dtype, cudaSt
 }
 
 }  // namespace sparsepr
+
+namespace sparsepr {
+
+// The one-CTA-per-head solve on ridge matrices that are already in L.ridgeG / ridgeB / spanS.
+sparsepr_status launch_ridge_solve(const Layout& L, cudaStream_t st) {
+  const int n1 = L.d + 1;
+  const size_t ssm = (size_t)n1 * n1 * sizeof(double);
+  cudaFuncSetAttribute(ridge_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
+  launch(ridge_solve_kernel, L.BH, 256, ssm, st, L);
+  SPR_LAUNCH_CHECK();
+  return SPARSEPR_OK;
+}
+
+}  // namespace sparsepr

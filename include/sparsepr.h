@@ -182,6 +182,33 @@ sparsepr_status sparsepr_set_kernel_events(sparsepr_plan_t* plan, int32_t kernel
 /* Number of CUDA kernels this library has launched since it was loaded (all plans). */
 int64_t sparsepr_launch_count(void);
 
+/* Allocation-free weighted ridge fit (no counterpart in the paper: an interface for callers
+ * that cannot allocate device memory).  Some callers cannot call cudaMalloc or hand this
+ * library scratch memory at the point where they fit the correction -- e.g. code running under
+ * a fixed memory pool that must not grow during a step, or a host runtime that only passes the
+ * tensors it already owns.  This entry point computes, for each of n_heads heads, the same
+ * fitted map A as sparsepr_fit_apply (weighted ridge of O_dense - O_sp on [O_sp, 1], lambda as
+ * in sparsepr_config, restricted to the span of the probe residuals) from probe rows the
+ * caller passes in, and allocates nothing.
+ *   osp_probe    float  [n_heads, P, d]   device: block-sparse output of the probe rows
+ *   odense_probe float  [n_heads, P, d]   device: exact output of the probe rows
+ *   probe_w      double [n_heads, P]      device: probe weights
+ *   A            double [n_heads, d+1, d] device, written (last row: intercept)
+ *   status_out   int32  [1] device or NULL: receives 0, or SPARSEPR_ERR_NUMERIC if a head's
+ *                system stayed indefinite after the jitter retries (that head's A is zero)
+ * Scratch: one fixed __device__ array inside the library (about 7.4 MB) that every GPU which
+ * loads the library reserves until the process exits.  Limits: 1 <= n_heads <= 16,
+ * d in {64, 128}, 0 <= P <= 4096; larger sizes return SPARSEPR_ERR_WORKSPACE and launch
+ * nothing.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current, so make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's contents: calls that
+ * overlap on the GPU (e.g. on two streams at once) race and give wrong results; serialise
+ * them.  Enqueued on `stream` (cudaStream_t as void*); returns without waiting. */
+sparsepr_status sparsepr_ridge_fit_static(const float* osp_probe, const float* odense_probe,
+                                          const double* probe_w, int32_t n_heads, int32_t P,
+                                          int32_t d, double lambda, double* A, int32_t* status_out,
+                                          void* stream);
+
 #ifdef __cplusplus
 }
 #endif
