@@ -189,6 +189,9 @@ def run_ours(args, w, world, rank, local):
     st = op.stats()
     pairs = sum(s["sparse_pairs"] for s in st)
     realised = statistics.mean(s["density"] for s in st)
+    part_stats = {"k_iters": [s["k_iters"] for s in st], "q_iters": [s["q_iters"] for s in st],
+                  "k_refined": sum(s["k_refined"] for s in st), "q_refined": sum(s["q_refined"] for s in st),
+                  "span_rank": [s["span_rank"] for s in st]}
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -269,6 +272,7 @@ def run_ours(args, w, world, rank, local):
                     "h2d_bytes_per_step": 3 * Q.numel() * elt, "d2h_bytes_per_step": O.numel() * O.element_size(),
                     "ms_per_step": e2e_ms},
             "gpu_launches": launches,
+            "partition": part_stats,
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:

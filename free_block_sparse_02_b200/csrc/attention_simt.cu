@@ -8,8 +8,9 @@
 // Operands are the group-permuted Q/K/V: query group g is rows [qoff_g, qoff_{g+1}) of Qp and
 // key group j is rows [koff_j, koff_{j+1}) of Kp/Vp.  A work item is one 64-row query tile of
 // one group; it streams the concatenation of its kept key groups in 64-key tiles with an
-// online softmax (running max and sum per row).  fp32 inputs are the f32 path of the
-// operator; the bf16 path runs on the tensor-core kernel.
+// online softmax (running max and sum per row).  This is the fp32 path of the operator (fp32
+// inputs need fp32 products for the 1e-4 output tolerance); bf16 inputs run on the
+// tensor-core kernel.
 #include <math.h>
 
 #include "common.cuh"
@@ -178,10 +179,11 @@ static sparsepr_status launch_simt(const Layout& L, cudaStream_t st, cudaEvent_t
   return SPARSEPR_OK;
 }
 
+// fp32 inputs run here; bf16 inputs run on the tensor-core kernel (attention_sm100.cu).
 sparsepr_status launch_attention(const Layout& L, cudaStream_t st, cudaEvent_t e0, cudaEvent_t e1) {
   if (L.dtype == SPARSEPR_F32)
     return L.d == 64 ? launch_simt<float, 64>(L, st, e0, e1) : launch_simt<float, 128>(L, st, e0, e1);
-  return L.d == 64 ? launch_simt<__nv_bfloat16, 64>(L, st, e0, e1) : launch_simt<__nv_bfloat16, 128>(L, st, e0, e1);
+  return launch_attention_tc(L, st, e0, e1);
 }
 
 }  // namespace sparsepr

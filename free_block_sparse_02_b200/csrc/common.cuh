@@ -34,15 +34,13 @@ struct Layout {
   float km_tol;
   double lambda;
   uint64_t seed;
-  int n_gram_parts;     // N-chunks of the key Gram reduction
 
   // status + per-head statistics
   int* status;                    // [1]
   sparsepr_head_stats* stats;     // [BH]
 
-  // key responses: metric M = Qs^T Qs / d and the key Gram for the objective constant
+  // key responses: metric M = Qs^T Qs / d and the objective constants
   double* M;                      // [BH, d, d]
-  double* gram_part;              // [BH, n_gram_parts, d, d]
   double* T0k;                    // [BH]  sum_t ||f_t||^2
   double* T0q;                    // [BH]  sum_q ||r~_q||^2
 
@@ -79,6 +77,16 @@ struct Layout {
   int* qlabel;                    // [BH, N]
   double* qJ;                     // [BH, iters_cap]
   int* qrefined;                  // [BH]
+
+  // bf16 operands of the tensor-core assignment: weights split into three bf16 terms
+  // (hi + mid + lo reproduces the fp64 value to ~2^-24 relative), features likewise for the
+  // normalised responses; group rows padded to a multiple of 16, response dims to 64
+  int Ckp, Cqp, Dq;
+  __nv_bfloat16* kWb;             // [3][BH, Ckp, d]
+  __nv_bfloat16* qWb;             // [3][BH, Cqp, Dq]
+  __nv_bfloat16* rb;              // [3][BH, N, Dq]
+  float* knorm;                   // [BH, N] ||k_t||_2 (rounding bound of the key scores)
+  float* rnorm;                   // [BH, N] ||r~_q||_2
 
   // group-contiguous order (stable counting sort)
   int* kperm;                     // [BH, N]   position -> token

@@ -88,15 +88,19 @@ __global__ void __launch_bounds__(256) ridge_gram_kernel(Layout L) {
   }
 }
 
-// In-place lower Cholesky of the n x n matrix in shared memory; false if a pivot is not > 0.
-__device__ bool chol_smem(double* G, int n, int ld) {
+// Shared memory of the solve: the (d+1)^2 system and a (d+1) x 33 block of right-hand sides.
+static size_t ridge_solve_smem(int d) { return (size_t)((d + 1) * (d + 1) + (d + 1) * 33) * sizeof(double); }
+
+// In-place lower Cholesky of the n x n matrix in shared memory; false if a pivot is not
+// above `tol` (or not finite).  Trailing update: thread rows i, columns j <= i.
+__device__ bool chol_smem_tol(double* G, int n, int ld, double tol) {
   __shared__ int fail;
   if (threadIdx.x == 0) fail = 0;
   __syncthreads();
   for (int k = 0; k < n; ++k) {
     if (threadIdx.x == 0) {
       const double piv = G[k * ld + k];
-      if (!(piv > 0.0) || !isfinite(piv)) fail = 1;
+      if (!(piv > tol) || !isfinite(piv)) fail = 1;
       else G[k * ld + k] = sqrt(piv);
     }
     __syncthreads();
@@ -105,14 +109,18 @@ __device__ bool chol_smem(double* G, int n, int ld) {
     for (int i = k + 1 + threadIdx.x; i < n; i += blockDim.x) G[i * ld + k] /= lkk;
     __syncthreads();
     const int m = n - k - 1;
-    for (int e = threadIdx.x; e < m * m; e += blockDim.x) {
-      const int i = k + 1 + e / m, j = k + 1 + e % m;
-      if (j <= i) G[i * ld + j] -= G[i * ld + k] * G[j * ld + k];
+    // (i, j) with k < j <= i < n: warp-strided rows, lanes over columns
+    const int nw = blockDim.x >> 5, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = k + 1 + w; i < n; i += nw) {
+      const double lik = G[i * ld + k];
+      for (int j = k + 1 + lane; j <= i; j += 32) G[i * ld + j] -= lik * G[j * ld + k];
     }
+    (void)m;
     __syncthreads();
   }
   return true;
 }
+__device__ bool chol_smem(double* G, int n, int ld) { return chol_smem_tol(G, n, ld, 0.0); }
 
 // One CTA per head: lam, Cholesky with up to three x10 jitter retries, the d right-hand sides,
 // then the residual-span basis by column-pivoted Gram-Schmidt on S = R^T W R and A <- A U U^T.
@@ -163,96 +171,156 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
     }
     return;
   }
-  // solve L L^T x = b for every column of B; A is the scratch of each thread's column
-  const double* Bg = L.ridgeB + (size_t)bh * n1 * d;
-  for (int c = tid; c < d; c += blockDim.x) {
-    for (int i = 0; i < n1; ++i) {
-      double v = Bg[i * d + c];
-      for (int k = 0; k < i; ++k) v -= G[i * n1 + k] * A[k * d + c];
-      A[i * d + c] = v / G[i * n1 + i];
-    }
-    for (int i = n1 - 1; i >= 0; --i) {
-      double v = A[i * d + c];
-      for (int k = i + 1; k < n1; ++k) v -= G[k * n1 + i] * A[k * d + c];
-      A[i * d + c] = v / G[i * n1 + i];
+  // solve L L^T X = B, 32 right-hand sides at a time: column c = tid / 8 of the chunk, eight
+  // threads (one warp quarter) share each row's dot product
+  {
+    const double* Bg = L.ridgeB + (size_t)bh * n1 * d;
+    double* Y = G + n1 * n1;  // [n1][33]
+    const int col = tid >> 3, sub = tid & 7;
+    for (int c0 = 0; c0 < d; c0 += 32) {
+      __syncthreads();
+      for (int e = tid; e < n1 * 32; e += blockDim.x) Y[(e >> 5) * 33 + (e & 31)] = Bg[(e >> 5) * d + c0 + (e & 31)];
+      __syncthreads();
+      for (int i = 0; i < n1; ++i) {
+        double part = 0.0;
+        for (int k = sub; k < i; k += 8) part += G[i * n1 + k] * Y[k * 33 + col];
+        part += __shfl_xor_sync(0xffffffffu, part, 4);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        if (sub == 0) Y[i * 33 + col] = (Y[i * 33 + col] - part) / G[i * n1 + i];
+        __syncwarp();
+      }
+      for (int i = n1 - 1; i >= 0; --i) {
+        double part = 0.0;
+        for (int k = i + 1 + sub; k < n1; k += 8) part += G[k * n1 + i] * Y[k * 33 + col];
+        part += __shfl_xor_sync(0xffffffffu, part, 4);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        if (sub == 0) Y[i * 33 + col] = (Y[i * 33 + col] - part) / G[i * n1 + i];
+        __syncwarp();
+      }
+      __syncthreads();
+      for (int e = tid; e < n1 * 32; e += blockDim.x) A[(e >> 5) * d + c0 + (e & 31)] = Y[(e >> 5) * 33 + (e & 31)];
     }
   }
   __syncthreads();
-  // span basis: columns of S (they span range(S) = span{R_p}); pivoted Gram-Schmidt in place
+  // span of the residual rows = range(S), S = R^T W R.  Full rank is the common case: a
+  // Cholesky of S whose pivots all stay above 1e-10 of the largest diagonal entry proves it,
+  // and then the projector is the identity.  Otherwise an orthonormal basis U of range(S) comes
+  // from column-pivoted Gram-Schmidt on the columns of S (column norms scale like
+  // eigenvalue^2, so the cut is 1e-20 of the largest squared norm).
   double* S = G;
   const double* Sg = L.spanS + (size_t)bh * d * d;
-  for (int e = tid; e < d * d; e += blockDim.x) S[e] = Sg[e];  // S[i*d + c]: column c, entry i
-  __shared__ double cn[128];
-  __shared__ int used[128];
+  __shared__ double s_dmax;
+  for (int e = tid; e < d * d; e += blockDim.x) S[e] = Sg[e];
   __syncthreads();
-  for (int c = tid; c < d; c += blockDim.x) {
-    double s = 0.0;
-    for (int i = 0; i < d; ++i) s += S[i * d + c] * S[i * d + c];
-    cn[c] = s;
-    used[c] = 0;
-  }
-  __syncthreads();
-  __shared__ double s_tol;
   if (tid == 0) {
     double mx = 0.0;
-    for (int c = 0; c < d; ++c) mx = fmax(mx, cn[c]);
-    // column norms of S scale like eigenvalue^2; the span keeps eigenvalues > 1e-10 of the top
-    s_tol = mx * 1e-20;
+    for (int i = 0; i < d; ++i) mx = fmax(mx, S[i * d + i]);
+    s_dmax = mx;
   }
   __syncthreads();
   int rank = 0;
   int basis[128];
-  for (int step = 0; step < d; ++step) {
-    if (tid == 0) {
-      int best = -1;
-      double bv = 0.0;
-      for (int c = 0; c < d; ++c)
-        if (!used[c] && cn[c] > bv) {
-          bv = cn[c];
-          best = c;
+  bool full = s_dmax > 0.0 && chol_smem_tol(S, d, d, 1e-10 * s_dmax);
+  if (full) {
+    rank = d;
+  } else if (s_dmax > 0.0) {
+    for (int e = tid; e < d * d; e += blockDim.x) S[e] = Sg[e];  // S[i*d + c]: column c, entry i
+    __shared__ double cn[128];
+    __shared__ int used[128];
+    __shared__ double s_tol;
+    __syncthreads();
+    // column norms: 2 threads per column
+    for (int c = tid >> 1; c < d; c += blockDim.x >> 1) {
+      double sacc = 0.0;
+      for (int i = tid & 1; i < d; i += 2) sacc += S[i * d + c] * S[i * d + c];
+      sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
+      if ((tid & 1) == 0) {
+        cn[c] = sacc;
+        used[c] = 0;
+      }
+    }
+    __syncthreads();
+    if (tid < 32) {
+      double mx = 0.0;
+      for (int c = tid; c < d; c += 32) mx = fmax(mx, cn[c]);
+      for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (tid == 0) s_tol = mx * 1e-20;
+    }
+    __syncthreads();
+    for (int step = 0; step < d; ++step) {
+      if (tid < 32) {  // pivot: unused column of largest remaining norm (lowest index on ties)
+        double bv = -1.0;
+        int bi = -1;
+        for (int c = tid; c < d; c += 32)
+          if (!used[c] && cn[c] > bv) {
+            bv = cn[c];
+            bi = c;
+          }
+        for (int o = 16; o > 0; o >>= 1) {
+          const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+          if (ov > bv || (ov == bv && oi >= 0 && (bi < 0 || oi < bi))) {
+            bv = ov;
+            bi = oi;
+          }
         }
-      s_piv = (best >= 0 && bv > s_tol && bv > 0.0) ? best : -1;
-      if (s_piv >= 0) {
-        used[s_piv] = 1;
-        double s = 0.0;
-        for (int i = 0; i < d; ++i) s += S[i * d + s_piv] * S[i * d + s_piv];
-        s_norm = sqrt(s);
+        double nrm = 0.0;
+        if (bi >= 0 && bv > s_tol && bv > 0.0)
+          for (int i = tid; i < d; i += 32) nrm += S[i * d + bi] * S[i * d + bi];
+        for (int o = 16; o > 0; o >>= 1) nrm += __shfl_xor_sync(0xffffffffu, nrm, o);
+        if (tid == 0) {
+          s_piv = (bi >= 0 && bv > s_tol && bv > 0.0) ? bi : -1;
+          if (s_piv >= 0) {
+            used[s_piv] = 1;
+            s_norm = sqrt(nrm);
+          }
+        }
       }
-    }
-    __syncthreads();
-    const int pv = s_piv;
-    if (pv < 0) break;
-    for (int i = tid; i < d; i += blockDim.x) S[i * d + pv] /= s_norm;
-    __syncthreads();
-    for (int c = tid; c < d; c += blockDim.x) {
-      if (used[c]) continue;
-      double dot = 0.0;
-      for (int i = 0; i < d; ++i) dot += S[i * d + pv] * S[i * d + c];
-      double s = 0.0;
-      for (int i = 0; i < d; ++i) {
-        const double v = S[i * d + c] - dot * S[i * d + pv];
-        S[i * d + c] = v;
-        s += v * v;
+      __syncthreads();
+      const int pv = s_piv;
+      if (pv < 0) break;
+      for (int i = tid; i < d; i += blockDim.x) S[i * d + pv] /= s_norm;
+      __syncthreads();
+      // remove the new direction from every unused column: 2 threads per column
+      for (int c = tid >> 1; c < d; c += blockDim.x >> 1) {
+        const bool act = !used[c];
+        double dot = 0.0;
+        if (act)
+          for (int i = tid & 1; i < d; i += 2) dot += S[i * d + pv] * S[i * d + c];
+        dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+        double sacc = 0.0;
+        if (act)
+          for (int i = tid & 1; i < d; i += 2) {
+            const double v = S[i * d + c] - dot * S[i * d + pv];
+            S[i * d + c] = v;
+            sacc += v * v;
+          }
+        sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
+        if (act && (tid & 1) == 0) cn[c] = sacc;
       }
-      cn[c] = s;
+      basis[rank++] = pv;
+      __syncthreads();
     }
-    basis[rank++] = pv;
-    __syncthreads();
   }
-  // A <- (A U) U^T, one row of A per thread
+  // A <- (A U) U^T, one row of A per thread.  A full-rank span is all of R^d: the projector is
+  // the identity and A is kept as solved.
   for (int a = tid; a < n1; a += blockDim.x) {
-    double t[128];
-    for (int r = 0; r < rank; ++r) {
-      double s = 0.0;
-      for (int i = 0; i < d; ++i) s += A[a * d + i] * S[i * d + basis[r]];
-      t[r] = s;
+    if (rank < d) {
+      double t[128];
+      for (int r = 0; r < rank; ++r) {
+        double sacc = 0.0;
+        for (int i = 0; i < d; ++i) sacc += A[a * d + i] * S[i * d + basis[r]];
+        t[r] = sacc;
+      }
+      for (int i = 0; i < d; ++i) {
+        double sacc = 0.0;
+        for (int r = 0; r < rank; ++r) sacc += t[r] * S[i * d + basis[r]];
+        A[a * d + i] = sacc;
+      }
     }
-    for (int i = 0; i < d; ++i) {
-      double s = 0.0;
-      for (int r = 0; r < rank; ++r) s += t[r] * S[i * d + basis[r]];
-      A[a * d + i] = s;
-      L.A32[((size_t)bh * n1 + a) * d + i] = (float)s;
-    }
+    for (int i = 0; i < d; ++i) L.A32[((size_t)bh * n1 + a) * d + i] = (float)A[a * d + i];
   }
   if (tid == 0) {
     st.lambda = lam;
@@ -314,7 +382,7 @@ sparsepr_status launch_fit_apply(const Layout& L, void* O, int out_dtype, cudaSt
     cudaFuncSetAttribute(ridge_gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm);
     launch(ridge_gram_kernel, dim3(L.BH, (n1 + kRidgeRows - 1) / kRidgeRows), 256, gsm, st, L);
   }
-  const size_t ssm = (size_t)n1 * n1 * sizeof(double);
+  const size_t ssm = ridge_solve_smem(d);
   cudaFuncSetAttribute(ridge_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
   launch(ridge_solve_kernel, L.BH, 256, ssm, st, L);
   SPR_LAUNCH_CHECK();
@@ -329,8 +397,7 @@ namespace sparsepr {
 
 // The one-CTA-per-head solve on ridge matrices that are already in L.ridgeG / ridgeB / spanS.
 sparsepr_status launch_ridge_solve(const Layout& L, cudaStream_t st) {
-  const int n1 = L.d + 1;
-  const size_t ssm = (size_t)n1 * n1 * sizeof(double);
+  const size_t ssm = ridge_solve_smem(L.d);
   cudaFuncSetAttribute(ridge_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
   launch(ridge_solve_kernel, L.BH, 256, ssm, st, L);
   SPR_LAUNCH_CHECK();

@@ -5,8 +5,11 @@
 
 namespace sparsepr {
 
-// Query rows per attention work item (the block-sparse pass tiles each query group by this).
+// Query rows per attention work item (the block-sparse pass tiles each query group by this):
+// 64 for the fp32 CUDA-core kernel, 128 (one MMA M) for the bf16 tensor-core kernel.
 constexpr int kAttnTileM = 64;
+constexpr int kAttnTileMTc = 128;
+inline int attn_tile_m(const Layout& L) { return L.dtype == SPARSEPR_BF16 ? kAttnTileMTc : kAttnTileM; }
 
 sparsepr_status launch_plan(const Layout& L, const void* Q, const void* K, bool warm, int iters,
                             cudaStream_t st);
@@ -14,8 +17,11 @@ sparsepr_status launch_installed_partition(const Layout& L, cudaStream_t st);
 sparsepr_status launch_permute(const Layout& L, const void* Q, const void* K, const void* V,
                                cudaStream_t st);
 sparsepr_status launch_attention(const Layout& L, cudaStream_t st, cudaEvent_t ev_start, cudaEvent_t ev_stop);
+sparsepr_status launch_attention_tc(const Layout& L, cudaStream_t st, cudaEvent_t ev_start, cudaEvent_t ev_stop);
 sparsepr_status launch_fit_apply(const Layout& L, void* O, int out_dtype, cudaStream_t st);
 sparsepr_status launch_ridge_solve(const Layout& L, cudaStream_t st);
+bool km_tc_supported(const Layout& L, bool keys);
+sparsepr_status launch_kmeans_assign_tc(const Layout& L, bool keys, const void* K, int it, cudaStream_t st);
 
 // Upper bound of the number of query tiles of one head: sum_g ceil(n_g / tile) <= N/tile + C_q.
 inline int max_query_tiles(const Layout& L, int tile) { return (L.N + tile - 1) / tile + L.Cq; }

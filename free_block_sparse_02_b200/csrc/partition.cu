@@ -36,53 +36,44 @@ __global__ void metric_kernel(Layout L, const T* __restrict__ Q) {
   L.M[((size_t)bh * L.d + a) * L.d + b] = acc / L.d;
 }
 
-// Partial key Gram G = sum_t k_t k_t^T over one N-chunk (fp64).  Used only for the constant
-// sum_t ||f_t||^2 = <M, G> of the k-means objective.
+// Objective constant sum_t ||f_t||^2 = sum_t k_t^T M k_t of the key k-means (it only scales the
+// relative stop test, so fp32 products with an fp64 block sum are ample).  64 keys per block;
+// M is staged in shared memory as fp32, thread (key p = tid/4, quarter q) forms d/4 entries of
+// M k_p and their dot with k_p.
 template <typename T>
-__global__ void __launch_bounds__(256) gram_part_kernel(Layout L, const T* __restrict__ K) {
-  extern __shared__ double sh_rows[];  // [32][d]
-  const int bh = blockIdx.x, part = blockIdx.y, d = L.d;
-  const int chunk = (L.N + L.n_gram_parts - 1) / L.n_gram_parts;
-  const int t0 = part * chunk, t1 = min(L.N, t0 + chunk);
-  const T* k = K + (size_t)bh * L.N * d;
-  const int ne = d * d;
-  double acc[64];
-#pragma unroll
-  for (int i = 0; i < 64; ++i) acc[i] = 0.0;
-  for (int base = t0; base < t1; base += 32) {
-    const int nr = min(32, t1 - base);
-    __syncthreads();
-    for (int e = threadIdx.x; e < nr * d; e += blockDim.x)
-      sh_rows[e] = (double)to_f32(k[(size_t)(base + e / d) * d + (e % d)]);
-    __syncthreads();
-    for (int r = 0; r < nr; ++r) {
-      const double* row = sh_rows + r * d;
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const int e = threadIdx.x + i * 256;
-        if (e < ne) acc[i] += row[e / d] * row[e % d];
-      }
-    }
-  }
-  double* out = L.gram_part + ((size_t)bh * L.n_gram_parts + part) * ne;
-#pragma unroll
-  for (int i = 0; i < 64; ++i) {
-    const int e = threadIdx.x + i * 256;
-    if (e < ne) out[e] = acc[i];
-  }
-}
-
-__global__ void __launch_bounds__(256) gram_reduce_kernel(Layout L) {
+__global__ void __launch_bounds__(256) key_norms_kernel(Layout L, const T* __restrict__ K) {
+  extern __shared__ float shm[];
+  const int d = L.d, bh = blockIdx.y, tid = threadIdx.x;
+  const int DP = d + 1;
+  float* Ms = shm;              // [d][DP]
+  float* Ks = Ms + d * DP;      // [64][DP]
   __shared__ double red[8];
-  const int bh = blockIdx.x, ne = L.d * L.d;
-  double v = 0.0;
-  for (int e = threadIdx.x; e < ne; e += blockDim.x) {
-    double g = 0.0;
-    for (int p = 0; p < L.n_gram_parts; ++p) g += L.gram_part[((size_t)bh * L.n_gram_parts + p) * ne + e];
-    v += g * L.M[(size_t)bh * ne + e];
+  const int p0 = blockIdx.x * 64, np = min(64, L.N - p0);
+  const double* M = L.M + (size_t)bh * d * d;
+  for (int e = tid; e < d * d; e += 256) Ms[(e / d) * DP + (e % d)] = (float)M[e];
+  for (int e = tid; e < 64 * d; e += 256) {
+    const int p = e / d, a = e % d;
+    Ks[p * DP + a] = p < np ? to_f32(K[((size_t)bh * L.N + p0 + p) * d + a]) : 0.f;
   }
-  v = block_sum(v, red);
-  if (threadIdx.x == 0) L.T0k[bh] = v;
+  __syncthreads();
+  const int p = tid >> 2, q = tid & 3, dq = d >> 2;
+  const float* kp = Ks + p * DP;
+  float part = 0.f;
+  for (int a = q * dq; a < (q + 1) * dq; ++a) {
+    const float* Mr = Ms + a * DP;
+    float u = 0.f;
+    for (int b = 0; b < d; ++b) u = fmaf(Mr[b], kp[b], u);
+    part = fmaf(u, kp[a], part);
+  }
+  part += __shfl_xor_sync(0xffffffffu, part, 1);
+  part += __shfl_xor_sync(0xffffffffu, part, 2);
+  if (tid < 64 && tid < np) {
+    float kk = 0.f;
+    for (int a = 0; a < d; ++a) kk = fmaf(Ks[tid * DP + a], Ks[tid * DP + a], kk);
+    L.knorm[(size_t)bh * L.N + p0 + tid] = sqrtf(kk);
+  }
+  const double tot = block_sum((q == 0 && p < np) ? (double)part : 0.0, red);
+  if (tid == 0) atomicAdd(L.T0k + bh, tot);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -166,6 +157,18 @@ __global__ void km_reset_kernel(Layout L, int which, int iters) {
 //   keys:    c_j (key space), W_j = M c_j, bias_j = c_j^T M c_j
 //   queries: nu_g (response space), W_g = nu_g, bias_g = ||nu_g||^2
 // ------------------------------------------------------------------------------------------
+// x = hi + mid + lo in bf16 (each term the bf16 rounding of what the previous ones left),
+// written at index i of three planes `plane` elements apart.
+__device__ __forceinline__ void split3(double x, __nv_bfloat16* base, size_t plane, size_t i) {
+  const __nv_bfloat16 h = __double2bfloat16(x);
+  const double r1 = x - (double)__bfloat162float(h);
+  const __nv_bfloat16 m = __double2bfloat16(r1);
+  const double r2 = r1 - (double)__bfloat162float(m);
+  base[i] = h;
+  base[plane + i] = m;
+  base[2 * plane + i] = __double2bfloat16(r2);
+}
+
 __device__ __forceinline__ bool km_should_stop(const double* J, int it, int iters, float tol) {
   if (it >= iters) return true;
   if (it >= 2 && tol >= 0.f) {
@@ -199,6 +202,7 @@ __global__ void __launch_bounds__(128) kprep_kernel(Layout L, int it, int iters)
     L.kW64[gj * d + a] = w;
     L.kW32[gj * d + a] = (float)w;
     L.ksum[gj * d + a] = 0.0;
+    split3(w, L.kWb, (size_t)L.BH * L.Ckp * d, ((size_t)bh * L.Ckp + j) * d + a);
   }
   const double bias = block_sum(a < d ? c[a] * w : 0.0, red);
   const double wn = block_sum(a < d ? w * w : 0.0, red);
@@ -231,6 +235,7 @@ __global__ void __launch_bounds__(128) qprep_kernel(Layout L, int it, int iters)
     nn += v * v;
     L.qW32[gg * D + a] = (float)v;
     L.qsum[gg * D + a] = 0.0;
+    split3(v, L.qWb, (size_t)L.BH * L.Cqp * L.Dq, ((size_t)bh * L.Cqp + g) * L.Dq + a);
   }
   nn = block_sum(nn, red);
   if (threadIdx.x == 0) {
@@ -242,16 +247,24 @@ __global__ void __launch_bounds__(128) qprep_kernel(Layout L, int it, int iters)
 }
 
 // ------------------------------------------------------------------------------------------
-// Lloyd step 2: assignment of 64 points per block against all groups, with fp64 sums.
-// Thread (pg, cg) = (tid / 16, tid % 16) scores points 4pg..4pg+3 against groups cg + 16i of
-// the current 64-group chunk.  Feature rows: keys (d dims, exact in fp32 and fp64) or the
-// normalised responses (C_k dims; fp32 copy for scoring, fp64 for tie-breaks and sums).
+// Lloyd step 2: assignment of 128 points per block against all groups, with fp64 sums.
+// Thread (pg, cg) = (tid / 16, tid % 16) scores points pg + 16 r (r < 8) against groups
+// cg + 16 i (i < 4) of the current 64-group chunk (register tile 8 x 4).  Feature rows: keys
+// (d dims; bf16/fp32 values are exact in fp32 and fp64) or the normalised responses (C_k dims;
+// an fp32 copy for scoring and sums, fp64 for the tie-break).  Each fp32 score carries a
+// rounding bound; a point whose two best scores are within it is re-decided over all groups in
+// fp64.  The chosen group's exact fp64 score feeds the objective.
 // ------------------------------------------------------------------------------------------
 struct KeyFeat {};
 struct QueryFeat {};
 
-constexpr int kAsgPts = 64;
+constexpr int kAsgPts = 128;
 constexpr int kAsgChunk = 64;
+
+inline size_t assign_smem_bytes(int D) {
+  return (size_t)(kAsgPts + kAsgChunk) * (D + 1) * 4 + kAsgChunk * 4 + kAsgPts * 4 /*xnorm*/ +
+         2 * kAsgPts * 4 /*lab, order*/ + kAsgPts * 4 /*refine*/ + kAsgPts * 8 /*a64*/;
+}
 
 template <typename T, typename Feat>
 __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* __restrict__ K, int it) {
@@ -273,49 +286,66 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
   const float* WN = kKeys ? L.kwnorm + (size_t)bh * C : L.qwnorm + (size_t)bh * C;
 
   extern __shared__ float smem[];
-  float* Xs = smem;                        // [64][DP]
-  float* Ws = Xs + kAsgPts * DP;           // [64][DP]
-  float* Bs = Ws + kAsgChunk * DP;         // [64]
-  float* xnorm = Bs + kAsgChunk;           // [64]
-  int* lab = (int*)(xnorm + kAsgPts);      // [64]
-  int* order = lab + kAsgPts;              // [64]
-  double* a64 = (double*)(order + kAsgPts);  // [64]
-  __shared__ float s_wmax, s_bmax;
-  __shared__ int s_refine[kAsgPts];
+  float* Xs = smem;                          // [128][DP]
+  float* Ws = Xs + kAsgPts * DP;             // [64][DP]
+  float* Bs = Ws + kAsgChunk * DP;           // [64]
+  float* xnorm = Bs + kAsgChunk;             // [128]
+  int* lab = (int*)(xnorm + kAsgPts);        // [128]
+  int* order = lab + kAsgPts;                // [128]
+  int* refine = order + kAsgPts;             // [128]
+  double* a64 = (double*)(refine + kAsgPts); // [128]
+  __shared__ float s_red[2][8];
   __shared__ double red[8];
 
-  const int tid = threadIdx.x;
-  // features
-  for (int e = tid; e < kAsgPts * D; e += 256) {
-    const int p = e / D, a = e % D;
-    float v = 0.f;
-    if (p < np) {
-      if constexpr (kKeys) v = to_f32(K[((size_t)bh * L.N + p0 + p) * D + a]);
-      else v = L.r32[((size_t)bh * L.N + p0 + p) * D + a];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // features: two threads per row, every other element
+  {
+    const int p = tid >> 1, h = tid & 1;
+    const size_t row = (size_t)bh * L.N + p0 + p;
+    for (int a = h; a < D; a += 2) {
+      float v = 0.f;
+      if (p < np) {
+        if constexpr (kKeys) v = to_f32(K[row * D + a]);
+        else v = L.r32[row * D + a];
+      }
+      Xs[p * DP + a] = v;
     }
-    Xs[p * DP + a] = v;
   }
-  if (tid == 0) {
+  // largest centroid-weight norm and |bias| (block max)
+  {
     float wm = 0.f, bm = 0.f;
-    for (int j = 0; j < C; ++j) {
+    for (int j = tid; j < C; j += 256) {
       wm = fmaxf(wm, WN[j]);
       bm = fmaxf(bm, fabsf(B32[j]));
     }
-    s_wmax = wm;
-    s_bmax = bm;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+    }
+    if (lane == 0) {
+      s_red[0][warp] = wm;
+      s_red[1][warp] = bm;
+    }
   }
   __syncthreads();
+  float s_wmax = 0.f, s_bmax = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    s_wmax = fmaxf(s_wmax, s_red[0][w]);
+    s_bmax = fmaxf(s_bmax, s_red[1][w]);
+  }
   if (tid < kAsgPts) {
     float s = 0.f;
-    for (int a = 0; a < D; ++a) s += Xs[tid * DP + a] * Xs[tid * DP + a];
+    for (int a = 0; a < D; ++a) s = fmaf(Xs[tid * DP + a], Xs[tid * DP + a], s);
     xnorm[tid] = sqrtf(s);
   }
 
   const int pg = tid >> 4, cg = tid & 15;
-  float b1[4], b2[4];
-  int i1[4];
+  float b1[8], b2[8];
+  int i1[8];
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
+  for (int r = 0; r < 8; ++r) {
     b1[r] = INFINITY;
     b2[r] = INFINITY;
     i1[r] = 0x7fffffff;
@@ -323,25 +353,26 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
   for (int c0 = 0; c0 < C; c0 += kAsgChunk) {
     const int nc = min(kAsgChunk, C - c0);
     __syncthreads();
-    for (int e = tid; e < kAsgChunk * D; e += 256) {
-      const int j = e / D, a = e % D;
-      Ws[j * DP + a] = j < nc ? W32[(size_t)(c0 + j) * D + a] : 0.f;
+    {
+      const int j = tid >> 2, q = tid & 3;
+      for (int a = q; a < D; a += 4) Ws[j * DP + a] = j < nc ? W32[(size_t)(c0 + j) * D + a] : 0.f;
+      if (tid < kAsgChunk) Bs[tid] = tid < nc ? B32[c0 + tid] : 0.f;
     }
-    if (tid < kAsgChunk) Bs[tid] = tid < nc ? B32[c0 + tid] : 0.f;
     __syncthreads();
-    float acc[4][4];
+    float acc[8][4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+    for (int r = 0; r < 8; ++r)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[r][i] = 0.f;
+#pragma unroll 2
     for (int a = 0; a < D; ++a) {
-      float x[4], w[4];
+      float x[8], w[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) x[r] = Xs[(pg * 4 + r) * DP + a];
+      for (int r = 0; r < 8; ++r) x[r] = Xs[(pg + 16 * r) * DP + a];
 #pragma unroll
       for (int i = 0; i < 4; ++i) w[i] = Ws[(cg + 16 * i) * DP + a];
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int r = 0; r < 8; ++r)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[r][i] = fmaf(x[r], w[i], acc[r][i]);
     }
@@ -349,10 +380,10 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
     for (int i = 0; i < 4; ++i) {
       const int j = cg + 16 * i;
       if (j >= nc) continue;
+      const int gj = c0 + j;
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
+      for (int r = 0; r < 8; ++r) {
         const float sc = Bs[j] - 2.f * acc[r][i];
-        const int gj = c0 + j;
         if (sc < b1[r] || (sc == b1[r] && gj < i1[r])) {
           b2[r] = b1[r];
           b1[r] = sc;
@@ -365,7 +396,7 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
   }
   // merge the 16 partial top-2 lists of each point (lanes of one half-warp)
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
+  for (int r = 0; r < 8; ++r) {
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) {
       const float ob1 = __shfl_xor_sync(0xffffffffu, b1[r], o);
@@ -383,63 +414,73 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
   const float u = 5.9604645e-8f;  // 2^-24
   if (cg == 0) {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int p = pg * 4 + r;
+    for (int r = 0; r < 8; ++r) {
+      const int p = pg + 16 * r;
       const float delta = 4.f * (D + 2) * u * xnorm[p] * s_wmax + 2.f * u * s_bmax;
       lab[p] = (i1[r] >= 0 && i1[r] < C) ? i1[r] : 0;  // non-finite scores never yield a bad label
-      s_refine[p] = (p < np) && !(b2[r] - b1[r] > 2.f * delta);
+      refine[p] = (p < np) && !(b2[r] - b1[r] > 2.f * delta);
     }
   }
   __syncthreads();
 
-  // fp64 re-decision of points whose best two scores are within the rounding bound, and the
-  // exact score of every chosen group (for the objective).
-  const int warp = tid >> 5, lane = tid & 31;
+  // fp64 re-decision of the (rare) points within the rounding bound: one warp per point, lanes
+  // over groups, lowest index on exact ties
   for (int p = warp; p < np; p += 8) {
+    if (!refine[p]) continue;
     const size_t row = (size_t)bh * L.N + p0 + p;
-    auto xval = [&](int a) -> double {
-      if constexpr (kKeys) return (double)to_f32(K[row * D + a]);
-      else return L.r64[row * D + a];
-    };
-    int best = lab[p];
-    double bestv;
-    if (s_refine[p]) {
-      bestv = INFINITY;
-      best = 0x7fffffff;
-      for (int j = 0; j < C; ++j) {
-        double dot = 0.0;
-        for (int a = lane; a < D; a += 32) dot += xval(a) * W64[(size_t)j * D + a];
-        dot = warp_sum(dot);
-        const double sc = B64[j] - 2.0 * dot;
-        if (sc < bestv) {  // ascending j: strict < keeps the lowest index on ties
-          bestv = sc;
-          best = j;
-        }
-      }
-    } else {
+    double bestv = INFINITY;
+    int best = 0x7fffffff;
+    for (int j = lane; j < C; j += 32) {
+      const double* w = W64 + (size_t)j * D;
       double dot = 0.0;
-      for (int a = lane; a < D; a += 32) dot += xval(a) * W64[(size_t)best * D + a];
-      dot = warp_sum(dot);
-      bestv = B64[best] - 2.0 * dot;
+      for (int a = 0; a < D; ++a) {
+        double x;
+        if constexpr (kKeys) x = (double)Xs[p * DP + a];
+        else x = L.r64[row * D + a];
+        dot += x * w[a];
+      }
+      const double sc = B64[j] - 2.0 * dot;
+      if (sc < bestv) {  // ascending j per lane: strict < keeps the lower index
+        bestv = sc;
+        best = j;
+      }
     }
-    if (lane == 0) {
-      lab[p] = (best >= 0 && best < C) ? best : 0;
-      a64[p] = bestv;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double ov = __shfl_xor_sync(0xffffffffu, bestv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, best, o);
+      if (ov < bestv || (ov == bestv && oi < best)) {
+        bestv = ov;
+        best = oi;
+      }
     }
+    if (lane == 0) lab[p] = (best >= 0 && best < C) ? best : 0;
   }
   __syncthreads();
-  // labels out, objective, refined count
+  // exact fp64 score of each point's group (objective): one thread per point
+  if (tid < np) {
+    const int l = lab[tid];
+    const double* w = W64 + (size_t)l * D;
+    const size_t row = (size_t)bh * L.N + p0 + tid;
+    double dot = 0.0;
+    for (int a = 0; a < D; ++a) {
+      double x;
+      if constexpr (kKeys) x = (double)Xs[tid * DP + a];
+      else x = L.r64[row * D + a];
+      dot += x * w[a];
+    }
+    a64[tid] = B64[l] - 2.0 * dot;
+  }
+  __syncthreads();
   int* labels = (kKeys ? L.klabel : L.qlabel) + (size_t)bh * L.N;
   if (tid < np) labels[p0 + tid] = lab[tid];
   const double jsum = block_sum(tid < np ? a64[tid] : 0.0, red);
-  int nref = 0;
-  if (tid < np) nref = s_refine[tid];
-  nref = __syncthreads_count(nref);
+  const int nref = __syncthreads_count(tid < np ? refine[tid] : 0);
   if (tid == 0) {
     atomicAdd((kKeys ? L.kJ : L.qJ) + (size_t)bh * L.iters_cap + it, jsum);
     if (nref) atomicAdd((kKeys ? L.krefined : L.qrefined) + bh, nref);
   }
-  // stable order of the block's points by label, then one fp64 atomic per (run, dim)
+  // stable order of the block's points by label, then fp64 sums per (run, dim)
   if (tid < np) {
     const int l = lab[tid];
     int rk = 0;
@@ -452,31 +493,28 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
   __syncthreads();
   double* sums = (kKeys ? L.ksum : L.qsum) + (size_t)bh * C * D;
   int* counts = (kKeys ? L.kcount : L.qcount) + (size_t)bh * C;
-  for (int a = tid; a < D; a += 256) {
-    double acc = 0.0;
-    for (int q = 0; q < np; ++q) {
-      const int p = order[q];
-      const size_t row = (size_t)bh * L.N + p0 + p;
-      double v;
-      if constexpr (kKeys) v = (double)to_f32(K[row * D + a]);
-      else v = L.r64[row * D + a];
-      acc += v;
-      if (q == np - 1 || lab[order[q + 1]] != lab[p]) {
-        atomicAdd(sums + (size_t)lab[p] * D + a, acc);
-        acc = 0.0;
+  const int nparts = D >= 256 ? 1 : 256 / D;
+  if (tid < nparts * D) {
+    const int a = tid % D, part = tid / D;
+    const int q0 = part * np / nparts, q1 = (part + 1) * np / nparts;
+    for (int a2 = a; a2 < D; a2 += (D >= 256 ? 256 : D)) {
+      double acc = 0.0;
+      for (int q = q0; q < q1; ++q) {
+        const int p = order[q];
+        acc += (double)Xs[p * DP + a2];
+        if (q == q1 - 1 || lab[order[q + 1]] != lab[p]) {
+          atomicAdd(sums + (size_t)lab[p] * D + a2, acc);
+          acc = 0.0;
+        }
       }
+      if (D < 256) break;
     }
   }
-  if (tid == 0) {
-    int run = 0;
-    for (int q = 0; q < np; ++q) {
-      ++run;
-      const int l = lab[order[q]];
-      if (q == np - 1 || lab[order[q + 1]] != l) {
-        atomicAdd(counts + l, run);
-        run = 0;
-      }
-    }
+  if (tid < np && (tid == 0 || lab[order[tid - 1]] != lab[order[tid]])) {
+    const int l = lab[order[tid]];
+    int q = tid + 1;
+    while (q < np && lab[order[q]] == l) ++q;
+    atomicAdd(counts + l, q - tid);
   }
 }
 
@@ -531,7 +569,26 @@ __global__ void __launch_bounds__(256) qresp_kernel(Layout L, const T* __restric
     const size_t o = ((size_t)bh * L.N + p0 + p) * Ck + j;
     L.r64[o] = v;
     L.r32[o] = (float)v;
+    split3(v, L.rb, (size_t)L.BH * L.N * L.Dq, ((size_t)bh * L.N + p0 + p) * L.Dq + j);
     nrm += v * v;
+  }
+  for (int e = tid; e < 32 * (L.Dq - Ck); e += 256) {  // zero the padding columns
+    const int p = e / (L.Dq - Ck), j = Ck + e % (L.Dq - Ck);
+    if (p >= np) continue;
+    const size_t o = ((size_t)bh * L.N + p0 + p) * L.Dq + j;
+    const size_t plane = (size_t)L.BH * L.N * L.Dq;
+    const __nv_bfloat16 z = __float2bfloat16(0.f);
+    L.rb[o] = z;
+    L.rb[plane + o] = z;
+    L.rb[2 * plane + o] = z;
+  }
+  if (tid < np) {
+    double q2 = 0.0;
+    for (int j = 0; j < Ck; ++j) {
+      const double v = rs[tid * Ck + j] * inv[tid];
+      q2 += v * v;
+    }
+    L.rnorm[(size_t)bh * L.N + p0 + tid] = (float)sqrt(q2);
   }
   nrm = block_sum(nrm, red);
   if (tid == 0) atomicAdd(L.T0q + bh, nrm);
@@ -823,8 +880,10 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
                                   cudaStream_t st) {
   const int d = L.d;
   launch(metric_kernel<T>, dim3(L.BH, d), 128, 0, st, L, Q);
-  launch(gram_part_kernel<T>, dim3(L.BH, L.n_gram_parts), 256, 32 * d * sizeof(double), st, L, K);
-  launch(gram_reduce_kernel, L.BH, 256, 0, st, L);
+  cudaMemsetAsync(L.T0k, 0, sizeof(double) * L.BH, st);
+  const size_t kn_smem = (size_t)(d + 64) * (d + 1) * sizeof(float);
+  cudaFuncSetAttribute(key_norms_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kn_smem);
+  launch(key_norms_kernel<T>, dim3((L.N + 63) / 64, L.BH), 256, kn_smem, st, L, K);
   if (!warm) {
     launch(km_draw_kernel, L.BH, 128, 0, st, L, 0, L.Ck);
     launch(kcent_init_kernel<T>, dim3(L.BH, L.Ck), 128, 0, st, L, K);
@@ -832,14 +891,23 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
   SPR_LAUNCH_CHECK();
   launch(km_reset_kernel, L.BH, 128, 0, st, L, 0, iters);
   cudaMemsetAsync(L.T0q, 0, sizeof(double) * L.BH, st);
-  const size_t asg_smem_k = (size_t)(kAsgPts + kAsgChunk) * (d + 1) * 4 + (kAsgChunk + kAsgPts) * 4 +
-                            2 * kAsgPts * 4 + kAsgPts * 8;
+  // bf16 inputs with at most 256 groups score on the tensor cores; otherwise on CUDA cores
+  const bool tc_keys = km_tc_supported(L, true), tc_queries = km_tc_supported(L, false);
+  cudaMemsetAsync(L.kWb, 0, (size_t)3 * L.BH * L.Ckp * d * 2, st);
+  cudaMemsetAsync(L.qWb, 0, (size_t)3 * L.BH * L.Cqp * L.Dq * 2, st);
+  const size_t asg_smem_k = assign_smem_bytes(d);
   const int nblk = (L.N + kAsgPts - 1) / kAsgPts;
   cudaFuncSetAttribute(kmeans_assign_kernel<T, KeyFeat>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asg_smem_k);
   for (int it = 0; it <= iters; ++it) {
     launch(kprep_kernel, dim3(L.BH, L.Ck), 128, 0, st, L, it, iters);
-    if (it < iters)
-      launch(kmeans_assign_kernel<T, KeyFeat>, dim3(nblk, L.BH), 256, asg_smem_k, st, L, K, it);
+    if (it < iters) {
+      if (tc_keys) {
+        const sparsepr_status s = launch_kmeans_assign_tc(L, true, K, it, st);
+        if (s != SPARSEPR_OK) return s;
+      } else {
+        launch(kmeans_assign_kernel<T, KeyFeat>, dim3(nblk, L.BH), 256, asg_smem_k, st, L, K, it);
+      }
+    }
   }
   SPR_LAUNCH_CHECK();
   const size_t qr_smem = (size_t)(2 * 32 * (d + 1) + 32 * L.Ck) * sizeof(double);
@@ -851,18 +919,23 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
   }
   launch(km_reset_kernel, L.BH, 128, 0, st, L, 1, iters);
   SPR_LAUNCH_CHECK();
-  const size_t asg_smem_q = (size_t)(kAsgPts + kAsgChunk) * (L.Ck + 1) * 4 + (kAsgChunk + kAsgPts) * 4 +
-                            2 * kAsgPts * 4 + kAsgPts * 8;
+  const size_t asg_smem_q = assign_smem_bytes(L.Ck);
   cudaFuncSetAttribute(kmeans_assign_kernel<T, QueryFeat>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asg_smem_q);
   for (int it = 0; it <= iters; ++it) {
     launch(qprep_kernel, dim3(L.BH, L.Cq), 128, 0, st, L, it, iters);
-    if (it < iters)
-      launch(kmeans_assign_kernel<T, QueryFeat>, dim3(nblk, L.BH), 256, asg_smem_q, st, L, K, it);
+    if (it < iters) {
+      if (tc_queries) {
+        const sparsepr_status s = launch_kmeans_assign_tc(L, false, K, it, st);
+        if (s != SPARSEPR_OK) return s;
+      } else {
+        launch(kmeans_assign_kernel<T, QueryFeat>, dim3(nblk, L.BH), 256, asg_smem_q, st, L, K, it);
+      }
+    }
   }
   SPR_LAUNCH_CHECK();
   launch(group_sort_kernel, dim3(L.BH, 2), 32, 0, st, L);
   launch(route_select_kernel<T>, dim3(L.BH, L.Cq), 128, 0, st, L, Q);
-  launch(route_build_kernel, L.BH, 256, 0, st, L, kAttnTileM);
+  launch(route_build_kernel, L.BH, 256, 0, st, L, attn_tile_m(L));
   cudaFuncSetAttribute(probe_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kProbeSmem);
   launch(probe_select_kernel, L.BH, 1024, kProbeSmem, st, L);
   launch(plan_stats_kernel, (L.BH + 127) / 128, 128, 0, st, L);
@@ -878,7 +951,7 @@ sparsepr_status launch_plan(const Layout& L, const void* Q, const void* K, bool 
 
 sparsepr_status launch_installed_partition(const Layout& L, cudaStream_t st) {
   launch(group_sort_kernel, dim3(L.BH, 2), 32, 0, st, L);
-  launch(route_build_kernel, L.BH, 256, 0, st, L, kAttnTileM);
+  launch(route_build_kernel, L.BH, 256, 0, st, L, attn_tile_m(L));
   launch(probe_index_kernel, L.BH, 1024, 0, st, L);
   SPR_LAUNCH_CHECK();
   return SPARSEPR_OK;

@@ -31,7 +31,6 @@ std::atomic<long long> sparsepr::g_launches{0};
 namespace {
 
 constexpr int kMaxKeyGroupsBuilt = 256;  // query-response dimension of the assignment kernel
-constexpr int kGramParts = 32;
 
 sparsepr_status validate(const sparsepr_config* c) {
   if (!c) return SPARSEPR_ERR_INVALID_ARG;
@@ -78,7 +77,6 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   L.km_tol = c.km_tol;
   L.lambda = c.lambda;
   L.seed = c.seed;
-  L.n_gram_parts = kGramParts;
   size_t off = 0;
   auto take = [&](auto*& ptr, size_t bytes) {
     using P_ = std::remove_reference_t<decltype(ptr)>;
@@ -89,7 +87,6 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   take(L.status, 4);
   take(L.stats, BH * sizeof(sparsepr_head_stats));
   take(L.M, BH * d * d * 8);
-  take(L.gram_part, BH * kGramParts * d * d * 8);
   take(L.T0k, BH * 8);
   take(L.T0q, BH * 8);
   take(L.init_ids, BH * std::max(Ck, Cq) * 4);
@@ -120,6 +117,14 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   take(L.qlabel, BH * N * 4);
   take(L.qJ, BH * cap * 8);
   take(L.qrefined, BH * 4);
+  L.Ckp = (c.n_kgroups + 15) / 16 * 16;
+  L.Cqp = (c.n_qgroups + 15) / 16 * 16;
+  L.Dq = (c.n_kgroups + 63) / 64 * 64;
+  take(L.kWb, 3 * BH * (size_t)L.Ckp * d * 2);
+  take(L.qWb, 3 * BH * (size_t)L.Cqp * L.Dq * 2);
+  take(L.rb, 3 * BH * N * (size_t)L.Dq * 2);
+  take(L.knorm, BH * N * 4);
+  take(L.rnorm, BH * N * 4);
   take(L.kperm, BH * N * 4);
   take(L.kinv, BH * N * 4);
   take(L.koff, BH * (Ck + 1) * 4);

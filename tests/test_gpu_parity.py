@@ -63,35 +63,59 @@ def compare_partition(op, res_list, w):
         np.testing.assert_allclose(kc[bh], r["kcent"], rtol=1e-9, atol=1e-9)
 
 
+def _close(name, got, exp, atol, rel_l2):
+    if exp.size == 0:
+        assert got.size == 0
+        return
+    diff = np.abs(got - exp)
+    rl2 = np.linalg.norm(got - exp) / max(np.linalg.norm(exp), 1e-30)
+    assert diff.max() <= atol, f"{name}: max-abs {diff.max():.3e} > {atol}"
+    assert rl2 <= rel_l2, f"{name}: rel-L2 {rl2:.3e} > {rel_l2}"
+
+
 def compare_outputs(op, out, qf, kf, vf, w, atol, rel_l2):
-    """Oracle steps 6-9 on the GPU's own partition vs the GPU outputs."""
+    """GPU outputs vs the oracle on the GPU's own partition, stage by stage:
+    1. block-sparse and probe attention vs the oracle's (the dtype's output bar);
+    2. the ridge fit vs the oracle's ridge on the GPU's own probe rows (both fp64: tight);
+    3. the corrected output vs the oracle's correction applied to the GPU's O_sp (fp32);
+    4. end to end vs the oracle's output (the dtype's bar) wherever the fit is well posed:
+       fp32 inputs, or at least d+1 probes -- with fewer probes than unknowns the ridge map
+       amplifies the bf16 rounding of the probe residuals;
+    5. mean error on evaluation rows no worse than the oracle's, up to the path's rounding."""
     kl, ql = op.query(S.Q_KLABELS), op.query(S.Q_QLABELS)
     route, probes, pw = op.query(S.Q_ROUTE).astype(bool), op.query(S.Q_PROBES), op.query(S.Q_PROBE_W)
-    osp = op.query(S.Q_OSP)
-    od = op.query(S.Q_ODENSE)
-    O_gpu = out.float().cpu().numpy().reshape(-1, w.N, w.d)
+    osp = op.query(S.Q_OSP).astype(np.float64)
+    od = op.query(S.Q_ODENSE).astype(np.float64)
+    A_gpu = op.query(S.Q_FIT)
+    O_gpu = out.float().cpu().numpy().reshape(-1, w.N, w.d).astype(np.float64)
     errs = []
     for bh in range(O_gpu.shape[0]):
-        ref = O.outputs_given_partition(qf[bh], kf[bh], vf[bh], ql[bh], kl[bh], route[bh], probes[bh],
-                                        pw[bh], w.lam)
-        for name, got, exp in (("O_sp", osp[bh], ref["osp"]), ("O_dense", od[bh], ref["odense"]),
-                               ("O", O_gpu[bh], ref["O"])):
-            if exp.size == 0:
-                assert got.size == 0
-                continue
-            diff = np.abs(got - exp)
-            rl2 = np.linalg.norm(got - exp) / max(np.linalg.norm(exp), 1e-30)
-            assert diff.max() <= atol, f"head {bh} {name}: max-abs {diff.max():.3e} > {atol}"
-            assert rl2 <= rel_l2, f"head {bh} {name}: rel-L2 {rl2:.3e} > {rel_l2}"
+        p = probes[bh]
+        ref = O.outputs_given_partition(qf[bh], kf[bh], vf[bh], ql[bh], kl[bh], route[bh], p, pw[bh], w.lam)
+        _close(f"head {bh} O_sp", osp[bh], ref["osp"], atol, rel_l2)
+        _close(f"head {bh} O_dense", od[bh], ref["odense"], atol, rel_l2)
+        A_ref, _ = O.ridge_fit(osp[bh][p], od[bh], pw[bh], w.lam)
+        if len(p):
+            A_ref = O.restrict_to_residual_span(A_ref, od[bh] - osp[bh][p], pw[bh])
+        scale = 1.0 + np.abs(A_ref).max()
+        assert np.abs(A_gpu[bh] - A_ref).max() <= 1e-6 * scale, f"head {bh} fit"
+        O_app = O.apply_correction(osp[bh], A_gpu[bh])
+        O_app[p] = od[bh]
+        _close(f"head {bh} apply", O_gpu[bh], O_app, 1e-4 * max(1.0, np.abs(O_app).max()), 1e-5)
+        if w.dtype == configs.F32 or len(p) >= w.d + 1:
+            _close(f"head {bh} O", O_gpu[bh], ref["O"], atol, rel_l2)
         # quality on evaluation rows: all rows of small heads, else 2048 strided rows (the
         # paper's metric sample per head, Table C.1), probes excluded
         rows = np.arange(w.N) if w.N <= 4096 else (np.arange(2048) * w.N) // 2048
-        rows = rows[~np.isin(rows, probes[bh])]
+        rows = rows[~np.isin(rows, p)]
         dense = O.attention(qf[bh][rows], kf[bh], vf[bh])
         e_gpu = O.row_errors(O_gpu[bh][rows], dense).mean()
         e_orc = O.row_errors(ref["O"][rows], dense).mean()
         errs.append((e_gpu, e_orc))
-        assert e_gpu <= e_orc * (1 + 1e-3) + 1e-4, f"head {bh}: mean error {e_gpu} > oracle {e_orc}"
+        # no worse than the oracle's, up to the rounding of the path's arithmetic: fp32 products
+        # (1e-4) or bf16 attention probabilities (relative rounding 2^-9, allowance 5e-3)
+        slack = 1e-4 if w.dtype == configs.F32 else 5e-3
+        assert e_gpu <= e_orc * (1 + 1e-3) + slack, f"head {bh}: mean error {e_gpu} > oracle {e_orc}"
     return errs
 
 
