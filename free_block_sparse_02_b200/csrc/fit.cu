@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
     if (tid == 0) {
       atomicCAS(L.status, kDevOk, kDevNumeric);
       st.fit_retries = retries;
+      st.span_rank = d;  // nothing to project: A is zero
     }
     for (int e = tid; e < n1 * d; e += blockDim.x) {
       A[e] = 0.0;
@@ -304,28 +305,55 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
       __syncthreads();
     }
   }
-  // A <- (A U) U^T, one row of A per thread.  A full-rank span is all of R^d: the projector is
-  // the identity and A is kept as solved.
-  for (int a = tid; a < n1; a += blockDim.x) {
-    if (rank < d) {
-      double t[128];
-      for (int r = 0; r < rank; ++r) {
-        double sacc = 0.0;
-        for (int i = 0; i < d; ++i) sacc += A[a * d + i] * S[i * d + basis[r]];
-        t[r] = sacc;
-      }
-      for (int i = 0; i < d; ++i) {
-        double sacc = 0.0;
-        for (int r = 0; r < rank; ++r) sacc += t[r] * S[i * d + basis[r]];
-        A[a * d + i] = sacc;
-      }
+  // hand the basis to the projection kernel: columns r < rank of spanS are U's columns
+  __syncthreads();
+  if (rank < d) {
+    double* U = L.spanS + (size_t)bh * d * d;
+    for (int e = tid; e < d * rank; e += blockDim.x) {
+      const int i = e / rank, r = e % rank;
+      U[i * d + r] = S[i * d + basis[r]];
     }
-    for (int i = 0; i < d; ++i) L.A32[((size_t)bh * n1 + a) * d + i] = (float)A[a * d + i];
   }
   if (tid == 0) {
     st.lambda = lam;
     st.fit_retries = retries;
     st.span_rank = rank;
+  }
+}
+
+// A <- (A U) U^T with U (d x rank) the residual-span basis; 8 rows of A per block.  A
+// full-rank span is all of R^d: the projector is the identity and A is only copied to fp32.
+__global__ void __launch_bounds__(256) ridge_project_kernel(Layout L) {
+  extern __shared__ double shp2[];
+  const int bh = blockIdx.x, d = L.d, n1 = d + 1, tid = threadIdx.x;
+  const int rank = L.P > 0 ? L.stats[bh].span_rank : d;
+  const int a0 = blockIdx.y * 8, na = min(8, n1 - a0);
+  double* A = L.A64 + (size_t)bh * n1 * d;
+  float* A32 = L.A32 + (size_t)bh * n1 * d;
+  if (rank >= d) {
+    for (int e = tid; e < na * d; e += blockDim.x) A32[(size_t)a0 * d + e] = (float)A[(size_t)a0 * d + e];
+    return;
+  }
+  double* U = shp2;                 // [d][rank]
+  double* Ar = U + d * rank;        // [8][d]
+  double* T = Ar + 8 * d;           // [8][rank]
+  const double* Ug = L.spanS + (size_t)bh * d * d;
+  for (int e = tid; e < d * rank; e += blockDim.x) U[e] = Ug[(e / rank) * d + (e % rank)];
+  for (int e = tid; e < na * d; e += blockDim.x) Ar[e] = A[(size_t)a0 * d + e];
+  __syncthreads();
+  for (int e = tid; e < na * rank; e += blockDim.x) {
+    const int r8 = e / rank, k = e % rank;
+    double acc = 0.0;
+    for (int i = 0; i < d; ++i) acc += Ar[r8 * d + i] * U[i * rank + k];
+    T[r8 * rank + k] = acc;
+  }
+  __syncthreads();
+  for (int e = tid; e < na * d; e += blockDim.x) {
+    const int r8 = e / d, i = e % d;
+    double acc = 0.0;
+    for (int k = 0; k < rank; ++k) acc += T[r8 * rank + k] * U[i * rank + k];
+    A[(size_t)a0 * d + e] = acc;
+    A32[(size_t)a0 * d + e] = (float)acc;
   }
 }
 
@@ -382,10 +410,8 @@ sparsepr_status launch_fit_apply(const Layout& L, void* O, int out_dtype, cudaSt
     cudaFuncSetAttribute(ridge_gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm);
     launch(ridge_gram_kernel, dim3(L.BH, (n1 + kRidgeRows - 1) / kRidgeRows), 256, gsm, st, L);
   }
-  const size_t ssm = ridge_solve_smem(d);
-  cudaFuncSetAttribute(ridge_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
-  launch(ridge_solve_kernel, L.BH, 256, ssm, st, L);
-  SPR_LAUNCH_CHECK();
+  const sparsepr_status s = launch_ridge_solve(L, st);
+  if (s != SPARSEPR_OK) return s;
   if (out_dtype == SPARSEPR_F32)
     return d == 64 ? launch_apply<float, 64>(L, O, st) : launch_apply<float, 128>(L, O, st);
   return d == 64 ? launch_apply<__nv_bfloat16, 64>(L, O, st) : launch_apply<__nv_bfloat16, 128>(L, O, st);
@@ -400,6 +426,9 @@ sparsepr_status launch_ridge_solve(const Layout& L, cudaStream_t st) {
   const size_t ssm = ridge_solve_smem(L.d);
   cudaFuncSetAttribute(ridge_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
   launch(ridge_solve_kernel, L.BH, 256, ssm, st, L);
+  const size_t psm = (size_t)(L.d * L.d + 8 * L.d + 8 * L.d) * sizeof(double);
+  cudaFuncSetAttribute(ridge_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
+  launch(ridge_project_kernel, dim3(L.BH, (L.d + 1 + 7) / 8), 256, psm, st, L);
   SPR_LAUNCH_CHECK();
   return SPARSEPR_OK;
 }

@@ -46,11 +46,11 @@ __host__ __device__ inline int km_tc_tmem_cols(int Np) {
 __host__ inline size_t km_tc_smem(int D, int Np, int xterms) {
   const size_t w = (size_t)3 * Np * D * 2;
   const size_t x = (size_t)xterms * kKmTile * D * 2;
-  return w + x + 1024 /*align*/ + 16384 /*bias, labels, order, list, scores, fp64 rows, barriers*/;
+  return w + x + 1024 /*align*/ + 24576 /*bias, labels, order, list, histogram, merge, scores, fp64 rows, barriers*/;
 }
 
 template <bool kKeys>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
     kmeans_assign_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                             Layout L, const __nv_bfloat16* __restrict__ K, int it, int tiles_per_cta) {
   const int bh = blockIdx.y;
@@ -76,13 +76,18 @@ __global__ void __launch_bounds__(128, 1)
   int* lab = (int*)(sB + 256);                       // [128]
   int* order = lab + kKmTile;                        // [128]
   int* rlist = order + kKmTile;                      // [128] points to re-decide
-  double* bval = (double*)(rlist + kKmTile);         // [128] score of the chosen group
-  double* xs64 = bval + kKmTile;                     // [4 warps][256] fp64 features
-  uint64_t* bars = (uint64_t*)(xs64 + 4 * 256);      // w_full, x_full, mma_done
+  int* hist = rlist + kKmTile;                       // [256] points per label in the tile
+  int* cursor = hist + 256;                          // [256] next slot per label
+  float* mb1 = (float*)(cursor + 256);               // [128] partial best / second / index
+  float* mb2 = mb1 + kKmTile;
+  int* mi1 = (int*)(mb2 + kKmTile);
+  double* bval = (double*)(mi1 + kKmTile);           // [128] score of the chosen group
+  double* xs64 = bval + kKmTile;                     // [8 warps][256] fp64 features
+  uint64_t* bars = (uint64_t*)(xs64 + 8 * 256);      // w_full, x_full, mma_done
   uint32_t* tmem_slot = (uint32_t*)(bars + 3);
   __shared__ volatile int s_abort;
   __shared__ float s_wmax, s_bmax;
-  __shared__ double red[4];
+  __shared__ double red[8];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const float* B32 = kKeys ? L.kbias32 + (size_t)bh * C : L.qbias32 + (size_t)bh * C;
@@ -102,10 +107,10 @@ __global__ void __launch_bounds__(128, 1)
     tmem_alloc(tmem_slot, tcols);
     tmem_relinquish();
   }
-  for (int j = tid; j < 256; j += 128) sB[j] = j < C ? B32[j] : INFINITY;
+  for (int j = tid; j < 256; j += blockDim.x) sB[j] = j < C ? B32[j] : INFINITY;
   {
     float wm = 0.f, bm = 0.f;
-    for (int j = tid; j < C; j += 128) {
+    for (int j = tid; j < C; j += blockDim.x) {
       wm = fmaxf(wm, WN[j]);
       bm = fmaxf(bm, fabsf(B32[j]));
     }
@@ -114,7 +119,7 @@ __global__ void __launch_bounds__(128, 1)
       wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
       bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
     }
-    __shared__ float pw[4], pb[4];
+    __shared__ float pw[8], pb[8];
     if (lane == 0) {
       pw[warp] = wm;
       pb[warp] = bm;
@@ -123,8 +128,13 @@ __global__ void __launch_bounds__(128, 1)
     __syncthreads();
     tc_fence_after();
     if (tid == 0) {
-      s_wmax = fmaxf(fmaxf(pw[0], pw[1]), fmaxf(pw[2], pw[3]));
-      s_bmax = fmaxf(fmaxf(pb[0], pb[1]), fmaxf(pb[2], pb[3]));
+      float a = 0.f, b = 0.f;
+      for (int w = 0; w < 8; ++w) {
+        a = fmaxf(a, pw[w]);
+        b = fmaxf(b, pb[w]);
+      }
+      s_wmax = a;
+      s_bmax = b;
     }
   }
   const uint32_t tmem = *tmem_slot;
@@ -142,6 +152,9 @@ __global__ void __launch_bounds__(128, 1)
   const float u = 4.76837158e-7f;  // 2^-21: covers the three-term split and fp32 accumulation
   double jsum = 0.0;
   int nref = 0;
+  __shared__ int s_nlist;
+  if (tid == 0) s_nlist = 0;
+  __syncthreads();
   for (int ti = 0; ti < ntile && !s_abort; ++ti) {
     const int p0 = (tile0 + ti) * kKmTile;
     const int np = min(kKmTile, L.N - p0);
@@ -174,14 +187,16 @@ __global__ void __launch_bounds__(128, 1)
       mma_commit(bars + 2);
     }
     __syncwarp();
-    // epilogue: thread tid = point p0 + tid, TMEM lane tid
+    // epilogue: point q = tid % 128 (TMEM lane q); warps w and w+4 read alternate 32-column
+    // chunks of that lane's scores, then merge
     const bool waited = mbar_wait(bars + 2, ti & 1, &s_abort);
     if (__syncthreads_or(!waited)) break;  // uniform: every thread leaves or none does
     tc_fence_after();
+    const int q = tid & 127, half = tid >> 7;
     float b1 = INFINITY, b2 = INFINITY;
     int i1 = 0x7fffffff;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    for (int c0 = 0; c0 < Np; c0 += 32) {
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    for (int c0 = half * 32; c0 < Np; c0 += 64) {
       uint32_t r[32];
       tmem_ld32(tmem + lane_base + c0, r);  // c0 + 32 <= tcols: tcols is a power of two >= 32, >= Np
       tmem_wait_ld();
@@ -199,23 +214,39 @@ __global__ void __launch_bounds__(128, 1)
         }
       }
     }
-    const bool valid = tid < np;
-    const size_t row = (size_t)bh * L.N + p0 + tid;
-    const float xn = valid ? (kKeys ? L.knorm[row] : L.rnorm[row]) : 0.f;
-    const float delta = 4.f * (Dreal + 8) * u * xn * s_wmax + 2.f * u * s_bmax;
-    const bool ref = valid && !(b2 - b1 > 2.f * delta);
-    __shared__ int s_nlist;
-    if (tid == 0) s_nlist = 0;
+    if (half == 1) {
+      mb1[q] = b1;
+      mb2[q] = b2;
+      mi1[q] = i1;
+    }
     __syncthreads();
-    lab[tid] = (i1 >= 0 && i1 < C) ? i1 : 0;
-    bval[tid] = valid ? (double)b1 : 0.0;  // fp32-grade score of the chosen group (objective)
-    if (ref) rlist[atomicAdd(&s_nlist, 1)] = tid;
-    nref += ref ? 1 : 0;
+    const int np_ = np;
+    if (half == 0) {
+      const float ob1 = mb1[q], ob2 = mb2[q];
+      const int oi1 = mi1[q];
+      if (ob1 < b1 || (ob1 == b1 && oi1 < i1)) {
+        b2 = fminf(b1, ob2);
+        b1 = ob1;
+        i1 = oi1;
+      } else {
+        b2 = fminf(b2, ob1);
+      }
+      const bool valid = q < np_;
+      const size_t row = (size_t)bh * L.N + p0 + q;
+      const float xn = valid ? (kKeys ? L.knorm[row] : L.rnorm[row]) : 0.f;
+      const float delta = 4.f * (Dreal + 8) * u * xn * s_wmax + 2.f * u * s_bmax;
+      const bool ref = valid && !(b2 - b1 > 2.f * delta);
+      lab[q] = (i1 >= 0 && i1 < C) ? i1 : 0;
+      bval[q] = valid ? (double)b1 : 0.0;  // fp32-grade score of the chosen group (objective)
+      if (ref) rlist[atomicAdd(&s_nlist, 1)] = q;
+      nref += ref ? 1 : 0;
+    }
+    for (int j = tid; j < C; j += blockDim.x) hist[j] = 0;
     __syncthreads();
     // fp64 re-decision over every group (lowest index on exact ties): one warp per listed
     // point, its features staged in shared memory, lanes over groups
     const int nlist = s_nlist;
-    for (int li = warp; li < nlist; li += 4) {
+    for (int li = warp; li < nlist; li += 8) {
       const int p = rlist[li];
       const size_t rr = (size_t)bh * L.N + p0 + p;
       double* xs = xs64 + warp * 256;
@@ -259,24 +290,37 @@ __global__ void __launch_bounds__(128, 1)
       __syncwarp();
     }
     __syncthreads();
-    const double bestv = bval[tid];
-    if (valid) ((kKeys ? L.klabel : L.qlabel) + (size_t)bh * L.N)[p0 + tid] = lab[tid];
+    if (tid < np_) {
+      ((kKeys ? L.klabel : L.qlabel) + (size_t)bh * L.N)[p0 + tid] = lab[tid];
+      jsum += bval[tid];
+      atomicAdd(&hist[lab[tid]], 1);
+    }
     tc_fence_before();
     __syncthreads();
-    jsum += valid ? bestv : 0.0;
-    // stable order by label, fp64 sums per (run, dim), counts per run
-    if (valid) {
-      const int l = lab[tid];
-      int rk = 0;
-      for (int q = 0; q < np; ++q) {
-        const int lq = lab[q];
-        rk += (lq < l) || (lq == l && q < tid);
+    // counting sort of the tile's points by label (order inside a label is irrelevant: each
+    // run's fp64 partial sums are exact for keys and fp32-grade values for responses)
+    if (warp == 0) {
+      int run = 0;
+      for (int c0 = 0; c0 < C; c0 += 32) {
+        const int j = c0 + lane;
+        const int v = j < C ? hist[j] : 0;
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (j < C) cursor[j] = run + x - v;
+        run += __shfl_sync(0xffffffffu, x, 31);
       }
-      order[rk] = tid;
     }
     __syncthreads();
-    double* sums = (kKeys ? L.ksum : L.qsum) + (size_t)bh * C * Dreal;
     int* counts = (kKeys ? L.kcount : L.qcount) + (size_t)bh * C;
+    for (int j = tid; j < C; j += blockDim.x)
+      if (hist[j]) atomicAdd(counts + j, hist[j]);
+    if (tid < np_) order[atomicAdd(&cursor[lab[tid]], 1)] = tid;
+    __syncthreads();
+    double* sums = (kKeys ? L.ksum : L.qsum) + (size_t)bh * C * Dreal;
     // feature (p, a) from the swizzled tile(s) in shared memory: keys exactly, responses as
     // hi + mid + lo (fp32-grade)
     auto feat = [&](int p, int a) -> double {
@@ -289,29 +333,24 @@ __global__ void __launch_bounds__(128, 1)
       }
       return v;
     };
-    const int nparts = Dreal >= 128 ? 1 : 128 / Dreal;
-    if (tid < nparts * Dreal || Dreal > 128) {
-      for (int a = tid % Dreal; a < Dreal; a += (Dreal > 128 ? 128 : Dreal)) {
-        const int part = Dreal > 128 ? 0 : tid / Dreal;
-        const int q0 = part * np / nparts, q1 = (part + 1) * np / nparts;
+    const int nparts = Dreal >= 256 ? 1 : 256 / Dreal;
+    if (tid < nparts * Dreal || Dreal > 256) {
+      for (int a = tid % Dreal; a < Dreal; a += (Dreal > 256 ? 256 : Dreal)) {
+        const int part = Dreal > 256 ? 0 : tid / Dreal;
+        const int q0 = part * np_ / nparts, q1 = (part + 1) * np_ / nparts;
         double acc = 0.0;
-        for (int q = q0; q < q1; ++q) {
-          const int p = order[q];
+        for (int qq = q0; qq < q1; ++qq) {
+          const int p = order[qq];
           acc += feat(p, a);
-          if (q == q1 - 1 || lab[order[q + 1]] != lab[p]) {
+          if (qq == q1 - 1 || lab[order[qq + 1]] != lab[p]) {
             atomicAdd(sums + (size_t)lab[p] * Dreal + a, acc);
             acc = 0.0;
           }
         }
-        if (Dreal <= 128) break;
+        if (Dreal <= 256) break;
       }
     }
-    if (valid && (tid == 0 || lab[order[tid - 1]] != lab[order[tid]])) {
-      const int l = lab[order[tid]];
-      int q = tid + 1;
-      while (q < np && lab[order[q]] == l) ++q;
-      atomicAdd(counts + l, q - tid);
-    }
+    if (tid == 0) s_nlist = 0;
     tc_fence_before();
     __syncthreads();
   }
@@ -360,10 +399,10 @@ sparsepr_status launch_kmeans_assign_tc(const Layout& L, bool keys, const void* 
   const dim3 grid((ntiles + tpc - 1) / tpc, L.BH);
   if (keys) {
     cudaFuncSetAttribute(kmeans_assign_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    launch(kmeans_assign_tc_kernel<true>, grid, dim3(128), smem, st, mX, mW, L, (const __nv_bfloat16*)K, it, tpc);
+    launch(kmeans_assign_tc_kernel<true>, grid, dim3(256), smem, st, mX, mW, L, (const __nv_bfloat16*)K, it, tpc);
   } else {
     cudaFuncSetAttribute(kmeans_assign_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    launch(kmeans_assign_tc_kernel<false>, grid, dim3(128), smem, st, mX, mW, L, (const __nv_bfloat16*)K, it, tpc);
+    launch(kmeans_assign_tc_kernel<false>, grid, dim3(256), smem, st, mX, mW, L, (const __nv_bfloat16*)K, it, tpc);
   }
   SPR_LAUNCH_CHECK();
   return SPARSEPR_OK;
