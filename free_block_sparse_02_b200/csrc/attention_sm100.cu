@@ -6,19 +6,21 @@
 // groups its group keeps, softmax over the retained keys only), and "exact attention on a
 // small set of query rows" for the probes.
 //
-// Work item = one 128-row tile of one query group (block-sparse pass) or of one head's probe
-// rows (dense pass).  Its keys are the concatenation of the kept key groups' rows in the
-// group-permuted K/V; they are streamed in 128-key tiles assembled from 16-row TMA boxes, so a
-// kept key group costs at most 15 padded (masked) rows, wherever it starts.
+// Work item = 256 query rows of one query group (block-sparse pass) or of one head's probe rows
+// (dense pass), as two 128-row MMA tiles Q0, Q1 that share every KV tile.  The keys are the
+// concatenation of the kept key groups' rows in the group-permuted K/V, streamed in 128-key
+// tiles assembled from 16-row TMA boxes, so a kept key group costs at most 15 padded (masked)
+// rows wherever it starts.
 //
-// CTA of 256 threads:  warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner),
-// warps 4..7 = softmax (thread t owns query row t of the tile: TMEM lane t).
-// TMEM (512 columns): S/P buffers at columns [0,128) and [128,256), O at [256, 256 + d).
-//   S_i = Q K_i^T (fp32) -> softmax reads S_i, writes P_i (bf16, packed) over S_i's columns ->
-//   O += P_i V_i with P_i taken from TMEM.  The MMA warp issues S_{i+1} before O += P_i V_i so
-//   the next scores are computed while the softmax of the current tile runs.
-// Online softmax in base 2 with lazy rescaling: the running max only moves (and O is
-// rescaled in TMEM) when a tile's max exceeds it by more than 8 (a factor 256).
+// CTA of 384 threads: warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner), warps 4..7
+// = softmax of Q0, warps 8..11 = softmax of Q1 (thread t of a group owns query row t of its tile:
+// TMEM lane t).  TMEM (512 columns): S0 [0,128), S1 [128,256), O0 at 256, O1 at 256 + d.
+// P_t (bf16, packed) overwrites the first 64 columns of S_t and feeds O_t += P_t V from TMEM.
+// The MMA warp issues  PV0(j), S0(j+1), PV1(j), S1(j+1)  so each softmax warpgroup works while
+// the tensor core runs the other tile's two MMAs (ping-pong).  tcgen05.mma operations of one
+// thread execute in issue order, which orders S_t(j+1) after the PV_t(j) that reads P_t(j).
+// Online softmax in base 2 with lazy rescaling: the running max only moves (and O is rescaled
+// in TMEM) when a tile's max exceeds it by more than 8 (a factor 256).
 // Every mbarrier wait is bounded; a wait that gives up sets the device status to
 // SPARSEPR_ERR_TIMEOUT and the CTA drains its copies, frees TMEM and exits.
 #include <math.h>
@@ -31,18 +33,20 @@ namespace sparsepr {
 
 using namespace sm100;
 
-constexpr int kTcTileM = 128;   // query rows per work item (MMA M)
+constexpr int kTcTileM = 128;   // query rows per MMA tile
 constexpr int kTcTileN = 128;   // keys per KV tile (MMA N of S, K of PV)
 constexpr int kSubRows = 16;    // rows per TMA box of K/V
 constexpr int kSubPerTile = kTcTileN / kSubRows;
 constexpr int kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+static_assert(kAttnTileMTc == 2 * kTcTileM, "a work item is two MMA tiles");
 
 template <int D>
 struct TcCfg {
   static constexpr int kKB = D / 64;                    // 64-column (128-byte) blocks of a row
   static constexpr int kStages = D == 64 ? 4 : 2;
-  static constexpr int kQBytes = kTcTileM * D * 2;
+  static constexpr int kQTileBytes = kTcTileM * D * 2;
+  static constexpr int kQBytes = 2 * kQTileBytes;
   static constexpr int kKVTileBytes = kTcTileN * D * 2;  // one of K or V
   static constexpr int kStageBytes = 2 * kKVTileBytes;
   static constexpr int kSmemTiles = kQBytes + kStages * kStageBytes;
@@ -77,48 +81,46 @@ __device__ __forceinline__ void next_tile(SegState& s, const int2* segs, int nse
 }
 
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQprobe,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, Layout L,
-                   int probe_tiles_per_head, int sparse_tiles_per_head) {
+                   int probe_items_per_head, int sparse_items_per_head) {
   using C = TcCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sQ = smem;
+  uint8_t* sQ = smem;                // tile t at t * kQTileBytes
   uint8_t* sKV = smem + C::kQBytes;  // stage s: K at s*kStageBytes, V right after
   uint64_t* bars = (uint64_t*)(smem + C::kSmemTiles);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + C::kStages;
-  uint64_t* s_full = kv_empty + C::kStages;  // [2]
-  uint64_t* s_free = s_full + 2;             // [2]
-  uint64_t* p_full = s_free + 2;             // [2]
-  uint64_t* o_bar = p_full + 2;
-  uint64_t* mma_done = o_bar + 1;
+  uint64_t* s_full = kv_empty + C::kStages;  // [2] per query tile
+  uint64_t* p_full = s_full + 2;             // [2]
+  uint64_t* o_bar = p_full + 2;              // [2]
+  uint64_t* mma_done = o_bar + 2;
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
   __shared__ int2 segs[kMaxGroups];
-  __shared__ int s_nseg, s_ntiles, s_qrow0, s_nrows, s_mode, s_bh;
+  __shared__ int s_nseg, s_ntiles, s_qrow0, s_rows0, s_rows1, s_mode, s_bh;
   __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // ---- work item
   if (tid == 0) {
-    const int nprobe_items = L.BH * probe_tiles_per_head;
+    const int nprobe_items = L.BH * probe_items_per_head;
     int item = blockIdx.x;
-    int mode, bh, qrow0 = 0, nrows = 0;
+    int mode, bh, qrow0 = 0, end = 0;
     if (item < nprobe_items) {
       mode = 1;
-      bh = item / probe_tiles_per_head;
-      const int t = item % probe_tiles_per_head;
-      qrow0 = t * kTcTileM;
-      nrows = min(kTcTileM, L.P - qrow0);
+      bh = item / probe_items_per_head;
+      qrow0 = (item % probe_items_per_head) * kAttnTileMTc;
+      end = L.P;
     } else {
       item -= nprobe_items;
       mode = 0;
-      bh = item / sparse_tiles_per_head;
-      const int x = item % sparse_tiles_per_head;
+      bh = item / sparse_items_per_head;
+      const int x = item % sparse_items_per_head;
       const int* toff = L.tile_off + (size_t)bh * (L.Cq + 1);
       if (x < toff[L.Cq]) {
         int lo = 0, hi = L.Cq - 1;
@@ -128,20 +130,22 @@ __global__ void __launch_bounds__(256, 1)
           else hi = mid - 1;
         }
         const int* qoff = L.qoff + (size_t)bh * (L.Cq + 1);
-        qrow0 = qoff[lo] + (x - toff[lo]) * kTcTileM;
-        nrows = min(kTcTileM, qoff[lo + 1] - qrow0);
+        qrow0 = qoff[lo] + (x - toff[lo]) * kAttnTileMTc;
+        end = qoff[lo + 1];
         s_nseg = lo;  // group id, replaced by the segment count below
       }
     }
     s_mode = mode;
     s_bh = bh;
     s_qrow0 = qrow0;
-    s_nrows = nrows;
+    s_rows0 = min(kTcTileM, end - qrow0);
+    s_rows1 = min(kTcTileM, end - qrow0 - kTcTileM);
     s_abort = 0;
   }
   __syncthreads();
-  if (s_nrows <= 0) return;  // uniform: no barrier, TMEM or copy has been touched yet
+  if (s_rows0 <= 0) return;  // uniform: no barrier, TMEM or copy has been touched yet
   const int mode = s_mode, bh = s_bh;
+  const int ntq = s_rows1 > 0 ? 2 : 1;
   if (tid == 0) {
     int nsub = 0;
     if (mode == 1) {
@@ -167,12 +171,11 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(kv_full + s, 1);
       mbar_init(kv_empty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(s_full + b, 1);
-      mbar_init(s_free + b, 1);
-      mbar_init(p_full + b, 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(s_full + t, 1);
+      mbar_init(p_full + t, 128);
+      mbar_init(o_bar + t, 1);
     }
-    mbar_init(o_bar, 1);
     mbar_init(mma_done, 1);
     fence_mbar_init();
   }
@@ -184,22 +187,23 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int nseg = s_nseg, ntiles = s_ntiles, qrow0 = s_qrow0, nrows = s_nrows;
-  const int row_base = bh * L.N;                 // first row of this head in the 2D K/V view
-  const int oob_row = L.BH * L.N;                // a box starting here is entirely zero-filled
-  int* status = L.status;
+  const int nseg = s_nseg, ntiles = s_ntiles, qrow0 = s_qrow0;
+  const int row_base = bh * L.N;   // first row of this head in the 2D K/V view
+  const int oob_row = L.BH * L.N;  // a box starting here is entirely zero-filled
 
   if (warp == 0) {
     // ================================================================ TMA producer
     if (lane == 0 && ntiles > 0) {
-      prefetch_tmap(mode == 1 ? &tmQprobe : &tmQ);
+      const CUtensorMap* qm = mode == 1 ? &tmQprobe : &tmQ;
+      prefetch_tmap(qm);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      mbar_arrive_expect_tx(q_full, C::kQBytes);
-      const CUtensorMap* qm = mode == 1 ? &tmQprobe : &tmQ;
+      mbar_arrive_expect_tx(q_full, ntq * C::kQTileBytes);
       const int qy = (mode == 1 ? bh * L.P : bh * L.N) + qrow0;
+      for (int t = 0; t < ntq; ++t)
 #pragma unroll
-      for (int kb = 0; kb < C::kKB; ++kb) tma_load_2d(sQ + kb * kTcTileM * 128, qm, q_full, kb * 64, qy);
+        for (int kb = 0; kb < C::kKB; ++kb)
+          tma_load_2d(sQ + t * C::kQTileBytes + kb * kTcTileM * 128, qm, q_full, kb * 64, qy + t * kTcTileM);
       SegState st{0, 0};
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
@@ -232,81 +236,87 @@ __global__ void __launch_bounds__(256, 1)
       const uint32_t idesc_s = idesc_bf16_f32(kTcTileM, kTcTileN, 0, 0);
       const uint32_t idesc_o = idesc_bf16_f32(kTcTileM, D, 0, 1);
       const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t t_o = tmem + 256;
-      bool ok = mbar_wait(q_full, 0, &s_abort);
-      auto issue_pv = [&](int j) -> bool {
-        const int bj = j & 1, sj = j % C::kStages;
-        if (!mbar_wait(p_full + bj, (j >> 1) & 1, &s_abort)) return false;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(sKV + sj * C::kStageBytes + C::kKVTileBytes);
-#pragma unroll
-        for (int ks = 0; ks < kTcTileN / 16; ++ks) {
-          // B = V (keys x d, d contiguous): 16 keys per step = 2048 bytes; LBO = next 64 d-columns
-          const uint64_t bdesc = sdesc_sw128(v_addr + ks * 2048, kTcTileN * 128, 1024);
-          mma_ts(t_o, tmem + bj * 128 + ks * 8, bdesc, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
-        }
-        mma_commit(kv_empty + sj);
-        mma_commit(s_free + bj);
-        mma_commit(o_bar);
-        return true;
-      };
-      for (int i = 0; ok && i < ntiles; ++i) {
-        const int s = i % C::kStages, b = i & 1;
-        if (!mbar_wait(kv_full + s, (i / C::kStages) & 1, &s_abort)) break;
-        if (i >= 2 && !mbar_wait(s_free + b, ((i >> 1) - 1) & 1, &s_abort)) break;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sKV + s * C::kStageBytes);
+      auto issue_s = [&](int t, int j) {  // S_t(j) = Q_t K_j^T
+        const uint32_t k_addr = smem_u32(sKV + (j % C::kStages) * C::kStageBytes);
+        const uint32_t qa = q_addr + t * C::kQTileBytes;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t koff = (ks >> 2) * (kTcTileN * 128) + (ks & 3) * 32;
           const uint32_t qoff = (ks >> 2) * (kTcTileM * 128) + (ks & 3) * 32;
-          mma_ss(tmem + b * 128, sdesc_sw128(q_addr + qoff, 16, 1024), sdesc_sw128(k_addr + koff, 16, 1024),
-                 idesc_s, ks > 0 ? 1u : 0u);
+          mma_ss(tmem + t * 128, sdesc_sw128(qa + qoff, 16, 1024), sdesc_sw128(k_addr + koff, 16, 1024), idesc_s,
+                 ks > 0 ? 1u : 0u);
         }
-        mma_commit(s_full + b);
-        if (i >= 1 && !issue_pv(i - 1)) {
-          ok = false;
-          break;
+        mma_commit(s_full + t);
+      };
+      auto issue_pv = [&](int t, int j) -> bool {  // O_t += P_t(j) V_j
+        if (!mbar_wait(p_full + t, j & 1, &s_abort)) return false;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(sKV + (j % C::kStages) * C::kStageBytes + C::kKVTileBytes);
+#pragma unroll
+        for (int ks = 0; ks < kTcTileN / 16; ++ks) {
+          // B = V (keys x d, d contiguous): 16 keys per step = 2048 bytes; LBO = next 64 d-columns
+          const uint64_t bdesc = sdesc_sw128(v_addr + ks * 2048, kTcTileN * 128, 1024);
+          mma_ts(tmem + 256 + t * D, tmem + t * 128 + ks * 8, bdesc, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
         }
+        mma_commit(o_bar + t);
+        return true;
+      };
+      bool ok = mbar_wait(q_full, 0, &s_abort) && mbar_wait(kv_full, 0, &s_abort);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (ntq == 2) issue_s(1, 0);
       }
-      if (ok && !s_abort) issue_pv(ntiles - 1);
+      for (int j = 0; ok && j < ntiles; ++j) {
+        const bool more = j + 1 < ntiles;
+        if (!issue_pv(0, j)) break;
+        if (more) {
+          if (!mbar_wait(kv_full + (j + 1) % C::kStages, ((j + 1) / C::kStages) & 1, &s_abort)) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (ntq == 2 && !issue_pv(1, j)) break;
+        mma_commit(kv_empty + j % C::kStages);  // K_j, V_j no longer read once these complete
+        if (more && ntq == 2) issue_s(1, j + 1);
+      }
       // every MMA issued by this thread has completed before TMEM is released
       mma_commit(mma_done);
       mbar_wait_drain(mma_done, 0);
     }
   } else if (warp >= 4) {
     // ================================================================ softmax + epilogue
-    const int row = tid - 128;  // TMEM lane and query row of the tile
+    const int t = (warp - 4) >> 2;  // query tile of this warpgroup
+    const int row = tid - 128 - t * 128;
+    const int rows_t = t == 0 ? s_rows0 : s_rows1;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + t * 128;
+    const uint32_t tO = tmem + lane_base + 256 + t * D;
     const float scale2 = 1.4426950408889634f / sqrtf((float)D);
     float m_used = -INFINITY, l = 0.f;
     SegState st{0, 0};
-    bool ok = ntiles > 0;
-    for (int i = 0; ok && i < ntiles; ++i) {
-      const int b = i & 1;
+    bool ok = ntiles > 0 && t < ntq;
+    for (int j = 0; ok && j < ntiles; ++j) {
       int rows[kSubPerTile], valid[kSubPerTile];
       next_tile(st, segs, nseg, row_base, oob_row, rows, valid);
-      if (!mbar_wait(s_full + b, (i >> 1) & 1, &s_abort)) {
+      if (!mbar_wait(s_full + t, j & 1, &s_abort)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float sc[kTcTileN];
+      // pass 1: row max over the valid keys
+      float tmax = -INFINITY;
 #pragma unroll
       for (int c = 0; c < kTcTileN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_base + b * 128 + c * 32, r);
+        tmem_ld32(tS + c * 32, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 32; ++k) sc[c * 32 + k] = __uint_as_float(r[k]);
+        for (int k = 0; k < 32; ++k) {
+          const int col = c * 32 + k;
+          if ((col & (kSubRows - 1)) < valid[col / kSubRows]) tmax = fmaxf(tmax, __uint_as_float(r[k]));
+        }
       }
-      float tmax = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kTcTileN; ++c) {
-        const bool v = (c & (kSubRows - 1)) < valid[c / kSubRows];
-        sc[c] = v ? sc[c] * scale2 : -INFINITY;
-        tmax = fmaxf(tmax, sc[c]);
-      }
+      tmax *= scale2;
       // lazy rescale: move the running max only when this tile exceeds it by > 2^8
       const bool need = (m_used == -INFINITY) ? (tmax > -INFINITY) : (tmax > m_used + kRescaleThreshold);
       float factor = 1.f;
@@ -315,9 +325,9 @@ __global__ void __launch_bounds__(256, 1)
         m_new = tmax;
         factor = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_new);
       }
-      if (__any_sync(0xffffffffu, need && i > 0)) {
-        // O holds P_0..P_{i-1} V: wait for the last of them, then scale this warp's rows
-        if (!mbar_wait(o_bar, (i - 1) & 1, &s_abort)) {
+      if (__any_sync(0xffffffffu, need && j > 0)) {
+        // O_t holds P_t(0..j-1) V (complete: S_t(j) was issued after the last of them)
+        if (!mbar_wait(o_bar + t, (j - 1) & 1, &s_abort)) {
           ok = false;
           break;
         }
@@ -325,58 +335,78 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
-          tmem_ld32(tmem + lane_base + 256 + c * 32, r);
+          tmem_ld32(tO + c * 32, r);
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * factor);
-          tmem_st32(tmem + lane_base + 256 + c * 32, r);
+          tmem_st32(tO + c * 32, r);
         }
         tmem_wait_st();
       }
       l *= factor;
       m_used = m_new;
-      // P = 2^(s - m) as packed bf16 over the first 64 columns of this S buffer
+      // pass 2: P = 2^(s*scale - m) as packed bf16 over the first 64 columns of S_t (each
+      // 64-key half is read before its 32 packed columns are written over already-read ones)
+      const float neg_m = -m_used;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
+        uint32_t ra[32], rb[32];
+        tmem_ld32(tS + c * 64, ra);
+        tmem_ld32(tS + c * 64 + 32, rb);
+        tmem_wait_ld();
+        uint32_t pk[32];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float p0 = ex2(sc[c * 64 + 2 * k] - m_used);
-          const float p1 = ex2(sc[c * 64 + 2 * k + 1] - m_used);
+        for (int k = 0; k < 16; ++k) {
+          const int c0 = c * 64 + 2 * k, c1 = c0 + 1;
+          const bool v0 = (c0 & (kSubRows - 1)) < valid[c0 / kSubRows];
+          const bool v1 = (c1 & (kSubRows - 1)) < valid[c1 / kSubRows];
+          const float p0 = v0 ? ex2(fmaf(__uint_as_float(ra[2 * k]), scale2, neg_m)) : 0.f;
+          const float p1 = v1 ? ex2(fmaf(__uint_as_float(ra[2 * k + 1]), scale2, neg_m)) : 0.f;
           l += p0 + p1;
-          r[k] = pack_bf16x2(p0, p1);
+          pk[k] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(tmem + lane_base + b * 128 + c * 32, r);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int c0 = c * 64 + 32 + 2 * k, c1 = c0 + 1;
+          const bool v0 = (c0 & (kSubRows - 1)) < valid[c0 / kSubRows];
+          const bool v1 = (c1 & (kSubRows - 1)) < valid[c1 / kSubRows];
+          const float p0 = v0 ? ex2(fmaf(__uint_as_float(rb[2 * k]), scale2, neg_m)) : 0.f;
+          const float p1 = v1 ? ex2(fmaf(__uint_as_float(rb[2 * k + 1]), scale2, neg_m)) : 0.f;
+          l += p0 + p1;
+          pk[16 + k] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + c * 32, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full + b);
+      mbar_arrive(p_full + t);
     }
-    // epilogue: O / l for the rows of this tile (a tile without keys outputs zeros)
-    if (ntiles == 0 && row < nrows) {
-      float* out = (mode == 1 ? L.Odense + ((size_t)bh * L.P + qrow0) * D : L.Osp + ((size_t)bh * L.N + qrow0) * D);
-      for (int c = 0; c < D; c += 4) *(float4*)(out + (size_t)row * D + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    if (ok && mbar_wait(o_bar, (ntiles - 1) & 1, &s_abort)) {
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      float* out = (mode == 1 ? L.Odense + ((size_t)bh * L.P + qrow0) * D : L.Osp + ((size_t)bh * L.N + qrow0) * D);
+    // epilogue: O_t / l for the rows of this tile (a tile without keys outputs zeros)
+    if (t < ntq) {
+      float* out = (mode == 1 ? L.Odense + ((size_t)bh * L.P + qrow0 + t * kTcTileM) * D
+                              : L.Osp + ((size_t)bh * L.N + qrow0 + t * kTcTileM) * D);
+      if (ntiles == 0 && row < rows_t)
+        for (int c = 0; c < D; c += 4) *(float4*)(out + (size_t)row * D + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (ok && mbar_wait(o_bar + t, (ntiles - 1) & 1, &s_abort)) {
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + 256 + c * 32, r);
-        tmem_wait_ld();
-        if (row < nrows) {
-          float4* o4 = (float4*)(out + (size_t)row * D + c * 32);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + c * 32, r);
+          tmem_wait_ld();
+          if (row < rows_t) {
+            float4* o4 = (float4*)(out + (size_t)row * D + c * 32);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            o4[k] = make_float4(__uint_as_float(r[4 * k]) * inv, __uint_as_float(r[4 * k + 1]) * inv,
-                                __uint_as_float(r[4 * k + 2]) * inv, __uint_as_float(r[4 * k + 3]) * inv);
+            for (int k = 0; k < 8; ++k)
+              o4[k] = make_float4(__uint_as_float(r[4 * k]) * inv, __uint_as_float(r[4 * k + 1]) * inv,
+                                  __uint_as_float(r[4 * k + 2]) * inv, __uint_as_float(r[4 * k + 3]) * inv);
+          }
         }
       }
     }
   }
-  if (s_abort && tid == 0) atomicCAS(status, kDevOk, kDevTimeout);
+  if (s_abort && tid == 0) atomicCAS(L.status, kDevOk, kDevTimeout);
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -394,18 +424,18 @@ static sparsepr_status launch_tc(const Layout& L, cudaStream_t st, cudaEvent_t e
   if (!make_tmap_bf16(&mQ, L.Qp, rows, D, kTcTileM) || !make_tmap_bf16(&mK, L.Kp, rows, D, kSubRows) ||
       !make_tmap_bf16(&mV, L.Vp, rows, D, kSubRows))
     return SPARSEPR_ERR_CUDA;
-  const int probe_tiles = (L.P + kTcTileM - 1) / kTcTileM;
-  if (probe_tiles > 0) {
+  const int probe_items = (L.P + kAttnTileMTc - 1) / kAttnTileMTc;
+  if (probe_items > 0) {
     if (!make_tmap_bf16(&mQp, L.Qprobe, (long long)L.BH * L.P, D, kTcTileM)) return SPARSEPR_ERR_CUDA;
   } else {
     mQp = mQ;
   }
-  const int sparse_tiles = max_query_tiles(L, kTcTileM);
-  const int items = L.BH * (probe_tiles + sparse_tiles);
+  const int sparse_items = max_query_tiles(L, kAttnTileMTc);
+  const int items = L.BH * (probe_items + sparse_items);
   cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (ev0) cudaEventRecord(ev0, st);
-  launch(attn_tc_kernel<D>, dim3(items), dim3(256), (size_t)C::kSmemBytes, st, mQ, mQp, mK, mV, L, probe_tiles,
-         sparse_tiles);
+  launch(attn_tc_kernel<D>, dim3(items), dim3(384), (size_t)C::kSmemBytes, st, mQ, mQp, mK, mV, L, probe_items,
+         sparse_items);
   if (ev1) cudaEventRecord(ev1, st);
   SPR_LAUNCH_CHECK();
   return SPARSEPR_OK;

@@ -6,9 +6,9 @@
 namespace sparsepr {
 
 // Query rows per attention work item (the block-sparse pass tiles each query group by this):
-// 64 for the fp32 CUDA-core kernel, 128 (one MMA M) for the bf16 tensor-core kernel.
+// 64 for the fp32 CUDA-core kernel, 256 (two 128-row MMA tiles) for the bf16 tensor-core kernel.
 constexpr int kAttnTileM = 64;
-constexpr int kAttnTileMTc = 128;
+constexpr int kAttnTileMTc = 256;
 inline int attn_tile_m(const Layout& L) { return L.dtype == SPARSEPR_BF16 ? kAttnTileMTc : kAttnTileM; }
 
 sparsepr_status launch_plan(const Layout& L, const void* Q, const void* K, bool warm, int iters,
