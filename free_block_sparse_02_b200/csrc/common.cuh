@@ -64,29 +64,34 @@ struct Layout {
   double* kJ;                     // [BH, iters_cap]
   int* krefined;                  // [BH]
 
-  // query responses and query k-means (features: RMS-normalised responses)
-  double* r64;                    // [BH, N, Ck]
-  float* r32;                     // [BH, N, Ck]
-  double* qcent;                  // [BH, Cq, Ck]
-  float* qW32;                    // [BH, Cq, Ck]
-  double* qbias64;                // [BH, Cq]
+  // query k-means.  The normalised responses are linear in the query,
+  //   r~_q = C q / (sqrt(d) rms_q),   rms_q^2 = q^T Gc q + 1e-12,   Gc = C^T C / (d C_k),
+  // (C = key-group centroids, rows c_j), so the iteration runs on the d-dim queries: the score
+  // of group g is ||nu_g||^2 - 2 (q . u_g) / rms_q with u_g = C^T nu_g / sqrt(d), and the group
+  // sums are sums of q / rms_q, projected back as nu_g = C S_g / (sqrt(d) n_g).
+  double* Gc;                     // [BH, d, d]
+  float* inv_rms;                 // [BH, N]   1 / rms_q
+  float* qxnorm;                  // [BH, N]   ||q|| / rms_q  (= ||r~_q|| bound for the score error)
+  double* qcent;                  // [BH, Cq, Ck] nu_g (response space)
+  double* qU64;                   // [BH, Cq, d]  u_g
+  float* qU32;                    // [BH, Cq, d]
+  double* qbias64;                // [BH, Cq]     ||nu_g||^2
   float* qbias32;                 // [BH, Cq]
-  float* qwnorm;                  // [BH, Cq]
-  double* qsum;                   // [BH, Cq, Ck]
+  float* qwnorm;                  // [BH, Cq]     ||u_g||_2
+  double* qsum;                   // [BH, Cq, d]  sums of q / rms_q
   int* qcount;                    // [BH, Cq]
   int* qlabel;                    // [BH, N]
   double* qJ;                     // [BH, iters_cap]
   int* qrefined;                  // [BH]
 
-  // bf16 operands of the tensor-core assignment: weights split into three bf16 terms
-  // (hi + mid + lo reproduces the fp64 value to ~2^-24 relative), features likewise for the
-  // normalised responses; group rows padded to a multiple of 16, response dims to 64
-  int Ckp, Cqp, Dq;
-  __nv_bfloat16* kWb;             // [3][BH, Ckp, d]
-  __nv_bfloat16* qWb;             // [3][BH, Cqp, Dq]
-  __nv_bfloat16* rb;              // [3][BH, N, Dq]
+  // bf16 operands of the tensor-core kernels: fp64 matrices split into three bf16 terms
+  // (hi + mid + lo reproduces the value to ~2^-24 relative); group rows padded to 16
+  int Ckp, Cqp;
+  __nv_bfloat16* kWb;             // [3][BH, Ckp, d]   W_j = M c_j
+  __nv_bfloat16* qWb;             // [3][BH, Cqp, d]   u_g
+  __nv_bfloat16* Mb;              // [3][BH, d, d]     M
+  __nv_bfloat16* Gcb;             // [3][BH, d, d]     Gc
   float* knorm;                   // [BH, N] ||k_t||_2 (rounding bound of the key scores)
-  float* rnorm;                   // [BH, N] ||r~_q||_2
 
   // group-contiguous order (stable counting sort)
   int* kperm;                     // [BH, N]   position -> token

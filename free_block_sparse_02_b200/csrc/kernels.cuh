@@ -21,7 +21,8 @@ sparsepr_status launch_attention_tc(const Layout& L, cudaStream_t st, cudaEvent_
 sparsepr_status launch_fit_apply(const Layout& L, void* O, int out_dtype, cudaStream_t st);
 sparsepr_status launch_ridge_solve(const Layout& L, cudaStream_t st);
 bool km_tc_supported(const Layout& L, bool keys);
-sparsepr_status launch_kmeans_assign_tc(const Layout& L, bool keys, const void* K, int it, cudaStream_t st);
+sparsepr_status launch_kmeans_assign_tc(const Layout& L, bool keys, const void* X, int it, cudaStream_t st);
+sparsepr_status launch_rowqf_tc(const Layout& L, int which, const void* X, cudaStream_t st);
 
 // Upper bound of the number of query tiles of one head: sum_g ceil(n_g / tile) <= N/tile + C_q.
 inline int max_query_tiles(const Layout& L, int tile) { return (L.N + tile - 1) / tile + L.Cq; }

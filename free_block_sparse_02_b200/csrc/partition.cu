@@ -5,18 +5,23 @@
 // responses to the key-group centroids (shared sparse routing); project page "SparsePR:
 // Training-Free Sparse Attention for Video Generation", method pipeline steps 01-03.
 //
-// Key responses f_t = Q_s k_t / sqrt(d) (s-dimensional) are never materialised: for a group
-// mean mu_j = Q_s c_j / sqrt(d) (c_j = mean of the member keys), linearity gives
-//   ||f_t - mu_j||^2 = (k_t - c_j)^T M (k_t - c_j),   M = Q_s^T Q_s / d,
-// so the assignment is argmin_j ( c_j^T M c_j - 2 k_t . (M c_j) ) over d-dimensional keys.
+// Neither response matrix is materialised; both k-means run on the d-dimensional inputs.
+// Keys: f_t = Q_s k_t / sqrt(d) (s dims).  For a group mean mu_j = Q_s c_j / sqrt(d) (c_j the
+// mean of the member keys), ||f_t - mu_j||^2 = (k_t - c_j)^T M (k_t - c_j) with
+// M = Q_s^T Q_s / d, so the label is argmin_j (c_j^T M c_j - 2 k_t . (M c_j)).
+// Queries: the per-query RMS-normalised responses (Table D.1, "Per query RMS") are
+// r~_q = C q / (sqrt(d) rms_q) with rms_q^2 = q^T Gc q + 1e-12, Gc = C^T C / (d C_k); for a group
+// mean nu_g of r~, ||r~_q - nu_g||^2 = ||r~_q||^2 + ||nu_g||^2 - 2 (q . u_g) / rms_q with
+// u_g = C^T nu_g / sqrt(d), and nu_g = C S_g / (sqrt(d) n_g) with S_g the sum of q / rms_q.
 //
-// Exactness: scores are computed in fp32 with a rigorous rounding bound; a point whose best
-// two scores are within that bound is re-decided over all groups in fp64, so labels agree
-// with an fp64 evaluation except at ties far below the fp32 resolution.  Group sums are fp64.
+// Exactness: scores carry a rigorous rounding bound; a point whose best two scores are within
+// it is re-decided over all groups in fp64, so labels agree with an fp64 evaluation except at
+// ties far below the fp32 resolution.  Group sums are fp64.
 #include <math.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "kmeans.cuh"
 
 namespace sparsepr {
 
@@ -36,44 +41,81 @@ __global__ void metric_kernel(Layout L, const T* __restrict__ Q) {
   L.M[((size_t)bh * L.d + a) * L.d + b] = acc / L.d;
 }
 
-// Objective constant sum_t ||f_t||^2 = sum_t k_t^T M k_t of the key k-means (it only scales the
-// relative stop test, so fp32 products with an fp64 block sum are ample).  64 keys per block;
-// M is staged in shared memory as fp32, thread (key p = tid/4, quarter q) forms d/4 entries of
-// M k_p and their dot with k_p.
+// fp64 [BH, d, d] matrices split into three bf16 planes (tensor-core operands).
+__global__ void split_mat_kernel(const double* __restrict__ src, __nv_bfloat16* __restrict__ dst, size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const double x = src[i];
+    const __nv_bfloat16 h = __double2bfloat16(x);
+    const double r1 = x - (double)__bfloat162float(h);
+    const __nv_bfloat16 m = __double2bfloat16(r1);
+    dst[i] = h;
+    dst[n + i] = m;
+    dst[2 * n + i] = __double2bfloat16(r1 - (double)__bfloat162float(m));
+  }
+}
+
+// Gc = C^T C / (d C_k) from the key-group centroids (fp64): rms_q^2 = q^T Gc q + 1e-12 is the
+// mean square of the query's responses to every key group.
+__global__ void gc_kernel(Layout L) {
+  const int bh = blockIdx.x, a = blockIdx.y, b = threadIdx.x, d = L.d;
+  if (b >= d) return;
+  const double* C = L.kcent + (size_t)bh * L.Ck * d;
+  double acc = 0.0;
+  for (int j = 0; j < L.Ck; ++j) acc += C[(size_t)j * d + a] * C[(size_t)j * d + b];
+  L.Gc[((size_t)bh * d + a) * d + b] = acc / ((double)d * L.Ck);
+}
+
+// Per-row quadratic forms on CUDA cores (the tensor-core version serves bf16 inputs).
+//   keys    (which 0): x^T M x summed into T0k (the constant of the key objective); ||x||.
+//   queries (which 1): ms = x^T Gc x; 1/rms, ||x||/rms, and C_k ms/(ms + 1e-12) = ||r~||^2
+//                      summed into T0q.
+// 64 rows per block; G staged in shared memory as fp32; thread (row p = tid/4, quarter q).
 template <typename T>
-__global__ void __launch_bounds__(256) key_norms_kernel(Layout L, const T* __restrict__ K) {
+__global__ void __launch_bounds__(256) rowqf_simt_kernel(Layout L, const T* __restrict__ X, int which) {
   extern __shared__ float shm[];
   const int d = L.d, bh = blockIdx.y, tid = threadIdx.x;
   const int DP = d + 1;
-  float* Ms = shm;              // [d][DP]
-  float* Ks = Ms + d * DP;      // [64][DP]
+  float* Gs = shm;              // [d][DP]
+  float* Xs = Gs + d * DP;      // [64][DP]
   __shared__ double red[8];
   const int p0 = blockIdx.x * 64, np = min(64, L.N - p0);
-  const double* M = L.M + (size_t)bh * d * d;
-  for (int e = tid; e < d * d; e += 256) Ms[(e / d) * DP + (e % d)] = (float)M[e];
+  const double* G = (which == 0 ? L.M : L.Gc) + (size_t)bh * d * d;
+  for (int e = tid; e < d * d; e += 256) Gs[(e / d) * DP + (e % d)] = (float)G[e];
   for (int e = tid; e < 64 * d; e += 256) {
     const int p = e / d, a = e % d;
-    Ks[p * DP + a] = p < np ? to_f32(K[((size_t)bh * L.N + p0 + p) * d + a]) : 0.f;
+    Xs[p * DP + a] = p < np ? to_f32(X[((size_t)bh * L.N + p0 + p) * d + a]) : 0.f;
   }
   __syncthreads();
   const int p = tid >> 2, q = tid & 3, dq = d >> 2;
-  const float* kp = Ks + p * DP;
-  float part = 0.f;
+  const float* xp = Xs + p * DP;
+  float part = 0.f, nn = 0.f;
   for (int a = q * dq; a < (q + 1) * dq; ++a) {
-    const float* Mr = Ms + a * DP;
+    const float* Gr = Gs + a * DP;
     float u = 0.f;
-    for (int b = 0; b < d; ++b) u = fmaf(Mr[b], kp[b], u);
-    part = fmaf(u, kp[a], part);
+    for (int b = 0; b < d; ++b) u = fmaf(Gr[b], xp[b], u);
+    part = fmaf(u, xp[a], part);
+    nn = fmaf(xp[a], xp[a], nn);
   }
   part += __shfl_xor_sync(0xffffffffu, part, 1);
   part += __shfl_xor_sync(0xffffffffu, part, 2);
-  if (tid < 64 && tid < np) {
-    float kk = 0.f;
-    for (int a = 0; a < d; ++a) kk = fmaf(Ks[tid * DP + a], Ks[tid * DP + a], kk);
-    L.knorm[(size_t)bh * L.N + p0 + tid] = sqrtf(kk);
+  nn += __shfl_xor_sync(0xffffffffu, nn, 1);
+  nn += __shfl_xor_sync(0xffffffffu, nn, 2);
+  double contrib = 0.0;
+  if (q == 0 && p < np) {
+    const size_t row = (size_t)bh * L.N + p0 + p;
+    if (which == 0) {
+      L.knorm[row] = sqrtf(nn);
+      contrib = part;
+    } else {
+      const double ms = (double)part;
+      const float inv = (float)(1.0 / sqrt(ms + 1e-12));
+      L.inv_rms[row] = inv;
+      L.qxnorm[row] = sqrtf(nn) * inv;
+      contrib = (double)L.Ck * ms / (ms + 1e-12);
+    }
   }
-  const double tot = block_sum((q == 0 && p < np) ? (double)part : 0.0, red);
-  if (tid == 0) atomicAdd(L.T0k + bh, tot);
+  const double tot = block_sum(contrib, red);
+  if (tid == 0) atomicAdd((which == 0 ? L.T0k : L.T0q) + bh, tot);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -132,11 +174,30 @@ __global__ void kcent_init_kernel(Layout L, const T* __restrict__ K) {
   L.kcent[((size_t)bh * L.Ck + j) * L.d + a] = (double)to_f32(K[((size_t)bh * L.N + t) * L.d + a]);
 }
 
-__global__ void qcent_init_kernel(Layout L) {
-  const int bh = blockIdx.x, g = blockIdx.y;
+// Cold start of the query groups: nu_g = r~ of the drawn query, in fp64.
+template <typename T>
+__global__ void __launch_bounds__(128) qcent_init_kernel(Layout L, const T* __restrict__ Q) {
+  __shared__ double qv[128];
+  __shared__ double red[4];
+  const int bh = blockIdx.x, g = blockIdx.y, d = L.d, Ck = L.Ck, tid = threadIdx.x;
   const int t = L.init_ids[(size_t)bh * max(L.Ck, L.Cq) + g];
-  for (int a = threadIdx.x; a < L.Ck; a += blockDim.x)
-    L.qcent[((size_t)bh * L.Cq + g) * L.Ck + a] = L.r64[((size_t)bh * L.N + t) * L.Ck + a];
+  if (tid < d) qv[tid] = (double)to_f32(Q[((size_t)bh * L.N + t) * d + tid]);
+  __syncthreads();
+  const double rsd = 1.0 / sqrt((double)d);
+  double* nu = L.qcent + ((size_t)bh * L.Cq + g) * Ck;
+  double ms = 0.0;
+  for (int j = tid; j < Ck; j += blockDim.x) {
+    const double* c = L.kcent + ((size_t)bh * Ck + j) * d;
+    double r = 0.0;
+    for (int a = 0; a < d; ++a) r += qv[a] * c[a];
+    r *= rsd;
+    nu[j] = r;
+    ms += r * r;
+  }
+  ms = block_sum(ms, red) / Ck;
+  const double inv = 1.0 / sqrt(ms + 1e-12);
+  __syncthreads();
+  for (int j = tid; j < Ck; j += blockDim.x) nu[j] *= inv;
 }
 
 // J arrays start at the objective constant; the stop marker starts at the iteration limit.
@@ -215,45 +276,67 @@ __global__ void __launch_bounds__(128) kprep_kernel(Layout L, int it, int iters)
 }
 
 __global__ void __launch_bounds__(128) qprep_kernel(Layout L, int it, int iters) {
+  __shared__ double Sv[128];
+  __shared__ double nuv[kMaxGroups];
   __shared__ double red[4];
-  const int bh = blockIdx.x, g = blockIdx.y, D = L.Ck;
+  const int bh = blockIdx.x, g = blockIdx.y, d = L.d, Ck = L.Ck, tid = threadIdx.x;
   if (it > L.stop_at[bh * 2 + 1]) return;
   const size_t gg = (size_t)bh * L.Cq + g;
-  double* nu = L.qcent + gg * D;
-  if (it > 0) {
+  double* nu = L.qcent + gg * Ck;
+  const double* C = L.kcent + (size_t)bh * Ck * d;
+  const double rsd = 1.0 / sqrt((double)d);
+  if (it > 0) {  // nu_g = C S_g / (sqrt(d) n_g): the mean normalised response of the members
     const int cnt = L.qcount[gg];
-    if (cnt > 0)
-      for (int a = threadIdx.x; a < D; a += blockDim.x) nu[a] = L.qsum[gg * D + a] / (double)cnt;
+    if (cnt > 0) {
+      if (tid < d) Sv[tid] = L.qsum[gg * d + tid] / (double)cnt;
+      __syncthreads();
+      for (int j = tid; j < Ck; j += blockDim.x) {
+        double acc = 0.0;
+        for (int a = 0; a < d; ++a) acc += C[(size_t)j * d + a] * Sv[a];
+        nu[j] = acc * rsd;
+      }
+    }
   }
   if (km_should_stop(L.qJ + (size_t)bh * L.iters_cap, it, iters, L.km_tol)) {
-    if (threadIdx.x == 0 && g == 0) L.stop_at[bh * 2 + 1] = it;
+    if (tid == 0 && g == 0) L.stop_at[bh * 2 + 1] = it;
     return;
   }
+  __syncthreads();
   double nn = 0.0;
-  for (int a = threadIdx.x; a < D; a += blockDim.x) {
-    const double v = nu[a];
+  for (int j = tid; j < Ck; j += blockDim.x) {
+    const double v = nu[j];
+    nuv[j] = v;
     nn += v * v;
-    L.qW32[gg * D + a] = (float)v;
-    L.qsum[gg * D + a] = 0.0;
-    split3(v, L.qWb, (size_t)L.BH * L.Cqp * L.Dq, ((size_t)bh * L.Cqp + g) * L.Dq + a);
   }
   nn = block_sum(nn, red);
-  if (threadIdx.x == 0) {
+  // u_g = C^T nu_g / sqrt(d)
+  double un = 0.0;
+  if (tid < d) {
+    double acc = 0.0;
+    for (int j = 0; j < Ck; ++j) acc += C[(size_t)j * d + tid] * nuv[j];
+    acc *= rsd;
+    L.qU64[gg * d + tid] = acc;
+    L.qU32[gg * d + tid] = (float)acc;
+    split3(acc, L.qWb, (size_t)L.BH * L.Cqp * d, ((size_t)bh * L.Cqp + g) * d + tid);
+    L.qsum[gg * d + tid] = 0.0;
+    un = acc * acc;
+  }
+  un = block_sum(un, red);
+  if (tid == 0) {
     L.qbias64[gg] = nn;
     L.qbias32[gg] = (float)nn;
     L.qcount[gg] = 0;
-    L.qwnorm[gg] = (float)sqrt(nn);
+    L.qwnorm[gg] = (float)sqrt(un);
   }
 }
 
 // ------------------------------------------------------------------------------------------
-// Lloyd step 2: assignment of 128 points per block against all groups, with fp64 sums.
-// Thread (pg, cg) = (tid / 16, tid % 16) scores points pg + 16 r (r < 8) against groups
-// cg + 16 i (i < 4) of the current 64-group chunk (register tile 8 x 4).  Feature rows: keys
-// (d dims; bf16/fp32 values are exact in fp32 and fp64) or the normalised responses (C_k dims;
-// an fp32 copy for scoring and sums, fp64 for the tie-break).  Each fp32 score carries a
-// rounding bound; a point whose two best scores are within it is re-decided over all groups in
-// fp64.  The chosen group's exact fp64 score feeds the objective.
+// Lloyd step 2 on CUDA cores (fp32 inputs, or more groups than the tensor-core kernel holds):
+// 128 points per block against all groups, register tile 8 points x 4 groups per thread
+// (pg = tid / 16, cg = tid % 16), groups in chunks of 64.  Feature rows are the inputs
+// themselves (keys, or queries scaled by 1/rms_q in the score); every bf16/fp32 input is exact
+// in fp32 and fp64.  A point whose two best fp32 scores are within the rounding bound is
+// re-decided over all groups in fp64.
 // ------------------------------------------------------------------------------------------
 struct KeyFeat {};
 struct QueryFeat {};
@@ -262,56 +345,49 @@ constexpr int kAsgPts = 128;
 constexpr int kAsgChunk = 64;
 
 inline size_t assign_smem_bytes(int D) {
-  return (size_t)(kAsgPts + kAsgChunk) * (D + 1) * 4 + kAsgChunk * 4 + kAsgPts * 4 /*xnorm*/ +
-         2 * kAsgPts * 4 /*lab, order*/ + kAsgPts * 4 /*refine*/ + kAsgPts * 8 /*a64*/;
+  return (size_t)(kAsgPts + kAsgChunk) * (D + 1) * 4 + kAsgChunk * 4 + kAsgPts * 4 /*scale*/ +
+         3 * kAsgPts * 4 /*lab, order, refine*/ + kAsgPts * 8 /*score*/ + 8 * 128 * 8 /*fp64 rows*/;
 }
 
 template <typename T, typename Feat>
-__global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* __restrict__ K, int it) {
+__global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* __restrict__ X, int it) {
   constexpr bool kKeys = std::is_same<Feat, KeyFeat>::value;
   const int bh = blockIdx.y;
   const int which = kKeys ? 0 : 1;
   if (it >= L.stop_at[bh * 2 + which]) return;
-  const int D = kKeys ? L.d : L.Ck;
+  const int D = L.d;
   const int C = kKeys ? L.Ck : L.Cq;
   const int DP = D + 1;
   const int p0 = blockIdx.x * kAsgPts;
   const int np = min(kAsgPts, L.N - p0);
   if (np <= 0) return;
 
-  const float* W32 = kKeys ? L.kW32 + (size_t)bh * C * D : L.qW32 + (size_t)bh * C * D;
-  const float* B32 = kKeys ? L.kbias32 + (size_t)bh * C : L.qbias32 + (size_t)bh * C;
-  const double* W64 = kKeys ? L.kW64 + (size_t)bh * C * D : L.qcent + (size_t)bh * C * D;
-  const double* B64 = kKeys ? L.kbias64 + (size_t)bh * C : L.qbias64 + (size_t)bh * C;
-  const float* WN = kKeys ? L.kwnorm + (size_t)bh * C : L.qwnorm + (size_t)bh * C;
+  const float* W32 = (kKeys ? L.kW32 : L.qU32) + (size_t)bh * C * D;
+  const float* B32 = (kKeys ? L.kbias32 : L.qbias32) + (size_t)bh * C;
+  const double* W64 = (kKeys ? L.kW64 : L.qU64) + (size_t)bh * C * D;
+  const double* B64 = (kKeys ? L.kbias64 : L.qbias64) + (size_t)bh * C;
+  const float* WN = (kKeys ? L.kwnorm : L.qwnorm) + (size_t)bh * C;
 
   extern __shared__ float smem[];
   float* Xs = smem;                          // [128][DP]
   float* Ws = Xs + kAsgPts * DP;             // [64][DP]
   float* Bs = Ws + kAsgChunk * DP;           // [64]
-  float* xnorm = Bs + kAsgChunk;             // [128]
-  int* lab = (int*)(xnorm + kAsgPts);        // [128]
+  float* scl = Bs + kAsgChunk;               // [128] per-point score scale
+  int* lab = (int*)(scl + kAsgPts);          // [128]
   int* order = lab + kAsgPts;                // [128]
   int* refine = order + kAsgPts;             // [128]
-  double* a64 = (double*)(refine + kAsgPts); // [128]
+  double* bval = (double*)(refine + kAsgPts);  // [128]
+  double* xs64 = bval + kAsgPts;             // [8 warps][128]
   __shared__ float s_red[2][8];
   __shared__ double red[8];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // features: two threads per row, every other element
   {
     const int p = tid >> 1, h = tid & 1;
     const size_t row = (size_t)bh * L.N + p0 + p;
-    for (int a = h; a < D; a += 2) {
-      float v = 0.f;
-      if (p < np) {
-        if constexpr (kKeys) v = to_f32(K[row * D + a]);
-        else v = L.r32[row * D + a];
-      }
-      Xs[p * DP + a] = v;
-    }
+    for (int a = h; a < D; a += 2) Xs[p * DP + a] = p < np ? to_f32(X[row * D + a]) : 0.f;
   }
-  // largest centroid-weight norm and |bias| (block max)
+  if (tid < kAsgPts) scl[tid] = kKeys ? 1.f : (tid < np ? L.inv_rms[(size_t)bh * L.N + p0 + tid] : 0.f);
   {
     float wm = 0.f, bm = 0.f;
     for (int j = tid; j < C; j += 256) {
@@ -334,11 +410,6 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
   for (int w = 0; w < 8; ++w) {
     s_wmax = fmaxf(s_wmax, s_red[0][w]);
     s_bmax = fmaxf(s_bmax, s_red[1][w]);
-  }
-  if (tid < kAsgPts) {
-    float s = 0.f;
-    for (int a = 0; a < D; ++a) s = fmaf(Xs[tid * DP + a], Xs[tid * DP + a], s);
-    xnorm[tid] = sqrtf(s);
   }
 
   const int pg = tid >> 4, cg = tid & 15;
@@ -383,7 +454,7 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
       const int gj = c0 + j;
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        const float sc = Bs[j] - 2.f * acc[r][i];
+        const float sc = Bs[j] - 2.f * acc[r][i] * scl[pg + 16 * r];
         if (sc < b1[r] || (sc == b1[r] && gj < i1[r])) {
           b2[r] = b1[r];
           b1[r] = sc;
@@ -394,7 +465,6 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
       }
     }
   }
-  // merge the 16 partial top-2 lists of each point (lanes of one half-warp)
 #pragma unroll
   for (int r = 0; r < 8; ++r) {
 #pragma unroll
@@ -416,71 +486,39 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int p = pg + 16 * r;
-      const float delta = 4.f * (D + 2) * u * xnorm[p] * s_wmax + 2.f * u * s_bmax;
+      const size_t row = (size_t)bh * L.N + p0 + p;
+      const float xn = p < np ? (kKeys ? L.knorm[row] : L.qxnorm[row]) : 0.f;
+      // |error of b - 2 s x.w| <= 2 (D+2) u ||x|| s ||w|| + u |b| (+ the scale's rounding); x4 margin
+      const float delta = 4.f * (D + 4) * u * xn * s_wmax + 2.f * u * s_bmax;
       lab[p] = (i1[r] >= 0 && i1[r] < C) ? i1[r] : 0;  // non-finite scores never yield a bad label
+      bval[p] = (double)b1[r];
       refine[p] = (p < np) && !(b2[r] - b1[r] > 2.f * delta);
     }
   }
   __syncthreads();
-
-  // fp64 re-decision of the (rare) points within the rounding bound: one warp per point, lanes
-  // over groups, lowest index on exact ties
   for (int p = warp; p < np; p += 8) {
     if (!refine[p]) continue;
-    const size_t row = (size_t)bh * L.N + p0 + p;
-    double bestv = INFINITY;
-    int best = 0x7fffffff;
-    for (int j = lane; j < C; j += 32) {
-      const double* w = W64 + (size_t)j * D;
-      double dot = 0.0;
-      for (int a = 0; a < D; ++a) {
-        double x;
-        if constexpr (kKeys) x = (double)Xs[p * DP + a];
-        else x = L.r64[row * D + a];
-        dot += x * w[a];
-      }
-      const double sc = B64[j] - 2.0 * dot;
-      if (sc < bestv) {  // ascending j per lane: strict < keeps the lower index
-        bestv = sc;
-        best = j;
-      }
+    double* xs = xs64 + warp * 128;
+    for (int a = lane; a < D; a += 32) xs[a] = (double)Xs[p * DP + a];
+    __syncwarp();
+    int best;
+    double bv;
+    redecide_fp64<kKeys>(L, bh, xs, D, C, W64, B64, best, bv);
+    if (lane == 0) {
+      lab[p] = best;
+      bval[p] = bv;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const double ov = __shfl_xor_sync(0xffffffffu, bestv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, best, o);
-      if (ov < bestv || (ov == bestv && oi < best)) {
-        bestv = ov;
-        best = oi;
-      }
-    }
-    if (lane == 0) lab[p] = (best >= 0 && best < C) ? best : 0;
-  }
-  __syncthreads();
-  // exact fp64 score of each point's group (objective): one thread per point
-  if (tid < np) {
-    const int l = lab[tid];
-    const double* w = W64 + (size_t)l * D;
-    const size_t row = (size_t)bh * L.N + p0 + tid;
-    double dot = 0.0;
-    for (int a = 0; a < D; ++a) {
-      double x;
-      if constexpr (kKeys) x = (double)Xs[tid * DP + a];
-      else x = L.r64[row * D + a];
-      dot += x * w[a];
-    }
-    a64[tid] = B64[l] - 2.0 * dot;
+    __syncwarp();
   }
   __syncthreads();
   int* labels = (kKeys ? L.klabel : L.qlabel) + (size_t)bh * L.N;
   if (tid < np) labels[p0 + tid] = lab[tid];
-  const double jsum = block_sum(tid < np ? a64[tid] : 0.0, red);
+  const double jsum = block_sum(tid < np ? bval[tid] : 0.0, red);
   const int nref = __syncthreads_count(tid < np ? refine[tid] : 0);
   if (tid == 0) {
     atomicAdd((kKeys ? L.kJ : L.qJ) + (size_t)bh * L.iters_cap + it, jsum);
     if (nref) atomicAdd((kKeys ? L.krefined : L.qrefined) + bh, nref);
   }
-  // stable order of the block's points by label, then fp64 sums per (run, dim)
   if (tid < np) {
     const int l = lab[tid];
     int rk = 0;
@@ -491,23 +529,21 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
     order[rk] = tid;
   }
   __syncthreads();
+  // group sums (fp64): keys x, queries x / rms (both products exact in fp64)
   double* sums = (kKeys ? L.ksum : L.qsum) + (size_t)bh * C * D;
   int* counts = (kKeys ? L.kcount : L.qcount) + (size_t)bh * C;
-  const int nparts = D >= 256 ? 1 : 256 / D;
+  const int nparts = 256 / D;
   if (tid < nparts * D) {
     const int a = tid % D, part = tid / D;
     const int q0 = part * np / nparts, q1 = (part + 1) * np / nparts;
-    for (int a2 = a; a2 < D; a2 += (D >= 256 ? 256 : D)) {
-      double acc = 0.0;
-      for (int q = q0; q < q1; ++q) {
-        const int p = order[q];
-        acc += (double)Xs[p * DP + a2];
-        if (q == q1 - 1 || lab[order[q + 1]] != lab[p]) {
-          atomicAdd(sums + (size_t)lab[p] * D + a2, acc);
-          acc = 0.0;
-        }
+    double acc = 0.0;
+    for (int q = q0; q < q1; ++q) {
+      const int p = order[q];
+      acc += (double)Xs[p * DP + a] * (double)scl[p];
+      if (q == q1 - 1 || lab[order[q + 1]] != lab[p]) {
+        atomicAdd(sums + (size_t)lab[p] * D + a, acc);
+        acc = 0.0;
       }
-      if (D < 256) break;
     }
   }
   if (tid < np && (tid == 0 || lab[order[tid - 1]] != lab[order[tid]])) {
@@ -516,82 +552,6 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
     while (q < np && lab[order[q]] == l) ++q;
     atomicAdd(counts + l, q - tid);
   }
-}
-
-// ------------------------------------------------------------------------------------------
-// a3: query responses r_q = q . c_j / sqrt(d) (fp64) and per-query RMS normalisation
-// (Table D.1, "Per query RMS"): r~ = r / sqrt(mean_j r_j^2 + 1e-12).  32 queries per block.
-// ------------------------------------------------------------------------------------------
-template <typename T>
-__global__ void __launch_bounds__(256) qresp_kernel(Layout L, const T* __restrict__ Q) {
-  extern __shared__ double shq[];
-  const int d = L.d, Ck = L.Ck, bh = blockIdx.y;
-  const int p0 = blockIdx.x * 32, np = min(32, L.N - p0);
-  double* qs = shq;                 // [32][d+1]
-  double* cs = qs + 32 * (d + 1);   // [32][d+1]
-  double* rs = cs + 32 * (d + 1);   // [32][Ck]
-  __shared__ double inv[32];
-  __shared__ double red[8];
-  const int tid = threadIdx.x;
-  for (int e = tid; e < 32 * d; e += 256) {
-    const int p = e / d, a = e % d;
-    qs[p * (d + 1) + a] = p < np ? (double)to_f32(Q[((size_t)bh * L.N + p0 + p) * d + a]) : 0.0;
-  }
-  const double rsd = 1.0 / sqrt((double)d);
-  for (int c0 = 0; c0 < Ck; c0 += 32) {
-    const int nc = min(32, Ck - c0);
-    __syncthreads();
-    for (int e = tid; e < 32 * d; e += 256) {
-      const int j = e / d, a = e % d;
-      cs[j * (d + 1) + a] = j < nc ? L.kcent[((size_t)bh * Ck + c0 + j) * d + a] : 0.0;
-    }
-    __syncthreads();
-    for (int e = tid; e < 32 * 32; e += 256) {
-      const int p = e >> 5, j = e & 31;
-      if (j >= nc) continue;
-      double acc = 0.0;
-      for (int a = 0; a < d; ++a) acc += qs[p * (d + 1) + a] * cs[j * (d + 1) + a];
-      rs[p * Ck + c0 + j] = acc * rsd;
-    }
-  }
-  __syncthreads();
-  if (tid < 32) {
-    double ms = 0.0;
-    for (int j = 0; j < Ck; ++j) ms += rs[tid * Ck + j] * rs[tid * Ck + j];
-    inv[tid] = 1.0 / sqrt(ms / Ck + 1e-12);
-  }
-  __syncthreads();
-  double nrm = 0.0;
-  for (int e = tid; e < 32 * Ck; e += 256) {
-    const int p = e / Ck, j = e % Ck;
-    if (p >= np) continue;
-    const double v = rs[p * Ck + j] * inv[p];
-    const size_t o = ((size_t)bh * L.N + p0 + p) * Ck + j;
-    L.r64[o] = v;
-    L.r32[o] = (float)v;
-    split3(v, L.rb, (size_t)L.BH * L.N * L.Dq, ((size_t)bh * L.N + p0 + p) * L.Dq + j);
-    nrm += v * v;
-  }
-  for (int e = tid; e < 32 * (L.Dq - Ck); e += 256) {  // zero the padding columns
-    const int p = e / (L.Dq - Ck), j = Ck + e % (L.Dq - Ck);
-    if (p >= np) continue;
-    const size_t o = ((size_t)bh * L.N + p0 + p) * L.Dq + j;
-    const size_t plane = (size_t)L.BH * L.N * L.Dq;
-    const __nv_bfloat16 z = __float2bfloat16(0.f);
-    L.rb[o] = z;
-    L.rb[plane + o] = z;
-    L.rb[2 * plane + o] = z;
-  }
-  if (tid < np) {
-    double q2 = 0.0;
-    for (int j = 0; j < Ck; ++j) {
-      const double v = rs[tid * Ck + j] * inv[tid];
-      q2 += v * v;
-    }
-    L.rnorm[(size_t)bh * L.N + p0 + tid] = (float)sqrt(q2);
-  }
-  nrm = block_sum(nrm, red);
-  if (tid == 0) atomicAdd(L.T0q + bh, nrm);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -879,25 +839,36 @@ template <typename T>
 static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool warm, int iters,
                                   cudaStream_t st) {
   const int d = L.d;
+  const bool tc = L.dtype == SPARSEPR_BF16;  // bf16 inputs: tensor-core quadratic forms
+  const size_t dd = (size_t)L.BH * d * d;
+  const int split_blocks = (int)((dd + 255) / 256 < 4096 ? (dd + 255) / 256 : 4096);
+  const size_t qf_smem = (size_t)(d + 64) * (d + 1) * sizeof(float);
+  cudaFuncSetAttribute(rowqf_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qf_smem);
+  // keys: metric M = Qs^T Qs / d, objective constant sum_t k_t^T M k_t, key norms
   launch(metric_kernel<T>, dim3(L.BH, d), 128, 0, st, L, Q);
   cudaMemsetAsync(L.T0k, 0, sizeof(double) * L.BH, st);
-  const size_t kn_smem = (size_t)(d + 64) * (d + 1) * sizeof(float);
-  cudaFuncSetAttribute(key_norms_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kn_smem);
-  launch(key_norms_kernel<T>, dim3((L.N + 63) / 64, L.BH), 256, kn_smem, st, L, K);
+  cudaMemsetAsync(L.T0q, 0, sizeof(double) * L.BH, st);
+  if (tc) {
+    launch(split_mat_kernel, split_blocks, 256, 0, st, (const double*)L.M, L.Mb, dd);
+    const sparsepr_status s = launch_rowqf_tc(L, 0, K, st);
+    if (s != SPARSEPR_OK) return s;
+  } else {
+    launch(rowqf_simt_kernel<T>, dim3((L.N + 63) / 64, L.BH), 256, qf_smem, st, L, K, 0);
+  }
   if (!warm) {
     launch(km_draw_kernel, L.BH, 128, 0, st, L, 0, L.Ck);
     launch(kcent_init_kernel<T>, dim3(L.BH, L.Ck), 128, 0, st, L, K);
   }
   SPR_LAUNCH_CHECK();
   launch(km_reset_kernel, L.BH, 128, 0, st, L, 0, iters);
-  cudaMemsetAsync(L.T0q, 0, sizeof(double) * L.BH, st);
   // bf16 inputs with at most 256 groups score on the tensor cores; otherwise on CUDA cores
   const bool tc_keys = km_tc_supported(L, true), tc_queries = km_tc_supported(L, false);
   cudaMemsetAsync(L.kWb, 0, (size_t)3 * L.BH * L.Ckp * d * 2, st);
-  cudaMemsetAsync(L.qWb, 0, (size_t)3 * L.BH * L.Cqp * L.Dq * 2, st);
-  const size_t asg_smem_k = assign_smem_bytes(d);
+  cudaMemsetAsync(L.qWb, 0, (size_t)3 * L.BH * L.Cqp * d * 2, st);
+  const size_t asg_smem = assign_smem_bytes(d);
   const int nblk = (L.N + kAsgPts - 1) / kAsgPts;
-  cudaFuncSetAttribute(kmeans_assign_kernel<T, KeyFeat>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asg_smem_k);
+  cudaFuncSetAttribute(kmeans_assign_kernel<T, KeyFeat>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asg_smem);
+  cudaFuncSetAttribute(kmeans_assign_kernel<T, QueryFeat>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asg_smem);
   for (int it = 0; it <= iters; ++it) {
     launch(kprep_kernel, dim3(L.BH, L.Ck), 128, 0, st, L, it, iters);
     if (it < iters) {
@@ -905,30 +876,34 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
         const sparsepr_status s = launch_kmeans_assign_tc(L, true, K, it, st);
         if (s != SPARSEPR_OK) return s;
       } else {
-        launch(kmeans_assign_kernel<T, KeyFeat>, dim3(nblk, L.BH), 256, asg_smem_k, st, L, K, it);
+        launch(kmeans_assign_kernel<T, KeyFeat>, dim3(nblk, L.BH), 256, asg_smem, st, L, K, it);
       }
     }
   }
   SPR_LAUNCH_CHECK();
-  const size_t qr_smem = (size_t)(2 * 32 * (d + 1) + 32 * L.Ck) * sizeof(double);
-  cudaFuncSetAttribute(qresp_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qr_smem);
-  launch(qresp_kernel<T>, dim3((L.N + 31) / 32, L.BH), 256, qr_smem, st, L, Q);
+  // queries: Gc from the key-group centroids, 1/rms_q, ||r~_q||, objective constant
+  launch(gc_kernel, dim3(L.BH, d), 128, 0, st, L);
+  if (tc) {
+    launch(split_mat_kernel, split_blocks, 256, 0, st, (const double*)L.Gc, L.Gcb, dd);
+    const sparsepr_status s = launch_rowqf_tc(L, 1, Q, st);
+    if (s != SPARSEPR_OK) return s;
+  } else {
+    launch(rowqf_simt_kernel<T>, dim3((L.N + 63) / 64, L.BH), 256, qf_smem, st, L, Q, 1);
+  }
   if (!warm) {
     launch(km_draw_kernel, L.BH, 128, 0, st, L, 1, L.Cq);
-    launch(qcent_init_kernel, dim3(L.BH, L.Cq), 128, 0, st, L);
+    launch(qcent_init_kernel<T>, dim3(L.BH, L.Cq), 128, 0, st, L, Q);
   }
   launch(km_reset_kernel, L.BH, 128, 0, st, L, 1, iters);
   SPR_LAUNCH_CHECK();
-  const size_t asg_smem_q = assign_smem_bytes(L.Ck);
-  cudaFuncSetAttribute(kmeans_assign_kernel<T, QueryFeat>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asg_smem_q);
   for (int it = 0; it <= iters; ++it) {
     launch(qprep_kernel, dim3(L.BH, L.Cq), 128, 0, st, L, it, iters);
     if (it < iters) {
       if (tc_queries) {
-        const sparsepr_status s = launch_kmeans_assign_tc(L, false, K, it, st);
+        const sparsepr_status s = launch_kmeans_assign_tc(L, false, Q, it, st);
         if (s != SPARSEPR_OK) return s;
       } else {
-        launch(kmeans_assign_kernel<T, QueryFeat>, dim3(nblk, L.BH), 256, asg_smem_q, st, L, K, it);
+        launch(kmeans_assign_kernel<T, QueryFeat>, dim3(nblk, L.BH), 256, asg_smem, st, L, Q, it);
       }
     }
   }

@@ -30,7 +30,6 @@ std::atomic<long long> sparsepr::g_launches{0};
 
 namespace {
 
-constexpr int kMaxKeyGroupsBuilt = 256;  // query-response dimension of the assignment kernel
 
 sparsepr_status validate(const sparsepr_config* c) {
   if (!c) return SPARSEPR_ERR_INVALID_ARG;
@@ -50,7 +49,6 @@ sparsepr_status validate(const sparsepr_config* c) {
   if (c->km_iters > 10000 || c->km_iters_warm > 10000) return SPARSEPR_ERR_INVALID_ARG;
   if ((double)c->B * c->H * c->N * 256.0 > 9.0e18) return SPARSEPR_ERR_INVALID_ARG;
   if (c->d != 64 && c->d != 128) return SPARSEPR_ERR_UNSUPPORTED;
-  if (c->n_kgroups > kMaxKeyGroupsBuilt) return SPARSEPR_ERR_UNSUPPORTED;
   return SPARSEPR_OK;
 }
 
@@ -105,26 +103,27 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   take(L.klabel, BH * N * 4);
   take(L.kJ, BH * cap * 8);
   take(L.krefined, BH * 4);
-  take(L.r64, BH * N * Ck * 8);
-  take(L.r32, BH * N * Ck * 4);
+  L.Ckp = (c.n_kgroups + 15) / 16 * 16;
+  L.Cqp = (c.n_qgroups + 15) / 16 * 16;
+  take(L.Gc, BH * d * d * 8);
+  take(L.inv_rms, BH * N * 4);
+  take(L.qxnorm, BH * N * 4);
   take(L.qcent, BH * Cq * Ck * 8);
-  take(L.qW32, BH * Cq * Ck * 4);
+  take(L.qU64, BH * Cq * d * 8);
+  take(L.qU32, BH * Cq * d * 4);
   take(L.qbias64, BH * Cq * 8);
   take(L.qbias32, BH * Cq * 4);
   take(L.qwnorm, BH * Cq * 4);
-  take(L.qsum, BH * Cq * Ck * 8);
+  take(L.qsum, BH * Cq * d * 8);
   take(L.qcount, BH * Cq * 4);
   take(L.qlabel, BH * N * 4);
   take(L.qJ, BH * cap * 8);
   take(L.qrefined, BH * 4);
-  L.Ckp = (c.n_kgroups + 15) / 16 * 16;
-  L.Cqp = (c.n_qgroups + 15) / 16 * 16;
-  L.Dq = (c.n_kgroups + 63) / 64 * 64;
   take(L.kWb, 3 * BH * (size_t)L.Ckp * d * 2);
-  take(L.qWb, 3 * BH * (size_t)L.Cqp * L.Dq * 2);
-  take(L.rb, 3 * BH * N * (size_t)L.Dq * 2);
+  take(L.qWb, 3 * BH * (size_t)L.Cqp * d * 2);
+  take(L.Mb, 3 * BH * d * d * 2);
+  take(L.Gcb, 3 * BH * d * d * 2);
   take(L.knorm, BH * N * 4);
-  take(L.rnorm, BH * N * 4);
   take(L.kperm, BH * N * 4);
   take(L.kinv, BH * N * 4);
   take(L.koff, BH * (Ck + 1) * 4);
