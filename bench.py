@@ -56,6 +56,22 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(values, world, device=None):
+    """Element-wise max of `values` over all ranks (one all_reduce MAX; identity at world 1).
+    Per-step device times are combined this way: the job takes as long as its slowest rank."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def whole_job_tflops(world, flops_per_call, ms_per_call):
+    """Throughput of the whole job: every rank runs one independent call of `flops_per_call`
+    (dense-equivalent) per step, and a step lasts `ms_per_call` (the max over ranks)."""
+    return world * flops_per_call / (ms_per_call * 1e-3) / 1e12
+
+
 def workload_config(w, extra=None):
     c = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "density": w.density, "s": w.s,
          "n_kgroups": w.n_kgroups, "n_qgroups": w.n_qgroups, "P": w.P,
@@ -219,10 +235,7 @@ def run_ours(args, w, world, rank, local):
     kern_ms = [a.elapsed_time(b) for a, b in kev]
     ms = statistics.mean(step_ms)
     kms = statistics.mean(kern_ms)
-    t = torch.tensor([ms, kms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max, kms_max = float(t[0]), float(t[1])
+    ms_max, kms_max = max_over_ranks([ms, kms], world, dev)
 
     # end to end through the public API with host buffers (pinned), copies inside the region
     Qh, Kh, Vh = Qc.pin_memory(), Kc.pin_memory(), Vc.pin_memory()
@@ -241,15 +254,12 @@ def run_ours(args, w, world, rank, local):
             e2e_ev[i - 1][1].record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in e2e_ev)
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t[0])
+    e2e_ms, = max_over_ranks([e2e_ms], world, dev)
 
     if rank == 0:
         pk = peaks()
         flops = w.dense_flops()
-        value = world * flops / (ms_max * 1e-3) / 1e12
+        value = whole_job_tflops(world, flops, ms_max)
         kflops = 4.0 * w.d * pairs
         achieved = kflops / (kms_max * 1e-3) / 1e12
         peak = pk["bf16_tflops"]
@@ -268,7 +278,7 @@ def run_ours(args, w, world, rank, local):
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
                          "peak_source": f"{pk['source']} bf16 dense (burst)",
                          "algorithmic": f"4*d*executed pairs = {kflops:.4g} flop per launch"},
-            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+            "e2e": {"value": whole_job_tflops(world, flops, e2e_ms), "unit": "TFLOPS",
                     "h2d_bytes_per_step": 3 * Q.numel() * elt, "d2h_bytes_per_step": O.numel() * O.element_size(),
                     "ms_per_step": e2e_ms},
             "gpu_launches": launches,
@@ -293,9 +303,13 @@ def main():
     ap.add_argument("--workload", type=int, default=1, help="index into configs.WORKLOADS")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload on this many heads instead (a smaller case for profilers)")
     args = ap.parse_args()
     world, rank, local = dist_env()
     w = configs.workload(args.workload)
+    if args.heads > 0:
+        w = configs.scaled_down(w, heads=args.heads)
     if args.impl == "reference":
         run_reference(args, w, world, rank)
     else:

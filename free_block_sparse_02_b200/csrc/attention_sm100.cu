@@ -39,6 +39,21 @@ constexpr int kSubRows = 16;    // rows per TMA box of K/V
 constexpr int kSubPerTile = kTcTileN / kSubRows;
 constexpr int kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kExpPolyEvery = 4;           // 1 in 4 exponential pairs on the FMA pipe (0: none)
+
+// 2^x on the FMA pipe for x <= kRescaleThreshold (0 below -125, so -inf gives 0): Cody-Waite
+// style reduction x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low mantissa
+// bits) and f in [-1/2, 1/2], then a cubic in f fitted to 2^f by least squares on relative error
+// at Chebyshev nodes with Lawson reweighting (max relative error 7.5e-5, far below the bf16
+// rounding of P), and n added to the exponent field.
+__device__ __forceinline__ float exp2_poly(float x) {
+  const float xc = fmaxf(x, -125.f);
+  const float t = xc + 12582912.f;
+  const float f = xc - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(0.0551716648f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
+  const float y = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  return x < -125.f ? 0.f : y;
+}
 static_assert(kAttnTileMTc == 2 * kTcTileM, "a work item is two MMA tiles");
 
 template <int D>
@@ -298,23 +313,35 @@ __global__ void __launch_bounds__(384, 1)
     for (int j = 0; ok && j < ntiles; ++j) {
       int rows[kSubPerTile], valid[kSubPerTile];
       next_tile(st, segs, nseg, row_base, oob_row, rows, valid);
-      if (!mbar_wait(s_full + t, j & 1, &s_abort)) {
+      bool full = true;  // every key of the tile is real (the same for every thread of the CTA)
+#pragma unroll
+      for (int b = 0; b < kSubPerTile; ++b) full = full && valid[b] == kSubRows;
+      // warp-uniform: the tcgen05.ld below needs every lane of the warp
+      const bool okw = mbar_wait(s_full + t, j & 1, &s_abort);
+      if (!__all_sync(0xffffffffu, okw)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // pass 1: row max over the valid keys
-      float tmax = -INFINITY;
+      // pass 1: row max over the real keys (four loads, one wait; eight independent chains)
+      float tmax;
+      {
+        uint32_t sv[kTcTileN];
 #pragma unroll
-      for (int c = 0; c < kTcTileN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + c * 32, r);
+        for (int c = 0; c < kTcTileN / 32; ++c)
+          tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
         tmem_wait_ld();
+        if (!full) {  // padded keys of partial boxes take no part
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const int col = c * 32 + k;
-          if ((col & (kSubRows - 1)) < valid[col / kSubRows]) tmax = fmaxf(tmax, __uint_as_float(r[k]));
+          for (int k = 0; k < kTcTileN; ++k)
+            if ((k & (kSubRows - 1)) >= valid[k / kSubRows]) sv[k] = __float_as_uint(-INFINITY);
         }
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sv[k]);
+#pragma unroll
+        for (int k = 8; k < kTcTileN; ++k) mx[k & 7] = fmaxf(mx[k & 7], __uint_as_float(sv[k]));
+        tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       }
       tmax *= scale2;
       // lazy rescale: move the running max only when this tile exceeds it by > 2^8
@@ -327,7 +354,8 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (__any_sync(0xffffffffu, need && j > 0)) {
         // O_t holds P_t(0..j-1) V (complete: S_t(j) was issued after the last of them)
-        if (!mbar_wait(o_bar + t, (j - 1) & 1, &s_abort)) {
+        const bool okw2 = mbar_wait(o_bar + t, (j - 1) & 1, &s_abort);
+        if (!__all_sync(0xffffffffu, okw2)) {
           ok = false;
           break;
         }
@@ -345,38 +373,40 @@ __global__ void __launch_bounds__(384, 1)
       }
       l *= factor;
       m_used = m_new;
-      // pass 2: P = 2^(s*scale - m) as packed bf16 over the first 64 columns of S_t (each
-      // 64-key half is read before its 32 packed columns are written over already-read ones)
+      // pass 2: P = 2^(s*scale - m) as packed bf16 over the first 64 columns of S_t, 64 keys at
+      // a time (each half is read before its 32 packed columns overwrite already-read ones).
+      // Padded keys are set to -inf first, so their probability is exactly 0.  Every
+      // kExpPolyEvery-th pair of exponentials runs on the FMA pipe (exp2_poly) to relieve the
+      // special-function unit.
       const float neg_m = -m_used;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t ra[32], rb[32];
-        tmem_ld32(tS + c * 64, ra);
-        tmem_ld32(tS + c * 64 + 32, rb);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sv[64];
+        tmem_ld32(tS + h * 64, *reinterpret_cast<uint32_t(*)[32]>(sv));
+        tmem_ld32(tS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
         tmem_wait_ld();
+        if (!full) {
+#pragma unroll
+          for (int k = 0; k < 64; ++k) {
+            const int col = h * 64 + k;
+            if ((col & (kSubRows - 1)) >= valid[col / kSubRows]) sv[k] = __float_as_uint(-INFINITY);
+          }
+        }
         uint32_t pk[32];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int c0 = c * 64 + 2 * k, c1 = c0 + 1;
-          const bool v0 = (c0 & (kSubRows - 1)) < valid[c0 / kSubRows];
-          const bool v1 = (c1 & (kSubRows - 1)) < valid[c1 / kSubRows];
-          const float p0 = v0 ? ex2(fmaf(__uint_as_float(ra[2 * k]), scale2, neg_m)) : 0.f;
-          const float p1 = v1 ? ex2(fmaf(__uint_as_float(ra[2 * k + 1]), scale2, neg_m)) : 0.f;
-          l += p0 + p1;
+        for (int k = 0; k < 32; ++k) {
+          const float x0 = fmaf(__uint_as_float(sv[2 * k]), scale2, neg_m);
+          const float x1 = fmaf(__uint_as_float(sv[2 * k + 1]), scale2, neg_m);
+          const bool poly = kExpPolyEvery > 0 && (k % kExpPolyEvery) == kExpPolyEvery - 1;
+          const float p0 = poly ? exp2_poly(x0) : ex2(x0);
+          const float p1 = poly ? exp2_poly(x1) : ex2(x1);
+          ls[k & 3] += p0 + p1;
           pk[k] = pack_bf16x2(p0, p1);
         }
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int c0 = c * 64 + 32 + 2 * k, c1 = c0 + 1;
-          const bool v0 = (c0 & (kSubRows - 1)) < valid[c0 / kSubRows];
-          const bool v1 = (c1 & (kSubRows - 1)) < valid[c1 / kSubRows];
-          const float p0 = v0 ? ex2(fmaf(__uint_as_float(rb[2 * k]), scale2, neg_m)) : 0.f;
-          const float p1 = v1 ? ex2(fmaf(__uint_as_float(rb[2 * k + 1]), scale2, neg_m)) : 0.f;
-          l += p0 + p1;
-          pk[16 + k] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tS + c * 32, pk);
+        tmem_st32(tS + h * 32, pk);
       }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full + t);

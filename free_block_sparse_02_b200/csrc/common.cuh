@@ -16,6 +16,7 @@ namespace sparsepr {
 
 constexpr int kMaxGroups = 1024;  // C_k, C_q upper bound (route rows fit one CTA's smem)
 constexpr int kMaxProbes = 4096;
+constexpr int kSortChunk = 4096;   // tokens per chunk of the parallel stable group sort
 
 // Device status word values (a subset of sparsepr_status).
 constexpr int kDevOk = 0;
@@ -70,7 +71,8 @@ struct Layout {
   // of group g is ||nu_g||^2 - 2 (q . u_g) / rms_q with u_g = C^T nu_g / sqrt(d), and the group
   // sums are sums of q / rms_q, projected back as nu_g = C S_g / (sqrt(d) n_g).
   double* Gc;                     // [BH, d, d]
-  float* inv_rms;                 // [BH, N]   1 / rms_q
+  float* inv_rms;                 // [BH, N]   1 / rms_q (scores)
+  double* inv_rms64;              // [BH, N]   1 / rms_q (group sums)
   float* qxnorm;                  // [BH, N]   ||q|| / rms_q  (= ||r~_q|| bound for the score error)
   double* qcent;                  // [BH, Cq, Ck] nu_g (response space)
   double* qU64;                   // [BH, Cq, d]  u_g
@@ -93,7 +95,15 @@ struct Layout {
   __nv_bfloat16* Gcb;             // [3][BH, d, d]     Gc
   float* knorm;                   // [BH, N] ||k_t||_2 (rounding bound of the key scores)
 
+  // points of the tensor-core assignment whose two best scores were within the rounding bound,
+  // re-decided in fp64 by the update pass: CTA c of the assignment grid appends to its own
+  // segment starting at (first tile of c) * 128, entries (row bh*N + p, float bits of the
+  // tentative score), and leaves the segment length in rcnt[c]
+  int2* rlist;                    // [BH * ceil(N/128) * 128]
+  int* rcnt;                      // [BH * ceil(N/128)]
+
   // group-contiguous order (stable counting sort)
+  int* sort_hist;                 // [BH, 2, ceil(N / kSortChunk), max(Ck, Cq)] chunk histograms
   int* kperm;                     // [BH, N]   position -> token
   int* kinv;                      // [BH, N]   token -> position
   int* koff;                      // [BH, Ck+1]

@@ -91,36 +91,30 @@ __global__ void __launch_bounds__(256) ridge_gram_kernel(Layout L) {
 // Shared memory of the solve: the (d+1)^2 system and a (d+1) x 33 block of right-hand sides.
 static size_t ridge_solve_smem(int d) { return (size_t)((d + 1) * (d + 1) + (d + 1) * 33) * sizeof(double); }
 
-// In-place lower Cholesky of the n x n matrix in shared memory; false if a pivot is not
-// above `tol` (or not finite).  Trailing update: thread rows i, columns j <= i.
-__device__ bool chol_smem_tol(double* G, int n, int ld, double tol) {
-  __shared__ int fail;
-  if (threadIdx.x == 0) fail = 0;
+// Cholesky G = L L^T of the n x n matrix in shared memory with one barrier per step: step k
+// reads column k of the (lower) trailing matrix, writes L's column k below the diagonal into
+// row k of the upper triangle (L_ik at G[k][i], i > k) and L_kk into diag[k], and updates the
+// trailing lower part G[i][j] -= G[i][k] G[j][k] / G[k][k] (k < j <= i) without touching
+// column k.  False if a pivot is not above `tol` (or not finite).
+__device__ bool chol_smem_tol(double* G, int n, int ld, double tol, double* diag) {
+  const int nthr = blockDim.x;
   __syncthreads();
   for (int k = 0; k < n; ++k) {
-    if (threadIdx.x == 0) {
-      const double piv = G[k * ld + k];
-      if (!(piv > tol) || !isfinite(piv)) fail = 1;
-      else G[k * ld + k] = sqrt(piv);
-    }
-    __syncthreads();
-    if (fail) return false;
-    const double lkk = G[k * ld + k];
-    for (int i = k + 1 + threadIdx.x; i < n; i += blockDim.x) G[i * ld + k] /= lkk;
-    __syncthreads();
-    const int m = n - k - 1;
-    // (i, j) with k < j <= i < n: warp-strided rows, lanes over columns
-    const int nw = blockDim.x >> 5, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const double piv = G[k * ld + k];
+    if (!(piv > tol) || !isfinite(piv)) return false;  // the same value in every thread
+    const double lkk = sqrt(piv), inv = 1.0 / lkk, ipiv = 1.0 / piv;
+    if (threadIdx.x == 0) diag[k] = lkk;
+    for (int i = k + 1 + threadIdx.x; i < n; i += nthr) G[k * ld + i] = G[i * ld + k] * inv;
+    // trailing pairs (i, j), k < j <= i < n: warp-strided rows, lanes over columns
+    const int nw = nthr >> 5, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = k + 1 + w; i < n; i += nw) {
-      const double lik = G[i * ld + k];
+      const double lik = G[i * ld + k] * ipiv;
       for (int j = k + 1 + lane; j <= i; j += 32) G[i * ld + j] -= lik * G[j * ld + k];
     }
-    (void)m;
     __syncthreads();
   }
   return true;
 }
-__device__ bool chol_smem(double* G, int n, int ld) { return chol_smem_tol(G, n, ld, 0.0); }
 
 // One CTA per head: lam, Cholesky with up to three x10 jitter retries, the d right-hand sides,
 // then the residual-span basis by column-pivoted Gram-Schmidt on S = R^T W R and A <- A U U^T.
@@ -129,6 +123,7 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
   const int bh = blockIdx.x, d = L.d, n1 = d + 1, tid = threadIdx.x;
   double* G = shs;  // [n1][n1], later S [d][d]
   __shared__ double red[8];
+  __shared__ double ldiag[129];  // diagonal of the Cholesky factor
   __shared__ int s_piv;
   __shared__ double s_norm;
   const double* Gg = L.ridgeG + (size_t)bh * n1 * n1;
@@ -156,7 +151,7 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
   for (; retries <= 3; ++retries) {
     for (int e = tid; e < n1 * n1; e += blockDim.x) G[e] = Gg[e] + ((e / n1) == (e % n1) ? lam : 0.0);
     __syncthreads();
-    ok = chol_smem(G, n1, n1);
+    ok = chol_smem_tol(G, n1, n1, 0.0, ldiag);
     if (ok) break;
     lam = lam > 0.0 ? lam * 10.0 : (tr > 0.0 ? 1e-12 * tr / n1 : 1e-30);
   }
@@ -182,22 +177,22 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
       __syncthreads();
       for (int e = tid; e < n1 * 32; e += blockDim.x) Y[(e >> 5) * 33 + (e & 31)] = Bg[(e >> 5) * d + c0 + (e & 31)];
       __syncthreads();
-      for (int i = 0; i < n1; ++i) {
+      for (int i = 0; i < n1; ++i) {  // L y = b, L_ik = G[k][i]
         double part = 0.0;
-        for (int k = sub; k < i; k += 8) part += G[i * n1 + k] * Y[k * 33 + col];
+        for (int k = sub; k < i; k += 8) part += G[k * n1 + i] * Y[k * 33 + col];
         part += __shfl_xor_sync(0xffffffffu, part, 4);
         part += __shfl_xor_sync(0xffffffffu, part, 2);
         part += __shfl_xor_sync(0xffffffffu, part, 1);
-        if (sub == 0) Y[i * 33 + col] = (Y[i * 33 + col] - part) / G[i * n1 + i];
+        if (sub == 0) Y[i * 33 + col] = (Y[i * 33 + col] - part) / ldiag[i];
         __syncwarp();
       }
-      for (int i = n1 - 1; i >= 0; --i) {
+      for (int i = n1 - 1; i >= 0; --i) {  // L^T x = y, (L^T)_ik = L_ki = G[i][k]
         double part = 0.0;
-        for (int k = i + 1 + sub; k < n1; k += 8) part += G[k * n1 + i] * Y[k * 33 + col];
+        for (int k = i + 1 + sub; k < n1; k += 8) part += G[i * n1 + k] * Y[k * 33 + col];
         part += __shfl_xor_sync(0xffffffffu, part, 4);
         part += __shfl_xor_sync(0xffffffffu, part, 2);
         part += __shfl_xor_sync(0xffffffffu, part, 1);
-        if (sub == 0) Y[i * 33 + col] = (Y[i * 33 + col] - part) / G[i * n1 + i];
+        if (sub == 0) Y[i * 33 + col] = (Y[i * 33 + col] - part) / ldiag[i];
         __syncwarp();
       }
       __syncthreads();
@@ -223,7 +218,7 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
   __syncthreads();
   int rank = 0;
   int basis[128];
-  bool full = s_dmax > 0.0 && chol_smem_tol(S, d, d, 1e-10 * s_dmax);
+  bool full = s_dmax > 0.0 && chol_smem_tol(S, d, d, 1e-10 * s_dmax, ldiag);
   if (full) {
     rank = d;
   } else if (s_dmax > 0.0) {
@@ -412,6 +407,7 @@ sparsepr_status launch_fit_apply(const Layout& L, void* O, int out_dtype, cudaSt
   }
   const sparsepr_status s = launch_ridge_solve(L, st);
   if (s != SPARSEPR_OK) return s;
+  if (L.dtype == SPARSEPR_BF16) return launch_apply_tc(L, O, out_dtype, st);
   if (out_dtype == SPARSEPR_F32)
     return d == 64 ? launch_apply<float, 64>(L, O, st) : launch_apply<float, 128>(L, O, st);
   return d == 64 ? launch_apply<__nv_bfloat16, 64>(L, O, st) : launch_apply<__nv_bfloat16, 128>(L, O, st);

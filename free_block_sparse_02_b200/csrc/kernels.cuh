@@ -19,9 +19,15 @@ sparsepr_status launch_permute(const Layout& L, const void* Q, const void* K, co
 sparsepr_status launch_attention(const Layout& L, cudaStream_t st, cudaEvent_t ev_start, cudaEvent_t ev_stop);
 sparsepr_status launch_attention_tc(const Layout& L, cudaStream_t st, cudaEvent_t ev_start, cudaEvent_t ev_stop);
 sparsepr_status launch_fit_apply(const Layout& L, void* O, int out_dtype, cudaStream_t st);
+// O = O_sp + [O_sp, 1] A on unprobed rows, O_dense on probe rows, in token order (tensor cores).
+sparsepr_status launch_apply_tc(const Layout& L, void* O, int out_dtype, cudaStream_t st);
 sparsepr_status launch_ridge_solve(const Layout& L, cudaStream_t st);
 bool km_tc_supported(const Layout& L, bool keys);
-sparsepr_status launch_kmeans_assign_tc(const Layout& L, bool keys, const void* X, int it, cudaStream_t st);
+int km_tc_grid(const Layout& L, bool keys);
+// One Lloyd iteration after the centroid update: tensor-core assignment, then the fp64
+// re-decisions, group sums and counts (both kernels over the same G tile ranges).
+sparsepr_status launch_kmeans_iteration_tc(const Layout& L, bool keys, const void* X, int it, int G,
+                                           cudaStream_t st);
 sparsepr_status launch_rowqf_tc(const Layout& L, int which, const void* X, cudaStream_t st);
 
 // Upper bound of the number of query tiles of one head: sum_g ceil(n_g / tile) <= N/tile + C_q.

@@ -1,4 +1,4 @@
-// k-means assignment and per-row quadratic forms of the partition on the tensor cores
+// k-means assignment, update and per-row quadratic forms of the partition on the tensor cores
 // (tcgen05, results in TMEM, operands by TMA).
 //
 // "Partition the Support, Reconstruct the Residual" (arXiv 2608.18484), abstract: keys are
@@ -8,15 +8,32 @@
 // Both k-means run on the d-dimensional inputs (see partition.cu): the score of point x against
 // group j is  s_j = b_j - 2 sigma_x (x . w_j)  with (keys) w = M c, b = c^T M c, sigma = 1, or
 // (queries) w = u = C^T nu / sqrt(d), b = ||nu||^2, sigma = 1/rms_q; the label is argmin_j s_j,
-// lowest j on ties.  The dot products of a 128-point tile against every group are one MMA chain:
-// X (128 x d, bf16, exact) times W^T (d x C), W split into three bf16 terms (hi + mid + lo)
-// accumulated in fp32 in TMEM, which gives fp32-grade dots.  The epilogue (two threads per
-// point, its TMEM lane) keeps the best two scores; a point whose two best are within a
-// rigorous rounding bound is re-decided over all groups in fp64 by one warp, so labels agree
-// with an fp64 evaluation.  The objective takes the chosen group's score; the group sums
-// (fp64, of sigma x) are accumulated per run of equal labels after a counting sort of the
-// tile and flushed with one atomic per (run, dim).
+// lowest j on ties.
+//
+// One Lloyd iteration on the tensor-core path is three kernels over the same static split of the
+// BH * ceil(N/128) point tiles into G contiguous ranges (one per CTA, ranges may cross heads):
+//
+//  assignment  Persistent and warp-specialised (384 threads): warp 0 streams 128-point tiles of
+//              X by TMA through a ring of shared-memory stages (and the head's three-term W when
+//              the head changes), warp 1 issues the MMA chain X (128 x d, bf16, exact) times W^T
+//              (d x C; W = hi + mid + lo in bf16, fp32 accumulation: fp32-grade dots) into one
+//              of two TMEM accumulators, and two epilogue warpgroups take alternate tiles: one
+//              thread per point (its TMEM lane) scans every group's score, keeps the best two,
+//              writes the label and adds the best score to the objective.  A point whose two
+//              best are within a rigorous rounding bound goes to the CTA's re-decision list.
+//  re-decide   Re-decides the listed points over all groups in fp64 (one warp each, all over
+//              the GPU; label and objective corrected).
+//  update      For chunks of up to 8192 points of one head,
+//              counting-sorts the points by label in shared memory and sums each group's run:
+//              one thread per (group, 8 dimensions) gathers the run's rows (consecutive threads
+//              read consecutive 16-byte pieces of a row), accumulates sigma x in fp64 registers
+//              and adds the result with one atomic per (group, dimension) per chunk.
+//
+// Labels therefore equal the argmin of an fp64 evaluation, and the group sums are fp64 sums of
+// the exact inputs (keys) or of the inputs times their fp64 scale 1/rms (queries).
 #include <math.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -28,6 +45,10 @@ namespace sparsepr {
 using namespace sm100;
 
 constexpr int kKmTile = 128;
+constexpr int kKmThreads = 384;   // warp 0 TMA, warp 1 MMA, warps 4..11 epilogue
+constexpr int kKmUpdThreads = 512;
+constexpr int kKmMaxStages = 4;
+constexpr int kKmUpdChunk = 8192;  // points of one head sorted and summed at a time by the update
 
 __host__ __device__ inline int km_tc_tmem_cols(int n) {
   int c = 32;
@@ -35,291 +56,482 @@ __host__ __device__ inline int km_tc_tmem_cols(int n) {
   return c;
 }
 
-__host__ inline size_t km_tc_smem(int D, int Np) {
-  const size_t w = (size_t)3 * Np * D * 2;
-  const size_t x = (size_t)kKmTile * D * 2;
-  return w + x + 1024 /*align*/ + 24576 /*bias, scale, labels, order, list, histogram, merge, scores, rows*/;
+// Shared memory of the assignment kernel: three-term W, `stages` X tiles, barriers, per-warp
+// bias copies.
+__host__ inline size_t km_assign_smem(int D, int Np, int stages) {
+  return (size_t)3 * Np * D * 2 + (size_t)stages * kKmTile * D * 2 + 1024 /*align*/ + 256 /*barriers*/ +
+         (size_t)8 * 256 * 4 /*bias*/;
 }
 
-// Tiles per CTA: enough CTAs for about four per SM; each loads the weights once for its tiles.
-static int tiles_per_cta(const Layout& L) {
-  const int ntiles = (L.N + kKmTile - 1) / kKmTile;
-  int tpc = (int)(((long long)ntiles * L.BH + 148 * 4 - 1) / (148 * 4));
-  return tpc < 1 ? 1 : (tpc > 16 ? 16 : tpc);
+// Shared memory of the update kernel: labels and sorted order of a chunk of points, per-group
+// offsets and cursors.
+__host__ inline size_t km_update_smem(int D, int C) {
+  (void)D;
+  return (size_t)2 * kKmUpdChunk * 4 /*labels, order*/ + (size_t)(2 * C + 1) * 4;
+}
+
+__device__ __forceinline__ int km_tiles_per_head(const Layout& L) { return (L.N + kKmTile - 1) / kKmTile; }
+
+// Tile range [t0, t1) of CTA c of G over T = BH * tiles_per_head tiles.
+__device__ __forceinline__ void km_range(long long T, int G, int c, int& t0, int& t1) {
+  t0 = (int)(T * c / G);
+  t1 = (int)(T * (c + 1) / G);
 }
 
 template <bool kKeys>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kKmThreads, 1)
     kmeans_assign_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                            Layout L, int it, int tiles_per_cta) {
-  const int bh = blockIdx.y;
+                            Layout L, int it, int G, int S) {
   const int which = kKeys ? 0 : 1;
-  if (it >= L.stop_at[bh * 2 + which]) return;
-  const int D = L.d;
+  const int D = L.d, KB = D / 64;
   const int C = kKeys ? L.Ck : L.Cq;
   const int Np = kKeys ? L.Ckp : L.Cqp;
-  const int KB = D / 64;
-  const int tile0 = blockIdx.x * tiles_per_cta;
-  const int ntiles_head = (L.N + kKmTile - 1) / kKmTile;
-  const int ntile = min(tiles_per_cta, ntiles_head - tile0);
-  if (ntile <= 0) return;
+  const int Npr = (Np + 31) & ~31;  // columns per TMEM accumulator: the epilogue reads 32 at a time
+  const int tph = km_tiles_per_head(L);
+  int t0, t1;
+  km_range((long long)L.BH * tph, G, blockIdx.x, t0, t1);
+  if (t0 >= t1) return;  // uniform, before any barrier or TMEM use
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sW = sm;                                   // [3 terms][KB][Np rows][128 B]
-  uint8_t* sX = sW + (size_t)3 * Np * D * 2;          // [KB][128 rows][128 B]
-  float* sB = (float*)(sX + (size_t)kKmTile * D * 2);  // [256] bias
-  float* scl = sB + 256;                             // [128] sigma of each point
-  int* lab = (int*)(scl + kKmTile);                  // [128]
-  int* order = lab + kKmTile;                        // [128]
-  int* rlist = order + kKmTile;                      // [128] points to re-decide
-  int* hist = rlist + kKmTile;                       // [256] points per label in the tile
-  int* cursor = hist + 256;                          // [256] next slot per label
-  float* mb1 = (float*)(cursor + 256);               // [128] partial best / second / index
-  float* mb2 = mb1 + kKmTile;
-  int* mi1 = (int*)(mb2 + kKmTile);
-  double* bval = (double*)(mi1 + kKmTile);           // [128] score of the chosen group
-  double* xs64 = bval + kKmTile;                     // [8 warps][128] fp64 features
-  uint64_t* bars = (uint64_t*)(xs64 + 8 * 128);      // w_full, x_full, mma_done
-  uint32_t* tmem_slot = (uint32_t*)(bars + 3);
+  uint8_t* sX = sW + (size_t)3 * Np * D * 2;          // [S][KB][128 rows][128 B]
+  uint64_t* bars = (uint64_t*)(sX + (size_t)S * kKmTile * D * 2);
+  uint64_t* x_full = bars;                            // [S]
+  uint64_t* x_empty = bars + kKmMaxStages;            // [S]
+  uint64_t* acc_full = bars + 2 * kKmMaxStages;       // [2]
+  uint64_t* acc_empty = acc_full + 2;                 // [2]
+  uint64_t* w_full = acc_empty + 2;
+  uint64_t* w_empty = w_full + 1;
+  uint64_t* mma_done = w_empty + 1;
+  uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
+  float* sBias = (float*)(bars + 32);                 // [8 epilogue warps][256]
   __shared__ volatile int s_abort;
-  __shared__ float s_wmax, s_bmax;
-  __shared__ int s_nlist;
-  __shared__ double red[8];
+  __shared__ int s_rcnt;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const float* B32 = (kKeys ? L.kbias32 : L.qbias32) + (size_t)bh * C;
-  const float* WN = (kKeys ? L.kwnorm : L.qwnorm) + (size_t)bh * C;
-  const double* W64 = (kKeys ? L.kW64 : L.qU64) + (size_t)bh * C * D;
-  const double* B64 = (kKeys ? L.kbias64 : L.qbias64) + (size_t)bh * C;
-  const uint32_t tcols = km_tc_tmem_cols(Np);
-
+  const uint32_t tcols = km_tc_tmem_cols(2 * Npr);
   if (tid == 0) {
     s_abort = 0;
-    s_nlist = 0;
-    mbar_init(bars + 0, 1);
-    mbar_init(bars + 1, 1);
-    mbar_init(bars + 2, 1);
+    s_rcnt = 0;
+    for (int s = 0; s < S; ++s) {
+      mbar_init(x_full + s, 1);
+      mbar_init(x_empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full + b, 1);
+      mbar_init(acc_empty + b, 128);
+    }
+    mbar_init(w_full, 1);
+    mbar_init(w_empty, 1);
+    mbar_init(mma_done, 1);
     fence_mbar_init();
   }
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, tcols);
     tmem_relinquish();
   }
-  for (int j = tid; j < 256; j += blockDim.x) sB[j] = j < C ? B32[j] : INFINITY;
-  {
-    float wm = 0.f, bm = 0.f;
-    for (int j = tid; j < C; j += blockDim.x) {
-      wm = fmaxf(wm, WN[j]);
-      bm = fmaxf(bm, fabsf(B32[j]));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
-    }
-    __shared__ float pw[8], pb[8];
-    if (lane == 0) {
-      pw[warp] = wm;
-      pb[warp] = bm;
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (tid == 0) {
-      float a = 0.f, b = 0.f;
-      for (int w = 0; w < 8; ++w) {
-        a = fmaxf(a, pw[w]);
-        b = fmaxf(b, pb[w]);
-      }
-      s_wmax = a;
-      s_bmax = b;
-    }
-  }
-  const uint32_t tmem = *tmem_slot;
-  if (tid == 0) {  // weights: 3 terms x KB column blocks, one TMA box of Np rows each
-    mbar_arrive_expect_tx(bars + 0, (uint32_t)(3 * Np * D * 2));
-    for (int t = 0; t < 3; ++t)
-      for (int kb = 0; kb < KB; ++kb)
-        tma_load_2d(sW + ((size_t)t * KB + kb) * Np * 128, &tmW, bars + 0, kb * 64, t * L.BH * Np + bh * Np);
-  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // every role walks the same tiles: those of heads whose loop has not stopped
+  auto active = [&](int t) { return it < L.stop_at[(t / tph) * 2 + which]; };
 
-  const uint32_t idesc = idesc_bf16_f32(kKmTile, Np, 0, 0);
-  // |error of b - 2 sigma x.w| <= 2 sigma ||x|| ||w|| (3D + 8) 2^-23 (three-term split, fp32
-  // accumulation) + 2^-23 |b|; a factor-2 margin on top
-  const float u = 1.1920929e-7f;  // 2^-23
-  double jsum = 0.0;
-  int nref = 0;
-  for (int ti = 0; ti < ntile && !s_abort; ++ti) {
-    const int p0 = (tile0 + ti) * kKmTile;
-    const int np = min(kKmTile, L.N - p0);
-    if (tid == 0) {
-      mbar_arrive_expect_tx(bars + 1, (uint32_t)(kKmTile * D * 2));
-      for (int kb = 0; kb < KB; ++kb)
-        tma_load_2d(sX + (size_t)kb * kKmTile * 128, &tmX, bars + 1, kb * 64, bh * L.N + p0);
-      const bool ok = (ti > 0 || mbar_wait(bars + 0, 0, &s_abort)) && mbar_wait(bars + 1, ti & 1, &s_abort);
-      if (ok) {
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmX);
+      prefetch_tmap(&tmW);
+      int i = 0, wloads = 0, cur = -1;
+      for (int t = t0; t < t1; ++t) {
+        if (!active(t)) continue;
+        const int bh = t / tph;
+        if (bh != cur) {  // the head's W, once the MMAs on the previous head's W have completed
+          if (wloads > 0 && !mbar_wait(w_empty, (wloads - 1) & 1, &s_abort)) break;
+          mbar_arrive_expect_tx(w_full, (uint32_t)(3 * Np * D * 2));
+          for (int term = 0; term < 3; ++term)
+            for (int kb = 0; kb < KB; ++kb)
+              tma_load_2d(sW + ((size_t)term * KB + kb) * Np * 128, &tmW, w_full, kb * 64,
+                          term * L.BH * Np + bh * Np);
+          ++wloads;
+          cur = bh;
+        }
+        const int s = i % S;
+        if (i >= S && !mbar_wait(x_empty + s, ((i / S) - 1) & 1, &s_abort)) break;
+        mbar_arrive_expect_tx(x_full + s, (uint32_t)(kKmTile * D * 2));
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_2d(sX + ((size_t)s * KB + kb) * kKmTile * 128, &tmX, x_full + s, kb * 64,
+                      bh * L.N + (t % tph) * kKmTile);
+        ++i;
+      }
+      // never leave with copies in flight into this CTA's shared memory
+      for (int j = max(0, i - S); j < i; ++j) mbar_wait_drain(x_full + (j % S), (j / S) & 1);
+      if (wloads > 0) mbar_wait_drain(w_full, (wloads - 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kKmTile, Np, 0, 0);
+      int i = 0, wl = 0, cur = -1;
+      for (int t = t0; t < t1; ++t) {
+        if (!active(t)) continue;
+        const int bh = t / tph;
+        if (bh != cur) {
+          if (wl > 0) mma_commit(w_empty);  // the previous head's W is free once these complete
+          if (!mbar_wait(w_full, wl & 1, &s_abort)) break;
+          ++wl;
+          cur = bh;
+        }
+        const int s = i % S, b = i & 1;
+        if (!mbar_wait(x_full + s, (i / S) & 1, &s_abort)) break;
+        if (i >= 2 && !mbar_wait(acc_empty + b, ((i >> 1) - 1) & 1, &s_abort)) break;
         tc_fence_after();
         uint32_t acc = 0;
-        for (int wt = 0; wt < 3; ++wt)
+        for (int term = 0; term < 3; ++term)
           for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t xa = smem_u32(sX + (size_t)(ks >> 2) * kKmTile * 128) + (ks & 3) * 32;
-            const uint32_t wa = smem_u32(sW + ((size_t)wt * KB + (ks >> 2)) * Np * 128) + (ks & 3) * 32;
-            mma_ss(tmem, sdesc_sw128(xa, 16, 1024), sdesc_sw128(wa, 16, 1024), idesc, acc);
+            const uint32_t xa = smem_u32(sX + ((size_t)s * KB + (ks >> 2)) * kKmTile * 128) + (ks & 3) * 32;
+            const uint32_t wa = smem_u32(sW + ((size_t)term * KB + (ks >> 2)) * Np * 128) + (ks & 3) * 32;
+            mma_ss(tmem + b * Npr, sdesc_sw128(xa, 16, 1024), sdesc_sw128(wa, 16, 1024), idesc, acc);
             acc = 1;
           }
+        mma_commit(x_empty + s);
+        mma_commit(acc_full + b);
+        ++i;
       }
-      mma_commit(bars + 2);
+      // every MMA issued by this thread has completed before TMEM is released
+      mma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
     }
-    if (tid < kKmTile) scl[tid] = kKeys ? 1.f : (tid < np ? L.inv_rms[(size_t)bh * L.N + p0 + tid] : 0.f);
-    // epilogue: point q = tid % 128 (TMEM lane q); warps w and w+4 read alternate 32-column
-    // chunks of that lane's scores, then merge
-    const bool waited = mbar_wait(bars + 2, ti & 1, &s_abort);
-    if (__syncthreads_or(!waited)) break;  // uniform: every thread leaves or none does
-    tc_fence_after();
-    const int q = tid & 127, half = tid >> 7;
-    const float sq = scl[q];
-    float b1 = INFINITY, b2 = INFINITY;
-    int i1 = 0x7fffffff;
+  } else if (warp >= 4) {
+    // ================================================================ epilogue
+    const int e = (warp - 4) >> 2;          // warpgroup: the CTA's active tiles k with k % 2 == e
+    const int q = tid - 128 - 128 * e;      // point of the tile = TMEM lane
+    const int ew = warp - 4;
+    float* bias = sBias + ew * 256;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    for (int c0 = half * 32; c0 < Np; c0 += 64) {
-      uint32_t r[32];
-      tmem_ld32(tmem + lane_base + c0, r);  // c0 + 32 <= tcols: tcols is a power of two >= 32, >= Np
-      tmem_wait_ld();
+    int* labels = kKeys ? L.klabel : L.qlabel;
+    double* Jarr = kKeys ? L.kJ : L.qJ;
+    int* refined = kKeys ? L.krefined : L.qrefined;
+    const float u = 1.1920929e-7f;  // 2^-23
+    double jsum = 0.0;
+    int nref = 0, cur = -1;
+    float wmax = 0.f, bmax = 0.f;
+    auto flush = [&](int bh) {  // this warp's objective and re-decision count of head bh
+      const double js = warp_sum(jsum);
+      const int nr = (int)warp_sum((double)nref);
+      if (lane == 0) {
+        atomicAdd(Jarr + (size_t)bh * L.iters_cap + it, js);
+        if (nr) atomicAdd(refined + bh, nr);
+      }
+      jsum = 0.0;
+      nref = 0;
+    };
+    auto next_active = [&](int t) {
+      while (t < t1 && !active(t)) ++t;
+      return t;
+    };
+    // per-point scalars of a tile: 1/rms (queries) and the norm in the rounding bound
+    auto scalars = [&](int t, float& sq, float& xn) {
+      sq = 0.f;
+      xn = 0.f;
+      if (t >= t1) return;
+      const int bh = t / tph, p0 = (t % tph) * kKmTile;
+      if (q < L.N - p0) {
+        const size_t row = (size_t)bh * L.N + p0 + q;
+        sq = kKeys ? 1.f : L.inv_rms[row];
+        xn = kKeys ? L.knorm[row] : L.qxnorm[row];
+      }
+    };
+    int t = next_active(t0), k = 0;
+    if (e == 1 && t < t1) {
+      t = next_active(t + 1);
+      k = 1;
+    }
+    float sq, xn;
+    scalars(t, sq, xn);
+    while (t < t1) {
+      int tn = next_active(t + 1);
+      if (tn < t1) tn = next_active(tn + 1);  // this warpgroup's next tile
+      float nsq, nxn;
+      scalars(tn, nsq, nxn);                  // in flight while this tile is scanned
+      const int bh = t / tph;
+      if (bh != cur) {
+        if (cur >= 0) flush(cur);
+        cur = bh;
+        // the head's biases (this warp's copy) and the maxima of the bound.  Columns C .. Npr-1
+        // (padded groups, and columns the MMA does not write) get +inf: their score is +inf or
+        // nan, which never wins.
+        const float* B32 = (kKeys ? L.kbias32 : L.qbias32) + (size_t)bh * C;
+        const float* WN = (kKeys ? L.kwnorm : L.qwnorm) + (size_t)bh * C;
+        __syncwarp();  // every lane is done with the previous head's copy
+        float wm = 0.f, bm = 0.f;
+        for (int j = lane; j < Npr; j += 32) {
+          const float bj = j < C ? B32[j] : INFINITY;
+          bias[j] = bj;
+          if (j < C) {
+            bm = fmaxf(bm, fabsf(bj));
+            wm = fmaxf(wm, WN[j]);
+          }
+        }
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const int j = c0 + k;
-        if (j >= C) break;
-        const float sc = sB[j] - 2.f * sq * __uint_as_float(r[k]);
-        if (sc < b1 || (sc == b1 && j < i1)) {
-          b2 = b1;
-          b1 = sc;
-          i1 = j;
-        } else if (sc < b2) {
-          b2 = sc;
+        for (int o = 16; o > 0; o >>= 1) {
+          wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+        }
+        wmax = wm;
+        bmax = bm;
+        __syncwarp();
+      }
+      const int p0 = (t % tph) * kKmTile;
+      const bool valid = q < L.N - p0;
+      const size_t row = (size_t)bh * L.N + p0 + q;
+      const int b = k & 1;
+      // warp-uniform: the tcgen05.ld below needs every lane of the warp
+      const bool okw = mbar_wait(acc_full + b, (k >> 1) & 1, &s_abort);
+      if (!__all_sync(0xffffffffu, okw)) break;
+      tc_fence_after();
+      const float m2s = -2.f * sq;
+      float b1 = INFINITY, b2 = INFINITY;
+      int i1 = -1;
+      for (int c0 = 0; c0 < Npr; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + b * Npr + c0, r);  // b * Npr + c0 + 32 <= 2 Npr <= tcols
+        tmem_wait_ld();
+#pragma unroll
+        for (int kk = 0; kk < 32; ++kk) {
+          // ascending j and strict <: the lowest index of equal scores wins
+          const float sc = fmaf(m2s, __uint_as_float(r[kk]), bias[c0 + kk]);
+          const bool lt = sc < b1;
+          b2 = lt ? b1 : fminf(b2, sc);
+          i1 = lt ? c0 + kk : i1;
+          b1 = lt ? sc : b1;
         }
       }
-    }
-    if (half == 1) {
-      mb1[q] = b1;
-      mb2[q] = b2;
-      mi1[q] = i1;
-    }
-    __syncthreads();
-    if (half == 0) {
-      const float ob1 = mb1[q], ob2 = mb2[q];
-      const int oi1 = mi1[q];
-      if (ob1 < b1 || (ob1 == b1 && oi1 < i1)) {
-        b2 = fminf(b1, ob2);
-        b1 = ob1;
-        i1 = oi1;
-      } else {
-        b2 = fminf(b2, ob1);
+      tc_fence_before();
+      mbar_arrive(acc_empty + b);
+      if (valid) {
+        const float delta = 4.f * (3 * D + 8) * u * xn * wmax + 4.f * u * bmax;
+        const bool ref = !(b2 - b1 > 2.f * delta);
+        labels[row] = (i1 >= 0 && i1 < C) ? i1 : 0;  // non-finite scores never yield a bad label
+        jsum += (double)b1;
+        if (ref) {
+          const int slot = atomicAdd(&s_rcnt, 1);
+          L.rlist[(size_t)t0 * kKmTile + slot] = make_int2((int)row, __float_as_int(b1));
+          ++nref;
+        }
       }
-      const bool valid = q < np;
-      const size_t row = (size_t)bh * L.N + p0 + q;
-      const float xn = valid ? (kKeys ? L.knorm[row] : L.qxnorm[row]) : 0.f;
-      const float delta = 4.f * (3 * D + 8) * u * xn * s_wmax + 4.f * u * s_bmax;
-      const bool ref = valid && !(b2 - b1 > 2.f * delta);
-      lab[q] = (i1 >= 0 && i1 < C) ? i1 : 0;  // non-finite scores never yield a bad label
-      bval[q] = valid ? (double)b1 : 0.0;
-      if (ref) rlist[atomicAdd(&s_nlist, 1)] = q;
-      nref += ref ? 1 : 0;
+      t = tn;
+      k += 2;
+      sq = nsq;
+      xn = nxn;
     }
-    for (int j = tid; j < C; j += blockDim.x) hist[j] = 0;
+    if (cur >= 0) flush(cur);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0) {
+    L.rcnt[blockIdx.x] = s_rcnt;
+    if (s_abort) atomicCAS(L.status, kDevOk, kDevTimeout);
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tcols);
+  }
+}
+
+// Exact fp64 value of a bf16 given by its 16 bits (normal numbers by moving the exponent and
+// mantissa fields; zero, subnormals, inf and nan through fp32).
+__device__ __forceinline__ double bf16_bits_to_f64(uint32_t b) {
+  const uint32_t ex = b & 0x7F80u;
+  if (ex == 0u || ex == 0x7F80u) return (double)__uint_as_float(b << 16);
+  // sign to bit 63, exponent + (1023 - 127) to bits 62..52, 7 mantissa bits to 51..45
+  const uint32_t hi = ((b & 0x8000u) << 16) | (((b & 0x7FFFu) << 13) + 0x38000000u);
+  return __hiloint2double((int)hi, 0);
+}
+
+// fp64 re-decision of the points the assignment listed: block (c, y) takes every
+// kKmRedecideSplit-th entry of CTA range c's list, one warp per point; the label and the
+// objective (its fp64 score minus the tentative fp32 one) are corrected in place.
+constexpr int kKmRedecideSplit = 4;
+
+template <bool kKeys>
+__global__ void __launch_bounds__(256) kmeans_redecide_kernel(const __nv_bfloat16* __restrict__ X, Layout L, int it,
+                                                              int G) {
+  __shared__ double xs_all[8][128];
+  const int D = L.d, C = kKeys ? L.Ck : L.Cq;
+  const int tph = km_tiles_per_head(L);
+  int t0, t1;
+  km_range((long long)L.BH * tph, G, blockIdx.x, t0, t1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nlist = min(max(L.rcnt[blockIdx.x], 0), max(t1 - t0, 0) * kKmTile);  // never past the segment
+  const int2* list = L.rlist + (size_t)t0 * kKmTile;
+  int* labels = kKeys ? L.klabel : L.qlabel;
+  double* Jarr = kKeys ? L.kJ : L.qJ;
+  double* xs = xs_all[warp];
+  for (int li = blockIdx.y * 8 + warp; li < nlist; li += 8 * kKmRedecideSplit) {
+    const int2 en = list[li];
+    const int row = en.x, bh = row / L.N;
+    for (int a = lane; a < D; a += 32) xs[a] = (double)__bfloat162float(X[(size_t)row * D + a]);
+    __syncwarp();
+    int best;
+    double bv;
+    const double* W64 = (kKeys ? L.kW64 : L.qU64) + (size_t)bh * C * D;
+    const double* B64 = (kKeys ? L.kbias64 : L.qbias64) + (size_t)bh * C;
+    redecide_fp64<kKeys>(L, bh, xs, D, C, W64, B64, best, bv);
+    if (lane == 0) {
+      labels[row] = best;
+      atomicAdd(Jarr + (size_t)bh * L.iters_cap + it, bv - (double)__int_as_float(en.y));
+    }
+    __syncwarp();
+  }
+}
+
+template <bool kKeys>
+__global__ void __launch_bounds__(kKmUpdThreads, 1)
+    kmeans_update_kernel(const __nv_bfloat16* __restrict__ X, Layout L, int it, int G) {
+  const int which = kKeys ? 0 : 1;
+  const int D = L.d;
+  const int C = kKeys ? L.Ck : L.Cq;
+  const int tph = km_tiles_per_head(L);
+  int t0, t1;
+  km_range((long long)L.BH * tph, G, blockIdx.x, t0, t1);
+  if (t0 >= t1) return;
+
+  extern __shared__ uint8_t smem_raw[];
+  int* lab = (int*)smem_raw;                   // [kKmUpdChunk] label of each point of the chunk
+  int* order = lab + kKmUpdChunk;              // [kKmUpdChunk] chunk points sorted by label
+  int* offs = order + kKmUpdChunk;             // [C + 1] start of each label's run
+  int* cursor = offs + (C + 1);                // [C] histogram, then next slot per label
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int* labels = kKeys ? L.klabel : L.qlabel;
+  double* sums_all = kKeys ? L.ksum : L.qsum;
+  int* counts_all = kKeys ? L.kcount : L.qcount;
+  const int octs = D / 8;  // threads per row: eight dimensions (16 bytes) each
+  int t = t0;
+  while (t < t1) {
+    const int bh = t / tph;
+    if (it >= L.stop_at[bh * 2 + which]) {  // this head's loop has stopped: skip its tiles
+      t = (bh + 1) * tph;
+      continue;
+    }
+    // chunk: tiles [t, te) of head bh, at most kKmUpdChunk points
+    const int te = min(min(t1, (bh + 1) * tph), t + kKmUpdChunk / kKmTile);
+    const int p_lo = (t % tph) * kKmTile;
+    const int p_hi = min(L.N, (te - 1) % tph * kKmTile + kKmTile);
+    const int n = p_hi - p_lo;
+    const size_t row0 = (size_t)bh * L.N + p_lo;
+    for (int j = tid; j < C; j += kKmUpdThreads) cursor[j] = 0;
     __syncthreads();
-    // fp64 re-decision over every group: one warp per listed point
-    const int nlist = s_nlist;
-    for (int li = warp; li < nlist; li += 8) {
-      const int p = rlist[li];
-      double* xs = xs64 + warp * 128;
-      for (int a = lane; a < D; a += 32) {
-        const int kb = a >> 6, w = a & 63;
-        const uint32_t off = (uint32_t)p * 128 + ((((w >> 3) ^ (p & 7)) << 4) | ((w & 7) << 1));
-        xs[a] = (double)__bfloat162float(*(const __nv_bfloat16*)(sX + (size_t)kb * kKmTile * 128 + off));
+    // histogram: lanes holding the same label add once (labels are spatially coherent)
+    for (int i0 = 0; i0 < n; i0 += kKmUpdThreads) {
+      const int i = i0 + tid;
+      int g = -1;
+      if (i < n) {
+        g = labels[row0 + i];
+        g = (g >= 0 && g < C) ? g : 0;
+        lab[i] = g;
       }
-      __syncwarp();
-      int best;
-      double bv;
-      redecide_fp64<kKeys>(L, bh, xs, D, C, W64, B64, best, bv);
-      if (lane == 0) {
-        lab[p] = best;
-        bval[p] = bv;
+      const unsigned act = __ballot_sync(0xffffffffu, i < n);
+      if (i < n) {
+        const unsigned same = __match_any_sync(act, g);
+        if (lane == __ffs(same) - 1) atomicAdd(&cursor[g], __popc(same));
       }
-      __syncwarp();
     }
     __syncthreads();
-    if (tid < np) {
-      ((kKeys ? L.klabel : L.qlabel) + (size_t)bh * L.N)[p0 + tid] = lab[tid];
-      jsum += bval[tid];
-      atomicAdd(&hist[lab[tid]], 1);
-    }
-    tc_fence_before();
-    __syncthreads();
-    // counting sort of the tile's points by label (the order inside a label is irrelevant:
-    // each run's fp64 partial sums of exact products are exact)
-    if (warp == 0) {
+    if (warp == 0) {  // exclusive prefix over the groups, and the counts
       int run = 0;
       for (int c0 = 0; c0 < C; c0 += 32) {
         const int j = c0 + lane;
-        const int v = j < C ? hist[j] : 0;
+        const int v = j < C ? cursor[j] : 0;
         int x = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const int y = __shfl_up_sync(0xffffffffu, x, o);
           if (lane >= o) x += y;
         }
-        if (j < C) cursor[j] = run + x - v;
+        if (j < C) {
+          offs[j] = run + x - v;
+          cursor[j] = run + x - v;
+          if (v) atomicAdd(counts_all + (size_t)bh * C + j, v);
+        }
         run += __shfl_sync(0xffffffffu, x, 31);
       }
+      if (lane == 0) offs[C] = run;
     }
     __syncthreads();
-    int* counts = (kKeys ? L.kcount : L.qcount) + (size_t)bh * C;
-    for (int j = tid; j < C; j += blockDim.x)
-      if (hist[j]) atomicAdd(counts + j, hist[j]);
-    if (tid < np) order[atomicAdd(&cursor[lab[tid]], 1)] = tid;
-    __syncthreads();
-    double* sums = (kKeys ? L.ksum : L.qsum) + (size_t)bh * C * D;
-    const int nparts = 256 / D;
-    {
-      const int a = tid % D, part = tid / D;
-      const int q0 = part * np / nparts, q1 = (part + 1) * np / nparts;
-      const int kb = a >> 6, w = a & 63;
-      const uint8_t* colbase = sX + (size_t)kb * kKmTile * 128;
-      double acc = 0.0;
-      for (int qq = q0; qq < q1; ++qq) {
-        const int p = order[qq];
-        const uint32_t off = (uint32_t)p * 128 + ((((w >> 3) ^ (p & 7)) << 4) | ((w & 7) << 1));
-        acc += (double)__bfloat162float(*(const __nv_bfloat16*)(colbase + off)) * (double)scl[p];
-        if (qq == q1 - 1 || lab[order[qq + 1]] != lab[p]) {
-          atomicAdd(sums + (size_t)lab[p] * D + a, acc);
-          acc = 0.0;
-        }
+    // scatter: lanes with the same label take consecutive slots from one atomic
+    for (int i0 = 0; i0 < n; i0 += kKmUpdThreads) {
+      const int i = i0 + tid;
+      const unsigned act = __ballot_sync(0xffffffffu, i < n);
+      if (i < n) {
+        const int g = lab[i];
+        const unsigned same = __match_any_sync(act, g);
+        const int leader = __ffs(same) - 1;
+        int base = 0;
+        if (lane == leader) base = atomicAdd(&cursor[g], __popc(same));
+        base = __shfl_sync(same, base, leader);
+        order[base + __popc(same & ((1u << lane) - 1))] = i;
       }
     }
-    if (tid == 0) s_nlist = 0;
-    tc_fence_before();
     __syncthreads();
-  }
-  const double js = block_sum(jsum, red);
-  const double nr = block_sum((double)nref, red);
-  if (tid == 0) {
-    atomicAdd((kKeys ? L.kJ : L.qJ) + (size_t)bh * L.iters_cap + it, js);
-    if (nr > 0.0) atomicAdd((kKeys ? L.krefined : L.qrefined) + bh, (int)nr);
-    if (s_abort) {
-      atomicCAS(L.status, kDevOk, kDevTimeout);
-      // never leave with copies in flight into this CTA's shared memory
-      mbar_wait_drain(bars + 0, 0);
-      for (int ti = 0; ti < ntile; ++ti) mbar_wait_drain(bars + 1, ti & 1);
+    // accumulation: item = (group, eight dimensions); consecutive threads read consecutive
+    // 16-byte pieces of the same rows; each item's run is summed in fp64 registers
+    const __nv_bfloat16* Xc = X + row0 * D;
+    const double* sig = L.inv_rms64 + row0;
+    double* sums = sums_all + (size_t)bh * C * D;
+    for (int item = tid; item < C * octs; item += kKmUpdThreads) {
+      const int g = item / octs, oc = item % octs;
+      const int q0 = offs[g], q1 = offs[g + 1];
+      if (q0 == q1) continue;
+      double r[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) r[k] = 0.0;
+      int q = q0;
+      for (; q + 4 <= q1; q += 4) {
+        int pidx[4];
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) pidx[u] = order[q + u];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = *(const uint4*)(Xc + (size_t)pidx[u] * D + 8 * oc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          if constexpr (kKeys) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              r[2 * k] += bf16_bits_to_f64(w[k] & 0xFFFFu);
+              r[2 * k + 1] += bf16_bits_to_f64(w[k] >> 16);
+            }
+          } else {
+            const double sg = sig[pidx[u]];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              r[2 * k] = fma(bf16_bits_to_f64(w[k] & 0xFFFFu), sg, r[2 * k]);
+              r[2 * k + 1] = fma(bf16_bits_to_f64(w[k] >> 16), sg, r[2 * k + 1]);
+            }
+          }
+        }
+      }
+      for (; q < q1; ++q) {
+        const int p = order[q];
+        const uint4 v = *(const uint4*)(Xc + (size_t)p * D + 8 * oc);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        const double sg = kKeys ? 1.0 : sig[p];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          r[2 * k] = fma(bf16_bits_to_f64(w[k] & 0xFFFFu), sg, r[2 * k]);
+          r[2 * k + 1] = fma(bf16_bits_to_f64(w[k] >> 16), sg, r[2 * k + 1]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) atomicAdd(sums + (size_t)g * D + 8 * oc + k, r[k]);
     }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, tcols);
+    __syncthreads();  // lab / order / offs are rewritten by the next chunk
+    t = te;
   }
 }
 
@@ -420,6 +632,7 @@ __global__ void __launch_bounds__(128, 1)
         const double ms = (double)qf;
         const float inv = (float)(1.0 / sqrt(ms + 1e-12));
         L.inv_rms[row] = inv;
+        L.inv_rms64[row] = 1.0 / sqrt(ms + 1e-12);
         L.qxnorm[row] = sqrtf(nn) * inv;
         tot += (double)L.Ck * ms / (ms + 1e-12);
       }
@@ -444,34 +657,85 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+
 // ----------------------------------------------------------------------------------- host
+static int km_stages(const Layout& L, int Np) {
+  const size_t budget = 227 * 1024;
+  const size_t fixed = km_assign_smem(L.d, Np, 0);
+  if (fixed >= budget) return 0;
+  const size_t per = (size_t)kKmTile * L.d * 2;
+  return (int)std::min<size_t>(kKmMaxStages, (budget - fixed) / per);
+}
+
 bool km_tc_supported(const Layout& L, bool keys) {
   if (L.dtype != SPARSEPR_BF16) return false;
   const int Np = keys ? L.Ckp : L.Cqp;
-  return Np <= 256 && km_tc_smem(L.d, Np) <= 227 * 1024;
+  const int C = keys ? L.Ck : L.Cq;
+  return Np <= 256 && km_stages(L, Np) >= 2 && km_update_smem(L.d, C) <= 227 * 1024;
 }
 
-sparsepr_status launch_kmeans_assign_tc(const Layout& L, bool keys, const void* X, int it, cudaStream_t st) {
+// CTAs of both k-means kernels: as many as fit the device at once (so the static ranges run in
+// one wave), at most one per tile.
+int km_tc_grid(const Layout& L, bool keys) {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  const int Np = keys ? L.Ckp : L.Cqp;
+  const int S = km_stages(L, Np);
+  const size_t smem = km_assign_smem(L.d, Np, S);
+  int occ = 1;
+  if (keys) {
+    cudaFuncSetAttribute(kmeans_assign_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kmeans_assign_tc_kernel<true>, kKmThreads, smem);
+  } else {
+    cudaFuncSetAttribute(kmeans_assign_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kmeans_assign_tc_kernel<false>, kKmThreads, smem);
+  }
+  occ = std::max(1, std::min(occ, 2));
+  const long long T = (long long)L.BH * ((L.N + kKmTile - 1) / kKmTile);
+  return (int)std::min<long long>(T, (long long)sms * occ);
+}
+
+sparsepr_status launch_kmeans_iteration_tc(const Layout& L, bool keys, const void* X, int it, int G,
+                                           cudaStream_t st) {
   CUtensorMap mX, mW;
   const int D = L.d;
   const int Np = keys ? L.Ckp : L.Cqp;
+  const int C = keys ? L.Ck : L.Cq;
   const void* wbase = keys ? (const void*)L.kWb : (const void*)L.qWb;
   if (!make_tmap_bf16(&mX, X, (long long)L.BH * L.N, D, kKmTile) ||
       !make_tmap_bf16(&mW, wbase, 3LL * L.BH * Np, D, Np))
     return SPARSEPR_ERR_CUDA;
-  const size_t smem = km_tc_smem(D, Np);
-  const int tpc = tiles_per_cta(L);
-  const int ntiles = (L.N + kKmTile - 1) / kKmTile;
-  const dim3 grid((ntiles + tpc - 1) / tpc, L.BH);
+  const int S = km_stages(L, Np);
+  const size_t smem_a = km_assign_smem(D, Np, S);
+  const size_t smem_u = km_update_smem(D, C);
+  const __nv_bfloat16* Xb = (const __nv_bfloat16*)X;
   if (keys) {
-    cudaFuncSetAttribute(kmeans_assign_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    launch(kmeans_assign_tc_kernel<true>, grid, dim3(256), smem, st, mX, mW, L, it, tpc);
+    cudaFuncSetAttribute(kmeans_assign_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
+    cudaFuncSetAttribute(kmeans_update_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_u);
+    launch(kmeans_assign_tc_kernel<true>, G, kKmThreads, smem_a, st, mX, mW, L, it, G, S);
+    launch(kmeans_redecide_kernel<true>, dim3(G, kKmRedecideSplit), 256, 0, st, Xb, L, it, G);
+    launch(kmeans_update_kernel<true>, G, kKmUpdThreads, smem_u, st, Xb, L, it, G);
   } else {
-    cudaFuncSetAttribute(kmeans_assign_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    launch(kmeans_assign_tc_kernel<false>, grid, dim3(256), smem, st, mX, mW, L, it, tpc);
+    cudaFuncSetAttribute(kmeans_assign_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
+    cudaFuncSetAttribute(kmeans_update_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_u);
+    launch(kmeans_assign_tc_kernel<false>, G, kKmThreads, smem_a, st, mX, mW, L, it, G, S);
+    launch(kmeans_redecide_kernel<false>, dim3(G, kKmRedecideSplit), 256, 0, st, Xb, L, it, G);
+    launch(kmeans_update_kernel<false>, G, kKmUpdThreads, smem_u, st, Xb, L, it, G);
   }
   SPR_LAUNCH_CHECK();
   return SPARSEPR_OK;
+}
+
+// Tiles per CTA of the row quadratic forms: enough CTAs for about four per SM.
+static int tiles_per_cta(const Layout& L) {
+  const int ntiles = (L.N + kKmTile - 1) / kKmTile;
+  int tpc = (int)(((long long)ntiles * L.BH + 148 * 4 - 1) / (148 * 4));
+  return tpc < 1 ? 1 : (tpc > 16 ? 16 : tpc);
 }
 
 sparsepr_status launch_rowqf_tc(const Layout& L, int which, const void* X, cudaStream_t st) {

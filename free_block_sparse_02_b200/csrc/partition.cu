@@ -19,6 +19,8 @@
 // ties far below the fp32 resolution.  Group sums are fp64.
 #include <math.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "kmeans.cuh"
@@ -26,19 +28,43 @@
 namespace sparsepr {
 
 // ------------------------------------------------------------------------------------------
-// a1 + a2 prologue: M = Q_s^T Q_s / d (fp64, exact products) per head.
+// a1 + a2 prologue: M = Q_s^T Q_s / d (fp64, exact products, summed over the samples in order)
+// per head.  Block (bh, y) computes rows [16 y, 16 y + 16) of M; the sampled rows are staged in
+// shared memory (fp32, exact for bf16 and fp32 inputs) 64 at a time.
 // ------------------------------------------------------------------------------------------
+constexpr int kMetricRows = 16;
+constexpr int kMetricChunk = 64;
+
 template <typename T>
-__global__ void metric_kernel(Layout L, const T* __restrict__ Q) {
-  const int bh = blockIdx.x, a = blockIdx.y, b = threadIdx.x;
-  if (b >= L.d) return;
-  const T* q = Q + (size_t)bh * L.N * L.d;
-  double acc = 0.0;
-  for (int i = 0; i < L.s; ++i) {
-    const long long row = ((2LL * i + 1) * L.N) / (2LL * L.s);
-    acc += (double)to_f32(q[row * L.d + a]) * (double)to_f32(q[row * L.d + b]);
+__global__ void __launch_bounds__(256) metric_kernel(Layout L, const T* __restrict__ Q) {
+  __shared__ float qs[kMetricChunk][128];
+  const int bh = blockIdx.x, a0 = blockIdx.y * kMetricRows, d = L.d, tid = threadIdx.x;
+  const int b = tid % d, lanes_per_b = 256 / d, r0 = tid / d;
+  constexpr int kMaxOut = kMetricRows / 2;  // d = 128: 8 rows per thread; d = 64: 4
+  const int nout = kMetricRows / lanes_per_b;
+  const T* q = Q + (size_t)bh * L.N * d;
+  double acc[kMaxOut];
+#pragma unroll
+  for (int k = 0; k < kMaxOut; ++k) acc[k] = 0.0;
+  for (int i0 = 0; i0 < L.s; i0 += kMetricChunk) {
+    const int ni = min(kMetricChunk, L.s - i0);
+    __syncthreads();
+    for (int e = tid; e < ni * d; e += 256) {
+      const int i = e / d, c = e % d;
+      const long long row = ((2LL * (i0 + i) + 1) * L.N) / (2LL * L.s);
+      qs[i][c] = to_f32(q[row * d + c]);
+    }
+    __syncthreads();
+    for (int i = 0; i < ni; ++i) {
+      const double xb = (double)qs[i][b];
+#pragma unroll
+      for (int k = 0; k < kMaxOut; ++k)
+        if (k < nout) acc[k] += (double)qs[i][a0 + r0 + k * lanes_per_b] * xb;
+    }
   }
-  L.M[((size_t)bh * L.d + a) * L.d + b] = acc / L.d;
+#pragma unroll
+  for (int k = 0; k < kMaxOut; ++k)
+    if (k < nout) L.M[((size_t)bh * d + a0 + r0 + k * lanes_per_b) * d + b] = acc[k] / d;
 }
 
 // fp64 [BH, d, d] matrices split into three bf16 planes (tensor-core operands).
@@ -110,6 +136,7 @@ __global__ void __launch_bounds__(256) rowqf_simt_kernel(Layout L, const T* __re
       const double ms = (double)part;
       const float inv = (float)(1.0 / sqrt(ms + 1e-12));
       L.inv_rms[row] = inv;
+      L.inv_rms64[row] = 1.0 / sqrt(ms + 1e-12);
       L.qxnorm[row] = sqrtf(nn) * inv;
       contrib = (double)L.Ck * ms / (ms + 1e-12);
     }
@@ -239,94 +266,199 @@ __device__ __forceinline__ bool km_should_stop(const double* J, int it, int iter
   return false;
 }
 
+constexpr int kPrepGroups = 8;  // groups per block of the centroid-update kernels
+
+// Sums of kPrepGroups values per thread over the block (128 threads): out[g] for g < n.
+__device__ __forceinline__ void block_sums8(const double (&v)[kPrepGroups], double* red /*[8][4]*/, double* out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int g = 0; g < kPrepGroups; ++g) {
+    const double x = warp_sum(v[g]);
+    if (lane == 0) red[g * 4 + warp] = x;
+  }
+  __syncthreads();
+  if (threadIdx.x < kPrepGroups) {
+    const double* r = red + threadIdx.x * 4;
+    out[threadIdx.x] = (r[0] + r[1]) + (r[2] + r[3]);
+  }
+  __syncthreads();
+}
+
+constexpr int kPrepRows = 128;  // rows of M or C staged in shared memory at a time (fp64)
+
+// Rows [r0, r0 + nr) of a row-major fp64 matrix with `cols` columns into shared memory, all
+// threads of the block loading together (coalesced, many loads in flight).
+__device__ __forceinline__ void stage_rows(double* dst, const double* __restrict__ src, int r0, int nr, int cols) {
+  const int n = nr * cols;
+  const double* s = src + (size_t)r0 * cols;
+  for (int e = threadIdx.x; e < n; e += blockDim.x) dst[e] = s[e];
+}
+
+// Keys, kPrepGroups groups per block (grid BH x ceil(C_k / 8), thread a = dimension):
+// c_j <- sum_j / n_j (groups that received points), the stop test, then W_j = M c_j (M staged in
+// shared memory, symmetric: thread a reads column a), bias_j = c_j^T W_j, ||W_j||, and the sums
+// zeroed.  Dynamic shared memory: min(d, kPrepRows) rows of M.
 __global__ void __launch_bounds__(128) kprep_kernel(Layout L, int it, int iters) {
-  __shared__ double c[128];
-  __shared__ double red[4];
-  const int bh = blockIdx.x, j = blockIdx.y, a = threadIdx.x, d = L.d;
+  extern __shared__ double Ms[];
+  __shared__ double c[kPrepGroups][128];
+  __shared__ double red[kPrepGroups * 4], bias_s[kPrepGroups], wn_s[kPrepGroups];
+  const int bh = blockIdx.x, j0 = blockIdx.y * kPrepGroups, a = threadIdx.x, d = L.d;
   if (it > L.stop_at[bh * 2 + 0]) return;
-  double* cj = L.kcent + ((size_t)bh * L.Ck + j) * d;
-  const size_t gj = (size_t)bh * L.Ck + j;
-  if (it > 0) {
-    const int cnt = L.kcount[gj];
-    if (cnt > 0 && a < d) cj[a] = L.ksum[gj * d + a] / (double)cnt;
+  const int ng = min(kPrepGroups, L.Ck - j0);
+  const size_t g0 = (size_t)bh * L.Ck + j0;
+  for (int g = 0; g < ng; ++g) {
+    double* cj = L.kcent + (g0 + g) * d;
+    if (it > 0) {
+      const int cnt = L.kcount[g0 + g];
+      if (cnt > 0 && a < d) cj[a] = L.ksum[(g0 + g) * d + a] / (double)cnt;
+    }
+    if (a < d) c[g][a] = cj[a];
   }
   if (km_should_stop(L.kJ + (size_t)bh * L.iters_cap, it, iters, L.km_tol)) {
-    if (a == 0 && j == 0) L.stop_at[bh * 2 + 0] = it;
+    if (a == 0 && blockIdx.y == 0) L.stop_at[bh * 2 + 0] = it;
     return;
   }
-  if (a < d) c[a] = cj[a];
-  __syncthreads();
-  double w = 0.0;
-  if (a < d) {
-    const double* Mr = L.M + ((size_t)bh * d + a) * d;
-    for (int b = 0; b < d; ++b) w += Mr[b] * c[b];
-    L.kW64[gj * d + a] = w;
-    L.kW32[gj * d + a] = (float)w;
-    L.ksum[gj * d + a] = 0.0;
-    split3(w, L.kWb, (size_t)L.BH * L.Ckp * d, ((size_t)bh * L.Ckp + j) * d + a);
+  double w[kPrepGroups];
+#pragma unroll
+  for (int g = 0; g < kPrepGroups; ++g) w[g] = 0.0;
+  const double* M = L.M + (size_t)bh * d * d;
+  for (int b0 = 0; b0 < d; b0 += kPrepRows) {
+    const int nb = min(kPrepRows, d - b0);
+    __syncthreads();
+    stage_rows(Ms, M, b0, nb, d);
+    __syncthreads();
+    if (a < d)
+      for (int bb = 0; bb < nb; ++bb) {
+        const double m = Ms[bb * d + a];  // M[b][a] = M[a][b]
+#pragma unroll
+        for (int g = 0; g < kPrepGroups; ++g) w[g] += m * c[g][b0 + bb];
+      }
   }
-  const double bias = block_sum(a < d ? c[a] * w : 0.0, red);
-  const double wn = block_sum(a < d ? w * w : 0.0, red);
-  if (a == 0) {
-    L.kbias64[gj] = bias;
-    L.kbias32[gj] = (float)bias;
+  double cb[kPrepGroups], wn[kPrepGroups];
+#pragma unroll
+  for (int g = 0; g < kPrepGroups; ++g) {
+    const bool on = a < d && g < ng;
+    cb[g] = on ? c[g][a] * w[g] : 0.0;
+    wn[g] = on ? w[g] * w[g] : 0.0;
+    if (on) {
+      const size_t gj = g0 + g;
+      L.kW64[gj * d + a] = w[g];
+      L.kW32[gj * d + a] = (float)w[g];
+      L.ksum[gj * d + a] = 0.0;
+      split3(w[g], L.kWb, (size_t)L.BH * L.Ckp * d, ((size_t)bh * L.Ckp + j0 + g) * d + a);
+    }
+  }
+  block_sums8(cb, red, bias_s);
+  block_sums8(wn, red, wn_s);
+  if (a < ng) {
+    const size_t gj = g0 + a;
+    L.kbias64[gj] = bias_s[a];
+    L.kbias32[gj] = (float)bias_s[a];
     L.kcount[gj] = 0;
-    L.kwnorm[gj] = (float)sqrt(wn);
+    L.kwnorm[gj] = (float)sqrt(wn_s[a]);
   }
 }
 
+// Queries, kPrepGroups groups per block (grid BH x ceil(C_q / 8)):
+// nu_g <- C S_g / (sqrt(d) n_g) (the mean normalised response of the members), the stop test,
+// then u_g = C^T nu_g / sqrt(d), bias ||nu_g||^2, ||u_g||, and the sums zeroed.  The key-group
+// centroids C are staged in shared memory kPrepRows rows at a time.
+// Dynamic shared memory: kPrepGroups * C_k doubles (nu of the block's groups), then
+// min(C_k, kPrepRows) rows of C.
 __global__ void __launch_bounds__(128) qprep_kernel(Layout L, int it, int iters) {
-  __shared__ double Sv[128];
-  __shared__ double nuv[kMaxGroups];
-  __shared__ double red[4];
-  const int bh = blockIdx.x, g = blockIdx.y, d = L.d, Ck = L.Ck, tid = threadIdx.x;
+  extern __shared__ double qsm[];
+  __shared__ double Sv[kPrepGroups][128];
+  __shared__ double red[kPrepGroups * 4], nn_s[kPrepGroups], un_s[kPrepGroups];
+  __shared__ int cnt_s[kPrepGroups];
+  const int bh = blockIdx.x, g0i = blockIdx.y * kPrepGroups, d = L.d, Ck = L.Ck, tid = threadIdx.x;
   if (it > L.stop_at[bh * 2 + 1]) return;
-  const size_t gg = (size_t)bh * L.Cq + g;
-  double* nu = L.qcent + gg * Ck;
+  double* nus = qsm;                             // [kPrepGroups][Ck]
+  double* Cs = qsm + (size_t)kPrepGroups * Ck;   // [kPrepRows][d]
+  const int ng = min(kPrepGroups, L.Cq - g0i);
+  const size_t g0 = (size_t)bh * L.Cq + g0i;
   const double* C = L.kcent + (size_t)bh * Ck * d;
   const double rsd = 1.0 / sqrt((double)d);
-  if (it > 0) {  // nu_g = C S_g / (sqrt(d) n_g): the mean normalised response of the members
-    const int cnt = L.qcount[gg];
-    if (cnt > 0) {
-      if (tid < d) Sv[tid] = L.qsum[gg * d + tid] / (double)cnt;
+  if (tid < kPrepGroups) cnt_s[tid] = (it > 0 && tid < ng) ? L.qcount[g0 + tid] : 0;
+  __syncthreads();
+  if (it > 0) {  // nu_g = C S_g / (sqrt(d) n_g) for the groups that received points
+#pragma unroll
+    for (int g = 0; g < kPrepGroups; ++g)
+      if (tid < d) Sv[g][tid] = cnt_s[g] > 0 ? L.qsum[(g0 + g) * d + tid] / (double)cnt_s[g] : 0.0;
+    for (int jc = 0; jc < Ck; jc += kPrepRows) {
+      const int nj = min(kPrepRows, Ck - jc);
       __syncthreads();
-      for (int j = tid; j < Ck; j += blockDim.x) {
-        double acc = 0.0;
-        for (int a = 0; a < d; ++a) acc += C[(size_t)j * d + a] * Sv[a];
-        nu[j] = acc * rsd;
+      stage_rows(Cs, C, jc, nj, d);
+      __syncthreads();
+      for (int jj = tid; jj < nj; jj += blockDim.x) {
+        double acc[kPrepGroups];
+#pragma unroll
+        for (int g = 0; g < kPrepGroups; ++g) acc[g] = 0.0;
+        const double* cj = Cs + (size_t)jj * d;
+        int aa = jj % d;  // rotated start: the lanes of a warp read different banks
+        for (int a = 0; a < d; ++a) {
+          const double x = cj[aa];
+#pragma unroll
+          for (int g = 0; g < kPrepGroups; ++g) acc[g] += x * Sv[g][aa];
+          aa = aa + 1 == d ? 0 : aa + 1;
+        }
+#pragma unroll
+        for (int g = 0; g < kPrepGroups; ++g)
+          if (g < ng && cnt_s[g] > 0) L.qcent[(g0 + g) * Ck + jc + jj] = acc[g] * rsd;
       }
     }
   }
   if (km_should_stop(L.qJ + (size_t)bh * L.iters_cap, it, iters, L.km_tol)) {
-    if (tid == 0 && g == 0) L.stop_at[bh * 2 + 1] = it;
+    if (tid == 0 && blockIdx.y == 0) L.stop_at[bh * 2 + 1] = it;
     return;
   }
   __syncthreads();
-  double nn = 0.0;
-  for (int j = tid; j < Ck; j += blockDim.x) {
-    const double v = nu[j];
-    nuv[j] = v;
-    nn += v * v;
+  double nn[kPrepGroups];
+#pragma unroll
+  for (int g = 0; g < kPrepGroups; ++g) nn[g] = 0.0;
+  for (int j = tid; j < Ck; j += blockDim.x)
+#pragma unroll
+    for (int g = 0; g < kPrepGroups; ++g) {
+      const double v = g < ng ? L.qcent[(g0 + g) * Ck + j] : 0.0;
+      nus[g * Ck + j] = v;
+      nn[g] += v * v;
+    }
+  block_sums8(nn, red, nn_s);  // (its barriers also publish nus)
+  // u_g = C^T nu_g / sqrt(d): thread = dimension, rows of C from shared memory
+  double uu[kPrepGroups], un[kPrepGroups];
+#pragma unroll
+  for (int g = 0; g < kPrepGroups; ++g) uu[g] = 0.0;
+  for (int jc = 0; jc < Ck; jc += kPrepRows) {
+    const int nj = min(kPrepRows, Ck - jc);
+    __syncthreads();
+    stage_rows(Cs, C, jc, nj, d);
+    __syncthreads();
+    if (tid < d)
+      for (int jj = 0; jj < nj; ++jj) {
+        const double x = Cs[(size_t)jj * d + tid];
+#pragma unroll
+        for (int g = 0; g < kPrepGroups; ++g) uu[g] += x * nus[g * Ck + jc + jj];
+      }
   }
-  nn = block_sum(nn, red);
-  // u_g = C^T nu_g / sqrt(d)
-  double un = 0.0;
-  if (tid < d) {
-    double acc = 0.0;
-    for (int j = 0; j < Ck; ++j) acc += C[(size_t)j * d + tid] * nuv[j];
-    acc *= rsd;
-    L.qU64[gg * d + tid] = acc;
-    L.qU32[gg * d + tid] = (float)acc;
-    split3(acc, L.qWb, (size_t)L.BH * L.Cqp * d, ((size_t)bh * L.Cqp + g) * d + tid);
-    L.qsum[gg * d + tid] = 0.0;
-    un = acc * acc;
+#pragma unroll
+  for (int g = 0; g < kPrepGroups; ++g) {
+    const bool on = tid < d && g < ng;
+    const double u = uu[g] * rsd;
+    un[g] = on ? u * u : 0.0;
+    if (on) {
+      const size_t gg = g0 + g;
+      L.qU64[gg * d + tid] = u;
+      L.qU32[gg * d + tid] = (float)u;
+      split3(u, L.qWb, (size_t)L.BH * L.Cqp * d, ((size_t)bh * L.Cqp + g0i + g) * d + tid);
+      L.qsum[gg * d + tid] = 0.0;
+    }
   }
-  un = block_sum(un, red);
-  if (tid == 0) {
-    L.qbias64[gg] = nn;
-    L.qbias32[gg] = (float)nn;
+  block_sums8(un, red, un_s);
+  if (tid < ng) {
+    const size_t gg = g0 + tid;
+    L.qbias64[gg] = nn_s[tid];
+    L.qbias32[gg] = (float)nn_s[tid];
     L.qcount[gg] = 0;
-    L.qwnorm[gg] = (float)sqrt(un);
+    L.qwnorm[gg] = (float)sqrt(un_s[tid]);
   }
 }
 
@@ -529,7 +661,7 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
     order[rk] = tid;
   }
   __syncthreads();
-  // group sums (fp64): keys x, queries x / rms (both products exact in fp64)
+  // group sums (fp64): keys x, queries x / rms with the fp64 scale
   double* sums = (kKeys ? L.ksum : L.qsum) + (size_t)bh * C * D;
   int* counts = (kKeys ? L.kcount : L.qcount) + (size_t)bh * C;
   const int nparts = 256 / D;
@@ -539,7 +671,7 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
     double acc = 0.0;
     for (int q = q0; q < q1; ++q) {
       const int p = order[q];
-      acc += (double)Xs[p * DP + a] * (double)scl[p];
+      acc += (double)Xs[p * DP + a] * (kKeys ? 1.0 : L.inv_rms64[(size_t)bh * L.N + p0 + p]);
       if (q == q1 - 1 || lab[order[q + 1]] != lab[p]) {
         atomicAdd(sums + (size_t)lab[p] * D + a, acc);
         acc = 0.0;
@@ -555,36 +687,100 @@ __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* _
 }
 
 // ------------------------------------------------------------------------------------------
-// a6 prologue: stable counting sort of the labels (one warp per (head, side)).  Members of a
-// group keep ascending token order.  perm[pos] = token, inv[token] = pos, off = group starts.
+// a6 prologue: stable counting sort of the labels, in parallel over chunks of kSortChunk
+// tokens.  Members of a group keep ascending token order.  perm[pos] = token,
+// inv[token] = pos, off = group starts.
+//   1. group_hist_kernel    per (chunk, head, side): label histogram of the chunk
+//   2. group_scan_kernel    per (head, side): group starts, and each chunk's start inside every
+//                           group (chunks in token order), in place of the histogram
+//   3. group_scatter_kernel per (chunk, head, side): one warp places the chunk's tokens in
+//                           token order from those starts
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(32) group_sort_kernel(Layout L) {
-  __shared__ int cursor[kMaxGroups + 1];
-  const int bh = blockIdx.x, side = blockIdx.y, lane = threadIdx.x;
+__device__ __forceinline__ int* sort_hist(const Layout& L, int bh, int side, int chunk) {
+  const int nch = (L.N + kSortChunk - 1) / kSortChunk, Cm = max(L.Ck, L.Cq);
+  return L.sort_hist + (((size_t)bh * 2 + side) * nch + chunk) * Cm;
+}
+
+__global__ void __launch_bounds__(256) group_hist_kernel(Layout L) {
+  __shared__ int h[kMaxGroups];
+  const int chunk = blockIdx.x, bh = blockIdx.y, side = blockIdx.z, tid = threadIdx.x, lane = tid & 31;
+  const int C = side == 0 ? L.Ck : L.Cq;
+  const int* labels = (side == 0 ? L.klabel : L.qlabel) + (size_t)bh * L.N;
+  for (int c = tid; c < C; c += blockDim.x) h[c] = 0;
+  __syncthreads();
+  const int t_lo = chunk * kSortChunk, t_hi = min(L.N, t_lo + kSortChunk);
+  for (int t0 = t_lo; t0 < t_hi; t0 += blockDim.x) {
+    const int t = t0 + tid;
+    const unsigned act = __ballot_sync(0xffffffffu, t < t_hi);
+    if (t < t_hi) {
+      const int l = labels[t];
+      const unsigned same = __match_any_sync(act, l);
+      if (lane == __ffs(same) - 1) atomicAdd(&h[l], __popc(same));
+    }
+  }
+  __syncthreads();
+  int* out = sort_hist(L, bh, side, chunk);
+  for (int c = tid; c < C; c += blockDim.x) out[c] = h[c];
+}
+
+__global__ void __launch_bounds__(1024) group_scan_kernel(Layout L) {
+  __shared__ int wsum[32];
+  const int bh = blockIdx.x, side = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int C = side == 0 ? L.Ck : L.Cq;
+  const int nch = (L.N + kSortChunk - 1) / kSortChunk;
+  int* off = (side == 0 ? L.koff : L.qoff) + (size_t)bh * (C + 1);
+  // totals per group (thread g walks the chunks)
+  int v = 0;
+  if (tid < C)
+    for (int ch = 0; ch < nch; ++ch) v += sort_hist(L, bh, side, ch)[tid];
+  // exclusive scan over the groups (C <= 1024 = blockDim)
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    wsum[lane] = w;
+  }
+  __syncthreads();
+  const int excl = x - v + (warp > 0 ? wsum[warp - 1] : 0);
+  if (tid < C) {
+    off[tid] = excl;
+    int run = excl;  // each chunk's start inside group tid, chunks in token order
+    for (int ch = 0; ch < nch; ++ch) {
+      int* hc = sort_hist(L, bh, side, ch);
+      const int n = hc[tid];
+      hc[tid] = run;
+      run += n;
+    }
+  }
+  if (tid == 0) off[C] = L.N;
+}
+
+__global__ void __launch_bounds__(32) group_scatter_kernel(Layout L) {
+  __shared__ int cursor[kMaxGroups];
+  const int chunk = blockIdx.x, bh = blockIdx.y, side = blockIdx.z, lane = threadIdx.x;
   const int C = side == 0 ? L.Ck : L.Cq;
   const int* labels = (side == 0 ? L.klabel : L.qlabel) + (size_t)bh * L.N;
   int* perm = (side == 0 ? L.kperm : L.qperm) + (size_t)bh * L.N;
   int* inv = (side == 0 ? L.kinv : L.qinv) + (size_t)bh * L.N;
-  int* off = (side == 0 ? L.koff : L.qoff) + (size_t)bh * (C + 1);
-  for (int c = lane; c <= C; c += 32) cursor[c] = 0;
-  __syncwarp();
-  for (int t = lane; t < L.N; t += 32) atomicAdd(&cursor[labels[t]], 1);
-  __syncwarp();
-  if (lane == 0) {
-    int run = 0;
-    for (int c = 0; c < C; ++c) {
-      const int n = cursor[c];
-      off[c] = run;
-      cursor[c] = run;
-      run += n;
-    }
-    off[C] = run;
-  }
+  const int* start = sort_hist(L, bh, side, chunk);
+  for (int c = lane; c < C; c += 32) cursor[c] = start[c];
   __syncwarp();
   const unsigned lt = (1u << lane) - 1u;
-  for (int base = 0; base < L.N; base += 32) {
+  const int t_lo = chunk * kSortChunk, t_hi = min(L.N, t_lo + kSortChunk);
+  for (int base = t_lo; base < t_hi; base += 32) {
     const int t = base + lane;
-    const bool valid = t < L.N;
+    const bool valid = t < t_hi;
     const int l = valid ? labels[t] : -1;
     const unsigned m = __match_any_sync(0xffffffffu, l);
     const int pos = valid ? cursor[l] + __popc(m & lt) : 0;
@@ -598,6 +794,13 @@ __global__ void __launch_bounds__(32) group_sort_kernel(Layout L) {
   }
 }
 
+static void launch_group_sort(const Layout& L, cudaStream_t st) {
+  const int nch = (L.N + kSortChunk - 1) / kSortChunk;
+  launch(group_hist_kernel, dim3(nch, L.BH, 2), 256, 0, st, L);
+  launch(group_scan_kernel, dim3(L.BH, 2), 1024, 0, st, L);
+  launch(group_scatter_kernel, dim3(nch, L.BH, 2), 32, 0, st, L);
+}
+
 // ------------------------------------------------------------------------------------------
 // a5: routing.  S[g,j] = (mean query of group g) . c_j / sqrt(d) + ln m_j over non-empty key
 // groups, visited by score (ties: lower j).  fixed_k > 0 keeps the first fixed_k; otherwise
@@ -605,8 +808,9 @@ __global__ void __launch_bounds__(32) group_sort_kernel(Layout L) {
 // closer to kappa = density*N - (s + C_k + P).
 // ------------------------------------------------------------------------------------------
 template <typename T>
-__global__ void __launch_bounds__(128) route_select_kernel(Layout L, const T* __restrict__ Q) {
+__global__ void __launch_bounds__(256) route_select_kernel(Layout L, const T* __restrict__ Q) {
   __shared__ double qbar[128];
+  __shared__ double qpart[4][128];
   __shared__ double S[kMaxGroups];
   __shared__ int ord[kMaxGroups];
   const int bh = blockIdx.x, g = blockIdx.y, d = L.d, Ck = L.Ck, tid = threadIdx.x;
@@ -616,11 +820,29 @@ __global__ void __launch_bounds__(128) route_select_kernel(Layout L, const T* __
   const int r0 = qoff[g], n = qoff[g + 1] - r0;
   for (int j = tid; j < Ck; j += blockDim.x) route[j] = 0;
   if (n == 0) return;
-  if (tid < d) {
+  {  // mean query of the group: thread (dimension, part) sums every parts-th member
+    const int parts = blockDim.x / d, a = tid % d, part = tid / d;
+    const int* perm = L.qperm + (size_t)bh * L.N + r0;
+    const T* Qh = Q + (size_t)bh * L.N * d + a;
     double acc = 0.0;
-    const int* perm = L.qperm + (size_t)bh * L.N;
-    for (int i = 0; i < n; ++i) acc += (double)to_f32(Q[((size_t)bh * L.N + perm[r0 + i]) * d + tid]);
-    qbar[tid] = acc / (double)n;
+    int i = part;
+    for (; i + 3 * parts < n; i += 4 * parts) {
+      const int t0 = perm[i], t1 = perm[i + parts], t2 = perm[i + 2 * parts], t3 = perm[i + 3 * parts];
+      const float x0 = to_f32(Qh[(size_t)t0 * d]), x1 = to_f32(Qh[(size_t)t1 * d]);
+      const float x2 = to_f32(Qh[(size_t)t2 * d]), x3 = to_f32(Qh[(size_t)t3 * d]);
+      acc += (double)x0;
+      acc += (double)x1;
+      acc += (double)x2;
+      acc += (double)x3;
+    }
+    for (; i < n; i += parts) acc += (double)to_f32(Qh[(size_t)perm[i] * d]);
+    qpart[part][a] = acc;
+    __syncthreads();
+    if (tid < d) {
+      double t = 0.0;
+      for (int q = 0; q < parts; ++q) t += qpart[q][tid];
+      qbar[tid] = t / (double)n;
+    }
   }
   __syncthreads();
   const double rsd = 1.0 / sqrt((double)d);
@@ -845,7 +1067,7 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
   const size_t qf_smem = (size_t)(d + 64) * (d + 1) * sizeof(float);
   cudaFuncSetAttribute(rowqf_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qf_smem);
   // keys: metric M = Qs^T Qs / d, objective constant sum_t k_t^T M k_t, key norms
-  launch(metric_kernel<T>, dim3(L.BH, d), 128, 0, st, L, Q);
+  launch(metric_kernel<T>, dim3(L.BH, d / kMetricRows), 256, 0, st, L, Q);
   cudaMemsetAsync(L.T0k, 0, sizeof(double) * L.BH, st);
   cudaMemsetAsync(L.T0q, 0, sizeof(double) * L.BH, st);
   if (tc) {
@@ -863,17 +1085,20 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
   launch(km_reset_kernel, L.BH, 128, 0, st, L, 0, iters);
   // bf16 inputs with at most 256 groups score on the tensor cores; otherwise on CUDA cores
   const bool tc_keys = km_tc_supported(L, true), tc_queries = km_tc_supported(L, false);
+  const int Gk = tc_keys ? km_tc_grid(L, true) : 0, Gq = tc_queries ? km_tc_grid(L, false) : 0;
   cudaMemsetAsync(L.kWb, 0, (size_t)3 * L.BH * L.Ckp * d * 2, st);
   cudaMemsetAsync(L.qWb, 0, (size_t)3 * L.BH * L.Cqp * d * 2, st);
   const size_t asg_smem = assign_smem_bytes(d);
   const int nblk = (L.N + kAsgPts - 1) / kAsgPts;
   cudaFuncSetAttribute(kmeans_assign_kernel<T, KeyFeat>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asg_smem);
   cudaFuncSetAttribute(kmeans_assign_kernel<T, QueryFeat>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asg_smem);
+  const size_t kprep_smem = (size_t)std::min(d, kPrepRows) * d * sizeof(double);
+  cudaFuncSetAttribute(kprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kprep_smem);
   for (int it = 0; it <= iters; ++it) {
-    launch(kprep_kernel, dim3(L.BH, L.Ck), 128, 0, st, L, it, iters);
+    launch(kprep_kernel, dim3(L.BH, (L.Ck + kPrepGroups - 1) / kPrepGroups), 128, kprep_smem, st, L, it, iters);
     if (it < iters) {
       if (tc_keys) {
-        const sparsepr_status s = launch_kmeans_assign_tc(L, true, K, it, st);
+        const sparsepr_status s = launch_kmeans_iteration_tc(L, true, K, it, Gk, st);
         if (s != SPARSEPR_OK) return s;
       } else {
         launch(kmeans_assign_kernel<T, KeyFeat>, dim3(nblk, L.BH), 256, asg_smem, st, L, K, it);
@@ -896,11 +1121,13 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
   }
   launch(km_reset_kernel, L.BH, 128, 0, st, L, 1, iters);
   SPR_LAUNCH_CHECK();
+  const size_t qprep_smem = ((size_t)kPrepGroups * L.Ck + (size_t)std::min(L.Ck, kPrepRows) * d) * sizeof(double);
+  cudaFuncSetAttribute(qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qprep_smem);
   for (int it = 0; it <= iters; ++it) {
-    launch(qprep_kernel, dim3(L.BH, L.Cq), 128, 0, st, L, it, iters);
+    launch(qprep_kernel, dim3(L.BH, (L.Cq + kPrepGroups - 1) / kPrepGroups), 128, qprep_smem, st, L, it, iters);
     if (it < iters) {
       if (tc_queries) {
-        const sparsepr_status s = launch_kmeans_assign_tc(L, false, Q, it, st);
+        const sparsepr_status s = launch_kmeans_iteration_tc(L, false, Q, it, Gq, st);
         if (s != SPARSEPR_OK) return s;
       } else {
         launch(kmeans_assign_kernel<T, QueryFeat>, dim3(nblk, L.BH), 256, asg_smem, st, L, Q, it);
@@ -908,8 +1135,8 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
     }
   }
   SPR_LAUNCH_CHECK();
-  launch(group_sort_kernel, dim3(L.BH, 2), 32, 0, st, L);
-  launch(route_select_kernel<T>, dim3(L.BH, L.Cq), 128, 0, st, L, Q);
+  launch_group_sort(L, st);
+  launch(route_select_kernel<T>, dim3(L.BH, L.Cq), 256, 0, st, L, Q);
   launch(route_build_kernel, L.BH, 256, 0, st, L, attn_tile_m(L));
   cudaFuncSetAttribute(probe_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kProbeSmem);
   launch(probe_select_kernel, L.BH, 1024, kProbeSmem, st, L);
@@ -925,7 +1152,7 @@ sparsepr_status launch_plan(const Layout& L, const void* Q, const void* K, bool 
 }
 
 sparsepr_status launch_installed_partition(const Layout& L, cudaStream_t st) {
-  launch(group_sort_kernel, dim3(L.BH, 2), 32, 0, st, L);
+  launch_group_sort(L, st);
   launch(route_build_kernel, L.BH, 256, 0, st, L, attn_tile_m(L));
   launch(probe_index_kernel, L.BH, 1024, 0, st, L);
   SPR_LAUNCH_CHECK();

@@ -195,8 +195,9 @@ inline EncodeTiledFn tmap_encode_fn() {
 }
 
 // Tensor map of a 2D bf16 view [rows, d] (d a multiple of 64): boxes of 64 columns (128 bytes,
-// 128-byte swizzle) x box_rows rows; reads past the last row return zeros.
-inline bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, int d, int box_rows) {
+// 128-byte swizzle unless `swizzle` is false) x box_rows rows; reads past the last row return zeros.
+inline bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, int d, int box_rows,
+                           bool swizzle = true) {
   EncodeTiledFn fn = tmap_encode_fn();
   if (!fn || rows <= 0 || d % 64 != 0 || box_rows < 1 || box_rows > 256) return false;
   cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
@@ -204,7 +205,8 @@ inline bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, int
   cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

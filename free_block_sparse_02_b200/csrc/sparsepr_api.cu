@@ -49,6 +49,8 @@ sparsepr_status validate(const sparsepr_config* c) {
   if (c->km_iters > 10000 || c->km_iters_warm > 10000) return SPARSEPR_ERR_INVALID_ARG;
   if ((double)c->B * c->H * c->N * 256.0 > 9.0e18) return SPARSEPR_ERR_INVALID_ARG;
   if (c->d != 64 && c->d != 128) return SPARSEPR_ERR_UNSUPPORTED;
+  // rows of the [B*H*N, d] views are int32 in the kernels (tiles of 128 rows)
+  if ((double)c->B * c->H * (((double)c->N + 127.0) / 128.0) * 128.0 > 2147483647.0) return SPARSEPR_ERR_UNSUPPORTED;
   return SPARSEPR_OK;
 }
 
@@ -107,6 +109,7 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   L.Cqp = (c.n_qgroups + 15) / 16 * 16;
   take(L.Gc, BH * d * d * 8);
   take(L.inv_rms, BH * N * 4);
+  take(L.inv_rms64, BH * N * 8);
   take(L.qxnorm, BH * N * 4);
   take(L.qcent, BH * Cq * Ck * 8);
   take(L.qU64, BH * Cq * d * 8);
@@ -124,6 +127,10 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   take(L.Mb, 3 * BH * d * d * 2);
   take(L.Gcb, 3 * BH * d * d * 2);
   take(L.knorm, BH * N * 4);
+  const size_t km_tiles = BH * (size_t)((N + 127) / 128);
+  take(L.rlist, km_tiles * 128 * 8);
+  take(L.rcnt, km_tiles * 4);
+  take(L.sort_hist, BH * 2 * ((N + kSortChunk - 1) / kSortChunk) * std::max(Ck, Cq) * 4);
   take(L.kperm, BH * N * 4);
   take(L.kinv, BH * N * 4);
   take(L.koff, BH * (Ck + 1) * 4);

@@ -48,7 +48,7 @@ extern "C" {
 typedef enum sparsepr_status {
   SPARSEPR_OK = 0,
   SPARSEPR_ERR_INVALID_ARG = 1,  /* null pointer, size out of range, inconsistent config     */
-  SPARSEPR_ERR_UNSUPPORTED = 2,  /* valid but not built: d not in {64,128}, too many groups  */
+  SPARSEPR_ERR_UNSUPPORTED = 2,  /* valid but not built: d not in {64,128}, or B*H*N above 2^31 rows */
   SPARSEPR_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed               */
   SPARSEPR_ERR_WORKSPACE = 4,    /* workspace null, too small or not 256-byte aligned         */
   SPARSEPR_ERR_NUMERIC = 5,      /* ridge system not positive definite after jitter retries  */
