@@ -72,6 +72,32 @@ def whole_job_tflops(world, flops_per_call, ms_per_call):
     return world * flops_per_call / (ms_per_call * 1e-3) / 1e12
 
 
+def source_hash(*rel):
+    import hashlib
+    h = hashlib.sha256()
+    for r in rel:
+        with open(os.path.join(ROOT, r), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(w):
+    """DRAM read + write bytes per attention launch from the committed ncu summary of this
+    workload, or None when there is none or the attention source changed since it was taken."""
+    import re
+    path = os.path.join(ROOT, "profiles", f"attn_tc_kernel_{w.name}.md")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        text = f.read()
+    m = re.search(r"^dram_bytes_per_launch:\s*(\d+)", text, re.M)
+    h = re.search(r"^source_sha256:\s*([0-9a-f]{64})", text, re.M)
+    cur = source_hash("free_block_sparse_02_b200/csrc/attention_sm100.cu", "free_block_sparse_02_b200/csrc/sm100.cuh")
+    if not m or not h or h.group(1) != cur:
+        return None
+    return int(m.group(1))
+
+
 def workload_config(w, extra=None):
     c = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "density": w.density, "s": w.s,
          "n_kgroups": w.n_kgroups, "n_qgroups": w.n_qgroups, "P": w.P,
@@ -128,6 +154,22 @@ class ClockSampler:
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(rows)}
+
+
+def km_rooflines(w, asg_ms, upd_ms, pk):
+    """HBM rooflines of one key k-means assignment and one update launch (first iteration of
+    the call): each reads every key once (2 d bytes, bf16) and writes (assignment) or reads
+    (update) its label (4 bytes)."""
+    units = w.B * w.H * w.N
+    by = units * (2 * w.d + 4)
+    out = {}
+    for name, t in (("assignment", asg_ms), ("update", upd_ms)):
+        if t > 0:
+            a = by / (t * 1e-3) / 1e9
+            out[name] = {"bound": "hbm", "achieved": a, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": a / pk["hbm_gbs"], "ms": t, "traffic": None,
+                         "algorithmic": f"{units} keys x (2d + 4) bytes = {by} bytes per launch"}
+    return out
 
 
 # ------------------------------------------------------------------------------------ CPU baseline
@@ -211,7 +253,10 @@ def run_ours(args, w, world, rank, local):
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for a, b in kev:  # torch creates the CUDA event on first record; the library records it again
+    # the first key k-means assignment and update launches of each timed call (tensor-core path)
+    km_ev = {kid: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)] for kid in (1, 2)}
+    for a, b in kev + km_ev[1] + km_ev[2]:  # torch creates the CUDA event on first record
         a.record(stream)
         b.record(stream)
     if world > 1:
@@ -222,6 +267,8 @@ def run_ours(args, w, world, rank, local):
     for i in range(args.steps):
         flush.zero_()                         # L2 flush between timed steps, outside the events
         op.set_kernel_events(*kev[i])
+        for kid in (1, 2):
+            op.set_kernel_events(*km_ev[kid][i], kernel=kid)
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
@@ -231,11 +278,16 @@ def run_ours(args, w, world, rank, local):
     launches = S.launch_count() - launches0
     clk = clocks.stop()
     op.set_kernel_events(None, None)
+    for kid in (1, 2):
+        op.set_kernel_events(None, None, kernel=kid)
     step_ms = [a.elapsed_time(b) for a, b in ev]
     kern_ms = [a.elapsed_time(b) for a, b in kev]
+    tc_km = w.dtype == configs.BF16  # the k-means hooks bracket the tensor-core path only
+    asg_ms = statistics.mean(a.elapsed_time(b) for a, b in km_ev[1]) if tc_km else 0.0
+    upd_ms = statistics.mean(a.elapsed_time(b) for a, b in km_ev[2]) if tc_km else 0.0
     ms = statistics.mean(step_ms)
     kms = statistics.mean(kern_ms)
-    ms_max, kms_max = max_over_ranks([ms, kms], world, dev)
+    ms_max, kms_max, asg_ms, upd_ms = max_over_ranks([ms, kms, asg_ms, upd_ms], world, dev)
 
     # end to end through the public API with host buffers (pinned), copies inside the region
     Qh, Kh, Vh = Qc.pin_memory(), Kc.pin_memory(), Vc.pin_memory()
@@ -274,10 +326,13 @@ def run_ours(args, w, world, rank, local):
             "ms_per_call": ms_max,
             "executed_tflops": world * (kflops + 4.0 * w.d * w.B * w.H * w.P * w.N) / (ms_max * 1e-3) / 1e12,
             "kernel_ms": {"block_sparse_attention": kms_max},
-            "roofline": {"bound": "tensor", "kernel": "block-sparse attention", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+            "roofline": {"bound": "tensor", "kernel": "block-sparse attention (the kernel the metric's % of "
+                                                         "bf16 peak refers to)",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "traffic": profiled_traffic(w),
                          "peak_source": f"{pk['source']} bf16 dense (burst)",
                          "algorithmic": f"4*d*executed pairs = {kflops:.4g} flop per launch"},
+            "roofline_kmeans": km_rooflines(w, asg_ms, upd_ms, pk) if tc_km else None,
             "e2e": {"value": whole_job_tflops(world, flops, e2e_ms), "unit": "TFLOPS",
                     "h2d_bytes_per_step": 3 * Q.numel() * elt, "d2h_bytes_per_step": O.numel() * O.element_size(),
                     "ms_per_step": e2e_ms},

@@ -185,11 +185,13 @@ class SparsePR:
         self.attention(Q, K, V, stream)
         return self.fit_apply(O, out_dtype, stream)
 
-    def set_kernel_events(self, start: "torch.cuda.Event", stop: "torch.cuda.Event"):
-        """Bracket the block-sparse attention kernel with two (already created) CUDA events."""
+    def set_kernel_events(self, start: "torch.cuda.Event", stop: "torch.cuda.Event", kernel: int = 0):
+        """Bracket one kernel launch with two (already created) CUDA events: kernel 0 = the
+        block-sparse attention, 1 = the first key k-means assignment, 2 = the first key k-means
+        update (SPARSEPR_KERNEL_* in the C header)."""
         h0 = ctypes.c_void_p(start.cuda_event) if start is not None else None
         h1 = ctypes.c_void_p(stop.cuda_event) if stop is not None else None
-        _check(self.lib.sparsepr_set_kernel_events(self.handle, 0, h0, h1), "sparsepr_set_kernel_events")
+        _check(self.lib.sparsepr_set_kernel_events(self.handle, int(kernel), h0, h1), "sparsepr_set_kernel_events")
 
     def sync(self):
         _check(self.lib.sparsepr_sync(self.handle), "sparsepr_sync")

@@ -39,7 +39,8 @@ constexpr int kSubRows = 16;    // rows per TMA box of K/V
 constexpr int kSubPerTile = kTcTileN / kSubRows;
 constexpr int kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kExpPolyEvery = 4;           // 1 in 4 exponential pairs on the FMA pipe (0: none)
+constexpr int kExpPolyEvery = 0;           // 1 in n exponential pairs on the FMA pipe (0: none; measured
+                                           // slower on sm_100a, where the exponentials are not the bound)
 
 // 2^x on the FMA pipe for x <= kRescaleThreshold (0 below -125, so -inf gives 0): Cody-Waite
 // style reduction x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low mantissa
@@ -59,34 +60,51 @@ static_assert(kAttnTileMTc == 2 * kTcTileM, "a work item is two MMA tiles");
 template <int D>
 struct TcCfg {
   static constexpr int kKB = D / 64;                    // 64-column (128-byte) blocks of a row
-  static constexpr int kStages = D == 64 ? 4 : 2;
+  static constexpr int kKS = D == 64 ? 4 : 3;           // K stages
+  static constexpr int kVS = D == 64 ? 4 : 2;           // V stages (K runs one tile ahead of V)
   static constexpr int kQTileBytes = kTcTileM * D * 2;
   static constexpr int kQBytes = 2 * kQTileBytes;
-  static constexpr int kKVTileBytes = kTcTileN * D * 2;  // one of K or V
-  static constexpr int kStageBytes = 2 * kKVTileBytes;
-  static constexpr int kSmemTiles = kQBytes + kStages * kStageBytes;
-  static constexpr int kSmemBytes = kSmemTiles + 1024 /* align */ + 1024 /* barriers etc */;
+  static constexpr int kKVTileBytes = kTcTileN * D * 2;  // one K or V tile
+  static constexpr int kSmemTiles = kQBytes + (kKS + kVS) * kKVTileBytes;
+  static constexpr int kSmemBytes = kSmemTiles + 1024 /* align */ + 512 /* barriers, tile validity */;
+};
+
+// The keys of a work item: probe items attend to all N keys of the head (one segment);
+// sparse items to the kept key groups' segments of the group-permuted K/V (offset, length),
+// read from the route list and the group offsets in global memory.
+struct Segs {
+  const int* list;  // kept key groups (sparse items)
+  const int* koff;  // key-group offsets of the head
+  int n;            // segments
+  int probe_len;    // > 0: probe item, one segment [0, probe_len)
+  __device__ __forceinline__ int2 at(int i) const {
+    if (probe_len > 0) return make_int2(0, probe_len);
+    const int j = list[i];
+    const int o = koff[j];
+    return make_int2(o, koff[j + 1] - o);
+  }
 };
 
 struct SegState {
-  int seg;   // index into the segment list
-  int off;   // rows already consumed in that segment
+  int seg;   // index of the current segment
+  int off;   // rows already consumed in it
+  int2 cur;  // the current segment (offset, length)
 };
 
 // Next KV tile: row of each 16-row box (global row of the 2D [BH*N, d] view) and its valid
 // row count (0 = box not used; it is then loaded from past the end of the tensor, all zeros).
-__device__ __forceinline__ void next_tile(SegState& s, const int2* segs, int nseg, int row_base, int oob_row,
+__device__ __forceinline__ void next_tile(SegState& s, const Segs& sg, int row_base, int oob_row,
                                           int (&rows)[kSubPerTile], int (&valid)[kSubPerTile]) {
 #pragma unroll
   for (int b = 0; b < kSubPerTile; ++b) {
-    while (s.seg < nseg && s.off >= segs[s.seg].y) {
+    while (s.seg < sg.n && s.off >= s.cur.y) {
       ++s.seg;
       s.off = 0;
+      if (s.seg < sg.n) s.cur = sg.at(s.seg);
     }
-    if (s.seg < nseg) {
-      const int2 sg = segs[s.seg];
-      rows[b] = row_base + sg.x + s.off;
-      valid[b] = min(kSubRows, sg.y - s.off);
+    if (s.seg < sg.n) {
+      rows[b] = row_base + s.cur.x + s.off;
+      valid[b] = min(kSubRows, s.cur.y - s.off);
       s.off += kSubRows;
     } else {
       rows[b] = oob_row;
@@ -104,18 +122,23 @@ __global__ void __launch_bounds__(384, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sQ = smem;                // tile t at t * kQTileBytes
-  uint8_t* sKV = smem + C::kQBytes;  // stage s: K at s*kStageBytes, V right after
+  uint8_t* sQ = smem;                            // tile t at t * kQTileBytes
+  uint8_t* sK = smem + C::kQBytes;               // K stage s at s * kKVTileBytes
+  uint8_t* sV = sK + C::kKS * C::kKVTileBytes;   // V stage s at s * kKVTileBytes
   uint64_t* bars = (uint64_t*)(smem + C::kSmemTiles);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = kv_full + C::kStages;
-  uint64_t* s_full = kv_empty + C::kStages;  // [2] per query tile
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + C::kKS;
+  uint64_t* v_full = k_empty + C::kKS;
+  uint64_t* v_empty = v_full + C::kVS;
+  uint64_t* s_full = v_empty + C::kVS;       // [2] per query tile
   uint64_t* p_full = s_full + 2;             // [2]
   uint64_t* o_bar = p_full + 2;              // [2]
   uint64_t* mma_done = o_bar + 2;
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
-  __shared__ int2 segs[kMaxGroups];
+  // valid rows of each 16-row box of the tile held in V stage s, written by the producer before
+  // the V copy (the softmax reads it after waiting on that copy)
+  int* tvalid = (int*)(tmem_slot + 2);       // [kVS][kSubPerTile]
   __shared__ int s_nseg, s_ntiles, s_qrow0, s_rows0, s_rows1, s_mode, s_bh;
   __shared__ volatile int s_abort;
 
@@ -161,30 +184,25 @@ __global__ void __launch_bounds__(384, 1)
   if (s_rows0 <= 0) return;  // uniform: no barrier, TMEM or copy has been touched yet
   const int mode = s_mode, bh = s_bh;
   const int ntq = s_rows1 > 0 ? 2 : 1;
+  const int g_item = s_nseg;  // sparse items: the query group
+  __syncthreads();
+  Segs sg;
+  sg.probe_len = mode == 1 ? L.N : 0;
+  sg.list = L.route_list + ((size_t)bh * L.Cq + (mode == 1 ? 0 : g_item)) * L.Ck;
+  sg.koff = L.koff + (size_t)bh * (L.Ck + 1);
+  sg.n = mode == 1 ? 1 : L.route_cnt[(size_t)bh * L.Cq + g_item];
   if (tid == 0) {
     int nsub = 0;
-    if (mode == 1) {
-      segs[0] = make_int2(0, L.N);
-      s_nseg = 1;
-      nsub = (L.N + kSubRows - 1) / kSubRows;
-    } else {
-      const int g = s_nseg;
-      const int cnt = L.route_cnt[(size_t)bh * L.Cq + g];
-      const int* list = L.route_list + ((size_t)bh * L.Cq + g) * L.Ck;
-      const int* koff = L.koff + (size_t)bh * (L.Ck + 1);
-      for (int i = 0; i < cnt; ++i) {
-        const int j = list[i];
-        const int len = koff[j + 1] - koff[j];
-        segs[i] = make_int2(koff[j], len);
-        nsub += (len + kSubRows - 1) / kSubRows;
-      }
-      s_nseg = cnt;
-    }
+    for (int i = 0; i < sg.n; ++i) nsub += (sg.at(i).y + kSubRows - 1) / kSubRows;
     s_ntiles = (nsub + kSubPerTile - 1) / kSubPerTile;
     mbar_init(q_full, 1);
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(kv_full + s, 1);
-      mbar_init(kv_empty + s, 1);
+    for (int s = 0; s < C::kKS; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < C::kVS; ++s) {
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full + t, 1);
@@ -202,7 +220,7 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int nseg = s_nseg, ntiles = s_ntiles, qrow0 = s_qrow0;
+  const int ntiles = s_ntiles, qrow0 = s_qrow0;
   const int row_base = bh * L.N;   // first row of this head in the 2D K/V view
   const int oob_row = L.BH * L.N;  // a box starting here is entirely zero-filled
 
@@ -219,31 +237,54 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int kb = 0; kb < C::kKB; ++kb)
           tma_load_2d(sQ + t * C::kQTileBytes + kb * kTcTileM * 128, qm, q_full, kb * 64, qy + t * kTcTileM);
-      SegState st{0, 0};
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int s = i % C::kStages;
-        if (!mbar_wait(kv_empty + s, ((i / C::kStages) & 1) ^ 1, &s_abort)) break;
-        int rows[kSubPerTile], valid[kSubPerTile];
-        next_tile(st, segs, nseg, row_base, oob_row, rows, valid);
-        uint8_t* sK = sKV + s * C::kStageBytes;
-        uint8_t* sV = sK + C::kKVTileBytes;
-        mbar_arrive_expect_tx(kv_full + s, C::kStageBytes);
+      // K(0), K(1), V(0), K(2), V(1), ...: K runs one tile ahead of V
+      SegState st{0, 0, sg.n > 0 ? sg.at(0) : make_int2(0, 0)};
+      int rows[kSubPerTile], valid[kSubPerTile], prows[kSubPerTile], pvalid[kSubPerTile];
+      int nk = 0, nv = 0;  // K and V tiles issued
+      auto load_k = [&](int i) -> bool {
+        const int s = i % C::kKS;
+        if (!mbar_wait(k_empty + s, ((i / C::kKS) & 1) ^ 1, &s_abort)) return false;
+        uint8_t* dst = sK + s * C::kKVTileBytes;
+        mbar_arrive_expect_tx(k_full + s, C::kKVTileBytes);
+#pragma unroll
+        for (int b = 0; b < kSubPerTile; ++b)
+#pragma unroll
+          for (int kb = 0; kb < C::kKB; ++kb)
+            tma_load_2d(dst + kb * kTcTileN * 128 + b * kSubRows * 128, &tmK, k_full + s, kb * 64, rows[b]);
+        ++nk;
+        return true;
+      };
+      auto load_v = [&](int i) -> bool {
+        const int s = i % C::kVS;
+        if (!mbar_wait(v_empty + s, ((i / C::kVS) & 1) ^ 1, &s_abort)) return false;
+#pragma unroll
+        for (int b = 0; b < kSubPerTile; ++b) tvalid[s * kSubPerTile + b] = pvalid[b];
+        uint8_t* dst = sV + s * C::kKVTileBytes;
+        mbar_arrive_expect_tx(v_full + s, C::kKVTileBytes);  // (release: tvalid is visible to its waiters)
+#pragma unroll
+        for (int b = 0; b < kSubPerTile; ++b)
+#pragma unroll
+          for (int kb = 0; kb < C::kKB; ++kb)
+            tma_load_2d(dst + kb * kTcTileN * 128 + b * kSubRows * 128, &tmV, v_full + s, kb * 64, prows[b]);
+        ++nv;
+        return true;
+      };
+      bool okp = true;
+      for (int i = 0; okp && i < ntiles; ++i) {
+        next_tile(st, sg, row_base, oob_row, rows, valid);
+        okp = load_k(i);
+        if (okp && i > 0) okp = load_v(i - 1);
 #pragma unroll
         for (int b = 0; b < kSubPerTile; ++b) {
-#pragma unroll
-          for (int kb = 0; kb < C::kKB; ++kb) {
-            const int off = kb * kTcTileN * 128 + b * kSubRows * 128;
-            tma_load_2d(sK + off, &tmK, kv_full + s, kb * 64, rows[b]);
-            tma_load_2d(sV + off, &tmV, kv_full + s, kb * 64, rows[b]);
-          }
+          prows[b] = rows[b];
+          pvalid[b] = valid[b];
         }
-        ++issued;
       }
+      if (okp && ntiles > 0) load_v(ntiles - 1);
       // drain: never leave with copies in flight into this CTA's shared memory
       mbar_wait_drain(q_full, 0);
-      for (int i = max(0, issued - C::kStages); i < issued; ++i)
-        mbar_wait_drain(kv_full + (i % C::kStages), (i / C::kStages) & 1);
+      for (int i = max(0, nk - C::kKS); i < nk; ++i) mbar_wait_drain(k_full + (i % C::kKS), (i / C::kKS) & 1);
+      for (int i = max(0, nv - C::kVS); i < nv; ++i) mbar_wait_drain(v_full + (i % C::kVS), (i / C::kVS) & 1);
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
@@ -252,7 +293,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t idesc_o = idesc_bf16_f32(kTcTileM, D, 0, 1);
       const uint32_t q_addr = smem_u32(sQ);
       auto issue_s = [&](int t, int j) {  // S_t(j) = Q_t K_j^T
-        const uint32_t k_addr = smem_u32(sKV + (j % C::kStages) * C::kStageBytes);
+        const uint32_t k_addr = smem_u32(sK + (j % C::kKS) * C::kKVTileBytes);
         const uint32_t qa = q_addr + t * C::kQTileBytes;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
@@ -266,7 +307,7 @@ __global__ void __launch_bounds__(384, 1)
       auto issue_pv = [&](int t, int j) -> bool {  // O_t += P_t(j) V_j
         if (!mbar_wait(p_full + t, j & 1, &s_abort)) return false;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(sKV + (j % C::kStages) * C::kStageBytes + C::kKVTileBytes);
+        const uint32_t v_addr = smem_u32(sV + (j % C::kVS) * C::kKVTileBytes);
 #pragma unroll
         for (int ks = 0; ks < kTcTileN / 16; ++ks) {
           // B = V (keys x d, d contiguous): 16 keys per step = 2048 bytes; LBO = next 64 d-columns
@@ -276,23 +317,28 @@ __global__ void __launch_bounds__(384, 1)
         mma_commit(o_bar + t);
         return true;
       };
-      bool ok = mbar_wait(q_full, 0, &s_abort) && mbar_wait(kv_full, 0, &s_abort);
+      bool ok = mbar_wait(q_full, 0, &s_abort) && mbar_wait(k_full, 0, &s_abort);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         if (ntq == 2) issue_s(1, 0);
+        mma_commit(k_empty);  // K_0 is free once S(0) completes
       }
       for (int j = 0; ok && j < ntiles; ++j) {
         const bool more = j + 1 < ntiles;
+        if (!mbar_wait(v_full + j % C::kVS, (j / C::kVS) & 1, &s_abort)) break;
         if (!issue_pv(0, j)) break;
         if (more) {
-          if (!mbar_wait(kv_full + (j + 1) % C::kStages, ((j + 1) / C::kStages) & 1, &s_abort)) break;
+          if (!mbar_wait(k_full + (j + 1) % C::kKS, ((j + 1) / C::kKS) & 1, &s_abort)) break;
           tc_fence_after();
           issue_s(0, j + 1);
         }
         if (ntq == 2 && !issue_pv(1, j)) break;
-        mma_commit(kv_empty + j % C::kStages);  // K_j, V_j no longer read once these complete
-        if (more && ntq == 2) issue_s(1, j + 1);
+        mma_commit(v_empty + j % C::kVS);  // V_j is no longer read once these complete
+        if (more) {
+          if (ntq == 2) issue_s(1, j + 1);
+          mma_commit(k_empty + (j + 1) % C::kKS);  // nor K_{j+1}
+        }
       }
       // every MMA issued by this thread has completed before TMEM is released
       mma_commit(mma_done);
@@ -308,19 +354,22 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tO = tmem + lane_base + 256 + t * D;
     const float scale2 = 1.4426950408889634f / sqrtf((float)D);
     float m_used = -INFINITY, l = 0.f;
-    SegState st{0, 0};
     bool ok = ntiles > 0 && t < ntq;
     for (int j = 0; ok && j < ntiles; ++j) {
-      int rows[kSubPerTile], valid[kSubPerTile];
-      next_tile(st, segs, nseg, row_base, oob_row, rows, valid);
-      bool full = true;  // every key of the tile is real (the same for every thread of the CTA)
-#pragma unroll
-      for (int b = 0; b < kSubPerTile; ++b) full = full && valid[b] == kSubRows;
-      // warp-uniform: the tcgen05.ld below needs every lane of the warp
-      const bool okw = mbar_wait(s_full + t, j & 1, &s_abort);
+      // warp-uniform: the tcgen05.ld below needs every lane of the warp.  The V copy of tile j
+      // is waited on too: it orders the producer's tile-validity words before their read.
+      const bool okw = mbar_wait(s_full + t, j & 1, &s_abort) &&
+                       mbar_wait(v_full + j % C::kVS, (j / C::kVS) & 1, &s_abort);
       if (!__all_sync(0xffffffffu, okw)) {
         ok = false;
         break;
+      }
+      int valid[kSubPerTile];
+      bool full = true;  // every key of the tile is real (the same for every thread of the CTA)
+#pragma unroll
+      for (int b = 0; b < kSubPerTile; ++b) {
+        valid[b] = tvalid[(j % C::kVS) * kSubPerTile + b];
+        full = full && valid[b] == kSubRows;
       }
       tc_fence_after();
       // pass 1: row max over the real keys (four loads, one wait; eight independent chains)

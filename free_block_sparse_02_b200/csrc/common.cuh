@@ -96,10 +96,12 @@ struct Layout {
   float* knorm;                   // [BH, N] ||k_t||_2 (rounding bound of the key scores)
 
   // points of the tensor-core assignment whose two best scores were within the rounding bound,
-  // re-decided in fp64 by the update pass: CTA c of the assignment grid appends to its own
-  // segment starting at (first tile of c) * 128, entries (row bh*N + p, float bits of the
-  // tentative score), and leaves the segment length in rcnt[c]
-  int2* rlist;                    // [BH * ceil(N/128) * 128]
+  // re-decided in fp64: CTA c of the assignment grid appends to its own segment starting at
+  // (first tile of c) * 128 and leaves the segment length in rcnt[c].  Entry: x = row bh*N + p,
+  // y = float bits of the tentative score, z = candidate count (bits 0..7; 255 = all groups) |
+  // candidate 0 << 8 | candidate 1 << 18, w = candidate 2 | candidate 3 << 16 (candidates: the
+  // groups whose fp32 score is within the bound of the best, ascending)
+  int4* rlist;                    // [BH * ceil(N/128) * 128]
   int* rcnt;                      // [BH * ceil(N/128)]
 
   // group-contiguous order (stable counting sort)

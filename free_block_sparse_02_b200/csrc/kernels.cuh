@@ -11,8 +11,15 @@ constexpr int kAttnTileM = 64;
 constexpr int kAttnTileMTc = 256;
 inline int attn_tile_m(const Layout& L) { return L.dtype == SPARSEPR_BF16 ? kAttnTileMTc : kAttnTileM; }
 
+// Optional events recorded around single launches (ids: SPARSEPR_KERNEL_*).
+struct KernelEvents {
+  static constexpr int kCount = 3;
+  cudaEvent_t start[kCount] = {};
+  cudaEvent_t stop[kCount] = {};
+};
+
 sparsepr_status launch_plan(const Layout& L, const void* Q, const void* K, bool warm, int iters,
-                            cudaStream_t st);
+                            cudaStream_t st, const KernelEvents& ev);
 sparsepr_status launch_installed_partition(const Layout& L, cudaStream_t st);
 sparsepr_status launch_permute(const Layout& L, const void* Q, const void* K, const void* V,
                                cudaStream_t st);
@@ -27,7 +34,7 @@ int km_tc_grid(const Layout& L, bool keys);
 // One Lloyd iteration after the centroid update: tensor-core assignment, then the fp64
 // re-decisions, group sums and counts (both kernels over the same G tile ranges).
 sparsepr_status launch_kmeans_iteration_tc(const Layout& L, bool keys, const void* X, int it, int G,
-                                           cudaStream_t st);
+                                           cudaStream_t st, const KernelEvents* ev = nullptr);
 sparsepr_status launch_rowqf_tc(const Layout& L, int which, const void* X, cudaStream_t st);
 
 // Upper bound of the number of query tiles of one head: sum_g ceil(n_g / tile) <= N/tile + C_q.

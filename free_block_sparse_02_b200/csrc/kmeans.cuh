@@ -5,36 +5,96 @@
 
 namespace sparsepr {
 
+// Sum over the 32 lanes of each of 32 values: afterwards lane l holds the total of v[l]
+// (recursive halving: 16 + 8 + 4 + 2 + 1 shuffles instead of 32 full warp sums).
+__device__ __forceinline__ double warp_transpose_sum32(double (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const bool up = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const double send = up ? v[i] : v[i + s];
+      const double keep = up ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return v[0];
+}
+
 // fp64 score of every group for one point (one warp), lowest index on exact ties; x staged in
-// xs (fp64, shared memory).  Lanes run over the dimensions, so every row of W (and of Gc) is
-// read coalesced; each dot is completed by a warp sum, identical in every lane.  Queries need
-// the exact scale 1/rms: ms = x^T Gc x.  Eight groups per step keep eight rows of loads in flight.
+// xs (fp64, shared memory).  Lanes run over the dimensions, so every row of W and Gc is read
+// coalesced.  Queries need the exact scale 1/rms: ms = x^T Gc x, each lane summing over its
+// columns and one warp sum at the end.  Group dots are formed 32 groups at a time and
+// transposed across the lanes (lane l gets group 32 c + l), then the lowest score wins.
+// The exact query scale 1/rms = 1/sqrt(x^T Gc x + 1e-12) (Gc in global or shared memory), one
+// warp: each lane sums over its columns, one warp sum at the end.
+__device__ __forceinline__ double query_scale_fp64(const double* Gc, const double* xs, const double (&xl)[4], int D) {
+  const int lane = threadIdx.x & 31;
+  double part = 0.0;
+#pragma unroll 4
+  for (int a = 0; a < D; ++a) {
+    double row = 0.0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (lane + 32 * k < D) row += Gc[(size_t)a * D + lane + 32 * k] * xl[k];
+    part += row * xs[a];
+  }
+  return 1.0 / sqrt(warp_sum(part) + 1e-12);
+}
+
+// fp64 argmin over a short candidate list (ascending group ids; the lowest id wins exact ties),
+// one warp; `scale` is 1 for keys.
+__device__ __forceinline__ void redecide_candidates(const double* xs, int D, const double* W64, const double* B64,
+                                                    double scale, const int* cand, int ncand, int& best_out,
+                                                    double& bestv_out) {
+  const int lane = threadIdx.x & 31;
+  double bv = INFINITY;
+  int bj = 0;
+  for (int c = 0; c < ncand; ++c) {
+    const int j = cand[c];
+    double part = 0.0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (lane + 32 * k < D) part += W64[(size_t)j * D + lane + 32 * k] * xs[lane + 32 * k];
+    const double sc = B64[j] - 2.0 * scale * warp_sum(part);
+    if (sc < bv) {
+      bv = sc;
+      bj = j;
+    }
+  }
+  best_out = bj;
+  bestv_out = bv;
+}
+
 template <bool kKeys>
 __device__ void redecide_fp64(const Layout& L, int bh, const double* xs, int D, int C, const double* W64,
-                              const double* B64, int& best_out, double& bestv_out) {
+                              const double* B64, int& best_out, double& bestv_out, const double* Gc_in = nullptr) {
   const int lane = threadIdx.x & 31;
   double xl[4];  // this lane's dimensions lane, lane + 32, ... (D <= 128)
 #pragma unroll
   for (int k = 0; k < 4; ++k) xl[k] = lane + 32 * k < D ? xs[lane + 32 * k] : 0.0;
   double scale = 1.0;
   if constexpr (!kKeys) {
-    const double* Gc = L.Gc + (size_t)bh * D * D;
-    double ms = 0.0;
+    const double* Gc = Gc_in ? Gc_in : L.Gc + (size_t)bh * D * D;
+    double part = 0.0;
+#pragma unroll 4
     for (int a = 0; a < D; ++a) {
-      double part = 0.0;
+      double row = 0.0;
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        if (lane + 32 * k < D) part += Gc[(size_t)a * D + lane + 32 * k] * xl[k];
-      ms += warp_sum(part) * xs[a];
+        if (lane + 32 * k < D) row += Gc[(size_t)a * D + lane + 32 * k] * xl[k];
+      part += row * xs[a];
     }
+    const double ms = warp_sum(part);
     scale = 1.0 / sqrt(ms + 1e-12);
   }
   double bv = INFINITY;
   int bj = 0x7fffffff;
-  for (int j0 = 0; j0 < C; j0 += 8) {
-    double part[8];
+  for (int j0 = 0; j0 < C; j0 += 32) {
+    double part[32];
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
+    for (int g = 0; g < 32; ++g) {
       part[g] = 0.0;
       if (j0 + g < C) {
         const double* w = W64 + (size_t)(j0 + g) * D;
@@ -43,16 +103,23 @@ __device__ void redecide_fp64(const Layout& L, int bh, const double* xs, int D, 
           if (lane + 32 * k < D) part[g] += w[lane + 32 * k] * xl[k];
       }
     }
-#pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      const double dot = warp_sum(part[g]);
-      if (j0 + g < C) {
-        const double sc = B64[j0 + g] - 2.0 * scale * dot;
-        if (sc < bv) {  // ascending j: strict < keeps the lower index
-          bv = sc;
-          bj = j0 + g;
-        }
+    const double dot = warp_transpose_sum32(part);  // group j0 + lane
+    const int j = j0 + lane;
+    if (j < C) {
+      const double sc = B64[j] - 2.0 * scale * dot;
+      if (sc < bv) {  // ascending j per lane: strict < keeps the lower index
+        bv = sc;
+        bj = j;
       }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+    if (ov < bv || (ov == bv && oj < bj)) {
+      bv = ov;
+      bj = oj;
     }
   }
   best_out = (bj >= 0 && bj < C) ? bj : 0;

@@ -67,7 +67,7 @@ __host__ inline size_t km_assign_smem(int D, int Np, int stages) {
 // offsets and cursors.
 __host__ inline size_t km_update_smem(int D, int C) {
   (void)D;
-  return (size_t)2 * kKmUpdChunk * 4 /*labels, order*/ + (size_t)(2 * C + 1) * 4;
+  return (size_t)2 * kKmUpdChunk * 4 /*labels, order*/ + (size_t)(3 * C + 1) * 4;
 }
 
 __device__ __forceinline__ int km_tiles_per_head(const Layout& L) { return (L.N + kKmTile - 1) / kKmTile; }
@@ -111,7 +111,8 @@ __global__ void __launch_bounds__(kKmThreads, 1)
   __shared__ int s_rcnt;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t tcols = km_tc_tmem_cols(2 * Npr);
+  // two accumulators of Npr columns; the epilogue reads 128 columns at a time from b * Npr
+  const uint32_t tcols = km_tc_tmem_cols(max(2 * Npr, Npr + 128 * ((Npr + 127) / 128)));
   if (tid == 0) {
     s_abort = 0;
     s_rcnt = 0;
@@ -267,7 +268,7 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         const float* WN = (kKeys ? L.kwnorm : L.qwnorm) + (size_t)bh * C;
         __syncwarp();  // every lane is done with the previous head's copy
         float wm = 0.f, bm = 0.f;
-        for (int j = lane; j < Npr; j += 32) {
+        for (int j = lane; j < 256; j += 32) {
           const float bj = j < C ? B32[j] : INFINITY;
           bias[j] = bj;
           if (j < C) {
@@ -295,30 +296,67 @@ __global__ void __launch_bounds__(kKmThreads, 1)
       const float m2s = -2.f * sq;
       float b1 = INFINITY, b2 = INFINITY;
       int i1 = -1;
-      for (int c0 = 0; c0 < Npr; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + b * Npr + c0, r);  // b * Npr + c0 + 32 <= 2 Npr <= tcols
+      for (int c0 = 0; c0 < Npr; c0 += 128) {  // four 32-column loads, one wait
+        // columns past this tile's Npr (the other accumulator, or unwritten TMEM inside the
+        // allocation: b * Npr + c0 + 128 <= tcols) have bias +inf and never win
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        const uint32_t ta = tmem + lane_base + b * Npr + c0;
+        tmem_ld32(ta, r0);
+        tmem_ld32(ta + 32, r1);
+        tmem_ld32(ta + 64, r2);
+        tmem_ld32(ta + 96, r3);
         tmem_wait_ld();
 #pragma unroll
-        for (int kk = 0; kk < 32; ++kk) {
+        for (int kk = 0; kk < 128; ++kk) {
+          const uint32_t rv = kk < 32 ? r0[kk & 31] : kk < 64 ? r1[kk & 31] : kk < 96 ? r2[kk & 31] : r3[kk & 31];
           // ascending j and strict <: the lowest index of equal scores wins
-          const float sc = fmaf(m2s, __uint_as_float(r[kk]), bias[c0 + kk]);
+          const float sc = fmaf(m2s, __uint_as_float(rv), bias[c0 + kk]);
           const bool lt = sc < b1;
           b2 = lt ? b1 : fminf(b2, sc);
           i1 = lt ? c0 + kk : i1;
           b1 = lt ? sc : b1;
         }
       }
+      const float delta = 4.f * (3 * D + 8) * u * xn * wmax + 4.f * u * bmax;
+      const bool ref = valid && !(b2 - b1 > 2.f * delta);
+      // candidates of a flagged point: every group whose fp32 score is within the bound of the
+      // best (the fp64 argmin is among them).  With at most 128 groups the warp reads its scores
+      // once more (warp-uniform branch, before the accumulator is released).
+      int nc = 255;
+      uint32_t cpk = 0;  // up to four candidate groups, 8 bits each
+      if (Npr <= 128 && __any_sync(0xffffffffu, ref)) {
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        const uint32_t ta = tmem + lane_base + b * Npr;
+        tmem_ld32(ta, r0);
+        tmem_ld32(ta + 32, r1);
+        tmem_ld32(ta + 64, r2);
+        tmem_ld32(ta + 96, r3);
+        tmem_wait_ld();
+        if (ref) {
+          const float thr = b1 + 2.5f * delta;
+          nc = 0;
+#pragma unroll
+          for (int kk = 0; kk < 128; ++kk) {
+            const uint32_t rv = kk < 32 ? r0[kk & 31] : kk < 64 ? r1[kk & 31] : kk < 96 ? r2[kk & 31] : r3[kk & 31];
+            const float sc = fmaf(m2s, __uint_as_float(rv), bias[kk]);
+            if (sc <= thr) {
+              if (nc < 4) cpk |= (uint32_t)kk << (8 * nc);
+              ++nc;
+            }
+          }
+          if (nc > 4 || nc == 0) nc = 255;
+        }
+      }
       tc_fence_before();
       mbar_arrive(acc_empty + b);
       if (valid) {
-        const float delta = 4.f * (3 * D + 8) * u * xn * wmax + 4.f * u * bmax;
-        const bool ref = !(b2 - b1 > 2.f * delta);
         labels[row] = (i1 >= 0 && i1 < C) ? i1 : 0;  // non-finite scores never yield a bad label
         jsum += (double)b1;
         if (ref) {
+          const int c0 = cpk & 0xFF, c1 = (cpk >> 8) & 0xFF, c2 = (cpk >> 16) & 0xFF, c3 = cpk >> 24;
           const int slot = atomicAdd(&s_rcnt, 1);
-          L.rlist[(size_t)t0 * kKmTile + slot] = make_int2((int)row, __float_as_int(b1));
+          L.rlist[(size_t)t0 * kKmTile + slot] =
+              make_int4((int)row, __float_as_int(b1), nc | (c0 << 8) | (c1 << 18), c2 | (c3 << 16));
           ++nref;
         }
       }
@@ -341,24 +379,20 @@ __global__ void __launch_bounds__(kKmThreads, 1)
   }
 }
 
-// Exact fp64 value of a bf16 given by its 16 bits (normal numbers by moving the exponent and
-// mantissa fields; zero, subnormals, inf and nan through fp32).
-__device__ __forceinline__ double bf16_bits_to_f64(uint32_t b) {
-  const uint32_t ex = b & 0x7F80u;
-  if (ex == 0u || ex == 0x7F80u) return (double)__uint_as_float(b << 16);
-  // sign to bit 63, exponent + (1023 - 127) to bits 62..52, 7 mantissa bits to 51..45
-  const uint32_t hi = ((b & 0x8000u) << 16) | (((b & 0x7FFFu) << 13) + 0x38000000u);
-  return __hiloint2double((int)hi, 0);
-}
+// Exact fp64 value of a bf16 given by its 16 bits (through its exact fp32 value).
+__device__ __forceinline__ double bf16_bits_to_f64(uint32_t b) { return (double)__uint_as_float(b << 16); }
 
 // fp64 re-decision of the points the assignment listed: block (c, y) takes every
 // kKmRedecideSplit-th entry of CTA range c's list, one warp per point; the label and the
-// objective (its fp64 score minus the tentative fp32 one) are corrected in place.
+// objective (its fp64 score minus the tentative fp32 one) are corrected in place.  Points with
+// a short candidate list evaluate only those groups; queries stage Gc in shared memory (dynamic:
+// d * d doubles) for the exact scale.
 constexpr int kKmRedecideSplit = 4;
 
 template <bool kKeys>
 __global__ void __launch_bounds__(256) kmeans_redecide_kernel(const __nv_bfloat16* __restrict__ X, Layout L, int it,
                                                               int G) {
+  extern __shared__ double Gcs[];  // queries: Gc of the current head
   __shared__ double xs_all[8][128];
   const int D = L.d, C = kKeys ? L.Ck : L.Cq;
   const int tph = km_tiles_per_head(L);
@@ -366,20 +400,68 @@ __global__ void __launch_bounds__(256) kmeans_redecide_kernel(const __nv_bfloat1
   km_range((long long)L.BH * tph, G, blockIdx.x, t0, t1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nlist = min(max(L.rcnt[blockIdx.x], 0), max(t1 - t0, 0) * kKmTile);  // never past the segment
-  const int2* list = L.rlist + (size_t)t0 * kKmTile;
+  if ((int)blockIdx.y * 8 >= nlist) return;  // no entry for this block (uniform)
+  const int4* list = L.rlist + (size_t)t0 * kKmTile;
   int* labels = kKeys ? L.klabel : L.qlabel;
   double* Jarr = kKeys ? L.kJ : L.qJ;
   double* xs = xs_all[warp];
-  for (int li = blockIdx.y * 8 + warp; li < nlist; li += 8 * kKmRedecideSplit) {
-    const int2 en = list[li];
-    const int row = en.x, bh = row / L.N;
+  int gc_head = -1;  // head whose Gc is staged (the range spans few heads; stage per change)
+  for (int li0 = blockIdx.y * 8; li0 < nlist; li0 += 8 * kKmRedecideSplit) {
+    const int li = li0 + warp;
+    int bh = -1;
+    int4 en = make_int4(0, 0, 0, 0);
+    if (li < nlist) {
+      en = list[li];
+      bh = en.x / L.N;
+    }
+    if constexpr (!kKeys) {  // the block's warps agree on the heads they need: stage on change
+      const int need = __shfl_sync(0xffffffffu, bh, 0);
+      __shared__ int s_need[8];
+      if (lane == 0) s_need[warp] = need;
+      __syncthreads();
+      int first = -1;
+      bool mixed = false;
+      for (int w = 0; w < 8; ++w)
+        if (s_need[w] >= 0) {
+          if (first < 0) first = s_need[w];
+          else if (s_need[w] != first) mixed = true;
+        }
+      if (!mixed && first >= 0 && first != gc_head) {
+        const double* src = L.Gc + (size_t)first * D * D;
+        for (int e = threadIdx.x; e < D * D / 2; e += blockDim.x)
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(Gcs + 2 * e)),
+                       "l"(src + 2 * e)
+                       : "memory");
+        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+        gc_head = first;
+      } else if (mixed) {
+        gc_head = -1;  // heads differ inside this round: read Gc from global memory
+      }
+      __syncthreads();
+    }
+    if (li >= nlist) continue;
+    const int row = en.x;
     for (int a = lane; a < D; a += 32) xs[a] = (double)__bfloat162float(X[(size_t)row * D + a]);
     __syncwarp();
     int best;
     double bv;
     const double* W64 = (kKeys ? L.kW64 : L.qU64) + (size_t)bh * C * D;
     const double* B64 = (kKeys ? L.kbias64 : L.qbias64) + (size_t)bh * C;
-    redecide_fp64<kKeys>(L, bh, xs, D, C, W64, B64, best, bv);
+    const double* Gc = (!kKeys && gc_head == bh) ? Gcs : L.Gc + (size_t)bh * D * D;
+    const int nc = en.z & 0xFF;
+    if (nc <= 4) {
+      int cand[4] = {(en.z >> 8) & 0x3FF, (en.z >> 18) & 0x3FF, en.w & 0xFFFF, (en.w >> 16) & 0xFFFF};
+      double scale = 1.0;
+      if constexpr (!kKeys) {
+        double xl[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) xl[k] = lane + 32 * k < D ? xs[lane + 32 * k] : 0.0;
+        scale = query_scale_fp64(Gc, xs, xl, D);
+      }
+      redecide_candidates(xs, D, W64, B64, scale, cand, nc, best, bv);
+    } else {
+      redecide_fp64<kKeys>(L, bh, xs, D, C, W64, B64, best, bv, Gc);
+    }
     if (lane == 0) {
       labels[row] = best;
       atomicAdd(Jarr + (size_t)bh * L.iters_cap + it, bv - (double)__int_as_float(en.y));
@@ -404,6 +486,8 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
   int* order = lab + kKmUpdChunk;              // [kKmUpdChunk] chunk points sorted by label
   int* offs = order + kKmUpdChunk;             // [C + 1] start of each label's run
   int* cursor = offs + (C + 1);                // [C] histogram, then next slot per label
+  int* byrun = cursor + C;                     // [C] groups by decreasing run length
+  __shared__ int s_next;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int* labels = kKeys ? L.klabel : L.qlabel;
@@ -476,14 +560,36 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
         order[base + __popc(same & ((1u << lane) - 1))] = i;
       }
     }
+    // groups by decreasing run length (longest first), for the dynamic schedule below
+    for (int g = tid; g < C; g += kKmUpdThreads) {
+      const int sz = offs[g + 1] - offs[g];
+      int rk = 0;
+      if (C <= 256)
+        for (int h = 0; h < C; ++h) {
+          const int sh = offs[h + 1] - offs[h];
+          rk += sh > sz || (sh == sz && h < g);
+        }
+      else
+        rk = g;
+      byrun[rk] = g;
+    }
+    if (tid == 0) s_next = 0;
     __syncthreads();
-    // accumulation: item = (group, eight dimensions); consecutive threads read consecutive
-    // 16-byte pieces of the same rows; each item's run is summed in fp64 registers
+    // accumulation: a warp takes the next 32 / octs groups (longest runs first); within it,
+    // item = (group, eight dimensions), consecutive lanes reading consecutive 16-byte pieces of
+    // the same rows; each item's run is summed in fp64 registers
     const __nv_bfloat16* Xc = X + row0 * D;
     const double* sig = L.inv_rms64 + row0;
     double* sums = sums_all + (size_t)bh * C * D;
-    for (int item = tid; item < C * octs; item += kKmUpdThreads) {
-      const int g = item / octs, oc = item % octs;
+    const int gpw = 32 / octs;
+    while (true) {
+      int k = 0;
+      if (lane == 0) k = atomicAdd(&s_next, 1);
+      k = __shfl_sync(0xffffffffu, k, 0);
+      if (k * gpw >= C) break;  // the same for the whole warp
+      const int gi = k * gpw + lane / octs;
+      if (gi >= C) continue;
+      const int g = byrun[gi], oc = lane % octs;
       const int q0 = offs[g], q1 = offs[g + 1];
       if (q0 == q1) continue;
       double r[8];
@@ -701,7 +807,11 @@ int km_tc_grid(const Layout& L, bool keys) {
 }
 
 sparsepr_status launch_kmeans_iteration_tc(const Layout& L, bool keys, const void* X, int it, int G,
-                                           cudaStream_t st) {
+                                           cudaStream_t st, const KernelEvents* ev) {
+  auto mark = [&](int id, bool stop) {
+    const cudaEvent_t e = ev ? (stop ? ev->stop[id] : ev->start[id]) : nullptr;
+    if (e) cudaEventRecord(e, st);
+  };
   CUtensorMap mX, mW;
   const int D = L.d;
   const int Np = keys ? L.Ckp : L.Cqp;
@@ -717,14 +827,20 @@ sparsepr_status launch_kmeans_iteration_tc(const Layout& L, bool keys, const voi
   if (keys) {
     cudaFuncSetAttribute(kmeans_assign_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
     cudaFuncSetAttribute(kmeans_update_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_u);
+    mark(SPARSEPR_KERNEL_KMEANS_ASSIGN, false);
     launch(kmeans_assign_tc_kernel<true>, G, kKmThreads, smem_a, st, mX, mW, L, it, G, S);
-    launch(kmeans_redecide_kernel<true>, dim3(G, kKmRedecideSplit), 256, 0, st, Xb, L, it, G);
+    mark(SPARSEPR_KERNEL_KMEANS_ASSIGN, true);
+    launch(kmeans_redecide_kernel<true>, dim3(G, kKmRedecideSplit), 256, 0, st, Xb, L, it, G);  // keys: no Gc
+    mark(SPARSEPR_KERNEL_KMEANS_UPDATE, false);
     launch(kmeans_update_kernel<true>, G, kKmUpdThreads, smem_u, st, Xb, L, it, G);
+    mark(SPARSEPR_KERNEL_KMEANS_UPDATE, true);
   } else {
     cudaFuncSetAttribute(kmeans_assign_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
     cudaFuncSetAttribute(kmeans_update_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_u);
     launch(kmeans_assign_tc_kernel<false>, G, kKmThreads, smem_a, st, mX, mW, L, it, G, S);
-    launch(kmeans_redecide_kernel<false>, dim3(G, kKmRedecideSplit), 256, 0, st, Xb, L, it, G);
+    const size_t smem_r = (size_t)D * D * sizeof(double);
+    cudaFuncSetAttribute(kmeans_redecide_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r);
+    launch(kmeans_redecide_kernel<false>, dim3(G, kKmRedecideSplit), 256, smem_r, st, Xb, L, it, G);
     launch(kmeans_update_kernel<false>, G, kKmUpdThreads, smem_u, st, Xb, L, it, G);
   }
   SPR_LAUNCH_CHECK();

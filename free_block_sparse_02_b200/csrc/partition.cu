@@ -38,6 +38,7 @@ constexpr int kMetricChunk = 64;
 template <typename T>
 __global__ void __launch_bounds__(256) metric_kernel(Layout L, const T* __restrict__ Q) {
   __shared__ float qs[kMetricChunk][128];
+  __shared__ long long rowi[kMetricChunk];
   const int bh = blockIdx.x, a0 = blockIdx.y * kMetricRows, d = L.d, tid = threadIdx.x;
   const int b = tid % d, lanes_per_b = 256 / d, r0 = tid / d;
   constexpr int kMaxOut = kMetricRows / 2;  // d = 128: 8 rows per thread; d = 64: 4
@@ -49,10 +50,11 @@ __global__ void __launch_bounds__(256) metric_kernel(Layout L, const T* __restri
   for (int i0 = 0; i0 < L.s; i0 += kMetricChunk) {
     const int ni = min(kMetricChunk, L.s - i0);
     __syncthreads();
+    if (tid < ni) rowi[tid] = ((2LL * (i0 + tid) + 1) * L.N) / (2LL * L.s);
+    __syncthreads();
     for (int e = tid; e < ni * d; e += 256) {
       const int i = e / d, c = e % d;
-      const long long row = ((2LL * (i0 + i) + 1) * L.N) / (2LL * L.s);
-      qs[i][c] = to_f32(q[row * d + c]);
+      qs[i][c] = to_f32(q[rowi[i] * d + c]);
     }
     __syncthreads();
     for (int i = 0; i < ni; ++i) {
@@ -286,12 +288,18 @@ __device__ __forceinline__ void block_sums8(const double (&v)[kPrepGroups], doub
 
 constexpr int kPrepRows = 128;  // rows of M or C staged in shared memory at a time (fp64)
 
-// Rows [r0, r0 + nr) of a row-major fp64 matrix with `cols` columns into shared memory, all
-// threads of the block loading together (coalesced, many loads in flight).
+// Rows [r0, r0 + nr) of a row-major fp64 matrix with `cols` (even) columns into shared memory
+// by 16-byte asynchronous copies, all issued before one wait (many in flight).  Both addresses
+// are 16-byte aligned: workspace regions are 256-byte aligned and rows hold an even count of
+// doubles.  The caller synchronises the block afterwards.
 __device__ __forceinline__ void stage_rows(double* dst, const double* __restrict__ src, int r0, int nr, int cols) {
-  const int n = nr * cols;
+  const int n16 = nr * cols / 2;
   const double* s = src + (size_t)r0 * cols;
-  for (int e = threadIdx.x; e < n; e += blockDim.x) dst[e] = s[e];
+  for (int e = threadIdx.x; e < n16; e += blockDim.x)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst + 2 * e)),
+                 "l"(s + 2 * e)
+                 : "memory");
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 // Keys, kPrepGroups groups per block (grid BH x ceil(C_k / 8), thread a = dimension):
@@ -768,6 +776,7 @@ __global__ void __launch_bounds__(1024) group_scan_kernel(Layout L) {
 
 __global__ void __launch_bounds__(32) group_scatter_kernel(Layout L) {
   __shared__ int cursor[kMaxGroups];
+  __shared__ int lab[kSortChunk];
   const int chunk = blockIdx.x, bh = blockIdx.y, side = blockIdx.z, lane = threadIdx.x;
   const int C = side == 0 ? L.Ck : L.Cq;
   const int* labels = (side == 0 ? L.klabel : L.qlabel) + (size_t)bh * L.N;
@@ -775,13 +784,15 @@ __global__ void __launch_bounds__(32) group_scatter_kernel(Layout L) {
   int* inv = (side == 0 ? L.kinv : L.qinv) + (size_t)bh * L.N;
   const int* start = sort_hist(L, bh, side, chunk);
   for (int c = lane; c < C; c += 32) cursor[c] = start[c];
+  const int t_lo = chunk * kSortChunk, t_hi = min(L.N, t_lo + kSortChunk);
+#pragma unroll 8
+  for (int t = t_lo + lane; t < t_hi; t += 32) lab[t - t_lo] = labels[t];  // loads in flight together
   __syncwarp();
   const unsigned lt = (1u << lane) - 1u;
-  const int t_lo = chunk * kSortChunk, t_hi = min(L.N, t_lo + kSortChunk);
   for (int base = t_lo; base < t_hi; base += 32) {
     const int t = base + lane;
     const bool valid = t < t_hi;
-    const int l = valid ? labels[t] : -1;
+    const int l = valid ? lab[t - t_lo] : -1;
     const unsigned m = __match_any_sync(0xffffffffu, l);
     const int pos = valid ? cursor[l] + __popc(m & lt) : 0;
     __syncwarp();
@@ -1054,12 +1065,41 @@ __global__ void permute_rows_kernel(Layout L, const void* __restrict__ src, void
   for (int c = lane; c < chunks; c += 32) o[c] = s[c];
 }
 
+// Q by the query-group order, K and V by the key-group order, in one pass: thread = one
+// 16-byte piece of a row of each (three independent loads in flight per piece).
+__global__ void __launch_bounds__(256) permute_qkv_kernel(Layout L, const void* __restrict__ Q,
+                                                          const void* __restrict__ K, const void* __restrict__ V) {
+  const int bh = blockIdx.y;
+  const size_t rb = (size_t)L.d * elt_size(L.dtype);
+  const int chunks = (int)(rb / 16);
+  const long long total = (long long)L.N * chunks;
+  const int* qp = L.qperm + (size_t)bh * L.N;
+  const int* kp = L.kperm + (size_t)bh * L.N;
+  const char* q = (const char*)Q + (size_t)bh * L.N * rb;
+  const char* k = (const char*)K + (size_t)bh * L.N * rb;
+  const char* v = (const char*)V + (size_t)bh * L.N * rb;
+  char* qo = (char*)L.Qp + (size_t)bh * L.N * rb;
+  char* ko = (char*)L.Kp + (size_t)bh * L.N * rb;
+  char* vo = (char*)L.Vp + (size_t)bh * L.N * rb;
+  for (long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x; p < total; p += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(p / chunks), c = (int)(p % chunks);
+    const size_t so = (size_t)c * 16, dofs = (size_t)r * rb + so;
+    const int tq = qp[r], tk = kp[r];
+    const uint4 a = *(const uint4*)(q + (size_t)tq * rb + so);
+    const uint4 b = *(const uint4*)(k + (size_t)tk * rb + so);
+    const uint4 e = *(const uint4*)(v + (size_t)tk * rb + so);
+    *(uint4*)(qo + dofs) = a;
+    *(uint4*)(ko + dofs) = b;
+    *(uint4*)(vo + dofs) = e;
+  }
+}
+
 // ------------------------------------------------------------------------------------------
 // Host launchers.
 // ------------------------------------------------------------------------------------------
 template <typename T>
 static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool warm, int iters,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, const KernelEvents& ev) {
   const int d = L.d;
   const bool tc = L.dtype == SPARSEPR_BF16;  // bf16 inputs: tensor-core quadratic forms
   const size_t dd = (size_t)L.BH * d * d;
@@ -1098,7 +1138,7 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
     launch(kprep_kernel, dim3(L.BH, (L.Ck + kPrepGroups - 1) / kPrepGroups), 128, kprep_smem, st, L, it, iters);
     if (it < iters) {
       if (tc_keys) {
-        const sparsepr_status s = launch_kmeans_iteration_tc(L, true, K, it, Gk, st);
+        const sparsepr_status s = launch_kmeans_iteration_tc(L, true, K, it, Gk, st, it == 0 ? &ev : nullptr);
         if (s != SPARSEPR_OK) return s;
       } else {
         launch(kmeans_assign_kernel<T, KeyFeat>, dim3(nblk, L.BH), 256, asg_smem, st, L, K, it);
@@ -1146,9 +1186,9 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
 }
 
 sparsepr_status launch_plan(const Layout& L, const void* Q, const void* K, bool warm, int iters,
-                            cudaStream_t st) {
-  if (L.dtype == SPARSEPR_F32) return plan_typed<float>(L, (const float*)Q, (const float*)K, warm, iters, st);
-  return plan_typed<__nv_bfloat16>(L, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, warm, iters, st);
+                            cudaStream_t st, const KernelEvents& ev) {
+  if (L.dtype == SPARSEPR_F32) return plan_typed<float>(L, (const float*)Q, (const float*)K, warm, iters, st, ev);
+  return plan_typed<__nv_bfloat16>(L, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, warm, iters, st, ev);
 }
 
 sparsepr_status launch_installed_partition(const Layout& L, cudaStream_t st) {
@@ -1161,10 +1201,11 @@ sparsepr_status launch_installed_partition(const Layout& L, cudaStream_t st) {
 
 sparsepr_status launch_permute(const Layout& L, const void* Q, const void* K, const void* V,
                                cudaStream_t st) {
-  const dim3 grid((L.N * 32 + 255) / 256, L.BH);
-  launch(permute_rows_kernel, grid, 256, 0, st, L, Q, L.Qp, L.qperm, L.N, L.N);
-  launch(permute_rows_kernel, grid, 256, 0, st, L, K, L.Kp, L.kperm, L.N, L.N);
-  launch(permute_rows_kernel, grid, 256, 0, st, L, V, L.Vp, L.kperm, L.N, L.N);
+  {
+    const long long pieces = (long long)L.N * (L.d * (long long)elt_size(L.dtype) / 16);
+    const int gx = (int)std::min<long long>((pieces + 1023) / 1024, 65535);  // about four pieces per thread
+    launch(permute_qkv_kernel, dim3(gx, L.BH), 256, 0, st, L, Q, K, V);
+  }
   if (L.P > 0)
     launch(permute_rows_kernel, dim3((L.P * 32 + 255) / 256, L.BH), 256, 0, st, L, Q, L.Qprobe, L.probe_tok, L.P, L.N);
   SPR_LAUNCH_CHECK();

@@ -22,8 +22,7 @@ struct sparsepr_plan_s {
   bool attended = false;    // attention ran on the current partition
   bool have_state = false;  // centroids of a previous plan exist (warm start)
   cudaStream_t last = nullptr;
-  cudaEvent_t ev_start = nullptr;  // optional timing hook around the block-sparse kernel
-  cudaEvent_t ev_stop = nullptr;
+  KernelEvents ev;  // optional timing hooks (see sparsepr_set_kernel_events)
 };
 
 std::atomic<long long> sparsepr::g_launches{0};
@@ -128,7 +127,7 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   take(L.Gcb, 3 * BH * d * d * 2);
   take(L.knorm, BH * N * 4);
   const size_t km_tiles = BH * (size_t)((N + 127) / 128);
-  take(L.rlist, km_tiles * 128 * 8);
+  take(L.rlist, km_tiles * 128 * 16);
   take(L.rcnt, km_tiles * 4);
   take(L.sort_hist, BH * 2 * ((N + kSortChunk - 1) / kSortChunk) * std::max(Ck, Cq) * 4);
   take(L.kperm, BH * N * 4);
@@ -238,7 +237,7 @@ sparsepr_status sparsepr_plan(sparsepr_plan_t* p, const void* Q, const void* K, 
   p->last = st;
   p->planned = false;
   p->attended = false;
-  sparsepr_status s = launch_plan(p->L, Q, K, warm, iters, st);
+  sparsepr_status s = launch_plan(p->L, Q, K, warm, iters, st, p->ev);
   if (s != SPARSEPR_OK) return s;
   p->planned = true;
   p->have_state = true;
@@ -292,7 +291,7 @@ sparsepr_status sparsepr_attention(sparsepr_plan_t* p, const void* Q, const void
   p->last = st;
   sparsepr_status s = launch_permute(p->L, Q, K, V, st);
   if (s != SPARSEPR_OK) return s;
-  s = launch_attention(p->L, st, p->ev_start, p->ev_stop);
+  s = launch_attention(p->L, st, p->ev.start[SPARSEPR_KERNEL_BLOCK_SPARSE], p->ev.stop[SPARSEPR_KERNEL_BLOCK_SPARSE]);
   if (s != SPARSEPR_OK) return s;
   p->attended = true;
   return SPARSEPR_OK;
@@ -366,10 +365,10 @@ void sparsepr_plan_destroy(sparsepr_plan_t* p) { delete p; }
 
 sparsepr_status sparsepr_set_kernel_events(sparsepr_plan_t* p, int32_t kernel, void* start_event,
                                            void* stop_event) {
-  if (!p || kernel != SPARSEPR_KERNEL_BLOCK_SPARSE) return SPARSEPR_ERR_INVALID_ARG;
+  if (!p || kernel < 0 || kernel >= KernelEvents::kCount) return SPARSEPR_ERR_INVALID_ARG;
   if ((start_event == nullptr) != (stop_event == nullptr)) return SPARSEPR_ERR_INVALID_ARG;
-  p->ev_start = (cudaEvent_t)start_event;
-  p->ev_stop = (cudaEvent_t)stop_event;
+  p->ev.start[kernel] = (cudaEvent_t)start_event;
+  p->ev.stop[kernel] = (cudaEvent_t)stop_event;
   return SPARSEPR_OK;
 }
 

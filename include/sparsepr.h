@@ -168,14 +168,19 @@ const char* sparsepr_status_string(sparsepr_status status);
 /* Library version, e.g. 100 for 0.1.0. */
 int32_t sparsepr_version(void);
 
-/* Kernels whose launches sparsepr_set_kernel_events can bracket. */
-enum { SPARSEPR_KERNEL_BLOCK_SPARSE = 0 };
+/* Kernels whose launches sparsepr_set_kernel_events can bracket:
+ *   BLOCK_SPARSE   the block-sparse (and probe-row) attention launch of sparsepr_attention;
+ *   KMEANS_ASSIGN  the first key-group k-means assignment launch of sparsepr_plan (bf16
+ *                  inputs, tensor-core path: one pass over all keys);
+ *   KMEANS_UPDATE  the first key-group k-means update launch of sparsepr_plan (group sums
+ *                  and counts: one pass over all keys). */
+enum { SPARSEPR_KERNEL_BLOCK_SPARSE = 0, SPARSEPR_KERNEL_KMEANS_ASSIGN = 1, SPARSEPR_KERNEL_KMEANS_UPDATE = 2 };
 
-/* Optional timing hook for measurement.  When set, sparsepr_attention records `start_event`
- * on its stream immediately before launching the block-sparse attention kernel and
- * `stop_event` immediately after it, so cudaEventElapsedTime gives that kernel's duration.
- * Events are cudaEvent_t handles passed as void*, created and owned by the caller; passing
- * NULL for both removes the hook.  Returns INVALID_ARG for an unknown kernel id. */
+/* Optional timing hook for measurement.  When set, the library records `start_event` on its
+ * stream immediately before launching the named kernel and `stop_event` immediately after it,
+ * so cudaEventElapsedTime gives that kernel's duration.  Events are cudaEvent_t handles passed
+ * as void*, created and owned by the caller; passing NULL for both removes the hook.  Returns
+ * INVALID_ARG for an unknown kernel id. */
 sparsepr_status sparsepr_set_kernel_events(sparsepr_plan_t* plan, int32_t kernel, void* start_event,
                                            void* stop_event);
 
