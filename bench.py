@@ -360,11 +360,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload on this many heads instead (a smaller case for profilers)")
+    ap.add_argument("--density", type=float, default=0.0, help="override the density target (sweeps)")
+    ap.add_argument("--probes", type=int, default=-1, help="override the probe budget P (sweeps)")
     args = ap.parse_args()
     world, rank, local = dist_env()
     w = configs.workload(args.workload)
     if args.heads > 0:
         w = configs.scaled_down(w, heads=args.heads)
+    if args.density > 0:
+        w = w.replace(density=args.density)
+    if args.probes >= 0:
+        w = w.replace(P=args.probes)
     if args.impl == "reference":
         run_reference(args, w, world, rank)
     else:

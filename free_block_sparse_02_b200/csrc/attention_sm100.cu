@@ -9,7 +9,7 @@
 // Work item = 256 query rows of one query group (block-sparse pass) or of one head's probe rows
 // (dense pass), as two 128-row MMA tiles Q0, Q1 that share every KV tile.  The keys are the
 // concatenation of the kept key groups' rows in the group-permuted K/V, streamed in 128-key
-// tiles assembled from 16-row TMA boxes, so a kept key group costs at most 15 padded (masked)
+// tiles assembled from 32-row TMA boxes, so a kept key group costs at most 31 padded (masked)
 // rows wherever it starts.
 //
 // CTA of 384 threads: warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner), warps 4..7
@@ -35,7 +35,7 @@ using namespace sm100;
 
 constexpr int kTcTileM = 128;   // query rows per MMA tile
 constexpr int kTcTileN = 128;   // keys per KV tile (MMA N of S, K of PV)
-constexpr int kSubRows = 16;    // rows per TMA box of K/V
+constexpr int kSubRows = 32;    // rows per TMA box of K/V (32: measured faster than 16 at d = 128)
 constexpr int kSubPerTile = kTcTileN / kSubRows;
 constexpr int kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -91,7 +91,7 @@ struct SegState {
   int2 cur;  // the current segment (offset, length)
 };
 
-// Next KV tile: row of each 16-row box (global row of the 2D [BH*N, d] view) and its valid
+// Next KV tile: row of each kSubRows-row box (global row of the 2D [BH*N, d] view) and its valid
 // row count (0 = box not used; it is then loaded from past the end of the tensor, all zeros).
 __device__ __forceinline__ void next_tile(SegState& s, const Segs& sg, int row_base, int oob_row,
                                           int (&rows)[kSubPerTile], int (&valid)[kSubPerTile]) {
@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* o_bar = p_full + 2;              // [2]
   uint64_t* mma_done = o_bar + 2;
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
-  // valid rows of each 16-row box of the tile held in V stage s, written by the producer before
+  // valid rows of each box of the tile held in V stage s, written by the producer before
   // the V copy (the softmax reads it after waiting on that copy)
   int* tvalid = (int*)(tmem_slot + 2);       // [kVS][kSubPerTile]
   __shared__ int s_nseg, s_ntiles, s_qrow0, s_rows0, s_rows1, s_mode, s_bh;
@@ -447,7 +447,8 @@ __global__ void __launch_bounds__(384, 1)
         for (int k = 0; k < 32; ++k) {
           const float x0 = fmaf(__uint_as_float(sv[2 * k]), scale2, neg_m);
           const float x1 = fmaf(__uint_as_float(sv[2 * k + 1]), scale2, neg_m);
-          const bool poly = kExpPolyEvery > 0 && (k % kExpPolyEvery) == kExpPolyEvery - 1;
+          constexpr int kEvery = kExpPolyEvery > 0 ? kExpPolyEvery : 1;
+          const bool poly = kExpPolyEvery > 0 && (k % kEvery) == kEvery - 1;
           const float p0 = poly ? exp2_poly(x0) : ex2(x0);
           const float p1 = poly ? exp2_poly(x1) : ex2(x1);
           ls[k & 3] += p0 + p1;

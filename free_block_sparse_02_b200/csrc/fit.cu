@@ -124,8 +124,6 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
   double* G = shs;  // [n1][n1], later S [d][d]
   __shared__ double red[8];
   __shared__ double ldiag[129];  // diagonal of the Cholesky factor
-  __shared__ int s_piv;
-  __shared__ double s_norm;
   const double* Gg = L.ridgeG + (size_t)bh * n1 * n1;
   double* A = L.A64 + (size_t)bh * n1 * d;
   sparsepr_head_stats& st = L.stats[bh];
@@ -222,83 +220,81 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
   if (full) {
     rank = d;
   } else if (s_dmax > 0.0) {
+    // Column-pivoted Gram-Schmidt with one barrier per step: every warp finds the same pivot
+    // (largest remaining squared norm cn, lowest index on ties); the unused columns remove
+    // their component along the pivot column v_p (v_c -= (v_p . v_c / |v_p|^2) v_p, the pivot
+    // column itself is normalised once at the end), tpc threads per column.
     for (int e = tid; e < d * d; e += blockDim.x) S[e] = Sg[e];  // S[i*d + c]: column c, entry i
     __shared__ double cn[128];
     __shared__ int used[128];
-    __shared__ double s_tol;
+    __shared__ double binv[128];
+    __shared__ int bcol[128];
+    const int tpc = blockDim.x / d, sub = tid % tpc;  // 4 (d = 64) or 2 (d = 128)
     __syncthreads();
-    // column norms: 2 threads per column
-    for (int c = tid >> 1; c < d; c += blockDim.x >> 1) {
+    for (int c = tid / tpc; c < d; c += blockDim.x / tpc) {
       double sacc = 0.0;
-      for (int i = tid & 1; i < d; i += 2) sacc += S[i * d + c] * S[i * d + c];
-      sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
-      if ((tid & 1) == 0) {
+      for (int i = sub; i < d; i += tpc) sacc += S[i * d + c] * S[i * d + c];
+      for (int o = 1; o < tpc; o <<= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
+      if (sub == 0) {
         cn[c] = sacc;
         used[c] = 0;
       }
     }
     __syncthreads();
-    if (tid < 32) {
-      double mx = 0.0;
-      for (int c = tid; c < d; c += 32) mx = fmax(mx, cn[c]);
-      for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      if (tid == 0) s_tol = mx * 1e-20;
-    }
-    __syncthreads();
+    const int lane = tid & 31;
+    double mx = 0.0;
+    for (int c = lane; c < d; c += 32) mx = fmax(mx, cn[c]);
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const double tol = mx * 1e-20;
     for (int step = 0; step < d; ++step) {
-      if (tid < 32) {  // pivot: unused column of largest remaining norm (lowest index on ties)
-        double bv = -1.0;
-        int bi = -1;
-        for (int c = tid; c < d; c += 32)
-          if (!used[c] && cn[c] > bv) {
-            bv = cn[c];
-            bi = c;
-          }
-        for (int o = 16; o > 0; o >>= 1) {
-          const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-          if (ov > bv || (ov == bv && oi >= 0 && (bi < 0 || oi < bi))) {
-            bv = ov;
-            bi = oi;
-          }
+      double bv = -1.0;
+      int bi = -1;
+      for (int c = lane; c < d; c += 32)
+        if (!used[c] && cn[c] > bv) {
+          bv = cn[c];
+          bi = c;
         }
-        double nrm = 0.0;
-        if (bi >= 0 && bv > s_tol && bv > 0.0)
-          for (int i = tid; i < d; i += 32) nrm += S[i * d + bi] * S[i * d + bi];
-        for (int o = 16; o > 0; o >>= 1) nrm += __shfl_xor_sync(0xffffffffu, nrm, o);
-        if (tid == 0) {
-          s_piv = (bi >= 0 && bv > s_tol && bv > 0.0) ? bi : -1;
-          if (s_piv >= 0) {
-            used[s_piv] = 1;
-            s_norm = sqrt(nrm);
-          }
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi >= 0 && (bi < 0 || oi < bi))) {
+          bv = ov;
+          bi = oi;
         }
       }
-      __syncthreads();
-      const int pv = s_piv;
-      if (pv < 0) break;
-      for (int i = tid; i < d; i += blockDim.x) S[i * d + pv] /= s_norm;
-      __syncthreads();
-      // remove the new direction from every unused column: 2 threads per column
-      for (int c = tid >> 1; c < d; c += blockDim.x >> 1) {
-        const bool act = !used[c];
+      if (!(bi >= 0 && bv > tol && bv > 0.0)) break;  // the same in every thread
+      const double inv2 = 1.0 / bv;
+      for (int c = tid / tpc; c < d; c += blockDim.x / tpc) {
+        const bool act = !used[c] && c != bi;
         double dot = 0.0;
         if (act)
-          for (int i = tid & 1; i < d; i += 2) dot += S[i * d + pv] * S[i * d + c];
-        dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+          for (int i = sub; i < d; i += tpc) dot += S[i * d + bi] * S[i * d + c];
+        for (int o = 1; o < tpc; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        dot *= inv2;
         double sacc = 0.0;
         if (act)
-          for (int i = tid & 1; i < d; i += 2) {
-            const double v = S[i * d + c] - dot * S[i * d + pv];
+          for (int i = sub; i < d; i += tpc) {
+            const double v = S[i * d + c] - dot * S[i * d + bi];
             S[i * d + c] = v;
             sacc += v * v;
           }
-        sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
-        if (act && (tid & 1) == 0) cn[c] = sacc;
+        for (int o = 1; o < tpc; o <<= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
+        if (act && sub == 0) cn[c] = sacc;
       }
-      basis[rank++] = pv;
+      if (tid == 0) {
+        used[bi] = 1;
+        bcol[rank] = bi;
+        binv[rank] = sqrt(inv2);
+      }
+      ++rank;
       __syncthreads();
     }
+    for (int e = tid; e < d * rank; e += blockDim.x) {  // normalise the basis columns
+      const int i = e / rank, r = e % rank;
+      S[i * d + bcol[r]] *= binv[r];
+    }
+    __syncthreads();
+    for (int r = 0; r < rank; ++r) basis[r] = bcol[r];
   }
   // hand the basis to the projection kernel: columns r < rank of spanS are U's columns
   __syncthreads();

@@ -23,7 +23,7 @@
 //              best are within a rigorous rounding bound goes to the CTA's re-decision list.
 //  re-decide   Re-decides the listed points over all groups in fp64 (one warp each, all over
 //              the GPU; label and objective corrected).
-//  update      For chunks of up to 8192 points of one head,
+//  update      For chunks of up to 16384 points of one head,
 //              counting-sorts the points by label in shared memory and sums each group's run:
 //              one thread per (group, 8 dimensions) gathers the run's rows (consecutive threads
 //              read consecutive 16-byte pieces of a row), accumulates sigma x in fp64 registers
@@ -48,7 +48,7 @@ constexpr int kKmTile = 128;
 constexpr int kKmThreads = 384;   // warp 0 TMA, warp 1 MMA, warps 4..11 epilogue
 constexpr int kKmUpdThreads = 512;
 constexpr int kKmMaxStages = 4;
-constexpr int kKmUpdChunk = 8192;  // points of one head sorted and summed at a time by the update
+constexpr int kKmUpdChunk = 16384;  // points of one head sorted and summed at a time by the update
 
 __host__ __device__ inline int km_tc_tmem_cols(int n) {
   int c = 32;
@@ -111,8 +111,7 @@ __global__ void __launch_bounds__(kKmThreads, 1)
   __shared__ int s_rcnt;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // two accumulators of Npr columns; the epilogue reads 128 columns at a time from b * Npr
-  const uint32_t tcols = km_tc_tmem_cols(max(2 * Npr, Npr + 128 * ((Npr + 127) / 128)));
+  const uint32_t tcols = km_tc_tmem_cols(2 * Npr);  // two accumulators of Npr columns
   if (tid == 0) {
     s_abort = 0;
     s_rcnt = 0;
@@ -296,21 +295,15 @@ __global__ void __launch_bounds__(kKmThreads, 1)
       const float m2s = -2.f * sq;
       float b1 = INFINITY, b2 = INFINITY;
       int i1 = -1;
-      for (int c0 = 0; c0 < Npr; c0 += 128) {  // four 32-column loads, one wait
-        // columns past this tile's Npr (the other accumulator, or unwritten TMEM inside the
-        // allocation: b * Npr + c0 + 128 <= tcols) have bias +inf and never win
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        const uint32_t ta = tmem + lane_base + b * Npr + c0;
-        tmem_ld32(ta, r0);
-        tmem_ld32(ta + 32, r1);
-        tmem_ld32(ta + 64, r2);
-        tmem_ld32(ta + 96, r3);
+      for (int c0 = 0; c0 < Npr; c0 += 32) {
+        // columns C .. Npr-1 (padded groups) have bias +inf and never win
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + b * Npr + c0, r);  // b * Npr + c0 + 32 <= 2 Npr <= tcols
         tmem_wait_ld();
 #pragma unroll
-        for (int kk = 0; kk < 128; ++kk) {
-          const uint32_t rv = kk < 32 ? r0[kk & 31] : kk < 64 ? r1[kk & 31] : kk < 96 ? r2[kk & 31] : r3[kk & 31];
+        for (int kk = 0; kk < 32; ++kk) {
           // ascending j and strict <: the lowest index of equal scores wins
-          const float sc = fmaf(m2s, __uint_as_float(rv), bias[c0 + kk]);
+          const float sc = fmaf(m2s, __uint_as_float(r[kk]), bias[c0 + kk]);
           const bool lt = sc < b1;
           b2 = lt ? b1 : fminf(b2, sc);
           i1 = lt ? c0 + kk : i1;
@@ -325,27 +318,25 @@ __global__ void __launch_bounds__(kKmThreads, 1)
       int nc = 255;
       uint32_t cpk = 0;  // up to four candidate groups, 8 bits each
       if (Npr <= 128 && __any_sync(0xffffffffu, ref)) {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        const uint32_t ta = tmem + lane_base + b * Npr;
-        tmem_ld32(ta, r0);
-        tmem_ld32(ta + 32, r1);
-        tmem_ld32(ta + 64, r2);
-        tmem_ld32(ta + 96, r3);
-        tmem_wait_ld();
-        if (ref) {
-          const float thr = b1 + 2.5f * delta;
-          nc = 0;
+        const float thr = b1 + 2.5f * delta;
+        int cnt = 0;
+#pragma unroll 1
+        for (int c0 = 0; c0 < Npr; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + b * Npr + c0, r);
+          tmem_wait_ld();
+          if (ref) {
 #pragma unroll
-          for (int kk = 0; kk < 128; ++kk) {
-            const uint32_t rv = kk < 32 ? r0[kk & 31] : kk < 64 ? r1[kk & 31] : kk < 96 ? r2[kk & 31] : r3[kk & 31];
-            const float sc = fmaf(m2s, __uint_as_float(rv), bias[kk]);
-            if (sc <= thr) {
-              if (nc < 4) cpk |= (uint32_t)kk << (8 * nc);
-              ++nc;
+            for (int kk = 0; kk < 32; ++kk) {
+              const float sc = fmaf(m2s, __uint_as_float(r[kk]), bias[c0 + kk]);
+              if (sc <= thr) {
+                if (cnt < 4) cpk |= (uint32_t)(c0 + kk) << (8 * cnt);
+                ++cnt;
+              }
             }
           }
-          if (nc > 4 || nc == 0) nc = 255;
         }
+        if (ref) nc = (cnt > 4 || cnt == 0) ? 255 : cnt;
       }
       tc_fence_before();
       mbar_arrive(acc_empty + b);
@@ -596,15 +587,15 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
 #pragma unroll
       for (int k = 0; k < 8; ++k) r[k] = 0.0;
       int q = q0;
-      for (; q + 4 <= q1; q += 4) {
-        int pidx[4];
-        uint4 v[4];
+      for (; q + 8 <= q1; q += 8) {  // eight rows in flight per lane
+        int pidx[8];
+        uint4 v[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) pidx[u] = order[q + u];
+        for (int u = 0; u < 8; ++u) pidx[u] = order[q + u];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) v[u] = *(const uint4*)(Xc + (size_t)pidx[u] * D + 8 * oc);
+        for (int u = 0; u < 8; ++u) v[u] = *(const uint4*)(Xc + (size_t)pidx[u] * D + 8 * oc);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
           const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
           if constexpr (kKeys) {
 #pragma unroll
