@@ -156,6 +156,38 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def output_quality(S, w, Q, K, V, O_main, main_probes, dev, n_eval=2048):
+    """Normalised output error of the call (Table 2's metric) on n_eval strided rows per head,
+    its probe rows excluded, against exact dense rows from a second operator whose n_eval
+    uniform probe rows are computed densely; and the same error for the semantic partition
+    without repair (Table 2's baseline), giving the error reduction.  Outside the timed region."""
+    import numpy as np
+    ev = min(n_eval, w.N, 4096)
+    dense_op = S.SparsePR(w, device=dev, P=ev, probe_mode=configs.PROBE_UNIFORM, repair=0)
+    dense_op(Q, K, V)
+    ref = dense_op.query(S.Q_ODENSE).astype(np.float64)          # [BH, ev, d]
+    rows = dense_op.query(S.Q_PROBES)                            # [BH, ev] ascending tokens
+    sem = S.SparsePR(w, device=dev, partition=configs.PARTITION_SEMANTIC, repair=0)
+    O_sem = sem(Q, K, V, out_dtype=O_main.dtype)
+    torch.cuda.synchronize(dev)
+    BH = w.B * w.H
+    O1 = O_main.float().reshape(BH, w.N, w.d).cpu().numpy().astype(np.float64)
+    O0 = O_sem.float().reshape(BH, w.N, w.d).cpu().numpy().astype(np.float64)
+    sem_probes = sem.query(S.Q_PROBES)
+    e1, e0 = [], []
+    for h in range(BH):
+        keep = ~np.isin(rows[h], main_probes[h]) & ~np.isin(rows[h], sem_probes[h])
+        r, t = ref[h][keep], rows[h][keep]
+        den = np.linalg.norm(r, axis=1) + 1e-8
+        e1.append(np.linalg.norm(O1[h][t] - r, axis=1) / den)
+        e0.append(np.linalg.norm(O0[h][t] - r, axis=1) / den)
+    e1, e0 = np.concatenate(e1), np.concatenate(e0)
+    return {"mean_err": float(e1.mean()), "p99_err": float(np.percentile(e1, 99)),
+            "semantic_no_repair_mean_err": float(e0.mean()),
+            "error_reduction": float(1.0 - e1.mean() / e0.mean()),
+            "eval_rows": f"{ev} strided rows per head minus probe rows; output dtype of the call"}
+
+
 def km_rooflines(w, asg_ms, upd_ms, pk):
     """HBM rooflines of one key k-means assignment and one update launch (first iteration of
     the call): each reads every key once (2 d bytes, bf16) and writes (assignment) or reads
@@ -340,6 +372,10 @@ def run_ours(args, w, world, rank, local):
             "partition": part_stats,
             "clocks": clk,
         }
+        try:
+            line["quality"] = output_quality(S, w, Q, K, V, O, op.query(S.Q_PROBES), dev)
+        except Exception as exc:  # reported, never fatal: the timing above stands on its own
+            line["quality"] = {"error": str(exc)[:200]}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = oracle_sample(w, args.cpu_budget)
             line["cpu_baseline"].pop("s_per_call", None)

@@ -20,6 +20,11 @@ BF16 = 1
 
 PROBE_UNIFORM = 0
 PROBE_STRATIFIED = 1
+# partitions: response-coupled (SparsePR: keys by their responses to sampled queries, queries
+# by their normalised responses to the key-group centroids) or semantic (k-means on the raw
+# keys and the raw queries; the baseline of the paper's Table 2)
+PARTITION_RESPONSE = 0
+PARTITION_SEMANTIC = 1
 
 
 @dataclasses.dataclass(frozen=True)
@@ -48,6 +53,8 @@ class Workload:
     calls: int = 1                    # consecutive calls (streaming workload)
     noise: float = 0.5
     seed: int = 20261202              # k-means initial-point draw (SplitMix64 streams)
+    partition: int = 0                # PARTITION_RESPONSE (SparsePR) or PARTITION_SEMANTIC
+    repair: int = 1                   # 1: fit and add the probe-residual correction; 0: none
 
     @property
     def n_tiles(self) -> int:

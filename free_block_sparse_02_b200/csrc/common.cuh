@@ -35,6 +35,8 @@ struct Layout {
   float km_tol;
   double lambda;
   uint64_t seed;
+  int semantic;         // 1: k-means on the raw keys and queries (M = I, Gc = I, scale 1)
+  int repair;           // 1: fit and add the probe-residual correction
 
   // status + per-head statistics
   int* status;                    // [1]

@@ -116,6 +116,38 @@ __device__ bool chol_smem_tol(double* G, int n, int ld, double tol, double* diag
   return true;
 }
 
+// In-place Gauss-Jordan inverse of the symmetric positive definite n x n matrix in shared
+// memory (no pivoting: the pivots of an SPD matrix are the Cholesky pivots squared and stay
+// positive), two barriers per step.  False if a pivot is not positive (or not finite).
+__device__ bool gj_inverse_spd(double* G, int n, int ld) {
+  const int nthr = blockDim.x;
+  __syncthreads();
+  for (int k = 0; k < n; ++k) {
+    const double p = G[k * ld + k];
+    if (!(p > 0.0) || !isfinite(p)) return false;  // the same value in every thread
+    const double inv = 1.0 / p;
+    // every (i, j) off row and column k: reads row k and column k, which this phase leaves alone
+    // (warps over rows, lanes over columns)
+    const int nw = nthr >> 5, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = w; i < n; i += nw) {
+      if (i == k) continue;
+      const double f = G[i * ld + k] * inv;
+      for (int j = lane; j < n; j += 32)
+        if (j != k) G[i * ld + j] -= f * G[k * ld + j];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < n; e += nthr) {
+      if (e != k) {
+        G[k * ld + e] *= inv;
+        G[e * ld + k] *= -inv;
+      }
+    }
+    if (threadIdx.x == 0) G[k * ld + k] = inv;
+    __syncthreads();
+  }
+  return true;
+}
+
 // One CTA per head: lam, Cholesky with up to three x10 jitter retries, the d right-hand sides,
 // then the residual-span basis by column-pivoted Gram-Schmidt on S = R^T W R and A <- A U U^T.
 __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
@@ -149,7 +181,7 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
   for (; retries <= 3; ++retries) {
     for (int e = tid; e < n1 * n1; e += blockDim.x) G[e] = Gg[e] + ((e / n1) == (e % n1) ? lam : 0.0);
     __syncthreads();
-    ok = chol_smem_tol(G, n1, n1, 0.0, ldiag);
+    ok = gj_inverse_spd(G, n1, n1);
     if (ok) break;
     lam = lam > 0.0 ? lam * 10.0 : (tr > 0.0 ? 1e-12 * tr / n1 : 1e-30);
   }
@@ -165,36 +197,27 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
     }
     return;
   }
-  // solve L L^T X = B, 32 right-hand sides at a time: column c = tid / 8 of the chunk, eight
-  // threads (one warp quarter) share each row's dot product
+  // A = (G + lam I)^-1 B, 32 columns of B at a time staged in shared memory (all loads in
+  // flight together); thread = (row, column) of the chunk
   {
     const double* Bg = L.ridgeB + (size_t)bh * n1 * d;
     double* Y = G + n1 * n1;  // [n1][33]
-    const int col = tid >> 3, sub = tid & 7;
     for (int c0 = 0; c0 < d; c0 += 32) {
       __syncthreads();
-      for (int e = tid; e < n1 * 32; e += blockDim.x) Y[(e >> 5) * 33 + (e & 31)] = Bg[(e >> 5) * d + c0 + (e & 31)];
+      for (int e = tid; e < n1 * 32; e += blockDim.x) Y[(e >> 5) * 33 + (e & 31)] = Bg[(size_t)(e >> 5) * d + c0 + (e & 31)];
       __syncthreads();
-      for (int i = 0; i < n1; ++i) {  // L y = b, L_ik = G[k][i]
-        double part = 0.0;
-        for (int k = sub; k < i; k += 8) part += G[k * n1 + i] * Y[k * 33 + col];
-        part += __shfl_xor_sync(0xffffffffu, part, 4);
-        part += __shfl_xor_sync(0xffffffffu, part, 2);
-        part += __shfl_xor_sync(0xffffffffu, part, 1);
-        if (sub == 0) Y[i * 33 + col] = (Y[i * 33 + col] - part) / ldiag[i];
-        __syncwarp();
+      for (int e = tid; e < n1 * 32; e += blockDim.x) {
+        const int a = e >> 5, j = e & 31;
+        const double* gr = G + a * n1;
+        double acc0 = 0.0, acc1 = 0.0;
+        int k = 0;
+        for (; k + 1 < n1; k += 2) {
+          acc0 += gr[k] * Y[k * 33 + j];
+          acc1 += gr[k + 1] * Y[(k + 1) * 33 + j];
+        }
+        if (k < n1) acc0 += gr[k] * Y[k * 33 + j];
+        A[(size_t)a * d + c0 + j] = acc0 + acc1;
       }
-      for (int i = n1 - 1; i >= 0; --i) {  // L^T x = y, (L^T)_ik = L_ki = G[i][k]
-        double part = 0.0;
-        for (int k = i + 1 + sub; k < n1; k += 8) part += G[i * n1 + k] * Y[k * 33 + col];
-        part += __shfl_xor_sync(0xffffffffu, part, 4);
-        part += __shfl_xor_sync(0xffffffffu, part, 2);
-        part += __shfl_xor_sync(0xffffffffu, part, 1);
-        if (sub == 0) Y[i * 33 + col] = (Y[i * 33 + col] - part) / ldiag[i];
-        __syncwarp();
-      }
-      __syncthreads();
-      for (int e = tid; e < n1 * 32; e += blockDim.x) A[(e >> 5) * d + c0 + (e & 31)] = Y[(e >> 5) * 33 + (e & 31)];
     }
   }
   __syncthreads();
@@ -224,7 +247,10 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
     // (largest remaining squared norm cn, lowest index on ties); the unused columns remove
     // their component along the pivot column v_p (v_c -= (v_p . v_c / |v_p|^2) v_p, the pivot
     // column itself is normalised once at the end), tpc threads per column.
-    for (int e = tid; e < d * d; e += blockDim.x) S[e] = Sg[e];  // S[i*d + c]: column c, entry i
+    // S[i*ld + c]: column c, entry i; rows padded to d + 1 so the tpc threads of a column,
+    // on rows i, i + 1, ..., read different banks
+    const int ld = d + 1;
+    for (int e = tid; e < d * d; e += blockDim.x) S[(e / d) * ld + (e % d)] = Sg[e];
     __shared__ double cn[128];
     __shared__ int used[128];
     __shared__ double binv[128];
@@ -233,7 +259,7 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
     __syncthreads();
     for (int c = tid / tpc; c < d; c += blockDim.x / tpc) {
       double sacc = 0.0;
-      for (int i = sub; i < d; i += tpc) sacc += S[i * d + c] * S[i * d + c];
+      for (int i = sub; i < d; i += tpc) sacc += S[i * ld + c] * S[i * ld + c];
       for (int o = 1; o < tpc; o <<= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
       if (sub == 0) {
         cn[c] = sacc;
@@ -268,14 +294,14 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
         const bool act = !used[c] && c != bi;
         double dot = 0.0;
         if (act)
-          for (int i = sub; i < d; i += tpc) dot += S[i * d + bi] * S[i * d + c];
+          for (int i = sub; i < d; i += tpc) dot += S[i * ld + bi] * S[i * ld + c];
         for (int o = 1; o < tpc; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
         dot *= inv2;
         double sacc = 0.0;
         if (act)
           for (int i = sub; i < d; i += tpc) {
-            const double v = S[i * d + c] - dot * S[i * d + bi];
-            S[i * d + c] = v;
+            const double v = S[i * ld + c] - dot * S[i * ld + bi];
+            S[i * ld + c] = v;
             sacc += v * v;
           }
         for (int o = 1; o < tpc; o <<= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
@@ -291,7 +317,7 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
     }
     for (int e = tid; e < d * rank; e += blockDim.x) {  // normalise the basis columns
       const int i = e / rank, r = e % rank;
-      S[i * d + bcol[r]] *= binv[r];
+      S[i * ld + bcol[r]] *= binv[r];
     }
     __syncthreads();
     for (int r = 0; r < rank; ++r) basis[r] = bcol[r];
@@ -302,7 +328,7 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
     double* U = L.spanS + (size_t)bh * d * d;
     for (int e = tid; e < d * rank; e += blockDim.x) {
       const int i = e / rank, r = e % rank;
-      U[i * d + r] = S[i * d + basis[r]];
+      U[i * d + r] = S[i * (d + 1) + basis[r]];  // the Gram-Schmidt rows are padded to d + 1
     }
   }
   if (tid == 0) {
@@ -394,15 +420,34 @@ static sparsepr_status launch_apply(const Layout& L, void* O, cudaStream_t st) {
   return SPARSEPR_OK;
 }
 
+// No correction (repair off): A = 0, so unprobed rows keep O_sp and probe rows take O_dense.
+__global__ void zero_fit_kernel(Layout L) {
+  const int bh = blockIdx.x, n = (L.d + 1) * L.d;
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    L.A64[(size_t)bh * n + e] = 0.0;
+    L.A32[(size_t)bh * n + e] = 0.f;
+  }
+  if (threadIdx.x == 0) {
+    L.stats[bh].lambda = 0.0;
+    L.stats[bh].fit_retries = 0;
+    L.stats[bh].span_rank = 0;
+  }
+}
+
 sparsepr_status launch_fit_apply(const Layout& L, void* O, int out_dtype, cudaStream_t st) {
   const int d = L.d, n1 = d + 1;
-  if (L.P > 0) {
+  if (!L.repair) {
+    launch(zero_fit_kernel, L.BH, 256, 0, st, L);
+    SPR_LAUNCH_CHECK();
+  } else if (L.P > 0) {
     const size_t gsm = (size_t)(kRidgeChunk * n1 + kRidgeChunk * d + kRidgeChunk) * sizeof(double);
     cudaFuncSetAttribute(ridge_gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm);
     launch(ridge_gram_kernel, dim3(L.BH, (n1 + kRidgeRows - 1) / kRidgeRows), 256, gsm, st, L);
   }
-  const sparsepr_status s = launch_ridge_solve(L, st);
-  if (s != SPARSEPR_OK) return s;
+  if (L.repair) {
+    const sparsepr_status s = launch_ridge_solve(L, st);
+    if (s != SPARSEPR_OK) return s;
+  }
   if (L.dtype == SPARSEPR_BF16) return launch_apply_tc(L, O, out_dtype, st);
   if (out_dtype == SPARSEPR_F32)
     return d == 64 ? launch_apply<float, 64>(L, O, st) : launch_apply<float, 128>(L, O, st);

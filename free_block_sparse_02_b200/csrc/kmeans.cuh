@@ -75,7 +75,7 @@ __device__ void redecide_fp64(const Layout& L, int bh, const double* xs, int D, 
 #pragma unroll
   for (int k = 0; k < 4; ++k) xl[k] = lane + 32 * k < D ? xs[lane + 32 * k] : 0.0;
   double scale = 1.0;
-  if constexpr (!kKeys) {
+  if (!kKeys && !L.semantic) {  // the semantic partition clusters the raw queries (scale 1)
     const double* Gc = Gc_in ? Gc_in : L.Gc + (size_t)bh * D * D;
     double part = 0.0;
 #pragma unroll 4

@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(256) kmeans_redecide_kernel(const __nv_bfloat1
     if (nc <= 4) {
       int cand[4] = {(en.z >> 8) & 0x3FF, (en.z >> 18) & 0x3FF, en.w & 0xFFFF, (en.w >> 16) & 0xFFFF};
       double scale = 1.0;
-      if constexpr (!kKeys) {
+      if (!kKeys && !L.semantic) {
         double xl[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) xl[k] = lane + 32 * k < D ? xs[lane + 32 * k] : 0.0;
@@ -727,11 +727,18 @@ __global__ void __launch_bounds__(128, 1)
         tot += (double)qf;
       } else {
         const double ms = (double)qf;
-        const float inv = (float)(1.0 / sqrt(ms + 1e-12));
-        L.inv_rms[row] = inv;
-        L.inv_rms64[row] = 1.0 / sqrt(ms + 1e-12);
-        L.qxnorm[row] = sqrtf(nn) * inv;
-        tot += (double)L.Ck * ms / (ms + 1e-12);
+        if (L.semantic) {  // raw queries: scale 1, objective constant ||q||^2
+          L.inv_rms[row] = 1.f;
+          L.inv_rms64[row] = 1.0;
+          L.qxnorm[row] = sqrtf(nn);
+          tot += ms;
+        } else {
+          const float inv = (float)(1.0 / sqrt(ms + 1e-12));
+          L.inv_rms[row] = inv;
+          L.inv_rms64[row] = 1.0 / sqrt(ms + 1e-12);
+          L.qxnorm[row] = sqrtf(nn) * inv;
+          tot += (double)L.Ck * ms / (ms + 1e-12);
+        }
       }
     }
     tc_fence_before();

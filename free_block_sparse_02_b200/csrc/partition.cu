@@ -43,6 +43,13 @@ __global__ void __launch_bounds__(256) metric_kernel(Layout L, const T* __restri
   const int b = tid % d, lanes_per_b = 256 / d, r0 = tid / d;
   constexpr int kMaxOut = kMetricRows / 2;  // d = 128: 8 rows per thread; d = 64: 4
   const int nout = kMetricRows / lanes_per_b;
+  if (L.semantic) {  // the semantic partition clusters the raw keys: Euclidean metric M = I
+    for (int k = 0; k < nout; ++k) {
+      const int a = a0 + r0 + k * lanes_per_b;
+      L.M[((size_t)bh * d + a) * d + b] = a == b ? 1.0 : 0.0;
+    }
+    return;
+  }
   const T* q = Q + (size_t)bh * L.N * d;
   double acc[kMaxOut];
 #pragma unroll
@@ -87,6 +94,10 @@ __global__ void split_mat_kernel(const double* __restrict__ src, __nv_bfloat16* 
 __global__ void gc_kernel(Layout L) {
   const int bh = blockIdx.x, a = blockIdx.y, b = threadIdx.x, d = L.d;
   if (b >= d) return;
+  if (L.semantic) {  // raw queries: the row quadratic form is ||q||^2
+    L.Gc[((size_t)bh * d + a) * d + b] = a == b ? 1.0 : 0.0;
+    return;
+  }
   const double* C = L.kcent + (size_t)bh * L.Ck * d;
   double acc = 0.0;
   for (int j = 0; j < L.Ck; ++j) acc += C[(size_t)j * d + a] * C[(size_t)j * d + b];
@@ -136,11 +147,18 @@ __global__ void __launch_bounds__(256) rowqf_simt_kernel(Layout L, const T* __re
       contrib = part;
     } else {
       const double ms = (double)part;
-      const float inv = (float)(1.0 / sqrt(ms + 1e-12));
-      L.inv_rms[row] = inv;
-      L.inv_rms64[row] = 1.0 / sqrt(ms + 1e-12);
-      L.qxnorm[row] = sqrtf(nn) * inv;
-      contrib = (double)L.Ck * ms / (ms + 1e-12);
+      if (L.semantic) {  // raw queries: scale 1, objective constant ||q||^2
+        L.inv_rms[row] = 1.f;
+        L.inv_rms64[row] = 1.0;
+        L.qxnorm[row] = sqrtf(nn);
+        contrib = ms;
+      } else {
+        const float inv = (float)(1.0 / sqrt(ms + 1e-12));
+        L.inv_rms[row] = inv;
+        L.inv_rms64[row] = 1.0 / sqrt(ms + 1e-12);
+        L.qxnorm[row] = sqrtf(nn) * inv;
+        contrib = (double)L.Ck * ms / (ms + 1e-12);
+      }
     }
   }
   const double tot = block_sum(contrib, red);
@@ -210,6 +228,10 @@ __global__ void __launch_bounds__(128) qcent_init_kernel(Layout L, const T* __re
   __shared__ double red[4];
   const int bh = blockIdx.x, g = blockIdx.y, d = L.d, Ck = L.Ck, tid = threadIdx.x;
   const int t = L.init_ids[(size_t)bh * max(L.Ck, L.Cq) + g];
+  if (L.semantic) {  // raw queries: the drawn query itself is the centroid
+    if (tid < d) L.qU64[((size_t)bh * L.Cq + g) * d + tid] = (double)to_f32(Q[((size_t)bh * L.N + t) * d + tid]);
+    return;
+  }
   if (tid < d) qv[tid] = (double)to_f32(Q[((size_t)bh * L.N + t) * d + tid]);
   __syncthreads();
   const double rsd = 1.0 / sqrt((double)d);
@@ -388,6 +410,37 @@ __global__ void __launch_bounds__(128) qprep_kernel(Layout L, int it, int iters)
   const double rsd = 1.0 / sqrt((double)d);
   if (tid < kPrepGroups) cnt_s[tid] = (it > 0 && tid < ng) ? L.qcount[g0 + tid] : 0;
   __syncthreads();
+  if (L.semantic) {  // raw queries: u_g = c_g = S_g / n_g (groups that received points), bias ||c_g||^2
+    if (it > 0 && tid < d)
+      for (int g = 0; g < ng; ++g)
+        if (cnt_s[g] > 0) L.qU64[(g0 + g) * d + tid] = L.qsum[(g0 + g) * d + tid] / (double)cnt_s[g];
+    if (km_should_stop(L.qJ + (size_t)bh * L.iters_cap, it, iters, L.km_tol)) {
+      if (tid == 0 && blockIdx.y == 0) L.stop_at[bh * 2 + 1] = it;
+      return;
+    }
+    double cc[kPrepGroups];
+#pragma unroll
+    for (int g = 0; g < kPrepGroups; ++g) {
+      const bool on = tid < d && g < ng;
+      const double u = on ? L.qU64[(g0 + g) * d + tid] : 0.0;
+      cc[g] = u * u;
+      if (on) {
+        const size_t gg = g0 + g;
+        L.qU32[gg * d + tid] = (float)u;
+        split3(u, L.qWb, (size_t)L.BH * L.Cqp * d, ((size_t)bh * L.Cqp + g0i + g) * d + tid);
+        L.qsum[gg * d + tid] = 0.0;
+      }
+    }
+    block_sums8(cc, red, nn_s);
+    if (tid < ng) {
+      const size_t gg = g0 + tid;
+      L.qbias64[gg] = nn_s[tid];
+      L.qbias32[gg] = (float)nn_s[tid];
+      L.qcount[gg] = 0;
+      L.qwnorm[gg] = (float)sqrt(nn_s[tid]);
+    }
+    return;
+  }
   if (it > 0) {  // nu_g = C S_g / (sqrt(d) n_g) for the groups that received points
 #pragma unroll
     for (int g = 0; g < kPrepGroups; ++g)

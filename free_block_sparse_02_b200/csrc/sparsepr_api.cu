@@ -46,6 +46,9 @@ sparsepr_status validate(const sparsepr_config* c) {
   if (!isfinite(c->lambda) || c->km_iters < 1 || c->km_iters_warm < 0 || !isfinite(c->km_tol))
     return SPARSEPR_ERR_INVALID_ARG;
   if (c->km_iters > 10000 || c->km_iters_warm > 10000) return SPARSEPR_ERR_INVALID_ARG;
+  if (c->partition != SPARSEPR_PARTITION_RESPONSE && c->partition != SPARSEPR_PARTITION_SEMANTIC)
+    return SPARSEPR_ERR_INVALID_ARG;
+  if (c->repair != 0 && c->repair != 1) return SPARSEPR_ERR_INVALID_ARG;
   if ((double)c->B * c->H * c->N * 256.0 > 9.0e18) return SPARSEPR_ERR_INVALID_ARG;
   if (c->d != 64 && c->d != 128) return SPARSEPR_ERR_UNSUPPORTED;
   // rows of the [B*H*N, d] views are int32 in the kernels (tiles of 128 rows)
@@ -76,6 +79,8 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   L.km_tol = c.km_tol;
   L.lambda = c.lambda;
   L.seed = c.seed;
+  L.semantic = c.partition == SPARSEPR_PARTITION_SEMANTIC;
+  L.repair = c.repair;
   size_t off = 0;
   auto take = [&](auto*& ptr, size_t bytes) {
     using P_ = std::remove_reference_t<decltype(ptr)>;

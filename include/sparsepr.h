@@ -79,7 +79,14 @@ typedef struct sparsepr_config {
                                0 = every plan starts cold                                      */
   float km_tol;             /* stop when J_prev - J <= km_tol * J_prev; < 0 = never early      */
   uint64_t seed;            /* k-means initial points: SplitMix64 stream seed + 2*(b*H+h) + stage */
+  int32_t partition;        /* SPARSEPR_PARTITION_RESPONSE (the paper's response-coupled
+                               partition) or SPARSEPR_PARTITION_SEMANTIC (k-means on the raw keys
+                               and the raw queries: the semantic baseline of Table 2)           */
+  int32_t repair;           /* 1: fit and add the probe-residual correction (the paper's method);
+                               0: unprobed rows keep their block-sparse output                  */
 } sparsepr_config;
+
+enum { SPARSEPR_PARTITION_RESPONSE = 0, SPARSEPR_PARTITION_SEMANTIC = 1 };
 
 /* Per-head statistics, read with sparsepr_plan_query(SPARSEPR_Q_STATS). */
 typedef struct sparsepr_head_stats {

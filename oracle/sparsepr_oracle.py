@@ -398,13 +398,17 @@ class WarmState:
     query_centroids: np.ndarray   # (C_q, C_k) normalised response space
 
 
-def outputs_given_partition(q, k, v, qlabels, klabels, route, probes, weights, lam_cfg):
-    """Steps 6-9 for a given partition, route table and probe set."""
+def outputs_given_partition(q, k, v, qlabels, klabels, route, probes, weights, lam_cfg, repair=1):
+    """Steps 6-9 for a given partition, route table and probe set (repair=0: no correction;
+    unprobed rows keep their sparse output, probe rows their exact one)."""
     osp = sparse_attention(q, k, v, qlabels, klabels, route)
     odense = attention(q[probes], k, v)
-    A, lam = ridge_fit(osp[probes], odense, weights, lam_cfg)
-    if len(probes):
-        A = restrict_to_residual_span(A, odense - osp[probes], weights)
+    if repair:
+        A, lam = ridge_fit(osp[probes], odense, weights, lam_cfg)
+        if len(probes):
+            A = restrict_to_residual_span(A, odense - osp[probes], weights)
+    else:
+        A, lam = np.zeros((q.shape[1] + 1, q.shape[1])), 0.0
     O = apply_correction(osp, A)
     O[probes] = odense
     return dict(osp=osp, odense=odense, A=A, lam=lam, O=O)
@@ -414,7 +418,10 @@ def call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int,
               warm: Optional[WarmState] = None, keep_history: bool = False,
               compute_outputs: bool = True) -> dict:
     """One (batch, head) of one call.  cfg needs: s, n_kgroups, n_qgroups, density, fixed_k,
-    P, probe_mode (0 uniform, 1 stratified), lam, km_iters, km_iters_warm, km_tol, seed."""
+    P, probe_mode (0 uniform, 1 stratified), lam, km_iters, km_iters_warm, km_tol, seed, and
+    optionally partition (0 response-coupled, 1 semantic) and repair (1 correct, 0 not)."""
+    if getattr(cfg, "partition", 0) == 1:
+        return semantic_call_head(q, k, v, cfg, bh, compute_outputs=compute_outputs)
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -472,8 +479,69 @@ def call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int,
                scores=S, kappa=kappa, route=route, sparse_pairs=sparse_pairs, density=density,
                probes=probes, weights=weights)
     if compute_outputs:
-        out.update(outputs_given_partition(q, k, v, qlabels, klabels, route, probes, weights, cfg.lam))
+        out.update(outputs_given_partition(q, k, v, qlabels, klabels, route, probes, weights, cfg.lam,
+                                           repair=getattr(cfg, "repair", 1)))
     return out
+
+
+def route_and_probe(q, klabels, qlabels, kcent, cfg):
+    """Steps 5 and 7 for a given partition: routes, realised density and probes."""
+    N = q.shape[0]
+    Ck, Cq = cfg.n_kgroups, cfg.n_qgroups
+    m = np.bincount(klabels, minlength=Ck)
+    n = np.bincount(qlabels, minlength=Cq)
+    S = routing_scores(query_responses(q, kcent), qlabels, Cq, m)
+    kappa = per_row_key_budget(cfg.density, N, cfg.s, Ck, cfg.P)
+    route = np.zeros((Cq, Ck), dtype=bool)
+    for g in range(Cq):
+        if n[g] > 0:
+            route[g, route_group(S[g], m, cfg.fixed_k, kappa)] = True
+    sparse_pairs = int(sum(int(n[g]) * int(m[route[g]].sum()) for g in range(Cq)))
+    density = (cfg.s * N + Ck * N + cfg.P * N + sparse_pairs) / float(N) ** 2
+    if cfg.probe_mode == 0:
+        probes, weights = probes_uniform(N, cfg.P)
+    else:
+        probes, weights = probes_stratified(qlabels, Cq, cfg.P)
+    return dict(ksizes=m, qsizes=n, scores=S, kappa=kappa, route=route, sparse_pairs=sparse_pairs,
+                density=density, probes=probes, weights=weights)
+
+
+def semantic_call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int,
+                       compute_outputs: bool = True) -> dict:
+    """The semantic partition of the paper's Table 2 baseline ("semantic block-sparse
+    attention"): Lloyd's k-means on the raw keys and on the raw queries (squared Euclidean
+    distance, the same seeded initial points, limits and stop rule as the response-coupled
+    partition), then the same routing, probes and (if cfg.repair) correction.
+    Reading: "semantic" groups tokens by their own feature vectors, with no response coupling."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    N = q.shape[0]
+    Ck, Cq = cfg.n_kgroups, cfg.n_qgroups
+    seed = getattr(cfg, "seed", 0)
+    tol = float(np.float32(cfg.km_tol))
+    ids = kmeans_init_ids(N, Ck, stream_seed(seed, bh, 0))
+    kk = lloyd(k, k[ids], cfg.km_iters, tol)
+    ids = kmeans_init_ids(N, Cq, stream_seed(seed, bh, 1))
+    qq = lloyd(q, q[ids], cfg.km_iters, tol)
+    out = dict(klabels=kk.labels, kcent=kk.centroids, kmeans_k=kk, qlabels=qq.labels, qcent=qq.centroids,
+               kmeans_q=qq)
+    out.update(route_and_probe(q, kk.labels, qq.labels, kk.centroids, cfg))
+    if compute_outputs:
+        out.update(outputs_given_partition(q, k, v, qq.labels, kk.labels, out["route"], out["probes"],
+                                           out["weights"], cfg.lam, repair=getattr(cfg, "repair", 1)))
+    return out
+
+
+def mean_error(O: np.ndarray, Oref: np.ndarray, rows: np.ndarray) -> float:
+    """Mean normalised attention-output error over the given rows (Table 2's metric)."""
+    return float(row_errors(O[rows], Oref[rows]).mean())
+
+
+def error_reduction(err_method: float, err_baseline: float) -> float:
+    """Relative error reduction of a method over a baseline, as in the abstract's 61.6-90.5%:
+    1 - err_method / err_baseline."""
+    return 1.0 - err_method / err_baseline
 
 
 def call(Q, K, V, cfg, warm: Optional[Sequence[WarmState]] = None, heads=None, **kw) -> List[dict]:

@@ -10,6 +10,8 @@ import json
 import math
 import os
 
+import types
+
 import numpy as np
 import pytest
 import scipy.linalg
@@ -386,6 +388,46 @@ def test_call_partition_is_consistent():
 
 def test_table2_error_reduction_arithmetic():
     t = _gold("table2_error_reduction.json")
-    red = [100 * (1 - b / a) for a, b in zip(t["semantic_mean"], t["sparsepr_mean"])]
+    red = [100 * O.error_reduction(b, a) for a, b in zip(t["semantic_mean"], t["sparsepr_mean"])]
     lo, hi = t["stated_reduction_range_pct"]
     assert round(min(red), 1) == lo and round(max(red), 1) == hi
+
+
+def test_mean_error_is_the_row_error_mean():
+    rng = np.random.default_rng(3)
+    O_, R_ = rng.standard_normal((6, 4)), rng.standard_normal((6, 4))
+    rows = np.array([0, 2, 5])
+    expect = np.mean([np.linalg.norm(O_[i] - R_[i]) / (np.linalg.norm(R_[i]) + 1e-8) for i in rows])
+    assert np.isclose(O.mean_error(O_, R_, rows), expect, rtol=1e-14)
+
+
+def test_repair_off_keeps_sparse_rows_and_exact_probes():
+    w = types.SimpleNamespace(s=8, n_kgroups=4, n_qgroups=4, density=0.5, fixed_k=2, P=6, probe_mode=0,
+                              lam=-1.0, km_iters=4, km_iters_warm=0, km_tol=-1.0, seed=5, repair=0)
+    q, k, v = (np.random.default_rng(i).standard_normal((64, 8)) for i in range(3))
+    r = O.call_head(q, k, v, w, 0)
+    unprobed = np.setdiff1d(np.arange(64), r["probes"])
+    assert np.array_equal(r["O"][unprobed], r["osp"][unprobed])
+    assert np.array_equal(r["O"][r["probes"]], r["odense"])
+    assert not np.any(r["A"])
+
+
+def test_semantic_partition_is_kmeans_on_the_raw_inputs():
+    """The semantic baseline's key groups are Lloyd's k-means of the raw keys (the same seeded
+    initial points and limits), pinned against scikit-learn from those initial centroids."""
+    from sklearn.cluster import KMeans
+    w = types.SimpleNamespace(s=8, n_kgroups=5, n_qgroups=3, density=0.5, fixed_k=2, P=6, probe_mode=0,
+                              lam=-1.0, km_iters=50, km_iters_warm=0, km_tol=-1.0, seed=9, partition=1,
+                              repair=0)
+    rng = np.random.default_rng(4)
+    centres = 4 * rng.standard_normal((5, 8))
+    k = centres[rng.integers(0, 5, 80)] + 0.3 * rng.standard_normal((80, 8))
+    q = centres[rng.integers(0, 5, 80)] + 0.3 * rng.standard_normal((80, 8))
+    v = rng.standard_normal((80, 8))
+    r = O.call_head(q, k, v, w, 2)
+    ids = O.kmeans_init_ids(80, 5, O.stream_seed(9, 2, 0))
+    km = KMeans(n_clusters=5, init=k[ids], n_init=1, max_iter=50, tol=0.0, algorithm="lloyd").fit(k)
+    assert np.array_equal(r["klabels"], km.labels_)
+    ids = O.kmeans_init_ids(80, 3, O.stream_seed(9, 2, 1))
+    kq = KMeans(n_clusters=3, init=q[ids], n_init=1, max_iter=50, tol=0.0, algorithm="lloyd").fit(q)
+    assert np.array_equal(r["qlabels"], kq.labels_)
