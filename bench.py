@@ -102,7 +102,9 @@ def workload_config(w, extra=None):
     c = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "density": w.density, "s": w.s,
          "n_kgroups": w.n_kgroups, "n_qgroups": w.n_qgroups, "P": w.P,
          "probes": "stratified" if w.probe_mode else "uniform", "km_iters": w.km_iters, "km_tol": w.km_tol,
-         "generator": f"clustered Gaussian tiles {w.tile} on grid {w.grid}" + (" + 3D RoPE" if w.rope else "")}
+         "generator": (f"clustered Gaussian tiles {w.tile} on grid {w.grid}" if w.recipe == "tiles" else
+                       f"smooth random field, length scales {w.field_ell}, logit contrast {w.field_tau}, "
+                       f"value offset {w.value_offset}, on grid {w.grid}") + (" + 3D RoPE" if w.rope else "")}
     if extra:
         c.update(extra)
     return c
@@ -398,6 +400,8 @@ def main():
                     help="run the workload on this many heads instead (a smaller case for profilers)")
     ap.add_argument("--density", type=float, default=0.0, help="override the density target (sweeps)")
     ap.add_argument("--probes", type=int, default=-1, help="override the probe budget P (sweeps)")
+    ap.add_argument("--inputs", default="tiles", choices=["tiles", "field"],
+                    help="input recipe: clustered Gaussian tiles (the workloads' own) or a smooth random field")
     args = ap.parse_args()
     world, rank, local = dist_env()
     w = configs.workload(args.workload)
@@ -407,6 +411,8 @@ def main():
         w = w.replace(density=args.density)
     if args.probes >= 0:
         w = w.replace(P=args.probes)
+    if args.inputs != w.recipe:
+        w = w.replace(recipe=args.inputs)
     if args.impl == "reference":
         run_reference(args, w, world, rank)
     else:

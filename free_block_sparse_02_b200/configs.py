@@ -55,6 +55,10 @@ class Workload:
     seed: int = 20261202              # k-means initial-point draw (SplitMix64 streams)
     partition: int = 0                # PARTITION_RESPONSE (SparsePR) or PARTITION_SEMANTIC
     repair: int = 1                   # 1: fit and add the probe-residual correction; 0: none
+    recipe: str = "tiles"             # input generator: "tiles" (clustered Gaussian) or "field"
+    field_tau: float = 4.0            # "field": peak logit contrast of the smooth field
+    field_ell: Tuple[float, float, float] = (2.0, 6.0, 6.0)  # "field": length scales (t, y, x)
+    value_offset: float = 1.0         # "field": scale of the value offset shared by all tokens
 
     @property
     def n_tiles(self) -> int:

@@ -17,6 +17,18 @@ Recipe (per head, one independent PCG64 stream per (b, h)):
     generator, not of the method.
   * streaming workloads: call c > 0 is x_c = 0.95 x_{c-1} + 0.31 N(0, I) for each of q, k, v
     (q-noise, k-noise, v-noise drawn in that order per call).
+
+Second recipe, "field" (opt-in; smooth activations whose sparse residual an affine map of the
+sparse output can predict, the regime of the paper's model activations):
+  * f(p) = sqrt(2/F) sum_j W_j cos(omega_j . p + b_j) over the token's (t, y, x) grid position p,
+    F = 256 random Fourier features, omega_j ~ N(0, diag(1/ell^2)), b_j ~ U[0, 2 pi),
+    W_j ~ N(0, I_d): a Gaussian random field, unit variance per dimension, correlation
+    exp(-|dp / ell|^2 / 2) between tokens
+  * q = a f(p) + noise N(0, I),  k = a f(p) + noise N(0, I),  a^2 = tau / sqrt(d), so that the
+    logit q.k / sqrt(d) of two nearby tokens is about tau above that of two distant ones
+  * v = g(p) + noise N(0, I) + c u, g a second independent field, u ~ N(0, I_d) one offset
+    shared by every token of the head
+  draws in the order (omega, b, W) of f, q-noise, k-noise, (omega, b, W) of g, v-noise, u.
 Values are produced in float64 and cast once to the workload dtype; the CUDA path and the
 oracle both consume the cast tensors.
 
@@ -74,6 +86,39 @@ def _apply_rope(x: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
     return out
 
 
+N_FEATURES = 256
+
+
+def grid_positions(w: Workload) -> np.ndarray:
+    """(N, 3) float64 (t, y, x) grid coordinates of the tokens in raster order."""
+    T, Y, X = w.grid
+    t, y, x = np.meshgrid(np.arange(T), np.arange(Y), np.arange(X), indexing="ij")
+    return np.stack([t.reshape(-1), y.reshape(-1), x.reshape(-1)], axis=1).astype(np.float64)
+
+
+def _random_field(rng: np.random.Generator, pos: np.ndarray, d: int, ell) -> np.ndarray:
+    """Random-Fourier-feature Gaussian field over the grid: (N, d), unit variance per dim."""
+    omega = rng.standard_normal((N_FEATURES, 3)) / np.asarray(ell, dtype=np.float64)[None, :]
+    phase = rng.uniform(0.0, 2.0 * np.pi, N_FEATURES)
+    W = rng.standard_normal((N_FEATURES, d))
+    out = np.empty((pos.shape[0], d))
+    for s in range(0, pos.shape[0], 16384):      # bounded temporaries on the large grids
+        out[s:s + 16384] = np.cos(pos[s:s + 16384] @ omega.T + phase) @ W
+    return out * np.sqrt(2.0 / N_FEATURES)
+
+
+def _field_qkv(w: Workload, rng: np.random.Generator):
+    pos = grid_positions(w)
+    f = _random_field(rng, pos, w.d, w.field_ell)
+    a = np.sqrt(w.field_tau / np.sqrt(w.d))
+    q = a * f + w.noise * rng.standard_normal((w.N, w.d))
+    k = a * f + w.noise * rng.standard_normal((w.N, w.d))
+    g = _random_field(rng, pos, w.d, w.field_ell)
+    v = g + w.noise * rng.standard_normal((w.N, w.d))
+    v += w.value_offset * rng.standard_normal((1, w.d))
+    return q, k, v
+
+
 def _head_stream(w: Workload, variant: int, bh: int) -> np.random.Generator:
     ss = np.random.SeedSequence(entropy=SEED_BASE + w.index, spawn_key=(variant,))
     child = ss.spawn(w.B * w.H)[bh]
@@ -85,12 +130,17 @@ def head_calls_f64(w: Workload, b: int, h: int, variant: int = 0,
     """Yield float64 (q, k, v), each (N, d), for consecutive calls of head (b, h)."""
     calls = w.calls if calls is None else calls
     rng = _head_stream(w, variant, b * w.H + h)
-    tiles = token_tiles(w)
-    assert tiles.shape[0] == w.N
-    mu = 2.0 * rng.standard_normal((w.n_tiles, w.d))
-    q = mu[tiles] + w.noise * rng.standard_normal((w.N, w.d))
-    k = mu[tiles] + w.noise * rng.standard_normal((w.N, w.d))
-    v = rng.standard_normal((w.N, w.d))
+    if w.recipe == "field":
+        q, k, v = _field_qkv(w, rng)
+    elif w.recipe == "tiles":
+        tiles = token_tiles(w)
+        assert tiles.shape[0] == w.N
+        mu = 2.0 * rng.standard_normal((w.n_tiles, w.d))
+        q = mu[tiles] + w.noise * rng.standard_normal((w.N, w.d))
+        k = mu[tiles] + w.noise * rng.standard_normal((w.N, w.d))
+        v = rng.standard_normal((w.N, w.d))
+    else:
+        raise ValueError(f"unknown input recipe {w.recipe!r}")
     if w.rope:
         cos, sin = _rope_angles(w)
         q = _apply_rope(q, cos, sin)

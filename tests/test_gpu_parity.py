@@ -226,6 +226,8 @@ EDGE = {
     # fewer groups than one 32-column TMEM chunk, and more point tiles than SMs (both accumulators)
     "few-groups-many-tiles": dict(base=1, grid=(16, 32, 32), heads=2, s=64, n_kgroups=8, n_qgroups=12, P=64,
                                   km_iters=6),
+    # smooth-field inputs: no cluster structure, so more points sit near group boundaries
+    "field-inputs": dict(base=1, grid=(8, 16, 32), heads=2, recipe="field"),
 }
 
 
