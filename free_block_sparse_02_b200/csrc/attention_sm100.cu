@@ -39,22 +39,59 @@ constexpr int kSubRows = 32;    // rows per TMA box of K/V (32: measured faster 
 constexpr int kSubPerTile = kTcTileN / kSubRows;
 constexpr int kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kExpPolyEvery = 0;           // 1 in n exponential pairs on the FMA pipe (0: none; measured
-                                           // slower on sm_100a, where the exponentials are not the bound)
+constexpr int kExpPolyEvery = 0;           // in tiles whose keys are all real, 1 in n exponential
+                                           // pairs runs on the FMA pipe (0: none)
 
-// 2^x on the FMA pipe for x <= kRescaleThreshold (0 below -125, so -inf gives 0): Cody-Waite
-// style reduction x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low mantissa
-// bits) and f in [-1/2, 1/2], then a cubic in f fitted to 2^f by least squares on relative error
-// at Chebyshev nodes with Lawson reweighting (max relative error 7.5e-5, far below the bf16
-// rounding of P), and n added to the exponent field.
-__device__ __forceinline__ float exp2_poly(float x) {
-  const float xc = fmaxf(x, -125.f);
-  const float t = xc + 12582912.f;
-  const float f = xc - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0.0551716648f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
-  const float y = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-  return x < -125.f ? 0.f : y;
+// 2^x for a pair of x <= kRescaleThreshold on the FMA pipe (f32x2), for x >= -125 (smaller x
+// give 2^-125 instead of 0: far below the bf16 rounding of P and of any row sum, which is
+// >= 1).  Cody-Waite style reduction x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in
+// the low mantissa bits) and f in [-1/2, 1/2], then a cubic in f fitted to 2^f by least
+// squares on relative error at Chebyshev nodes with Lawson reweighting (max relative error
+// 7.5e-5), and n added to the exponent field.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t shifter = f2_pack(12582912.f, 12582912.f);
+  const uint64_t t = f2_add(xc, shifter);
+  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);
+  uint64_t p = f2_fma(f2_pack(0.0551716648f, 0.0551716648f), f, f2_pack(0.2426111251f, 0.2426111251f));
+  p = f2_fma(p, f, f2_pack(0.6932609677f, 0.6932609677f));
+  p = f2_fma(p, f, f2_pack(0.9999280572f, 0.9999280572f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+                 __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
 }
+
+// Exponentials of one half row of S (64 scores in sv, as fp32 bits) into 32 packed bf16 pairs,
+// adding them to the row sum.  kFull: every key of the tile is real (no -inf scores), so the
+// polynomial pairs may run; otherwise every exponential is on the special-function unit,
+// where 2^-inf = 0 exactly.
+template <bool kFull>
+__device__ __forceinline__ void exp_half(const uint32_t (&sv)[64], float scale2, float neg_m, uint32_t (&pk)[32],
+                                         uint64_t (&acc)[2]) {
+  const uint64_t sc = f2_pack(scale2, scale2), nm = f2_pack(neg_m, neg_m);
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1])), sc, nm);
+    uint64_t e;
+    if (kFull && kExpPolyEvery > 0 && (k % (kExpPolyEvery > 0 ? kExpPolyEvery : 1)) == kExpPolyEvery - 1) {
+      e = exp2_poly2(x);
+    } else {
+      float x0, x1;
+      f2_unpack(x, x0, x1);
+      e = f2_pack(ex2(x0), ex2(x1));
+    }
+    acc[k & 1] = f2_add(acc[k & 1], e);
+    float p0, p1;
+    f2_unpack(e, p0, p1);
+    pk[k] = pack_bf16x2(p0, p1);
+  }
+}
+
 static_assert(kAttnTileMTc == 2 * kTcTileM, "a work item is two MMA tiles");
 
 template <int D>
@@ -385,12 +422,18 @@ __global__ void __launch_bounds__(384, 1)
           for (int k = 0; k < kTcTileN; ++k)
             if ((k & (kSubRows - 1)) >= valid[k / kSubRows]) sv[k] = __float_as_uint(-INFINITY);
         }
+        // eight chains over columns c + 8i, three inputs per maximum
         float mx[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sv[k]);
+        for (int c = 0; c < 8; ++c) {
+          float m = fmax3(__uint_as_float(sv[c]), __uint_as_float(sv[c + 8]), __uint_as_float(sv[c + 16]));
 #pragma unroll
-        for (int k = 8; k < kTcTileN; ++k) mx[k & 7] = fmaxf(mx[k & 7], __uint_as_float(sv[k]));
-        tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+          for (int i = 3; i + 1 < kTcTileN / 8; i += 2)
+            m = fmax3(m, __uint_as_float(sv[c + 8 * i]), __uint_as_float(sv[c + 8 * i + 8]));
+          if ((kTcTileN / 8 - 3) % 2) m = fmaxf(m, __uint_as_float(sv[c + kTcTileN - 8]));
+          mx[c] = m;
+        }
+        tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7]));
       }
       tmax *= scale2;
       // lazy rescale: move the running max only when this tile exceeds it by > 2^8
@@ -424,39 +467,32 @@ __global__ void __launch_bounds__(384, 1)
       m_used = m_new;
       // pass 2: P = 2^(s*scale - m) as packed bf16 over the first 64 columns of S_t, 64 keys at
       // a time (each half is read before its 32 packed columns overwrite already-read ones).
-      // Padded keys are set to -inf first, so their probability is exactly 0.  Every
-      // kExpPolyEvery-th pair of exponentials runs on the FMA pipe (exp2_poly) to relieve the
-      // special-function unit.
+      // Padded keys are set to -inf first, so their probability is exactly 0.
       const float neg_m = -m_used;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t sv[64];
         tmem_ld32(tS + h * 64, *reinterpret_cast<uint32_t(*)[32]>(sv));
         tmem_ld32(tS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
         tmem_wait_ld();
-        if (!full) {
+        uint32_t pk[32];
+        if (full) {
+          exp_half<true>(sv, scale2, neg_m, pk, acc);
+        } else {
 #pragma unroll
           for (int k = 0; k < 64; ++k) {
             const int col = h * 64 + k;
             if ((col & (kSubRows - 1)) >= valid[col / kSubRows]) sv[k] = __float_as_uint(-INFINITY);
           }
-        }
-        uint32_t pk[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float x0 = fmaf(__uint_as_float(sv[2 * k]), scale2, neg_m);
-          const float x1 = fmaf(__uint_as_float(sv[2 * k + 1]), scale2, neg_m);
-          constexpr int kEvery = kExpPolyEvery > 0 ? kExpPolyEvery : 1;
-          const bool poly = kExpPolyEvery > 0 && (k % kEvery) == kEvery - 1;
-          const float p0 = poly ? exp2_poly(x0) : ex2(x0);
-          const float p1 = poly ? exp2_poly(x1) : ex2(x1);
-          ls[k & 3] += p0 + p1;
-          pk[k] = pack_bf16x2(p0, p1);
+          exp_half<false>(sv, scale2, neg_m, pk, acc);
         }
         tmem_st32(tS + h * 32, pk);
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      float a0, a1, a2, a3;
+      f2_unpack(acc[0], a0, a1);
+      f2_unpack(acc[1], a2, a3);
+      l += (a0 + a1) + (a2 + a3);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full + t);

@@ -49,6 +49,9 @@ constexpr int kKmThreads = 384;   // warp 0 TMA, warp 1 MMA, warps 4..11 epilogu
 constexpr int kKmUpdThreads = 512;
 constexpr int kKmMaxStages = 4;
 constexpr int kKmUpdChunk = 16384;  // points of one head sorted and summed at a time by the update
+constexpr int kKmUpdItemRows = 64;   // rows of one accumulation item: a group's run is split into
+                                     // pieces of at most this many rows, summed by different warps
+__host__ __device__ constexpr int km_upd_max_items(int C) { return kKmUpdChunk / kKmUpdItemRows + C; }
 
 __host__ __device__ inline int km_tc_tmem_cols(int n) {
   int c = 32;
@@ -67,7 +70,8 @@ __host__ inline size_t km_assign_smem(int D, int Np, int stages) {
 // offsets and cursors.
 __host__ inline size_t km_update_smem(int D, int C) {
   (void)D;
-  return (size_t)2 * kKmUpdChunk * 4 /*labels, order*/ + (size_t)(3 * C + 1) * 4;
+  return (size_t)2 * kKmUpdChunk * 4 /*labels, order*/ + (size_t)(3 * C + 2) * 4 /*offs, cursor, ioff*/ +
+         (size_t)2 * km_upd_max_items(C) * 4 /*item group, item start*/;
 }
 
 __device__ __forceinline__ int km_tiles_per_head(const Layout& L) { return (L.N + kKmTile - 1) / kKmTile; }
@@ -477,7 +481,9 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
   int* order = lab + kKmUpdChunk;              // [kKmUpdChunk] chunk points sorted by label
   int* offs = order + kKmUpdChunk;             // [C + 1] start of each label's run
   int* cursor = offs + (C + 1);                // [C] histogram, then next slot per label
-  int* byrun = cursor + C;                     // [C] groups by decreasing run length
+  int* ioff = cursor + C;                      // [C + 1] first accumulation item of each label
+  int* item_g = ioff + (C + 1);                // [km_upd_max_items] group of each item
+  int* item_s = item_g + km_upd_max_items(C);  // [km_upd_max_items] first slot of `order` of each item
   __shared__ int s_next;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -516,25 +522,35 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
       }
     }
     __syncthreads();
-    if (warp == 0) {  // exclusive prefix over the groups, and the counts
-      int run = 0;
+    if (warp == 0) {  // exclusive prefixes over the groups (slots and items), and the counts
+      int run = 0, irun = 0;
       for (int c0 = 0; c0 < C; c0 += 32) {
         const int j = c0 + lane;
         const int v = j < C ? cursor[j] : 0;
-        int x = v;
+        const int nv = (v + kKmUpdItemRows - 1) / kKmUpdItemRows;
+        int x = v, y = nv;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, x, o);
-          if (lane >= o) x += y;
+          const int a = __shfl_up_sync(0xffffffffu, x, o);
+          const int b = __shfl_up_sync(0xffffffffu, y, o);
+          if (lane >= o) {
+            x += a;
+            y += b;
+          }
         }
         if (j < C) {
           offs[j] = run + x - v;
           cursor[j] = run + x - v;
+          ioff[j] = irun + y - nv;
           if (v) atomicAdd(counts_all + (size_t)bh * C + j, v);
         }
         run += __shfl_sync(0xffffffffu, x, 31);
+        irun += __shfl_sync(0xffffffffu, y, 31);
       }
-      if (lane == 0) offs[C] = run;
+      if (lane == 0) {
+        offs[C] = run;
+        ioff[C] = irun;
+      }
     }
     __syncthreads();
     // scatter: lanes with the same label take consecutive slots from one atomic
@@ -551,38 +567,33 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
         order[base + __popc(same & ((1u << lane) - 1))] = i;
       }
     }
-    // groups by decreasing run length (longest first), for the dynamic schedule below
+    // the item table: group g's run is cut into pieces of at most kKmUpdItemRows rows
     for (int g = tid; g < C; g += kKmUpdThreads) {
-      const int sz = offs[g + 1] - offs[g];
-      int rk = 0;
-      if (C <= 256)
-        for (int h = 0; h < C; ++h) {
-          const int sh = offs[h + 1] - offs[h];
-          rk += sh > sz || (sh == sz && h < g);
-        }
-      else
-        rk = g;
-      byrun[rk] = g;
+      const int q0 = offs[g], q1 = offs[g + 1];
+      for (int i = ioff[g], q = q0; q < q1; ++i, q += kKmUpdItemRows) {
+        item_g[i] = g;
+        item_s[i] = q;
+      }
     }
     if (tid == 0) s_next = 0;
     __syncthreads();
-    // accumulation: a warp takes the next 32 / octs groups (longest runs first); within it,
-    // item = (group, eight dimensions), consecutive lanes reading consecutive 16-byte pieces of
-    // the same rows; each item's run is summed in fp64 registers
+    // accumulation: a warp takes the next 32 / octs items; within it, consecutive lanes read
+    // consecutive 16-byte pieces (eight dimensions) of the same rows; each item's rows are summed
+    // in fp64 registers and added to the group's sums with one atomic per dimension
     const __nv_bfloat16* Xc = X + row0 * D;
     const double* sig = L.inv_rms64 + row0;
     double* sums = sums_all + (size_t)bh * C * D;
     const int gpw = 32 / octs;
+    const int nitems = ioff[C];
     while (true) {
       int k = 0;
       if (lane == 0) k = atomicAdd(&s_next, 1);
       k = __shfl_sync(0xffffffffu, k, 0);
-      if (k * gpw >= C) break;  // the same for the whole warp
-      const int gi = k * gpw + lane / octs;
-      if (gi >= C) continue;
-      const int g = byrun[gi], oc = lane % octs;
-      const int q0 = offs[g], q1 = offs[g + 1];
-      if (q0 == q1) continue;
+      if (k * gpw >= nitems) break;  // the same for the whole warp
+      const int ii = k * gpw + lane / octs;
+      if (ii >= nitems) continue;
+      const int g = item_g[ii], oc = lane % octs;
+      const int q0 = item_s[ii], q1 = min(q0 + kKmUpdItemRows, offs[g + 1]);
       double r[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) r[k] = 0.0;
