@@ -50,6 +50,7 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bflo
 
 template <typename To, int D>
 __global__ void __launch_bounds__(kApThreads, 1) apply_tc_kernel(Layout L, To* __restrict__ O, int G) {
+  pdl_entry();
   using C = ApCfg<D>;
   const int tph = (L.N + kApTile - 1) / kApTile;
   const long long T = (long long)L.BH * tph;

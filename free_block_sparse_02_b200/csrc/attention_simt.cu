@@ -35,6 +35,7 @@ __device__ __forceinline__ int virt_to_row(int v, const int* segpre, const int* 
 // mode 1: probe rows, blockIdx.x = 64-row tile of the head's probe rows, all keys.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) attn_simt_kernel(Layout L, int mode) {
+  pdl_entry();
   constexpr int DP = D + 1;
   extern __shared__ float sm[];
   float* Qs = sm;                              // [64][DP]

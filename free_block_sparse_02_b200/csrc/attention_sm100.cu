@@ -155,6 +155,7 @@ __global__ void __launch_bounds__(384, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQprobe,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, Layout L,
                    int probe_items_per_head, int sparse_items_per_head) {
+  pdl_entry();
   using C = TcCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);

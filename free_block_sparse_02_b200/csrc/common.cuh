@@ -179,11 +179,31 @@ __host__ __device__ inline size_t elt_size(int dtype) { return dtype == SPARSEPR
 // Kernels launched by this library since it was loaded (read by sparsepr_launch_count).
 extern std::atomic<long long> g_launches;
 
-// Every kernel of the library is launched through this helper, which counts the launch.
+// Programmatic dependent launch.  Every kernel of the library starts with pdl_entry(): it waits
+// until the kernels before it in the stream have completed and their memory is visible (the
+// same ordering as a plain launch), then allows the next kernel's CTAs to be launched.  The
+// launch work and CTA start of kernel n+1 so overlap the tail of kernel n.
+__device__ __forceinline__ void pdl_entry() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Every kernel of the library is launched through this helper, which counts the launch and
+// marks it as programmatically dependent on the previous kernel in the stream.
 template <typename... KArgs, typename... Args>
 inline void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                    Args&&... args) {
-  kernel<<<grid, block, smem, st>>>(std::forward<Args>(args)...);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
   g_launches.fetch_add(1, std::memory_order_relaxed);
 }
 

@@ -25,6 +25,7 @@ constexpr int kRidgeChunk = 32;  // probes staged per step
 // G = X^T W X ((d+1)^2), B = X^T W R ((d+1) x d), S = R^T W R (d x d): rows
 // [8 y, 8 y + 8) of each, summed over the probes in a fixed order.
 __global__ void __launch_bounds__(256) ridge_gram_kernel(Layout L) {
+  pdl_entry();
   extern __shared__ double shr[];
   const int bh = blockIdx.x, d = L.d, n1 = d + 1, P = L.P, tid = threadIdx.x;
   double* X = shr;                       // [32][n1]
@@ -151,6 +152,7 @@ __device__ bool gj_inverse_spd(double* G, int n, int ld) {
 // One CTA per head: lam, Cholesky with up to three x10 jitter retries, the d right-hand sides,
 // then the residual-span basis by column-pivoted Gram-Schmidt on S = R^T W R and A <- A U U^T.
 __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
+  pdl_entry();
   extern __shared__ double shs[];
   const int bh = blockIdx.x, d = L.d, n1 = d + 1, tid = threadIdx.x;
   double* G = shs;  // [n1][n1], later S [d][d]
@@ -341,6 +343,7 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
 // A <- (A U) U^T with U (d x rank) the residual-span basis; 8 rows of A per block.  A
 // full-rank span is all of R^d: the projector is the identity and A is only copied to fp32.
 __global__ void __launch_bounds__(256) ridge_project_kernel(Layout L) {
+  pdl_entry();
   extern __shared__ double shp2[];
   const int bh = blockIdx.x, d = L.d, n1 = d + 1, tid = threadIdx.x;
   const int rank = L.P > 0 ? L.stats[bh].span_rank : d;
@@ -378,6 +381,7 @@ __global__ void __launch_bounds__(256) ridge_project_kernel(Layout L) {
 // rows per block, written back to original token order.
 template <typename To, int D>
 __global__ void __launch_bounds__(256) apply_kernel(Layout L, To* __restrict__ O) {
+  pdl_entry();
   extern __shared__ float sha[];
   float* As = sha;                  // [(D+1)][D]
   float* Xs = As + (D + 1) * D;     // [64][D]
@@ -422,6 +426,7 @@ static sparsepr_status launch_apply(const Layout& L, void* O, cudaStream_t st) {
 
 // No correction (repair off): A = 0, so unprobed rows keep O_sp and probe rows take O_dense.
 __global__ void zero_fit_kernel(Layout L) {
+  pdl_entry();
   const int bh = blockIdx.x, n = (L.d + 1) * L.d;
   for (int e = threadIdx.x; e < n; e += blockDim.x) {
     L.A64[(size_t)bh * n + e] = 0.0;

@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(256) ridge_gram_rows_kernel(const float* __res
                                                               const double* __restrict__ pw, int P, int d,
                                                               double* __restrict__ G, double* __restrict__ B,
                                                               double* __restrict__ S) {
+  pdl_entry();
   extern __shared__ double shx[];
   constexpr int kRows = 8, kChunk = 32;
   const int bh = blockIdx.x, n1 = d + 1, tid = threadIdx.x;

@@ -37,6 +37,7 @@ constexpr int kMetricChunk = 64;
 
 template <typename T>
 __global__ void __launch_bounds__(256) metric_kernel(Layout L, const T* __restrict__ Q) {
+  pdl_entry();
   __shared__ float qs[kMetricChunk][128];
   __shared__ long long rowi[kMetricChunk];
   const int bh = blockIdx.x, a0 = blockIdx.y * kMetricRows, d = L.d, tid = threadIdx.x;
@@ -78,6 +79,7 @@ __global__ void __launch_bounds__(256) metric_kernel(Layout L, const T* __restri
 
 // fp64 [BH, d, d] matrices split into three bf16 planes (tensor-core operands).
 __global__ void split_mat_kernel(const double* __restrict__ src, __nv_bfloat16* __restrict__ dst, size_t n) {
+  pdl_entry();
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
     const double x = src[i];
     const __nv_bfloat16 h = __double2bfloat16(x);
@@ -92,6 +94,7 @@ __global__ void split_mat_kernel(const double* __restrict__ src, __nv_bfloat16* 
 // Gc = C^T C / (d C_k) from the key-group centroids (fp64): rms_q^2 = q^T Gc q + 1e-12 is the
 // mean square of the query's responses to every key group.
 __global__ void gc_kernel(Layout L) {
+  pdl_entry();
   const int bh = blockIdx.x, a = blockIdx.y, b = threadIdx.x, d = L.d;
   if (b >= d) return;
   if (L.semantic) {  // raw queries: the row quadratic form is ||q||^2
@@ -111,6 +114,7 @@ __global__ void gc_kernel(Layout L) {
 // 64 rows per block; G staged in shared memory as fp32; thread (row p = tid/4, quarter q).
 template <typename T>
 __global__ void __launch_bounds__(256) rowqf_simt_kernel(Layout L, const T* __restrict__ X, int which) {
+  pdl_entry();
   extern __shared__ float shm[];
   const int d = L.d, bh = blockIdx.y, tid = threadIdx.x;
   const int DP = d + 1;
@@ -179,6 +183,7 @@ __device__ __forceinline__ uint64_t splitmix64_next(uint64_t& state) {
 // One thread per head.  The slots touched by C swaps live in a shared-memory hash map
 // (slot -> value), so the identity array of N slots is never written.
 __global__ void km_draw_kernel(Layout L, int stage, int C) {
+  pdl_entry();
   constexpr int kTab = 4096;  // >= 2 * 2 * kMaxGroups
   __shared__ int keys[kTab];
   __shared__ int vals[kTab];
@@ -215,6 +220,7 @@ __global__ void km_draw_kernel(Layout L, int stage, int C) {
 
 template <typename T>
 __global__ void kcent_init_kernel(Layout L, const T* __restrict__ K) {
+  pdl_entry();
   const int bh = blockIdx.x, j = blockIdx.y, a = threadIdx.x;
   if (a >= L.d) return;
   const int t = L.init_ids[(size_t)bh * max(L.Ck, L.Cq) + j];
@@ -224,6 +230,7 @@ __global__ void kcent_init_kernel(Layout L, const T* __restrict__ K) {
 // Cold start of the query groups: nu_g = r~ of the drawn query, in fp64.
 template <typename T>
 __global__ void __launch_bounds__(128) qcent_init_kernel(Layout L, const T* __restrict__ Q) {
+  pdl_entry();
   __shared__ double qv[128];
   __shared__ double red[4];
   const int bh = blockIdx.x, g = blockIdx.y, d = L.d, Ck = L.Ck, tid = threadIdx.x;
@@ -253,6 +260,7 @@ __global__ void __launch_bounds__(128) qcent_init_kernel(Layout L, const T* __re
 
 // J arrays start at the objective constant; the stop marker starts at the iteration limit.
 __global__ void km_reset_kernel(Layout L, int which, int iters) {
+  pdl_entry();
   const int bh = blockIdx.x;
   double* J = (which == 0 ? L.kJ : L.qJ) + (size_t)bh * L.iters_cap;
   const double c = which == 0 ? L.T0k[bh] : L.T0q[bh];
@@ -329,6 +337,7 @@ __device__ __forceinline__ void stage_rows(double* dst, const double* __restrict
 // shared memory, symmetric: thread a reads column a), bias_j = c_j^T W_j, ||W_j||, and the sums
 // zeroed.  Dynamic shared memory: min(d, kPrepRows) rows of M.
 __global__ void __launch_bounds__(128) kprep_kernel(Layout L, int it, int iters) {
+  pdl_entry();
   extern __shared__ double Ms[];
   __shared__ double c[kPrepGroups][128];
   __shared__ double red[kPrepGroups * 4], bias_s[kPrepGroups], wn_s[kPrepGroups];
@@ -396,6 +405,7 @@ __global__ void __launch_bounds__(128) kprep_kernel(Layout L, int it, int iters)
 // Dynamic shared memory: kPrepGroups * C_k doubles (nu of the block's groups), then
 // min(C_k, kPrepRows) rows of C.
 __global__ void __launch_bounds__(128) qprep_kernel(Layout L, int it, int iters) {
+  pdl_entry();
   extern __shared__ double qsm[];
   __shared__ double Sv[kPrepGroups][128];
   __shared__ double red[kPrepGroups * 4], nn_s[kPrepGroups], un_s[kPrepGroups];
@@ -544,6 +554,7 @@ inline size_t assign_smem_bytes(int D) {
 
 template <typename T, typename Feat>
 __global__ void __launch_bounds__(256) kmeans_assign_kernel(Layout L, const T* __restrict__ X, int it) {
+  pdl_entry();
   constexpr bool kKeys = std::is_same<Feat, KeyFeat>::value;
   const int bh = blockIdx.y;
   const int which = kKeys ? 0 : 1;
@@ -763,6 +774,7 @@ __device__ __forceinline__ int* sort_hist(const Layout& L, int bh, int side, int
 }
 
 __global__ void __launch_bounds__(256) group_hist_kernel(Layout L) {
+  pdl_entry();
   __shared__ int h[kMaxGroups];
   const int chunk = blockIdx.x, bh = blockIdx.y, side = blockIdx.z, tid = threadIdx.x, lane = tid & 31;
   const int C = side == 0 ? L.Ck : L.Cq;
@@ -785,6 +797,7 @@ __global__ void __launch_bounds__(256) group_hist_kernel(Layout L) {
 }
 
 __global__ void __launch_bounds__(1024) group_scan_kernel(Layout L) {
+  pdl_entry();
   __shared__ int wsum[32];
   const int bh = blockIdx.x, side = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = side == 0 ? L.Ck : L.Cq;
@@ -828,6 +841,7 @@ __global__ void __launch_bounds__(1024) group_scan_kernel(Layout L) {
 }
 
 __global__ void __launch_bounds__(32) group_scatter_kernel(Layout L) {
+  pdl_entry();
   __shared__ int cursor[kMaxGroups];
   __shared__ int lab[kSortChunk];
   const int chunk = blockIdx.x, bh = blockIdx.y, side = blockIdx.z, lane = threadIdx.x;
@@ -873,6 +887,7 @@ static void launch_group_sort(const Layout& L, cudaStream_t st) {
 // ------------------------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(256) route_select_kernel(Layout L, const T* __restrict__ Q) {
+  pdl_entry();
   __shared__ double qbar[128];
   __shared__ double qpart[4][128];
   __shared__ double S[kMaxGroups];
@@ -956,6 +971,7 @@ __global__ void __launch_bounds__(256) route_select_kernel(Layout L, const T* __
 // Route lists (ascending key-group ids), visible keys per group, query-tile prefix and the
 // realised density.  One block per head.
 __global__ void __launch_bounds__(256) route_build_kernel(Layout L, int tile_m) {
+  pdl_entry();
   __shared__ int tiles[kMaxGroups + 1];
   __shared__ long long pairs[kMaxGroups];
   const int bh = blockIdx.x, Ck = L.Ck, Cq = L.Cq;
@@ -1003,6 +1019,7 @@ constexpr size_t kProbeSmem = kMaxProbes * (sizeof(double) + sizeof(int)) + kMax
                               (2 * kMaxGroups + 1) * sizeof(int);
 
 __global__ void __launch_bounds__(1024) probe_select_kernel(Layout L) {
+  pdl_entry();
   extern __shared__ double shp[];
   double* cw = shp;                                  // [kMaxProbes]
   long long* rem = (long long*)(cw + kMaxProbes);    // [kMaxGroups]
@@ -1081,6 +1098,7 @@ __global__ void __launch_bounds__(1024) probe_select_kernel(Layout L) {
 
 // probe_of from an installed probe list (sparsepr_set_partition).
 __global__ void probe_index_kernel(Layout L) {
+  pdl_entry();
   const int bh = blockIdx.x;
   int* pof = L.probe_of + (size_t)bh * L.N;
   for (int t = threadIdx.x; t < L.N; t += blockDim.x) pof[t] = -1;
@@ -1090,6 +1108,7 @@ __global__ void probe_index_kernel(Layout L) {
 
 // Per-head k-means statistics after both loops.
 __global__ void plan_stats_kernel(Layout L) {
+  pdl_entry();
   const int bh = blockIdx.x * blockDim.x + threadIdx.x;
   if (bh >= L.BH) return;
   sparsepr_head_stats& st = L.stats[bh];
@@ -1107,6 +1126,7 @@ __global__ void plan_stats_kernel(Layout L) {
 // ------------------------------------------------------------------------------------------
 __global__ void permute_rows_kernel(Layout L, const void* __restrict__ src, void* __restrict__ dst,
                                     const int* __restrict__ perm, int rows_per_head, int src_rows_per_head) {
+  pdl_entry();
   const int bh = blockIdx.y;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= rows_per_head) return;
@@ -1122,6 +1142,7 @@ __global__ void permute_rows_kernel(Layout L, const void* __restrict__ src, void
 // 16-byte piece of a row of each (three independent loads in flight per piece).
 __global__ void __launch_bounds__(256) permute_qkv_kernel(Layout L, const void* __restrict__ Q,
                                                           const void* __restrict__ K, const void* __restrict__ V) {
+  pdl_entry();
   const int bh = blockIdx.y;
   const size_t rb = (size_t)L.d * elt_size(L.dtype);
   const int chunks = (int)(rb / 16);

@@ -307,3 +307,71 @@ def test_out_of_order_calls_are_rejected():
     op.plan(Q, K)
     with pytest.raises(S.SparsePRError):
         op.fit_apply(out_dtype=torch.float32)
+
+
+def _sparse_rows(q, k, v, rows, qlabels, klabels, route):
+    """Block-sparse attention output of the given rows only (the oracle's definition, row by row
+    grouped by query group): each row attends to the keys of the groups its group keeps."""
+    out = np.zeros((len(rows), v.shape[1]))
+    for g in np.unique(qlabels[rows]):
+        sel = np.flatnonzero(qlabels[rows] == g)
+        keys = np.flatnonzero(route[g][klabels])
+        out[sel] = O.attention(q[rows[sel]], k[keys], v[keys])
+    return out
+
+
+def test_dit13b_full_size_sampled():
+    """The 13B-DiT-shaped layer at its full size (24 heads x 118,800 tokens, d = 128), launched
+    as the benchmark launches it: one call over all heads, bf16 output.  On the first and the
+    last head: the oracle's key and query groups equal the GPU's (up to the oracle's near-ties),
+    its routes, probes and weights equal the GPU's, and -- on the GPU's partition -- the probe
+    rows' dense outputs, 256 sampled rows' block-sparse outputs, the fitted map and those rows'
+    corrected outputs match the oracle's computed one row at a time."""
+    w = configs.workload(2)
+    Q, K, V = gen.make_qkv(w)
+    op, out = run_gpu(w, Q, K, V, out_dtype=torch.bfloat16)
+    kl, ql = op.query(S.Q_KLABELS), op.query(S.Q_QLABELS)
+    route, probes, pw = op.query(S.Q_ROUTE).astype(bool), op.query(S.Q_PROBES), op.query(S.Q_PROBE_W)
+    kc, st, A_gpu = op.query(S.Q_KCENT), op.stats(), op.query(S.Q_FIT)
+    osp_all = op.query(S.Q_OSP)
+    od_all = op.query(S.Q_ODENSE)
+    for h in (0, w.H - 1):
+        q, k, v = gen.as_f64(Q[0, h]), gen.as_f64(K[0, h]), gen.as_f64(V[0, h])
+        r = O.call_head(q, k, v, w, h, compute_outputs=False)
+        labels_match(kl[h], r["kmeans_k"], f"head {h} key groups")
+        labels_match(ql[h], r["kmeans_q"], f"head {h} query groups")
+        if np.array_equal(kl[h], r["klabels"]) and np.array_equal(ql[h], r["qlabels"]):
+            ref_route, ref_probes, ref_w, ref_pairs = r["route"], r["probes"], r["weights"], r["sparse_pairs"]
+        else:
+            ref_route, ref_probes, ref_w, ref_pairs = oracle_routing_on(q, kl[h], ql[h], kc[h], w)
+        assert np.array_equal(route[h], ref_route), f"head {h} routes"
+        assert np.array_equal(probes[h], ref_probes), f"head {h} probes"
+        np.testing.assert_allclose(pw[h], ref_w, rtol=1e-12)
+        assert st[h]["sparse_pairs"] == ref_pairs
+        p = probes[h]
+        od = od_all[h].astype(np.float64)
+        od_ref = O.attention(q[p], k, v)
+        _close(f"head {h} O_dense", od, od_ref, 2e-2, 1e-2)
+        osp = osp_all[h].astype(np.float64)
+        rows = (np.arange(256) * w.N) // 256
+        rows = rows[~np.isin(rows, p)]
+        ref_sp = _sparse_rows(q, k, v, np.concatenate([rows, p]), ql[h], kl[h], route[h])
+        ref_rows_sp, ref_p_sp = ref_sp[:len(rows)], ref_sp[len(rows):]
+        _close(f"head {h} O_sp rows", osp[rows], ref_rows_sp, 2e-2, 1e-2)
+        _close(f"head {h} O_sp probes", osp[p], ref_p_sp, 2e-2, 1e-2)
+        # the fit on the GPU's own probe rows (both sides fp64)
+        A_full, _ = O.ridge_fit(osp[p], od, pw[h], w.lam)
+        A_ref = O.restrict_to_residual_span(A_full, od - osp[p], pw[h])
+        fit_matches(A_gpu[h], A_full, A_ref, od - osp[p], pw[h], f"head {h} fit")
+        got = out[0, h].float().cpu().numpy().astype(np.float64)
+        # corrected rows: the GPU's O_sp through the GPU's map, to the bf16 output's rounding
+        _close(f"head {h} apply", got[rows], O.apply_correction(osp[rows], A_gpu[h]), 2e-2, 1e-2)
+        assert np.abs(got[p] - od).max() <= 2e-2, f"head {h} probe rows"
+        # end to end on the sampled rows: the oracle's rows through the oracle's own map, the bar
+        # scaled by the map's gain (it carries the block-sparse rounding into the rows)
+        A_orc_full, _ = O.ridge_fit(ref_p_sp, od_ref, pw[h], w.lam)
+        A_orc = O.restrict_to_residual_span(A_orc_full, od_ref - ref_p_sp, pw[h])
+        ref_rows = O.apply_correction(ref_rows_sp, A_orc)
+        A_lin = A_orc[:-1]
+        _close(f"head {h} O rows", got[rows], ref_rows, 2e-2 * (1.0 + np.abs(A_lin).sum(axis=0).max()),
+               1e-2 * (1.0 + np.linalg.norm(A_lin, 2)))
