@@ -191,17 +191,32 @@ def output_quality(S, w, Q, K, V, O_main, main_probes, dev, n_eval=2048):
 
 
 def km_rooflines(w, asg_ms, upd_ms, pk):
-    """HBM rooflines of one key k-means assignment and one update launch (first iteration of
-    the call): each reads every key once (2 d bytes, bf16) and writes (assignment) or reads
-    (update) its label (4 bytes)."""
+    """Rooflines of one key k-means assignment and one update launch (first iteration of the
+    call).  Both read every key once (2 d bytes, bf16) and write (assignment) or read (update)
+    its label (4 bytes).  The assignment also runs the tensor-core products of every key with
+    the three bf16 terms of the C_p (padded) group weights, 3 x 2 x C_p x d flops per key: at
+    the large shapes that, not HBM, is its bound, and it is reported against the bf16 peak with
+    the HBM fraction beside it.  The update is HBM-bound."""
     units = w.B * w.H * w.N
     by = units * (2 * w.d + 4)
+    cp = (w.n_kgroups + 15) // 16 * 16
+    fl = units * 3 * 2 * cp * w.d
     out = {}
-    for name, t in (("assignment", asg_ms), ("update", upd_ms)):
-        if t > 0:
-            a = by / (t * 1e-3) / 1e9
-            out[name] = {"bound": "hbm", "achieved": a, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": a / pk["hbm_gbs"], "ms": t, "traffic": None,
+    if asg_ms > 0:
+        s = asg_ms * 1e-3
+        t_hbm, t_tc = by / (pk["hbm_gbs"] * 1e9), fl / (pk["bf16_tflops"] * 1e12)
+        hbm = {"achieved": by / s / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": by / s / 1e9 / pk["hbm_gbs"]}
+        tc = {"achieved": fl / s / 1e12, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+              "frac": fl / s / 1e12 / pk["bf16_tflops"]}
+        main, other = (tc, hbm) if t_tc >= t_hbm else (hbm, tc)
+        out["assignment"] = {"bound": "tensor" if t_tc >= t_hbm else "hbm", **main, "ms": asg_ms, "traffic": None,
+                             "other": other,
+                             "algorithmic": f"{units} keys x (2d + 4) bytes = {by} bytes and x 6 C_p d = {fl} "
+                                            f"flops per launch"}
+    if upd_ms > 0:
+        a = by / (upd_ms * 1e-3) / 1e9
+        out["update"] = {"bound": "hbm", "achieved": a, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": a / pk["hbm_gbs"], "ms": upd_ms, "traffic": None,
                          "algorithmic": f"{units} keys x (2d + 4) bytes = {by} bytes per launch"}
     return out
 

@@ -45,20 +45,22 @@ constexpr int kExpPolyEvery = 0;           // in tiles whose keys are all real, 
 // 2^x for a pair of x <= kRescaleThreshold on the FMA pipe (f32x2), for x >= -125 (smaller x
 // give 2^-125 instead of 0: far below the bf16 rounding of P and of any row sum, which is
 // >= 1).  Cody-Waite style reduction x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in
-// the low mantissa bits) and f in [-1/2, 1/2], then a cubic in f fitted to 2^f by least
+// the low mantissa bits) and f in [-1/2, 1/2], then a quintic in f fitted to 2^f by least
 // squares on relative error at Chebyshev nodes with Lawson reweighting (max relative error
-// 7.5e-5), and n added to the exponent field.
+// 2.3e-7 in fp32 Horner evaluation, about that of the special-function unit), and n added to
+// the exponent field.
 __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
   float x0, x1;
   f2_unpack(x, x0, x1);
   const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const uint64_t shifter = f2_pack(12582912.f, 12582912.f);
-  const uint64_t t = f2_add(xc, shifter);
+  const uint64_t t = f2_add(xc, f2_pack(12582912.f, 12582912.f));
   const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));
   const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);
-  uint64_t p = f2_fma(f2_pack(0.0551716648f, 0.0551716648f), f, f2_pack(0.2426111251f, 0.2426111251f));
-  p = f2_fma(p, f, f2_pack(0.6932609677f, 0.6932609677f));
-  p = f2_fma(p, f, f2_pack(0.9999280572f, 0.9999280572f));
+  uint64_t p = f2_fma(f2_pack(0.001327647129f, 0.001327647129f), f, f2_pack(0.009675540961f, 0.009675540961f));
+  p = f2_fma(p, f, f2_pack(0.05550713092f, 0.05550713092f));
+  p = f2_fma(p, f, f2_pack(0.2402212024f, 0.2402212024f));
+  p = f2_fma(p, f, f2_pack(0.693146944f, 0.693146944f));
+  p = f2_fma(p, f, f2_pack(1.000000119f, 1.000000119f));
   float p0, p1, t0, t1;
   f2_unpack(p, p0, p1);
   f2_unpack(t, t0, t1);
