@@ -149,80 +149,12 @@ __device__ bool gj_inverse_spd(double* G, int n, int ld) {
   return true;
 }
 
-// One CTA per head: lam, Cholesky with up to three x10 jitter retries, the d right-hand sides,
-// then the residual-span basis by column-pivoted Gram-Schmidt on S = R^T W R and A <- A U U^T.
-__global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
-  pdl_entry();
-  extern __shared__ double shs[];
-  const int bh = blockIdx.x, d = L.d, n1 = d + 1, tid = threadIdx.x;
-  double* G = shs;  // [n1][n1], later S [d][d]
-  __shared__ double red[8];
-  __shared__ double ldiag[129];  // diagonal of the Cholesky factor
-  const double* Gg = L.ridgeG + (size_t)bh * n1 * n1;
-  double* A = L.A64 + (size_t)bh * n1 * d;
+// The residual-span basis of head bh (role 1 of ridge_solve_kernel): span of the residual rows
+// = range(S), S = R^T W R, whose rank goes to the head's statistics and whose basis (when the
+// rank is below d) goes to spanS for the projection kernel.
+__device__ __noinline__ void ridge_span_basis(const Layout& L, int bh, double* G, double* ldiag) {
+  const int d = L.d, tid = threadIdx.x;
   sparsepr_head_stats& st = L.stats[bh];
-
-  if (L.P == 0) {
-    for (int e = tid; e < n1 * d; e += blockDim.x) {
-      A[e] = 0.0;
-      L.A32[(size_t)bh * n1 * d + e] = 0.f;
-    }
-    if (tid == 0) {
-      st.lambda = 0.0;
-      st.fit_retries = 0;
-      st.span_rank = 0;
-    }
-    return;
-  }
-  double tr = 0.0;
-  for (int i = tid; i < n1; i += blockDim.x) tr += Gg[i * n1 + i];
-  tr = block_sum(tr, red);
-  double lam = L.lambda >= 0.0 ? L.lambda : 1e-3 * tr / n1;
-  int retries = 0;
-  bool ok = false;
-  for (; retries <= 3; ++retries) {
-    for (int e = tid; e < n1 * n1; e += blockDim.x) G[e] = Gg[e] + ((e / n1) == (e % n1) ? lam : 0.0);
-    __syncthreads();
-    ok = gj_inverse_spd(G, n1, n1);
-    if (ok) break;
-    lam = lam > 0.0 ? lam * 10.0 : (tr > 0.0 ? 1e-12 * tr / n1 : 1e-30);
-  }
-  if (!ok) {
-    if (tid == 0) {
-      atomicCAS(L.status, kDevOk, kDevNumeric);
-      st.fit_retries = retries;
-      st.span_rank = d;  // nothing to project: A is zero
-    }
-    for (int e = tid; e < n1 * d; e += blockDim.x) {
-      A[e] = 0.0;
-      L.A32[(size_t)bh * n1 * d + e] = 0.f;
-    }
-    return;
-  }
-  // A = (G + lam I)^-1 B, 32 columns of B at a time staged in shared memory (all loads in
-  // flight together); thread = (row, column) of the chunk
-  {
-    const double* Bg = L.ridgeB + (size_t)bh * n1 * d;
-    double* Y = G + n1 * n1;  // [n1][33]
-    for (int c0 = 0; c0 < d; c0 += 32) {
-      __syncthreads();
-      for (int e = tid; e < n1 * 32; e += blockDim.x) Y[(e >> 5) * 33 + (e & 31)] = Bg[(size_t)(e >> 5) * d + c0 + (e & 31)];
-      __syncthreads();
-      for (int e = tid; e < n1 * 32; e += blockDim.x) {
-        const int a = e >> 5, j = e & 31;
-        const double* gr = G + a * n1;
-        double acc0 = 0.0, acc1 = 0.0;
-        int k = 0;
-        for (; k + 1 < n1; k += 2) {
-          acc0 += gr[k] * Y[k * 33 + j];
-          acc1 += gr[k + 1] * Y[(k + 1) * 33 + j];
-        }
-        if (k < n1) acc0 += gr[k] * Y[k * 33 + j];
-        A[(size_t)a * d + c0 + j] = acc0 + acc1;
-      }
-    }
-  }
-  __syncthreads();
   // span of the residual rows = range(S), S = R^T W R.  Full rank is the common case: a
   // Cholesky of S whose pivots all stay above 1e-10 of the largest diagonal entry proves it,
   // and then the projector is the identity.  Otherwise an orthonormal basis U of range(S) comes
@@ -240,7 +172,7 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
   }
   __syncthreads();
   int rank = 0;
-  int basis[128];
+  __shared__ int bcol[128];  // pivot columns in basis order
   bool full = s_dmax > 0.0 && chol_smem_tol(S, d, d, 1e-10 * s_dmax, ldiag);
   if (full) {
     rank = d;
@@ -256,7 +188,6 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
     __shared__ double cn[128];
     __shared__ int used[128];
     __shared__ double binv[128];
-    __shared__ int bcol[128];
     const int tpc = blockDim.x / d, sub = tid % tpc;  // 4 (d = 64) or 2 (d = 128)
     __syncthreads();
     for (int c = tid / tpc; c < d; c += blockDim.x / tpc) {
@@ -322,7 +253,6 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
       S[i * ld + bcol[r]] *= binv[r];
     }
     __syncthreads();
-    for (int r = 0; r < rank; ++r) basis[r] = bcol[r];
   }
   // hand the basis to the projection kernel: columns r < rank of spanS are U's columns
   __syncthreads();
@@ -330,13 +260,96 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
     double* U = L.spanS + (size_t)bh * d * d;
     for (int e = tid; e < d * rank; e += blockDim.x) {
       const int i = e / rank, r = e % rank;
-      U[i * d + r] = S[i * (d + 1) + basis[r]];  // the Gram-Schmidt rows are padded to d + 1
+      U[i * d + r] = S[i * (d + 1) + bcol[r]];  // the Gram-Schmidt rows are padded to d + 1
+    }
+  }
+  if (tid == 0) st.span_rank = rank;
+}
+
+// Two CTAs per head, which run at the same time: role 0 takes lam, the inverse of G + lam I
+// with up to three x10 jitter retries and the d right-hand sides; role 1 takes the residual-span
+// basis (a full-rank test, else column-pivoted Gram-Schmidt on S = R^T W R).  The projection
+// A <- A U U^T follows in ridge_project_kernel.
+__global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
+  pdl_entry();
+  extern __shared__ double shs[];
+  const int bh = blockIdx.x >> 1, role = blockIdx.x & 1, d = L.d, n1 = d + 1, tid = threadIdx.x;
+  double* G = shs;  // [n1][n1], later S [d][d]
+  __shared__ double red[8];
+  __shared__ double ldiag[129];  // diagonal of the Cholesky factor
+  const double* Gg = L.ridgeG + (size_t)bh * n1 * n1;
+  double* A = L.A64 + (size_t)bh * n1 * d;
+  sparsepr_head_stats& st = L.stats[bh];
+
+  if (L.P == 0) {
+    if (role == 0) {
+      for (int e = tid; e < n1 * d; e += blockDim.x) {
+        A[e] = 0.0;
+        L.A32[(size_t)bh * n1 * d + e] = 0.f;
+      }
+      if (tid == 0) {
+        st.lambda = 0.0;
+        st.fit_retries = 0;
+      }
+    } else if (tid == 0) {
+      st.span_rank = 0;
+    }
+    return;
+  }
+  if (role == 1) {
+    ridge_span_basis(L, bh, shs, ldiag);
+    return;
+  }
+  double tr = 0.0;
+  for (int i = tid; i < n1; i += blockDim.x) tr += Gg[i * n1 + i];
+  tr = block_sum(tr, red);
+  double lam = L.lambda >= 0.0 ? L.lambda : 1e-3 * tr / n1;
+  int retries = 0;
+  bool ok = false;
+  for (; retries <= 3; ++retries) {
+    for (int e = tid; e < n1 * n1; e += blockDim.x) G[e] = Gg[e] + ((e / n1) == (e % n1) ? lam : 0.0);
+    __syncthreads();
+    ok = gj_inverse_spd(G, n1, n1);
+    if (ok) break;
+    lam = lam > 0.0 ? lam * 10.0 : (tr > 0.0 ? 1e-12 * tr / n1 : 1e-30);
+  }
+  if (!ok) {
+    if (tid == 0) {
+      atomicCAS(L.status, kDevOk, kDevNumeric);
+      st.fit_retries = retries;  // A is zero; its projection stays zero
+    }
+    for (int e = tid; e < n1 * d; e += blockDim.x) {
+      A[e] = 0.0;
+      L.A32[(size_t)bh * n1 * d + e] = 0.f;
+    }
+    return;
+  }
+  // A = (G + lam I)^-1 B, 32 columns of B at a time staged in shared memory (all loads in
+  // flight together); thread = (row, column) of the chunk
+  {
+    const double* Bg = L.ridgeB + (size_t)bh * n1 * d;
+    double* Y = G + n1 * n1;  // [n1][33]
+    for (int c0 = 0; c0 < d; c0 += 32) {
+      __syncthreads();
+      for (int e = tid; e < n1 * 32; e += blockDim.x) Y[(e >> 5) * 33 + (e & 31)] = Bg[(size_t)(e >> 5) * d + c0 + (e & 31)];
+      __syncthreads();
+      for (int e = tid; e < n1 * 32; e += blockDim.x) {
+        const int a = e >> 5, j = e & 31;
+        const double* gr = G + a * n1;
+        double acc0 = 0.0, acc1 = 0.0;
+        int k = 0;
+        for (; k + 1 < n1; k += 2) {
+          acc0 += gr[k] * Y[k * 33 + j];
+          acc1 += gr[k + 1] * Y[(k + 1) * 33 + j];
+        }
+        if (k < n1) acc0 += gr[k] * Y[k * 33 + j];
+        A[(size_t)a * d + c0 + j] = acc0 + acc1;
+      }
     }
   }
   if (tid == 0) {
     st.lambda = lam;
     st.fit_retries = retries;
-    st.span_rank = rank;
   }
 }
 
@@ -463,11 +476,12 @@ sparsepr_status launch_fit_apply(const Layout& L, void* O, int out_dtype, cudaSt
 
 namespace sparsepr {
 
-// The one-CTA-per-head solve on ridge matrices that are already in L.ridgeG / ridgeB / spanS.
+// The solve (two CTAs per head) and the projection on ridge matrices that are already in
+// L.ridgeG / ridgeB / spanS.
 sparsepr_status launch_ridge_solve(const Layout& L, cudaStream_t st) {
   const size_t ssm = ridge_solve_smem(L.d);
   cudaFuncSetAttribute(ridge_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
-  launch(ridge_solve_kernel, L.BH, 256, ssm, st, L);
+  launch(ridge_solve_kernel, 2 * L.BH, 256, ssm, st, L);  // two roles per head
   const size_t psm = (size_t)(L.d * L.d + 8 * L.d + 8 * L.d) * sizeof(double);
   cudaFuncSetAttribute(ridge_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
   launch(ridge_project_kernel, dim3(L.BH, (L.d + 1 + 7) / 8), 256, psm, st, L);
