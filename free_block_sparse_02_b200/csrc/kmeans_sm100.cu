@@ -69,9 +69,9 @@ __host__ inline size_t km_assign_smem(int D, int Np, int stages) {
 // Shared memory of the update kernel: labels and sorted order of a chunk of points, per-group
 // offsets and cursors.
 __host__ inline size_t km_update_smem(int D, int C) {
-  (void)D;
-  return (size_t)2 * kKmUpdChunk * 4 /*labels, order*/ + (size_t)(3 * C + 2) * 4 /*offs, cursor, ioff*/ +
-         (size_t)2 * km_upd_max_items(C) * 4 /*item group, item start*/;
+  const size_t chunk = (size_t)2 * kKmUpdChunk * 4 /*labels, order*/ + (size_t)(3 * C + 2) * 4 /*offs, cursor, ioff*/ +
+                       (size_t)2 * km_upd_max_items(C) * 4 /*item group, item start*/;
+  return std::max(chunk, (size_t)D * D * sizeof(double) /*Gc during the re-decision*/);
 }
 
 __device__ __forceinline__ int km_tiles_per_head(const Layout& L) { return (L.N + kKmTile - 1) / kKmTile; }
@@ -414,32 +414,29 @@ __global__ void __launch_bounds__(kKmThreads, 1)
 // Exact fp64 value of a bf16 given by its 16 bits (through its exact fp32 value).
 __device__ __forceinline__ double bf16_bits_to_f64(uint32_t b) { return (double)__uint_as_float(b << 16); }
 
-// fp64 re-decision of the points the assignment listed: block (c, y) takes every
-// kKmRedecideSplit-th entry of CTA range c's list, one warp per point; the label and the
-// objective (its fp64 score minus the tentative fp32 one) are corrected in place.  Points with
-// a short candidate list evaluate only those groups; queries stage Gc in shared memory (dynamic:
-// d * d doubles) for the exact scale.
-constexpr int kKmRedecideSplit = 4;
+// fp64 re-decision of the points the assignment listed for CTA range c, run by the update
+// kernel's CTA c before it reads the labels (the ranges of the two kernels are the same): the
+// CTA's warps take every kKmUpdWarps-th entry, one warp per point; the label and the objective
+// (its fp64 score minus the tentative fp32 one) are corrected in place.  Points with a short
+// candidate list evaluate only those groups; queries stage Gc in shared memory (gcs: d * d
+// doubles, free until the update's chunk loop) for the exact scale.  Every thread of the CTA
+// calls this (it has block barriers).
+constexpr int kKmUpdWarps = kKmUpdThreads / 32;
 
 template <bool kKeys>
-__global__ void __launch_bounds__(256) kmeans_redecide_kernel(const __nv_bfloat16* __restrict__ X, Layout L, int it,
-                                                              int G) {
-  pdl_entry();
-  extern __shared__ double Gcs[];  // queries: Gc of the current head
-  __shared__ double xs_all[8][128];
+__device__ __forceinline__ void redecide_range(const __nv_bfloat16* __restrict__ X, const Layout& L, int it, int t0,
+                                               int t1, double* gcs) {
+  __shared__ double xs_all[kKmUpdWarps][128];
+  __shared__ int s_need[kKmUpdWarps];
   const int D = L.d, C = kKeys ? L.Ck : L.Cq;
-  const int tph = km_tiles_per_head(L);
-  int t0, t1;
-  km_range((long long)L.BH * tph, G, blockIdx.x, t0, t1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nlist = min(max(L.rcnt[blockIdx.x], 0), max(t1 - t0, 0) * kKmTile);  // never past the segment
-  if ((int)blockIdx.y * 8 >= nlist) return;  // no entry for this block (uniform)
   const int4* list = L.rlist + (size_t)t0 * kKmTile;
   int* labels = kKeys ? L.klabel : L.qlabel;
   double* Jarr = kKeys ? L.kJ : L.qJ;
   double* xs = xs_all[warp];
   int gc_head = -1;  // head whose Gc is staged (the range spans few heads; stage per change)
-  for (int li0 = blockIdx.y * 8; li0 < nlist; li0 += 8 * kKmRedecideSplit) {
+  for (int li0 = 0; li0 < nlist; li0 += kKmUpdWarps) {  // the same trip count in every thread
     const int li = li0 + warp;
     int bh = -1;
     int4 en = make_int4(0, 0, 0, 0);
@@ -447,14 +444,13 @@ __global__ void __launch_bounds__(256) kmeans_redecide_kernel(const __nv_bfloat1
       en = list[li];
       bh = en.x / L.N;
     }
-    if constexpr (!kKeys) {  // the block's warps agree on the heads they need: stage on change
+    if constexpr (!kKeys) {  // the CTA's warps agree on the heads they need: stage on change
       const int need = __shfl_sync(0xffffffffu, bh, 0);
-      __shared__ int s_need[8];
       if (lane == 0) s_need[warp] = need;
       __syncthreads();
       int first = -1;
       bool mixed = false;
-      for (int w = 0; w < 8; ++w)
+      for (int w = 0; w < kKmUpdWarps; ++w)
         if (s_need[w] >= 0) {
           if (first < 0) first = s_need[w];
           else if (s_need[w] != first) mixed = true;
@@ -462,7 +458,7 @@ __global__ void __launch_bounds__(256) kmeans_redecide_kernel(const __nv_bfloat1
       if (!mixed && first >= 0 && first != gc_head) {
         const double* src = L.Gc + (size_t)first * D * D;
         for (int e = threadIdx.x; e < D * D / 2; e += blockDim.x)
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(Gcs + 2 * e)),
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(gcs + 2 * e)),
                        "l"(src + 2 * e)
                        : "memory");
         asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
@@ -480,7 +476,7 @@ __global__ void __launch_bounds__(256) kmeans_redecide_kernel(const __nv_bfloat1
     double bv;
     const double* W64 = (kKeys ? L.kW64 : L.qU64) + (size_t)bh * C * D;
     const double* B64 = (kKeys ? L.kbias64 : L.qbias64) + (size_t)bh * C;
-    const double* Gc = (!kKeys && gc_head == bh) ? Gcs : L.Gc + (size_t)bh * D * D;
+    const double* Gc = (!kKeys && gc_head == bh) ? gcs : L.Gc + (size_t)bh * D * D;
     const int nc = en.z & 0xFF;
     if (nc <= 4) {
       int cand[4] = {(en.z >> 8) & 0x3FF, (en.z >> 18) & 0x3FF, en.w & 0xFFFF, (en.w >> 16) & 0xFFFF};
@@ -501,6 +497,7 @@ __global__ void __launch_bounds__(256) kmeans_redecide_kernel(const __nv_bfloat1
     }
     __syncwarp();
   }
+  __syncthreads();  // final labels are visible to the whole CTA; gcs is free again
 }
 
 template <bool kKeys>
@@ -516,6 +513,9 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
   if (t0 >= t1) return;
 
   extern __shared__ uint8_t smem_raw[];
+  // the re-decision of the points the assignment flagged in this range comes first; it may
+  // use the start of the dynamic shared memory for Gc (d * d doubles <= the two chunk arrays)
+  redecide_range<kKeys>(X, L, it, t0, t1, (double*)smem_raw);
   int* lab = (int*)smem_raw;                   // [kKmUpdChunk] label of each point of the chunk
   int* order = lab + kKmUpdChunk;              // [kKmUpdChunk] chunk points sorted by label
   int* offs = order + kKmUpdChunk;             // [C + 1] start of each label's run
@@ -879,7 +879,6 @@ sparsepr_status launch_kmeans_iteration_tc(const Layout& L, bool keys, const voi
     mark(SPARSEPR_KERNEL_KMEANS_ASSIGN, false);
     launch(kmeans_assign_tc_kernel<true>, G, kKmThreads, smem_a, st, mX, mW, L, it, G, S);
     mark(SPARSEPR_KERNEL_KMEANS_ASSIGN, true);
-    launch(kmeans_redecide_kernel<true>, dim3(G, kKmRedecideSplit), 256, 0, st, Xb, L, it, G);  // keys: no Gc
     mark(SPARSEPR_KERNEL_KMEANS_UPDATE, false);
     launch(kmeans_update_kernel<true>, G, kKmUpdThreads, smem_u, st, Xb, L, it, G);
     mark(SPARSEPR_KERNEL_KMEANS_UPDATE, true);
@@ -887,9 +886,6 @@ sparsepr_status launch_kmeans_iteration_tc(const Layout& L, bool keys, const voi
     cudaFuncSetAttribute(kmeans_assign_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
     cudaFuncSetAttribute(kmeans_update_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_u);
     launch(kmeans_assign_tc_kernel<false>, G, kKmThreads, smem_a, st, mX, mW, L, it, G, S);
-    const size_t smem_r = (size_t)D * D * sizeof(double);
-    cudaFuncSetAttribute(kmeans_redecide_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r);
-    launch(kmeans_redecide_kernel<false>, dim3(G, kKmRedecideSplit), 256, smem_r, st, Xb, L, it, G);
     launch(kmeans_update_kernel<false>, G, kKmUpdThreads, smem_u, st, Xb, L, it, G);
   }
   SPR_LAUNCH_CHECK();
