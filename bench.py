@@ -101,7 +101,8 @@ def profiled_traffic(w):
 def workload_config(w, extra=None):
     c = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "density": w.density, "s": w.s,
          "n_kgroups": w.n_kgroups, "n_qgroups": w.n_qgroups, "P": w.P,
-         "probes": "stratified" if w.probe_mode else "uniform", "km_iters": w.km_iters, "km_tol": w.km_tol,
+         "probes": ["uniform", "stratified", "random"][w.probe_mode], "km_iters": w.km_iters, "km_tol": w.km_tol,
+         "lam": w.lam, "correction": "mean" if w.correction == 1 else "affine",
          "generator": (f"clustered Gaussian tiles {w.tile} on grid {w.grid}" if w.recipe == "tiles" else
                        f"smooth random field, length scales {w.field_ell}, logit contrast {w.field_tau}, "
                        f"value offset {w.value_offset}, on grid {w.grid}") + (" + 3D RoPE" if w.rope else "")}
@@ -415,6 +416,11 @@ def main():
                     help="run the workload on this many heads instead (a smaller case for profilers)")
     ap.add_argument("--density", type=float, default=0.0, help="override the density target (sweeps)")
     ap.add_argument("--probes", type=int, default=-1, help="override the probe budget P (sweeps)")
+    ap.add_argument("--probe-mode", default=None, choices=["uniform", "stratified", "random"],
+                    help="override the probe selection (Table 4 sweeps)")
+    ap.add_argument("--correction", default=None, choices=["affine", "mean"],
+                    help="override the correction family (Table 4 sweeps)")
+    ap.add_argument("--lam", type=float, default=None, help="override the ridge lambda (>= 0 absolute)")
     ap.add_argument("--inputs", default="tiles", choices=["tiles", "field"],
                     help="input recipe: clustered Gaussian tiles (the workloads' own) or a smooth random field")
     args = ap.parse_args()
@@ -428,6 +434,13 @@ def main():
         w = w.replace(P=args.probes)
     if args.inputs != w.recipe:
         w = w.replace(recipe=args.inputs)
+    if args.probe_mode is not None:
+        w = w.replace(probe_mode={"uniform": configs.PROBE_UNIFORM, "stratified": configs.PROBE_STRATIFIED,
+                                  "random": configs.PROBE_RANDOM}[args.probe_mode])
+    if args.correction is not None:
+        w = w.replace(correction=configs.CORRECTION_MEAN if args.correction == "mean" else configs.CORRECTION_AFFINE)
+    if args.lam is not None:
+        w = w.replace(lam=args.lam)
     if args.impl == "reference":
         run_reference(args, w, world, rank)
     else:

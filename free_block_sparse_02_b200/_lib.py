@@ -38,7 +38,8 @@ class Config(ctypes.Structure):
                 ("n_qgroups", ctypes.c_int32), ("density", ctypes.c_float), ("fixed_k", ctypes.c_int32),
                 ("P", ctypes.c_int32), ("probe_mode", ctypes.c_int32), ("lambda_", ctypes.c_double),
                 ("km_iters", ctypes.c_int32), ("km_iters_warm", ctypes.c_int32), ("km_tol", ctypes.c_float),
-                ("seed", ctypes.c_uint64), ("partition", ctypes.c_int32), ("repair", ctypes.c_int32)]
+                ("seed", ctypes.c_uint64), ("partition", ctypes.c_int32), ("repair", ctypes.c_int32),
+                ("correction", ctypes.c_int32)]
 
 
 class HeadStats(ctypes.Structure):
@@ -97,7 +98,8 @@ def config_from(w, **over) -> Config:
                   fixed_k=g("fixed_k"), P=g("P"), probe_mode=g("probe_mode"), lambda_=g("lam"),
                   km_iters=g("km_iters"), km_iters_warm=g("km_iters_warm"), km_tol=g("km_tol"),
                   seed=g("seed"), partition=over.get("partition", getattr(w, "partition", 0)),
-                  repair=over.get("repair", getattr(w, "repair", 1)))
+                  repair=over.get("repair", getattr(w, "repair", 1)),
+                  correction=over.get("correction", getattr(w, "correction", 0)))
 
 
 def workspace_size(cfg: Config) -> int:

@@ -20,6 +20,10 @@ BF16 = 1
 
 PROBE_UNIFORM = 0
 PROBE_STRATIFIED = 1
+PROBE_RANDOM = 2
+# correction families (Table 4): the affine map of [O_sp, 1] (SparsePR) or the mean-only one
+CORRECTION_AFFINE = 0
+CORRECTION_MEAN = 1
 # partitions: response-coupled (SparsePR: keys by their responses to sampled queries, queries
 # by their normalised responses to the key-group centroids) or semantic (k-means on the raw
 # keys and the raw queries; the baseline of the paper's Table 2)
@@ -55,6 +59,7 @@ class Workload:
     seed: int = 20261202              # k-means initial-point draw (SplitMix64 streams)
     partition: int = 0                # PARTITION_RESPONSE (SparsePR) or PARTITION_SEMANTIC
     repair: int = 1                   # 1: fit and add the probe-residual correction; 0: none
+    correction: int = 0               # CORRECTION_AFFINE (SparsePR) or CORRECTION_MEAN
     recipe: str = "tiles"             # input generator: "tiles" (clustered Gaussian) or "field"
     field_tau: float = 4.0            # "field": peak logit contrast of the smooth field
     field_ell: Tuple[float, float, float] = (2.0, 6.0, 6.0)  # "field": length scales (t, y, x)

@@ -37,6 +37,7 @@ struct Layout {
   uint64_t seed;
   int semantic;         // 1: k-means on the raw keys and queries (M = I, Gc = I, scale 1)
   int repair;           // 1: fit and add the probe-residual correction
+  int correction;       // SPARSEPR_CORRECTION_AFFINE / _MEAN
 
   // status + per-head statistics
   int* status;                    // [1]

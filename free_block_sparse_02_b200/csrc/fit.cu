@@ -300,6 +300,21 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
     ridge_span_basis(L, bh, shs, ldiag);
     return;
   }
+  if (L.correction == SPARSEPR_CORRECTION_MEAN) {
+    // Table 4 "Mean-only": the constant feature alone, A_lin = 0 and intercept
+    // (sum w + lam)^-1 sum w R, i.e. row d of B over G[d][d] (+ lam; lam < 0 selects
+    // 1e-3 * sum w, the rule of the 1 x 1 Gram)
+    const double sw = Gg[(size_t)d * n1 + d];
+    const double lam = L.lambda >= 0.0 ? L.lambda : 1e-3 * sw;
+    const double* Bg = L.ridgeB + (size_t)bh * n1 * d;
+    const double den = sw + lam;
+    for (int e = tid; e < n1 * d; e += blockDim.x) A[e] = (e >= d * d && den > 0.0) ? Bg[e] / den : 0.0;
+    if (tid == 0) {
+      st.lambda = lam;
+      st.fit_retries = 0;
+    }
+    return;
+  }
   double tr = 0.0;
   for (int i = tid; i < n1; i += blockDim.x) tr += Gg[i * n1 + i];
   tr = block_sum(tr, red);

@@ -1015,8 +1015,9 @@ __global__ void __launch_bounds__(256) route_build_kernel(Layout L, int tile_m) 
 // (P n_g mod N, ties to the lower g); member floor((2i+1) n_g / (2 m_g)) of group g in token
 // order; weight n_g / m_g scaled to sum P.  Output in ascending token order.
 // ------------------------------------------------------------------------------------------
+constexpr int kProbeTab = 4 * kMaxProbes;  // random mode: open-addressing table of the swapped slots
 constexpr size_t kProbeSmem = kMaxProbes * (sizeof(double) + sizeof(int)) + kMaxGroups * sizeof(long long) +
-                              (2 * kMaxGroups + 1) * sizeof(int);
+                              (2 * kMaxGroups + 1) * sizeof(int) + 2 * kProbeTab * sizeof(int);
 
 __global__ void __launch_bounds__(1024) probe_select_kernel(Layout L) {
   pdl_entry();
@@ -1037,6 +1038,42 @@ __global__ void __launch_bounds__(1024) probe_select_kernel(Layout L) {
       cw[i] = 1.0;
     }
     if (tid == 0) s_sum = (double)P;
+  } else if (L.probe_mode == SPARSEPR_PROBE_RANDOM) {
+    // P distinct rows: partial Fisher-Yates over [0, N) driven by SplitMix64 on the head's
+    // probe stream (seed + 2^63 + 2 bh); the few slots a draw touches (at most 2P) live in an
+    // open-addressing table (load <= 1/2)
+    int* hk = slot + kMaxGroups + 1;  // [kProbeTab] slot index, -1 = empty
+    int* hv = hk + kProbeTab;         // [kProbeTab] value now in that slot
+    for (int i = tid; i < kProbeTab; i += blockDim.x) hk[i] = -1;
+    for (int i = tid; i < P; i += blockDim.x) cw[i] = 1.0;
+    __syncthreads();
+    if (tid == 0) {
+      auto slot_ref = [&](int sl) -> int* {
+        unsigned h = ((unsigned)sl * 2654435761u) >> 18;  // 14 bits: kProbeTab = 16384
+        while (true) {
+          if (hk[h] == sl) return &hv[h];
+          if (hk[h] == -1) {
+            hk[h] = sl;
+            hv[h] = sl;
+            return &hv[h];
+          }
+          h = (h + 1) & (kProbeTab - 1);
+        }
+      };
+      uint64_t state = L.seed + (1ULL << 63) + 2ULL * (uint64_t)bh;
+      const uint64_t n = (uint64_t)N;
+      for (int i = 0; i < P; ++i) {
+        const uint64_t r = splitmix64_next(state);
+        const int j = i + (int)(r % (n - (uint64_t)i));
+        int* pi = slot_ref(i);
+        int* pj = slot_ref(j);
+        const int vi = *pi, vj = *pj;
+        *pi = vj;
+        *pj = vi;
+        ctok[i] = vj;
+      }
+      s_sum = (double)P;
+    }
   } else {
     const int* qoff = L.qoff + (size_t)bh * (Cq + 1);
     const int* qperm = L.qperm + (size_t)bh * N;

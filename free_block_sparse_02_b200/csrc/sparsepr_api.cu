@@ -41,7 +41,8 @@ sparsepr_status validate(const sparsepr_config* c) {
   if (c->fixed_k < 0) return SPARSEPR_ERR_INVALID_ARG;
   if (c->fixed_k == 0 && !(c->density > 0.f && c->density <= 1.f)) return SPARSEPR_ERR_INVALID_ARG;
   if (c->P < 0 || c->P > c->N || c->P > kMaxProbes) return SPARSEPR_ERR_INVALID_ARG;
-  if (c->probe_mode != SPARSEPR_PROBE_UNIFORM && c->probe_mode != SPARSEPR_PROBE_STRATIFIED)
+  if (c->probe_mode != SPARSEPR_PROBE_UNIFORM && c->probe_mode != SPARSEPR_PROBE_STRATIFIED &&
+      c->probe_mode != SPARSEPR_PROBE_RANDOM)
     return SPARSEPR_ERR_INVALID_ARG;
   if (!isfinite(c->lambda) || c->km_iters < 1 || c->km_iters_warm < 0 || !isfinite(c->km_tol))
     return SPARSEPR_ERR_INVALID_ARG;
@@ -49,6 +50,8 @@ sparsepr_status validate(const sparsepr_config* c) {
   if (c->partition != SPARSEPR_PARTITION_RESPONSE && c->partition != SPARSEPR_PARTITION_SEMANTIC)
     return SPARSEPR_ERR_INVALID_ARG;
   if (c->repair != 0 && c->repair != 1) return SPARSEPR_ERR_INVALID_ARG;
+  if (c->correction != SPARSEPR_CORRECTION_AFFINE && c->correction != SPARSEPR_CORRECTION_MEAN)
+    return SPARSEPR_ERR_INVALID_ARG;
   if ((double)c->B * c->H * c->N * 256.0 > 9.0e18) return SPARSEPR_ERR_INVALID_ARG;
   if (c->d != 64 && c->d != 128) return SPARSEPR_ERR_UNSUPPORTED;
   // rows of the [B*H*N, d] views are int32 in the kernels (tiles of 128 rows)
@@ -81,6 +84,7 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   L.seed = c.seed;
   L.semantic = c.partition == SPARSEPR_PARTITION_SEMANTIC;
   L.repair = c.repair;
+  L.correction = c.correction;
   size_t off = 0;
   auto take = [&](auto*& ptr, size_t bytes) {
     using P_ = std::remove_reference_t<decltype(ptr)>;

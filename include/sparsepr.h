@@ -57,7 +57,10 @@ typedef enum sparsepr_status {
 } sparsepr_status;
 
 enum { SPARSEPR_F32 = 0, SPARSEPR_BF16 = 1 };
-enum { SPARSEPR_PROBE_UNIFORM = 0, SPARSEPR_PROBE_STRATIFIED = 1 };
+/* Probe rows (Table 4, probe selection): uniform rows floor((2i+1)N/(2P)); query-group stratified
+   (the paper's reference setting); or P distinct rows drawn at random (partial Fisher-Yates on
+   SplitMix64 stream seed + 2^63 + 2*(b*H+h)), weight 1 each. */
+enum { SPARSEPR_PROBE_UNIFORM = 0, SPARSEPR_PROBE_STRATIFIED = 1, SPARSEPR_PROBE_RANDOM = 2 };
 
 /* Parameters of one call, as the paper states the problem (abstract; Table C.1; Table 4). */
 typedef struct sparsepr_config {
@@ -72,7 +75,7 @@ typedef struct sparsepr_config {
   int32_t fixed_k;          /* > 0: every query group keeps exactly min(fixed_k, non-empty)
                                key groups and `density` is ignored                              */
   int32_t P;                /* probe rows per head, 0 <= P <= min(N, 4096)                     */
-  int32_t probe_mode;       /* SPARSEPR_PROBE_UNIFORM or SPARSEPR_PROBE_STRATIFIED              */
+  int32_t probe_mode;       /* SPARSEPR_PROBE_UNIFORM, _STRATIFIED or _RANDOM                   */
   double lambda;            /* ridge lambda >= 0; < 0 selects 1e-3 * tr(X^T W X) / (d+1)       */
   int32_t km_iters;         /* Lloyd iteration limit of a cold plan (>= 1)                     */
   int32_t km_iters_warm;    /* limit of a re-plan warm-started from the previous centroids;
@@ -84,7 +87,13 @@ typedef struct sparsepr_config {
                                and the raw queries: the semantic baseline of Table 2)           */
   int32_t repair;           /* 1: fit and add the probe-residual correction (the paper's method);
                                0: unprobed rows keep their block-sparse output                  */
+  int32_t correction;       /* SPARSEPR_CORRECTION_AFFINE (the affine map of [O_sp, 1], the
+                               paper's method) or SPARSEPR_CORRECTION_MEAN (Table 4 "Mean-only":
+                               the weighted mean probe residual, (sum w + lambda)^-1 sum w R,
+                               lambda < 0 selecting 1e-3 * sum w)                               */
 } sparsepr_config;
+
+enum { SPARSEPR_CORRECTION_AFFINE = 0, SPARSEPR_CORRECTION_MEAN = 1 };
 
 enum { SPARSEPR_PARTITION_RESPONSE = 0, SPARSEPR_PARTITION_SEMANTIC = 1 };
 

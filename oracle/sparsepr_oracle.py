@@ -97,6 +97,12 @@ def stream_seed(seed: int, bh: int, stage: int) -> int:
     return (seed + 2 * bh + stage) & _MASK64
 
 
+def probe_stream_seed(seed: int, bh: int) -> int:
+    """Seed of head bh's random probe rows: the k-means streams offset by 2^63, so that no
+    k-means stream of any head coincides with it."""
+    return (seed + (1 << 63) + 2 * bh) & _MASK64
+
+
 # ----------------------------------------------------------------------------------------------
 # Step 1: sampled query rows (abstract: "how their keys respond to sampled queries").
 # ----------------------------------------------------------------------------------------------
@@ -294,6 +300,24 @@ def probes_uniform(N: int, P: int):
     return ((2 * i + 1) * N) // (2 * P), np.ones(P)
 
 
+def probes_random(N: int, P: int, seed: int, bh: int):
+    """Table 4 "Random probes": P distinct rows drawn uniformly at random (the partial
+    Fisher-Yates draw of the k-means initial points, on the head's probe stream), in ascending
+    token order, weight 1 each."""
+    ids = np.sort(np.array(kmeans_init_ids(N, P, probe_stream_seed(seed, bh)), dtype=np.int64))
+    return ids, np.ones(P)
+
+
+def select_probes(cfg, qlabels: np.ndarray, n_qgroups: int, N: int, bh: int):
+    """The probe rows and weights of the configured mode: 0 uniform, 1 query-group stratified
+    (the paper's reference setting), 2 random."""
+    if cfg.probe_mode == 0:
+        return probes_uniform(N, cfg.P)
+    if cfg.probe_mode == 2:
+        return probes_random(N, cfg.P, getattr(cfg, "seed", 0), bh)
+    return probes_stratified(qlabels, n_qgroups, cfg.P)
+
+
 def probes_stratified(qlabels: np.ndarray, n_qgroups: int, P: int):
     """Table 4 "Query group stratified probes" (the reference setting).
 
@@ -398,13 +422,28 @@ class WarmState:
     query_centroids: np.ndarray   # (C_q, C_k) normalised response space
 
 
-def outputs_given_partition(q, k, v, qlabels, klabels, route, probes, weights, lam_cfg, repair=1):
+def mean_fit(osp_p: np.ndarray, odense_p: np.ndarray, w: np.ndarray, lam_cfg: float):
+    """Table 4 "Mean-only" correction family: the weighted ridge with the constant feature
+    alone, A_lin = 0 and intercept (sum_p w_p + lam)^-1 sum_p w_p R_p (lam by the same rule on
+    the 1 x 1 Gram).  Returns A of shape (d+1, d) and lam."""
+    P, d = osp_p.shape
+    A = np.zeros((d + 1, d))
+    if P == 0:
+        return A, 0.0
+    Am, lam = weighted_ridge(np.ones((P, 1)), odense_p - osp_p, w, lam_cfg)
+    A[-1] = Am[0]
+    return A, lam
+
+
+def outputs_given_partition(q, k, v, qlabels, klabels, route, probes, weights, lam_cfg, repair=1, correction=0):
     """Steps 6-9 for a given partition, route table and probe set (repair=0: no correction;
-    unprobed rows keep their sparse output, probe rows their exact one)."""
+    unprobed rows keep their sparse output, probe rows their exact one; correction=1: the
+    mean-only family instead of the affine map of [O_sp, 1])."""
     osp = sparse_attention(q, k, v, qlabels, klabels, route)
     odense = attention(q[probes], k, v)
     if repair:
-        A, lam = ridge_fit(osp[probes], odense, weights, lam_cfg)
+        fit = mean_fit if correction == 1 else ridge_fit
+        A, lam = fit(osp[probes], odense, weights, lam_cfg)
         if len(probes):
             A = restrict_to_residual_span(A, odense - osp[probes], weights)
     else:
@@ -418,8 +457,9 @@ def call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int,
               warm: Optional[WarmState] = None, keep_history: bool = False,
               compute_outputs: bool = True) -> dict:
     """One (batch, head) of one call.  cfg needs: s, n_kgroups, n_qgroups, density, fixed_k,
-    P, probe_mode (0 uniform, 1 stratified), lam, km_iters, km_iters_warm, km_tol, seed, and
-    optionally partition (0 response-coupled, 1 semantic) and repair (1 correct, 0 not)."""
+    P, probe_mode (0 uniform, 1 stratified, 2 random), lam, km_iters, km_iters_warm, km_tol,
+    seed, and optionally partition (0 response-coupled, 1 semantic), repair (1 correct, 0 not)
+    and correction (0 affine map of [O_sp, 1], 1 mean-only)."""
     if getattr(cfg, "partition", 0) == 1:
         return semantic_call_head(q, k, v, cfg, bh, compute_outputs=compute_outputs)
     q = np.asarray(q, dtype=np.float64)
@@ -469,10 +509,7 @@ def call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int,
     density = (cfg.s * N + Ck * N + cfg.P * N + sparse_pairs) / float(N) ** 2
 
     # 7: probes.
-    if cfg.probe_mode == 0:
-        probes, weights = probes_uniform(N, cfg.P)
-    else:
-        probes, weights = probes_stratified(qlabels, Cq, cfg.P)
+    probes, weights = select_probes(cfg, qlabels, Cq, N, bh)
 
     out = dict(sample_rows=rows, klabels=klabels, kcent=kcent, kmeans_k=kk, R=R, Rt=Rt,
                qlabels=qlabels, qcent=qq.centroids, kmeans_q=qq, ksizes=m, qsizes=n,
@@ -480,11 +517,12 @@ def call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int,
                probes=probes, weights=weights)
     if compute_outputs:
         out.update(outputs_given_partition(q, k, v, qlabels, klabels, route, probes, weights, cfg.lam,
-                                           repair=getattr(cfg, "repair", 1)))
+                                           repair=getattr(cfg, "repair", 1),
+                                           correction=getattr(cfg, "correction", 0)))
     return out
 
 
-def route_and_probe(q, klabels, qlabels, kcent, cfg):
+def route_and_probe(q, klabels, qlabels, kcent, cfg, bh: int = 0):
     """Steps 5 and 7 for a given partition: routes, realised density and probes."""
     N = q.shape[0]
     Ck, Cq = cfg.n_kgroups, cfg.n_qgroups
@@ -498,10 +536,7 @@ def route_and_probe(q, klabels, qlabels, kcent, cfg):
             route[g, route_group(S[g], m, cfg.fixed_k, kappa)] = True
     sparse_pairs = int(sum(int(n[g]) * int(m[route[g]].sum()) for g in range(Cq)))
     density = (cfg.s * N + Ck * N + cfg.P * N + sparse_pairs) / float(N) ** 2
-    if cfg.probe_mode == 0:
-        probes, weights = probes_uniform(N, cfg.P)
-    else:
-        probes, weights = probes_stratified(qlabels, Cq, cfg.P)
+    probes, weights = select_probes(cfg, qlabels, Cq, N, bh)
     return dict(ksizes=m, qsizes=n, scores=S, kappa=kappa, route=route, sparse_pairs=sparse_pairs,
                 density=density, probes=probes, weights=weights)
 
@@ -526,10 +561,11 @@ def semantic_call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int
     qq = lloyd(q, q[ids], cfg.km_iters, tol)
     out = dict(klabels=kk.labels, kcent=kk.centroids, kmeans_k=kk, qlabels=qq.labels, qcent=qq.centroids,
                kmeans_q=qq)
-    out.update(route_and_probe(q, kk.labels, qq.labels, kk.centroids, cfg))
+    out.update(route_and_probe(q, kk.labels, qq.labels, kk.centroids, cfg, bh))
     if compute_outputs:
         out.update(outputs_given_partition(q, k, v, qq.labels, kk.labels, out["route"], out["probes"],
-                                           out["weights"], cfg.lam, repair=getattr(cfg, "repair", 1)))
+                                           out["weights"], cfg.lam, repair=getattr(cfg, "repair", 1),
+                                           correction=getattr(cfg, "correction", 0)))
     return out
 
 

@@ -41,8 +41,8 @@ def labels_match(gpu_labels, km: O.KMeansResult, what: str):
         assert np.all(km.near_tie_mask[mism]), f"{what}: mismatches outside the oracle's near-ties"
 
 
-def oracle_routing_on(q, klabels, qlabels, kcent, w):
-    """The oracle's routing and probe choice (steps 5 and 7) on a given partition."""
+def oracle_routing_on(q, klabels, qlabels, kcent, w, bh=0):
+    """The oracle's routing and probe choice (steps 5 and 7) on a given partition of head bh."""
     Ck, Cq = w.n_kgroups, w.n_qgroups
     m = np.bincount(klabels, minlength=Ck)
     n = np.bincount(qlabels, minlength=Cq)
@@ -52,10 +52,7 @@ def oracle_routing_on(q, klabels, qlabels, kcent, w):
     for g in range(Cq):
         if n[g] > 0:
             route[g, O.route_group(S[g], m, w.fixed_k, kappa)] = True
-    if w.probe_mode == 0:
-        probes, weights = O.probes_uniform(q.shape[0], w.P)
-    else:
-        probes, weights = O.probes_stratified(qlabels, Cq, w.P)
+    probes, weights = O.select_probes(w, qlabels, Cq, q.shape[0], bh)
     pairs = int(sum(int(n[g]) * int(m[route[g]].sum()) for g in range(Cq)))
     return route, probes, weights, pairs
 
@@ -82,7 +79,7 @@ def compare_partition(op, res_list, w, qf=None):
             np.testing.assert_allclose(kc[bh], r["kcent"], rtol=1e-9, atol=1e-9)
         else:
             assert qf is not None, "labels differ at near-ties: pass the inputs to re-derive the routing"
-            ref_route, ref_probes, ref_w, ref_pairs = oracle_routing_on(qf[bh], kl[bh], ql[bh], kc[bh], w)
+            ref_route, ref_probes, ref_w, ref_pairs = oracle_routing_on(qf[bh], kl[bh], ql[bh], kc[bh], w, bh)
         assert np.array_equal(route[bh].astype(bool), ref_route), f"head {bh} routes"
         assert np.array_equal(probes[bh], ref_probes), f"head {bh} probes"
         np.testing.assert_allclose(pw[bh], ref_w, rtol=1e-12)
@@ -150,11 +147,12 @@ def compare_outputs(op, out, qf, kf, vf, w, atol, rel_l2):
     for bh in range(O_gpu.shape[0]):
         p = probes[bh]
         ref = O.outputs_given_partition(qf[bh], kf[bh], vf[bh], ql[bh], kl[bh], route[bh], p, pw[bh], w.lam,
-                                        repair=w.repair)
+                                        repair=w.repair, correction=w.correction)
         _close(f"head {bh} O_sp", osp[bh], ref["osp"], atol, rel_l2)
         _close(f"head {bh} O_dense", od[bh], ref["odense"], atol, rel_l2)
         if w.repair:
-            A_full, _ = O.ridge_fit(osp[bh][p], od[bh], pw[bh], w.lam)
+            fit = O.mean_fit if w.correction == configs.CORRECTION_MEAN else O.ridge_fit
+            A_full, _ = fit(osp[bh][p], od[bh], pw[bh], w.lam)
             A_ref = O.restrict_to_residual_span(A_full, od[bh] - osp[bh][p], pw[bh]) if len(p) else A_full
             fit_matches(A_gpu[bh], A_full, A_ref, od[bh] - osp[bh][p], pw[bh], f"head {bh} fit")
         else:
@@ -228,6 +226,13 @@ EDGE = {
                                   km_iters=6),
     # smooth-field inputs: no cluster structure, so more points sit near group boundaries
     "field-inputs": dict(base=1, grid=(8, 16, 32), heads=2, recipe="field"),
+    # Table 4's other probe selection and correction family, and the pages' absolute lambda = 1
+    "random-probes": dict(base=1, grid=(4, 16, 32), heads=2, s=64, n_kgroups=16, n_qgroups=12, P=80,
+                          probe_mode=configs.PROBE_RANDOM, km_iters=6),
+    "mean-only": dict(base=1, grid=(4, 16, 32), heads=2, s=64, n_kgroups=16, n_qgroups=12, P=80,
+                      correction=configs.CORRECTION_MEAN, km_iters=6),
+    "lambda-one-d128": dict(base=2, grid=(3, 10, 20), heads=2, s=96, n_kgroups=16, n_qgroups=12, P=160, lam=1.0,
+                            km_iters=8),
 }
 
 
@@ -343,7 +348,7 @@ def test_dit13b_full_size_sampled():
         if np.array_equal(kl[h], r["klabels"]) and np.array_equal(ql[h], r["qlabels"]):
             ref_route, ref_probes, ref_w, ref_pairs = r["route"], r["probes"], r["weights"], r["sparse_pairs"]
         else:
-            ref_route, ref_probes, ref_w, ref_pairs = oracle_routing_on(q, kl[h], ql[h], kc[h], w)
+            ref_route, ref_probes, ref_w, ref_pairs = oracle_routing_on(q, kl[h], ql[h], kc[h], w, h)
         assert np.array_equal(route[h], ref_route), f"head {h} routes"
         assert np.array_equal(probes[h], ref_probes), f"head {h} probes"
         np.testing.assert_allclose(pw[h], ref_w, rtol=1e-12)

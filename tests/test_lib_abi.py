@@ -51,7 +51,8 @@ def test_workspace_size_for_every_workload(lib):
     ("d", 96, 2), ("d", 0, 2), ("N", 0, 1), ("s", 0, 1), ("s", 2000, 1), ("n_kgroups", 0, 1),
     ("n_kgroups", 1025, 1), ("n_kgroups", 2000, 1), ("n_qgroups", 2000, 1), ("P", -1, 1),
     ("P", 5000, 1), ("probe_mode", 7, 1), ("dtype", 3, 1), ("km_iters", 0, 1), ("km_iters_warm", -2, 1),
-    ("partition", 2, 1), ("partition", -1, 1), ("repair", 2, 1), ("repair", -1, 1),
+    ("partition", 2, 1), ("partition", -1, 1), ("repair", 2, 1), ("repair", -1, 1), ("probe_mode", 3, 1),
+    ("probe_mode", -1, 1), ("correction", 2, 1), ("correction", -1, 1),
 ])
 def test_invalid_configs_are_rejected_on_the_host(lib, field, value, code):
     w = configs.workload(0)
@@ -62,6 +63,13 @@ def test_invalid_configs_are_rejected_on_the_host(lib, field, value, code):
 
 def test_semantic_partition_without_repair_is_accepted(lib):
     cfg = _lib.config_from(configs.workload(1), partition=configs.PARTITION_SEMANTIC, repair=0)
+    n = ctypes.c_size_t(0)
+    assert lib.sparsepr_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == 0 and n.value > 0
+
+
+def test_random_probes_and_mean_only_correction_are_accepted(lib):
+    cfg = _lib.config_from(configs.workload(1), probe_mode=configs.PROBE_RANDOM,
+                           correction=configs.CORRECTION_MEAN)
     n = ctypes.c_size_t(0)
     assert lib.sparsepr_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == 0 and n.value > 0
 

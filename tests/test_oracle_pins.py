@@ -412,6 +412,43 @@ def test_repair_reduces_error_on_smooth_field_inputs():
     assert O.error_reduction(err["sparsepr"], err["semantic"]) > 0.5, err
 
 
+def test_random_probes_are_the_seeded_fisher_yates_draw():
+    """Random probe rows: P distinct rows of [0, N), ascending, weight 1; the same rows as a
+    brute-force partial Fisher-Yates over an explicit array driven by the SplitMix64 outputs;
+    a different head (or seed) gives a different draw; P = N gives every row."""
+    N, P, seed = 500, 40, 77
+    ids, w = O.probes_random(N, P, seed, bh=3)
+    assert ids.shape == (P,) and np.all(np.diff(ids) > 0) and ids.min() >= 0 and ids.max() < N
+    assert np.all(w == 1.0)
+    rng = O.SplitMix64((seed + (1 << 63) + 2 * 3) & ((1 << 64) - 1))
+    arr = list(range(N))
+    for i in range(P):
+        j = i + rng.next() % (N - i)
+        arr[i], arr[j] = arr[j], arr[i]
+    assert np.array_equal(ids, np.sort(arr[:P]))
+    assert not np.array_equal(ids, O.probes_random(N, P, seed, bh=4)[0])
+    assert np.array_equal(O.probes_random(64, 64, seed, bh=0)[0], np.arange(64))
+    # the probe stream never coincides with a k-means stream of any head
+    assert all(O.probe_stream_seed(seed, b) != O.stream_seed(seed, h, st)
+               for b in range(8) for h in range(8) for st in (0, 1))
+
+
+def test_mean_only_correction_is_the_weighted_mean_residual():
+    """Table 4's mean-only family: no linear part and the weighted mean probe residual as the
+    intercept (lambda = 0), shrunk by lambda otherwise, and the automatic lambda is 1e-3 of the
+    weight sum."""
+    rng = np.random.default_rng(11)
+    osp, od = rng.standard_normal((30, 5)), rng.standard_normal((30, 5))
+    w = rng.uniform(0.5, 2.0, 30)
+    A, lam = O.mean_fit(osp, od, w, 0.0)
+    assert lam == 0.0 and not np.any(A[:-1])
+    np.testing.assert_allclose(A[-1], (w[:, None] * (od - osp)).sum(0) / w.sum(), rtol=1e-13)
+    A1, _ = O.mean_fit(osp, od, w, 2.5)
+    np.testing.assert_allclose(A1[-1], (w[:, None] * (od - osp)).sum(0) / (w.sum() + 2.5), rtol=1e-13)
+    _, lam_auto = O.mean_fit(osp, od, w, -1.0)
+    assert np.isclose(lam_auto, 1e-3 * w.sum(), rtol=1e-13)
+
+
 def test_mean_error_is_the_row_error_mean():
     rng = np.random.default_rng(3)
     O_, R_ = rng.standard_normal((6, 4)), rng.standard_normal((6, 4))
