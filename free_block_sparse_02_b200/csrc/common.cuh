@@ -38,6 +38,7 @@ struct Layout {
   int semantic;         // 1: k-means on the raw keys and queries (M = I, Gc = I, scale 1)
   int repair;           // 1: fit and add the probe-residual correction
   int correction;       // SPARSEPR_CORRECTION_AFFINE / _MEAN
+  int trunc_rank;       // 0: whole residual span; r: its r leading eigenvectors
 
   // status + per-head statistics
   int* status;                    // [1]

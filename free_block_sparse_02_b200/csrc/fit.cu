@@ -149,6 +149,117 @@ __device__ bool gj_inverse_spd(double* G, int n, int ld) {
   return true;
 }
 
+// The r leading eigenvectors of S = R^T W R (Table D.2's output truncation), by the parallel
+// cyclic Jacobi method in fp64 (Golub & Van Loan, "Matrix Computations", the symmetric Schur
+// rotation and the round-robin ordering): S in shared memory, the accumulated rotations V in the
+// head's spanS (global, where S came from).  A round applies d/2 disjoint rotations, chosen by the
+// circle method so that every (p, q) pair meets once per sweep; sweeps run until the
+// off-diagonal mass is below 1e-30 of the total (squared) or kJacobiSweeps.  The eigenvectors of
+// eigenvalue above 1e-10 of the largest are ranked by eigenvalue (ties: lower index) and the
+// first min(r, count) become the basis; the count goes to span_rank.
+constexpr int kJacobiSweeps = 30;
+
+__device__ __noinline__ void span_basis_truncated(const Layout& L, int bh, double* S) {
+  const int d = L.d, tid = threadIdx.x, nt = blockDim.x, half = d / 2;
+  double* V = L.spanS + (size_t)bh * d * d;
+  __shared__ double rc[64], rs[64];
+  __shared__ int rp[64], rq[64];
+  __shared__ double ev[128];
+  __shared__ int order[128];
+  __shared__ double red2[2][8];
+  __shared__ int s_kept;
+  for (int e = tid; e < d * d; e += nt) S[e] = V[e];
+  __syncthreads();
+  for (int e = tid; e < d * d; e += nt) V[e] = (e / d == e % d) ? 1.0 : 0.0;
+  __syncthreads();
+  for (int sweep = 0; sweep < kJacobiSweeps; ++sweep) {
+    double off = 0.0, tot = 0.0;
+    for (int e = tid; e < d * d; e += nt) {
+      const double x = S[e] * S[e];
+      tot += x;
+      if (e / d != e % d) off += x;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      off += __shfl_xor_sync(0xffffffffu, off, o);
+      tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    }
+    if ((tid & 31) == 0) {
+      red2[0][tid >> 5] = off;
+      red2[1][tid >> 5] = tot;
+    }
+    __syncthreads();
+    off = 0.0;
+    tot = 0.0;
+    for (int w = 0; w < nt / 32; ++w) {
+      off += red2[0][w];
+      tot += red2[1][w];
+    }
+    __syncthreads();
+    if (!(off > 1e-30 * tot)) break;  // the same in every thread (also for a zero S)
+    for (int round = 0; round < d - 1; ++round) {
+      if (tid < half) {
+        const int k = tid;
+        const int a = k == 0 ? 0 : 1 + (k - 1 + round) % (d - 1);
+        const int b = 1 + (d - 2 - k + round) % (d - 1);
+        const int p = min(a, b), q = max(a, b);
+        const double apq = S[p * d + q];
+        double c = 1.0, sn = 0.0;
+        if (apq != 0.0) {
+          const double tau = (S[q * d + q] - S[p * d + p]) / (2.0 * apq);
+          const double t = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
+          c = 1.0 / sqrt(1.0 + t * t);
+          sn = t * c;
+        }
+        rp[k] = p;
+        rq[k] = q;
+        rc[k] = c;
+        rs[k] = sn;
+      }
+      __syncthreads();
+      for (int e = tid; e < half * d; e += nt) {  // S <- S J (columns p, q of every row)
+        const int k = e / d, i = e % d, p = rp[k], q = rq[k];
+        const double c = rc[k], sn = rs[k], x = S[i * d + p], y = S[i * d + q];
+        S[i * d + p] = c * x - sn * y;
+        S[i * d + q] = sn * x + c * y;
+      }
+      __syncthreads();
+      for (int e = tid; e < half * d; e += nt) {  // S <- J^T S (rows p, q), V <- V J
+        const int k = e / d, j = e % d, p = rp[k], q = rq[k];
+        const double c = rc[k], sn = rs[k];
+        const double x = S[p * d + j], y = S[q * d + j];
+        S[p * d + j] = c * x - sn * y;
+        S[q * d + j] = sn * x + c * y;
+        const double u = V[j * d + p], v = V[j * d + q];
+        V[j * d + p] = c * u - sn * v;
+        V[j * d + q] = sn * u + c * v;
+      }
+      __syncthreads();
+    }
+  }
+  // eigenvalues, the kept ones ranked by size, the leading min(r, kept) columns of V
+  for (int i = tid; i < d; i += nt) ev[i] = S[i * d + i];
+  __syncthreads();
+  double top = 0.0;
+  for (int i = 0; i < d; ++i) top = fmax(top, ev[i]);
+  const double thr = 1e-10 * top;
+  if (tid == 0) s_kept = 0;
+  __syncthreads();
+  for (int i = tid; i < d; i += nt) {
+    if (top > 0.0 && ev[i] > thr) {
+      int rk = 0;
+      for (int j = 0; j < d; ++j) rk += ev[j] > thr && (ev[j] > ev[i] || (ev[j] == ev[i] && j < i));
+      order[rk] = i;
+      atomicAdd(&s_kept, 1);
+    }
+  }
+  __syncthreads();
+  const int rank = min(L.trunc_rank, s_kept);
+  for (int e = tid; e < d * rank; e += nt) S[e] = V[(e / rank) * d + order[e % rank]];  // [d][rank]
+  __syncthreads();
+  for (int e = tid; e < d * rank; e += nt) V[(e / rank) * d + e % rank] = S[e];  // U[i*d + r]
+  if (tid == 0) L.stats[bh].span_rank = rank;
+}
+
 // The residual-span basis of head bh (role 1 of ridge_solve_kernel): span of the residual rows
 // = range(S), S = R^T W R, whose rank goes to the head's statistics and whose basis (when the
 // rank is below d) goes to spanS for the projection kernel.
@@ -297,7 +408,10 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
     return;
   }
   if (role == 1) {
-    ridge_span_basis(L, bh, shs, ldiag);
+    if (L.trunc_rank > 0 && L.trunc_rank < d)
+      span_basis_truncated(L, bh, shs);
+    else
+      ridge_span_basis(L, bh, shs, ldiag);
     return;
   }
   if (L.correction == SPARSEPR_CORRECTION_MEAN) {

@@ -52,6 +52,7 @@ sparsepr_status validate(const sparsepr_config* c) {
   if (c->repair != 0 && c->repair != 1) return SPARSEPR_ERR_INVALID_ARG;
   if (c->correction != SPARSEPR_CORRECTION_AFFINE && c->correction != SPARSEPR_CORRECTION_MEAN)
     return SPARSEPR_ERR_INVALID_ARG;
+  if (c->trunc_rank < 0 || c->trunc_rank > c->d) return SPARSEPR_ERR_INVALID_ARG;
   if ((double)c->B * c->H * c->N * 256.0 > 9.0e18) return SPARSEPR_ERR_INVALID_ARG;
   if (c->d != 64 && c->d != 128) return SPARSEPR_ERR_UNSUPPORTED;
   // rows of the [B*H*N, d] views are int32 in the kernels (tiles of 128 rows)
@@ -85,6 +86,7 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   L.semantic = c.partition == SPARSEPR_PARTITION_SEMANTIC;
   L.repair = c.repair;
   L.correction = c.correction;
+  L.trunc_rank = c.trunc_rank;
   size_t off = 0;
   auto take = [&](auto*& ptr, size_t bytes) {
     using P_ = std::remove_reference_t<decltype(ptr)>;

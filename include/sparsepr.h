@@ -91,6 +91,9 @@ typedef struct sparsepr_config {
                                paper's method) or SPARSEPR_CORRECTION_MEAN (Table 4 "Mean-only":
                                the weighted mean probe residual, (sum w + lambda)^-1 sum w R,
                                lambda < 0 selecting 1e-3 * sum w)                               */
+  int32_t trunc_rank;       /* 0: the map's outputs restricted to the whole probe-residual span
+                               (the identity on the ridge solution); 1 <= r <= d: to the r leading
+                               eigenvectors of R^T W R (Table D.2's output truncation)           */
 } sparsepr_config;
 
 enum { SPARSEPR_CORRECTION_AFFINE = 0, SPARSEPR_CORRECTION_MEAN = 1 };

@@ -382,24 +382,31 @@ def weighted_ridge(X: np.ndarray, R: np.ndarray, w: np.ndarray, lam_cfg: float):
     return A, lam
 
 
-def residual_span_basis(R: np.ndarray, w: np.ndarray) -> np.ndarray:
+def residual_span_basis(R: np.ndarray, w: np.ndarray, rank: int = 0) -> np.ndarray:
     """Orthonormal basis (d, r) of the span of the probe residual rows: eigenvectors of
-    R^T W R with eigenvalue above SPAN_REL_TOL of the largest (none if all are zero)."""
+    R^T W R with eigenvalue above SPAN_REL_TOL of the largest (none if all are zero).
+    rank > 0 truncates it to the `rank` eigenvectors of largest eigenvalue (Table D.2's output
+    truncation; reading: the low-rank probe-residual subspace is the leading one)."""
     d = R.shape[1]
     Sg = R.T @ (w[:, None] * R)
     ev, U = np.linalg.eigh(Sg)
     top = ev.max() if ev.size else 0.0
     if not top > 0:
         return np.zeros((d, 0))
-    return U[:, ev > SPAN_REL_TOL * top]
+    keep = ev > SPAN_REL_TOL * top
+    U, ev = U[:, keep], ev[keep]
+    if rank > 0 and U.shape[1] > rank:
+        U = U[:, np.argsort(-ev, kind="stable")[:rank]]
+    return U
 
 
-def restrict_to_residual_span(A: np.ndarray, R: np.ndarray, w: np.ndarray) -> np.ndarray:
+def restrict_to_residual_span(A: np.ndarray, R: np.ndarray, w: np.ndarray, rank: int = 0) -> np.ndarray:
     """Project the fitted map's outputs onto the probe-residual subspace (arXiv abstract:
     "within the output subspace observed in the probe residuals"): A <- A U U^T.
-    Without truncation the ridge solution already lies in that span (each output of A is a
-    combination of residual rows), so this is the identity up to rounding."""
-    U = residual_span_basis(R, w)
+    Without truncation (rank 0) the ridge solution already lies in that span (each output of A
+    is a combination of residual rows), so this is the identity up to rounding; with rank r the
+    outputs keep only their part along the r leading residual directions."""
+    U = residual_span_basis(R, w, rank)
     return A @ U @ U.T
 
 
@@ -435,17 +442,19 @@ def mean_fit(osp_p: np.ndarray, odense_p: np.ndarray, w: np.ndarray, lam_cfg: fl
     return A, lam
 
 
-def outputs_given_partition(q, k, v, qlabels, klabels, route, probes, weights, lam_cfg, repair=1, correction=0):
+def outputs_given_partition(q, k, v, qlabels, klabels, route, probes, weights, lam_cfg, repair=1, correction=0,
+                            trunc_rank=0):
     """Steps 6-9 for a given partition, route table and probe set (repair=0: no correction;
     unprobed rows keep their sparse output, probe rows their exact one; correction=1: the
-    mean-only family instead of the affine map of [O_sp, 1])."""
+    mean-only family instead of the affine map of [O_sp, 1]; trunc_rank r > 0: the map's outputs
+    restricted to the r leading residual directions)."""
     osp = sparse_attention(q, k, v, qlabels, klabels, route)
     odense = attention(q[probes], k, v)
     if repair:
         fit = mean_fit if correction == 1 else ridge_fit
         A, lam = fit(osp[probes], odense, weights, lam_cfg)
         if len(probes):
-            A = restrict_to_residual_span(A, odense - osp[probes], weights)
+            A = restrict_to_residual_span(A, odense - osp[probes], weights, trunc_rank)
     else:
         A, lam = np.zeros((q.shape[1] + 1, q.shape[1])), 0.0
     O = apply_correction(osp, A)
@@ -458,8 +467,9 @@ def call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int,
               compute_outputs: bool = True) -> dict:
     """One (batch, head) of one call.  cfg needs: s, n_kgroups, n_qgroups, density, fixed_k,
     P, probe_mode (0 uniform, 1 stratified, 2 random), lam, km_iters, km_iters_warm, km_tol,
-    seed, and optionally partition (0 response-coupled, 1 semantic), repair (1 correct, 0 not)
-    and correction (0 affine map of [O_sp, 1], 1 mean-only)."""
+    seed, and optionally partition (0 response-coupled, 1 semantic), repair (1 correct, 0 not),
+    correction (0 affine map of [O_sp, 1], 1 mean-only) and trunc_rank (0 none, r > 0 the r
+    leading residual directions)."""
     if getattr(cfg, "partition", 0) == 1:
         return semantic_call_head(q, k, v, cfg, bh, compute_outputs=compute_outputs)
     q = np.asarray(q, dtype=np.float64)
@@ -518,7 +528,8 @@ def call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int,
     if compute_outputs:
         out.update(outputs_given_partition(q, k, v, qlabels, klabels, route, probes, weights, cfg.lam,
                                            repair=getattr(cfg, "repair", 1),
-                                           correction=getattr(cfg, "correction", 0)))
+                                           correction=getattr(cfg, "correction", 0),
+                                           trunc_rank=getattr(cfg, "trunc_rank", 0)))
     return out
 
 
@@ -565,7 +576,8 @@ def semantic_call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int
     if compute_outputs:
         out.update(outputs_given_partition(q, k, v, qq.labels, kk.labels, out["route"], out["probes"],
                                            out["weights"], cfg.lam, repair=getattr(cfg, "repair", 1),
-                                           correction=getattr(cfg, "correction", 0)))
+                                           correction=getattr(cfg, "correction", 0),
+                                           trunc_rank=getattr(cfg, "trunc_rank", 0)))
     return out
 
 

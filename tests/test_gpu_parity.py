@@ -147,13 +147,14 @@ def compare_outputs(op, out, qf, kf, vf, w, atol, rel_l2):
     for bh in range(O_gpu.shape[0]):
         p = probes[bh]
         ref = O.outputs_given_partition(qf[bh], kf[bh], vf[bh], ql[bh], kl[bh], route[bh], p, pw[bh], w.lam,
-                                        repair=w.repair, correction=w.correction)
+                                        repair=w.repair, correction=w.correction, trunc_rank=w.trunc_rank)
         _close(f"head {bh} O_sp", osp[bh], ref["osp"], atol, rel_l2)
         _close(f"head {bh} O_dense", od[bh], ref["odense"], atol, rel_l2)
         if w.repair:
             fit = O.mean_fit if w.correction == configs.CORRECTION_MEAN else O.ridge_fit
             A_full, _ = fit(osp[bh][p], od[bh], pw[bh], w.lam)
-            A_ref = O.restrict_to_residual_span(A_full, od[bh] - osp[bh][p], pw[bh]) if len(p) else A_full
+            A_ref = (O.restrict_to_residual_span(A_full, od[bh] - osp[bh][p], pw[bh], w.trunc_rank) if len(p)
+                     else A_full)
             fit_matches(A_gpu[bh], A_full, A_ref, od[bh] - osp[bh][p], pw[bh], f"head {bh} fit")
         else:
             assert not np.any(A_gpu[bh]), f"head {bh}: no correction without repair"
@@ -233,6 +234,15 @@ EDGE = {
                       correction=configs.CORRECTION_MEAN, km_iters=6),
     "lambda-one-d128": dict(base=2, grid=(3, 10, 20), heads=2, s=96, n_kgroups=16, n_qgroups=12, P=160, lam=1.0,
                             km_iters=8),
+    # more than 256 groups (the pages' own configuration has 1000 key and 300 query groups): the
+    # CUDA-core k-means path for bf16, and key groups of a few rows (sub-box segments)
+    # Table D.2's output truncation: the map restricted to the r leading residual directions
+    "truncated-span-d64": dict(base=1, grid=(4, 16, 32), heads=2, s=64, n_kgroups=16, n_qgroups=12, P=96,
+                               trunc_rank=8, km_iters=6),
+    "truncated-span-d128": dict(base=2, grid=(3, 10, 20), heads=2, s=96, n_kgroups=16, n_qgroups=12, P=160,
+                                trunc_rank=16, km_iters=8),
+    "many-groups": dict(base=1, grid=(4, 16, 32), heads=1, s=128, n_kgroups=600, n_qgroups=300, P=64, lam=1.0,
+                        km_iters=5),
 }
 
 

@@ -52,7 +52,8 @@ def test_workspace_size_for_every_workload(lib):
     ("n_kgroups", 1025, 1), ("n_kgroups", 2000, 1), ("n_qgroups", 2000, 1), ("P", -1, 1),
     ("P", 5000, 1), ("probe_mode", 7, 1), ("dtype", 3, 1), ("km_iters", 0, 1), ("km_iters_warm", -2, 1),
     ("partition", 2, 1), ("partition", -1, 1), ("repair", 2, 1), ("repair", -1, 1), ("probe_mode", 3, 1),
-    ("probe_mode", -1, 1), ("correction", 2, 1), ("correction", -1, 1),
+    ("probe_mode", -1, 1), ("correction", 2, 1), ("correction", -1, 1), ("trunc_rank", -1, 1),
+    ("trunc_rank", 65, 1),
 ])
 def test_invalid_configs_are_rejected_on_the_host(lib, field, value, code):
     w = configs.workload(0)

@@ -449,6 +449,26 @@ def test_mean_only_correction_is_the_weighted_mean_residual():
     assert np.isclose(lam_auto, 1e-3 * w.sum(), rtol=1e-13)
 
 
+def test_truncated_span_is_the_leading_right_singular_subspace():
+    """Output truncation to rank r keeps the r leading eigenvectors of R^T W R, i.e. the r
+    leading right singular vectors of W^(1/2) R (checked against the SVD); rank >= the
+    numerical rank is the untruncated restriction; the projected map keeps exactly its part
+    along those directions."""
+    rng = np.random.default_rng(21)
+    P, d = 40, 6
+    R = rng.standard_normal((P, d)) @ np.diag([5.0, 3.0, 2.0, 1.0, 0.5, 0.1])
+    w = rng.uniform(0.5, 2.0, P)
+    _, _, Vt = np.linalg.svd(np.sqrt(w)[:, None] * R)
+    for r in (1, 2, 4):
+        U = O.residual_span_basis(R, w, r)
+        assert U.shape == (d, r)
+        np.testing.assert_allclose(U @ U.T, Vt[:r].T @ Vt[:r], atol=1e-12)
+    A = rng.standard_normal((d + 1, d))
+    np.testing.assert_allclose(O.restrict_to_residual_span(A, R, w, 2), A @ Vt[:2].T @ Vt[:2], atol=1e-12)
+    np.testing.assert_allclose(O.restrict_to_residual_span(A, R, w, d), O.restrict_to_residual_span(A, R, w, 0),
+                               atol=1e-12)
+
+
 def test_mean_error_is_the_row_error_mean():
     rng = np.random.default_rng(3)
     O_, R_ = rng.standard_normal((6, 4)), rng.standard_normal((6, 4))
