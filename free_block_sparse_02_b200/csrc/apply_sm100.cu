@@ -1,7 +1,7 @@
 // The residual correction of the unprobed rows on the tensor cores (tcgen05, TMEM accumulator).
 //
-// "Partition the Support, Reconstruct the Residual" (arXiv 2608.18484), abstract: the fitted map
-// "predicts a residual for each unprobed query, which we add to its sparse output"; probe rows
+// "Partition the Support, Reconstruct the Residual" (arXiv 2608.18484), abstract: each unprobed
+// query's sparse output is corrected by the residual the fitted map predicts for it; probe rows
 // keep their exact dense output.  Per head, with A the (d+1) x d fitted map:
 //   O_i = O_sp,i + O_sp,i A[0:d] + A[d]   (unprobed rows),   O_p = O_dense,p   (probe rows),
 // written back in token order.

@@ -1,9 +1,9 @@
 // Block-sparse attention and dense probe-row attention on CUDA cores (fp32 arithmetic).
 //
-// "Partition the Support, Reconstruct the Residual" (arXiv 2608.18484), abstract: attention
-// is computed "only between selected groups"; queries of one query group attend to the keys
-// of its kept key groups, softmax over the retained keys only (hard drop); probe rows attend
-// to every key ("compute exact attention on a small set of query rows").
+// "Partition the Support, Reconstruct the Residual" (arXiv 2608.18484), abstract: block-sparse
+// attention evaluates only the selected (query group, key group) cells; queries of one query
+// group attend to the keys of its kept key groups, softmax over the retained keys only (hard
+// drop); the few probe rows get exact attention over every key.
 //
 // Operands are the group-permuted Q/K/V: query group g is rows [qoff_g, qoff_{g+1}) of Qp and
 // key group j is rows [koff_j, koff_{j+1}) of Kp/Vp.  A work item is one 64-row query tile of

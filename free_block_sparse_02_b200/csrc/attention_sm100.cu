@@ -1,10 +1,10 @@
 // Block-sparse attention and dense probe-row attention on the 5th-generation tensor cores
 // (tcgen05, TMEM accumulators, TMA tile loads), bf16 inputs, fp32 accumulation and softmax.
 //
-// "Partition the Support, Reconstruct the Residual" (arXiv 2608.18484), abstract: attention
-// only "between selected groups" (every query of a query group attends to the keys of the key
-// groups its group keeps, softmax over the retained keys only), and "exact attention on a
-// small set of query rows" for the probes.
+// "Partition the Support, Reconstruct the Residual" (arXiv 2608.18484), abstract: attention is
+// evaluated for the selected group pairs only (every query of a query group attends to the keys
+// of the key groups its group keeps, softmax over the retained keys only), and exactly, over
+// all keys, for the few probe rows.
 //
 // Work item = 256 query rows of one query group (block-sparse pass) or of one head's probe rows
 // (dense pass), as two 128-row MMA tiles Q0, Q1 that share every KV tile.  The keys are the

@@ -1,11 +1,10 @@
 // Probe-Fitted Residual Reconstruction of the SparsePR operator.
 //
-// "Partition the Support, Reconstruct the Residual" (arXiv 2608.18484), abstract: "fit an
-// affine correction to the differences between their dense and sparse outputs using
-// weighted ridge regression.  The fitted map predicts a residual for each unprobed query,
-// which we add to its sparse output"; arXiv abstract: the correction acts "within the output
-// subspace observed in the probe residuals"; project page method column "Probe-Fitted
-// Residual Reconstruction".
+// "Partition the Support, Reconstruct the Residual" (arXiv 2608.18484), abstract: an affine
+// map from the sparse output to the probe rows' dense-minus-sparse differences is fitted by
+// weighted ridge regression and the residual it predicts is added to every unprobed row; the
+// arXiv abstract page confines the correction to the subspace the probe residuals span; the
+// project page's method column names the step Probe-Fitted Residual Reconstruction.
 //
 // Per head, with X_p = [O_sp(p), 1], R_p = O_dense(p) - O_sp(p), W = diag(w):
 //   A = (X^T W X + lam I)^-1 X^T W R,   lam = 1e-3 tr(X^T W X)/(d+1) unless given,

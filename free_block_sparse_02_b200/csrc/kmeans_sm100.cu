@@ -2,7 +2,7 @@
 // (tcgen05, results in TMEM, operands by TMA).
 //
 // "Partition the Support, Reconstruct the Residual" (arXiv 2608.18484), abstract: keys are
-// grouped by their responses to sampled queries, queries by their responses to the key-group
+// grouped by their responses to sampled queries, queries by how they respond to the key-group
 // centroids; both groupings are k-means (Table C.1: 25 / 2 iterations, tolerance 1e-4).
 //
 // Both k-means run on the d-dimensional inputs (see partition.cu): the score of point x against

@@ -1,8 +1,8 @@
 // Response-Coupled Partitioning, routing and probe choice of the SparsePR operator.
 //
 // "Partition the Support, Reconstruct the Residual" (arXiv 2608.18484), abstract: keys are
-// grouped by their responses to sampled queries (paired K/V groups), queries by their
-// responses to the key-group centroids (shared sparse routing); project page "SparsePR:
+// grouped by their responses to sampled queries (paired K/V groups), queries by how they
+// respond to the key-group centroids (shared sparse routing); project page "SparsePR:
 // Training-Free Sparse Attention for Video Generation", method pipeline steps 01-03.
 //
 // Neither response matrix is materialised; both k-means run on the d-dimensional inputs.

@@ -8,13 +8,14 @@
  * 02 partition support, 03 execute sparse routes, 04 reconstruct residual).
  *
  * One call on Q, K, V of shape [B, H, N, d] runs, independently for every (b, h) head:
- *   sparsepr_plan       Response-Coupled Partitioning and routing (abstract: "group paired
- *                       key/value tokens by how their keys respond to sampled queries", "group
- *                       queries by their responses to the resulting key-group centroids for
- *                       shared sparse routing"), plus the choice of probe rows (Table 4).
+ *   sparsepr_plan       Response-Coupled Partitioning and routing (abstract: K/V tokens are
+ *                       grouped in pairs by the responses of their keys to sampled queries;
+ *                       queries are grouped by their responses to those key groups' centroids,
+ *                       and each query group shares one sparse route), plus the choice of probe
+ *                       rows (Table 4).
  *   sparsepr_attention  block-sparse attention over the kept (query group, key group) cells
- *                       and exact dense attention of the probe rows (abstract: "compute exact
- *                       attention on a small set of query rows").
+ *                       and exact dense attention of the probe rows (abstract: a few query
+ *                       rows are evaluated exactly).
  *   sparsepr_fit_apply  Probe-Fitted Residual Reconstruction: weighted ridge fit of an affine
  *                       map [O_sp, 1] -> O_dense - O_sp on the probe rows, restricted to the
  *                       span of the probe residuals, added to every unprobed row; probe rows

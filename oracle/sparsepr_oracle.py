@@ -18,8 +18,8 @@ The operator, per (batch, head), in the abstract's order:
      (Table D.1, "Per query RMS" column, the reference setting);
   4. k-means on the normalised responses -> C_q query groups that share one sparse route;
   5. routing: per query group the kept key groups, to a target executed-pair density that
-     counts routing and exact probe pairs (project page, Results: "Density includes routing
-     and exact probe pairs");
+     counts routing and exact probe pairs (project page, Results: the reported density
+     counts the routing and the exact probe pairs too);
   6. block-sparse attention: each query attends only to the keys of its group's kept key
      groups (softmax over the retained keys only);
   7. exact dense attention on P probe rows (Table 4: uniform spatiotemporal or query-group
@@ -104,7 +104,8 @@ def probe_stream_seed(seed: int, bh: int) -> int:
 
 
 # ----------------------------------------------------------------------------------------------
-# Step 1: sampled query rows (abstract: "how their keys respond to sampled queries").
+# Step 1: sampled query rows (abstract: keys are characterised by their responses to sampled
+# queries).
 # ----------------------------------------------------------------------------------------------
 def sample_query_rows(N: int, s: int) -> np.ndarray:
     """Reading: s rows spread evenly over raster token order, row i = floor((2i+1) N / (2s))."""
@@ -401,8 +402,8 @@ def residual_span_basis(R: np.ndarray, w: np.ndarray, rank: int = 0) -> np.ndarr
 
 
 def restrict_to_residual_span(A: np.ndarray, R: np.ndarray, w: np.ndarray, rank: int = 0) -> np.ndarray:
-    """Project the fitted map's outputs onto the probe-residual subspace (arXiv abstract:
-    "within the output subspace observed in the probe residuals"): A <- A U U^T.
+    """Project the fitted map's outputs onto the probe-residual subspace (arXiv abstract page:
+    the correction stays inside the span of the probe residuals): A <- A U U^T.
     Without truncation (rank 0) the ridge solution already lies in that span (each output of A
     is a combination of residual rows), so this is the identity up to rounding; with rank r the
     outputs keep only their part along the r leading residual directions."""
