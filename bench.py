@@ -85,6 +85,8 @@ def profiled_traffic(w):
     """DRAM read + write bytes per attention launch from the committed ncu summary of this
     workload, or None when there is none or the attention source changed since it was taken."""
     import re
+    if w != configs.workload(w.index):  # a sweep or a cut of the workload: not what was profiled
+        return None
     path = os.path.join(ROOT, "profiles", f"attn_tc_kernel_{w.name}.md")
     if not os.path.exists(path):
         return None
