@@ -89,7 +89,13 @@ __global__ void __launch_bounds__(256) ridge_gram_kernel(Layout L) {
 }
 
 // Shared memory of the solve: the (d+1)^2 system and a (d+1) x 33 block of right-hand sides.
-static size_t ridge_solve_smem(int d) { return (size_t)((d + 1) * (d + 1) + (d + 1) * 33) * sizeof(double); }
+// Dynamic shared memory of ridge_solve_kernel: G + lam I and 32 staged columns of B (role 0),
+// S (role 1); at d <= 64 also room for the Jacobi rotations next to S (2 d^2 doubles).
+__host__ __device__ inline size_t ridge_solve_smem(int d) {
+  const size_t base = (size_t)((d + 1) * (d + 1) + (d + 1) * 33) * sizeof(double);
+  const size_t jac = d <= 64 ? (size_t)2 * d * d * sizeof(double) : 0;
+  return base > jac ? base : jac;
+}
 
 // Cholesky G = L L^T of the n x n matrix in shared memory with one barrier per step: step k
 // reads column k of the (lower) trailing matrix, writes L's column k below the diagonal into
@@ -150,8 +156,8 @@ __device__ bool gj_inverse_spd(double* G, int n, int ld) {
 
 // The r leading eigenvectors of S = R^T W R (Table D.2's output truncation), by the parallel
 // cyclic Jacobi method in fp64 (Golub & Van Loan, "Matrix Computations", the symmetric Schur
-// rotation and the round-robin ordering): S in shared memory, the accumulated rotations V in the
-// head's spanS (global, where S came from).  A round applies d/2 disjoint rotations, chosen by the
+// rotation and the round-robin ordering): S in shared memory, the accumulated rotations V next to
+// it when both fit (d = 64), else in the head's spanS (global, where S came from).  A round applies d/2 disjoint rotations, chosen by the
 // circle method so that every (p, q) pair meets once per sweep; sweeps run until the
 // off-diagonal mass is below 1e-30 of the total (squared) or kJacobiSweeps.  The eigenvectors of
 // eigenvalue above 1e-10 of the largest are ranked by eigenvalue (ties: lower index) and the
@@ -160,14 +166,16 @@ constexpr int kJacobiSweeps = 30;
 
 __device__ __noinline__ void span_basis_truncated(const Layout& L, int bh, double* S) {
   const int d = L.d, tid = threadIdx.x, nt = blockDim.x, half = d / 2;
-  double* V = L.spanS + (size_t)bh * d * d;
+  double* Ug = L.spanS + (size_t)bh * d * d;
+  // the rotations accumulate in shared memory next to S when both fit (d = 64), else in L2
+  double* V = (size_t)2 * d * d * sizeof(double) <= ridge_solve_smem(d) ? S + d * d : Ug;
   __shared__ double rc[64], rs[64];
   __shared__ int rp[64], rq[64];
   __shared__ double ev[128];
   __shared__ int order[128];
   __shared__ double red2[2][8];
   __shared__ int s_kept;
-  for (int e = tid; e < d * d; e += nt) S[e] = V[e];
+  for (int e = tid; e < d * d; e += nt) S[e] = Ug[e];
   __syncthreads();
   for (int e = tid; e < d * d; e += nt) V[e] = (e / d == e % d) ? 1.0 : 0.0;
   __syncthreads();
@@ -255,7 +263,7 @@ __device__ __noinline__ void span_basis_truncated(const Layout& L, int bh, doubl
   const int rank = min(L.trunc_rank, s_kept);
   for (int e = tid; e < d * rank; e += nt) S[e] = V[(e / rank) * d + order[e % rank]];  // [d][rank]
   __syncthreads();
-  for (int e = tid; e < d * rank; e += nt) V[(e / rank) * d + e % rank] = S[e];  // U[i*d + r]
+  for (int e = tid; e < d * rank; e += nt) Ug[(e / rank) * d + e % rank] = S[e];  // U[i*d + r]
   if (tid == 0) L.stats[bh].span_rank = rank;
 }
 
