@@ -4,14 +4,16 @@
 One step = one whole operator call (plan: response-coupled partitioning, routing, probes;
 attention: block-sparse + dense probe rows; fit_apply: weighted ridge + residual add) over
 one batch of seeded synthetic video-latent Q/K/V of the chosen workload (default: the
-mid-size bf16 call, B=1 H=8 N=16384 d=64 at 22% density).
+13B-DiT-720p-shaped layer, B=1 H=24 N=118800 d=128 at 22% density, the largest single-GPU
+configuration at that density).
 
-  python bench.py [--gpus N --steps K --warmup W] [--workload I] [--impl reference]
+  python bench.py [--gpus N --steps K --warmup W] [--workload I] [--shard heads] [--impl reference]
 
 Prints one JSON line (rank 0).  `value` is dense-equivalent TFLOPS of all ranks
 (4*B*H*N^2*d per call / device time); `ms_per_step` is milliseconds per call (max over
 ranks).  With N > 1 (torchrun) every rank runs its own independent call on its own inputs
-(heads never exchange data: weak scaling, no collective on the data path).
+(weak scaling, no collective on the data path); with --shard heads the ranks split ONE call by
+heads (strong scaling; --gather adds an NCCL all-gather of the output inside the timed region).
 """
 from __future__ import annotations
 
@@ -66,24 +68,46 @@ def max_over_ranks(values, world, device=None):
     return [float(x) for x in t]
 
 
+def sum_over_ranks(values, world, device=None):
+    """Element-wise sum of `values` over all ranks (identity at world 1)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t]
+
+
 def whole_job_tflops(world, flops_per_call, ms_per_call):
     """Throughput of the whole job: every rank runs one independent call of `flops_per_call`
     (dense-equivalent) per step, and a step lasts `ms_per_call` (the max over ranks)."""
     return world * flops_per_call / (ms_per_call * 1e-3) / 1e12
 
 
+def _strip_comments(text: str) -> str:
+    """C/C++/CUDA source without comments, trailing blanks and empty lines: the code a
+    profile's counters belong to (a comment edit does not void them)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+
+
 def source_hash(*rel):
+    """sha256 of the given sources (paths relative to the repository root), comments stripped."""
     import hashlib
     h = hashlib.sha256()
     for r in rel:
-        with open(os.path.join(ROOT, r), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, r), encoding="utf-8") as f:
+            h.update(_strip_comments(f.read()).encode())
     return h.hexdigest()
+
+
+ATTN_SOURCES = ("free_block_sparse_02_b200/csrc/attention_sm100.cu", "free_block_sparse_02_b200/csrc/sm100.cuh")
 
 
 def profiled_traffic(w):
     """DRAM read + write bytes per attention launch from the committed ncu summary of this
-    workload, or None when there is none or the attention source changed since it was taken."""
+    workload, or None when there is none or the attention code changed since it was taken."""
     import re
     if w != configs.workload(w.index):  # a sweep or a cut of the workload: not what was profiled
         return None
@@ -94,8 +118,7 @@ def profiled_traffic(w):
         text = f.read()
     m = re.search(r"^dram_bytes_per_launch:\s*(\d+)", text, re.M)
     h = re.search(r"^source_sha256:\s*([0-9a-f]{64})", text, re.M)
-    cur = source_hash("free_block_sparse_02_b200/csrc/attention_sm100.cu", "free_block_sparse_02_b200/csrc/sm100.cuh")
-    if not m or not h or h.group(1) != cur:
+    if not m or not h or h.group(1) != source_hash(*ATTN_SOURCES):
         return None
     return int(m.group(1))
 
@@ -172,25 +195,36 @@ def output_quality(S, w, Q, K, V, O_main, main_probes, dev, n_eval=2048):
     dense_op(Q, K, V)
     ref = dense_op.query(S.Q_ODENSE).astype(np.float64)          # [BH, ev, d]
     rows = dense_op.query(S.Q_PROBES)                            # [BH, ev] ascending tokens
+    del dense_op
     sem = S.SparsePR(w, device=dev, partition=configs.PARTITION_SEMANTIC, repair=0)
     O_sem = sem(Q, K, V, out_dtype=O_main.dtype)
     torch.cuda.synchronize(dev)
     BH = w.B * w.H
-    O1 = O_main.float().reshape(BH, w.N, w.d).cpu().numpy().astype(np.float64)
-    O0 = O_sem.float().reshape(BH, w.N, w.d).cpu().numpy().astype(np.float64)
+    # the uniform evaluation rows are the same in every head: gather them on the device
+    idx = torch.from_numpy(rows[0].astype(np.int64)).to(dev)
+    assert (rows == rows[0][None, :]).all()
+    O1 = O_main.reshape(BH, w.N, w.d).index_select(1, idx).float().cpu().numpy().astype(np.float64)
+    O0 = O_sem.reshape(BH, w.N, w.d).index_select(1, idx).float().cpu().numpy().astype(np.float64)
     sem_probes = sem.query(S.Q_PROBES)
+    del sem, O_sem
     e1, e0 = [], []
     for h in range(BH):
         keep = ~np.isin(rows[h], main_probes[h]) & ~np.isin(rows[h], sem_probes[h])
-        r, t = ref[h][keep], rows[h][keep]
+        r = ref[h][keep]
         den = np.linalg.norm(r, axis=1) + 1e-8
-        e1.append(np.linalg.norm(O1[h][t] - r, axis=1) / den)
-        e0.append(np.linalg.norm(O0[h][t] - r, axis=1) / den)
+        e1.append(np.linalg.norm(O1[h][keep] - r, axis=1) / den)
+        e0.append(np.linalg.norm(O0[h][keep] - r, axis=1) / den)
     e1, e0 = np.concatenate(e1), np.concatenate(e0)
     return {"mean_err": float(e1.mean()), "p99_err": float(np.percentile(e1, 99)),
             "semantic_no_repair_mean_err": float(e0.mean()),
             "error_reduction": float(1.0 - e1.mean() / e0.mean()),
             "eval_rows": f"{ev} strided rows per head minus probe rows; output dtype of the call"}
+
+
+QUALITY_NOTE_TILES = ("clustered-tile inputs have independent N(0,1) values: the residual of a dropped key group "
+                      "is an average of unrelated noise, which no affine map of the sparse output predicts, so "
+                      "the fitted correction can raise the error on them (a property of these inputs, not a "
+                      "parity result); quality_field shows the same operator on smooth-field inputs")
 
 
 def km_rooflines(w, asg_ms, upd_ms, pk):
@@ -224,55 +258,131 @@ def km_rooflines(w, asg_ms, upd_ms, pk):
     return out
 
 
+def attention_flops(w, sparse_pairs):
+    """Algorithmic flops of one attention launch: 4 d per executed query-key pair, counting the
+    block-sparse pairs of every row and the probe rows' dense pairs (P N per head), which the
+    same launch computes.  Padding rows and masked keys are not counted."""
+    return 4.0 * w.d * (sparse_pairs + w.B * w.H * w.P * w.N)
+
+
 # ------------------------------------------------------------------------------------ CPU baseline
-def oracle_sample(w, budget_s: float, max_heads=None):
-    """Time the fp64 oracle on whole heads of the workload until `budget_s` is spent."""
-    from oracle import sparsepr_oracle as O
+def _oracle_cores():
     try:
         from threadpoolctl import threadpool_info
-        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=os.cpu_count())
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=os.cpu_count())
     except Exception:
-        cores = os.cpu_count()
-    times = []
-    h = 0
-    max_heads = max_heads or w.H
-    while h < max_heads and (sum(times) < budget_s or not times):
-        Q, K, V = gen.make_qkv(w, heads=[(0, h)])
-        q, k, v = (gen.as_f64(x)[0, h] for x in (Q, K, V))
+        return os.cpu_count()
+
+
+class OracleSample:
+    """The fp64 oracle, as it stands, on a bounded sample of one call of workload `w`.
+
+    One head's partition (steps 1-5 and the probe choice: call_head without outputs) runs once
+    and is timed.  A step then runs the oracle's output steps on that partition: the
+    block-sparse attention of one slice of the query groups (groups g with g mod S = step mod S,
+    S = min(8, C_q) slices, so S consecutive steps cover every group once), the probe rows'
+    dense attention, the ridge fit, its restriction to the residual span and the corrected
+    output.  The time of a whole call is estimated as
+        B * H * (partition + S * mean block-sparse slice time + mean time of the rest),
+    every term measured; it is an extrapolation over heads and slices, and says so."""
+
+    def __init__(self, w, head=0):
+        import numpy as np
+        from oracle import sparsepr_oracle as O
+        self.O, self.np, self.w = O, np, w
+        b, h = divmod(head, w.H)
+        Q, K, V = gen.make_qkv(w, heads=[(b, h)])
+        self.q, self.k, self.v = (gen.as_f64(x)[b, h] for x in (Q, K, V))
         t0 = time.perf_counter()
-        O.call_head(q, k, v, w, h)
-        times.append(time.perf_counter() - t0)
-        h += 1
-    per_call_s = statistics.mean(times) * w.B * w.H
-    return {"value": w.dense_flops() / per_call_s / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
-            "sample": f"{len(times)} of {w.B * w.H} heads of one call (fp64 NumPy oracle, whole per-head "
-                      f"call), mean {statistics.mean(times):.2f} s/head extrapolated x{w.B * w.H}",
-            "s_per_call": per_call_s}
+        self.r = O.call_head(self.q, self.k, self.v, w, head, compute_outputs=False)
+        self.t_part = time.perf_counter() - t0
+        self.slices = max(1, min(8, w.n_qgroups))
+        self.t_sparse, self.t_rest = [], []
+
+    def step(self, i, record=True):
+        O, np, r = self.O, self.np, self.r
+        sel = (np.arange(self.w.n_qgroups) % self.slices) == (i % self.slices)
+        route = r["route"] & sel[:, None]
+        t0 = time.perf_counter()
+        osp = O.sparse_attention(self.q, self.k, self.v, r["qlabels"], r["klabels"], route)
+        t1 = time.perf_counter()
+        p, wts = r["probes"], r["weights"]
+        od = O.attention(self.q[p], self.k, self.v)
+        if len(p):
+            A, _ = O.ridge_fit(osp[p], od, wts, self.w.lam)
+            A = O.restrict_to_residual_span(A, od - osp[p], wts)
+        else:
+            A = np.zeros((self.w.d + 1, self.w.d))
+        out = O.apply_correction(osp, A)
+        out[p] = od
+        t2 = time.perf_counter()
+        if record:
+            self.t_sparse.append(t1 - t0)
+            self.t_rest.append(t2 - t1)
+        return t2 - t0
+
+    def s_per_call(self):
+        per_head = self.t_part + self.slices * statistics.mean(self.t_sparse) + statistics.mean(self.t_rest)
+        return self.w.B * self.w.H * per_head
+
+    def describe(self):
+        return (f"head 0 of {self.w.B * self.w.H}: its partition once ({self.t_part:.1f} s), then per step the "
+                f"block-sparse attention of 1/{self.slices} of its query groups (a different slice each step) "
+                f"plus its probe rows, ridge fit and correction; call time extrapolated as "
+                f"{self.w.B * self.w.H} x (partition + {self.slices} x slice + rest)")
+
+
+def oracle_baseline(w):
+    """cpu_baseline: the oracle's partition of one head plus one output step (about 10-30 s of
+    CPU work at the large shapes), extrapolated to the call."""
+    s = OracleSample(w)
+    s.step(0)
+    per_call = s.s_per_call()
+    return {"value": w.dense_flops() / per_call / 1e12, "unit": "TFLOPS", "cores": _oracle_cores(), "kind": "oracle",
+            "sample": s.describe() + " (one step)", "s_per_call_extrapolated": per_call}
 
 
 def run_reference(args, w, world, rank):
     if rank != 0:
         return
-    for _ in range(args.warmup):
-        oracle_sample(w, 0.0, max_heads=1)
+    t_start = time.perf_counter()
+    s = OracleSample(w)
+    for i in range(args.warmup):
+        s.step(i, record=False)
     t0 = time.perf_counter()
-    runs = [oracle_sample(w, 0.0, max_heads=1) for _ in range(args.steps)]
-    wall = time.perf_counter() - t0
-    s_per_call = statistics.mean(r["s_per_call"] for r in runs)
-    val = w.dense_flops() / s_per_call / 1e12
+    steps = [s.step(args.warmup + i) for i in range(args.steps)]
+    timed = time.perf_counter() - t0
+    per_call = s.s_per_call()
+    val = w.dense_flops() / per_call / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": s_per_call * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(steps) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w, {"l2": "n/a (CPU)"}),
-            "cpu_baseline": {"kind": "oracle", "cores": runs[0]["cores"], "value": val, "unit": "TFLOPS",
-                             "sample": "each step: head 0 of the call through the fp64 NumPy oracle, "
-                                       f"extrapolated x{w.B * w.H} heads"},
+            "oracle_s_per_call_extrapolated": per_call,
+            "oracle_partition_s_per_head": s.t_part,
+            "cpu_baseline": {"kind": "oracle", "cores": _oracle_cores(), "value": val, "unit": "TFLOPS",
+                             "sample": s.describe()},
             "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-            "wall_s": wall}
+            "timed_s": timed, "wall_s": time.perf_counter() - t_start}
     print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------------------------ GPU arm
+def _rank_inputs(w, world, rank, shard):
+    """(local workload, Q, K, V on the CPU, bh0, bh1).  Replicas: every rank draws the whole call
+    from its own generator variant.  Head shards: the rank draws only its heads of the one call
+    (variant 0) and runs them as a call of B = 1 with the seed of its first head."""
+    from free_block_sparse_02_b200 import shard as SH
+    if not shard or world == 1:
+        Q, K, V = gen.make_qkv(w, variant=rank if not shard else 0)
+        return w, Q, K, V, 0, w.B * w.H
+    wl, bh0, bh1 = SH.shard_workload(w, world, rank)
+    if wl is None:
+        raise SystemExit(f"--shard heads: rank {rank} of {world} has no head of the {w.B * w.H}-head call")
+    Q, K, V = gen.make_qkv(w, variant=0, heads=[divmod(bh, w.H) for bh in range(bh0, bh1)])
+    return wl, *(SH.local_slice(x, bh0, bh1).contiguous() for x in (Q, K, V)), bh0, bh1
+
+
 def run_ours(args, w, world, rank, local):
     from free_block_sparse_02_b200 import _lib as S
     import torch.distributed as dist
@@ -282,15 +392,24 @@ def run_ours(args, w, world, rank, local):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     S.load()
-    Qc, Kc, Vc = gen.make_qkv(w, variant=rank)
+    shard = args.shard == "heads" and world > 1
+    wl, Qc, Kc, Vc, bh0, bh1 = _rank_inputs(w, world, rank, args.shard == "heads")
     Q, K, V = Qc.to(dev), Kc.to(dev), Vc.to(dev)
-    op = S.SparsePR(w, device=dev)
+    op = S.SparsePR(wl, device=dev)
     O = torch.empty(Q.shape, dtype=Q.dtype, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    gather = None
+    if shard and args.gather:
+        per = -(-w.B * w.H // world)
+        gather = (torch.zeros((per, w.N, w.d), dtype=Q.dtype, device=dev),
+                  torch.empty((world * per, w.N, w.d), dtype=Q.dtype, device=dev))
 
     def step():
         op(Q, K, V, O=O)
+        if gather is not None:
+            gather[0][:bh1 - bh0].copy_(O.reshape(bh1 - bh0, w.N, w.d))
+            dist.all_gather_into_tensor(gather[1], gather[0])
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -301,7 +420,7 @@ def run_ours(args, w, world, rank, local):
     realised = statistics.mean(s["density"] for s in st)
     part_stats = {"k_iters": [s["k_iters"] for s in st], "q_iters": [s["q_iters"] for s in st],
                   "k_refined": sum(s["k_refined"] for s in st), "q_refined": sum(s["q_refined"] for s in st),
-                  "span_rank": [s["span_rank"] for s in st]}
+                  "span_rank": [s["span_rank"] for s in st], "fit_retries": sum(s["fit_retries"] for s in st)}
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -336,17 +455,24 @@ def run_ours(args, w, world, rank, local):
     kern_ms = [a.elapsed_time(b) for a, b in kev]
     # the k-means hooks bracket the tensor-core path only: bf16 inputs with at most 256 (padded)
     # key groups; above that the key k-means runs on the CUDA cores and the events stay unset
-    tc_km = w.dtype == configs.BF16 and (w.n_kgroups + 15) // 16 * 16 <= 256
+    tc_km = wl.dtype == configs.BF16 and (wl.n_kgroups + 15) // 16 * 16 <= 256
     asg_ms = statistics.mean(a.elapsed_time(b) for a, b in km_ev[1]) if tc_km else 0.0
     upd_ms = statistics.mean(a.elapsed_time(b) for a, b in km_ev[2]) if tc_km else 0.0
     ms = statistics.mean(step_ms)
     kms = statistics.mean(kern_ms)
     ms_max, kms_max, asg_ms, upd_ms = max_over_ranks([ms, kms, asg_ms, upd_ms], world, dev)
+    # attention roofline per rank: this rank's launch, the slowest rank's time
+    kflops = attention_flops(wl, pairs)
+    kflops_min, = [-x for x in max_over_ranks([-kflops], world, dev)]
+    # executed pairs of the whole job (block-sparse and probe rows, all ranks)
+    executed, = sum_over_ranks([kflops], world, dev)
 
     # end to end through the public API with host buffers (pinned), copies inside the region
     Qh, Kh, Vh = Qc.pin_memory(), Kc.pin_memory(), Vc.pin_memory()
     Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
     for i in range(args.steps + 1):
         flush.zero_()
         if i > 0:
@@ -364,47 +490,74 @@ def run_ours(args, w, world, rank, local):
 
     if rank == 0:
         pk = peaks()
-        flops = w.dense_flops()
-        value = whole_job_tflops(world, flops, ms_max)
-        kflops = 4.0 * w.d * pairs
+        # whole-job throughput: replicas run `world` calls per step, head shards one call
+        job_flops = w.dense_flops() * (1 if shard else world)
+        value = job_flops / (ms_max * 1e-3) / 1e12
         achieved = kflops / (kms_max * 1e-3) / 1e12
         peak = pk["bf16_tflops"]
         elt = Q.element_size()
+        if shard:
+            par = f"one call split by heads over {world} GPUs ({wl.H} or so heads each, no data-path collective" + \
+                  (", NCCL all-gather of O inside the timed region)" if gather is not None else ")")
+        else:
+            par = f"{world} independent calls, one per GPU"
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+            "scaling": "strong" if shard else "weak",
             "vs_baseline": None, "dtype": "bf16" if w.dtype == configs.BF16 else "f32", "data": "synthetic",
             "config": workload_config(w, {"l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
-                                          "realised_density": realised,
-                                          "parallelism": f"{world} independent calls, one per GPU"}),
+                                          "realised_density": realised, "parallelism": par}),
             "ms_per_call": ms_max,
-            "executed_tflops": world * (kflops + 4.0 * w.d * w.B * w.H * w.P * w.N) / (ms_max * 1e-3) / 1e12,
+            "executed_tflops": executed / (ms_max * 1e-3) / 1e12,
             "kernel_ms": {"block_sparse_attention": kms_max},
-            "roofline": {"bound": "tensor", "kernel": "block-sparse attention (the kernel the metric's % of "
-                                                         "bf16 peak refers to)",
+            "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel: block-sparse attention and the dense probe "
+                                                        "rows (the kernel the metric's % of bf16 peak refers to)",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                         "traffic": profiled_traffic(w),
-                         "peak_source": f"{pk['source']} bf16 dense (burst)",
-                         "algorithmic": f"4*d*executed pairs = {kflops:.4g} flop per launch"},
-            "roofline_kmeans": km_rooflines(w, asg_ms, upd_ms, pk) if tc_km else None,
-            "e2e": {"value": whole_job_tflops(world, flops, e2e_ms), "unit": "TFLOPS",
+                         "traffic": profiled_traffic(wl),
+                         "peak_source": f"{pk['source']} bf16 dense (burst), MEASURED_PEAKS.json",
+                         "algorithmic": f"4*d*(executed sparse pairs + P*N*heads) = {kflops:.4g} flop per launch "
+                                        f"(rank 0; smallest over ranks {kflops_min:.4g})"},
+            "roofline_kmeans": km_rooflines(wl, asg_ms, upd_ms, pk) if tc_km else None,
+            "e2e": {"value": job_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
                     "h2d_bytes_per_step": 3 * Q.numel() * elt, "d2h_bytes_per_step": O.numel() * O.element_size(),
                     "ms_per_step": e2e_ms},
             "gpu_launches": launches,
             "partition": part_stats,
             "clocks": clk,
         }
-        try:
-            line["quality"] = output_quality(S, w, Q, K, V, O, op.query(S.Q_PROBES), dev)
-        except Exception as exc:  # reported, never fatal: the timing above stands on its own
-            line["quality"] = {"error": str(exc)[:200]}
+        if not args.no_quality:
+            try:
+                q = output_quality(S, wl, Q, K, V, O, op.query(S.Q_PROBES), dev)
+                if wl.recipe == "tiles":
+                    q["note"] = QUALITY_NOTE_TILES
+                line["quality"] = q
+            except Exception as exc:  # reported, never fatal: the timing above stands on its own
+                line["quality"] = {"error": str(exc)[:200]}
+            if world == 1 and wl.recipe == "tiles":
+                try:
+                    line["quality_field"] = field_quality(S, wl, dev)
+                except Exception as exc:
+                    line["quality_field"] = {"error": str(exc)[:200]}
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = oracle_sample(w, args.cpu_budget)
-            line["cpu_baseline"].pop("s_per_call", None)
+            line["cpu_baseline"] = oracle_baseline(w)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def field_quality(S, w, dev, heads=2):
+    """The same operator and error metric on smooth-field inputs of the workload's shape
+    (`heads` heads): inputs whose block-sparse residual an affine map of the sparse output can
+    predict, as the paper's model activations are."""
+    wf = configs.scaled_down(w, heads=min(heads, w.H)).replace(recipe="field")
+    Q, K, V = (x.to(dev) for x in gen.make_qkv(wf))
+    op = S.SparsePR(wf, device=dev)
+    O = op(Q, K, V)
+    q = output_quality(S, wf, Q, K, V, O, op.query(S.Q_PROBES), dev)
+    q["inputs"] = f"smooth random field on the workload's grid, {wf.H} heads"
+    return q
 
 
 def main():
@@ -413,9 +566,12 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", type=int, default=1, help="index into configs.WORKLOADS")
-    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--workload", type=int, default=2, help="index into configs.WORKLOADS")
+    ap.add_argument("--shard", default="none", choices=["none", "heads"],
+                    help="multi-GPU: independent calls per rank (none) or one call split by heads")
+    ap.add_argument("--gather", action="store_true", help="--shard heads: all-gather O inside the timed region")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-quality", action="store_true", help="skip the output-error report (after the timing)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload on this many heads instead (a smaller case for profilers)")
     ap.add_argument("--density", type=float, default=0.0, help="override the density target (sweeps)")

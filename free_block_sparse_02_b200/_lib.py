@@ -76,6 +76,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sparsepr_version": (i32, []),
         "sparsepr_set_kernel_events": (i32, [vp, i32, vp, vp]),
         "sparsepr_launch_count": (ctypes.c_int64, []),
+        "sparsepr_set_wait_limit": (i32, [vp, i32, ctypes.c_int64]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -196,6 +197,11 @@ class SparsePR:
         h0 = ctypes.c_void_p(start.cuda_event) if start is not None else None
         h1 = ctypes.c_void_p(stop.cuda_event) if stop is not None else None
         _check(self.lib.sparsepr_set_kernel_events(self.handle, int(kernel), h0, h1), "sparsepr_set_kernel_events")
+
+    def set_wait_limit(self, cycles: int, kernel: int = 0):
+        """Test hook of the timeout path: the given kernel's bounded device-side waits give up
+        after `cycles` SM cycles (0 restores the default of about 1 s)."""
+        _check(self.lib.sparsepr_set_wait_limit(self.handle, int(kernel), int(cycles)), "sparsepr_set_wait_limit")
 
     def sync(self):
         _check(self.lib.sparsepr_sync(self.handle), "sparsepr_sync")

@@ -183,6 +183,12 @@ __global__ void __launch_bounds__(384, 1)
   __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // Every wait below gives up after the default limit, or after L.attn_wait_limit cycles when
+  // the test hook of the timeout path sets one; a wait that gives up sets s_abort.
+  const long long wlim = L.attn_wait_limit;
+  auto wt = [wlim](uint64_t* bar, uint32_t parity) -> bool {
+    return wlim > 0 ? mbar_wait_limit(bar, parity, &s_abort, wlim) : mbar_wait(bar, parity, &s_abort);
+  };
 
   // ---- work item
   if (tid == 0) {
@@ -283,7 +289,7 @@ __global__ void __launch_bounds__(384, 1)
       int nk = 0, nv = 0;  // K and V tiles issued
       auto load_k = [&](int i) -> bool {
         const int s = i % C::kKS;
-        if (!mbar_wait(k_empty + s, ((i / C::kKS) & 1) ^ 1, &s_abort)) return false;
+        if (!wt(k_empty + s, ((i / C::kKS) & 1) ^ 1)) return false;
         uint8_t* dst = sK + s * C::kKVTileBytes;
         mbar_arrive_expect_tx(k_full + s, C::kKVTileBytes);
 #pragma unroll
@@ -296,7 +302,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       auto load_v = [&](int i) -> bool {
         const int s = i % C::kVS;
-        if (!mbar_wait(v_empty + s, ((i / C::kVS) & 1) ^ 1, &s_abort)) return false;
+        if (!wt(v_empty + s, ((i / C::kVS) & 1) ^ 1)) return false;
 #pragma unroll
         for (int b = 0; b < kSubPerTile; ++b) tvalid[s * kSubPerTile + b] = pvalid[b];
         uint8_t* dst = sV + s * C::kKVTileBytes;
@@ -345,7 +351,7 @@ __global__ void __launch_bounds__(384, 1)
         mma_commit(s_full + t);
       };
       auto issue_pv = [&](int t, int j) -> bool {  // O_t += P_t(j) V_j
-        if (!mbar_wait(p_full + t, j & 1, &s_abort)) return false;
+        if (!wt(p_full + t, j & 1)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(sV + (j % C::kVS) * C::kKVTileBytes);
 #pragma unroll
@@ -357,7 +363,7 @@ __global__ void __launch_bounds__(384, 1)
         mma_commit(o_bar + t);
         return true;
       };
-      bool ok = mbar_wait(q_full, 0, &s_abort) && mbar_wait(k_full, 0, &s_abort);
+      bool ok = wt(q_full, 0) && wt(k_full, 0);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -366,10 +372,10 @@ __global__ void __launch_bounds__(384, 1)
       }
       for (int j = 0; ok && j < ntiles; ++j) {
         const bool more = j + 1 < ntiles;
-        if (!mbar_wait(v_full + j % C::kVS, (j / C::kVS) & 1, &s_abort)) break;
+        if (!wt(v_full + j % C::kVS, (j / C::kVS) & 1)) break;
         if (!issue_pv(0, j)) break;
         if (more) {
-          if (!mbar_wait(k_full + (j + 1) % C::kKS, ((j + 1) / C::kKS) & 1, &s_abort)) break;
+          if (!wt(k_full + (j + 1) % C::kKS, ((j + 1) / C::kKS) & 1)) break;
           tc_fence_after();
           issue_s(0, j + 1);
         }
@@ -398,8 +404,8 @@ __global__ void __launch_bounds__(384, 1)
     for (int j = 0; ok && j < ntiles; ++j) {
       // warp-uniform: the tcgen05.ld below needs every lane of the warp.  The V copy of tile j
       // is waited on too: it orders the producer's tile-validity words before their read.
-      const bool okw = mbar_wait(s_full + t, j & 1, &s_abort) &&
-                       mbar_wait(v_full + j % C::kVS, (j / C::kVS) & 1, &s_abort);
+      const bool okw = wt(s_full + t, j & 1) &&
+                       wt(v_full + j % C::kVS, (j / C::kVS) & 1);
       if (!__all_sync(0xffffffffu, okw)) {
         ok = false;
         break;
@@ -449,7 +455,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (__any_sync(0xffffffffu, need && j > 0)) {
         // O_t holds P_t(0..j-1) V (complete: S_t(j) was issued after the last of them)
-        const bool okw2 = mbar_wait(o_bar + t, (j - 1) & 1, &s_abort);
+        const bool okw2 = wt(o_bar + t, (j - 1) & 1);
         if (!__all_sync(0xffffffffu, okw2)) {
           ok = false;
           break;
@@ -506,7 +512,9 @@ __global__ void __launch_bounds__(384, 1)
                               : L.Osp + ((size_t)bh * L.N + qrow0 + t * kTcTileM) * D);
       if (ntiles == 0 && row < rows_t)
         for (int c = 0; c < D; c += 4) *(float4*)(out + (size_t)row * D + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (ok && mbar_wait(o_bar + t, (ntiles - 1) & 1, &s_abort)) {
+      // warp-uniform: the tcgen05.ld below needs every lane of the warp
+      const bool oke = ok && wt(o_bar + t, (ntiles - 1) & 1);
+      if (__all_sync(0xffffffffu, oke)) {
         tc_fence_after();
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
@@ -525,9 +533,10 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
   }
-  if (s_abort && tid == 0) atomicCAS(L.status, kDevOk, kDevTimeout);
   tc_fence_before();
   __syncthreads();
+  // after the barrier every wait of the CTA has ended, so a late give-up is not missed
+  if (s_abort && tid == 0) atomicCAS(L.status, kDevOk, kDevTimeout);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

@@ -39,6 +39,8 @@ struct Layout {
   int repair;           // 1: fit and add the probe-residual correction
   int correction;       // SPARSEPR_CORRECTION_AFFINE / _MEAN
   int trunc_rank;       // 0: whole residual span; r: its r leading eigenvectors
+  long long attn_wait_limit;  // > 0: the attention kernel's bounded waits give up after this
+                              // many cycles (test hook of the timeout path); 0: the default
 
   // status + per-head statistics
   int* status;                    // [1]

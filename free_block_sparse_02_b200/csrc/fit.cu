@@ -452,7 +452,7 @@ __global__ void __launch_bounds__(256) ridge_solve_kernel(Layout L) {
   if (!ok) {
     if (tid == 0) {
       atomicCAS(L.status, kDevOk, kDevNumeric);
-      st.fit_retries = retries;  // A is zero; its projection stays zero
+      st.fit_retries = retries - 1;  // the three jitter retries all failed; A is zero
     }
     for (int e = tid; e < n1 * d; e += blockDim.x) {
       A[e] = 0.0;

@@ -16,6 +16,8 @@
 
 #include <mutex>
 
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -37,22 +39,58 @@ static __device__ __align__(256) double g_ridge_scratch[kStaticDoubles];
 
 constexpr int kMaxDevices = 64;
 static std::mutex g_scratch_mu;
-static double* g_scratch_addr[kMaxDevices] = {};
+struct ScratchAddr {
+  unsigned long long ctx_id;  // the context the address belongs to (0 = not looked up yet)
+  double* addr;
+};
+static ScratchAddr g_scratch_addr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device.  The array's name is only a
-// host-side stand-in in host code, so the address is looked up once per device with
-// cudaGetSymbolAddress (with that device current) and cached.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (cuCtxGetId: never reused within a
+// process), or 0 when there is none or the driver does not provide it.
+static unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = (CtxGetCurrentFn)p;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = (CtxGetIdFn)p;
+    looked_up = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device.  In host code the array's name is
+// only a host-side stand-in, so the address is looked up with cudaGetSymbolAddress, with the
+// device current, the first time a device is used, and cached together with the id of the
+// context it was taken in.  A later call under another context of that device (after a
+// cudaDeviceReset the module is loaded again, possibly at another address) looks it up again.
 static sparsepr_status scratch_address(double** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SPARSEPR_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return SPARSEPR_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  ScratchAddr& e = g_scratch_addr[dev];
+  const unsigned long long id = current_context_id();
+  if (!e.addr || id == 0 || id != e.ctx_id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_ridge_scratch) != cudaSuccess || p == nullptr) return SPARSEPR_ERR_CUDA;
-    g_scratch_addr[dev] = (double*)p;
+    e.addr = (double*)p;
+    e.ctx_id = current_context_id();  // the lookup itself makes the primary context current
   }
-  *out = g_scratch_addr[dev];
+  *out = e.addr;
   return SPARSEPR_OK;
 }
 
@@ -133,7 +171,8 @@ extern "C" sparsepr_status sparsepr_ridge_fit_static(const float* osp_probe, con
                                                      void* stream) {
   if (!A || (P > 0 && (!osp_probe || !odense_probe || !probe_w)) || !isfinite(lambda))
     return SPARSEPR_ERR_INVALID_ARG;
-  if (n_heads < 1 || P < 0 || (d != 64 && d != 128)) return SPARSEPR_ERR_INVALID_ARG;
+  if (n_heads < 1 || P < 0) return SPARSEPR_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SPARSEPR_ERR_UNSUPPORTED;
   if (n_heads > kStaticMaxHeads || d > kStaticMaxDim || P > kStaticMaxProbes) return SPARSEPR_ERR_WORKSPACE;
   double* base = nullptr;
   sparsepr_status s = scratch_address(&base);

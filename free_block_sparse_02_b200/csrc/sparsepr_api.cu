@@ -385,4 +385,11 @@ sparsepr_status sparsepr_set_kernel_events(sparsepr_plan_t* p, int32_t kernel, v
 
 int64_t sparsepr_launch_count(void) { return (int64_t)g_launches.load(); }
 
+sparsepr_status sparsepr_set_wait_limit(sparsepr_plan_t* p, int32_t kernel, int64_t cycles) {
+  if (!p || cycles < 0) return SPARSEPR_ERR_INVALID_ARG;
+  if (kernel != SPARSEPR_KERNEL_BLOCK_SPARSE) return SPARSEPR_ERR_UNSUPPORTED;
+  p->L.attn_wait_limit = (long long)cycles;
+  return SPARSEPR_OK;
+}
+
 }  // extern "C"

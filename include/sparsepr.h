@@ -107,7 +107,10 @@ typedef struct sparsepr_head_stats {
   int32_t q_iters;          /* ... for the query groups                                         */
   int32_t k_refined;        /* key labels decided by the float64 tie-break at the last pass     */
   int32_t q_refined;        /* query labels decided by the float64 tie-break at the last pass   */
-  int32_t fit_retries;      /* ridge jitter retries (lambda x10 each); 0 normally               */
+  int32_t fit_retries;      /* ridge jitter retries, 0..3; 0 normally.  A failed attempt retries
+                               with lambda x10 (lambda = 0: 1e-12 tr(G)/(d+1) first); when the
+                               third retry fails too the head's A is zero and the status word
+                               is SPARSEPR_ERR_NUMERIC                                           */
   int32_t span_rank;        /* rank of the probe-residual span                                  */
   int64_t sparse_pairs;     /* executed (query, key) pairs of the block-sparse pass             */
   double density;           /* realised density: (s*N + C_k*N + P*N + sparse_pairs) / N^2      */
@@ -207,14 +210,28 @@ sparsepr_status sparsepr_set_kernel_events(sparsepr_plan_t* plan, int32_t kernel
 /* Number of CUDA kernels this library has launched since it was loaded (all plans). */
 int64_t sparsepr_launch_count(void);
 
+/* Test hook of the timeout path (no counterpart in the paper).  Every device-side wait of the
+ * library is bounded: by default it gives up after about 2e9 SM cycles (about 1 s), sets the
+ * device status word to SPARSEPR_ERR_TIMEOUT, lets the copies and tensor-core operations it
+ * started finish, frees its tensor memory and returns, so the context stays usable.  This call
+ * sets, for the plan's later launches of `kernel`, a limit of `cycles` SM cycles on each such
+ * wait (0 restores the default).  Only SPARSEPR_KERNEL_BLOCK_SPARSE is accepted (other ids:
+ * SPARSEPR_ERR_UNSUPPORTED; cycles < 0: SPARSEPR_ERR_INVALID_ARG).  With a limit of a few
+ * hundred cycles the attention launch gives up, its output rows are left unwritten, and the
+ * next sparsepr_sync returns SPARSEPR_ERR_TIMEOUT (and clears it); the plan, its workspace and
+ * the context stay usable for the next call.  Enqueues nothing. */
+sparsepr_status sparsepr_set_wait_limit(sparsepr_plan_t* plan, int32_t kernel, int64_t cycles);
+
 /* Allocation-free weighted ridge fit (no counterpart in the paper: an interface for callers
  * that cannot allocate device memory).  Some callers cannot call cudaMalloc or hand this
  * library scratch memory at the point where they fit the correction -- e.g. code running under
  * a fixed memory pool that must not grow during a step, or a host runtime that only passes the
- * tensors it already owns.  This entry point computes, for each of n_heads heads, the same
- * fitted map A as sparsepr_fit_apply (weighted ridge of O_dense - O_sp on [O_sp, 1], lambda as
- * in sparsepr_config, restricted to the span of the probe residuals) from probe rows the
- * caller passes in, and allocates nothing.
+ * tensors it already owns.  This entry point fits, for each of n_heads heads, the affine map A
+ * that sparsepr_fit_apply fits with the default settings (correction SPARSEPR_CORRECTION_AFFINE,
+ * trunc_rank 0): the weighted ridge of O_dense - O_sp on [O_sp, 1], lambda as in
+ * sparsepr_config, restricted to the whole span of the probe residuals.  It has no mean-only
+ * family and no output truncation; for plans that use either, its A differs from theirs.  The
+ * probe rows come from the caller and nothing is allocated.
  *   osp_probe    float  [n_heads, P, d]   device: block-sparse output of the probe rows
  *   odense_probe float  [n_heads, P, d]   device: exact output of the probe rows
  *   probe_w      double [n_heads, P]      device: probe weights
@@ -223,12 +240,13 @@ int64_t sparsepr_launch_count(void);
  *                system stayed indefinite after the jitter retries (that head's A is zero)
  * Scratch: one fixed __device__ array inside the library (about 7.4 MB) that every GPU which
  * loads the library reserves until the process exits.  Limits: 1 <= n_heads <= 16,
- * d in {64, 128}, 0 <= P <= 4096; larger sizes return SPARSEPR_ERR_WORKSPACE and launch
- * nothing.  The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current, so make that first call before any stream
- * capture.  All calls share the one array and it keeps the last call's contents: calls that
- * overlap on the GPU (e.g. on two streams at once) race and give wrong results; serialise
- * them.  Enqueued on `stream` (cudaStream_t as void*); returns without waiting. */
+ * 0 <= P <= 4096 (larger sizes return SPARSEPR_ERR_WORKSPACE and launch nothing); d must be 64
+ * or 128 (else SPARSEPR_ERR_UNSUPPORTED).  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current and keeps it for that device's
+ * context, so make that first call before any stream capture.  All calls share the one array
+ * and it keeps the last call's contents: calls that overlap on the GPU (e.g. on two streams at
+ * once) race and give wrong results; serialise them.  Enqueued on `stream` (cudaStream_t as
+ * void*); returns without waiting. */
 sparsepr_status sparsepr_ridge_fit_static(const float* osp_probe, const float* odense_probe,
                                           const double* probe_w, int32_t n_heads, int32_t P,
                                           int32_t d, double lambda, double* A, int32_t* status_out,

@@ -50,3 +50,32 @@ def test_whole_job_throughput_counts_every_rank():
     one = bench.whole_job_tflops(1, flops, 3.2)
     assert one == pytest.approx(flops / 3.2e-3 / 1e12)
     assert bench.whole_job_tflops(4, flops, 3.2) == pytest.approx(4 * one)
+
+
+def test_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    a = "// header\nint f(int x) {  /* twice */\n  return 2 * x;  // doubled\n}\n"
+    b = "int f(int x) {\n\n  return 2 * x;\n}\n/* a new note\n spanning lines */\n"
+    c = "int f(int x) {\n  return 3 * x;\n}\n"
+    for name, text in (("a.cu", a), ("b.cu", b), ("c.cu", c)):
+        (tmp_path / name).write_text(text)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.source_hash("a.cu") == bench.source_hash("b.cu")
+    assert bench.source_hash("a.cu") != bench.source_hash("c.cu")
+
+
+def test_attention_flops_count_the_probe_rows():
+    w = configs.workload(2)
+    pairs = 69_700_000_000
+    assert bench.attention_flops(w, pairs) == pytest.approx(4 * 128 * (pairs + 24 * 512 * 118800))
+    assert bench.attention_flops(w.replace(P=0), pairs) == pytest.approx(4 * 128 * pairs)
+
+
+def test_oracle_sample_extrapolates_from_measured_parts():
+    w = configs.workload(0)
+    s = bench.OracleSample(w)
+    for i in range(3):
+        assert s.step(i) > 0
+    assert s.t_part > 0 and len(s.t_sparse) == 3
+    assert s.s_per_call() == pytest.approx(
+        w.B * w.H * (s.t_part + s.slices * sum(s.t_sparse) / 3 + sum(s.t_rest) / 3))
+    assert "extrapolated" in s.describe()

@@ -507,3 +507,86 @@ def test_semantic_partition_is_kmeans_on_the_raw_inputs():
     ids = O.kmeans_init_ids(80, 3, O.stream_seed(9, 2, 1))
     kq = KMeans(n_clusters=3, init=q[ids], n_init=1, max_iter=50, tol=0.0, algorithm="lloyd").fit(q)
     assert np.array_equal(r["qlabels"], kq.labels_)
+
+
+# ---------------------------------------------------------------- warm start (streaming calls)
+class _WarmCfg:
+    s, n_kgroups, n_qgroups, density, fixed_k, P, probe_mode = 16, 6, 5, 0.5, 0, 6, 1
+    lam, km_tol, seed = -1.0, -1.0, 31
+
+    def __init__(self, km_iters, km_iters_warm):
+        self.km_iters, self.km_iters_warm = km_iters, km_iters_warm
+
+
+def _rms_rows(C):
+    return np.sqrt(np.mean(C * C, axis=1))
+
+
+def test_warm_start_restarts_lloyd_where_the_previous_call_stopped():
+    """On the same inputs, a call of a Lloyd iterations followed by a warm-started call of b
+    iterations must end where one cold call of a + b iterations ends: the state of Lloyd's method
+    is its centroids, and the warm start hands them over (keys in key space, re-projected through
+    the sampled queries; queries in the previous call's response coordinates, unchanged).  The
+    key groups have converged by iteration a, so both calls see the same response coordinates;
+    the query groups have not, so the pin has teeth: a warm start that re-normalised the carried
+    query centroids, or restarted from the seeded points, would end elsewhere."""
+    q, k, v = _small_inputs(39)
+    a, b = 4, 4
+    ra = O.call_head(q, k, v, _WarmCfg(a, 0), 2, compute_outputs=False)
+    rab = O.call_head(q, k, v, _WarmCfg(a + b, 0), 2, compute_outputs=False)
+    # preconditions: keys converged by a; queries still moving between a and a + b; the carried
+    # query centroids are not unit-RMS rows (re-normalising them would move them)
+    assert np.array_equal(ra["klabels"], rab["klabels"])
+    assert not np.array_equal(ra["qlabels"], rab["qlabels"])
+    assert np.abs(_rms_rows(ra["qcent"]) - 1.0).max() > 1e-2
+    rw = O.call_head(q, k, v, _WarmCfg(a, b), 2, warm=O.warm_state(ra), compute_outputs=False)
+    assert rw["kmeans_k"].n_iter == b and rw["kmeans_q"].n_iter == b
+    assert np.array_equal(rw["klabels"], rab["klabels"])
+    assert np.array_equal(rw["qlabels"], rab["qlabels"])
+    np.testing.assert_allclose(rw["kmeans_q"].objective, rab["kmeans_q"].objective[a:], rtol=1e-12)
+    np.testing.assert_allclose(rw["qcent"], rab["qcent"], rtol=1e-12, atol=1e-12)
+    # the same restart from re-normalised query centroids does not reproduce it
+    bad = O.WarmState(key_centroids=ra["kcent"], query_centroids=O.rms_normalize(ra["qcent"]))
+    rb = O.call_head(q, k, v, _WarmCfg(a, b), 2, warm=bad, compute_outputs=False)
+    assert not np.allclose(rb["kmeans_q"].objective, rab["kmeans_q"].objective[a:], rtol=1e-9)
+
+
+def test_warm_start_key_step_uses_the_current_calls_metric():
+    """Call 2 sees new queries and keys.  With one warm iteration its key labels are the first
+    assignment from the previous call's key-space centroids c_j, in call 2's response space:
+    argmin_j (k_t - c_j)^T M2 (k_t - c_j) with M2 = Qs2^T Qs2 / d, evaluated here in key space (the
+    metric identity, not the oracle's response-space projection).  The previous call's metric M1
+    would give other labels on these inputs."""
+    rng = np.random.default_rng(22)
+    N, d = 120, 8
+    q1, k1, v1 = rng.standard_normal((N, d)), rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    stretch = np.array([4.0, 0.25, 3.0, 0.5, 1.0, 2.0, 0.3, 1.5])
+    q2, k2, v2 = q1 * stretch + 0.3 * rng.standard_normal((N, d)), rng.standard_normal((N, d)), v1
+    cfg = _WarmCfg(6, 1)
+    r1 = O.call_head(q1, k1, v1, cfg, 0, compute_outputs=False)
+    r2 = O.call_head(q2, k2, v2, cfg, 0, warm=O.warm_state(r1), compute_outputs=False)
+    C = r1["kcent"]
+    rows = O.sample_query_rows(N, cfg.s)
+    M2 = q2[rows].T @ q2[rows] / d
+    M1 = q1[rows].T @ q1[rows] / d
+
+    def labels_under(M):
+        D = np.array([[(kt - c) @ M @ (kt - c) for c in C] for kt in k2])
+        return np.argmin(D, axis=1)
+
+    assert r2["kmeans_k"].n_iter == 1
+    assert np.array_equal(r2["klabels"], labels_under(M2))
+    assert not np.array_equal(labels_under(M1), labels_under(M2))
+
+
+def test_warm_start_from_converged_centroids_is_a_fixed_point():
+    """A call warm-started from the converged state of the same inputs keeps every label and the
+    objectives after one iteration."""
+    q, k, v = _small_inputs(23)
+    r = O.call_head(q, k, v, _WarmCfg(60, 0), 1, compute_outputs=False, keep_history=True)
+    hk, hq = r["kmeans_k"].label_history, r["kmeans_q"].label_history
+    assert np.array_equal(hk[-1], hk[-2]) and np.array_equal(hq[-1], hq[-2])  # converged
+    rw = O.call_head(q, k, v, _WarmCfg(60, 1), 1, warm=O.warm_state(r), compute_outputs=False)
+    assert np.array_equal(rw["klabels"], r["klabels"]) and np.array_equal(rw["qlabels"], r["qlabels"])
+    np.testing.assert_allclose(rw["kmeans_k"].objective[0], r["kmeans_k"].objective[-1], rtol=1e-12)
+    np.testing.assert_allclose(rw["kmeans_q"].objective[0], r["kmeans_q"].objective[-1], rtol=1e-12)
