@@ -36,6 +36,7 @@ from free_block_sparse_02_b200 import configs, gen  # noqa: E402
 
 METRIC = "SparsePR ms/call & dense-equiv TFLOPS at 22% density; % bf16 TC peak"
 L2_FLUSH_BYTES = 256 << 20
+KM_W_TERMS = 2  # bf16 terms of the group weights in the k-means assignment's products
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -128,6 +129,7 @@ def workload_config(w, extra=None):
          "n_kgroups": w.n_kgroups, "n_qgroups": w.n_qgroups, "P": w.P,
          "probes": ["uniform", "stratified", "random"][w.probe_mode], "km_iters": w.km_iters, "km_tol": w.km_tol,
          "lam": w.lam, "correction": "mean" if w.correction == 1 else "affine", "trunc_rank": w.trunc_rank,
+         "key_rank": w.key_rank,
          "generator": (f"clustered Gaussian tiles {w.tile} on grid {w.grid}" if w.recipe == "tiles" else
                        f"smooth random field, length scales {w.field_ell}, logit contrast {w.field_tau}, "
                        f"value offset {w.value_offset}, on grid {w.grid}") + (" + 3D RoPE" if w.rope else "")}
@@ -231,13 +233,13 @@ def km_rooflines(w, asg_ms, upd_ms, pk):
     """Rooflines of one key k-means assignment and one update launch (first iteration of the
     call).  Both read every key once (2 d bytes, bf16) and write (assignment) or read (update)
     its label (4 bytes).  The assignment also runs the tensor-core products of every key with
-    the three bf16 terms of the C_p (padded) group weights, 3 x 2 x C_p x d flops per key: at
-    the large shapes that, not HBM, is its bound, and it is reported against the bf16 peak with
-    the HBM fraction beside it.  The update is HBM-bound."""
+    the two bf16 terms (hi, mid) of the C_p (padded) group weights, 2 x 2 x C_p x d flops per
+    key: at the large shapes that, not HBM, is its bound, and it is reported against the bf16
+    peak with the HBM fraction beside it.  The update is HBM-bound."""
     units = w.B * w.H * w.N
     by = units * (2 * w.d + 4)
     cp = (w.n_kgroups + 15) // 16 * 16
-    fl = units * 3 * 2 * cp * w.d
+    fl = units * KM_W_TERMS * 2 * cp * w.d
     out = {}
     if asg_ms > 0:
         s = asg_ms * 1e-3
@@ -248,8 +250,8 @@ def km_rooflines(w, asg_ms, upd_ms, pk):
         main, other = (tc, hbm) if t_tc >= t_hbm else (hbm, tc)
         out["assignment"] = {"bound": "tensor" if t_tc >= t_hbm else "hbm", **main, "ms": asg_ms, "traffic": None,
                              "other": other,
-                             "algorithmic": f"{units} keys x (2d + 4) bytes = {by} bytes and x 6 C_p d = {fl} "
-                                            f"flops per launch"}
+                             "algorithmic": f"{units} keys x (2d + 4) bytes = {by} bytes and x {2 * KM_W_TERMS} C_p d = "
+                                            f"{fl} flops per launch"}
     if upd_ms > 0:
         a = by / (upd_ms * 1e-3) / 1e9
         out["update"] = {"bound": "hbm", "achieved": a, "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -582,6 +584,7 @@ def main():
                     help="override the correction family (Table 4 sweeps)")
     ap.add_argument("--lam", type=float, default=None, help="override the ridge lambda (>= 0 absolute)")
     ap.add_argument("--trunc-rank", type=int, default=0, help="restrict the map to the r leading residual directions")
+    ap.add_argument("--key-rank", type=int, default=0, help="key-response rank r_K (Table C.1; 0 = full)")
     ap.add_argument("--kgroups", type=int, default=0, help="override the key-group count C_k")
     ap.add_argument("--qgroups", type=int, default=0, help="override the query-group count C_q")
     ap.add_argument("--sampled", type=int, default=0, help="override the sampled-query count s")
@@ -607,6 +610,8 @@ def main():
         w = w.replace(lam=args.lam)
     if args.trunc_rank > 0:
         w = w.replace(trunc_rank=args.trunc_rank)
+    if args.key_rank > 0:
+        w = w.replace(key_rank=args.key_rank)
     if args.kgroups > 0:
         w = w.replace(n_kgroups=args.kgroups)
     if args.qgroups > 0:

@@ -39,7 +39,7 @@ class Config(ctypes.Structure):
                 ("P", ctypes.c_int32), ("probe_mode", ctypes.c_int32), ("lambda_", ctypes.c_double),
                 ("km_iters", ctypes.c_int32), ("km_iters_warm", ctypes.c_int32), ("km_tol", ctypes.c_float),
                 ("seed", ctypes.c_uint64), ("partition", ctypes.c_int32), ("repair", ctypes.c_int32),
-                ("correction", ctypes.c_int32), ("trunc_rank", ctypes.c_int32)]
+                ("correction", ctypes.c_int32), ("trunc_rank", ctypes.c_int32), ("key_rank", ctypes.c_int32)]
 
 
 class HeadStats(ctypes.Structure):
@@ -101,7 +101,8 @@ def config_from(w, **over) -> Config:
                   seed=g("seed"), partition=over.get("partition", getattr(w, "partition", 0)),
                   repair=over.get("repair", getattr(w, "repair", 1)),
                   correction=over.get("correction", getattr(w, "correction", 0)),
-                  trunc_rank=over.get("trunc_rank", getattr(w, "trunc_rank", 0)))
+                  trunc_rank=over.get("trunc_rank", getattr(w, "trunc_rank", 0)),
+                  key_rank=over.get("key_rank", getattr(w, "key_rank", 0)))
 
 
 def workspace_size(cfg: Config) -> int:

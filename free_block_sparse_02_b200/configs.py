@@ -61,6 +61,7 @@ class Workload:
     repair: int = 1                   # 1: fit and add the probe-residual correction; 0: none
     correction: int = 0               # CORRECTION_AFFINE (SparsePR) or CORRECTION_MEAN
     trunc_rank: int = 0               # 0: whole residual span; r: its r leading directions
+    key_rank: int = 0                 # 0: full key responses; r: their r leading directions (r_K)
     recipe: str = "tiles"             # input generator: "tiles" (clustered Gaussian) or "field"
     field_tau: float = 4.0            # "field": peak logit contrast of the smooth field
     field_ell: Tuple[float, float, float] = (2.0, 6.0, 6.0)  # "field": length scales (t, y, x)

@@ -9,7 +9,7 @@
 // Work item = 256 query rows of one query group (block-sparse pass) or of one head's probe rows
 // (dense pass), as two 128-row MMA tiles Q0, Q1 that share every KV tile.  The keys are the
 // concatenation of the kept key groups' rows in the group-permuted K/V, streamed in 128-key
-// tiles assembled from 32-row TMA boxes, so a kept key group costs at most 31 padded (masked)
+// tiles assembled from 64-row TMA boxes, so a kept key group costs at most 63 padded (masked)
 // rows wherever it starts.
 //
 // CTA of 384 threads: warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner), warps 4..7
@@ -35,9 +35,13 @@ using namespace sm100;
 
 constexpr int kTcTileM = 128;   // query rows per MMA tile
 constexpr int kTcTileN = 128;   // keys per KV tile (MMA N of S, K of PV)
-constexpr int kSubRows = 32;    // rows per TMA box of K/V (32: measured faster than 16 at d = 128)
+constexpr int kSubRows = 64;    // rows per TMA box of K/V (64: 1.5% faster than 32 at the 13B-DiT
+                                // shape, which was 3% faster than 16)
 constexpr int kSubPerTile = kTcTileN / kSubRows;
 constexpr int kTmemCols = 512;
+constexpr int kRegsCtl = 152;      // registers per thread of warps 0-3 (TMA, MMA, two idle warps)
+constexpr int kRegsSoftmax = 176;  // ... of the two softmax warpgroups
+static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= 384 * 168, "register split above the launch's registers");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kExpPolyEvery = 0;           // in tiles whose keys are all real, 1 in n exponential
                                            // pairs runs on the FMA pipe (0: none)
@@ -45,10 +49,9 @@ constexpr int kExpPolyEvery = 0;           // in tiles whose keys are all real, 
 // 2^x for a pair of x <= kRescaleThreshold on the FMA pipe (f32x2), for x >= -125 (smaller x
 // give 2^-125 instead of 0: far below the bf16 rounding of P and of any row sum, which is
 // >= 1).  Cody-Waite style reduction x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in
-// the low mantissa bits) and f in [-1/2, 1/2], then a quintic in f fitted to 2^f by least
-// squares on relative error at Chebyshev nodes with Lawson reweighting (max relative error
-// 2.3e-7 in fp32 Horner evaluation, about that of the special-function unit), and n added to
-// the exponent field.
+// the low mantissa bits) and f in [-1/2, 1/2], then a cubic in f fitted to 2^f by least squares
+// on relative error at Chebyshev nodes with Lawson reweighting (max relative error 7.5e-5 in fp32
+// Horner evaluation, 26 times below the bf16 rounding of P), and n added to the exponent field.
 __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
   float x0, x1;
   f2_unpack(x, x0, x1);
@@ -56,11 +59,9 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
   const uint64_t t = f2_add(xc, f2_pack(12582912.f, 12582912.f));
   const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));
   const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);
-  uint64_t p = f2_fma(f2_pack(0.001327647129f, 0.001327647129f), f, f2_pack(0.009675540961f, 0.009675540961f));
-  p = f2_fma(p, f, f2_pack(0.05550713092f, 0.05550713092f));
-  p = f2_fma(p, f, f2_pack(0.2402212024f, 0.2402212024f));
-  p = f2_fma(p, f, f2_pack(0.693146944f, 0.693146944f));
-  p = f2_fma(p, f, f2_pack(1.000000119f, 1.000000119f));
+  uint64_t p = f2_fma(f2_pack(0.05517166853f, 0.05517166853f), f, f2_pack(0.24261114001f, 0.24261114001f));
+  p = f2_fma(p, f, f2_pack(0.69326096773f, 0.69326096773f));
+  p = f2_fma(p, f, f2_pack(0.99992805719f, 0.99992805719f));
   float p0, p1, t0, t1;
   f2_unpack(p, p0, p1);
   f2_unpack(t, t0, t1);
@@ -68,10 +69,10 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
                  __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
 }
 
-// Exponentials of one half row of S (64 scores in sv, as fp32 bits) into 32 packed bf16 pairs,
-// adding them to the row sum.  kFull: every key of the tile is real (no -inf scores), so the
-// polynomial pairs may run; otherwise every exponential is on the special-function unit,
-// where 2^-inf = 0 exactly.
+// Exponentials of 64 scores of a row of S (fp32 bits) into 32 packed bf16 pairs, adding them to
+// the row sum.  kFull: every key of the tile is real (no -inf scores), so the polynomial pairs
+// may run; otherwise every exponential is on the special-function unit, where 2^-inf = 0
+// exactly.
 template <bool kFull>
 __device__ __forceinline__ void exp_half(const uint32_t (&sv)[64], float scale2, float neg_m, uint32_t (&pk)[32],
                                          uint64_t (&acc)[2]) {
@@ -269,6 +270,12 @@ __global__ void __launch_bounds__(384, 1)
   const int ntiles = s_ntiles, qrow0 = s_qrow0;
   const int row_base = bh * L.N;   // first row of this head in the 2D K/V view
   const int oob_row = L.BH * L.N;  // a box starting here is entirely zero-filled
+  // registers: the TMA / MMA warpgroup gives a share to the two softmax warpgroups, which hold a
+  // whole row of S in registers (128 x kRegsCtl + 256 x kRegsSoftmax = 384 x 168, the launch's)
+  if (warp < 4)
+    regs_release<kRegsCtl>();
+  else
+    regs_take<kRegsSoftmax>();
 
   if (warp == 0) {
     // ================================================================ TMA producer
@@ -418,20 +425,20 @@ __global__ void __launch_bounds__(384, 1)
         full = full && valid[b] == kSubRows;
       }
       tc_fence_after();
-      // pass 1: row max over the real keys (four loads, one wait; eight independent chains)
+      // the row's kTcTileN scores in registers: four loads, one wait
+      uint32_t sv[kTcTileN];
+#pragma unroll
+      for (int c = 0; c < kTcTileN / 32; ++c)
+        tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
+      tmem_wait_ld();
+      if (!full) {  // padded keys of partial boxes take no part: -inf, probability exactly 0
+#pragma unroll
+        for (int k = 0; k < kTcTileN; ++k)
+          if ((k & (kSubRows - 1)) >= valid[k / kSubRows]) sv[k] = __float_as_uint(-INFINITY);
+      }
+      // row max: eight chains over columns c + 8i, three inputs per maximum
       float tmax;
       {
-        uint32_t sv[kTcTileN];
-#pragma unroll
-        for (int c = 0; c < kTcTileN / 32; ++c)
-          tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
-        tmem_wait_ld();
-        if (!full) {  // padded keys of partial boxes take no part
-#pragma unroll
-          for (int k = 0; k < kTcTileN; ++k)
-            if ((k & (kSubRows - 1)) >= valid[k / kSubRows]) sv[k] = __float_as_uint(-INFINITY);
-        }
-        // eight chains over columns c + 8i, three inputs per maximum
         float mx[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -453,6 +460,22 @@ __global__ void __launch_bounds__(384, 1)
         m_new = tmax;
         factor = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_new);
       }
+      l *= factor;
+      m_used = m_new;
+      // P = 2^(s*scale - m) as packed bf16 over the first kTcTileN/2 columns of S_t (every score
+      // is already in registers, so the packed columns may overwrite them)
+      uint64_t acc[2] = {0ull, 0ull};
+#pragma unroll
+      for (int h = 0; h < kTcTileN / 64; ++h) {  // 64 scores -> 32 packed columns at a time
+        uint32_t pk[32];
+        if (full)
+          exp_half<true>(*reinterpret_cast<const uint32_t(*)[64]>(sv + h * 64), scale2, -m_used, pk, acc);
+        else
+          exp_half<false>(*reinterpret_cast<const uint32_t(*)[64]>(sv + h * 64), scale2, -m_used, pk, acc);
+        tmem_st32(tS + h * 32, pk);
+      }
+      // a moved maximum rescales O_t before PV_t(j) adds to it (the arrival below releases that
+      // MMA); here, after P, the row's scores no longer occupy registers
       if (__any_sync(0xffffffffu, need && j > 0)) {
         // O_t holds P_t(0..j-1) V (complete: S_t(j) was issued after the last of them)
         const bool okw2 = wt(o_bar + t, (j - 1) & 1);
@@ -470,33 +493,6 @@ __global__ void __launch_bounds__(384, 1)
           for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * factor);
           tmem_st32(tO + c * 32, r);
         }
-        tmem_wait_st();
-      }
-      l *= factor;
-      m_used = m_new;
-      // pass 2: P = 2^(s*scale - m) as packed bf16 over the first 64 columns of S_t, 64 keys at
-      // a time (each half is read before its 32 packed columns overwrite already-read ones).
-      // Padded keys are set to -inf first, so their probability is exactly 0.
-      const float neg_m = -m_used;
-      uint64_t acc[2] = {0ull, 0ull};
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t sv[64];
-        tmem_ld32(tS + h * 64, *reinterpret_cast<uint32_t(*)[32]>(sv));
-        tmem_ld32(tS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-        tmem_wait_ld();
-        uint32_t pk[32];
-        if (full) {
-          exp_half<true>(sv, scale2, neg_m, pk, acc);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 64; ++k) {
-            const int col = h * 64 + k;
-            if ((col & (kSubRows - 1)) >= valid[col / kSubRows]) sv[k] = __float_as_uint(-INFINITY);
-          }
-          exp_half<false>(sv, scale2, neg_m, pk, acc);
-        }
-        tmem_st32(tS + h * 32, pk);
       }
       float a0, a1, a2, a3;
       f2_unpack(acc[0], a0, a1);

@@ -17,6 +17,8 @@ namespace sparsepr {
 constexpr int kMaxGroups = 1024;  // C_k, C_q upper bound (route rows fit one CTA's smem)
 constexpr int kMaxProbes = 4096;
 constexpr int kSortChunk = 4096;   // tokens per chunk of the parallel stable group sort
+constexpr int kKmChunkGroups = 256;  // groups per launch of the tensor-core k-means assignment
+constexpr int kGramChunk = 4096;     // keys per partial Gram of the key-response rank projection
 
 // Device status word values (a subset of sparsepr_status).
 constexpr int kDevOk = 0;
@@ -41,6 +43,8 @@ struct Layout {
   int trunc_rank;       // 0: whole residual span; r: its r leading eigenvectors
   long long attn_wait_limit;  // > 0: the attention kernel's bounded waits give up after this
                               // many cycles (test hook of the timeout path); 0: the default
+  int key_rank;         // 0 < r < d: the key k-means metric restricted to the r leading
+                        // directions of the key responses (r_K); else the full metric
 
   // status + per-head statistics
   int* status;                    // [1]
@@ -50,6 +54,14 @@ struct Layout {
   double* M;                      // [BH, d, d]
   double* T0k;                    // [BH]  sum_t ||f_t||^2
   double* T0q;                    // [BH]  sum_q ||r~_q||^2
+
+  // key-response rank projection (key_rank in (0, d)): partial and total K^T K, the factor of
+  // M, the eigenvectors of L^T K^T K L and a product scratch
+  double* kgram_part;             // [BH, ceil(N / kGramChunk), d, d]
+  double* kgram;                  // [BH, d, d]
+  double* kr_L;                   // [BH, d, d]
+  double* kr_V;                   // [BH, d, d]
+  double* kr_T;                   // [BH, d, d]
 
   // k-means shared scratch
   int* init_ids;                  // [BH, max(Ck, Cq)]
@@ -100,6 +112,10 @@ struct Layout {
   __nv_bfloat16* Mb;              // [3][BH, d, d]     M
   __nv_bfloat16* Gcb;             // [3][BH, d, d]     Gc
   float* knorm;                   // [BH, N] ||k_t||_2 (rounding bound of the key scores)
+  // running best two scores of every point across the group chunks of one assignment (more
+  // than kKmChunkGroups groups): {best bits, second bits, best group, 0}; null when unused
+  int4* ktop;                     // [BH, N]
+  int4* qtop;                     // [BH, N]
 
   // points of the tensor-core assignment whose two best scores were within the rounding bound,
   // re-decided in fp64: CTA c of the assignment grid appends to its own segment starting at

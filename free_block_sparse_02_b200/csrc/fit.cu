@@ -15,6 +15,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "linalg.cuh"
 
 namespace sparsepr {
 
@@ -97,31 +98,6 @@ __host__ __device__ inline size_t ridge_solve_smem(int d) {
   return base > jac ? base : jac;
 }
 
-// Cholesky G = L L^T of the n x n matrix in shared memory with one barrier per step: step k
-// reads column k of the (lower) trailing matrix, writes L's column k below the diagonal into
-// row k of the upper triangle (L_ik at G[k][i], i > k) and L_kk into diag[k], and updates the
-// trailing lower part G[i][j] -= G[i][k] G[j][k] / G[k][k] (k < j <= i) without touching
-// column k.  False if a pivot is not above `tol` (or not finite).
-__device__ bool chol_smem_tol(double* G, int n, int ld, double tol, double* diag) {
-  const int nthr = blockDim.x;
-  __syncthreads();
-  for (int k = 0; k < n; ++k) {
-    const double piv = G[k * ld + k];
-    if (!(piv > tol) || !isfinite(piv)) return false;  // the same value in every thread
-    const double lkk = sqrt(piv), inv = 1.0 / lkk, ipiv = 1.0 / piv;
-    if (threadIdx.x == 0) diag[k] = lkk;
-    for (int i = k + 1 + threadIdx.x; i < n; i += nthr) G[k * ld + i] = G[i * ld + k] * inv;
-    // trailing pairs (i, j), k < j <= i < n: warp-strided rows, lanes over columns
-    const int nw = nthr >> 5, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = k + 1 + w; i < n; i += nw) {
-      const double lik = G[i * ld + k] * ipiv;
-      for (int j = k + 1 + lane; j <= i; j += 32) G[i * ld + j] -= lik * G[j * ld + k];
-    }
-    __syncthreads();
-  }
-  return true;
-}
-
 // In-place Gauss-Jordan inverse of the symmetric positive definite n x n matrix in shared
 // memory (no pivoting: the pivots of an SPD matrix are the Cholesky pivots squared and stay
 // positive), two barriers per step.  False if a pivot is not positive (or not finite).
@@ -155,94 +131,22 @@ __device__ bool gj_inverse_spd(double* G, int n, int ld) {
 }
 
 // The r leading eigenvectors of S = R^T W R (Table D.2's output truncation), by the parallel
-// cyclic Jacobi method in fp64 (Golub & Van Loan, "Matrix Computations", the symmetric Schur
-// rotation and the round-robin ordering): S in shared memory, the accumulated rotations V next to
-// it when both fit (d = 64), else in the head's spanS (global, where S came from).  A round applies d/2 disjoint rotations, chosen by the
-// circle method so that every (p, q) pair meets once per sweep; sweeps run until the
-// off-diagonal mass is below 1e-30 of the total (squared) or kJacobiSweeps.  The eigenvectors of
-// eigenvalue above 1e-10 of the largest are ranked by eigenvalue (ties: lower index) and the
-// first min(r, count) become the basis; the count goes to span_rank.
-constexpr int kJacobiSweeps = 30;
+// cyclic Jacobi method (jacobi_eig): S in shared memory, the accumulated rotations V next to it
+// when both fit (d = 64), else in the head's spanS (global, where S came from).  The
+// eigenvectors of eigenvalue above 1e-10 of the largest are ranked by eigenvalue (ties: lower
+// index) and the first min(r, count) become the basis; the count goes to span_rank.
 
 __device__ __noinline__ void span_basis_truncated(const Layout& L, int bh, double* S) {
-  const int d = L.d, tid = threadIdx.x, nt = blockDim.x, half = d / 2;
+  const int d = L.d, tid = threadIdx.x, nt = blockDim.x;
   double* Ug = L.spanS + (size_t)bh * d * d;
   // the rotations accumulate in shared memory next to S when both fit (d = 64), else in L2
   double* V = (size_t)2 * d * d * sizeof(double) <= ridge_solve_smem(d) ? S + d * d : Ug;
-  __shared__ double rc[64], rs[64];
-  __shared__ int rp[64], rq[64];
   __shared__ double ev[128];
   __shared__ int order[128];
-  __shared__ double red2[2][8];
   __shared__ int s_kept;
   for (int e = tid; e < d * d; e += nt) S[e] = Ug[e];
   __syncthreads();
-  for (int e = tid; e < d * d; e += nt) V[e] = (e / d == e % d) ? 1.0 : 0.0;
-  __syncthreads();
-  for (int sweep = 0; sweep < kJacobiSweeps; ++sweep) {
-    double off = 0.0, tot = 0.0;
-    for (int e = tid; e < d * d; e += nt) {
-      const double x = S[e] * S[e];
-      tot += x;
-      if (e / d != e % d) off += x;
-    }
-    for (int o = 16; o > 0; o >>= 1) {
-      off += __shfl_xor_sync(0xffffffffu, off, o);
-      tot += __shfl_xor_sync(0xffffffffu, tot, o);
-    }
-    if ((tid & 31) == 0) {
-      red2[0][tid >> 5] = off;
-      red2[1][tid >> 5] = tot;
-    }
-    __syncthreads();
-    off = 0.0;
-    tot = 0.0;
-    for (int w = 0; w < nt / 32; ++w) {
-      off += red2[0][w];
-      tot += red2[1][w];
-    }
-    __syncthreads();
-    if (!(off > 1e-30 * tot)) break;  // the same in every thread (also for a zero S)
-    for (int round = 0; round < d - 1; ++round) {
-      if (tid < half) {
-        const int k = tid;
-        const int a = k == 0 ? 0 : 1 + (k - 1 + round) % (d - 1);
-        const int b = 1 + (d - 2 - k + round) % (d - 1);
-        const int p = min(a, b), q = max(a, b);
-        const double apq = S[p * d + q];
-        double c = 1.0, sn = 0.0;
-        if (apq != 0.0) {
-          const double tau = (S[q * d + q] - S[p * d + p]) / (2.0 * apq);
-          const double t = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
-          c = 1.0 / sqrt(1.0 + t * t);
-          sn = t * c;
-        }
-        rp[k] = p;
-        rq[k] = q;
-        rc[k] = c;
-        rs[k] = sn;
-      }
-      __syncthreads();
-      for (int e = tid; e < half * d; e += nt) {  // S <- S J (columns p, q of every row)
-        const int k = e / d, i = e % d, p = rp[k], q = rq[k];
-        const double c = rc[k], sn = rs[k], x = S[i * d + p], y = S[i * d + q];
-        S[i * d + p] = c * x - sn * y;
-        S[i * d + q] = sn * x + c * y;
-      }
-      __syncthreads();
-      for (int e = tid; e < half * d; e += nt) {  // S <- J^T S (rows p, q), V <- V J
-        const int k = e / d, j = e % d, p = rp[k], q = rq[k];
-        const double c = rc[k], sn = rs[k];
-        const double x = S[p * d + j], y = S[q * d + j];
-        S[p * d + j] = c * x - sn * y;
-        S[q * d + j] = sn * x + c * y;
-        const double u = V[j * d + p], v = V[j * d + q];
-        V[j * d + p] = c * u - sn * v;
-        V[j * d + q] = sn * u + c * v;
-      }
-      __syncthreads();
-    }
-  }
+  jacobi_eig(S, V, d);
   // eigenvalues, the kept ones ranked by size, the leading min(r, kept) columns of V
   for (int i = tid; i < d; i += nt) ev[i] = S[i * d + i];
   __syncthreads();

@@ -36,6 +36,8 @@ int km_tc_grid(const Layout& L, bool keys);
 sparsepr_status launch_kmeans_iteration_tc(const Layout& L, bool keys, const void* X, int it, int G,
                                            cudaStream_t st, const KernelEvents* ev = nullptr);
 sparsepr_status launch_rowqf_tc(const Layout& L, int which, const void* X, cudaStream_t st);
+// M <- its rank-r_K restriction to the leading key-response directions (key_rank in (0, d)).
+sparsepr_status launch_key_rank(const Layout& L, const void* K, cudaStream_t st);
 
 // Upper bound of the number of query tiles of one head: sum_g ceil(n_g / tile) <= N/tile + C_q.
 inline int max_query_tiles(const Layout& L, int tile) { return (L.N + tile - 1) / tile + L.Cq; }

@@ -45,6 +45,9 @@ namespace sparsepr {
 using namespace sm100;
 
 constexpr int kKmTile = 128;
+// bf16 terms of W in the assignment's products: hi + mid leaves |w - hi - mid| <= 2^-18 |w|, an
+// error the rounding bound below covers (the split error is a few percent of the bound)
+constexpr int kKmWTerms = 2;
 constexpr int kKmThreads = 384;   // warp 0 TMA, warp 1 MMA, warps 4..11 epilogue
 constexpr int kKmUpdThreads = 512;
 constexpr int kKmMaxStages = 4;
@@ -59,10 +62,10 @@ __host__ __device__ inline int km_tc_tmem_cols(int n) {
   return c;
 }
 
-// Shared memory of the assignment kernel: three-term W, `stages` X tiles, barriers, per-warp
-// bias copies.
+// Shared memory of the assignment kernel: the kKmWTerms-term W, `stages` X tiles, barriers,
+// per-warp bias copies.
 __host__ inline size_t km_assign_smem(int D, int Np, int stages) {
-  return (size_t)3 * Np * D * 2 + (size_t)stages * kKmTile * D * 2 + 1024 /*align*/ + 256 /*barriers*/ +
+  return (size_t)kKmWTerms * Np * D * 2 + (size_t)stages * kKmTile * D * 2 + 1024 /*align*/ + 256 /*barriers*/ +
          (size_t)8 * 256 * 4 /*bias*/;
 }
 
@@ -82,16 +85,25 @@ __device__ __forceinline__ void km_range(long long T, int G, int c, int& t0, int
   t1 = (int)(T * (c + 1) / G);
 }
 
+// Groups are scored in chunks of at most kKmChunk (all of W of a chunk sits in shared memory
+// and a chunk's scores in one TMEM accumulator).  With more groups than that, one launch per
+// chunk: chunk ci covers groups [c0, c0 + cn); every launch but the last merges its best two
+// scores into each point's running best two (ktop / qtop), and the last one writes the label.
+constexpr int kKmChunk = kKmChunkGroups;
+
 template <bool kKeys>
 __global__ void __launch_bounds__(kKmThreads, 1)
     kmeans_assign_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                            Layout L, int it, int G, int S) {
+                            Layout L, int it, int G, int S, int c0g, int cn, int ci, int nci) {
   pdl_entry();
   const int which = kKeys ? 0 : 1;
   const int D = L.d, KB = D / 64;
   const int C = kKeys ? L.Ck : L.Cq;
-  const int Np = kKeys ? L.Ckp : L.Cqp;
+  const int NpAll = kKeys ? L.Ckp : L.Cqp;      // padded groups of the head's W rows
+  const int Np = nci == 1 ? NpAll : (cn + 15) / 16 * 16;  // padded groups of this chunk
   const int Npr = (Np + 31) & ~31;  // score columns: the epilogue reads 32 at a time
+  const bool first = ci == 0, last = ci == nci - 1;
+  int4* top = kKeys ? L.ktop : L.qtop;  // running best two of every point across chunks
   // With at most 128 (padded) groups, a multiple of 32, the hi and mid terms of W form one B
   // operand of 2 Np rows (one N = 2 Np MMA per K step writes X W_hi and X W_mid side by side)
   // and the lo term adds into the hi half (N = Np): 16 MMAs per tile instead of 24, measured
@@ -106,8 +118,8 @@ __global__ void __launch_bounds__(kKmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sW = sm;                                   // [KB][3 terms][Np rows][128 B]
-  uint8_t* sX = sW + (size_t)3 * Np * D * 2;          // [S][KB][128 rows][128 B]
+  uint8_t* sW = sm;                                   // [KB][kKmWTerms terms][Np rows][128 B]
+  uint8_t* sX = sW + (size_t)kKmWTerms * Np * D * 2;  // [S][KB][128 rows][128 B]
   uint64_t* bars = (uint64_t*)(sX + (size_t)S * kKmTile * D * 2);
   uint64_t* x_full = bars;                            // [S]
   uint64_t* x_empty = bars + kKmMaxStages;            // [S]
@@ -161,11 +173,11 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         const int bh = t / tph;
         if (bh != cur) {  // the head's W, once the MMAs on the previous head's W have completed
           if (wloads > 0 && !mbar_wait(w_empty, (wloads - 1) & 1, &s_abort)) break;
-          mbar_arrive_expect_tx(w_full, (uint32_t)(3 * Np * D * 2));
-          for (int term = 0; term < 3; ++term)
+          mbar_arrive_expect_tx(w_full, (uint32_t)(kKmWTerms * Np * D * 2));
+          for (int term = 0; term < kKmWTerms; ++term)
             for (int kb = 0; kb < KB; ++kb)
-              tma_load_2d(sW + ((size_t)kb * 3 + term) * Np * 128, &tmW, w_full, kb * 64,
-                          term * L.BH * Np + bh * Np);
+              tma_load_2d(sW + ((size_t)kb * kKmWTerms + term) * Np * 128, &tmW, w_full, kb * 64,
+                          term * L.BH * NpAll + bh * NpAll + c0g);
           ++wloads;
           cur = bh;
         }
@@ -201,7 +213,8 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         if (i >= 2 && !mbar_wait(acc_empty + b, ((i >> 1) - 1) & 1, &s_abort)) break;
         tc_fence_after();
         auto wdesc = [&](int term, int ks) {  // K step ks of W term `term` (rows contiguous per kb)
-          return sdesc_sw128(smem_u32(sW + ((size_t)(ks >> 2) * 3 + term) * Np * 128) + (ks & 3) * 32, 16, 1024);
+          return sdesc_sw128(smem_u32(sW + ((size_t)(ks >> 2) * kKmWTerms + term) * Np * 128) + (ks & 3) * 32, 16,
+                             1024);
         };
         auto xdesc = [&](int ks) {
           return sdesc_sw128(smem_u32(sX + ((size_t)s * KB + (ks >> 2)) * kKmTile * 128) + (ks & 3) * 32, 16, 1024);
@@ -209,11 +222,11 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         if (stack) {
           for (int ks = 0; ks < D / 16; ++ks) {
             mma_ss(tmem + b * A, xdesc(ks), wdesc(0, ks), idesc2, ks > 0 ? 1u : 0u);  // [X W_hi | X W_mid]
-            mma_ss(tmem + b * A, xdesc(ks), wdesc(2, ks), idesc, 1u);                 // X W_lo into the hi half
+            if (kKmWTerms == 3) mma_ss(tmem + b * A, xdesc(ks), wdesc(2, ks), idesc, 1u);  // X W_lo into hi
           }
         } else {
           uint32_t acc = 0;
-          for (int term = 0; term < 3; ++term)
+          for (int term = 0; term < kKmWTerms; ++term)
             for (int ks = 0; ks < D / 16; ++ks) {
               mma_ss(tmem + b * A, xdesc(ks), wdesc(term, ks), idesc, acc);
               acc = 1;
@@ -298,7 +311,7 @@ __global__ void __launch_bounds__(kKmThreads, 1)
       scalars(tn, nsq, nxn);                  // in flight while this tile is scanned
       const int bh = t / tph;
       if (bh != cur) {
-        if (cur >= 0) flush(cur);
+        if (cur >= 0 && last) flush(cur);
         cur = bh;
         // the head's biases (this warp's copy) and the maxima of the bound.  Columns C .. Npr-1
         // (padded groups, and columns the MMA does not write) get +inf: their score is +inf or
@@ -307,13 +320,10 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         const float* WN = (kKeys ? L.kwnorm : L.qwnorm) + (size_t)bh * C;
         __syncwarp();  // every lane is done with the previous head's copy
         float wm = 0.f, bm = 0.f;
-        for (int j = lane; j < 256; j += 32) {
-          const float bj = j < C ? B32[j] : INFINITY;
-          bias[j] = bj;
-          if (j < C) {
-            bm = fmaxf(bm, fabsf(bj));
-            wm = fmaxf(wm, WN[j]);
-          }
+        for (int j = lane; j < kKmChunk; j += 32) bias[j] = j < cn ? B32[c0g + j] : INFINITY;
+        for (int j = lane; j < C; j += 32) {  // the bound takes the maxima over all groups
+          bm = fmaxf(bm, fabsf(B32[j]));
+          wm = fmaxf(wm, WN[j]);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -349,17 +359,43 @@ __global__ void __launch_bounds__(kKmThreads, 1)
           b1 = lt ? sc : b1;
         }
       }
-      // rounding bound of the fp32 scores: 3D products in one fp32 chain, plus the epilogue's
-      // operations (the stacked form sums 2D and D products in two chains and adds them once,
-      // which the same bound covers)
-      const float delta = 4.f * (3 * D + 8) * u * xn * wmax + 4.f * u * bmax;
+      if (!first && valid) {  // merge with the best two of the earlier chunks (lower indices win ties)
+        const int4 pv = top[row];
+        const float pb1 = __int_as_float(pv.x), pb2 = __int_as_float(pv.y);
+        if (b1 < pb1) {
+          b2 = fminf(pb1, b2);
+          i1 += c0g;
+        } else {
+          b2 = fminf(pb2, b1);
+          b1 = pb1;
+          i1 = pv.z;
+        }
+      } else if (i1 >= 0) {
+        i1 += c0g;
+      }
+      if (!last) {  // not the last chunk: keep the running best two for the next launch
+        tc_fence_before();
+        mbar_arrive(acc_empty + b);
+        if (valid) top[row] = make_int4(__float_as_int(b1), __float_as_int(b2), i1, 0);
+        t = tn;
+        k += 2;
+        sq = nsq;
+        xn = nxn;
+        continue;
+      }
+      // rounding bound of the fp32 scores: kKmWTerms * D products in one fp32 chain, plus the
+      // epilogue's operations (the stacked form sums the terms in two chains and adds them once,
+      // which the same bound covers), plus, with two terms, the split error 2^-18 |x| |w|
+      const float delta = kKmWTerms == 3
+                              ? 4.f * (3 * D + 8) * u * xn * wmax + 4.f * u * bmax
+                              : (4.f * (2 * D + 8) * u + 4.f * 3.81469727e-6f) * xn * wmax + 4.f * u * bmax;
       const bool ref = valid && !(b2 - b1 > 2.f * delta);
       // candidates of a flagged point: every group whose fp32 score is within the bound of the
       // best (the fp64 argmin is among them).  With at most 128 groups the warp reads its scores
       // once more (warp-uniform branch, before the accumulator is released).
       int nc = 255;
       uint32_t cpk = 0;  // up to four candidate groups, 8 bits each
-      if (Npr <= 128 && __any_sync(0xffffffffu, ref)) {
+      if (nci == 1 && Npr <= 128 && __any_sync(0xffffffffu, ref)) {
         const float thr = b1 + 2.5f * delta;
         int cnt = 0;
 #pragma unroll 1
@@ -397,12 +433,12 @@ __global__ void __launch_bounds__(kKmThreads, 1)
       sq = nsq;
       xn = nxn;
     }
-    if (cur >= 0) flush(cur);
+    if (cur >= 0 && last) flush(cur);
   }
   tc_fence_before();
   __syncthreads();
   if (tid == 0) {
-    L.rcnt[blockIdx.x] = s_rcnt;
+    if (last) L.rcnt[blockIdx.x] = s_rcnt;
     if (s_abort) atomicCAS(L.status, kDevOk, kDevTimeout);
   }
   if (warp == 1) {
@@ -822,11 +858,18 @@ static int km_stages(const Layout& L, int Np) {
   return (int)std::min<size_t>(kKmMaxStages, (budget - fixed) / per);
 }
 
+// Padded groups of one assignment launch: all of them, or a chunk of kKmChunk.
+static int km_chunk_rows(const Layout& L, bool keys) {
+  const int Np = keys ? L.Ckp : L.Cqp;
+  return Np <= kKmChunk ? Np : kKmChunk;
+}
+
 bool km_tc_supported(const Layout& L, bool keys) {
   if (L.dtype != SPARSEPR_BF16) return false;
-  const int Np = keys ? L.Ckp : L.Cqp;
   const int C = keys ? L.Ck : L.Cq;
-  return Np <= 256 && km_stages(L, Np) >= 2 && km_update_smem(L.d, C) <= 227 * 1024;
+  const bool chunked = (keys ? L.Ckp : L.Cqp) > kKmChunk;
+  if (chunked && !(keys ? L.ktop : L.qtop)) return false;
+  return km_stages(L, km_chunk_rows(L, keys)) >= 2 && km_update_smem(L.d, C) <= 227 * 1024;
 }
 
 // CTAs of both k-means kernels: as many as fit the device at once (so the static ranges run in
@@ -839,7 +882,7 @@ int km_tc_grid(const Layout& L, bool keys) {
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms <= 0) sms = 148;
   }
-  const int Np = keys ? L.Ckp : L.Cqp;
+  const int Np = km_chunk_rows(L, keys);
   const int S = km_stages(L, Np);
   const size_t smem = km_assign_smem(L.d, Np, S);
   int occ = 1;
@@ -863,31 +906,31 @@ sparsepr_status launch_kmeans_iteration_tc(const Layout& L, bool keys, const voi
   };
   CUtensorMap mX, mW;
   const int D = L.d;
-  const int Np = keys ? L.Ckp : L.Cqp;
+  const int NpAll = keys ? L.Ckp : L.Cqp;
   const int C = keys ? L.Ck : L.Cq;
   const void* wbase = keys ? (const void*)L.kWb : (const void*)L.qWb;
-  if (!make_tmap_bf16(&mX, X, (long long)L.BH * L.N, D, kKmTile) ||
-      !make_tmap_bf16(&mW, wbase, 3LL * L.BH * Np, D, Np))
-    return SPARSEPR_ERR_CUDA;
-  const int S = km_stages(L, Np);
-  const size_t smem_a = km_assign_smem(D, Np, S);
+  if (!make_tmap_bf16(&mX, X, (long long)L.BH * L.N, D, kKmTile)) return SPARSEPR_ERR_CUDA;
+  const int nci = NpAll <= kKmChunk ? 1 : (C + kKmChunk - 1) / kKmChunk;
+  const int S = km_stages(L, km_chunk_rows(L, keys));
+  const size_t smem_a = km_assign_smem(D, km_chunk_rows(L, keys), S);
   const size_t smem_u = km_update_smem(D, C);
   const __nv_bfloat16* Xb = (const __nv_bfloat16*)X;
-  if (keys) {
-    cudaFuncSetAttribute(kmeans_assign_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
-    cudaFuncSetAttribute(kmeans_update_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_u);
-    mark(SPARSEPR_KERNEL_KMEANS_ASSIGN, false);
-    launch(kmeans_assign_tc_kernel<true>, G, kKmThreads, smem_a, st, mX, mW, L, it, G, S);
-    mark(SPARSEPR_KERNEL_KMEANS_ASSIGN, true);
-    mark(SPARSEPR_KERNEL_KMEANS_UPDATE, false);
-    launch(kmeans_update_kernel<true>, G, kKmUpdThreads, smem_u, st, Xb, L, it, G);
-    mark(SPARSEPR_KERNEL_KMEANS_UPDATE, true);
-  } else {
-    cudaFuncSetAttribute(kmeans_assign_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
-    cudaFuncSetAttribute(kmeans_update_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_u);
-    launch(kmeans_assign_tc_kernel<false>, G, kKmThreads, smem_a, st, mX, mW, L, it, G, S);
-    launch(kmeans_update_kernel<false>, G, kKmUpdThreads, smem_u, st, Xb, L, it, G);
+  auto assign = keys ? kmeans_assign_tc_kernel<true> : kmeans_assign_tc_kernel<false>;
+  auto update = keys ? kmeans_update_kernel<true> : kmeans_update_kernel<false>;
+  cudaFuncSetAttribute(assign, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
+  cudaFuncSetAttribute(update, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_u);
+  if (keys) mark(SPARSEPR_KERNEL_KMEANS_ASSIGN, false);
+  for (int ci = 0; ci < nci; ++ci) {
+    // chunk ci: groups [c0, c0 + cn), W rows [c0, c0 + round16(cn)) of each head and term
+    const int c0 = ci * kKmChunk, cn = nci == 1 ? C : std::min(kKmChunk, C - c0);
+    const int rows = nci == 1 ? NpAll : (cn + 15) / 16 * 16;
+    if (!make_tmap_bf16(&mW, wbase, 3LL * L.BH * NpAll, D, rows)) return SPARSEPR_ERR_CUDA;
+    launch(assign, G, kKmThreads, smem_a, st, mX, mW, L, it, G, S, c0, cn, ci, nci);
   }
+  if (keys) mark(SPARSEPR_KERNEL_KMEANS_ASSIGN, true);
+  if (keys) mark(SPARSEPR_KERNEL_KMEANS_UPDATE, false);
+  launch(update, G, kKmUpdThreads, smem_u, st, Xb, L, it, G);
+  if (keys) mark(SPARSEPR_KERNEL_KMEANS_UPDATE, true);
   SPR_LAUNCH_CHECK();
   return SPARSEPR_OK;
 }

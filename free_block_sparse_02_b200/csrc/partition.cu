@@ -1219,6 +1219,10 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
   cudaFuncSetAttribute(rowqf_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qf_smem);
   // keys: metric M = Qs^T Qs / d, objective constant sum_t k_t^T M k_t, key norms
   launch(metric_kernel<T>, dim3(L.BH, d / kMetricRows), 256, 0, st, L, Q);
+  if (L.kgram) {  // key-response rank r_K: M <- M_r before anything uses M
+    const sparsepr_status s = launch_key_rank(L, K, st);
+    if (s != SPARSEPR_OK) return s;
+  }
   cudaMemsetAsync(L.T0k, 0, sizeof(double) * L.BH, st);
   cudaMemsetAsync(L.T0q, 0, sizeof(double) * L.BH, st);
   if (tc) {

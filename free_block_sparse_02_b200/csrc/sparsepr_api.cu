@@ -53,6 +53,7 @@ sparsepr_status validate(const sparsepr_config* c) {
   if (c->correction != SPARSEPR_CORRECTION_AFFINE && c->correction != SPARSEPR_CORRECTION_MEAN)
     return SPARSEPR_ERR_INVALID_ARG;
   if (c->trunc_rank < 0 || c->trunc_rank > c->d) return SPARSEPR_ERR_INVALID_ARG;
+  if (c->key_rank < 0 || c->key_rank > c->d) return SPARSEPR_ERR_INVALID_ARG;
   if ((double)c->B * c->H * c->N * 256.0 > 9.0e18) return SPARSEPR_ERR_INVALID_ARG;
   if (c->d != 64 && c->d != 128) return SPARSEPR_ERR_UNSUPPORTED;
   // rows of the [B*H*N, d] views are int32 in the kernels (tiles of 128 rows)
@@ -87,6 +88,7 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   L.repair = c.repair;
   L.correction = c.correction;
   L.trunc_rank = c.trunc_rank;
+  L.key_rank = c.key_rank;
   size_t off = 0;
   auto take = [&](auto*& ptr, size_t bytes) {
     using P_ = std::remove_reference_t<decltype(ptr)>;
@@ -99,6 +101,13 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   take(L.M, BH * d * d * 8);
   take(L.T0k, BH * 8);
   take(L.T0q, BH * 8);
+  if (c.key_rank > 0 && c.key_rank < c.d && c.partition == SPARSEPR_PARTITION_RESPONSE) {
+    take(L.kgram_part, BH * ((N + kGramChunk - 1) / kGramChunk) * d * d * 8);
+    take(L.kgram, BH * d * d * 8);
+    take(L.kr_L, BH * d * d * 8);
+    take(L.kr_V, BH * d * d * 8);
+    take(L.kr_T, BH * d * d * 8);
+  }
   take(L.init_ids, BH * std::max(Ck, Cq) * 4);
   take(L.fy, 4);  // unused: the draw keeps its slots in shared memory
   take(L.iters_run, BH * 2 * 4);
@@ -137,6 +146,8 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   take(L.Mb, 3 * BH * d * d * 2);
   take(L.Gcb, 3 * BH * d * d * 2);
   take(L.knorm, BH * N * 4);
+  if (L.Ckp > kKmChunkGroups) take(L.ktop, BH * N * 16);
+  if (L.Cqp > kKmChunkGroups) take(L.qtop, BH * N * 16);
   const size_t km_tiles = BH * (size_t)((N + 127) / 128);
   take(L.rlist, km_tiles * 128 * 16);
   take(L.rcnt, km_tiles * 4);

@@ -95,6 +95,11 @@ typedef struct sparsepr_config {
   int32_t trunc_rank;       /* 0: the map's outputs restricted to the whole probe-residual span
                                (the identity on the ridge solution); 1 <= r <= d: to the r leading
                                eigenvectors of R^T W R (Table D.2's output truncation)           */
+  int32_t key_rank;         /* Table C.1's key response rank r_K.  0 (or d): the key k-means sees
+                               the full key responses; 0 < r < d: the N x s key responses are taken
+                               in the basis of their r leading right singular vectors (the best
+                               rank-r approximation, not centred) before the key k-means.  0..d;
+                               the semantic partition ignores it                                */
 } sparsepr_config;
 
 enum { SPARSEPR_CORRECTION_AFFINE = 0, SPARSEPR_CORRECTION_MEAN = 1 };

@@ -205,6 +205,18 @@ def lloyd(X: np.ndarray, init_centroids: np.ndarray, iters: int, tol: float,
                         stop_margin=stop_margin, label_history=hist)
 
 
+def key_response_basis(F: np.ndarray, rank: int) -> Optional[np.ndarray]:
+    """Table C.1 "Key response rank r_K" (48 in the paper's runs).  Reading: the N x s key
+    responses are taken in the basis of their r_K leading right singular vectors (the best
+    rank-r_K approximation of the response matrix, not centred), so k-means sees the r_K-dim
+    coordinates F V_r.  Returns V_r (s x r), or None when rank is 0 (off) or not below the
+    response matrix's rank bound min(N, s) (the projection would keep every distance)."""
+    if rank <= 0 or rank >= min(F.shape):
+        return None
+    _, _, Vt = np.linalg.svd(F, full_matrices=False)
+    return Vt[:rank].T
+
+
 # ----------------------------------------------------------------------------------------------
 # Step 3: query responses to the key-group centroids, per-query RMS normalisation.
 # ----------------------------------------------------------------------------------------------
@@ -469,8 +481,9 @@ def call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int,
     """One (batch, head) of one call.  cfg needs: s, n_kgroups, n_qgroups, density, fixed_k,
     P, probe_mode (0 uniform, 1 stratified, 2 random), lam, km_iters, km_iters_warm, km_tol,
     seed, and optionally partition (0 response-coupled, 1 semantic), repair (1 correct, 0 not),
-    correction (0 affine map of [O_sp, 1], 1 mean-only) and trunc_rank (0 none, r > 0 the r
-    leading residual directions)."""
+    correction (0 affine map of [O_sp, 1], 1 mean-only), trunc_rank (0 none, r > 0 the r
+    leading residual directions) and key_rank (0 none, r > 0 the key responses in their r
+    leading right singular directions, Table C.1's r_K)."""
     if getattr(cfg, "partition", 0) == 1:
         return semantic_call_head(q, k, v, cfg, bh, compute_outputs=compute_outputs)
     q = np.asarray(q, dtype=np.float64)
@@ -486,11 +499,16 @@ def call_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, cfg, bh: int,
     rows = sample_query_rows(N, cfg.s)
     Qs = q[rows]
     F = (k @ Qs.T) * scale
+    Vr = key_response_basis(F, getattr(cfg, "key_rank", 0))
+    if Vr is not None:
+        F = F @ Vr
     if warm is None:
         ids = kmeans_init_ids(N, Ck, stream_seed(seed, bh, 0))
         C0, S0, iters = F[ids], k[ids], cfg.km_iters
     else:
         C0 = (warm.key_centroids @ Qs.T) * scale
+        if Vr is not None:
+            C0 = C0 @ Vr
         S0, iters = warm.key_centroids, cfg.km_iters_warm
     kk = lloyd(F, C0, iters, tol, shadow=k, shadow_init=S0, keep_history=keep_history)
     klabels = kk.labels

@@ -15,13 +15,14 @@ PEAKS = {"hbm_gbs": 6557.4, "bf16_tflops": 1629.0}
 
 
 def test_assignment_roofline_is_the_binding_one():
-    """13B-DiT layer: 6 C_p d = 98,304 flops and 2d + 4 = 260 bytes per key, so the tensor time
-    (flops / peak) exceeds the HBM time; the mid-size shape (d = 64, C_p = 64) is HBM-bound."""
+    """13B-DiT layer: 4 C_p d = 65,536 flops (two bf16 terms of W) and 2d + 4 = 260 bytes per
+    key, so the tensor time (flops / peak) exceeds the HBM time; the mid-size shape (d = 64,
+    C_p = 64) is HBM-bound."""
     big = bench.km_rooflines(configs.workload(2), 0.378, 0.244, PEAKS)
     assert big["assignment"]["bound"] == "tensor" and big["assignment"]["unit"] == "TFLOP/s"
     assert big["assignment"]["other"]["unit"] == "GB/s"
     keys = 24 * 118800
-    assert big["assignment"]["achieved"] == pytest.approx(keys * 6 * 128 * 128 / 0.378e-3 / 1e12)
+    assert big["assignment"]["achieved"] == pytest.approx(keys * 4 * 128 * 128 / 0.378e-3 / 1e12)
     assert big["update"]["bound"] == "hbm"
     assert big["update"]["achieved"] == pytest.approx(keys * 260 / 0.244e-3 / 1e9)
     mid = bench.km_rooflines(configs.workload(1), 0.0205, 0.0246, PEAKS)

@@ -104,9 +104,13 @@ def check_head(w, g, h, q, k, v, warm=None, log=None, case="", n_rows=256):
         bar = "scaled"
         _close(f"{case} head {h} O rows (bar x gain)", got[rows], ref_rows, 2e-2 * gain_inf, 1e-2 * gain_2)
     if log is not None:
-        den = np.linalg.norm(ref_rows, axis=1) + 1e-8
-        log.append(dict(case=case, head=h, gain_inf=float(gain_inf), gain_2=float(gain_2), e2e=bar, slack=0.0,
-                        e_gpu=float((np.linalg.norm(got[rows] - ref_rows, axis=1) / den).mean()), e_orc=0.0))
+        # the sampled rows' errors against the exact dense rows: the GPU's and the oracle's
+        dense = O.attention(q[rows], k, v)
+        log.append(dict(case=case, head=h, gain_inf=float(gain_inf), gain_2=float(gain_2), e2e=bar,
+                        e2e_abs=float(np.abs(got[rows] - ref_rows).max()),
+                        e2e_rl2=float(np.linalg.norm(got[rows] - ref_rows) / np.linalg.norm(ref_rows)), slack=0.0,
+                        e_gpu=float(O.row_errors(got[rows], dense).mean()),
+                        e_orc=float(O.row_errors(ref_rows, dense).mean())))
     if same:
         return O.warm_state(r)
     return O.WarmState(key_centroids=g.kc[h], query_centroids=g.qc[h])

@@ -174,6 +174,9 @@ def compare_outputs(op, out, qf, kf, vf, w, atol, rel_l2, log=None, case=""):
         gain_inf = 1.0 + np.abs(A_lin).sum(axis=0).max()
         gain_2 = 1.0 + np.linalg.norm(A_lin, 2)
         bar = "stage-only"
+        d_e2e = np.abs(O_gpu[bh] - ref["O"])
+        e2e_abs = float(d_e2e.max()) if d_e2e.size else 0.0
+        e2e_rl2 = float(np.linalg.norm(O_gpu[bh] - ref["O"]) / max(np.linalg.norm(ref["O"]), 1e-30))
         if w.dtype == configs.F32 or len(p) >= w.d + 1:
             if gain_inf <= 1.1 and gain_2 <= 1.1:
                 bar = "flat"
@@ -195,7 +198,8 @@ def compare_outputs(op, out, qf, kf, vf, w, atol, rel_l2, log=None, case=""):
         slack = (1e-4 if w.dtype == configs.F32 else 5e-3) * gain_2
         if log is not None:
             log.append(dict(case=case or w.name, head=bh, gain_inf=float(gain_inf), gain_2=float(gain_2), e2e=bar,
-                            slack=float(slack), e_gpu=float(e_gpu), e_orc=float(e_orc)))
+                            e2e_abs=e2e_abs, e2e_rl2=e2e_rl2, slack=float(slack), e_gpu=float(e_gpu),
+                            e_orc=float(e_orc)))
         assert e_gpu <= e_orc * (1 + 1e-3) + slack, f"head {bh}: mean error {e_gpu} > oracle {e_orc}"
     return errs
 
@@ -259,6 +263,18 @@ EDGE = {
                                 trunc_rank=16, km_iters=8),
     "many-groups": dict(base=1, grid=(4, 16, 32), heads=1, s=128, n_kgroups=600, n_qgroups=300, P=64, lam=1.0,
                         km_iters=5),
+    # 129-256 groups: one assignment launch without the stacked hi|mid form; and more than 256
+    # at d = 128 (group chunks of 256, the last one ragged), on two heads
+    "groups-200-d128": dict(base=2, grid=(3, 10, 40), heads=2, s=96, n_kgroups=200, n_qgroups=144, P=160,
+                            km_iters=5),
+    "groups-1000-d128": dict(base=2, grid=(3, 20, 40), heads=2, s=256, n_kgroups=1000, n_qgroups=300, P=64,
+                             lam=1.0, km_iters=4),
+    # Table C.1's key response rank r_K: the key k-means on the r leading response directions;
+    # with s >= d (positive definite M: Cholesky factor) and s < d (singular M: eigen factor)
+    "key-rank-d128": dict(base=2, grid=(3, 10, 40), heads=2, s=256, n_kgroups=16, n_qgroups=12, P=160, key_rank=8,
+                          km_iters=6),
+    "key-rank-few-samples": dict(base=1, grid=(4, 16, 32), heads=1, s=32, n_kgroups=16, n_qgroups=12, P=80,
+                                 key_rank=16, km_iters=6),
 }
 
 

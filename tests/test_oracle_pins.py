@@ -590,3 +590,58 @@ def test_warm_start_from_converged_centroids_is_a_fixed_point():
     assert np.array_equal(rw["klabels"], r["klabels"]) and np.array_equal(rw["qlabels"], r["qlabels"])
     np.testing.assert_allclose(rw["kmeans_k"].objective[0], r["kmeans_k"].objective[-1], rtol=1e-12)
     np.testing.assert_allclose(rw["kmeans_q"].objective[0], r["kmeans_q"].objective[-1], rtol=1e-12)
+
+
+# ---------------------------------------------------------------- key response rank (Table C.1 r_K)
+def test_key_response_basis_is_the_best_rank_r_approximation():
+    """Eckart-Young: projecting the responses on their r leading right singular vectors leaves
+    exactly the energy of the trailing eigenvalues of F^T F (a separate symmetric eigensolver)."""
+    rng = np.random.default_rng(41)
+    F = rng.standard_normal((200, 12)) @ rng.standard_normal((12, 30))
+    for r in (1, 5, 11):
+        Vr = O.key_response_basis(F, r)
+        assert Vr.shape == (30, r)
+        np.testing.assert_allclose(Vr.T @ Vr, np.eye(r), atol=1e-12)
+        resid = np.linalg.norm(F - F @ Vr @ Vr.T) ** 2
+        ev = np.sort(np.linalg.eigvalsh(F.T @ F))[::-1]
+        np.testing.assert_allclose(resid, ev[r:].sum(), rtol=1e-9, atol=1e-9 * ev[0])
+    assert O.key_response_basis(F, 0) is None and O.key_response_basis(F, 30) is None
+
+
+class _RankCfg(_WarmCfg):
+    def __init__(self, key_rank):
+        super().__init__(8, 0)
+        self.key_rank = key_rank
+
+
+def test_key_rank_at_or_above_the_response_rank_changes_nothing():
+    """F = K Qs^T / sqrt(d) has rank <= d, so its d leading singular directions keep every
+    distance: the key groups equal the unprojected ones."""
+    q, k, v = _small_inputs(42)
+    d = q.shape[1]
+    full = O.call_head(q, k, v, _RankCfg(0), 0, compute_outputs=False)
+    same = O.call_head(q, k, v, _RankCfg(d), 0, compute_outputs=False)
+    assert np.array_equal(full["klabels"], same["klabels"])
+    np.testing.assert_allclose(same["kmeans_k"].objective, full["kmeans_k"].objective, rtol=1e-9)
+
+
+def test_key_rank_equals_metric_kmeans_in_key_space():
+    """k-means on the rank-r response coordinates equals Euclidean k-means (scikit-learn) on the
+    keys mapped by L Z_r, where M = Qs^T Qs / d = L L^T (Cholesky) and Z_r holds the r leading
+    eigenvectors of L^T (K^T K) L: a different route through d x d matrices only."""
+    from sklearn.cluster import KMeans
+    q, k, v = _small_inputs(43, N=120, d=8)
+    cfg = _RankCfg(3)
+    r = O.call_head(q, k, v, cfg, 0, compute_outputs=False)
+    d = q.shape[1]
+    Qs = q[O.sample_query_rows(q.shape[0], cfg.s)]
+    Lc = np.linalg.cholesky(Qs.T @ Qs / d)
+    ev, Z = np.linalg.eigh(Lc.T @ (k.T @ k) @ Lc)
+    Zr = Z[:, np.argsort(-ev)[:cfg.key_rank]]
+    Y = k @ Lc @ Zr
+    ids = O.kmeans_init_ids(q.shape[0], cfg.n_kgroups, O.stream_seed(cfg.seed, 0, 0))
+    km = KMeans(n_clusters=cfg.n_kgroups, init=Y[ids], n_init=1, max_iter=cfg.km_iters, tol=0.0,
+                algorithm="lloyd").fit(Y)
+    assert np.array_equal(r["klabels"], km.labels_)
+    # and the rank matters on these inputs
+    assert not np.array_equal(r["klabels"], O.call_head(q, k, v, _RankCfg(0), 0, compute_outputs=False)["klabels"])
