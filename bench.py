@@ -243,10 +243,10 @@ def km_rooflines(w, asg_ms, upd_ms, pk):
     out = {}
     if asg_ms > 0:
         s = asg_ms * 1e-3
-        t_hbm, t_tc = by / (pk["hbm_gbs"] * 1e9), fl / (pk["bf16_tflops"] * 1e12)
+        tpk = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])  # inside a long step
+        t_hbm, t_tc = by / (pk["hbm_gbs"] * 1e9), fl / (tpk * 1e12)
         hbm = {"achieved": by / s / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": by / s / 1e9 / pk["hbm_gbs"]}
-        tc = {"achieved": fl / s / 1e12, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-              "frac": fl / s / 1e12 / pk["bf16_tflops"]}
+        tc = {"achieved": fl / s / 1e12, "peak": tpk, "unit": "TFLOP/s", "frac": fl / s / 1e12 / tpk}
         main, other = (tc, hbm) if t_tc >= t_hbm else (hbm, tc)
         out["assignment"] = {"bound": "tensor" if t_tc >= t_hbm else "hbm", **main, "ms": asg_ms, "traffic": None,
                              "other": other,
@@ -496,7 +496,10 @@ def run_ours(args, w, world, rank, local):
         job_flops = w.dense_flops() * (1 if shard else world)
         value = job_flops / (ms_max * 1e-3) / 1e12
         achieved = kflops / (kms_max * 1e-3) / 1e12
-        peak = pk["bf16_tflops"]
+        # the kernel is timed inside a long step (a whole call, calls back to back under the
+        # power cap): the sustained bf16 figure is its peak; the burst figure is given beside it
+        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        burst = pk["bf16_tflops"]
         elt = Q.element_size()
         if shard:
             par = f"one call split by heads over {world} GPUs ({wl.H} or so heads each, no data-path collective" + \
@@ -517,7 +520,9 @@ def run_ours(args, w, world, rank, local):
                                                         "rows (the kernel the metric's % of bf16 peak refers to)",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "traffic": profiled_traffic(wl),
-                         "peak_source": f"{pk['source']} bf16 dense (burst), MEASURED_PEAKS.json",
+                         "peak_source": f"{pk['source']} bf16 dense, sustained (the kernel runs inside a long "
+                                        f"step), MEASURED_PEAKS.json",
+                         "peak_burst": burst, "frac_of_burst": achieved / burst,
                          "algorithmic": f"4*d*(executed sparse pairs + P*N*heads) = {kflops:.4g} flop per launch "
                                         f"(rank 0; smallest over ranks {kflops_min:.4g})"},
             "roofline_kmeans": km_rooflines(wl, asg_ms, upd_ms, pk) if tc_km else None,

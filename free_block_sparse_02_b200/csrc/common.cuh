@@ -105,7 +105,8 @@ struct Layout {
   int* qrefined;                  // [BH]
 
   // bf16 operands of the tensor-core kernels: fp64 matrices split into three bf16 terms
-  // (hi + mid + lo reproduces the value to ~2^-24 relative); group rows padded to 16
+  // (hi + mid + lo reproduces the value to ~2^-24 relative; the k-means assignment reads hi and
+  // mid, the row quadratic forms all three); group rows padded to 16
   int Ckp, Cqp;
   __nv_bfloat16* kWb;             // [3][BH, Ckp, d]   W_j = M c_j
   __nv_bfloat16* qWb;             // [3][BH, Cqp, d]   u_g
