@@ -165,7 +165,7 @@ __device__ __noinline__ void span_basis_truncated(const Layout& L, int bh, doubl
   }
   __syncthreads();
   const int rank = min(L.trunc_rank, s_kept);
-  for (int e = tid; e < d * rank; e += nt) S[e] = V[(e / rank) * d + order[e % rank]];  // [d][rank]
+  for (int e = tid; e < d * rank; e += nt) S[e] = V[order[e % rank] * d + e / rank];  // [d][rank] (V: rows)
   __syncthreads();
   for (int e = tid; e < d * rank; e += nt) Ug[(e / rank) * d + e % rank] = S[e];  // U[i*d + r]
   if (tid == 0) L.stats[bh].span_rank = rank;

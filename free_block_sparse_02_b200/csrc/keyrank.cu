@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(256) key_rank_kernel(Layout L) {
   double* M = L.M + bh * dd;
   const double* G = L.kgram + bh * dd;
   double* Lf = L.kr_L + bh * dd;  // the factor L (d x d, row-major)
-  double* V = L.kr_V + bh * dd;   // eigenvectors (columns)
+  double* V = L.kr_V + bh * dd;   // eigenvectors (rows, as jacobi_eig leaves them)
   double* T = L.kr_T + bh * dd;   // G L, later Y = L Z_r (d x r)
   // factor of M: Cholesky when M is positive definite, else E D^(1/2)
   for (size_t e = tid; e < dd; e += nt) sS[e] = M[e];
@@ -100,8 +100,8 @@ __global__ void __launch_bounds__(256) key_rank_kernel(Layout L) {
     __syncthreads();
     jacobi_eig(sS, V, d);
     for (size_t e = tid; e < dd; e += nt) {
-      const int k = (int)(e % d);  // L = E D^(1/2): column k of E times sqrt(lambda_k)
-      Lf[e] = V[e] * sqrt(fmax(sS[k * d + k], 0.0));
+      const int i = (int)(e / d), k = (int)(e % d);  // L = E D^(1/2): E[i][k] = row k of V, entry i
+      Lf[e] = V[(size_t)k * d + i] * sqrt(fmax(sS[k * d + k], 0.0));
     }
   }
   __syncthreads();
@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(256) key_rank_kernel(Layout L) {
   for (int e = tid; e < d * r; e += nt) {
     const int i = e / r, q = e % r, col = order[q];
     double s = 0.0;
-    for (int m = 0; m < d; ++m) s += Lf[(size_t)i * d + m] * V[(size_t)m * d + col];
+    for (int m = 0; m < d; ++m) s += Lf[(size_t)i * d + m] * V[(size_t)col * d + m];
     T[e] = s;
   }
   __syncthreads();

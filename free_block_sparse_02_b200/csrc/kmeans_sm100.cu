@@ -726,6 +726,8 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
 //   keys    (which 0): T0k += sum x^T M x;  knorm = ||x||
 //   queries (which 1): ms = x^T Gc x;  inv_rms = 1/sqrt(ms + 1e-12);  qxnorm = ||x|| inv_rms;
 //                      T0q += C_k ms / (ms + 1e-12)   (= ||r~||^2)
+// Two X stages and two TMEM accumulators: the products of tile i + 1 run while the threads
+// read tile i, and the copy of tile i + 2 is issued as soon as tile i's stage is read.
 __global__ void __launch_bounds__(128, 1)
     rowqf_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmG, Layout L,
                     int which, int tiles_per_cta) {
@@ -738,19 +740,26 @@ __global__ void __launch_bounds__(128, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const size_t xbytes = (size_t)kKmTile * D * 2;
   uint8_t* sG = sm;                              // [3][KB][D rows][128 B]
-  uint8_t* sX = sG + (size_t)3 * D * D * 2;      // [KB][128 rows][128 B]
-  uint64_t* bars = (uint64_t*)(sX + (size_t)kKmTile * D * 2);
-  uint32_t* tmem_slot = (uint32_t*)(bars + 3);
+  uint8_t* sX = sG + (size_t)3 * D * D * 2;      // [2 stages][KB][128 rows][128 B]
+  uint64_t* g_full = (uint64_t*)(sX + 2 * xbytes);
+  uint64_t* x_full = g_full + 1;                 // [2]
+  uint64_t* mma_done = x_full + 2;               // [2]
+  uint64_t* mma_all = mma_done + 2;              // every product of the CTA (before TMEM is freed)
+  uint32_t* tmem_slot = (uint32_t*)(mma_all + 1);
   __shared__ volatile int s_abort;
   __shared__ double red[4];
   const int tid = threadIdx.x, warp = tid >> 5;
-  const uint32_t tcols = km_tc_tmem_cols(D);
+  const uint32_t tcols = km_tc_tmem_cols(2 * D);
   if (tid == 0) {
     s_abort = 0;
-    mbar_init(bars + 0, 1);
-    mbar_init(bars + 1, 1);
-    mbar_init(bars + 2, 1);
+    mbar_init(g_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(x_full + b, 1);
+      mbar_init(mma_done + b, 1);
+    }
+    mbar_init(mma_all, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -761,50 +770,62 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint32_t idesc = idesc_bf16_f32(kKmTile, D, 0, 0);
+  int issued = 0;  // X copies issued (thread 0)
+  auto load_x = [&](int ti) {  // thread 0: tile ti into stage ti & 1
+    const int b = ti & 1;
+    mbar_arrive_expect_tx(x_full + b, (uint32_t)xbytes);
+    for (int kb = 0; kb < KB; ++kb)
+      tma_load_2d(sX + b * xbytes + (size_t)kb * kKmTile * 128, &tmX, x_full + b, kb * 64,
+                  bh * L.N + (tile0 + ti) * kKmTile);
+    ++issued;
+  };
+  auto issue_mma = [&](int ti) -> bool {  // thread 0: U_ti = X_ti G into accumulator ti & 1
+    const int b = ti & 1;
+    if (!mbar_wait(x_full + b, (ti >> 1) & 1, &s_abort)) return false;
+    tc_fence_after();
+    uint32_t acc = 0;
+    for (int gt = 0; gt < 3; ++gt)
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t xa = smem_u32(sX + b * xbytes + (size_t)(ks >> 2) * kKmTile * 128) + (ks & 3) * 32;
+        const uint32_t ga = smem_u32(sG + ((size_t)gt * KB + (ks >> 2)) * D * 128) + (ks & 3) * 32;
+        mma_ss(tmem + b * D, sdesc_sw128(xa, 16, 1024), sdesc_sw128(ga, 16, 1024), idesc, acc);
+        acc = 1;
+      }
+    mma_commit(mma_done + b);
+    return true;
+  };
   if (tid == 0) {
-    mbar_arrive_expect_tx(bars + 0, (uint32_t)(3 * D * D * 2));
+    mbar_arrive_expect_tx(g_full, (uint32_t)(3 * D * D * 2));
     for (int t = 0; t < 3; ++t)
       for (int kb = 0; kb < KB; ++kb)
-        tma_load_2d(sG + ((size_t)t * KB + kb) * D * 128, &tmG, bars + 0, kb * 64, t * L.BH * D + bh * D);
+        tma_load_2d(sG + ((size_t)t * KB + kb) * D * 128, &tmG, g_full, kb * 64, t * L.BH * D + bh * D);
+    load_x(0);
+    if (ntile > 1) load_x(1);
+    if (mbar_wait(g_full, 0, &s_abort)) issue_mma(0);
   }
-  const uint32_t idesc = idesc_bf16_f32(kKmTile, D, 0, 0);
   double tot = 0.0;
-  for (int ti = 0; ti < ntile && !s_abort; ++ti) {
+  for (int ti = 0; ti < ntile; ++ti) {
+    const int b = ti & 1;
+    if (tid == 0 && ti + 1 < ntile && !s_abort) issue_mma(ti + 1);  // runs while tile ti is read
+    const bool waited = !s_abort && mbar_wait(mma_done + b, (ti >> 1) & 1, &s_abort);
+    if (__syncthreads_or(!waited)) break;  // uniform: every thread leaves or none does
+    tc_fence_after();
     const int p0 = (tile0 + ti) * kKmTile;
     const int np = min(kKmTile, L.N - p0);
-    if (tid == 0) {
-      mbar_arrive_expect_tx(bars + 1, (uint32_t)(kKmTile * D * 2));
-      for (int kb = 0; kb < KB; ++kb)
-        tma_load_2d(sX + (size_t)kb * kKmTile * 128, &tmX, bars + 1, kb * 64, bh * L.N + p0);
-      const bool ok = (ti > 0 || mbar_wait(bars + 0, 0, &s_abort)) && mbar_wait(bars + 1, ti & 1, &s_abort);
-      if (ok) {
-        tc_fence_after();
-        uint32_t acc = 0;
-        for (int gt = 0; gt < 3; ++gt)
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t xa = smem_u32(sX + (size_t)(ks >> 2) * kKmTile * 128) + (ks & 3) * 32;
-            const uint32_t ga = smem_u32(sG + ((size_t)gt * KB + (ks >> 2)) * D * 128) + (ks & 3) * 32;
-            mma_ss(tmem, sdesc_sw128(xa, 16, 1024), sdesc_sw128(ga, 16, 1024), idesc, acc);
-            acc = 1;
-          }
-      }
-      mma_commit(bars + 2);
-    }
-    const bool waited = mbar_wait(bars + 2, ti & 1, &s_abort);
-    if (__syncthreads_or(!waited)) break;
-    tc_fence_after();
     const int p = tid;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint8_t* xs = sX + b * xbytes;
     float qf = 0.f, nn = 0.f;
     for (int c0 = 0; c0 < D; c0 += 32) {
       uint32_t r[32];
-      tmem_ld32(tmem + lane_base + c0, r);
+      tmem_ld32(tmem + lane_base + b * D + c0, r);
       tmem_wait_ld();
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
         const int a = c0 + k, kb = a >> 6, w = a & 63;
         const uint32_t off = (uint32_t)p * 128 + ((((w >> 3) ^ (p & 7)) << 4) | ((w & 7) << 1));
-        const float x = __bfloat162float(*(const __nv_bfloat16*)(sX + (size_t)kb * kKmTile * 128 + off));
+        const float x = __bfloat162float(*(const __nv_bfloat16*)(xs + (size_t)kb * kKmTile * 128 + off));
         qf = fmaf(x, __uint_as_float(r[k]), qf);
         nn = fmaf(x, x, nn);
       }
@@ -831,16 +852,21 @@ __global__ void __launch_bounds__(128, 1)
       }
     }
     tc_fence_before();
-    __syncthreads();
+    __syncthreads();  // stage b and accumulator b are read: the copy of tile ti + 2 may land in b
+    if (tid == 0 && ti + 2 < ntile && !s_abort) load_x(ti + 2);
   }
   tot = block_sum(tot, red);
   if (tid == 0) {
     atomicAdd((which == 0 ? L.T0k : L.T0q) + bh, tot);
     if (s_abort) {
       atomicCAS(L.status, kDevOk, kDevTimeout);
-      mbar_wait_drain(bars + 0, 0);
-      for (int ti = 0; ti < ntile; ++ti) mbar_wait_drain(bars + 1, ti & 1);
+      // never leave with copies or products in flight: the last copies issued into each stage,
+      // and every product committed so far
+      mbar_wait_drain(g_full, 0);
+      for (int ti = max(0, issued - 2); ti < issued; ++ti) mbar_wait_drain(x_full + (ti & 1), (ti >> 1) & 1);
     }
+    mma_commit(mma_all);  // arrives once every MMA this thread issued has completed
+    mbar_wait_drain(mma_all, 0);
   }
   tc_fence_before();
   __syncthreads();
@@ -849,7 +875,6 @@ __global__ void __launch_bounds__(128, 1)
     tmem_dealloc(tmem, tcols);
   }
 }
-
 
 // ----------------------------------------------------------------------------------- host
 static int km_stages(const Layout& L, int Np) {
@@ -951,7 +976,7 @@ sparsepr_status launch_rowqf_tc(const Layout& L, int which, const void* X, cudaS
   if (!make_tmap_bf16(&mX, X, (long long)L.BH * L.N, D, kKmTile) ||
       !make_tmap_bf16(&mG, gbase, 3LL * L.BH * D, D, D))
     return SPARSEPR_ERR_CUDA;
-  const size_t smem = (size_t)3 * D * D * 2 + (size_t)kKmTile * D * 2 + 1024 + 64;
+  const size_t smem = (size_t)3 * D * D * 2 + (size_t)2 * kKmTile * D * 2 + 1024 + 64;
   const int tpc = tiles_per_cta(L);
   const int ntiles = (L.N + kKmTile - 1) / kKmTile;
   cudaFuncSetAttribute(rowqf_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -42,14 +42,15 @@ constexpr int kJacobiSweeps = 30;
 // Schur rotation and the round-robin ordering).  A round applies d/2 disjoint rotations, chosen
 // by the circle method so that every (p, q) pair meets once per sweep; sweeps run until the
 // off-diagonal Frobenius norm is below 1e-13 of the matrix's, or kJacobiSweeps.  On return S is
-// diagonal up to that tolerance (the eigenvalues) and V (d x d, shared or global memory,
-// initialised here to I) holds the eigenvectors as columns.
-static __device__ __noinline__ void jacobi_eig(double* S, double* V, int d) {
+// diagonal up to that tolerance (the eigenvalues) and Vt (d x d, shared or global memory,
+// initialised here to I) holds the eigenvectors as ROWS: row p is the eigenvector of S[p][p].
+// Rows, so that a rotation of the pair (p, q) reads and writes two contiguous rows.
+static __device__ __noinline__ void jacobi_eig(double* S, double* Vt, int d) {
   const int tid = threadIdx.x, nt = blockDim.x, half = d / 2;
   __shared__ double rc[64], rs[64];
   __shared__ int rp[64], rq[64];
   __shared__ double red2[2][32];
-  for (int e = tid; e < d * d; e += nt) V[e] = (e / d == e % d) ? 1.0 : 0.0;
+  for (int e = tid; e < d * d; e += nt) Vt[e] = (e / d == e % d) ? 1.0 : 0.0;
   __syncthreads();
   for (int sweep = 0; sweep < kJacobiSweeps; ++sweep) {
     double off = 0.0, tot = 0.0;
@@ -97,22 +98,24 @@ static __device__ __noinline__ void jacobi_eig(double* S, double* V, int d) {
         rs[k] = sn;
       }
       __syncthreads();
-      for (int e = tid; e < half * d; e += nt) {  // S <- S J (columns p, q of every row)
-        const int k = e / d, i = e % d, p = rp[k], q = rq[k];
+      // S <- S J (columns p, q of every row); consecutive threads take different pairs of the
+      // same row, so their shared-memory words fall in different banks
+      for (int e = tid; e < half * d; e += nt) {
+        const int k = e % half, i = e / half, p = rp[k], q = rq[k];
         const double c = rc[k], sn = rs[k], x = S[i * d + p], y = S[i * d + q];
         S[i * d + p] = c * x - sn * y;
         S[i * d + q] = sn * x + c * y;
       }
       __syncthreads();
-      for (int e = tid; e < half * d; e += nt) {  // S <- J^T S (rows p, q), V <- V J
+      for (int e = tid; e < half * d; e += nt) {  // S <- J^T S (rows p, q), V <- V J (rows of Vt)
         const int k = e / d, j = e % d, p = rp[k], q = rq[k];
         const double c = rc[k], sn = rs[k];
         const double x = S[p * d + j], y = S[q * d + j];
         S[p * d + j] = c * x - sn * y;
         S[q * d + j] = sn * x + c * y;
-        const double u = V[j * d + p], v = V[j * d + q];
-        V[j * d + p] = c * u - sn * v;
-        V[j * d + q] = sn * u + c * v;
+        const double u = Vt[p * d + j], v = Vt[q * d + j];
+        Vt[p * d + j] = c * u - sn * v;
+        Vt[q * d + j] = sn * u + c * v;
       }
       __syncthreads();
     }
