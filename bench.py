@@ -260,6 +260,27 @@ def km_rooflines(w, asg_ms, upd_ms, pk):
     return out
 
 
+def km_loop_roofline(w, loop_ms, k_iters, pk):
+    """The key k-means of a mid-size call as one launch (every Lloyd iteration; the keys stay in
+    shared memory, read from HBM once).  Its time is set by the per-iteration chain (scoring,
+    fp64 re-decision, group sums, two head barriers, the centroid step), not by a throughput
+    roofline: reported per iteration, with the tensor-core flops of the scoring against the bf16
+    peak for scale."""
+    units = w.B * w.H * w.N
+    cp = (w.n_kgroups + 15) // 16 * 16
+    it = max(k_iters) if k_iters else 0
+    fl = units * KM_W_TERMS * 2 * cp * w.d * it
+    tpk = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    s = loop_ms * 1e-3
+    return {"loop": {"bound": "latency", "ms": loop_ms, "iterations": it,
+                     "ms_per_iteration": loop_ms / it if it else None,
+                     "tensor": {"achieved": fl / s / 1e12 if s > 0 else None, "peak": tpk, "unit": "TFLOP/s",
+                                "frac": fl / s / 1e12 / tpk if s > 0 else None},
+                     "hbm_bytes": units * 2 * w.d,
+                     "algorithmic": f"{units} keys read once ({units * 2 * w.d} bytes); {it} iterations of "
+                                    f"{2 * KM_W_TERMS} C_p d flops per key on the tensor cores"}}
+
+
 def attention_flops(w, sparse_pairs):
     """Algorithmic flops of one attention launch: 4 d per executed query-key pair, counting the
     block-sparse pairs of every row and the probe rows' dense pairs (P N per head), which the
@@ -428,8 +449,8 @@ def run_ours(args, w, world, rank, local):
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     # the first key k-means assignment and update launches of each timed call (tensor-core path)
     km_ev = {kid: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(args.steps)] for kid in (1, 2)}
-    for a, b in kev + km_ev[1] + km_ev[2]:  # torch creates the CUDA event on first record
+                   for _ in range(args.steps)] for kid in (1, 2, 3)}
+    for a, b in kev + km_ev[1] + km_ev[2] + km_ev[3]:  # torch creates the CUDA event on first record
         a.record(stream)
         b.record(stream)
     if world > 1:
@@ -440,7 +461,7 @@ def run_ours(args, w, world, rank, local):
     for i in range(args.steps):
         flush.zero_()                         # L2 flush between timed steps, outside the events
         op.set_kernel_events(*kev[i])
-        for kid in (1, 2):
+        for kid in (1, 2, 3):
             op.set_kernel_events(*km_ev[kid][i], kernel=kid)
         ev[i][0].record(stream)
         step()
@@ -451,18 +472,22 @@ def run_ours(args, w, world, rank, local):
     launches = S.launch_count() - launches0
     clk = clocks.stop()
     op.set_kernel_events(None, None)
-    for kid in (1, 2):
+    for kid in (1, 2, 3):
         op.set_kernel_events(None, None, kernel=kid)
     step_ms = [a.elapsed_time(b) for a, b in ev]
     kern_ms = [a.elapsed_time(b) for a, b in kev]
-    # the k-means hooks bracket the tensor-core path only: bf16 inputs with at most 256 (padded)
-    # key groups; above that the key k-means runs on the CUDA cores and the events stay unset
-    tc_km = wl.dtype == configs.BF16 and (wl.n_kgroups + 15) // 16 * 16 <= 256
+    # the k-means hooks bracket the first assignment and update of the per-iteration tensor-core
+    # path (bf16 inputs, at most 256 padded key groups; above that the key k-means runs on the
+    # CUDA cores and the events stay unset), or, when the whole key loop runs in one launch, that
+    # launch
+    km_loop = int(op.query(S.Q_KM_PATH)[0]) == 1
+    tc_km = wl.dtype == configs.BF16 and (wl.n_kgroups + 15) // 16 * 16 <= 256 and not km_loop
     asg_ms = statistics.mean(a.elapsed_time(b) for a, b in km_ev[1]) if tc_km else 0.0
     upd_ms = statistics.mean(a.elapsed_time(b) for a, b in km_ev[2]) if tc_km else 0.0
+    loop_ms = statistics.mean(a.elapsed_time(b) for a, b in km_ev[3]) if km_loop else 0.0
     ms = statistics.mean(step_ms)
     kms = statistics.mean(kern_ms)
-    ms_max, kms_max, asg_ms, upd_ms = max_over_ranks([ms, kms, asg_ms, upd_ms], world, dev)
+    ms_max, kms_max, asg_ms, upd_ms, loop_ms = max_over_ranks([ms, kms, asg_ms, upd_ms, loop_ms], world, dev)
     # attention roofline per rank: this rank's launch, the slowest rank's time
     kflops = attention_flops(wl, pairs)
     kflops_min, = [-x for x in max_over_ranks([-kflops], world, dev)]
@@ -525,7 +550,8 @@ def run_ours(args, w, world, rank, local):
                          "peak_burst": burst, "frac_of_burst": achieved / burst,
                          "algorithmic": f"4*d*(executed sparse pairs + P*N*heads) = {kflops:.4g} flop per launch "
                                         f"(rank 0; smallest over ranks {kflops_min:.4g})"},
-            "roofline_kmeans": km_rooflines(wl, asg_ms, upd_ms, pk) if tc_km else None,
+            "roofline_kmeans": (km_rooflines(wl, asg_ms, upd_ms, pk) if tc_km else
+                                km_loop_roofline(wl, loop_ms, part_stats["k_iters"], pk) if km_loop else None),
             "e2e": {"value": job_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
                     "h2d_bytes_per_step": 3 * Q.numel() * elt, "d2h_bytes_per_step": O.numel() * O.element_size(),
                     "ms_per_step": e2e_ms},

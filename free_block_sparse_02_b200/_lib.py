@@ -23,7 +23,9 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "CU
           4: "workspace", 5: "numeric", 6: "timeout", 7: "call out of order"}
 
 Q_KLABELS, Q_QLABELS, Q_ROUTE, Q_PROBES, Q_PROBE_W, Q_FIT, Q_KCENT, Q_QCENT, Q_OSP, Q_ODENSE, \
-    Q_STATS, Q_KOBJ, Q_QOBJ = range(1, 14)
+    Q_STATS, Q_KOBJ, Q_QOBJ, Q_KM_PATH = range(1, 15)
+# kernels a pair of events can bracket (SPARSEPR_KERNEL_* in the C header)
+KERNEL_BLOCK_SPARSE, KERNEL_KMEANS_ASSIGN, KERNEL_KMEANS_UPDATE, KERNEL_KMEANS_LOOP = range(4)
 
 
 class SparsePRError(RuntimeError):
@@ -77,6 +79,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sparsepr_set_kernel_events": (i32, [vp, i32, vp, vp]),
         "sparsepr_launch_count": (ctypes.c_int64, []),
         "sparsepr_set_wait_limit": (i32, [vp, i32, ctypes.c_int64]),
+        "sparsepr_set_kmeans_path": (i32, [vp, i32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -194,7 +197,7 @@ class SparsePR:
     def set_kernel_events(self, start: "torch.cuda.Event", stop: "torch.cuda.Event", kernel: int = 0):
         """Bracket one kernel launch with two (already created) CUDA events: kernel 0 = the
         block-sparse attention, 1 = the first key k-means assignment, 2 = the first key k-means
-        update (SPARSEPR_KERNEL_* in the C header)."""
+        update, 3 = the whole key k-means loop when it runs in one launch (KERNEL_*)."""
         h0 = ctypes.c_void_p(start.cuda_event) if start is not None else None
         h1 = ctypes.c_void_p(stop.cuda_event) if stop is not None else None
         _check(self.lib.sparsepr_set_kernel_events(self.handle, int(kernel), h0, h1), "sparsepr_set_kernel_events")
@@ -203,6 +206,11 @@ class SparsePR:
         """Test hook of the timeout path: the given kernel's bounded device-side waits give up
         after `cycles` SM cycles (0 restores the default of about 1 s)."""
         _check(self.lib.sparsepr_set_wait_limit(self.handle, int(kernel), int(cycles)), "sparsepr_set_wait_limit")
+
+    def set_kmeans_path(self, mode: int):
+        """Test hook of the k-means paths: 1 launches the steps of every Lloyd iteration
+        separately even where the whole loop fits one launch; 0 restores the automatic choice."""
+        _check(self.lib.sparsepr_set_kmeans_path(self.handle, int(mode)), "sparsepr_set_kmeans_path")
 
     def sync(self):
         _check(self.lib.sparsepr_sync(self.handle), "sparsepr_sync")
@@ -218,6 +226,7 @@ class SparsePR:
             Q_KCENT: (np.float64, (BH, c.n_kgroups, c.d)), Q_QCENT: (np.float64, (BH, c.n_qgroups, c.n_kgroups)),
             Q_OSP: (np.float32, (BH, c.N, c.d)), Q_ODENSE: (np.float32, (BH, c.P, c.d)),
             Q_KOBJ: (np.float64, (BH, c.km_iters)), Q_QOBJ: (np.float64, (BH, c.km_iters)),
+            Q_KM_PATH: (np.int32, (2,)),
         }[what]
         out = np.empty(spec[1], dtype=spec[0])
         _check(self.lib.sparsepr_plan_query(self.handle, what, out.ctypes.data_as(ctypes.c_void_p), out.nbytes),

@@ -19,6 +19,7 @@ constexpr int kMaxProbes = 4096;
 constexpr int kSortChunk = 4096;   // tokens per chunk of the parallel stable group sort
 constexpr int kKmChunkGroups = 256;  // groups per launch of the tensor-core k-means assignment
 constexpr int kGramChunk = 4096;     // keys per partial Gram of the key-response rank projection
+constexpr int kKmLoopMaxCtas = 160;  // CTAs of one whole-loop k-means launch at most (>= the SMs)
 
 // Device status word values (a subset of sparsepr_status).
 constexpr int kDevOk = 0;
@@ -45,6 +46,10 @@ struct Layout {
                               // many cycles (test hook of the timeout path); 0: the default
   int key_rank;         // 0 < r < d: the key k-means metric restricted to the r leading
                         // directions of the key responses (r_K); else the full metric
+  int km_steps;         // 1: k-means one launch per step of every iteration even where the
+                        // whole loop fits one launch (test hook); 0: the faster path
+  long long km_wait_limit;  // > 0: the whole-loop k-means head barriers give up after this many
+                            // cycles (test hook of its timeout path); 0: the default
 
   // status + per-head statistics
   int* status;                    // [1]
@@ -64,7 +69,7 @@ struct Layout {
   double* kr_T;                   // [BH, d, d]
 
   // k-means shared scratch
-  int* init_ids;                  // [BH, max(Ck, Cq)]
+  int* init_ids;                  // [BH, Ck + Cq] initial points: keys, then queries
   int* fy;                        // [BH, N] Fisher-Yates slots
   int* iters_run;                 // [BH, 2] iterations for keys / queries (run-time state)
   int* stop_at;                   // [BH, 2] iteration at which the loop stopped
@@ -117,6 +122,14 @@ struct Layout {
   // than kKmChunkGroups groups): {best bits, second bits, best group, 0}; null when unused
   int4* ktop;                     // [BH, N]
   int4* qtop;                     // [BH, N]
+  // whole-loop k-means (mid-size calls: every Lloyd iteration of a side in one launch, G CTAs
+  // per head): each CTA's partial group sums, counts and objective, the head barrier counters
+  // and the abort flag; null when no side qualifies
+  int klp_G;                      // CTAs per head the partial arrays hold
+  double* klp_sum;                // [BH, klp_G, max C, d]
+  int* klp_cnt;                   // [BH, klp_G, max C]
+  double* klp_J;                  // [BH, klp_G]
+  unsigned* klp_bar;              // [BH + 1]: head counters, then the abort flag
 
   // points of the tensor-core assignment whose two best scores were within the rounding bound,
   // re-decided in fp64: CTA c of the assignment grid appends to its own segment starting at

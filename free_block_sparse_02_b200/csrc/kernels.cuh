@@ -13,7 +13,7 @@ inline int attn_tile_m(const Layout& L) { return L.dtype == SPARSEPR_BF16 ? kAtt
 
 // Optional events recorded around single launches (ids: SPARSEPR_KERNEL_*).
 struct KernelEvents {
-  static constexpr int kCount = 3;
+  static constexpr int kCount = 4;
   cudaEvent_t start[kCount] = {};
   cudaEvent_t stop[kCount] = {};
 };
@@ -35,6 +35,12 @@ int km_tc_grid(const Layout& L, bool keys);
 // re-decisions, group sums and counts (both kernels over the same G tile ranges).
 sparsepr_status launch_kmeans_iteration_tc(const Layout& L, bool keys, const void* X, int it, int G,
                                            cudaStream_t st, const KernelEvents* ev = nullptr);
+// Whole-loop k-means (kmeans_loop.cu): CTAs per head and resident tiles per CTA when `ctas`
+// CTAs can be co-resident, 0 when the side does not qualify; whether the plan's workspace and
+// the device allow it; the launch (every Lloyd iteration of one side, the stop test included).
+int km_loop_ctas_per_head(int BH, int N, int d, int dtype, int C, int Ck, bool keys, int ctas, int* cap_out);
+bool km_loop_supported(const Layout& L, bool keys);
+sparsepr_status launch_kmeans_loop(const Layout& L, bool keys, const void* X, int iters, cudaStream_t st);
 sparsepr_status launch_rowqf_tc(const Layout& L, int which, const void* X, cudaStream_t st);
 // M <- its rank-r_K restriction to the leading key-response directions (key_rank in (0, d)).
 sparsepr_status launch_key_rank(const Layout& L, const void* K, cudaStream_t st);

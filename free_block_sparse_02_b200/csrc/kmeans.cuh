@@ -5,6 +5,45 @@
 
 namespace sparsepr {
 
+// TMEM columns to allocate for n accumulator columns: a power of two, at least 32.
+__host__ __device__ inline int km_tc_tmem_cols(int n) {
+  int c = 32;
+  while (c < n) c <<= 1;
+  return c;
+}
+
+// A load of data that other CTAs of the same launch may have rewritten (kCg: served by L2, never
+// by a stale L1 line), or a plain load.
+template <bool kCg, typename T>
+__device__ __forceinline__ T ld_w(const T* p) {
+  if constexpr (kCg) return __ldcg(p);
+  else return *p;
+}
+
+// x = hi + mid + lo in bf16 (each term the bf16 rounding of what the previous ones left),
+// written at index i of three planes `plane` elements apart.
+__device__ __forceinline__ void split3(double x, __nv_bfloat16* base, size_t plane, size_t i) {
+  const __nv_bfloat16 h = __double2bfloat16(x);
+  const double r1 = x - (double)__bfloat162float(h);
+  const __nv_bfloat16 m = __double2bfloat16(r1);
+  const double r2 = r1 - (double)__bfloat162float(m);
+  base[i] = h;
+  base[plane + i] = m;
+  base[2 * plane + i] = __double2bfloat16(r2);
+}
+
+__device__ __forceinline__ bool km_should_stop(const double* J, int it, int iters, float tol) {
+  if (it >= iters) return true;
+  if (it >= 2 && tol >= 0.f) {
+    const double Jp = J[it - 2], Jc = J[it - 1];
+    return Jp - Jc <= (double)tol * Jp;
+  }
+  return false;
+}
+
+// Exact fp64 value of a bf16 given by its 16 bits (through its exact fp32 value).
+__device__ __forceinline__ double bf16_bits_to_f64(uint32_t b) { return (double)__uint_as_float(b << 16); }
+
 // Sum over the 32 lanes of each of 32 values: afterwards lane l holds the total of v[l]
 // (recursive halving: 16 + 8 + 4 + 2 + 1 shuffles instead of 32 full warp sums).
 __device__ __forceinline__ double warp_transpose_sum32(double (&v)[32]) {
@@ -22,11 +61,6 @@ __device__ __forceinline__ double warp_transpose_sum32(double (&v)[32]) {
   return v[0];
 }
 
-// fp64 score of every group for one point (one warp), lowest index on exact ties; x staged in
-// xs (fp64, shared memory).  Lanes run over the dimensions, so every row of W and Gc is read
-// coalesced.  Queries need the exact scale 1/rms: ms = x^T Gc x, each lane summing over its
-// columns and one warp sum at the end.  Group dots are formed 32 groups at a time and
-// transposed across the lanes (lane l gets group 32 c + l), then the lowest score wins.
 // The exact query scale 1/rms = 1/sqrt(x^T Gc x + 1e-12) (Gc in global or shared memory), one
 // warp: each lane sums over its columns, one warp sum at the end.
 __device__ __forceinline__ double query_scale_fp64(const double* Gc, const double* xs, const double (&xl)[4], int D) {
@@ -45,6 +79,7 @@ __device__ __forceinline__ double query_scale_fp64(const double* Gc, const doubl
 
 // fp64 argmin over a short candidate list (ascending group ids; the lowest id wins exact ties),
 // one warp; `scale` is 1 for keys.
+template <bool kCg = false>
 __device__ __forceinline__ void redecide_candidates(const double* xs, int D, const double* W64, const double* B64,
                                                     double scale, const int* cand, int ncand, int& best_out,
                                                     double& bestv_out) {
@@ -56,8 +91,8 @@ __device__ __forceinline__ void redecide_candidates(const double* xs, int D, con
     double part = 0.0;
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-      if (lane + 32 * k < D) part += W64[(size_t)j * D + lane + 32 * k] * xs[lane + 32 * k];
-    const double sc = B64[j] - 2.0 * scale * warp_sum(part);
+      if (lane + 32 * k < D) part += ld_w<kCg>(W64 + (size_t)j * D + lane + 32 * k) * xs[lane + 32 * k];
+    const double sc = ld_w<kCg>(B64 + j) - 2.0 * scale * warp_sum(part);
     if (sc < bv) {
       bv = sc;
       bj = j;
@@ -67,7 +102,12 @@ __device__ __forceinline__ void redecide_candidates(const double* xs, int D, con
   bestv_out = bv;
 }
 
-template <bool kKeys>
+// fp64 score of every group for one point (one warp), lowest index on exact ties; x staged in
+// xs (fp64, shared memory).  Lanes run over the dimensions, so every row of W and Gc is read
+// coalesced.  Queries need the exact scale 1/rms: ms = x^T Gc x, each lane summing over its
+// columns and one warp sum at the end.  Group dots are formed 32 groups at a time and
+// transposed across the lanes (lane l gets group 32 c + l), then the lowest score wins.
+template <bool kKeys, bool kCg = false>
 __device__ void redecide_fp64(const Layout& L, int bh, const double* xs, int D, int C, const double* W64,
                               const double* B64, int& best_out, double& bestv_out, const double* Gc_in = nullptr) {
   const int lane = threadIdx.x & 31;
@@ -100,13 +140,13 @@ __device__ void redecide_fp64(const Layout& L, int bh, const double* xs, int D, 
         const double* w = W64 + (size_t)(j0 + g) * D;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          if (lane + 32 * k < D) part[g] += w[lane + 32 * k] * xl[k];
+          if (lane + 32 * k < D) part[g] += ld_w<kCg>(w + lane + 32 * k) * xl[k];
       }
     }
     const double dot = warp_transpose_sum32(part);  // group j0 + lane
     const int j = j0 + lane;
     if (j < C) {
-      const double sc = B64[j] - 2.0 * scale * dot;
+      const double sc = ld_w<kCg>(B64 + j) - 2.0 * scale * dot;
       if (sc < bv) {  // ascending j per lane: strict < keeps the lower index
         bv = sc;
         bj = j;

@@ -58,11 +58,6 @@ constexpr int kKmUpdItemRows = 64;   // rows of one accumulation item: a group's
                                      // pieces of at most this many rows, summed by different warps
 __host__ __device__ constexpr int km_upd_max_items(int C) { return kKmUpdChunk / kKmUpdItemRows + C; }
 
-__host__ __device__ inline int km_tc_tmem_cols(int n) {
-  int c = 32;
-  while (c < n) c <<= 1;
-  return c;
-}
 
 // Shared memory of the assignment kernel: the kKmWTerms-term W, `stages` X tiles, barriers,
 // per-warp bias copies.
@@ -448,9 +443,6 @@ __global__ void __launch_bounds__(kKmThreads, 1)
     tmem_dealloc(tmem, tcols);
   }
 }
-
-// Exact fp64 value of a bf16 given by its 16 bits (through its exact fp32 value).
-__device__ __forceinline__ double bf16_bits_to_f64(uint32_t b) { return (double)__uint_as_float(b << 16); }
 
 // fp64 re-decision of the points the assignment listed for CTA range c, run by the update
 // kernel's CTA c before it reads the labels (the ranges of the two kernels are the same): the

@@ -180,14 +180,16 @@ __device__ __forceinline__ uint64_t splitmix64_next(uint64_t& state) {
   return z ^ (z >> 31);
 }
 
-// One thread per head.  The slots touched by C swaps live in a shared-memory hash map
-// (slot -> value), so the identity array of N slots is never written.
-__global__ void km_draw_kernel(Layout L, int stage, int C) {
+// One thread per (head, side): block (bh, stage) draws the key (stage 0) or query (stage 1)
+// initial points of head bh.  The draws depend on the seed alone, so both sides run in one
+// launch.  The slots touched by C swaps live in a shared-memory hash map (slot -> value), so the
+// identity array of N slots is never written.
+__global__ void km_draw_kernel(Layout L) {
   pdl_entry();
   constexpr int kTab = 4096;  // >= 2 * 2 * kMaxGroups
   __shared__ int keys[kTab];
   __shared__ int vals[kTab];
-  const int bh = blockIdx.x;
+  const int bh = blockIdx.x, stage = blockIdx.y, C = stage == 0 ? L.Ck : L.Cq;
   for (int i = threadIdx.x; i < kTab; i += blockDim.x) keys[i] = -1;
   __syncthreads();
   if (threadIdx.x != 0) return;
@@ -205,7 +207,7 @@ __global__ void km_draw_kernel(Layout L, int stage, int C) {
   };
   uint64_t state = L.seed + 2ULL * (uint64_t)bh + (uint64_t)stage;
   const uint64_t n = (uint64_t)L.N;
-  int* out = L.init_ids + (size_t)bh * max(L.Ck, L.Cq);
+  int* out = L.init_ids + (size_t)bh * (L.Ck + L.Cq) + (stage == 0 ? 0 : L.Ck);
   for (int i = 0; i < C; ++i) {
     const uint64_t r = splitmix64_next(state);
     const int j = i + (int)(r % (n - (uint64_t)i));
@@ -223,7 +225,7 @@ __global__ void kcent_init_kernel(Layout L, const T* __restrict__ K) {
   pdl_entry();
   const int bh = blockIdx.x, j = blockIdx.y, a = threadIdx.x;
   if (a >= L.d) return;
-  const int t = L.init_ids[(size_t)bh * max(L.Ck, L.Cq) + j];
+  const int t = L.init_ids[(size_t)bh * (L.Ck + L.Cq) + j];
   L.kcent[((size_t)bh * L.Ck + j) * L.d + a] = (double)to_f32(K[((size_t)bh * L.N + t) * L.d + a]);
 }
 
@@ -234,7 +236,7 @@ __global__ void __launch_bounds__(128) qcent_init_kernel(Layout L, const T* __re
   __shared__ double qv[128];
   __shared__ double red[4];
   const int bh = blockIdx.x, g = blockIdx.y, d = L.d, Ck = L.Ck, tid = threadIdx.x;
-  const int t = L.init_ids[(size_t)bh * max(L.Ck, L.Cq) + g];
+  const int t = L.init_ids[(size_t)bh * (L.Ck + L.Cq) + L.Ck + g];
   if (L.semantic) {  // raw queries: the drawn query itself is the centroid
     if (tid < d) L.qU64[((size_t)bh * L.Cq + g) * d + tid] = (double)to_f32(Q[((size_t)bh * L.N + t) * d + tid]);
     return;
@@ -277,27 +279,6 @@ __global__ void km_reset_kernel(Layout L, int which, int iters) {
 //   keys:    c_j (key space), W_j = M c_j, bias_j = c_j^T M c_j
 //   queries: nu_g (response space), W_g = nu_g, bias_g = ||nu_g||^2
 // ------------------------------------------------------------------------------------------
-// x = hi + mid + lo in bf16 (each term the bf16 rounding of what the previous ones left),
-// written at index i of three planes `plane` elements apart.
-__device__ __forceinline__ void split3(double x, __nv_bfloat16* base, size_t plane, size_t i) {
-  const __nv_bfloat16 h = __double2bfloat16(x);
-  const double r1 = x - (double)__bfloat162float(h);
-  const __nv_bfloat16 m = __double2bfloat16(r1);
-  const double r2 = r1 - (double)__bfloat162float(m);
-  base[i] = h;
-  base[plane + i] = m;
-  base[2 * plane + i] = __double2bfloat16(r2);
-}
-
-__device__ __forceinline__ bool km_should_stop(const double* J, int it, int iters, float tol) {
-  if (it >= iters) return true;
-  if (it >= 2 && tol >= 0.f) {
-    const double Jp = J[it - 2], Jc = J[it - 1];
-    return Jp - Jc <= (double)tol * Jp;
-  }
-  return false;
-}
-
 constexpr int kPrepGroups = 8;  // groups per block of the centroid-update kernels
 
 // Sums of kPrepGroups values per thread over the block (128 threads): out[g] for g < n.
@@ -1233,7 +1214,7 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
     launch(rowqf_simt_kernel<T>, dim3((L.N + 63) / 64, L.BH), 256, qf_smem, st, L, K, 0);
   }
   if (!warm) {
-    launch(km_draw_kernel, L.BH, 128, 0, st, L, 0, L.Ck);
+    launch(km_draw_kernel, dim3(L.BH, 2), 128, 0, st, L);  // both sides' initial points
     launch(kcent_init_kernel<T>, dim3(L.BH, L.Ck), 128, 0, st, L, K);
   }
   SPR_LAUNCH_CHECK();
@@ -1249,14 +1230,22 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
   cudaFuncSetAttribute(kmeans_assign_kernel<T, QueryFeat>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asg_smem);
   const size_t kprep_smem = (size_t)std::min(d, kPrepRows) * d * sizeof(double);
   cudaFuncSetAttribute(kprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kprep_smem);
-  for (int it = 0; it <= iters; ++it) {
-    launch(kprep_kernel, dim3(L.BH, (L.Ck + kPrepGroups - 1) / kPrepGroups), 128, kprep_smem, st, L, it, iters);
-    if (it < iters) {
-      if (tc_keys) {
-        const sparsepr_status s = launch_kmeans_iteration_tc(L, true, K, it, Gk, st, it == 0 ? &ev : nullptr);
-        if (s != SPARSEPR_OK) return s;
-      } else {
-        launch(kmeans_assign_kernel<T, KeyFeat>, dim3(nblk, L.BH), 256, asg_smem, st, L, K, it);
+  if (km_loop_supported(L, true)) {  // mid-size calls: the whole loop in one launch
+    const cudaEvent_t e0 = ev.start[SPARSEPR_KERNEL_KMEANS_LOOP], e1 = ev.stop[SPARSEPR_KERNEL_KMEANS_LOOP];
+    if (e0) cudaEventRecord(e0, st);
+    const sparsepr_status s = launch_kmeans_loop(L, true, K, iters, st);
+    if (s != SPARSEPR_OK) return s;
+    if (e1) cudaEventRecord(e1, st);
+  } else {
+    for (int it = 0; it <= iters; ++it) {
+      launch(kprep_kernel, dim3(L.BH, (L.Ck + kPrepGroups - 1) / kPrepGroups), 128, kprep_smem, st, L, it, iters);
+      if (it < iters) {
+        if (tc_keys) {
+          const sparsepr_status s = launch_kmeans_iteration_tc(L, true, K, it, Gk, st, it == 0 ? &ev : nullptr);
+          if (s != SPARSEPR_OK) return s;
+        } else {
+          launch(kmeans_assign_kernel<T, KeyFeat>, dim3(nblk, L.BH), 256, asg_smem, st, L, K, it);
+        }
       }
     }
   }
@@ -1271,21 +1260,25 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
     launch(rowqf_simt_kernel<T>, dim3((L.N + 63) / 64, L.BH), 256, qf_smem, st, L, Q, 1);
   }
   if (!warm) {
-    launch(km_draw_kernel, L.BH, 128, 0, st, L, 1, L.Cq);
     launch(qcent_init_kernel<T>, dim3(L.BH, L.Cq), 128, 0, st, L, Q);
   }
   launch(km_reset_kernel, L.BH, 128, 0, st, L, 1, iters);
   SPR_LAUNCH_CHECK();
   const size_t qprep_smem = ((size_t)kPrepGroups * L.Ck + (size_t)std::min(L.Ck, kPrepRows) * d) * sizeof(double);
   cudaFuncSetAttribute(qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qprep_smem);
-  for (int it = 0; it <= iters; ++it) {
-    launch(qprep_kernel, dim3(L.BH, (L.Cq + kPrepGroups - 1) / kPrepGroups), 128, qprep_smem, st, L, it, iters);
-    if (it < iters) {
-      if (tc_queries) {
-        const sparsepr_status s = launch_kmeans_iteration_tc(L, false, Q, it, Gq, st);
-        if (s != SPARSEPR_OK) return s;
-      } else {
-        launch(kmeans_assign_kernel<T, QueryFeat>, dim3(nblk, L.BH), 256, asg_smem, st, L, Q, it);
+  if (km_loop_supported(L, false)) {
+    const sparsepr_status s = launch_kmeans_loop(L, false, Q, iters, st);
+    if (s != SPARSEPR_OK) return s;
+  } else {
+    for (int it = 0; it <= iters; ++it) {
+      launch(qprep_kernel, dim3(L.BH, (L.Cq + kPrepGroups - 1) / kPrepGroups), 128, qprep_smem, st, L, it, iters);
+      if (it < iters) {
+        if (tc_queries) {
+          const sparsepr_status s = launch_kmeans_iteration_tc(L, false, Q, it, Gq, st);
+          if (s != SPARSEPR_OK) return s;
+        } else {
+          launch(kmeans_assign_kernel<T, QueryFeat>, dim3(nblk, L.BH), 256, asg_smem, st, L, Q, it);
+        }
       }
     }
   }

@@ -108,7 +108,7 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
     take(L.kr_V, BH * d * d * 8);
     take(L.kr_T, BH * d * d * 8);
   }
-  take(L.init_ids, BH * std::max(Ck, Cq) * 4);
+  take(L.init_ids, BH * (Ck + Cq) * 4);
   take(L.fy, 4);  // unused: the draw keeps its slots in shared memory
   take(L.iters_run, BH * 2 * 4);
   take(L.stop_at, BH * 2 * 4);
@@ -148,6 +148,21 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   take(L.knorm, BH * N * 4);
   if (L.Ckp > kKmChunkGroups) take(L.ktop, BH * N * 16);
   if (L.Cqp > kKmChunkGroups) take(L.qtop, BH * N * 16);
+  {  // whole-loop k-means: partials for the most CTAs per head either side could use
+    const int Gk = km_loop_ctas_per_head(c.B * c.H, c.N, c.d, c.dtype, c.n_kgroups, c.n_kgroups, true,
+                                         kKmLoopMaxCtas, nullptr);
+    const int Gq = km_loop_ctas_per_head(c.B * c.H, c.N, c.d, c.dtype, c.n_qgroups, c.n_kgroups, false,
+                                         kKmLoopMaxCtas, nullptr);
+    const int G = std::max(Gk, Gq);
+    if (G > 0) {
+      L.klp_G = G;
+      const size_t Cm = std::max(Gk > 0 ? Ck : 0, Gq > 0 ? Cq : 0);
+      take(L.klp_sum, BH * G * Cm * d * 8);
+      take(L.klp_cnt, BH * G * Cm * 4);
+      take(L.klp_J, BH * G * 8);
+      take(L.klp_bar, (BH + 1) * 4);
+    }
+  }
   const size_t km_tiles = BH * (size_t)((N + 127) / 128);
   take(L.rlist, km_tiles * 128 * 16);
   take(L.rcnt, km_tiles * 4);
@@ -350,6 +365,12 @@ sparsepr_status sparsepr_plan_query(const sparsepr_plan_t* p, int32_t what, void
     case SPARSEPR_Q_QCENT: return copy_out(dst, bytes, L.qcent, BH * L.Cq * L.Ck);
     case SPARSEPR_Q_ODENSE: return copy_out(dst, bytes, L.Odense, BH * L.P * d);
     case SPARSEPR_Q_STATS: return copy_out(dst, bytes, L.stats, BH);
+    case SPARSEPR_Q_KM_PATH: {
+      const int32_t path[2] = {km_loop_supported(L, true) ? 1 : 0, km_loop_supported(L, false) ? 1 : 0};
+      if (bytes != sizeof(path)) return SPARSEPR_ERR_INVALID_ARG;
+      memcpy(dst, path, sizeof(path));
+      return SPARSEPR_OK;
+    }
     case SPARSEPR_Q_OSP: {
       if (bytes != BH * N * d * 4) return SPARSEPR_ERR_INVALID_ARG;
       std::vector<float> tmp(BH * N * d);
@@ -396,10 +417,17 @@ sparsepr_status sparsepr_set_kernel_events(sparsepr_plan_t* p, int32_t kernel, v
 
 int64_t sparsepr_launch_count(void) { return (int64_t)g_launches.load(); }
 
+sparsepr_status sparsepr_set_kmeans_path(sparsepr_plan_t* p, int32_t mode) {
+  if (!p || (mode != 0 && mode != 1)) return SPARSEPR_ERR_INVALID_ARG;
+  p->L.km_steps = mode;
+  return SPARSEPR_OK;
+}
+
 sparsepr_status sparsepr_set_wait_limit(sparsepr_plan_t* p, int32_t kernel, int64_t cycles) {
   if (!p || cycles < 0) return SPARSEPR_ERR_INVALID_ARG;
-  if (kernel != SPARSEPR_KERNEL_BLOCK_SPARSE) return SPARSEPR_ERR_UNSUPPORTED;
-  p->L.attn_wait_limit = (long long)cycles;
+  if (kernel == SPARSEPR_KERNEL_BLOCK_SPARSE) p->L.attn_wait_limit = (long long)cycles;
+  else if (kernel == SPARSEPR_KERNEL_KMEANS_LOOP) p->L.km_wait_limit = (long long)cycles;
+  else return SPARSEPR_ERR_UNSUPPORTED;
   return SPARSEPR_OK;
 }
 

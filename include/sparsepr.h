@@ -138,7 +138,10 @@ enum {
   SPARSEPR_Q_ODENSE = 10,   /* float  [B*H, P, d]    exact output of the probe rows            */
   SPARSEPR_Q_STATS = 11,    /* sparsepr_head_stats [B*H]                                        */
   SPARSEPR_Q_KOBJ = 12,     /* double [B*H, km_iters] key objective per iteration (0 = not run) */
-  SPARSEPR_Q_QOBJ = 13      /* double [B*H, km_iters] query objective per iteration             */
+  SPARSEPR_Q_QOBJ = 13,     /* double [B*H, km_iters] query objective per iteration             */
+  SPARSEPR_Q_KM_PATH = 14   /* int32  [2]            k-means path of the keys, then the queries:
+                             * 0 one launch per step of every iteration, 1 one launch for the
+                             * whole loop (see SPARSEPR_KERNEL_KMEANS_LOOP)                      */
 };
 
 typedef struct sparsepr_plan_s sparsepr_plan_t;
@@ -201,8 +204,18 @@ int32_t sparsepr_version(void);
  *   KMEANS_ASSIGN  the first key-group k-means assignment launch of sparsepr_plan (bf16
  *                  inputs, tensor-core path: one pass over all keys);
  *   KMEANS_UPDATE  the first key-group k-means update launch of sparsepr_plan (group sums
- *                  and counts: one pass over all keys). */
-enum { SPARSEPR_KERNEL_BLOCK_SPARSE = 0, SPARSEPR_KERNEL_KMEANS_ASSIGN = 1, SPARSEPR_KERNEL_KMEANS_UPDATE = 2 };
+ *                  and counts: one pass over all keys);
+ *   KMEANS_LOOP    the key-group k-means launch of sparsepr_plan when the whole loop runs in
+ *                  one launch (bf16 calls whose keys fit in the shared memory of the SMs,
+ *                  at most 128 groups; SPARSEPR_Q_KM_PATH tells which path ran): every
+ *                  iteration, the stop test included.  The two hooks above are then not
+ *                  recorded. */
+enum {
+  SPARSEPR_KERNEL_BLOCK_SPARSE = 0,
+  SPARSEPR_KERNEL_KMEANS_ASSIGN = 1,
+  SPARSEPR_KERNEL_KMEANS_UPDATE = 2,
+  SPARSEPR_KERNEL_KMEANS_LOOP = 3
+};
 
 /* Optional timing hook for measurement.  When set, the library records `start_event` on its
  * stream immediately before launching the named kernel and `stop_event` immediately after it,
@@ -220,12 +233,24 @@ int64_t sparsepr_launch_count(void);
  * device status word to SPARSEPR_ERR_TIMEOUT, lets the copies and tensor-core operations it
  * started finish, frees its tensor memory and returns, so the context stays usable.  This call
  * sets, for the plan's later launches of `kernel`, a limit of `cycles` SM cycles on each such
- * wait (0 restores the default).  Only SPARSEPR_KERNEL_BLOCK_SPARSE is accepted (other ids:
- * SPARSEPR_ERR_UNSUPPORTED; cycles < 0: SPARSEPR_ERR_INVALID_ARG).  With a limit of a few
- * hundred cycles the attention launch gives up, its output rows are left unwritten, and the
- * next sparsepr_sync returns SPARSEPR_ERR_TIMEOUT (and clears it); the plan, its workspace and
- * the context stay usable for the next call.  Enqueues nothing. */
+ * wait (0 restores the default).  SPARSEPR_KERNEL_BLOCK_SPARSE (the attention launch's waits)
+ * and SPARSEPR_KERNEL_KMEANS_LOOP (the barriers between the CTAs of one head in the whole-loop
+ * k-means launch) are accepted; other ids give SPARSEPR_ERR_UNSUPPORTED, cycles < 0
+ * SPARSEPR_ERR_INVALID_ARG.  With a limit of a few hundred cycles the attention launch gives
+ * up and its output rows are left unwritten; the whole-loop k-means gives up at its first head
+ * barrier and leaves every point of the side in group 0.  The next sparsepr_sync then returns
+ * SPARSEPR_ERR_TIMEOUT (and clears it); the plan, its workspace and the context stay usable for
+ * the next call.  Enqueues nothing. */
 sparsepr_status sparsepr_set_wait_limit(sparsepr_plan_t* plan, int32_t kernel, int64_t cycles);
+
+/* Test hook of the k-means paths (no counterpart in the paper).  A bf16 call with at most 128
+ * groups on a side, whose points fit in the shared memory of the SMs (mid-size calls), runs that
+ * side's whole Lloyd loop in one cooperative launch; other calls launch the steps of every
+ * iteration separately.  Both compute the same labels and centroids.  mode 1 makes the plan's
+ * later sparsepr_plan calls use the per-iteration launches everywhere (so that both paths can be
+ * checked on the same inputs); mode 0 restores the automatic choice.  Other modes:
+ * SPARSEPR_ERR_INVALID_ARG.  Enqueues nothing. */
+sparsepr_status sparsepr_set_kmeans_path(sparsepr_plan_t* plan, int32_t mode);
 
 /* Allocation-free weighted ridge fit (no counterpart in the paper: an interface for callers
  * that cannot allocate device memory).  Some callers cannot call cudaMalloc or hand this

@@ -10,6 +10,10 @@
    give up, drain its copies, free its tensor memory and return, sparsepr_sync must return
    SPARSEPR_ERR_TIMEOUT, and, with the default limit restored, the next call on the same plan
    must be clean and correct.
+3. The same for the barriers between the CTAs of one head in the whole-loop k-means launch:
+   with a limit of one cycle the first CTA to reach a barrier gives up before the other fifteen
+   arrive, every CTA of the launch leaves (the abort flag), every point is left in group 0, and
+   the call reports SPARSEPR_ERR_TIMEOUT; the next call with the default limit is clean.
 """
 import numpy as np
 import pytest
@@ -108,4 +112,21 @@ def test_attention_wait_limit_gives_timeout_and_the_next_call_is_clean():
     assert e.value.status == TIMEOUT
     op.sync()  # cleared
     op.set_wait_limit(0)
+    _clean_call_matches_oracle(op, w, Q, K, V)
+
+
+def test_kmeans_loop_wait_limit_gives_timeout_and_the_next_call_is_clean():
+    w = _workload()  # 2 heads of 2048 points: 16 CTAs per head in the whole-loop k-means
+    Q, K, V = gen.make_qkv(w)
+    op = S.SparsePR(w)
+    assert list(op.query(S.Q_KM_PATH)) == [1, 1]
+    op.set_wait_limit(1, kernel=S.KERNEL_KMEANS_LOOP)
+    op(Q.cuda(), K.cuda(), V.cuda(), out_dtype=torch.float32)
+    torch.cuda.synchronize()  # the launches returned: no barrier was left spinning
+    with pytest.raises(S.SparsePRError) as e:
+        op.sync()
+    assert e.value.status == TIMEOUT
+    op.sync()  # cleared
+    assert not np.any(op.query(S.Q_KLABELS)) and not np.any(op.query(S.Q_QLABELS)), "aborted loops leave group 0"
+    op.set_wait_limit(0, kernel=S.KERNEL_KMEANS_LOOP)
     _clean_call_matches_oracle(op, w, Q, K, V)

@@ -24,8 +24,11 @@ def _built():
     S.load()
 
 
-def run_gpu(w, Q, K, V, out_dtype=torch.float32, **over):
+def run_gpu(w, Q, K, V, out_dtype=torch.float32, km_path=0, **over):
+    """One call through the C ABI; km_path 1 forces the per-iteration k-means launches."""
     op = S.SparsePR(w, **over)
+    if km_path:
+        op.set_kmeans_path(km_path)
     Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
     out = op(Qd, Kd, Vd, out_dtype=out_dtype)
     torch.cuda.synchronize()
@@ -292,8 +295,46 @@ def test_edge_cases(name, parity_log):
     compare_outputs(op, out, qf, kf, vf, w, *tol, log=parity_log, case=name)
 
 
+# Cases the whole-loop k-means takes (bf16, at most 128 groups, points resident in shared
+# memory), run again with the k-means forced onto one launch per step, the path of the large
+# calls: both paths must give the oracle's partition on the same inputs.
+LOOP_CASES = ["ragged-uniform", "d128-bf16", "few-groups-many-tiles", "key-rank-d128"]
+
+
+@pytest.mark.parametrize("name", LOOP_CASES)
+def test_kmeans_paths_both_match_oracle(name, parity_log):
+    e = dict(EDGE[name])
+    base = configs.workload(e.pop("base"))
+    w = configs.scaled_down(base, heads=e.pop("heads"), grid=e.pop("grid"), **e)
+    Q, K, V = gen.make_qkv(w)
+    qf, kf, vf = flat(Q), flat(K), flat(V)
+    res = O.call(qf[None], kf[None], vf[None], w)
+    labels = []
+    for path in (0, 1):
+        op, out = run_gpu(w, Q, K, V, km_path=path)
+        assert list(op.query(S.Q_KM_PATH)) == ([1, 1] if path == 0 else [0, 0])
+        compare_partition(op, res, w, qf)
+        labels.append((op.query(S.Q_KLABELS), op.query(S.Q_QLABELS)))
+        if path == 1:
+            compare_outputs(op, out, qf, kf, vf, w, 2e-2, 1e-2, log=parity_log, case=f"{name} per-iteration k-means")
+    assert all(np.array_equal(a, b) for a, b in zip(*labels)), "the two k-means paths disagree"
+
+
+def test_mid_bf16_two_heads_per_iteration_kmeans(parity_log):
+    w = configs.scaled_down(configs.workload(1), heads=2)
+    Q, K, V = gen.make_qkv(w)
+    qf, kf, vf = flat(Q), flat(K), flat(V)
+    res = O.call(qf[None], kf[None], vf[None], w)
+    op, out = run_gpu(w, Q, K, V, km_path=1)
+    assert list(op.query(S.Q_KM_PATH)) == [0, 0]
+    compare_partition(op, res, w, qf)
+    compare_outputs(op, out, qf, kf, vf, w, atol=2e-2, rel_l2=1e-2, log=parity_log,
+                    case="mid-bf16 2 heads per-iteration k-means")
+
+
+@pytest.mark.parametrize("km_path", [0, 1], ids=["auto", "per-iteration"])
 @pytest.mark.parametrize("repair", [0, 1])
-def test_semantic_partition_matches_oracle(repair, parity_log):
+def test_semantic_partition_matches_oracle(repair, km_path, parity_log):
     """The semantic baseline (k-means on the raw keys and queries), with and without the
     probe-residual correction, against the oracle's."""
     w = configs.scaled_down(configs.workload(1), heads=2, grid=(4, 16, 32))
@@ -302,9 +343,10 @@ def test_semantic_partition_matches_oracle(repair, parity_log):
     Q, K, V = gen.make_qkv(w)
     qf, kf, vf = flat(Q), flat(K), flat(V)
     res = O.call(qf[None], kf[None], vf[None], w)
-    op, out = run_gpu(w, Q, K, V)
+    op, out = run_gpu(w, Q, K, V, km_path=km_path)
     compare_partition(op, res, w, qf)
-    compare_outputs(op, out, qf, kf, vf, w, 2e-2, 1e-2, log=parity_log, case=f"semantic repair={repair}")
+    compare_outputs(op, out, qf, kf, vf, w, 2e-2, 1e-2, log=parity_log,
+                    case=f"semantic repair={repair}" + (" per-iteration k-means" if km_path else ""))
 
 
 def test_installed_oracle_partition_gives_oracle_outputs():
@@ -326,11 +368,14 @@ def test_installed_oracle_partition_gives_oracle_outputs():
     assert np.linalg.norm(got - r["O"]) / np.linalg.norm(r["O"]) <= 1e-2
 
 
-def test_streaming_warm_start_matches_oracle(parity_log):
+@pytest.mark.parametrize("km_path", [0, 1], ids=["auto", "per-iteration"])
+def test_streaming_warm_start_matches_oracle(km_path, parity_log):
     w = configs.scaled_down(configs.workload(4), heads=1, grid=(3, 8, 20), s=48, n_kgroups=8,
                             n_qgroups=8, P=24, calls=3)
     calls = gen.make_stream(w)
     op = S.SparsePR(w)
+    if km_path:
+        op.set_kmeans_path(km_path)
     warm = None
     for c, (Q, K, V) in enumerate(calls):
         qf, kf, vf = flat(Q), flat(K), flat(V)
