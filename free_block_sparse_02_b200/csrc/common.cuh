@@ -122,6 +122,10 @@ struct Layout {
   // than kKmChunkGroups groups): {best bits, second bits, best group, 0}; null when unused
   int4* ktop;                     // [BH, N]
   int4* qtop;                     // [BH, N]
+  // each point's label in the iteration before (the per-iteration update moves the group sums
+  // by the points whose label changed)
+  int* kprev;                     // [BH, N]
+  int* qprev;                     // [BH, N]
   // whole-loop k-means (mid-size calls: every Lloyd iteration of a side in one launch, G CTAs
   // per head): each CTA's partial group sums, counts and objective, the head barrier counters
   // and the abort flag; null when no side qualifies

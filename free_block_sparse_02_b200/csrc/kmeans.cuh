@@ -66,7 +66,7 @@ __device__ __forceinline__ double warp_transpose_sum32(double (&v)[32]) {
 __device__ __forceinline__ double query_scale_fp64(const double* Gc, const double* xs, const double (&xl)[4], int D) {
   const int lane = threadIdx.x & 31;
   double part = 0.0;
-#pragma unroll 4
+#pragma unroll 16
   for (int a = 0; a < D; ++a) {
     double row = 0.0;
 #pragma unroll
@@ -84,18 +84,29 @@ __device__ __forceinline__ void redecide_candidates(const double* xs, int D, con
                                                     double scale, const int* cand, int ncand, int& best_out,
                                                     double& bestv_out) {
   const int lane = threadIdx.x & 31;
+  // every candidate's W row piece and bias first (all loads in flight), then the scores
+  double wv[4][4], bb[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int j = c < ncand ? cand[c] : 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      wv[c][k] = (c < ncand && lane + 32 * k < D) ? ld_w<kCg>(W64 + (size_t)j * D + lane + 32 * k) : 0.0;
+    bb[c] = c < ncand ? ld_w<kCg>(B64 + j) : 0.0;
+  }
   double bv = INFINITY;
   int bj = 0;
-  for (int c = 0; c < ncand; ++c) {
-    const int j = cand[c];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    if (c >= ncand) break;
     double part = 0.0;
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-      if (lane + 32 * k < D) part += ld_w<kCg>(W64 + (size_t)j * D + lane + 32 * k) * xs[lane + 32 * k];
-    const double sc = ld_w<kCg>(B64 + j) - 2.0 * scale * warp_sum(part);
+      if (lane + 32 * k < D) part += wv[c][k] * xs[lane + 32 * k];
+    const double sc = bb[c] - 2.0 * scale * warp_sum(part);
     if (sc < bv) {
       bv = sc;
-      bj = j;
+      bj = cand[c];
     }
   }
   best_out = bj;

@@ -12,8 +12,8 @@
 //    contiguous point tiles [r T / G, (r + 1) T / G) of its head in shared memory for the whole
 //    loop: X is read from HBM once, not twice per iteration.
 //  * Per iteration: the head's two-term W (hi, mid) and biases are copied into shared memory;
-//    the tensor cores score every resident tile (tcgen05, two TMEM accumulators, one epilogue
-//    warpgroup per accumulator); flagged points are re-decided in fp64; each group's points are
+//    the tensor cores score every resident tile (tcgen05, up to four TMEM accumulators, two
+//    epilogue warpgroups); flagged points are re-decided in fp64; each group's points are
 //    summed in fp64 (one warp per group, sorted runs, fixed order) and written as this CTA's
 //    partial sums.  A head barrier; then CTA r owns groups [r C / G, (r + 1) C / G): it adds the
 //    G partials of each owned group in CTA order, updates the centroid, takes the stop test (the
@@ -48,14 +48,21 @@ constexpr int kKlMaxKGroups = 256;   // key groups the query step stages per own
 constexpr size_t kKlStaticSmem = 10 * 1024;  // bound of the kernel's static shared memory
 
 // Shared memory of the loop kernel for `cap` resident tiles: X, the two W terms, per point
-// (label, sorted order, 1/rms in fp32 and fp64, bound norm, re-decision entry), per-warp fp64
-// staging of one point, biases, group offsets, barriers.
+// (label, sorted order, 1/rms in fp32 and fp64, bound norm, re-decision entry), the scratch,
+// biases, group offsets, barriers.
 // At least 120 KB, so that two CTAs never share an SM: each may hold all 512 TMEM columns, and a
 // CTA blocked in the allocator would never reach the head barrier its partner waits at.
+// Scratch doubles shared by three phases that never overlap: the per-warp fp64 copy of a point
+// being re-decided (128 per warp), the run pieces of the group sums (2 D per warp) and the
+// slices of the centroid step's products (kKlThreads / D slices x kKlBatch x D = 1536).
+__host__ __device__ constexpr int km_loop_scratch(int D) {
+  return kKlWarps * 128 > kKlWarps * 2 * D ? kKlWarps * 128 : kKlWarps * 2 * D;
+}
+
 __host__ __device__ inline size_t km_loop_smem(int D, int Np, int C, int cap) {
   const size_t pts = (size_t)cap * kKlTile;
   const size_t need = 1024 /*align*/ + pts * D * 2 + (size_t)2 * Np * D * 2 + pts * (4 + 4 + 4 + 4 + 8 + 16) +
-                      (size_t)kKlWarps * 128 * 8 + (size_t)Np * 4 + (size_t)(2 * C + 2) * 4 + 128 /*barriers*/;
+                      (size_t)km_loop_scratch(D) * 8 + (size_t)Np * 4 + (size_t)(2 * C + 2) * 4 + 128 /*barriers*/;
   return need > (size_t)120 * 1024 ? need : (size_t)120 * 1024;
 }
 
@@ -76,15 +83,16 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // Barrier of the G CTAs of one head: the n-th call of every CTA of the head returns once all of
-// them have made it (counter target G n).  Bounded: gives up, sets the launch's abort flag and
+// them have made it (counter target G n): a release addition, then acquire loads.  Bounded: gives up, sets the launch's abort flag and
 // returns false after `limit` cycles, or as soon as another CTA has set the flag.  Called by
 // every thread of the CTA (block barriers on both sides).
 __device__ __forceinline__ bool head_barrier(unsigned* ctr, unsigned target, int* gabort, volatile int* s_abort,
                                              long long limit) {
   __syncthreads();
   if (threadIdx.x == 0 && !*s_abort) {
-    __threadfence();
-    atomicAdd(ctr, 1u);
+    // release: the CTA's writes before the block barrier above are visible to every CTA whose
+    // acquire load sees this addition
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(ctr), "r"(1u) : "memory");
     const long long t0 = clock64();
     while (ld_acquire_u32(ctr) < target) {
       if (ld_volatile_i32(gabort)) {
@@ -97,9 +105,8 @@ __device__ __forceinline__ bool head_barrier(unsigned* ctr, unsigned target, int
         break;
       }
     }
-    __threadfence();
   }
-  __syncthreads();
+  __syncthreads();  // the acquire above orders the whole CTA's later reads (block barrier)
   return !*s_abort;
 }
 
@@ -135,8 +142,8 @@ __global__ void __launch_bounds__(kKlThreads, 1)
   float* xn = sq + pts;                                      // [pts] norm in the rounding bound
   double* sig = (double*)(xn + pts);                         // [pts] scale of the group sums
   int4* flags = (int4*)(sig + pts);                          // [pts] re-decision entries
-  double* xs_all = (double*)(flags + pts);                   // [kKlWarps][128]
-  float* sbias = (float*)(xs_all + kKlWarps * 128);          // [Np]
+  double* xs_all = (double*)(flags + pts);                   // scratch: km_loop_scratch(D) doubles
+  float* sbias = (float*)(xs_all + km_loop_scratch(D));      // [Np]
   int* offs = (int*)(sbias + Np);                            // [C + 1]
   int* cursor = offs + C + 1;                                // [C + 1]
   uint64_t* bars = (uint64_t*)(((uintptr_t)(cursor + C + 1) + 7) & ~(uintptr_t)7);
@@ -146,7 +153,7 @@ __global__ void __launch_bounds__(kKlThreads, 1)
   uint64_t* mma_done = bars + 9;
   uint32_t* tmem_slot = (uint32_t*)(bars + 10);
   __shared__ volatile int s_abort;
-  __shared__ int s_nflag, s_next;
+  __shared__ int s_nflag, s_nchg;
   __shared__ float s_wmax, s_bmax;
   __shared__ double s_red[kKlWarps], s_redc[kKlWarps];
   __shared__ double s_red8[2 * kKlBatch][kKlWarps];
@@ -201,66 +208,121 @@ __global__ void __launch_bounds__(kKlThreads, 1)
   // ------------------------------------------------------------- centroid step of owned groups
   // update: c <- (sum of the G partial sums) / count for groups that received points (keys: c in
   // key space; queries: nu = C S / (sqrt(d) n), or the raw mean in the semantic partition);
-  // weights: the score weights, bias and norm of the next assignment.
+  // weights: the score weights, bias and norm of the next assignment.  The matrix-vector
+  // products are split over every thread (thread = (dimension, slice of the inner index), 16
+  // loads in flight), the slices' sums staged in wpart and added in a fixed order: the operands
+  // come from L2, and one thread walking a whole column would wait for each load in turn.
+  double* wpart = xs_all;             // [nsplit][kKlBatch][D]: the re-decision staging, free here
+  const int nsplit = kKlThreads / D;  // 6 (d = 64) or 3 (d = 128): nsplit * kKlBatch * D = 1536
   auto centroid_step = [&](bool update, bool weights) {
+    const double* Cg = L.kcent + (size_t)bh * L.Ck * D;  // key-group centroids (the query side's C)
     for (int gb = j0; gb < j1; gb += kKlBatch) {
       const int nb = min(kKlBatch, j1 - gb);
       const int Vd = (kKeys || L.semantic) ? D : L.Ck;  // length of a centroid vector
-      __syncthreads();  // cb is free
+      __syncthreads();  // cb and wpart are free
       if (update) {
-        // mean of the members' (scaled) inputs, in cb (D entries per group); counts in s_gred
-        for (int e = tid; e < nb * D; e += kKlThreads) {
+        // counts: warp g of the batch, lanes over the head's CTAs
+        if (warp < nb) {
+          int c = 0;
+          for (int q = lane; q < G; q += 32) c += __ldcg(L.klp_cnt + (hc + q) * C + gb + warp);
+          c = __reduce_add_sync(0xffffffffu, c);
+          if (lane == 0) s_gred[warp][0] = (double)c;
+        }
+        // sums of the G partials of (group g, dimension a), 16 CTAs' loads in flight per batch; the
+        // old centroid (kept where no point joined) fetched alongside
+        double tot[2] = {0.0, 0.0}, old[2] = {0.0, 0.0};
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int e = tid + i * kKlThreads;
+          if (e >= nb * D) continue;
           const int g = e / D, a = e % D, j = gb + g;
-          int cnt = 0;
-          double s = 0.0;
-#pragma unroll 6
-          for (int q = 0; q < G; ++q) {  // independent loads (every CTA wrote every group)
-            cnt += __ldcg(L.klp_cnt + (hc + q) * C + j);
-            s += __ldcg(L.klp_sum + ((hc + q) * C + j) * D + a);
+          if (kKeys) old[i] = L.kcent[((size_t)bh * C + j) * D + a];
+          else if (L.semantic) old[i] = L.qU64[((size_t)bh * C + j) * D + a];
+          const double* src = L.klp_sum + (hc * C + j) * D + a;  // CTA q's value at src[q C D]
+          for (int q0 = 0; q0 < G; q0 += 16) {
+            double v[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) v[k] = q0 + k < G ? __ldcg(src + (size_t)(q0 + k) * C * D) : 0.0;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) tot[i] += v[k];
           }
-          cb[g][a] = cnt > 0 ? s / (double)cnt : 0.0;
-          if (a == 0) s_gred[g][0] = (double)cnt;
+        }
+        __syncthreads();  // counts in s_gred
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int e = tid + i * kKlThreads;
+          if (e >= nb * D) continue;
+          const int g = e / D, a = e % D;
+          const double cnt = s_gred[g][0];
+          const double mean = cnt > 0.0 ? tot[i] / cnt : 0.0;
+          if (kKeys || L.semantic) {  // the new centroid, or the old one where no point joined
+            cb[g][a] = cnt > 0.0 ? mean : old[i];
+            if (cnt > 0.0) (kKeys ? L.kcent : L.qU64)[((size_t)bh * C + gb + g) * D + a] = mean;
+          } else {
+            cb[g][a] = mean;  // S_g / n_g, projected to nu below
+          }
         }
         __syncthreads();
-        if (kKeys) {
-          for (int e = tid; e < nb * D; e += kKlThreads) {
-            const int g = e / D, a = e % D;
-            if (s_gred[g][0] > 0.0) L.kcent[((size_t)bh * C + gb + g) * D + a] = cb[g][a];
-          }
-        } else if (L.semantic) {
-          for (int e = tid; e < nb * D; e += kKlThreads) {
-            const int g = e / D, a = e % D;
-            if (s_gred[g][0] > 0.0) L.qU64[((size_t)bh * C + gb + g) * D + a] = cb[g][a];
-          }
-        } else {
-          // nu_g[j] = C[j] . S_g / sqrt(d): one warp per key group j, lanes over the dimensions
-          const double* Ck = L.kcent + (size_t)bh * L.Ck * D;
-          for (int j = warp; j < L.Ck; j += kKlWarps) {
-            double cj[4];
+        if (!kKeys && !L.semantic) {
+          // nu_g[j] = C[j] . S_g / sqrt(d): thread j (one per key group) reads its row of C in
+          // 16-byte pieces, eight in flight; nu replaces S_g in cb (the old nu where no point
+          // joined)
+          double acc[kKlBatch], oldnu[kKlBatch];
+          const int j = tid;
+          if (j < L.Ck) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) cj[k] = lane + 32 * k < D ? Ck[(size_t)j * D + lane + 32 * k] : 0.0;
-            for (int g = 0; g < nb; ++g) {
-              double part = 0.0;
+            for (int g = 0; g < kKlBatch; ++g) {
+              acc[g] = 0.0;
+              oldnu[g] = g < nb ? L.qcent[((size_t)bh * C + gb + g) * L.Ck + j] : 0.0;
+            }
+            const double2* row = (const double2*)(Cg + (size_t)j * D);
+#pragma unroll 8
+            for (int a2 = 0; a2 < D / 2; ++a2) {
+              const double2 v = row[a2];
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                if (lane + 32 * k < D) part += cj[k] * cb[g][lane + 32 * k];
-              part = warp_sum(part);
-              if (lane == 0 && s_gred[g][0] > 0.0) L.qcent[((size_t)bh * C + gb + g) * L.Ck + j] = part * rsd;
+              for (int g = 0; g < kKlBatch; ++g) acc[g] += v.x * cb[g][2 * a2] + v.y * cb[g][2 * a2 + 1];
             }
           }
+          __syncthreads();  // every thread has read S from cb
+          if (j < L.Ck)
+            for (int g = 0; g < nb; ++g) {
+              const bool joined = s_gred[g][0] > 0.0;
+              cb[g][j] = joined ? acc[g] * rsd : oldnu[g];
+              if (joined) L.qcent[((size_t)bh * C + gb + g) * L.Ck + j] = acc[g] * rsd;
+            }
+          __syncthreads();
         }
-        __syncthreads();  // centroids written; cb is reused below
       }
       if (!weights) continue;
-      // the (possibly updated) centroid vectors of the batch into cb
-      const double* cent = kKeys ? L.kcent : (L.semantic ? L.qU64 : L.qcent);
-      for (int e = tid; e < nb * Vd; e += kKlThreads) {
-        const int g = e / Vd, a = e % Vd;
-        cb[g][a] = cent[((size_t)bh * C + gb + g) * Vd + a];
+      if (!update) {  // the initial centroid vectors of the batch into cb
+        const double* cent = kKeys ? L.kcent : (L.semantic ? L.qU64 : L.qcent);
+        for (int e = tid; e < nb * Vd; e += kKlThreads) {
+          const int g = e / Vd, a = e % Vd;
+          cb[g][a] = cent[((size_t)bh * C + gb + g) * Vd + a];
+        }
+        __syncthreads();
+      }
+      // w[g][a] = sum_k Op[k][a] cb[g][k]: keys Op = M (symmetric, so its column a is row a read
+      // down), queries Op = C (k over the key groups, then / sqrt(d)); the semantic queries take
+      // w = cb.  Thread (a, slice): the slice's partial sums of every group of the batch.
+      const int Kin = kKeys ? D : (L.semantic ? 0 : L.Ck);
+      if (Kin > 0) {
+        const int a = tid % D, part = tid / D;
+        const int k0 = part * Kin / nsplit, k1 = (part + 1) * Kin / nsplit;
+        const double* Op = (kKeys ? L.M + (size_t)bh * D * D : Cg) + a;  // element (k, a) at Op[k * D]
+        double acc[kKlBatch];
+#pragma unroll
+        for (int g = 0; g < kKlBatch; ++g) acc[g] = 0.0;
+#pragma unroll 16
+        for (int k = k0; k < k1; ++k) {
+          const double m = Op[(size_t)k * D];
+#pragma unroll
+          for (int g = 0; g < kKlBatch; ++g) acc[g] += m * cb[g][k];
+        }
+#pragma unroll
+        for (int g = 0; g < kKlBatch; ++g) wpart[((size_t)part * kKlBatch + g) * D + a] = acc[g];
       }
       __syncthreads();
-      // w (thread = (group, dimension)): keys M c (M symmetric: column reads), queries C^T nu / sqrt(d)
-      // or the raw mean; then bias and norm by warp sums
       double pb[kKlBatch], pn[kKlBatch];
 #pragma unroll
       for (int g = 0; g < kKlBatch; ++g) pb[g] = pn[g] = 0.0;
@@ -269,16 +331,13 @@ __global__ void __launch_bounds__(kKlThreads, 1)
         const int e = tid + k * kKlThreads;
         if (e >= nb * D) continue;
         const int g = e / D, a = e % D;
-        double w = 0.0;
-        if (kKeys) {
-          const double* M = L.M + (size_t)bh * D * D;
-          for (int b = 0; b < D; ++b) w += M[(size_t)b * D + a] * cb[g][b];
-        } else if (L.semantic) {
-          w = cb[g][a];
+        double w;
+        if (Kin > 0) {
+          w = 0.0;
+          for (int q = 0; q < nsplit; ++q) w += wpart[((size_t)q * kKlBatch + g) * D + a];
+          if (!kKeys) w *= rsd;
         } else {
-          const double* Ck = L.kcent + (size_t)bh * L.Ck * D;
-          for (int j = 0; j < L.Ck; ++j) w += Ck[(size_t)j * D + a] * cb[g][j];
-          w *= rsd;
+          w = cb[g][a];
         }
         const size_t gj = (size_t)bh * C + gb + g;
         if (kKeys) {
@@ -340,11 +399,14 @@ __global__ void __launch_bounds__(kKlThreads, 1)
         const int use = it * nt + k, b = use % NACC, n = use / NACC;
         if (n >= 1 && !mbar_wait(acc_empty + b, (n - 1) & 1, &s_abort)) break;
         tc_fence_after();
+        // both W terms stacked as one operand of 2 Np rows: [X W_hi | X W_mid] side by side (one
+        // chain per term, added in the epilogue; the rounding bound covers both forms).  Measured
+        // faster here than one chain of both terms into Np columns.
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t xd =
               sdesc_sw128(smem_u32(sX + ((size_t)k * KB + (ks >> 2)) * kKlTile * 128) + (ks & 3) * 32, 16, 1024);
           const uint64_t wd = sdesc_sw128(smem_u32(sW + (size_t)(ks >> 2) * 2 * Np * 128) + (ks & 3) * 32, 16, 1024);
-          mma_ss(tmem + b * A, xd, wd, idesc2, ks > 0 ? 1u : 0u);  // [X W_hi | X W_mid]
+          mma_ss(tmem + b * A, xd, wd, idesc2, ks > 0 ? 1u : 0u);
         }
         mma_commit(acc_full + b);
       }
@@ -471,7 +533,17 @@ __global__ void __launch_bounds__(kKlThreads, 1)
   auto group_sums = [&]() {
     for (int j = tid; j <= C; j += kKlThreads) cursor[j] = 0;
     __syncthreads();
-    for (int p = tid; p < npts; p += kKlThreads) atomicAdd(&cursor[lab[p]], 1);
+    // histogram: lanes holding the same label add once (labels are spatially coherent)
+    for (int p0 = 0; p0 < npts; p0 += kKlThreads) {
+      const int p = p0 + tid;
+      const bool v = p < npts;
+      const int g = v ? lab[p] : -1;
+      const unsigned act = __ballot_sync(0xffffffffu, v);
+      if (v) {
+        const unsigned same = __match_any_sync(act, g);
+        if (lane == __ffs(same) - 1) atomicAdd(&cursor[g], __popc(same));
+      }
+    }
     __syncthreads();
     if (warp == 0) {  // exclusive prefix over the groups
       int run = 0;
@@ -493,57 +565,166 @@ __global__ void __launch_bounds__(kKlThreads, 1)
       if (lane == 0) offs[C] = run;
     }
     __syncthreads();
-    for (int p = tid; p < npts; p += kKlThreads) order[atomicAdd(&cursor[lab[p]], 1)] = p;
-    if (tid == 0) s_next = 0;
-    __syncthreads();
-    // one warp per group: lanes over the dimensions (d = 64: two per lane, d = 128: four), the
-    // group's points in their sorted order; the CTA's count and sum of every group it holds
-    const int per = D / 32;
-    while (true) {
-      int g = 0;
-      if (lane == 0) g = atomicAdd(&s_next, 1);
-      g = __shfl_sync(0xffffffffu, g, 0);
-      if (g >= C) break;
-      const int q0 = offs[g], q1 = offs[g + 1];
-      if (lane == 0) __stcg(L.klp_cnt + (hc + r) * C + g, q1 - q0);
-      const int a0 = lane * per;
-      // four rows in flight, each into its own accumulators (an empty group writes zeros)
-      double acc[4][4];
-#pragma unroll
-      for (int u2 = 0; u2 < 4; ++u2)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[u2][k] = 0.0;
-      auto add_row = [&](double (&ac)[4], int p) {
-        const double sc = kKeys ? 1.0 : sig[p];
-        const __nv_bfloat16* xp = x_at(p, a0);  // `per` consecutive dimensions of one 16-byte piece
-        if (per == 2) {
-          const uint32_t v = *(const uint32_t*)xp;
-          ac[0] = fma(bf16_bits_to_f64(v & 0xFFFFu), sc, ac[0]);
-          ac[1] = fma(bf16_bits_to_f64(v >> 16), sc, ac[1]);
-        } else {
-          const uint2 v = *(const uint2*)xp;
-          ac[0] = fma(bf16_bits_to_f64(v.x & 0xFFFFu), sc, ac[0]);
-          ac[1] = fma(bf16_bits_to_f64(v.x >> 16), sc, ac[1]);
-          ac[2] = fma(bf16_bits_to_f64(v.y & 0xFFFFu), sc, ac[2]);
-          ac[3] = fma(bf16_bits_to_f64(v.y >> 16), sc, ac[3]);
-        }
-      };
-      int qq = q0;
-      for (; qq + 4 <= q1; qq += 4) {
-        const int pa = order[qq], pb2 = order[qq + 1], pc = order[qq + 2], pd = order[qq + 3];
-        add_row(acc[0], pa);
-        add_row(acc[1], pb2);
-        add_row(acc[2], pc);
-        add_row(acc[3], pd);
+    for (int p0 = 0; p0 < npts; p0 += kKlThreads) {  // scatter: one atomic per label per warp
+      const int p = p0 + tid;
+      const bool v = p < npts;
+      const int g = v ? lab[p] : -1;
+      const unsigned act = __ballot_sync(0xffffffffu, v);
+      if (v) {
+        const unsigned same = __match_any_sync(act, g);
+        const int leader = __ffs(same) - 1;
+        int base = 0;
+        if (lane == leader) base = atomicAdd(&cursor[g], __popc(same));
+        base = __shfl_sync(same, base, leader);
+        order[base + __popc(same & ((1u << lane) - 1))] = p;
       }
-      if (qq < q1) add_row(acc[0], order[qq]);  // the last 0..3 rows
-      if (qq + 1 < q1) add_row(acc[1], order[qq + 1]);
-      if (qq + 2 < q1) add_row(acc[2], order[qq + 2]);
+    }
+    __syncthreads();
+    // Balanced sums.  Warp w takes the sorted positions [s0, s1) = [w n / 12, (w + 1) n / 12);
+    // lanes run over the dimensions (d = 64: two per lane, d = 128: four), four rows in flight.
+    // A run (one group's points) that lies inside the slice is written to the CTA's partial sums
+    // at once.  A run that crosses a slice boundary leaves its piece in shared memory: slot 0 for
+    // the run the slice starts in when it began before s0, slot 1 for the run the slice ends in
+    // when it goes on past s1.  After a barrier the pieces of each crossing run are added in warp
+    // order, and absent groups get zeros.
+    const int per = D / 32, a0 = lane * per;
+    double* pieces = xs_all;  // [kKlWarps][2][D]: the re-decision staging, free here
+    auto slice_lo = [&](int w) { return (int)((long long)npts * w / kKlWarps); };
+    auto add_row = [&](double (&ac)[4], int p) {
+      const double sc = kKeys ? 1.0 : sig[p];
+      const __nv_bfloat16* xp = x_at(p, a0);  // `per` consecutive dimensions of one 16-byte piece
+      if (per == 2) {
+        const uint32_t v = *(const uint32_t*)xp;
+        ac[0] = fma(bf16_bits_to_f64(v & 0xFFFFu), sc, ac[0]);
+        ac[1] = fma(bf16_bits_to_f64(v >> 16), sc, ac[1]);
+      } else {
+        const uint2 v = *(const uint2*)xp;
+        ac[0] = fma(bf16_bits_to_f64(v.x & 0xFFFFu), sc, ac[0]);
+        ac[1] = fma(bf16_bits_to_f64(v.x >> 16), sc, ac[1]);
+        ac[2] = fma(bf16_bits_to_f64(v.y & 0xFFFFu), sc, ac[2]);
+        ac[3] = fma(bf16_bits_to_f64(v.y >> 16), sc, ac[3]);
+      }
+    };
+    const int s0 = slice_lo(warp), s1 = slice_lo(warp + 1);
+    if (s0 < s1) {
+      int g = lab[order[s0]];
+      while (true) {
+        const int q0 = offs[g], q1 = offs[g + 1];
+        const int b0 = max(q0, s0), b1 = min(q1, s1);
+        double acc[4][4];
+#pragma unroll
+        for (int u2 = 0; u2 < 4; ++u2)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) acc[u2][k] = 0.0;
+        int qq = b0;
+        for (; qq + 4 <= b1; qq += 4) {
+          const int pa = order[qq], pb2 = order[qq + 1], pc = order[qq + 2], pd = order[qq + 3];
+          add_row(acc[0], pa);
+          add_row(acc[1], pb2);
+          add_row(acc[2], pc);
+          add_row(acc[3], pd);
+        }
+        if (qq < b1) add_row(acc[0], order[qq]);  // the last 0..3 rows
+        if (qq + 1 < b1) add_row(acc[1], order[qq + 1]);
+        if (qq + 2 < b1) add_row(acc[2], order[qq + 2]);
+        const bool inside = q0 >= s0 && q1 <= s1;
+        double* dst = inside ? L.klp_sum + ((hc + r) * C + g) * D + a0 : pieces + ((size_t)warp * 2 + (q0 < s0 ? 0 : 1)) * D + a0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (k < per) {
+            const double v = (acc[0][k] + acc[1][k]) + (acc[2][k] + acc[3][k]);
+            if (inside) __stcg(dst + k, v);
+            else dst[k] = v;
+          }
+        if (inside && lane == 0) __stcg(L.klp_cnt + (hc + r) * C + g, q1 - q0);
+        if (b1 >= s1) break;
+        g = lab[order[b1]];  // the next group present (the sort is by group)
+      }
+    }
+    __syncthreads();
+    for (int g = warp; g < C; g += kKlWarps) {
+      const int q0 = offs[g], q1 = offs[g + 1];
+      int wf = 0, wl = 0;  // slices holding the run's first and last positions
+      for (int w2 = 1; w2 < kKlWarps; ++w2) {
+        if (slice_lo(w2) <= q0) wf = w2;
+        if (slice_lo(w2) <= q1 - 1) wl = w2;
+      }
+      if (q1 > q0 && wf == wl) continue;  // inside one slice: written by its warp
+      double v[4] = {0.0, 0.0, 0.0, 0.0};
+      if (q1 > q0)
+        for (int w2 = wf; w2 <= wl; ++w2) {
+          if (slice_lo(w2) == slice_lo(w2 + 1)) continue;  // an empty slice (fewer points than warps)
+          const double* pc = pieces + ((size_t)w2 * 2 + (q0 < slice_lo(w2) ? 0 : 1)) * D + a0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (k < per) v[k] += pc[k];
+        }
       double* dst = L.klp_sum + ((hc + r) * C + g) * D + a0;
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        if (k < per) __stcg(dst + k, (acc[0][k] + acc[1][k]) + (acc[2][k] + acc[3][k]));
+        if (k < per) __stcg(dst + k, v[k]);
+      if (lane == 0) __stcg(L.klp_cnt + (hc + r) * C + g, q1 - q0);
     }
+  };
+
+  // ------------------------------------------------------------- partial sums by label changes
+  // From the second iteration of the launch on, the CTA's partial sums and counts (its own
+  // slice of klp_sum / klp_cnt, kept from the iteration before) move only by the points whose
+  // label changed: the point leaves its old group's sum and joins its new group's (fp64 atomics,
+  // one warp per point, lanes over the dimensions).  Key sums of bf16 inputs are exact in fp64,
+  // so this equals summing every point again; query sums (scaled by 1/rms) agree to rounding.
+  // `prev` (the sort's order array, free after the first iteration) holds the labels of the
+  // iteration before; the changed points are listed in the re-decision entries' space.
+  auto delta_sums = [&]() {
+    int* prev = order;
+    int* changed = (int*)flags;
+    if (tid == 0) s_nchg = 0;
+    __syncthreads();
+    for (int p0 = 0; p0 < npts; p0 += kKlThreads) {
+      const int p = p0 + tid;
+      const bool ch = p < npts && lab[p] != prev[p];
+      const unsigned m = __ballot_sync(0xffffffffu, ch);
+      int base = 0;
+      if (lane == 0 && m) base = atomicAdd(&s_nchg, __popc(m));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (ch) changed[base + __popc(m & ((1u << lane) - 1))] = p;
+    }
+    __syncthreads();
+    const int nchg = s_nchg;
+    const int per = D / 32, a0 = lane * per;
+    double* part = L.klp_sum + (hc + r) * C * D;
+    int* pcnt = L.klp_cnt + (hc + r) * C;
+    for (int i = warp; i < nchg; i += kKlWarps) {
+      const int p = changed[i];
+      const int g0 = prev[p], g1 = lab[p];
+      const double sc = kKeys ? 1.0 : sig[p];
+      const __nv_bfloat16* xp = x_at(p, a0);
+      double v[4];
+      if (per == 2) {
+        const uint32_t u = *(const uint32_t*)xp;
+        v[0] = bf16_bits_to_f64(u & 0xFFFFu) * sc;
+        v[1] = bf16_bits_to_f64(u >> 16) * sc;
+        v[2] = v[3] = 0.0;
+      } else {
+        const uint2 u = *(const uint2*)xp;
+        v[0] = bf16_bits_to_f64(u.x & 0xFFFFu) * sc;
+        v[1] = bf16_bits_to_f64(u.x >> 16) * sc;
+        v[2] = bf16_bits_to_f64(u.y & 0xFFFFu) * sc;
+        v[3] = bf16_bits_to_f64(u.y >> 16) * sc;
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (k < per) {
+          atomicAdd(part + (size_t)g0 * D + a0 + k, -v[k]);
+          atomicAdd(part + (size_t)g1 * D + a0 + k, v[k]);
+        }
+      if (lane == 0) {
+        atomicAdd(pcnt + g0, -1);
+        atomicAdd(pcnt + g1, 1);
+      }
+    }
+    __syncthreads();  // every warp has read its points' previous labels
+    for (int i = tid; i < nchg; i += kKlThreads) prev[changed[i]] = lab[changed[i]];
   };
 
   // ------------------------------------------------------------- head-wide W into shared memory
@@ -551,21 +732,29 @@ __global__ void __launch_bounds__(kKlThreads, 1)
     const __nv_bfloat16* Wb = kKeys ? L.kWb : L.qWb;
     const size_t plane = (size_t)L.BH * Npg * D;
     const int nchunk = KB * 2 * Np * 8;  // 16-byte pieces of both terms
+    const float* B32 = (kKeys ? L.kbias32 : L.qbias32) + (size_t)bh * C;
+    const float* WN = (kKeys ? L.kwnorm : L.qwnorm) + (size_t)bh * C;
+    // the bias of group tid and (warp 0) the inputs of the bound's maxima, loaded with W
+    const float bj = tid < C ? __ldcg(B32 + tid) : INFINITY;
+    float bmx[4], wmx[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int j = lane + 32 * k;
+      const bool on = warp == 0 && j < C;
+      bmx[k] = on ? fabsf(__ldcg(B32 + j)) : 0.f;
+      wmx[k] = on ? __ldcg(WN + j) : 0.f;
+    }
+#pragma unroll 4
     for (int e = tid; e < nchunk; e += kKlThreads) {
       const int c = e & 7, n = (e >> 3) % Np, rest = (e >> 3) / Np, term = rest & 1, kb = rest >> 1;
       const uint4 v = n < Npg ? __ldcg((const uint4*)(Wb + term * plane + ((size_t)bh * Npg + n) * D + kb * 64 + c * 8))
                               : make_uint4(0u, 0u, 0u, 0u);  // rows past the global padding
       *(uint4*)(sW + ((size_t)(kb * 2 + term) * Np + n) * 128 + ((c ^ (n & 7)) << 4)) = v;
     }
-    const float* B32 = (kKeys ? L.kbias32 : L.qbias32) + (size_t)bh * C;
-    const float* WN = (kKeys ? L.kwnorm : L.qwnorm) + (size_t)bh * C;
-    for (int j = tid; j < Np; j += kKlThreads) sbias[j] = j < C ? __ldcg(B32 + j) : INFINITY;
-    if (warp == 0) {  // maxima of the rounding bound over all groups
-      float wm = 0.f, bm = 0.f;
-      for (int j = lane; j < C; j += 32) {
-        bm = fmaxf(bm, fabsf(__ldcg(B32 + j)));
-        wm = fmaxf(wm, __ldcg(WN + j));
-      }
+    if (tid < Np) sbias[tid] = bj;  // padded groups: +inf (Np <= 128 < the block's threads)
+    if (warp == 0) {  // maxima of the rounding bound over all groups (C <= 128)
+      float wm = fmaxf(fmaxf(wmx[0], wmx[1]), fmaxf(wmx[2], wmx[3]));
+      float bm = fmaxf(fmaxf(bmx[0], bmx[1]), fmaxf(bmx[2], bmx[3]));
       wm = warp_max(wm);
       bm = warp_max(bm);
       if (lane == 0) {
@@ -600,16 +789,30 @@ __global__ void __launch_bounds__(kKlThreads, 1)
       for (int w = 0; w < kKlWarps; ++w) js += s_redc[w];
       s_J = js;
     }
-    group_sums();
+    if (it == 0) {
+      group_sums();
+      __syncthreads();
+      for (int p = tid; p < npts; p += kKlThreads) order[p] = lab[p];  // the labels the next deltas start from
+    } else {
+      delta_sums();
+    }
     __syncthreads();
     if (tid == 0) {
       __stcg(L.klp_J + hc + r, s_J);
       if (s_nflag) atomicAdd((kKeys ? L.krefined : L.qrefined) + bh, s_nflag);
     }
     if (!head_barrier(hbar, G * ++nbar, gabort, &s_abort, blim)) break;
-    // the objective of this assignment, summed in CTA order by every CTA of the head
-    double Jc = T0;
-    for (int q = 0; q < G; ++q) Jc += __ldcg(L.klp_J + hc + q);
+    // the objective of this assignment: warp 0 loads the head's G shares at once (lane q takes
+    // CTAs q, q + 32, ...) and adds them in a fixed order, so every CTA of the head gets the same
+    // value
+    if (warp == 0) {
+      double js = 0.0;
+      for (int q = lane; q < G; q += 32) js += __ldcg(L.klp_J + hc + q);
+      js = warp_sum(js);
+      if (lane == 0) s_J = T0 + js;
+    }
+    __syncthreads();
+    const double Jc = s_J;
     if (r == 0 && tid == 0) Jarr[it] = Jc;
     const int nx = it + 1;  // the stop test before assignment nx
     const bool stop = nx >= P.iters || (nx >= 2 && L.km_tol >= 0.f && Jprev - Jc <= (double)L.km_tol * Jprev);

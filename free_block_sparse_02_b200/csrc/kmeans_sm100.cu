@@ -24,12 +24,14 @@
 //              a rigorous rounding bound goes to the CTA's re-decision list.  More than 256
 //              groups: one launch per chunk of 256, the best two carried between launches.
 //  update      First re-decides the points its range's assignment CTA listed, in fp64 (one warp
-//              each; label and objective corrected); then, for chunks of up to 16384 points of
+//              each; label and objective corrected); then, for chunks of up to 12288 points of
 //              one head, counting-sorts the points by label in shared memory and sums each
 //              group's run: one thread per (group, 8 dimensions) gathers the run's rows
 //              (consecutive threads read consecutive 16-byte pieces of a row), accumulates
 //              sigma x in fp64 registers and adds the result with one atomic per (group,
-//              dimension) per chunk.
+//              dimension) per chunk.  From the second iteration on only the points whose label
+//              changed are summed, as -x under the old label and +x under the new one: the
+//              group sums are running totals, not recomputed.
 //
 // Labels therefore equal the argmin of an fp64 evaluation, and the group sums are fp64 sums of
 // the exact inputs (keys) or of the inputs times their fp64 scale 1/rms (queries).
@@ -53,7 +55,9 @@ constexpr int kKmWTerms = 2;
 constexpr int kKmThreads = 384;   // warp 0 TMA, warp 1 MMA, warps 4..11 epilogue
 constexpr int kKmUpdThreads = 512;
 constexpr int kKmMaxStages = 3;  // 3 measured 2% faster than 4 at the 13B-DiT shape
-constexpr int kKmUpdChunk = 16384;  // points of one head sorted and summed at a time by the update
+constexpr int kKmUpdChunk = 12288;  // entries of one head sorted and summed at a time by the update
+                                    // (points, or two per label change)
+constexpr size_t kKmUpdStaticSmem = 17 * 1024;  // bound of the update kernel's static shared memory
 constexpr int kKmUpdItemRows = 64;   // rows of one accumulation item: a group's run is split into
                                      // pieces of at most this many rows, summed by different warps
 __host__ __device__ constexpr int km_upd_max_items(int C) { return kKmUpdChunk / kKmUpdItemRows + C; }
@@ -69,7 +73,8 @@ __host__ inline size_t km_assign_smem(int D, int Np, int stages) {
 // Shared memory of the update kernel: labels and sorted order of a chunk of points, per-group
 // offsets and cursors.
 __host__ inline size_t km_update_smem(int D, int C) {
-  const size_t chunk = (size_t)2 * kKmUpdChunk * 4 /*labels, order*/ + (size_t)(3 * C + 2) * 4 /*offs, cursor, ioff*/ +
+  const size_t chunk = (size_t)3 * kKmUpdChunk * 4 /*labels, order, entries*/ +
+                       (size_t)(4 * C + 2) * 4 /*offs, cursor, ioff, signed counts*/ +
                        (size_t)2 * km_upd_max_items(C) * 4 /*item group, item start*/;
   return std::max(chunk, (size_t)D * D * sizeof(double) /*Gc during the re-decision*/);
 }
@@ -546,14 +551,24 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
   // the re-decision of the points the assignment flagged in this range comes first; it may
   // use the start of the dynamic shared memory for Gc (d * d doubles <= the two chunk arrays)
   redecide_range<kKeys>(X, L, it, t0, t1, (double*)smem_raw);
-  int* lab = (int*)smem_raw;                   // [kKmUpdChunk] label of each point of the chunk
-  int* order = lab + kKmUpdChunk;              // [kKmUpdChunk] chunk points sorted by label
-  int* offs = order + kKmUpdChunk;             // [C + 1] start of each label's run
+  int* lab = (int*)smem_raw;                   // [kKmUpdChunk] label (key) of each entry of the chunk
+  int* order = lab + kKmUpdChunk;              // [kKmUpdChunk] entries sorted by label
+  int* ent = order + kKmUpdChunk;              // [kKmUpdChunk] entry codes (label changes only)
+  int* offs = ent + kKmUpdChunk;               // [C + 1] start of each label's run
   int* cursor = offs + (C + 1);                // [C] histogram, then next slot per label
   int* ioff = cursor + C;                      // [C + 1] first accumulation item of each label
-  int* item_g = ioff + (C + 1);                // [km_upd_max_items] group of each item
+  int* sdc = ioff + (C + 1);                   // [C] signed count changes (label changes only)
+  int* item_g = sdc + C;                       // [km_upd_max_items] group of each item
   int* item_s = item_g + km_upd_max_items(C);  // [km_upd_max_items] first slot of `order` of each item
-  __shared__ int s_next;
+  __shared__ int s_next, s_nent;
+  // From the second iteration on (tensor-core path), the sums and counts move only by the
+  // points whose label changed since the iteration before: each such point is two entries, -x
+  // under its old label and +x under its new one (code 2 i + 1 and 2 i), summed through the same
+  // sort and items as a full pass.  Key sums of bf16 inputs are exact in fp64, so this equals a
+  // full pass; query sums (scaled by 1/rms) agree to rounding.  The first iteration sums every
+  // point and records the labels in prev.
+  const bool delta = it > 0;
+  int* prev = kKeys ? L.kprev : L.qprev;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int* labels = kKeys ? L.klabel : L.qlabel;
@@ -567,22 +582,61 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
       t = (bh + 1) * tph;
       continue;
     }
-    // chunk: tiles [t, te) of head bh, at most kKmUpdChunk points
-    const int te = min(min(t1, (bh + 1) * tph), t + kKmUpdChunk / kKmTile);
+    // chunk: tiles [t, te) of head bh, at most kKmUpdChunk points (half as many with label
+    // changes: two entries each)
+    const int te = min(min(t1, (bh + 1) * tph), t + (delta ? kKmUpdChunk / 2 : kKmUpdChunk) / kKmTile);
     const int p_lo = (t % tph) * kKmTile;
     const int p_hi = min(L.N, (te - 1) % tph * kKmTile + kKmTile);
-    const int n = p_hi - p_lo;
+    const int np = p_hi - p_lo;
     const size_t row0 = (size_t)bh * L.N + p_lo;
-    for (int j = tid; j < C; j += kKmUpdThreads) cursor[j] = 0;
+    for (int j = tid; j < C; j += kKmUpdThreads) {
+      cursor[j] = 0;
+      sdc[j] = 0;
+    }
+    if (tid == 0) s_nent = 0;
     __syncthreads();
+    if (delta) {  // the entries of the points whose label changed
+      for (int i0 = 0; i0 < np; i0 += kKmUpdThreads) {
+        const int i = i0 + tid;
+        int gn = 0, go = 0;
+        if (i < np) {
+          gn = labels[row0 + i];
+          go = prev[row0 + i];
+          gn = (gn >= 0 && gn < C) ? gn : 0;
+          go = (go >= 0 && go < C) ? go : 0;
+        }
+        const bool ch = i < np && gn != go;
+        const unsigned m = __ballot_sync(0xffffffffu, ch);
+        int base = 0;
+        if (lane == 0 && m) base = atomicAdd(&s_nent, 2 * __popc(m));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (ch) {
+          const int k = base + 2 * __popc(m & ((1u << lane) - 1));
+          lab[k] = go;
+          ent[k] = 2 * i + 1;
+          lab[k + 1] = gn;
+          ent[k + 1] = 2 * i;
+          prev[row0 + i] = gn;
+          atomicAdd(&sdc[go], -1);
+          atomicAdd(&sdc[gn], 1);
+        }
+      }
+      __syncthreads();
+    }
+    const int n = delta ? s_nent : np;  // entries of the chunk
     // histogram: lanes holding the same label add once (labels are spatially coherent)
     for (int i0 = 0; i0 < n; i0 += kKmUpdThreads) {
       const int i = i0 + tid;
       int g = -1;
       if (i < n) {
-        g = labels[row0 + i];
-        g = (g >= 0 && g < C) ? g : 0;
-        lab[i] = g;
+        if (delta) {
+          g = lab[i];
+        } else {
+          g = labels[row0 + i];
+          g = (g >= 0 && g < C) ? g : 0;
+          lab[i] = g;
+          prev[row0 + i] = g;
+        }
       }
       const unsigned act = __ballot_sync(0xffffffffu, i < n);
       if (i < n) {
@@ -611,7 +665,8 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
           offs[j] = run + x - v;
           cursor[j] = run + x - v;
           ioff[j] = irun + y - nv;
-          if (v) atomicAdd(counts_all + (size_t)bh * C + j, v);
+          const int dc = delta ? sdc[j] : v;  // count change of the group
+          if (dc) atomicAdd(counts_all + (size_t)bh * C + j, dc);
         }
         run += __shfl_sync(0xffffffffu, x, 31);
         irun += __shfl_sync(0xffffffffu, y, 31);
@@ -667,37 +722,44 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
 #pragma unroll
       for (int k = 0; k < 8; ++k) r[k] = 0.0;
       int q = q0;
+      // entry at sorted slot q: its point and its factor (+1 or -1 for a label change; times the
+      // point's 1/rms for queries)
+      auto entry = [&](int q, int& p, double& f) {
+        const int e = order[q];
+        if (delta) {
+          const int code = ent[e];
+          p = code >> 1;
+          f = (code & 1) ? -1.0 : 1.0;
+        } else {
+          p = e;
+          f = 1.0;
+        }
+        if constexpr (!kKeys) f *= sig[p];
+      };
       for (; q + 8 <= q1; q += 8) {  // eight rows in flight per lane
         int pidx[8];
+        double fac[8];
         uint4 v[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) pidx[u] = order[q + u];
+        for (int u = 0; u < 8; ++u) entry(q + u, pidx[u], fac[u]);
 #pragma unroll
         for (int u = 0; u < 8; ++u) v[u] = *(const uint4*)(Xc + (size_t)pidx[u] * D + 8 * oc);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-          if constexpr (kKeys) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              r[2 * k] += bf16_bits_to_f64(w[k] & 0xFFFFu);
-              r[2 * k + 1] += bf16_bits_to_f64(w[k] >> 16);
-            }
-          } else {
-            const double sg = sig[pidx[u]];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              r[2 * k] = fma(bf16_bits_to_f64(w[k] & 0xFFFFu), sg, r[2 * k]);
-              r[2 * k + 1] = fma(bf16_bits_to_f64(w[k] >> 16), sg, r[2 * k + 1]);
-            }
+          for (int k = 0; k < 4; ++k) {  // (with factor 1 an exact addition)
+            r[2 * k] = fma(bf16_bits_to_f64(w[k] & 0xFFFFu), fac[u], r[2 * k]);
+            r[2 * k + 1] = fma(bf16_bits_to_f64(w[k] >> 16), fac[u], r[2 * k + 1]);
           }
         }
       }
       for (; q < q1; ++q) {
-        const int p = order[q];
+        int p;
+        double sg;
+        entry(q, p, sg);
         const uint4 v = *(const uint4*)(Xc + (size_t)p * D + 8 * oc);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        const double sg = kKeys ? 1.0 : sig[p];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           r[2 * k] = fma(bf16_bits_to_f64(w[k] & 0xFFFFu), sg, r[2 * k]);
@@ -888,7 +950,7 @@ bool km_tc_supported(const Layout& L, bool keys) {
   const int C = keys ? L.Ck : L.Cq;
   const bool chunked = (keys ? L.Ckp : L.Cqp) > kKmChunk;
   if (chunked && !(keys ? L.ktop : L.qtop)) return false;
-  return km_stages(L, km_chunk_rows(L, keys)) >= 2 && km_update_smem(L.d, C) <= 227 * 1024;
+  return km_stages(L, km_chunk_rows(L, keys)) >= 2 && km_update_smem(L.d, C) + kKmUpdStaticSmem <= 227 * 1024;
 }
 
 // CTAs of both k-means kernels: as many as fit the device at once (so the static ranges run in

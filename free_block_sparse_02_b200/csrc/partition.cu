@@ -316,8 +316,11 @@ __device__ __forceinline__ void stage_rows(double* dst, const double* __restrict
 // Keys, kPrepGroups groups per block (grid BH x ceil(C_k / 8), thread a = dimension):
 // c_j <- sum_j / n_j (groups that received points), the stop test, then W_j = M c_j (M staged in
 // shared memory, symmetric: thread a reads column a), bias_j = c_j^T W_j, ||W_j||, and the sums
-// zeroed.  Dynamic shared memory: min(d, kPrepRows) rows of M.
-__global__ void __launch_bounds__(128) kprep_kernel(Layout L, int it, int iters) {
+// zeroed for a pass over every point: always before the first assignment, and before each one
+// when `keep` is 0 (the CUDA-core path sums every point each iteration; the tensor-core path
+// only moves the sums by label changes after the first).  Dynamic shared memory:
+// min(d, kPrepRows) rows of M.
+__global__ void __launch_bounds__(128) kprep_kernel(Layout L, int it, int iters, int keep) {
   pdl_entry();
   extern __shared__ double Ms[];
   __shared__ double c[kPrepGroups][128];
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(128) kprep_kernel(Layout L, int it, int iters)
       const size_t gj = g0 + g;
       L.kW64[gj * d + a] = w[g];
       L.kW32[gj * d + a] = (float)w[g];
-      L.ksum[gj * d + a] = 0.0;
+      if (!keep || it == 0) L.ksum[gj * d + a] = 0.0;
       split3(w[g], L.kWb, (size_t)L.BH * L.Ckp * d, ((size_t)bh * L.Ckp + j0 + g) * d + a);
     }
   }
@@ -374,18 +377,18 @@ __global__ void __launch_bounds__(128) kprep_kernel(Layout L, int it, int iters)
     const size_t gj = g0 + a;
     L.kbias64[gj] = bias_s[a];
     L.kbias32[gj] = (float)bias_s[a];
-    L.kcount[gj] = 0;
+    if (!keep || it == 0) L.kcount[gj] = 0;
     L.kwnorm[gj] = (float)sqrt(wn_s[a]);
   }
 }
 
 // Queries, kPrepGroups groups per block (grid BH x ceil(C_q / 8)):
 // nu_g <- C S_g / (sqrt(d) n_g) (the mean normalised response of the members), the stop test,
-// then u_g = C^T nu_g / sqrt(d), bias ||nu_g||^2, ||u_g||, and the sums zeroed.  The key-group
-// centroids C are staged in shared memory kPrepRows rows at a time.
+// then u_g = C^T nu_g / sqrt(d), bias ||nu_g||^2, ||u_g||, and the sums zeroed as in
+// kprep_kernel.  The key-group centroids C are staged in shared memory kPrepRows rows at a time.
 // Dynamic shared memory: kPrepGroups * C_k doubles (nu of the block's groups), then
 // min(C_k, kPrepRows) rows of C.
-__global__ void __launch_bounds__(128) qprep_kernel(Layout L, int it, int iters) {
+__global__ void __launch_bounds__(128) qprep_kernel(Layout L, int it, int iters, int keep) {
   pdl_entry();
   extern __shared__ double qsm[];
   __shared__ double Sv[kPrepGroups][128];
@@ -419,7 +422,7 @@ __global__ void __launch_bounds__(128) qprep_kernel(Layout L, int it, int iters)
         const size_t gg = g0 + g;
         L.qU32[gg * d + tid] = (float)u;
         split3(u, L.qWb, (size_t)L.BH * L.Cqp * d, ((size_t)bh * L.Cqp + g0i + g) * d + tid);
-        L.qsum[gg * d + tid] = 0.0;
+        if (!keep || it == 0) L.qsum[gg * d + tid] = 0.0;
       }
     }
     block_sums8(cc, red, nn_s);
@@ -427,7 +430,7 @@ __global__ void __launch_bounds__(128) qprep_kernel(Layout L, int it, int iters)
       const size_t gg = g0 + tid;
       L.qbias64[gg] = nn_s[tid];
       L.qbias32[gg] = (float)nn_s[tid];
-      L.qcount[gg] = 0;
+      if (!keep || it == 0) L.qcount[gg] = 0;
       L.qwnorm[gg] = (float)sqrt(nn_s[tid]);
     }
     return;
@@ -501,7 +504,7 @@ __global__ void __launch_bounds__(128) qprep_kernel(Layout L, int it, int iters)
       L.qU64[gg * d + tid] = u;
       L.qU32[gg * d + tid] = (float)u;
       split3(u, L.qWb, (size_t)L.BH * L.Cqp * d, ((size_t)bh * L.Cqp + g0i + g) * d + tid);
-      L.qsum[gg * d + tid] = 0.0;
+      if (!keep || it == 0) L.qsum[gg * d + tid] = 0.0;
     }
   }
   block_sums8(un, red, un_s);
@@ -509,7 +512,7 @@ __global__ void __launch_bounds__(128) qprep_kernel(Layout L, int it, int iters)
     const size_t gg = g0 + tid;
     L.qbias64[gg] = nn_s[tid];
     L.qbias32[gg] = (float)nn_s[tid];
-    L.qcount[gg] = 0;
+    if (!keep || it == 0) L.qcount[gg] = 0;
     L.qwnorm[gg] = (float)sqrt(un_s[tid]);
   }
 }
@@ -1238,7 +1241,8 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
     if (e1) cudaEventRecord(e1, st);
   } else {
     for (int it = 0; it <= iters; ++it) {
-      launch(kprep_kernel, dim3(L.BH, (L.Ck + kPrepGroups - 1) / kPrepGroups), 128, kprep_smem, st, L, it, iters);
+      launch(kprep_kernel, dim3(L.BH, (L.Ck + kPrepGroups - 1) / kPrepGroups), 128, kprep_smem, st, L, it, iters,
+             tc_keys ? 1 : 0);
       if (it < iters) {
         if (tc_keys) {
           const sparsepr_status s = launch_kmeans_iteration_tc(L, true, K, it, Gk, st, it == 0 ? &ev : nullptr);
@@ -1271,7 +1275,8 @@ static sparsepr_status plan_typed(const Layout& L, const T* Q, const T* K, bool 
     if (s != SPARSEPR_OK) return s;
   } else {
     for (int it = 0; it <= iters; ++it) {
-      launch(qprep_kernel, dim3(L.BH, (L.Cq + kPrepGroups - 1) / kPrepGroups), 128, qprep_smem, st, L, it, iters);
+      launch(qprep_kernel, dim3(L.BH, (L.Cq + kPrepGroups - 1) / kPrepGroups), 128, qprep_smem, st, L, it, iters,
+             tc_queries ? 1 : 0);
       if (it < iters) {
         if (tc_queries) {
           const sparsepr_status s = launch_kmeans_iteration_tc(L, false, Q, it, Gq, st);

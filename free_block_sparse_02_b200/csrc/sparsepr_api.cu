@@ -148,6 +148,8 @@ size_t carve(const sparsepr_config& c, char* base, Layout& L) {
   take(L.knorm, BH * N * 4);
   if (L.Ckp > kKmChunkGroups) take(L.ktop, BH * N * 16);
   if (L.Cqp > kKmChunkGroups) take(L.qtop, BH * N * 16);
+  take(L.kprev, BH * N * 4);
+  take(L.qprev, BH * N * 4);
   {  // whole-loop k-means: partials for the most CTAs per head either side could use
     const int Gk = km_loop_ctas_per_head(c.B * c.H, c.N, c.d, c.dtype, c.n_kgroups, c.n_kgroups, true,
                                          kKmLoopMaxCtas, nullptr);
