@@ -264,32 +264,38 @@ __global__ void __launch_bounds__(kKlThreads, 1)
         }
         __syncthreads();
         if (!kKeys && !L.semantic) {
-          // nu_g[j] = C[j] . S_g / sqrt(d): thread j (one per key group) reads its row of C in
-          // 16-byte pieces, eight in flight; nu replaces S_g in cb (the old nu where no point
-          // joined)
-          double acc[kKlBatch], oldnu[kKlBatch];
-          const int j = tid;
-          if (j < L.Ck) {
+          // nu_g[j] = C[j] . S_g / sqrt(d): thread (j, slice of the dimensions), every load of the
+          // slice in flight, the slices' sums staged in wpart and added in a fixed order; nu
+          // replaces S_g in cb (the old nu where no point joined)
+          const int nsl = kKlThreads / L.Ck;  // slices per key group (>= 1: C_k <= 256)
+          {
+            const int j = tid % L.Ck, sl = tid / L.Ck;
+            if (sl < nsl) {
+              const int a0s = 2 * (sl * (D / 2) / nsl), a1s = 2 * ((sl + 1) * (D / 2) / nsl);
+              double acc[kKlBatch];
 #pragma unroll
-            for (int g = 0; g < kKlBatch; ++g) {
-              acc[g] = 0.0;
-              oldnu[g] = g < nb ? L.qcent[((size_t)bh * C + gb + g) * L.Ck + j] : 0.0;
-            }
-            const double2* row = (const double2*)(Cg + (size_t)j * D);
-#pragma unroll 8
-            for (int a2 = 0; a2 < D / 2; ++a2) {
-              const double2 v = row[a2];
+              for (int g = 0; g < kKlBatch; ++g) acc[g] = 0.0;
+              const double* row = Cg + (size_t)j * D;
+#pragma unroll 16
+              for (int a = a0s; a < a1s; a += 2) {
+                const double2 v = *(const double2*)(row + a);
 #pragma unroll
-              for (int g = 0; g < kKlBatch; ++g) acc[g] += v.x * cb[g][2 * a2] + v.y * cb[g][2 * a2 + 1];
+                for (int g = 0; g < kKlBatch; ++g) acc[g] += v.x * cb[g][a] + v.y * cb[g][a + 1];
+              }
+#pragma unroll
+              for (int g = 0; g < kKlBatch; ++g) wpart[((size_t)sl * kKlBatch + g) * L.Ck + j] = acc[g];
             }
           }
           __syncthreads();  // every thread has read S from cb
-          if (j < L.Ck)
-            for (int g = 0; g < nb; ++g) {
-              const bool joined = s_gred[g][0] > 0.0;
-              cb[g][j] = joined ? acc[g] * rsd : oldnu[g];
-              if (joined) L.qcent[((size_t)bh * C + gb + g) * L.Ck + j] = acc[g] * rsd;
-            }
+          for (int e = tid; e < nb * L.Ck; e += kKlThreads) {
+            const int g = e / L.Ck, j = e % L.Ck;
+            double nu = 0.0;
+            for (int sl = 0; sl < nsl; ++sl) nu += wpart[((size_t)sl * kKlBatch + g) * L.Ck + j];
+            nu *= rsd;
+            const bool joined = s_gred[g][0] > 0.0;
+            cb[g][j] = joined ? nu : L.qcent[((size_t)bh * C + gb + g) * L.Ck + j];
+            if (joined) L.qcent[((size_t)bh * C + gb + g) * L.Ck + j] = nu;
+          }
           __syncthreads();
         }
       }
@@ -860,9 +866,10 @@ int km_loop_ctas_per_head(int BH, int N, int d, int dtype, int C, int Ck, bool k
   if (Np > 128) return 0;
   if (!keys && Ck > kKlMaxKGroups) return 0;
   const int tph = (N + kKlTile - 1) / kKlTile;
-  const int G = std::min(tph, ctas / BH);
+  int G = std::min(tph, ctas / BH);
   if (G < 1) return 0;
   const int cap = (tph + G - 1) / G;
+  G = (tph + cap - 1) / cap;  // the fewest CTAs with that many tiles each: fewer partials per group
   if (km_loop_smem(d, Np, C, cap) + kKlStaticSmem > (size_t)227 * 1024) return 0;
   if (cap_out) *cap_out = cap;
   return G;
