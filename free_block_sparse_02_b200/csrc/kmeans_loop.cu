@@ -444,9 +444,18 @@ __global__ void __launch_bounds__(kKlThreads, 1)
         for (int c0 = 0; c0 < Np; c0 += 32) {
           float rr[32];
           load_dots(c0, rr);
+          float bq[8][4];  // the biases four at a time (16-byte shared-memory loads)
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 v4 = reinterpret_cast<const float4*>(sbias + c0)[k4];
+            bq[k4][0] = v4.x;
+            bq[k4][1] = v4.y;
+            bq[k4][2] = v4.z;
+            bq[k4][3] = v4.w;
+          }
 #pragma unroll
           for (int kk = 0; kk < 32; ++kk) {
-            const float sc = fmaf(m2s, rr[kk], sbias[c0 + kk]);  // padded groups: bias +inf
+            const float sc = fmaf(m2s, rr[kk], bq[kk >> 2][kk & 3]);  // padded groups: bias +inf
             const bool lt = sc < b1;
             b2 = lt ? b1 : fminf(b2, sc);
             i1 = lt ? c0 + kk : i1;

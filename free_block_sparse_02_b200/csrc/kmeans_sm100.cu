@@ -351,10 +351,20 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         // columns C .. Npr-1 (padded groups) have bias +inf and never win
         float r[32];
         load_dots(b, c0, r);
+        float bq[8][4];
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const float4 v4 = reinterpret_cast<const float4*>(bias + c0)[k4];
+          bq[k4][0] = v4.x;
+          bq[k4][1] = v4.y;
+          bq[k4][2] = v4.z;
+          bq[k4][3] = v4.w;
+        }
 #pragma unroll
         for (int kk = 0; kk < 32; ++kk) {
-          // ascending j and strict <: the lowest index of equal scores wins
-          const float sc = fmaf(m2s, r[kk], bias[c0 + kk]);
+          // ascending j and strict <: the lowest index of equal scores wins (the biases are read
+          // four at a time: 16-byte shared-memory loads, a quarter of the load instructions)
+          const float sc = fmaf(m2s, r[kk], bq[kk >> 2][kk & 3]);
           const bool lt = sc < b1;
           b2 = lt ? b1 : fminf(b2, sc);
           i1 = lt ? c0 + kk : i1;
