@@ -593,8 +593,30 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
       continue;
     }
     // chunk: tiles [t, te) of head bh, at most kKmUpdChunk points (half as many with label
-    // changes: two entries each)
-    const int te = min(min(t1, (bh + 1) * tph), t + (delta ? kKmUpdChunk / 2 : kKmUpdChunk) / kKmTile);
+    // changes: two entries each).  With label changes, the changed points of the head's whole
+    // segment of the range are counted first: when their entries fit, the segment is one chunk
+    // (after the first iterations few points change, and one sort serves the whole segment).
+    const int te_seg = min(t1, (bh + 1) * tph);
+    int te = min(te_seg, t + (delta ? kKmUpdChunk / 2 : kKmUpdChunk) / kKmTile);
+    auto changed = [&](size_t row) {  // the comparison of the entry pass below
+      int gn = labels[row], go = prev[row];
+      gn = (gn >= 0 && gn < C) ? gn : 0;
+      go = (go >= 0 && go < C) ? go : 0;
+      return gn != go;
+    };
+    if (delta && te < te_seg) {
+      const int q_lo = (t % tph) * kKmTile, q_hi = min(L.N, (te_seg - 1) % tph * kKmTile + kKmTile);
+      const size_t r0 = (size_t)bh * L.N + q_lo;
+      if (tid == 0) s_nent = 0;
+      __syncthreads();
+      int c = 0;
+      for (int i = tid; i < q_hi - q_lo; i += kKmUpdThreads) c += changed(r0 + i) ? 1 : 0;
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (lane == 0 && c) atomicAdd(&s_nent, c);
+      __syncthreads();
+      if (2 * s_nent <= kKmUpdChunk) te = te_seg;
+      __syncthreads();  // s_nent is reset below
+    }
     const int p_lo = (t % tph) * kKmTile;
     const int p_hi = min(L.N, (te - 1) % tph * kKmTile + kKmTile);
     const int np = p_hi - p_lo;
@@ -615,7 +637,7 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
           gn = (gn >= 0 && gn < C) ? gn : 0;
           go = (go >= 0 && go < C) ? go : 0;
         }
-        const bool ch = i < np && gn != go;
+        const bool ch = i < np && gn != go;  // (the same test as `changed`)
         const unsigned m = __ballot_sync(0xffffffffu, ch);
         int base = 0;
         if (lane == 0 && m) base = atomicAdd(&s_nent, 2 * __popc(m));

@@ -297,7 +297,9 @@ __device__ __forceinline__ void block_sums8(const double (&v)[kPrepGroups], doub
   __syncthreads();
 }
 
-constexpr int kPrepRows = 128;  // rows of M or C staged in shared memory at a time (fp64)
+constexpr int kPrepRows = 32;  // rows of M or C staged in shared memory at a time (fp64): 32 rows keep
+                               // a block at 32 KB at d = 128, so several blocks share an SM and their
+                               // staging overlaps (128 rows held one block per SM)
 
 // Rows [r0, r0 + nr) of a row-major fp64 matrix with `cols` (even) columns into shared memory
 // by 16-byte asynchronous copies, all issued before one wait (many in flight).  Both addresses
