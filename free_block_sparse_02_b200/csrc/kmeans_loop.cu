@@ -13,9 +13,10 @@
 //    loop: X is read from HBM once, not twice per iteration.
 //  * Per iteration: the head's two-term W (hi, mid) and biases are copied into shared memory;
 //    the tensor cores score every resident tile (tcgen05, up to four TMEM accumulators, two
-//    epilogue warpgroups); flagged points are re-decided in fp64; each group's points are
-//    summed in fp64 (one warp per group, sorted runs, fixed order) and written as this CTA's
-//    partial sums.  A head barrier; then CTA r owns groups [r C / G, (r + 1) C / G): it adds the
+//    epilogue warpgroups); flagged points are re-decided in fp64; the CTA's partial group sums
+//    are formed in fp64 (the first iteration sums every point, each warp an equal slice of the
+//    points sorted by label; later iterations move the partials by the points whose label
+//    changed).  A head barrier; then CTA r owns groups [r C / G, (r + 1) C / G): it adds the
 //    G partials of each owned group in CTA order, updates the centroid, takes the stop test (the
 //    objective is summed in the same order by every CTA of the head, so all of them decide
 //    alike) and, unless the loop stops, forms the next W, bias and norm of its groups.  A second

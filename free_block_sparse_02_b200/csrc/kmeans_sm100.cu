@@ -907,13 +907,22 @@ __global__ void __launch_bounds__(128, 1)
       uint32_t r[32];
       tmem_ld32(tmem + lane_base + b * D + c0, r);
       tmem_wait_ld();
+      // the row's elements eight at a time (16-byte shared-memory loads of the swizzled tile),
+      // in the same order: element a = c0 + k, k ascending
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const int a = c0 + k, kb = a >> 6, w = a & 63;
-        const uint32_t off = (uint32_t)p * 128 + ((((w >> 3) ^ (p & 7)) << 4) | ((w & 7) << 1));
-        const float x = __bfloat162float(*(const __nv_bfloat16*)(xs + (size_t)kb * kKmTile * 128 + off));
-        qf = fmaf(x, __uint_as_float(r[k]), qf);
-        nn = fmaf(x, x, nn);
+      for (int k8 = 0; k8 < 4; ++k8) {
+        const int a = c0 + 8 * k8, kb = a >> 6, w = a & 63;
+        const uint32_t off = (uint32_t)p * 128 + (((w >> 3) ^ (p & 7)) << 4);
+        const uint4 v = *(const uint4*)(xs + (size_t)kb * kKmTile * 128 + off);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float x0 = __uint_as_float(wv[u] << 16), x1 = __uint_as_float(wv[u] & 0xFFFF0000u);
+          qf = fmaf(x0, __uint_as_float(r[8 * k8 + 2 * u]), qf);
+          nn = fmaf(x0, x0, nn);
+          qf = fmaf(x1, __uint_as_float(r[8 * k8 + 2 * u + 1]), qf);
+          nn = fmaf(x1, x1, nn);
+        }
       }
     }
     if (p < np) {
