@@ -610,7 +610,17 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
       if (tid == 0) s_nent = 0;
       __syncthreads();
       int c = 0;
-      for (int i = tid; i < q_hi - q_lo; i += kKmUpdThreads) c += changed(r0 + i) ? 1 : 0;
+      const int nq = q_hi - q_lo;
+      for (int i0 = tid; i0 < nq; i0 += 8 * kKmUpdThreads) {  // eight points per thread in flight
+        bool chg[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * kKmUpdThreads;
+          chg[u] = i < nq && changed(r0 + i);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) c += chg[u] ? 1 : 0;
+      }
       c = __reduce_add_sync(0xffffffffu, c);
       if (lane == 0 && c) atomicAdd(&s_nent, c);
       __syncthreads();
@@ -627,30 +637,35 @@ __global__ void __launch_bounds__(kKmUpdThreads, 1)
     }
     if (tid == 0) s_nent = 0;
     __syncthreads();
-    if (delta) {  // the entries of the points whose label changed
-      for (int i0 = 0; i0 < np; i0 += kKmUpdThreads) {
-        const int i = i0 + tid;
-        int gn = 0, go = 0;
-        if (i < np) {
-          gn = labels[row0 + i];
-          go = prev[row0 + i];
-          gn = (gn >= 0 && gn < C) ? gn : 0;
-          go = (go >= 0 && go < C) ? go : 0;
+    if (delta) {  // the entries of the points whose label changed (eight rounds' loads in flight)
+      for (int i00 = 0; i00 < np; i00 += 8 * kKmUpdThreads) {
+        int gnv[8], gov[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i00 + u * kKmUpdThreads + tid;
+          gnv[u] = i < np ? labels[row0 + i] : 0;
+          gov[u] = i < np ? prev[row0 + i] : 0;
         }
-        const bool ch = i < np && gn != go;  // (the same test as `changed`)
-        const unsigned m = __ballot_sync(0xffffffffu, ch);
-        int base = 0;
-        if (lane == 0 && m) base = atomicAdd(&s_nent, 2 * __popc(m));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        if (ch) {
-          const int k = base + 2 * __popc(m & ((1u << lane) - 1));
-          lab[k] = go;
-          ent[k] = 2 * i + 1;
-          lab[k + 1] = gn;
-          ent[k + 1] = 2 * i;
-          prev[row0 + i] = gn;
-          atomicAdd(&sdc[go], -1);
-          atomicAdd(&sdc[gn], 1);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i00 + u * kKmUpdThreads + tid;
+          const int gn = (gnv[u] >= 0 && gnv[u] < C) ? gnv[u] : 0;
+          const int go = (gov[u] >= 0 && gov[u] < C) ? gov[u] : 0;
+          const bool ch = i < np && gn != go;  // (the same test as `changed`)
+          const unsigned m = __ballot_sync(0xffffffffu, ch);
+          int base = 0;
+          if (lane == 0 && m) base = atomicAdd(&s_nent, 2 * __popc(m));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (ch) {
+            const int k = base + 2 * __popc(m & ((1u << lane) - 1));
+            lab[k] = go;
+            ent[k] = 2 * i + 1;
+            lab[k + 1] = gn;
+            ent[k + 1] = 2 * i;
+            prev[row0 + i] = gn;
+            atomicAdd(&sdc[go], -1);
+            atomicAdd(&sdc[gn], 1);
+          }
         }
       }
       __syncthreads();
