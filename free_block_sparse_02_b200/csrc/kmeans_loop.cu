@@ -48,11 +48,6 @@ constexpr int kKlBatch = 4;          // owned groups updated together in the cen
 constexpr int kKlMaxKGroups = 256;   // key groups the query step stages per owned group
 constexpr size_t kKlStaticSmem = 10 * 1024;  // bound of the kernel's static shared memory
 
-// Shared memory of the loop kernel for `cap` resident tiles: X, the two W terms, per point
-// (label, sorted order, 1/rms in fp32 and fp64, bound norm, re-decision entry), the scratch,
-// biases, group offsets, barriers.
-// At least 120 KB, so that two CTAs never share an SM: each may hold all 512 TMEM columns, and a
-// CTA blocked in the allocator would never reach the head barrier its partner waits at.
 // Scratch doubles shared by three phases that never overlap: the per-warp fp64 copy of a point
 // being re-decided (128 per warp), the run pieces of the group sums (2 D per warp) and the
 // slices of the centroid step's products (kKlThreads / D slices x kKlBatch x D = 1536).
@@ -60,6 +55,11 @@ __host__ __device__ constexpr int km_loop_scratch(int D) {
   return kKlWarps * 128 > kKlWarps * 2 * D ? kKlWarps * 128 : kKlWarps * 2 * D;
 }
 
+// Shared memory of the loop kernel for `cap` resident tiles: X, the two W terms, per point
+// (label, sorted order, 1/rms in fp32 and fp64, bound norm, re-decision entry), the scratch,
+// biases, group offsets, barriers.  At least 120 KB, so that two CTAs never share an SM: each
+// may hold all 512 TMEM columns, and a CTA blocked in the allocator would never reach the head
+// barrier its partner waits at.
 __host__ __device__ inline size_t km_loop_smem(int D, int Np, int C, int cap) {
   const size_t pts = (size_t)cap * kKlTile;
   const size_t need = 1024 /*align*/ + pts * D * 2 + (size_t)2 * Np * D * 2 + pts * (4 + 4 + 4 + 4 + 8 + 16) +
@@ -84,9 +84,9 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // Barrier of the G CTAs of one head: the n-th call of every CTA of the head returns once all of
-// them have made it (counter target G n): a release addition, then acquire loads.  Bounded: gives up, sets the launch's abort flag and
-// returns false after `limit` cycles, or as soon as another CTA has set the flag.  Called by
-// every thread of the CTA (block barriers on both sides).
+// them have made it (counter target G n): a release addition, then acquire loads.  Bounded: it
+// gives up, sets the launch's abort flag and returns false after `limit` cycles, or as soon as
+// another CTA has set the flag.  Called by every thread of the CTA (block barriers on both sides).
 __device__ __forceinline__ bool head_barrier(unsigned* ctr, unsigned target, int* gabort, volatile int* s_abort,
                                              long long limit) {
   __syncthreads();
@@ -138,11 +138,13 @@ __global__ void __launch_bounds__(kKlThreads, 1)
   uint8_t* sX = sm;                                          // [cap][KB][128 rows][128 B]
   uint8_t* sW = sX + pts * D * 2;                            // [KB][2 terms][Np rows][128 B]
   int* lab = (int*)(sW + (size_t)2 * Np * D * 2);            // [pts]
-  int* order = lab + pts;                                    // [pts] points sorted by label
+  int* order = lab + pts;                                    // [pts] points sorted by label (first
+                                                             // iteration), then the labels before
   float* sq = (float*)(order + pts);                         // [pts] 1/rms (queries), 1 (keys)
   float* xn = sq + pts;                                      // [pts] norm in the rounding bound
   double* sig = (double*)(xn + pts);                         // [pts] scale of the group sums
-  int4* flags = (int4*)(sig + pts);                          // [pts] re-decision entries
+  int4* flags = (int4*)(sig + pts);                          // [pts] re-decision entries, then the
+                                                             // points whose label changed
   double* xs_all = (double*)(flags + pts);                   // scratch: km_loop_scratch(D) doubles
   float* sbias = (float*)(xs_all + km_loop_scratch(D));      // [Np]
   int* offs = (int*)(sbias + Np);                            // [C + 1]

@@ -101,4 +101,35 @@ def test_null_and_misaligned_arguments(lib):
     assert lib.sparsepr_attention(None, None, None, None, None) == 1
     assert lib.sparsepr_fit_apply(None, None, 0, None) == 1
     assert lib.sparsepr_sync(None) == 1
+    assert lib.sparsepr_set_wait_limit(None, 0, 100) == 1
+    assert lib.sparsepr_set_kmeans_path(None, 0) == 1
+    assert lib.sparsepr_set_kernel_events(None, 3, None, None) == 1
     lib.sparsepr_plan_destroy(None)
+
+
+def test_whole_loop_kmeans_partials_are_carved_only_where_a_side_qualifies(lib):
+    """The whole-loop k-means needs per-CTA partial sums in the workspace: a bf16 call with at
+    most 128 groups whose points fit in the SMs' shared memory gets them (the mid-size call), a
+    call too large to keep its points resident does not (the 13B-DiT layer), and an fp32 call
+    never does.  The sizes differ by exactly those buffers when the side's shape changes."""
+    def size(w):
+        cfg = _lib.config_from(w)
+        n = ctypes.c_size_t()
+        assert lib.sparsepr_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == 0
+        return n.value
+    mid = configs.workload(1)
+    # the same call with 200 key and query groups does not qualify (more than 128 groups)
+    many = mid.replace(n_kgroups=200, n_qgroups=200)
+    # extra bytes of the larger group count alone, measured on an fp32 call (never qualifies)
+    f32 = mid.replace(dtype=configs.F32)
+    grow = size(f32.replace(n_kgroups=200, n_qgroups=200)) - size(f32)
+    assert size(many) - size(mid) < grow, "the qualifying call must carry extra partial buffers"
+    big = configs.workload(2)
+    assert size(big.replace(dtype=configs.F32)) - size(big) == size_difference_of_inputs(big)
+
+
+def size_difference_of_inputs(w):
+    """Workspace bytes that depend on the input dtype alone: the permuted Q, K, V and the probe
+    queries, at 4 bytes (fp32) against 2 (bf16) per element."""
+    BH = w.B * w.H
+    return 2 * (3 * BH * w.N * w.d + BH * max(w.P, 1) * w.d)
