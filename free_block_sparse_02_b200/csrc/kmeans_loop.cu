@@ -898,27 +898,44 @@ static int device_sms() {
   return sms;
 }
 
-bool km_loop_supported(const Layout& L, bool keys) {
+// The launch shape of one side's whole loop on the current device: CTAs per head, resident tiles
+// per CTA and shared memory, or false when the side does not qualify (shape, workspace, test
+// hook) or its CTAs could not all be co-resident (cooperative launch support, occupancy).
+static bool km_loop_config(const Layout& L, bool keys, int& G, int& cap, size_t& smem) {
   if (!L.klp_sum || L.km_steps) return false;
   const int C = keys ? L.Ck : L.Cq;
-  const int G = km_loop_ctas_per_head(L.BH, L.N, L.d, L.dtype, C, L.Ck, keys, std::min(device_sms(), kKmLoopMaxCtas),
-                                      nullptr);
-  return G > 0 && G <= L.klp_G;
-}
-
-sparsepr_status launch_kmeans_loop(const Layout& L, bool keys, const void* X, int iters, cudaStream_t st) {
-  const int C = keys ? L.Ck : L.Cq;
-  int cap = 0;
-  const int G = km_loop_ctas_per_head(L.BH, L.N, L.d, L.dtype, C, L.Ck, keys, std::min(device_sms(), kKmLoopMaxCtas),
-                                      &cap);
-  if (G < 1 || G > L.klp_G) return SPARSEPR_ERR_UNSUPPORTED;
+  cap = 0;
+  G = km_loop_ctas_per_head(L.BH, L.N, L.d, L.dtype, C, L.Ck, keys, std::min(device_sms(), kKmLoopMaxCtas), &cap);
+  if (G < 1 || G > L.klp_G) return false;
+  int dev = 0, coop = 0;
+  cudaGetDevice(&dev);
+  if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop) {
+    (void)cudaGetLastError();  // a failed query must not read as a failed launch later
+    return false;
+  }
   const int Np = ((keys ? L.Ckp : L.Cqp) + 31) & ~31;
-  const size_t smem = km_loop_smem(L.d, Np, C, cap);
+  smem = km_loop_smem(L.d, Np, C, cap);
   auto kern = keys ? kmeans_loop_kernel<true> : kmeans_loop_kernel<false>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   int occ = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kKlThreads, smem);
-  if (occ < 1 || (long long)occ * device_sms() < (long long)L.BH * G) return SPARSEPR_ERR_UNSUPPORTED;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kKlThreads, smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  return occ >= 1 && (long long)occ * device_sms() >= (long long)L.BH * G;
+}
+
+bool km_loop_supported(const Layout& L, bool keys) {
+  int G, cap;
+  size_t smem;
+  return km_loop_config(L, keys, G, cap, smem);
+}
+
+sparsepr_status launch_kmeans_loop(const Layout& L, bool keys, const void* X, int iters, cudaStream_t st) {
+  int G, cap;
+  size_t smem;
+  if (!km_loop_config(L, keys, G, cap, smem)) return SPARSEPR_ERR_UNSUPPORTED;
+  auto kern = keys ? kmeans_loop_kernel<true> : kmeans_loop_kernel<false>;
   CUtensorMap mX;
   if (!make_tmap_bf16(&mX, X, (long long)L.BH * L.N, L.d, kKlTile)) return SPARSEPR_ERR_CUDA;
   // head barrier counters and the abort flag start at zero
