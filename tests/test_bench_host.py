@@ -30,6 +30,19 @@ def test_assignment_roofline_is_the_binding_one():
     assert bench.km_rooflines(configs.workload(1), 0.0, 0.0, PEAKS) == {}
 
 
+def test_whole_loop_kmeans_is_reported_per_iteration():
+    """Mid-size call, key side as one launch of 24 iterations in 0.5 ms: time per iteration,
+    and the scoring's tensor flops (4 C_p d per key per iteration) against the sustained peak."""
+    w = configs.workload(1)
+    r = bench.km_loop_roofline(w, 0.5, [16, 24, 15], PEAKS)["loop"]
+    assert r["bound"] == "latency" and r["iterations"] == 24
+    assert r["ms_per_iteration"] == pytest.approx(0.5 / 24)
+    keys = 8 * 16384
+    assert r["tensor"]["achieved"] == pytest.approx(keys * 4 * 64 * 64 * 24 / 0.5e-3 / 1e12)
+    assert r["tensor"]["peak"] == PEAKS["bf16_tflops_sustained"]
+    assert r["hbm_bytes"] == keys * 2 * 64  # the keys are read from HBM once per call
+
+
 def test_profiled_traffic_is_only_reported_for_the_profiled_configuration():
     w = configs.workload(1)
     assert bench.profiled_traffic(w.replace(P=64)) is None
