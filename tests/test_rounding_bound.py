@@ -7,7 +7,9 @@ three bf16 terms (hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid)), th
 fmaf(-2 sigma, dot, b32).  The claim: every fp32 score is within
     delta = 4 (3d + 8) 2^-23 ||sigma x|| max_j ||w_j|| + 4 2^-23 max_j |b_j|
 of the exact score, so the fp64 argmin is among the groups whose fp32 score is within 2.5 delta
-of the fp32 best.  This emulation shares nothing with the CUDA code; it restates the arithmetic."""
+of the fp32 best.  Also: the running fp64 group sums of bf16 keys, moved by label changes,
+equal fresh sums exactly.  This emulation shares nothing with the CUDA code; it restates the
+arithmetic."""
 import numpy as np
 
 
@@ -94,3 +96,36 @@ def test_two_term_split_bound_covers_keys_and_queries():
     assert check(d=128, C=64, n=96, wscale=1.0, bscale=50.0, sigma=1.0, seed=4, terms=2) < 1.0
     assert check(d=64, C=48, n=128, wscale=0.3, bscale=5.0, sigma=0.37, seed=5, terms=2) < 1.0
     assert check(d=64, C=32, n=64, wscale=100.0, bscale=1e5, sigma=1.0, seed=6, terms=2) < 1.0
+
+
+def _bf16(x):
+    """Round float32 values to bf16 (round to nearest even) and return them as float64."""
+    b = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16 << 16
+    return b.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def test_running_group_sums_of_bf16_keys_equal_fresh_sums():
+    """The k-means update keeps each group's fp64 sum of member keys as a running total, moved
+    by -x under a point's old label and +x under its new one, in whatever order the atomics
+    land.  For bf16 keys of the workloads' scale every partial sum is exactly representable in
+    fp64 (8-bit significands, an exponent spread of a few tens of bits, at most 2^17 terms), so
+    the running totals equal the sums formed afresh, bit for bit."""
+    rng = np.random.default_rng(7)
+    n, d, C = 4096, 16, 32
+    x = _bf16(rng.standard_normal((n, d)).astype(np.float32) * 2.0)
+    lab = rng.integers(0, C, n)
+    run = np.zeros((C, d))
+    for p in rng.permutation(n):  # the first iteration: every point, in a shuffled order
+        run[lab[p]] += x[p]
+    for _ in range(6):  # later iterations: about a tenth of the points change group
+        new = lab.copy()
+        ch = rng.random(n) < 0.1
+        new[ch] = rng.integers(0, C, ch.sum())
+        for p in rng.permutation(np.flatnonzero(new != lab)):
+            run[lab[p]] -= x[p]
+            run[new[p]] += x[p]
+        lab = new
+        fresh = np.zeros((C, d))
+        np.add.at(fresh, lab, x)
+        assert np.array_equal(run, fresh)
