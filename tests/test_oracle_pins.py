@@ -1,10 +1,11 @@
 """Pins of the fp64 oracle to things other than itself (CPU only).
 
-Each test checks one oracle function against a closed form, a library routine (torch SDPA,
-scikit-learn k-means, numpy lstsq, scipy orth), brute force on a tiny input, or a hand-worked
-fixture under tests/golden/ whose derivation is written in the fixture.  They are chosen so
-that a plausible slip (a dropped term, a wrong sign or scale, a transposed operand, an
-off-by-one in a sampling formula) fails at least one of them.
+Each test checks one oracle function, or a whole call from its own partition, against a closed
+form, a library routine (torch SDPA, scikit-learn k-means, numpy lstsq and SVD, scipy orth),
+brute force on a tiny input, or a hand-worked fixture under tests/golden/ whose derivation is
+written in the fixture.  They are chosen so that a plausible slip (a dropped term, a wrong sign
+or scale, a transposed operand, an off-by-one in a sampling formula, a swapped argument in the
+call) fails at least one of them; test_oracle_mutations.py plants such slips and checks that.
 """
 import json
 import math
@@ -162,6 +163,13 @@ def test_lloyd_tolerance_stop_rule():
         assert a - b > 1e-2 * a
     never = O.lloyd(X, X[:8], iters=7, tol=-1.0)
     assert never.n_iter == 7
+    # tol = 0: the run ends at the first iteration that leaves the objective unchanged (a fixed
+    # point of Lloyd's map gives bit-identical centroids, so the decrease is exactly 0)
+    zero = O.lloyd(X, X[:8], iters=200, tol=0.0)
+    assert zero.n_iter < 200 and zero.objective[-1] == zero.objective[-2]
+    assert all(a > b for a, b in zip(zero.objective[:-2], zero.objective[1:-1]))
+    # the earliest stop is at iteration 1: a start at a fixed point takes exactly two iterations
+    assert O.lloyd(X, zero.centroids, iters=10, tol=0.0).n_iter == 2
 
 
 def test_near_tie_margin_flags_equidistant_point():
@@ -384,6 +392,86 @@ def test_call_partition_is_consistent():
     r2 = O.call_head(q, k, v, cfg, 3, warm=O.warm_state(r))
     assert r2["kmeans_k"].n_iter <= cfg.km_iters_warm
     assert np.array_equal(r2["klabels"], r["klabels"])
+
+
+class _Cfg53(_Cfg):
+    """Unequal group counts (5 key groups, 3 query groups), so that a swapped label array or
+    group count in the call changes the result."""
+    n_kgroups, n_qgroups = 5, 3
+
+
+def test_call_routes_and_sparse_rows_follow_its_partition():
+    """The later stages of a whole call, checked from the call's own partition by other routes,
+    for the response-coupled and the semantic partition alike:
+    - the routing scores by pooling: the response of the group's mean query to each key-group
+      centroid (the member keys' means) plus ln m_j;
+    - the per-row key budget by the density it must reach with the routing and probe pairs;
+    - the block-sparse rows by torch SDPA under the mask route[g(q), j(k)];
+    - the stratified probes by their per-group counts."""
+    q, k, v = _small_inputs(17)
+    N, d = q.shape
+    for partition in (0, 1):
+        cfg = _Cfg53()
+        cfg.partition = partition
+        r = O.call_head(q, k, v, cfg, 1)
+        kl, ql = r["klabels"], r["qlabels"]
+        m = np.bincount(kl, minlength=cfg.n_kgroups)
+        n = np.bincount(ql, minlength=cfg.n_qgroups)
+        assert np.count_nonzero(m) > 1 and np.count_nonzero(n) > 1
+        cent = np.array([k[kl == j].mean(0) if m[j] else np.zeros(d) for j in range(cfg.n_kgroups)])
+        for g in np.flatnonzero(n):
+            pooled = cent @ q[ql == g].mean(0) / math.sqrt(d) + np.log(np.maximum(m, 1))
+            np.testing.assert_allclose(r["scores"][g][m > 0], pooled[m > 0], rtol=1e-12, atol=1e-12)
+            assert np.all(np.isneginf(r["scores"][g][m == 0]))
+        # the budget leaves room for s*N routing, C_k*N centroid and P*N probe pairs
+        assert abs((r["kappa"] + cfg.s + cfg.n_kgroups + cfg.P) / N - float(np.float32(cfg.density))) < 1e-12
+        np.testing.assert_allclose(r["osp"], _sdpa(q, k, v, r["route"][ql][:, kl]), rtol=1e-12, atol=1e-12)
+        per_group = np.bincount(ql[r["probes"]], minlength=cfg.n_qgroups)
+        assert per_group.sum() == cfg.P and np.all(np.abs(per_group - cfg.P * n / N) < 1.0)
+
+
+def _fit_rows(r):
+    X = np.hstack([r["osp"][r["probes"]], np.ones((len(r["probes"]), 1))])
+    return X, r["odense"] - r["osp"][r["probes"]], r["weights"]
+
+
+def test_call_fit_is_the_weighted_ridge_of_its_probe_residuals():
+    """The map a whole call applies, checked from its own probe rows by other routes.
+    - The ridge solution: augmented least squares (numpy lstsq) on X = [O_sp(p), 1],
+      R = O_dense(p) - O_sp(p) and the call's probe weights, with lam the call reports.
+    - The residual span: the right singular vectors of W^(1/2) R (numpy SVD) whose squared
+      singular value is above 1e-10 of the largest.  With P < d that span is a proper subspace,
+      so a projection on another one would show.
+    - The map: the ridge solution times the projector on that span.  With a truncation rank r
+      the projector is on the r leading vectors.
+    - The mean-only family: no linear part, and the shrunk weighted mean residual, in the same
+      span, as the intercept."""
+    q, k, v = _small_inputs(18)
+    cfg = _Cfg53()
+    r = O.call_head(q, k, v, cfg, 0)
+    X, R, w = _fit_rows(r)
+    d = q.shape[1]
+    assert len(w) < d and np.ptp(w) > 0            # a proper span and unequal weights
+    lam = r["lam"]
+    Xa = np.vstack([np.sqrt(w)[:, None] * X, math.sqrt(lam) * np.eye(d + 1)])
+    Ra = np.vstack([np.sqrt(w)[:, None] * R, np.zeros((d + 1, d))])
+    A_ridge = np.linalg.lstsq(Xa, Ra, rcond=None)[0]
+    _, sv, Vt = np.linalg.svd(np.sqrt(w)[:, None] * R)
+    V = Vt[:int(np.sum(sv ** 2 > 1e-10 * sv[0] ** 2))].T
+    assert V.shape[1] < d
+    scale = np.abs(A_ridge).max()
+    np.testing.assert_allclose(r["A"], A_ridge @ V @ V.T, rtol=0, atol=1e-9 * scale)
+
+    cfg.trunc_rank = 2
+    rt = O.call_head(q, k, v, cfg, 0)
+    assert np.array_equal(rt["probes"], r["probes"])
+    np.testing.assert_allclose(rt["A"], A_ridge @ V[:, :2] @ V[:, :2].T, rtol=0, atol=1e-9 * scale)
+
+    cfg.trunc_rank, cfg.correction = 0, 1
+    rm = O.call_head(q, k, v, cfg, 0)
+    assert not np.any(rm["A"][:-1])
+    mean = (w[:, None] * R).sum(0) / (w.sum() + rm["lam"])
+    np.testing.assert_allclose(rm["A"][-1], mean @ V @ V.T, rtol=0, atol=1e-12 * np.abs(mean).max())
 
 
 def test_table2_error_reduction_arithmetic():
