@@ -916,7 +916,12 @@ static bool km_loop_config(const Layout& L, bool keys, int& G, int& cap, size_t&
   const int Np = ((keys ? L.Ckp : L.Cqp) + 31) & ~31;
   smem = km_loop_smem(L.d, Np, C, cap);
   auto kern = keys ? kmeans_loop_kernel<true> : kmeans_loop_kernel<false>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // A failure here falls back to the per-iteration launches, so its error must not linger for
+  // their launch checks to report.
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
   int occ = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kKlThreads, smem) != cudaSuccess) {
     (void)cudaGetLastError();
