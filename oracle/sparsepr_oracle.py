@@ -285,7 +285,7 @@ def route_group(S_row: np.ndarray, ksizes: np.ndarray, fixed_k: int, kappa: floa
 # Steps 6 and 7: attention.
 # ----------------------------------------------------------------------------------------------
 def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
-    """softmax(q k^T / sqrt(d)) v, row-wise, float64."""
+    """softmax(q k^T / sqrt(d)) v, row-wise, float64.  With no keys the rows are the empty sum, 0."""
     if k.shape[0] == 0:
         return np.zeros((q.shape[0], v.shape[1]))
     s = (q @ k.T) / math.sqrt(q.shape[1])

@@ -56,6 +56,12 @@ MUTANTS = [
      ["lloyd_tolerance_stop_rule"]),
     ("first-stop-at-two", "lloyd", "if tol >= 0 and it >= 1:", "if tol >= 0 and it >= 2:",
      ["lloyd_tolerance_stop_rule"]),
+    ("objective-after-update", "lloyd", "        if tol >= 0 and it >= 1:",
+     "        J_hist[-1] = float(((X - C[labels]) ** 2).sum())\n        if tol >= 0 and it >= 1:",
+     ["lloyd_objective_non_increasing_and_fixed_point", "lloyd_tolerance_stop_rule"]),
+    ("near-tie-mask-last-only", "lloyd", "tie_mask |= nt", "tie_mask = nt", ["near_tie_margin_flags_equidistant_point"]),
+    ("margin-absolute", "assign", "(d2 - d1) / np.where(d1 > 0, d1, 1.0)", "(d2 - d1)",
+     ["near_tie_margin_flags_equidistant_point"]),
     ("shadow-sum", "lloyd", "S[j] = shadow[members].mean(axis=0)", "S[j] = shadow[members].sum(axis=0)",
      ["lloyd_empty_group_keeps_centroid_and_shadow"]),
     ("key-basis-trailing", "key_response_basis", "return Vt[:rank].T", "return Vt[-rank:].T",
@@ -100,6 +106,8 @@ MUTANTS = [
      ["dense_attention_matches_torch_sdpa"]),
     ("softmax-axis", "attention", "p /= p.sum(axis=1, keepdims=True)", "p /= p.sum(axis=0, keepdims=True)",
      ["dense_attention_matches_torch_sdpa"]),
+    ("no-keys-nan", "attention", "return np.zeros((q.shape[0], v.shape[1]))",
+     "return np.full((q.shape[0], v.shape[1]), np.nan)", ["sparse_attention_matches_masked_sdpa"]),
     ("sparse-query-labels", "sparse_attention", "route[g][klabels]", "route[g][qlabels]",
      ["sparse_attention_matches_masked_sdpa"]),
     ("sparse-mask-after-softmax", "sparse_attention", "out[rows] = attention(q[rows], k[keys], v[keys])",
@@ -119,6 +127,11 @@ MUTANTS = [
      "(i * int(n[g])) // int(m[g])", ["probes_stratified_hand_cases"]),
     ("stratified-weights-unscaled", "probes_stratified", "wts = wts * (P / wts.sum())", "wts = wts",
      ["probes_stratified_hand_cases", "probes_stratified_invariants"]),
+    ("stratified-weights-inverted", "probes_stratified", "wts.append(float(n[g]) / float(m[g]))",
+     "wts.append(float(m[g]) / float(n[g]))", ["probes_stratified_hand_cases"]),
+    ("stratified-unsorted", "probes_stratified", "toks, wts = toks[o], wts[o]", "pass",
+     ["probes_stratified_invariants"]),
+    ("uniform-weights", "probes_uniform", "np.ones(P)", "np.full(P, 2.0)", ["probes_uniform_formula"]),
     ("stratified-rounded-share", "probes_stratified", "base = (P * n) // N", "base = (P * n + N // 2) // N",
      ["probes_stratified_hand_cases"]),
     # ridge fit, span, correction
@@ -141,6 +154,8 @@ MUTANTS = [
      ["truncated_span_is_the_leading_right_singular_subspace"]),
     ("span-trailing", "residual_span_basis", "np.argsort(-ev, kind=\"stable\")", "np.argsort(ev, kind=\"stable\")",
      ["truncated_span_is_the_leading_right_singular_subspace"]),
+    ("truncation-off-by-one", "residual_span_basis", "if rank > 0 and U.shape[1] > rank:",
+     "if rank > 0 and U.shape[1] > rank + 1:", ["truncated_span_is_the_leading_right_singular_subspace"]),
     ("span-not-applied", "restrict_to_residual_span", "return A @ U @ U.T", "return A", ["residual_span_projection"]),
     ("apply-intercept-first", "apply_correction", "osp @ A[:-1] + A[-1][None, :]", "osp @ A[1:] + A[0][None, :]",
      ["apply_correction_and_row_errors"]),
@@ -170,6 +185,14 @@ MUTANTS = [
     # the whole call
     ("call-key-sizes-from-queries", "call_head", "m = np.bincount(klabels, minlength=Ck)",
      "m = np.bincount(qlabels, minlength=Ck)", ["call_partition_is_consistent"]),
+    ("call-density-drops-centroid-pairs", "call_head", "density = (cfg.s * N + Ck * N + cfg.P * N + sparse_pairs)",
+     "density = (cfg.s * N + cfg.P * N + sparse_pairs)",
+     ["call_with_every_group_kept_is_dense", "call_routes_and_sparse_rows_follow_its_partition"]),
+    ("call-pairs-without-group-sizes", "call_head", "sparse_pairs = int(sum(int(n[g]) * int(m[route[g]].sum())",
+     "sparse_pairs = int(sum(int(m[route[g]].sum())",
+     ["call_with_every_group_kept_is_dense", "call_routes_and_sparse_rows_follow_its_partition"]),
+    ("warm-runs-cold-limit", "call_head", "S0, iters = warm.key_centroids, cfg.km_iters_warm",
+     "S0, iters = warm.key_centroids, cfg.km_iters", ["warm_start_key_step_uses_the_current_calls_metric"]),
     ("call-routes-on-normalised-responses", "call_head", "S = routing_scores(R, qlabels, Cq, m)",
      "S = routing_scores(Rt, qlabels, Cq, m)", ["call_routes_and_sparse_rows_follow_its_partition"]),
     ("call-budget-with-query-groups", "call_head", "per_row_key_budget(cfg.density, N, cfg.s, Ck, cfg.P)",
@@ -187,6 +210,9 @@ MUTANTS = [
      ["warm_start_restarts_lloyd_where_the_previous_call_stopped"]),
     ("semantic-keys-from-queries", "semantic_call_head", "kk = lloyd(k, k[ids], cfg.km_iters, tol)",
      "kk = lloyd(q, q[ids], cfg.km_iters, tol)", ["semantic_partition_is_kmeans_on_the_raw_inputs"]),
+    ("semantic-density-drops-centroid-pairs", "route_and_probe",
+     "density = (cfg.s * N + Ck * N + cfg.P * N + sparse_pairs)", "density = (cfg.s * N + cfg.P * N + sparse_pairs)",
+     ["call_routes_and_sparse_rows_follow_its_partition"]),
     ("semantic-routes-on-scaled-responses", "route_and_probe", "routing_scores(query_responses(q, kcent),",
      "routing_scores(2.0 * query_responses(q, kcent),", ["call_routes_and_sparse_rows_follow_its_partition"]),
     ("error-reduction-inverted", "error_reduction", "1.0 - err_method / err_baseline",

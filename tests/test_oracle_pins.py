@@ -101,6 +101,12 @@ def test_sparse_attention_matches_masked_sdpa():
                                rtol=1e-12, atol=1e-12)
     full = np.ones((3, 4), dtype=bool)
     np.testing.assert_allclose(O.sparse_attention(q, k, v, ql, kl, full), O.attention(q, k, v), atol=1e-13)
+    # a query group that keeps no key group has no keys to attend to: its rows are the empty sum, 0
+    none = route.copy()
+    none[1] = False
+    out = O.sparse_attention(q, k, v, ql, kl, none)
+    assert np.all(out[ql == 1] == 0.0)
+    np.testing.assert_allclose(out[ql != 1], _sdpa(q, k, v, mask)[ql != 1], rtol=1e-12, atol=1e-12)
 
 
 # ---------------------------------------------------------------- k-means
@@ -126,6 +132,10 @@ def test_lloyd_objective_non_increasing_and_fixed_point():
     res = O.lloyd(X, X[:12], iters=50, tol=0.0)
     J = np.array(res.objective)
     assert np.all(np.diff(J) <= 1e-9 * J[:-1])
+    # J_0 is recorded at the first assignment: each point's squared distance to its nearest
+    # initial centroid, by brute force
+    J0 = sum(min(float(np.sum((x - c) ** 2)) for c in X[:12]) for x in X)
+    assert J[0] == pytest.approx(J0, rel=1e-12)
     again = O.lloyd(X, res.centroids, iters=1, tol=0.0)
     assert np.array_equal(again.labels, res.labels)
     np.testing.assert_allclose(again.centroids, res.centroids, atol=1e-13)
@@ -177,6 +187,13 @@ def test_near_tie_margin_flags_equidistant_point():
     labels, d1, margin = O.assign(X, np.array([[0.0], [2.0]]))
     assert list(labels) == [0, 0, 1]          # the midpoint goes to the lower index
     assert margin[1] == 0.0 and margin[0] == np.inf
+    # the margin is relative: x = 0.5 against centroids 0 and 2 has d1 = 0.25, d2 = 2.25
+    _, _, m = O.assign(np.array([[0.5]]), np.array([[0.0], [2.0]]))
+    assert m[0] == pytest.approx(8.0, rel=1e-15)
+    # a near-tie at any iteration stays flagged: the midpoint ties only at the first assignment
+    # (centroids 0 and 2), and after the update (0.5 and 2) it does not
+    res = O.lloyd(X, np.array([[0.0], [2.0]]), iters=3, tol=-1.0)
+    assert res.near_ties == [1, 0, 0] and list(res.near_tie_mask) == [False, True, False]
 
 
 def test_key_response_kmeans_equals_metric_kmeans_in_key_space():
@@ -407,6 +424,7 @@ def test_call_routes_and_sparse_rows_follow_its_partition():
       centroid (the member keys' means) plus ln m_j;
     - the per-row key budget by the density it must reach with the routing and probe pairs;
     - the block-sparse rows by torch SDPA under the mask route[g(q), j(k)];
+    - the executed pairs and the realised density by counting that mask;
     - the stratified probes by their per-group counts."""
     q, k, v = _small_inputs(17)
     N, d = q.shape
@@ -425,7 +443,12 @@ def test_call_routes_and_sparse_rows_follow_its_partition():
             assert np.all(np.isneginf(r["scores"][g][m == 0]))
         # the budget leaves room for s*N routing, C_k*N centroid and P*N probe pairs
         assert abs((r["kappa"] + cfg.s + cfg.n_kgroups + cfg.P) / N - float(np.float32(cfg.density))) < 1e-12
-        np.testing.assert_allclose(r["osp"], _sdpa(q, k, v, r["route"][ql][:, kl]), rtol=1e-12, atol=1e-12)
+        mask = r["route"][ql][:, kl]
+        np.testing.assert_allclose(r["osp"], _sdpa(q, k, v, mask), rtol=1e-12, atol=1e-12)
+        # executed pairs counted on the mask, and the realised density they give with the
+        # routing, centroid and probe pairs
+        assert r["sparse_pairs"] == int(mask.sum())
+        assert r["density"] == pytest.approx((cfg.s + cfg.n_kgroups + cfg.P) / N + mask.sum() / N ** 2, rel=1e-14)
         per_group = np.bincount(ql[r["probes"]], minlength=cfg.n_qgroups)
         assert per_group.sum() == cfg.P and np.all(np.abs(per_group - cfg.P * n / N) < 1.0)
 
@@ -547,7 +570,7 @@ def test_truncated_span_is_the_leading_right_singular_subspace():
     R = rng.standard_normal((P, d)) @ np.diag([5.0, 3.0, 2.0, 1.0, 0.5, 0.1])
     w = rng.uniform(0.5, 2.0, P)
     _, _, Vt = np.linalg.svd(np.sqrt(w)[:, None] * R)
-    for r in (1, 2, 4):
+    for r in (1, 2, 4, 5):                          # 5: one direction fewer than the span
         U = O.residual_span_basis(R, w, r)
         assert U.shape == (d, r)
         np.testing.assert_allclose(U @ U.T, Vt[:r].T @ Vt[:r], atol=1e-12)
