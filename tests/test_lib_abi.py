@@ -133,3 +133,60 @@ def size_difference_of_inputs(w):
     queries, at 4 bytes (fp32) against 2 (bf16) per element."""
     BH = w.B * w.H
     return 2 * (3 * BH * w.N * w.d + BH * max(w.P, 1) * w.d)
+
+
+def _header_layout(tmp_path, structs, constants):
+    """Sizes, field offsets and constant values as a C compiler sees them in include/sparsepr.h:
+    a small C program prints them."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "sparsepr.h"', "int main(void) {"]
+    for cname, fields in structs.items():
+        lines.append(f'  printf("size {cname} %zu\\n", sizeof({cname}));')
+        for f in fields:
+            lines.append(f'  printf("offset {cname}.{f} %zu\\n", offsetof({cname}, {f}));')
+    for c in constants:
+        lines.append(f'  printf("const {c} %d\\n", (int){c});')
+    lines += ["  return 0;", "}"]
+    src, exe = tmp_path / "layout.c", tmp_path / "layout"
+    src.write_text("\n".join(lines) + "\n")
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    return {k: int(v) for k, v in (line.rsplit(" ", 1) for line in out.splitlines())}
+
+
+def test_binding_structs_and_constants_match_the_header(tmp_path):
+    """The ctypes mirrors of sparsepr_config and sparsepr_head_stats have the header's size and
+    field offsets, and the binding's constants equal the header's enumerators, so a change on
+    one side that the other misses fails here instead of corrupting calls."""
+    mirrors = {"sparsepr_config": _lib.Config, "sparsepr_head_stats": _lib.HeadStats}
+    c_field = lambda f: "lambda" if f == "lambda_" else f
+    structs = {c: [c_field(f) for f, _ in m._fields_] for c, m in mirrors.items()}
+    consts = {
+        "SPARSEPR_F32": _lib.SPARSEPR_F32, "SPARSEPR_BF16": _lib.SPARSEPR_BF16,
+        "SPARSEPR_PROBE_UNIFORM": configs.PROBE_UNIFORM, "SPARSEPR_PROBE_STRATIFIED": configs.PROBE_STRATIFIED,
+        "SPARSEPR_PROBE_RANDOM": configs.PROBE_RANDOM,
+        "SPARSEPR_CORRECTION_AFFINE": configs.CORRECTION_AFFINE, "SPARSEPR_CORRECTION_MEAN": configs.CORRECTION_MEAN,
+        "SPARSEPR_PARTITION_RESPONSE": configs.PARTITION_RESPONSE,
+        "SPARSEPR_PARTITION_SEMANTIC": configs.PARTITION_SEMANTIC,
+        "SPARSEPR_KERNEL_BLOCK_SPARSE": _lib.KERNEL_BLOCK_SPARSE,
+        "SPARSEPR_KERNEL_KMEANS_ASSIGN": _lib.KERNEL_KMEANS_ASSIGN,
+        "SPARSEPR_KERNEL_KMEANS_UPDATE": _lib.KERNEL_KMEANS_UPDATE,
+        "SPARSEPR_KERNEL_KMEANS_LOOP": _lib.KERNEL_KMEANS_LOOP,
+        "SPARSEPR_OK": 0, "SPARSEPR_ERR_STATE": max(_lib.STATUS),
+    }
+    consts.update({"SPARSEPR_" + n: getattr(_lib, n) for n in dir(_lib) if n.startswith("Q_")})
+    got = _header_layout(tmp_path, structs, consts)
+    for cname, m in mirrors.items():
+        assert got[f"size {cname}"] == ctypes.sizeof(m), cname
+        for f, _ in m._fields_:
+            assert got[f"offset {cname}.{c_field(f)}"] == getattr(m, f).offset, (cname, f)
+    for c, v in consts.items():
+        assert got[f"const {c}"] == v, c
+    # every query enumerator of the header has a binding constant
+    text = open(os.path.join(ROOT, "include", "sparsepr.h")).read()
+    assert set(re.findall(r"\b(SPARSEPR_Q_[A-Z_]+)\s*=", text)) == {c for c in consts if c.startswith("SPARSEPR_Q_")}
