@@ -62,6 +62,38 @@ def test_invalid_configs_are_rejected_on_the_host(lib, field, value, code):
     assert lib.sparsepr_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == code
 
 
+@pytest.mark.parametrize("base,over,code", [
+    (0, dict(B=0), 1), (0, dict(H=0), 1), (0, dict(n_qgroups=0), 1), (0, dict(fixed_k=-1), 1),
+    (1, dict(density=1.5), 1), (1, dict(density=float("nan")), 1), (0, dict(P=2000), 1),
+    (0, dict(N=500, n_kgroups=600), 1), (0, dict(N=500, n_qgroups=501), 1),
+    (0, dict(lam=float("nan")), 1), (0, dict(lam=float("inf")), 1), (0, dict(km_tol=float("nan")), 1),
+    (0, dict(km_iters=10001), 1), (0, dict(km_iters_warm=10001), 1),
+    (0, dict(key_rank=-1), 1), (0, dict(key_rank=65), 1),
+    # sizes: a call whose element count overflows 64-bit offsets is invalid; one whose row count
+    # overflows the kernels' int32 row index is valid but not built
+    (0, dict(B=2**31 - 1, H=2**31 - 1, N=2**31 - 1, s=1, n_kgroups=1, n_qgroups=1, P=0), 1),
+    (2, dict(H=20000), 2),
+])
+def test_config_ranges_of_the_header_are_enforced(lib, base, over, code):
+    """Every range the header states for a sparsepr_config field is checked on the host, with
+    the status code the header gives (INVALID_ARG for a value outside its range, UNSUPPORTED for
+    a valid call this build does not run)."""
+    cfg = _lib.config_from(configs.workload(base), **over)
+    n = ctypes.c_size_t(0)
+    assert lib.sparsepr_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == code
+
+
+def test_range_edges_are_accepted(lib):
+    """The inclusive ends of the ranges pass: s = N, C_k = C_q = N, P = N, density = 1,
+    trunc_rank = key_rank = d, and the iteration caps."""
+    w = configs.workload(0).replace(N=512)
+    for over in (dict(s=512), dict(n_kgroups=512, n_qgroups=512), dict(P=512), dict(density=1.0, fixed_k=0),
+                 dict(trunc_rank=64, key_rank=64), dict(km_iters=10000, km_iters_warm=10000)):
+        cfg = _lib.config_from(w, **over)
+        n = ctypes.c_size_t(0)
+        assert lib.sparsepr_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == 0, over
+
+
 def test_semantic_partition_without_repair_is_accepted(lib):
     cfg = _lib.config_from(configs.workload(1), partition=configs.PARTITION_SEMANTIC, repair=0)
     n = ctypes.c_size_t(0)
