@@ -222,3 +222,24 @@ def test_binding_structs_and_constants_match_the_header(tmp_path):
     # every query enumerator of the header has a binding constant
     text = open(os.path.join(ROOT, "include", "sparsepr.h")).read()
     assert set(re.findall(r"\b(SPARSEPR_Q_[A-Z_]+)\s*=", text)) == {c for c in consts if c.startswith("SPARSEPR_Q_")}
+
+
+def test_static_ridge_fit_rejects_bad_arguments_before_any_device_call(lib):
+    """sparsepr_ridge_fit_static checks its arguments first, with the header's codes: null
+    pointers, a non-finite lambda, no heads or a negative P are INVALID_ARG; d outside
+    {64, 128} is UNSUPPORTED; more than 16 heads or 4096 probe rows exceed its fixed scratch
+    (WORKSPACE).  The pointers below are never dereferenced: each case returns before the first
+    device call."""
+    f = lib.sparsepr_ridge_fit_static
+    vp = ctypes.c_void_p
+    f.restype = ctypes.c_int32
+    f.argtypes = [vp, vp, vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_double, vp, vp, vp]
+    fake = 4096
+    ok = dict(osp=fake, od=fake, w=fake, heads=2, P=48, d=64, lam=-1.0, A=fake)
+    cases = [(dict(A=None), 1), (dict(osp=None), 1), (dict(od=None), 1), (dict(w=None), 1),
+             (dict(lam=float("nan")), 1), (dict(lam=float("inf")), 1), (dict(heads=0), 1), (dict(P=-1), 1),
+             (dict(d=96), 2), (dict(d=0), 2), (dict(heads=17), 4), (dict(P=4097), 4)]
+    for over, code in cases:
+        a = dict(ok, **over)
+        got = f(a["osp"], a["od"], a["w"], a["heads"], a["P"], a["d"], a["lam"], a["A"], None, None)
+        assert got == code, over
