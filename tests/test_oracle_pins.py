@@ -502,6 +502,12 @@ def test_table2_error_reduction_arithmetic():
     red = [100 * O.error_reduction(b, a) for a, b in zip(t["semantic_mean"], t["sparsepr_mean"])]
     lo, hi = t["stated_reduction_range_pct"]
     assert round(min(red), 1) == lo and round(max(red), 1) == hi
+    # Figure 4(a): the gain of the response-coupled partition, SparsePR against the semantic
+    # partition with the same probe repair, for the mean and the p99 error
+    for ours, base, key in (("sparsepr_mean", "semantic_repair_mean", "fig4_mean_range_pct"),
+                            ("sparsepr_p99", "semantic_repair_p99", "fig4_p99_range_pct")):
+        red = [100 * O.error_reduction(a, b) for a, b in zip(t[ours], t[base])]
+        assert [round(min(red), 1), round(max(red), 1)] == t[key], (key, red)
 
 
 def test_repair_reduces_error_on_smooth_field_inputs():
