@@ -122,7 +122,10 @@ __global__ void __launch_bounds__(256) key_rank_kernel(Layout L) {
   __syncthreads();
   jacobi_eig(sS, V, d);
   // the r leading eigenvalues (descending, ties to the lower index)
-  for (int i = tid; i < d; i += nt) ev[i] = sS[i * d + i];
+  for (int i = tid; i < d; i += nt) {
+    const double e = sS[i * d + i];
+    ev[i] = isnan(e) ? -INFINITY : e;  // NaN (from non-finite inputs) ranks last: order[] stays a permutation
+  }
   __syncthreads();
   for (int i = tid; i < d; i += nt) {
     int rk = 0;

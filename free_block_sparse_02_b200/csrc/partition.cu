@@ -919,6 +919,9 @@ __global__ void __launch_bounds__(256) route_select_kernel(Layout L, const T* __
       double dot = 0.0;
       for (int a = 0; a < d; ++a) dot += qbar[a] * c[a];
       v = dot * rsd + log((double)m);
+      // a non-finite input can make a score NaN; ranking it as -inf keeps the rank count below
+      // a strict total order, so ord[] is a permutation and every index written from it is valid
+      if (isnan(v)) v = -INFINITY;
     }
     S[j] = v;
   }
