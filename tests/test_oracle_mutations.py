@@ -9,10 +9,9 @@ for one test only. The pins of test_oracle_pins.py named beside the mutant must 
 A control runs every listed pin against an unchanged recompiled copy of the same function. This
 shows that a failure comes from the planted change and not from the recompilation.
 
-Left out on purpose are mutants that change no result the method defines. Examples: the order
-of the sampled query rows (a permutation of the response columns keeps every distance); a
-shift of the softmax by the global instead of the row maximum; a strict against a non-strict
-test on a continuous objective.
+Left out on purpose are mutants that change no result the method defines. Two examples: the
+order of the sampled query rows, since a permutation of the response columns keeps every
+distance; and a shift of the softmax by the global instead of the row maximum.
 """
 import __future__
 import inspect
